@@ -1,0 +1,244 @@
+"""fp64 CPU oracle for the rotated low-bit linear -- TEST INFRASTRUCTURE ONLY.
+
+Only the tests, the smoke check and the benchmark's CPU-baseline leg may import
+this package. It is a ctypes front end to ``harp_oracle.c`` (plain fp64 C, see that
+file's header for the passages of "HARP: Hadamard-Preconditioned Adaptive Rotation
+Processor for Extreme LLM Quantization" each function follows). It shares nothing
+with the CUDA library: no code, headers, tables or helpers.
+
+Parity status: every function here is pinned by the ``-m "not gpu"`` tests in
+``tests/test_oracle_pins.py`` (Sylvester-Hadamard identity, orthogonality, exact
+change of basis, brute-force quantizer argmin, pack round trip with hand-built
+bytes, block-diagonal split, the theta = -pi/4 diagonal case, a dense
+stride-permutation construction and hand-computed golden fixtures).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+_i64 = ctypes.c_int64
+_int = ctypes.c_int
+_dp = ctypes.POINTER(ctypes.c_double)
+_u8p = ctypes.POINTER(ctypes.c_uint8)
+_i8p = ctypes.POINTER(ctypes.c_int8)
+_u16p = ctypes.POINTER(ctypes.c_uint16)
+
+
+class _Linear(ctypes.Structure):
+    _fields_ = [("n_in", _i64), ("n_out", _i64), ("w_in", _i64), ("w_out", _i64),
+                ("bits", _i64), ("group", _i64),
+                ("thV", _dp), ("sV", _i8p), ("thU", _dp), ("sU", _i8p),
+                ("packed", _u8p), ("scale_zero", _u16p)]
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        L.ora_butterfly_fwd.argtypes = [_i64, _i64, _i64, _dp, _i8p, _dp]
+        L.ora_butterfly_inv.argtypes = [_i64, _i64, _i64, _dp, _i8p, _dp]
+        L.ora_rotate_weights.argtypes = [_i64, _i64, _i64, _i64, _dp, _i8p, _dp, _i8p, _dp]
+        L.ora_quantize.argtypes = [_i64, _i64, _int, _int, _dp, _u8p, _u16p, _u16p]
+        L.ora_pack.argtypes = [_i64, _i64, _int, _u8p, _u8p]
+        L.ora_unpack.argtypes = [_i64, _i64, _int, _u8p, _u8p]
+        L.ora_packed_bytes.argtypes = [_i64, _i64, _int]
+        L.ora_packed_bytes.restype = _i64
+        L.ora_linear_fwd.argtypes = [ctypes.POINTER(_Linear), _i64, _dp, _dp]
+        L.ora_dense_rotated_fwd.argtypes = [_i64, _i64, _i64, _i64, _dp, _i8p, _dp, _i8p, _dp,
+                                            _i64, _dp, _dp]
+        L.ora_stack_step.argtypes = [_i64, ctypes.POINTER(_Linear), _i64, _i64, _i64, _i64, _i64,
+                                     ctypes.c_double, _i64, _dp, _dp]
+        L.ora_f16_from_f64.argtypes = [ctypes.c_double]
+        L.ora_f16_from_f64.restype = ctypes.c_uint16
+        L.ora_f16_to_f64.argtypes = [ctypes.c_uint16]
+        L.ora_f16_to_f64.restype = ctypes.c_double
+        L.ora_set_threads.argtypes = [_int]
+        L.ora_get_threads.restype = _int
+        _lib = L
+    return _lib
+
+
+def _d(a):
+    return a.ctypes.data_as(_dp)
+
+
+def _f64(a):
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _i8(a):
+    return np.ascontiguousarray(a, dtype=np.int8)
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise ValueError(f"oracle {what}: invalid arguments (rc={rc})")
+
+
+def set_threads(n: int) -> None:
+    lib().ora_set_threads(int(n))
+
+
+def get_threads() -> int:
+    return int(lib().ora_get_threads())
+
+
+# ---------------------------------------------------------------- fp16 bits
+def f16_from_f64(v) -> np.ndarray:
+    v = np.asarray(v, dtype=np.float64)
+    f = lib().ora_f16_from_f64
+    return np.array([f(float(t)) for t in v.ravel()], dtype=np.uint16).reshape(v.shape)
+
+
+def f16_to_f64(h) -> np.ndarray:
+    h = np.asarray(h, dtype=np.uint16)
+    f = lib().ora_f16_to_f64
+    return np.array([f(int(t)) for t in h.ravel()], dtype=np.float64).reshape(h.shape)
+
+
+# ---------------------------------------------------------------- butterfly
+def _bfly(fn, x, theta, sign, w):
+    x = _f64(x).copy()
+    one = x.ndim == 1
+    x2 = x.reshape(1, -1) if one else x
+    n = x2.shape[1]
+    th = _f64(theta)
+    sg = _i8(sign)
+    assert th.size == (n // 2) * int(np.log2(w)) and sg.size == n
+    _check(fn(n, int(w), x2.shape[0], _d(th), sg.ctypes.data_as(_i8p), _d(x2)), "butterfly")
+    return x2.reshape(-1) if one else x2
+
+
+def butterfly_fwd(x, theta, sign, w):
+    """F(theta, s, w) x: signs first, then stages of stride 1, 2, ..., w/2."""
+    return _bfly(lib().ora_butterfly_fwd, x, theta, sign, w)
+
+
+def butterfly_inv(x, theta, sign, w):
+    """F(theta, s, w)^T x: stages of stride w/2, ..., 1, then signs."""
+    return _bfly(lib().ora_butterfly_inv, x, theta, sign, w)
+
+
+# ---------------------------------------------------------------- offline prep
+def rotate_weights(W, thV, sV, w_in, thU, sU, w_out):
+    """W' = U W V^T with V = F_V and U^T = F_U."""
+    Wr = _f64(W).copy()
+    n_out, n_in = Wr.shape
+    thV, thU = _f64(thV), _f64(thU)
+    sV, sU = _i8(sV), _i8(sU)
+    _check(lib().ora_rotate_weights(n_out, n_in, int(w_in), int(w_out), _d(thV),
+                                    sV.ctypes.data_as(_i8p), _d(thU), sU.ctypes.data_as(_i8p),
+                                    _d(Wr)), "rotate")
+    return Wr
+
+
+def quantize(Wr, bits, group=64):
+    """Returns (q uint8 [n_out, n_in], scale16 uint16 [n_out, ng], zero16 uint16 [n_out, ng])."""
+    Wr = _f64(Wr)
+    n_out, n_in = Wr.shape
+    q = np.zeros((n_out, n_in), np.uint8)
+    s = np.zeros((n_out, n_in // group), np.uint16)
+    z = np.zeros((n_out, n_in // group), np.uint16)
+    _check(lib().ora_quantize(n_out, n_in, int(bits), int(group), _d(Wr), q.ctypes.data_as(_u8p),
+                              s.ctypes.data_as(_u16p), z.ctypes.data_as(_u16p)), "quantize")
+    return q, s, z
+
+
+def pack(q, bits):
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    n_out, n_in = q.shape
+    out = np.zeros(int(lib().ora_packed_bytes(n_out, n_in, int(bits))), np.uint8)
+    _check(lib().ora_pack(n_out, n_in, int(bits), q.ctypes.data_as(_u8p), out.ctypes.data_as(_u8p)),
+           "pack")
+    return out
+
+
+def unpack(packed, n_out, n_in, bits):
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    q = np.zeros((n_out, n_in), np.uint8)
+    _check(lib().ora_unpack(n_out, n_in, int(bits), packed.ctypes.data_as(_u8p),
+                            q.ctypes.data_as(_u8p)), "unpack")
+    return q
+
+
+def scale_zero(scale16, zero16):
+    """Interleaves the fp16 bits into the [n_out][n_in/group] {scale, zero} pair layout."""
+    return np.ascontiguousarray(np.stack([scale16, zero16], axis=-1).astype(np.uint16))
+
+
+# ---------------------------------------------------------------- layers
+class Layer:
+    """One rotated low-bit linear as the oracle sees it (all arrays host numpy)."""
+
+    def __init__(self, n_in, n_out, bits, w_in, w_out, thV, sV, thU, sU, packed, sz, group=64):
+        self.n_in, self.n_out, self.bits, self.group = int(n_in), int(n_out), int(bits), int(group)
+        self.w_in, self.w_out = int(w_in), int(w_out)
+        self.thV, self.thU = _f64(thV), _f64(thU)
+        self.sV, self.sU = _i8(sV), _i8(sU)
+        self.packed = np.ascontiguousarray(packed, dtype=np.uint8)
+        self.sz = np.ascontiguousarray(sz, dtype=np.uint16)
+        assert self.packed.size == n_out * n_in * bits // 8
+        assert self.sz.size == n_out * (n_in // group) * 2
+
+    def cstruct(self):
+        return _Linear(self.n_in, self.n_out, self.w_in, self.w_out, self.bits, self.group,
+                       _d(self.thV), self.sV.ctypes.data_as(_i8p), _d(self.thU),
+                       self.sU.ctypes.data_as(_i8p), self.packed.ctypes.data_as(_u8p),
+                       self.sz.ctypes.data_as(_u16p))
+
+
+def prepare_layer(W, bits, w_in, w_out, thV, sV, thU, sU, group=64):
+    """Rotate, quantize and pack a weight matrix; returns (Layer, q, scale16, zero16, W')."""
+    n_out, n_in = np.shape(W)
+    Wr = rotate_weights(W, thV, sV, w_in, thU, sU, w_out)
+    q, s, z = quantize(Wr, bits, group)
+    lay = Layer(n_in, n_out, bits, w_in, w_out, thV, sV, thU, sU, pack(q, bits), scale_zero(s, z),
+                group)
+    return lay, q, s, z, Wr
+
+
+def linear_fwd(layer: Layer, x):
+    """y = F_U(dequant(codes) . F_V(x)); x [batch, n_in] -> y [batch, n_out] (fp64)."""
+    x = _f64(x)
+    one = x.ndim == 1
+    x2 = x.reshape(1, -1) if one else x
+    y = np.zeros((x2.shape[0], layer.n_out), np.float64)
+    st = layer.cstruct()
+    _check(lib().ora_linear_fwd(ctypes.byref(st), x2.shape[0], _d(x2), _d(y)), "linear")
+    return y.reshape(-1) if one else y
+
+
+def dense_rotated_fwd(Wr, thV, sV, w_in, thU, sU, w_out, x):
+    """F_U(W' F_V(x)) with an unquantized rotated matrix."""
+    Wr = _f64(Wr)
+    n_out, n_in = Wr.shape
+    x = _f64(x)
+    one = x.ndim == 1
+    x2 = x.reshape(1, -1) if one else x
+    y = np.zeros((x2.shape[0], n_out), np.float64)
+    thV, thU, sV, sU = _f64(thV), _f64(thU), _i8(sV), _i8(sU)
+    _check(lib().ora_dense_rotated_fwd(n_out, n_in, int(w_in), int(w_out), _d(thV),
+                                       sV.ctypes.data_as(_i8p), _d(thU), sU.ctypes.data_as(_i8p),
+                                       _d(Wr), x2.shape[0], _d(x2), _d(y)), "dense")
+    return y.reshape(-1) if one else y
+
+
+def stack_step(layers, hidden, ffn, n_heads, n_kv_heads, head_dim, x, eps=1e-5):
+    """One decode step through len(layers)//7 blocks (q, k, v, o, gate, up, down each)."""
+    assert len(layers) % 7 == 0
+    arr = (_Linear * len(layers))(*[l.cstruct() for l in layers])
+    x = _f64(x)
+    one = x.ndim == 1
+    x2 = x.reshape(1, -1) if one else x
+    out = np.zeros_like(x2)
+    _check(lib().ora_stack_step(len(layers) // 7, arr, hidden, ffn, n_heads, n_kv_heads, head_dim,
+                                float(eps), x2.shape[0], _d(x2), _d(out)), "stack")
+    return out.reshape(-1) if one else out

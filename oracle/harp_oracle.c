@@ -1,0 +1,415 @@
+/*
+ * harp_oracle.c -- TEST INFRASTRUCTURE, not part of the product.
+ *
+ * A plain, slow, fp64 CPU statement of what the rotated low-bit linear computes.
+ * Only the tests, the smoke check and the benchmark's CPU-baseline leg load it.
+ * It shares no code, header, table or helper with the CUDA library; the two meet
+ * only through the seeded input generators.
+ *
+ * Source: "HARP: Hadamard-Preconditioned Adaptive Rotation Processor for Extreme
+ * LLM Quantization" (gist.science explanation of arXiv 2605.29843):
+ *   Sec. 2.1 (Arquitetura Central)  -- the rotation is a product of sparse stride
+ *                                      stages, each a block-diagonal orthogonal B_t
+ *                                      between stride permutations; radix-2 here.
+ *   Sec. 2.2 (Pre-condicionamento)  -- block B_{t,c}(theta) = Q_{t,c}(theta) G_2 with
+ *                                      Q a Givens rotation and G_2 the normalised
+ *                                      Sylvester Hadamard; Theta = 0 gives the fixed
+ *                                      randomized Hadamard transform.
+ *   Sec. 5 (Exatidao vs. Aproximacao) -- an exact change of basis: the full-precision
+ *                                      layer is preserved, only the quantizer's
+ *                                      coordinates change.
+ * The pages leave the codebook to the backend (Sec. 2.4, Compatibilidade); the
+ * quantizer below is this library's stand-in: group-wise uniform scalar codes,
+ * b in {2,3,4} bits, an fp16 scale and an fp16 zero per group of 64 columns.
+ *
+ * Readings taken where the pages are silent (each is listed in the design notes):
+ *   - 2x2 block: Givens(theta) * H_2 = [[cos p, sin p], [sin p, -cos p]], p = pi/4 + theta.
+ *   - F = S_{m-1} ... S_1 S_0 D: the sign diagonal D first, then stage t = 0..m-1
+ *     pairs (i, i + 2^t) inside each w-wide block; pairs are numbered, per stage,
+ *     in increasing order of their first index.
+ *   - n not a power of two: F is block-diagonal with w-wide blocks (w a power of two).
+ *   - Every 2x2 block is symmetric, so F^T applies the stages in reverse, then D.
+ *
+ * Arithmetic is fp64 throughout; fp32/bf16 inputs convert to fp64 exactly.
+ * Parallelism (OpenMP) only splits independent rows or vectors; it never changes
+ * the order of any sum.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORA_OK 0
+#define ORA_EINVAL 1
+
+static const double ORA_PI = 3.14159265358979323846264338327950288;
+
+static int ora_log2_exact(int64_t w) {
+  if (w < 1) return -1;
+  int m = 0;
+  while (((int64_t)1 << m) < w) ++m;
+  return (((int64_t)1 << m) == w) ? m : -1;
+}
+
+/* ------------------------------------------------------------------ threads */
+void ora_set_threads(int n) {
+#ifdef _OPENMP
+  if (n > 0) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}
+
+int ora_get_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+
+/* ------------------------------------------------------------------ fp16
+ * IEEE 754 binary16 from fp64, round to nearest, ties to even, written from the
+ * format's definition (1 sign bit, 5 exponent bits with bias 15, 10 fraction bits;
+ * subnormals below 2^-14; overflow to infinity at and above 65520).
+ */
+uint16_t ora_f16_from_f64(double v) {
+  uint16_t sign = 0;
+  if (signbit(v)) { sign = 0x8000u; v = -v; }
+  if (isnan(v)) return (uint16_t)(sign | 0x7e00u);
+  if (v == 0.0) return sign;
+  int e2;
+  frexp(v, &e2);            /* v = f * 2^e2, f in [0.5, 1) -> exponent of v is e2 - 1 */
+  int e = e2 - 1;
+  if (e < -14) e = -14;      /* subnormal range shares the quantum 2^-24 */
+  double quantum = ldexp(1.0, e - 10);
+  double m = v / quantum;    /* exact: division by a power of two */
+  double r = nearbyint(m);   /* default rounding mode: nearest, ties to even */
+  /* r in [1024, 2048] for normals; rounding may carry into the next binade */
+  if (r >= 2048.0) { r = r / 2.0; e += 1; }
+  if (e > 15) return (uint16_t)(sign | 0x7c00u);
+  if (r < 1024.0) {          /* subnormal (only possible when e == -14) */
+    return (uint16_t)(sign | (uint16_t)r);
+  }
+  uint16_t exp_bits = (uint16_t)(e + 15);
+  uint16_t frac = (uint16_t)((int)r - 1024);
+  return (uint16_t)(sign | (exp_bits << 10) | frac);
+}
+
+double ora_f16_to_f64(uint16_t h) {
+  int s = (h >> 15) & 1, e = (h >> 10) & 0x1f, f = h & 0x3ff;
+  double v;
+  if (e == 0) v = ldexp((double)f, -24);
+  else if (e == 31) v = f ? NAN : INFINITY;
+  else v = ldexp((double)(1024 + f), e - 25);
+  return s ? -v : v;
+}
+
+/* ------------------------------------------------------------------ butterfly
+ * theta: [m][n/2] (m = log2 w), sign: [n] of +-1, x: [batch][n], in place.
+ */
+static void ora_stage(int64_t n, int64_t w, int t, const double* theta_t, double* x) {
+  const int64_t h = (int64_t)1 << t;
+  for (int64_t k = 0; k < n / w; ++k) {
+    double* blk = x + k * w;
+    for (int64_t i = 0; i < w; ++i) {
+      if (i & h) continue;
+      const int64_t p = k * (w / 2) + ((i >> (t + 1)) << t) + (i & (h - 1));
+      const double psi = ORA_PI / 4.0 + theta_t[p];
+      const double c = cos(psi), s = sin(psi);
+      const double a = blk[i], b = blk[i + h];
+      blk[i] = c * a + s * b;
+      blk[i + h] = s * a - c * b;
+    }
+  }
+}
+
+static int ora_check_bfly(int64_t n, int64_t w) {
+  if (n <= 0 || w < 2 || n % w) return -1;
+  return ora_log2_exact(w);
+}
+
+int ora_butterfly_fwd(int64_t n, int64_t w, int64_t batch, const double* theta,
+                      const int8_t* sign, double* x) {
+  const int m = ora_check_bfly(n, w);
+  if (m < 1 || batch < 0) return ORA_EINVAL;
+#pragma omp parallel for schedule(static)
+  for (int64_t b = 0; b < batch; ++b) {
+    double* v = x + b * n;
+    for (int64_t i = 0; i < n; ++i) v[i] *= (double)sign[i];
+    for (int t = 0; t < m; ++t) ora_stage(n, w, t, theta + (int64_t)t * (n / 2), v);
+  }
+  return ORA_OK;
+}
+
+int ora_butterfly_inv(int64_t n, int64_t w, int64_t batch, const double* theta,
+                      const int8_t* sign, double* x) {
+  const int m = ora_check_bfly(n, w);
+  if (m < 1 || batch < 0) return ORA_EINVAL;
+#pragma omp parallel for schedule(static)
+  for (int64_t b = 0; b < batch; ++b) {
+    double* v = x + b * n;
+    for (int t = m - 1; t >= 0; --t) ora_stage(n, w, t, theta + (int64_t)t * (n / 2), v);
+    for (int64_t i = 0; i < n; ++i) v[i] *= (double)sign[i];
+  }
+  return ORA_OK;
+}
+
+/* ------------------------------------------------------------------ rotate
+ * W' = U W V^T with V = F(theta_V, s_V, w_in) and U^T = F(theta_U, s_U, w_out):
+ * every row r becomes F_V(W_r), then every column j becomes F_U^T(W'_{:,j}).
+ * W: [n_out][n_in] row-major, in place.
+ */
+int ora_rotate_weights(int64_t n_out, int64_t n_in, int64_t w_in, int64_t w_out,
+                       const double* thV, const int8_t* sV, const double* thU,
+                       const int8_t* sU, double* W) {
+  if (ora_check_bfly(n_in, w_in) < 1 || ora_check_bfly(n_out, w_out) < 1) return ORA_EINVAL;
+  int rc = ora_butterfly_fwd(n_in, w_in, n_out, thV, sV, W);
+  if (rc) return rc;
+  int bad = 0;
+#pragma omp parallel
+  {
+    double* col = (double*)malloc(sizeof(double) * (size_t)n_out);
+    if (!col) {
+#pragma omp atomic write
+      bad = 1;
+    } else {
+#pragma omp for schedule(static)
+      for (int64_t j = 0; j < n_in; ++j) {
+        for (int64_t r = 0; r < n_out; ++r) col[r] = W[r * n_in + j];
+        ora_butterfly_inv(n_out, w_out, 1, thU, sU, col);
+        for (int64_t r = 0; r < n_out; ++r) W[r * n_in + j] = col[r];
+      }
+      free(col);
+    }
+  }
+  return bad ? ORA_EINVAL : ORA_OK;
+}
+
+/* ------------------------------------------------------------------ quantize
+ * Per row r and group g (group consecutive columns of W'):
+ *   zero16  = fp16(min), scale16 = fp16((max - min) / (2^b - 1)), 1 if that is 0,
+ *   q       = clamp(round_half_even((w - zero16) / scale16), 0, 2^b - 1),
+ *   dequant = scale16 * q + zero16.
+ * q: [n_out][n_in] one code per byte; scale16, zero16: [n_out][n_in/group] fp16 bits.
+ */
+int ora_quantize(int64_t n_out, int64_t n_in, int bits, int group, const double* Wr,
+                 uint8_t* q, uint16_t* scale16, uint16_t* zero16) {
+  if (bits < 2 || bits > 4 || group < 1 || n_in % group) return ORA_EINVAL;
+  const double L = (double)((1 << bits) - 1);
+  const int64_t ng = n_in / group;
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < n_out; ++r) {
+    for (int64_t g = 0; g < ng; ++g) {
+      const double* w = Wr + r * n_in + g * group;
+      double mn = w[0], mx = w[0];
+      for (int j = 1; j < group; ++j) {
+        if (w[j] < mn) mn = w[j];
+        if (w[j] > mx) mx = w[j];
+      }
+      uint16_t zb = ora_f16_from_f64(mn);
+      uint16_t sb = ora_f16_from_f64((mx - mn) / L);
+      if (ora_f16_to_f64(sb) == 0.0) sb = 0x3c00u; /* 1.0 */
+      const double z = ora_f16_to_f64(zb), s = ora_f16_to_f64(sb);
+      for (int j = 0; j < group; ++j) {
+        double v = nearbyint((w[j] - z) / s);
+        if (!(v >= 0.0)) v = 0.0; /* also maps NaN to 0 */
+        if (v > L) v = L;
+        q[r * n_in + g * group + j] = (uint8_t)v;
+      }
+      scale16[r * ng + g] = sb;
+      zero16[r * ng + g] = zb;
+    }
+  }
+  return ORA_OK;
+}
+
+/* ------------------------------------------------------------------ pack
+ * Canonical packed layout, row-major by output row; e = r * n_in + j:
+ *   b = 2 or 4: code e sits in little-endian 32-bit word (e * b) / 32 at bit (e * b) % 32;
+ *   b = 3     : a 2-bit plane of (q & 3) laid out as for b = 2 (n_out*n_in/4 bytes),
+ *               then a 1-bit plane of (q >> 2): word e / 32, bit e % 32.
+ * Total bytes: n_out * n_in * b / 8.
+ */
+static void ora_put_bits(uint8_t* buf, int64_t bitpos, unsigned v, int nb) {
+  for (int k = 0; k < nb; ++k) {
+    const int64_t p = bitpos + k;
+    const uint8_t bit = (uint8_t)((v >> k) & 1u);
+    /* little-endian words: bit p of the stream is bit (p % 8) of byte p / 8 */
+    buf[p >> 3] = (uint8_t)((buf[p >> 3] & ~(1u << (p & 7))) | (bit << (p & 7)));
+  }
+}
+
+static unsigned ora_get_bits(const uint8_t* buf, int64_t bitpos, int nb) {
+  unsigned v = 0;
+  for (int k = 0; k < nb; ++k) {
+    const int64_t p = bitpos + k;
+    v |= (unsigned)((buf[p >> 3] >> (p & 7)) & 1u) << k;
+  }
+  return v;
+}
+
+int64_t ora_packed_bytes(int64_t n_out, int64_t n_in, int bits) {
+  return n_out * n_in * bits / 8;
+}
+
+int ora_pack(int64_t n_out, int64_t n_in, int bits, const uint8_t* q, uint8_t* packed) {
+  if (bits < 2 || bits > 4 || n_in % 32) return ORA_EINVAL;
+  const int64_t N = n_out * n_in;
+  memset(packed, 0, (size_t)ora_packed_bytes(n_out, n_in, bits));
+  if (bits == 3) {
+    uint8_t* hi = packed + N / 4;
+    for (int64_t e = 0; e < N; ++e) {
+      ora_put_bits(packed, e * 2, q[e] & 3u, 2);
+      ora_put_bits(hi, e, (q[e] >> 2) & 1u, 1);
+    }
+  } else {
+    for (int64_t e = 0; e < N; ++e) ora_put_bits(packed, e * bits, q[e], bits);
+  }
+  return ORA_OK;
+}
+
+int ora_unpack(int64_t n_out, int64_t n_in, int bits, const uint8_t* packed, uint8_t* q) {
+  if (bits < 2 || bits > 4 || n_in % 32) return ORA_EINVAL;
+  const int64_t N = n_out * n_in;
+  if (bits == 3) {
+    const uint8_t* hi = packed + N / 4;
+    for (int64_t e = 0; e < N; ++e)
+      q[e] = (uint8_t)(ora_get_bits(packed, e * 2, 2) | (ora_get_bits(hi, e, 1) << 2));
+  } else {
+    for (int64_t e = 0; e < N; ++e) q[e] = (uint8_t)ora_get_bits(packed, e * bits, bits);
+  }
+  return ORA_OK;
+}
+
+/* ------------------------------------------------------------------ linear */
+typedef struct {
+  int64_t n_in, n_out, w_in, w_out;
+  int64_t bits, group;
+  const double* thV;
+  const int8_t* sV;
+  const double* thU;
+  const int8_t* sU;
+  const uint8_t* packed;      /* canonical layout above */
+  const uint16_t* scale_zero; /* [n_out][n_in/group][2]: {scale16, zero16} */
+} ora_linear;
+
+/* code of element (r, j) read straight from the canonical packed layout */
+static unsigned ora_code_at(const ora_linear* L, int64_t r, int64_t j) {
+  const int64_t e = r * L->n_in + j;
+  if (L->bits == 3) {
+    const uint8_t* hi = L->packed + (L->n_out * L->n_in) / 4;
+    return ora_get_bits(L->packed, e * 2, 2) | (ora_get_bits(hi, e, 1) << 2);
+  }
+  return ora_get_bits(L->packed, e * L->bits, (int)L->bits);
+}
+
+/* y = F_U( dequant(codes) . F_V(x) ), x: [batch][n_in], y: [batch][n_out] */
+int ora_linear_fwd(const ora_linear* L, int64_t batch, const double* x, double* y) {
+  if (ora_check_bfly(L->n_in, L->w_in) < 1 || ora_check_bfly(L->n_out, L->w_out) < 1) return ORA_EINVAL;
+  if (L->group < 1 || L->n_in % L->group) return ORA_EINVAL;
+  const int64_t n_in = L->n_in, n_out = L->n_out, ng = n_in / L->group;
+  double* xt = (double*)malloc(sizeof(double) * (size_t)(batch * n_in));
+  if (!xt && batch) return ORA_EINVAL;
+  memcpy(xt, x, sizeof(double) * (size_t)(batch * n_in));
+  ora_butterfly_fwd(n_in, L->w_in, batch, L->thV, L->sV, xt);
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < n_out; ++r) {
+    for (int64_t b = 0; b < batch; ++b) {
+      double acc = 0.0;
+      for (int64_t j = 0; j < n_in; ++j) {
+        const int64_t g = j / L->group;
+        const double s = ora_f16_to_f64(L->scale_zero[(r * ng + g) * 2 + 0]);
+        const double z = ora_f16_to_f64(L->scale_zero[(r * ng + g) * 2 + 1]);
+        const double wdq = s * (double)ora_code_at(L, r, j) + z;
+        acc += wdq * xt[b * n_in + j];
+      }
+      y[b * n_out + r] = acc;
+    }
+  }
+  free(xt);
+  return ora_butterfly_fwd(n_out, L->w_out, batch, L->thU, L->sU, y);
+}
+
+/* Same composition with an unquantized rotated matrix Wr (used to check that the
+ * rotation is an exact change of basis: F_U(Wr F_V(x)) must equal W x). */
+int ora_dense_rotated_fwd(int64_t n_out, int64_t n_in, int64_t w_in, int64_t w_out,
+                          const double* thV, const int8_t* sV, const double* thU,
+                          const int8_t* sU, const double* Wr, int64_t batch,
+                          const double* x, double* y) {
+  if (ora_check_bfly(n_in, w_in) < 1 || ora_check_bfly(n_out, w_out) < 1) return ORA_EINVAL;
+  double* xt = (double*)malloc(sizeof(double) * (size_t)(batch * n_in));
+  if (!xt && batch) return ORA_EINVAL;
+  memcpy(xt, x, sizeof(double) * (size_t)(batch * n_in));
+  ora_butterfly_fwd(n_in, w_in, batch, thV, sV, xt);
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < n_out; ++r)
+    for (int64_t b = 0; b < batch; ++b) {
+      double acc = 0.0;
+      for (int64_t j = 0; j < n_in; ++j) acc += Wr[r * n_in + j] * xt[b * n_in + j];
+      y[b * n_out + r] = acc;
+    }
+  free(xt);
+  return ora_butterfly_fwd(n_out, w_out, batch, thU, sU, y);
+}
+
+/* ------------------------------------------------------------------ stack step
+ * One decode step through n_layers Llama-shaped blocks whose seven linears are all
+ * rotated low-bit layers, in the order q, k, v, o, gate, up, down:
+ *   n1 = rms(x); v = v_proj(n1); a = v repeated per key/value group (a one-key
+ *   attention returns its value; q_proj and k_proj are evaluated all the same);
+ *   h = x + o_proj(a); n2 = rms(h); x' = h + down(silu(gate(n2)) * up(n2)),
+ *   rms(u) = u / sqrt(mean(u^2) + eps), silu(g) = g / (1 + exp(-g)).
+ * x, out: [batch][hidden].
+ */
+static void ora_rms(int64_t n, double eps, const double* u, double* o) {
+  double ss = 0.0;
+  for (int64_t i = 0; i < n; ++i) ss += u[i] * u[i];
+  const double inv = 1.0 / sqrt(ss / (double)n + eps);
+  for (int64_t i = 0; i < n; ++i) o[i] = u[i] * inv;
+}
+
+int ora_stack_step(int64_t n_layers, const ora_linear* lin, int64_t hidden, int64_t ffn,
+                   int64_t n_heads, int64_t n_kv_heads, int64_t head_dim, double eps,
+                   int64_t batch, const double* x, double* out) {
+  if (n_kv_heads < 1 || n_heads % n_kv_heads) return ORA_EINVAL;
+  const int64_t dq = n_heads * head_dim, dkv = n_kv_heads * head_dim, rep = n_heads / n_kv_heads;
+  const size_t B = (size_t)batch;
+  double* h = (double*)malloc(sizeof(double) * B * (size_t)hidden);
+  double* nrm = (double*)malloc(sizeof(double) * B * (size_t)hidden);
+  double* q = (double*)malloc(sizeof(double) * B * (size_t)dq);
+  double* k = (double*)malloc(sizeof(double) * B * (size_t)dkv);
+  double* v = (double*)malloc(sizeof(double) * B * (size_t)dkv);
+  double* a = (double*)malloc(sizeof(double) * B * (size_t)dq);
+  double* o = (double*)malloc(sizeof(double) * B * (size_t)hidden);
+  double* g = (double*)malloc(sizeof(double) * B * (size_t)ffn);
+  double* u = (double*)malloc(sizeof(double) * B * (size_t)ffn);
+  int rc = ORA_OK;
+  if (!h || !nrm || !q || !k || !v || !a || !o || !g || !u) { rc = ORA_EINVAL; goto done; }
+  memcpy(out, x, sizeof(double) * B * (size_t)hidden);
+  for (int64_t l = 0; l < n_layers && rc == ORA_OK; ++l) {
+    const ora_linear* L = lin + 7 * l;
+    for (int64_t b = 0; b < batch; ++b) ora_rms(hidden, eps, out + b * hidden, nrm + b * hidden);
+    rc |= ora_linear_fwd(&L[0], batch, nrm, q);
+    rc |= ora_linear_fwd(&L[1], batch, nrm, k);
+    rc |= ora_linear_fwd(&L[2], batch, nrm, v);
+    for (int64_t b = 0; b < batch; ++b)
+      for (int64_t hh = 0; hh < n_heads; ++hh)
+        for (int64_t d = 0; d < head_dim; ++d)
+          a[b * dq + hh * head_dim + d] = v[b * dkv + (hh / rep) * head_dim + d];
+    rc |= ora_linear_fwd(&L[3], batch, a, o);
+    for (size_t i = 0; i < B * (size_t)hidden; ++i) h[i] = out[i] + o[i];
+    for (int64_t b = 0; b < batch; ++b) ora_rms(hidden, eps, h + b * hidden, nrm + b * hidden);
+    rc |= ora_linear_fwd(&L[4], batch, nrm, g);
+    rc |= ora_linear_fwd(&L[5], batch, nrm, u);
+    for (size_t i = 0; i < B * (size_t)ffn; ++i) g[i] = g[i] / (1.0 + exp(-g[i])) * u[i];
+    rc |= ora_linear_fwd(&L[6], batch, g, o);
+    for (size_t i = 0; i < B * (size_t)hidden; ++i) out[i] = h[i] + o[i];
+  }
+done:
+  free(h); free(nrm); free(q); free(k); free(v); free(a); free(o); free(g); free(u);
+  return rc;
+}

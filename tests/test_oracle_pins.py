@@ -1,0 +1,365 @@
+"""Pins for the fp64 oracle, checked against what the HARP pages and mathematics fix.
+
+Source: "HARP: Hadamard-Preconditioned Adaptive Rotation Processor for Extreme LLM
+Quantization" (gist.science): Sec. 2.1 (stride stages of block-diagonal orthogonal
+B_t between stride permutations), Sec. 2.2 (B = Q(theta) G_2, Givens Q, normalised
+Sylvester G_2; Theta = 0 recovers the randomized Hadamard transform), Sec. 1 and 5
+(an exact, orthogonal change of basis that preserves the full-precision layer).
+Each test is chosen so that a plausible slip in the oracle (a dropped stage, a
+wrong sign, a transposed factor, a mis-numbered pair, a wrong rounding rule) fails.
+"""
+import math
+
+import numpy as np
+import pytest
+import scipy.linalg
+
+from conftest import read_golden
+
+pytestmark = pytest.mark.filterwarnings("ignore::RuntimeWarning")
+
+
+def _rand_theta(rng, n, w, scale):
+    m = int(math.log2(w))
+    return rng.uniform(-scale, scale, size=(m, n // 2))
+
+
+def _rand_sign(rng, n):
+    return (rng.integers(0, 2, n) * 2 - 1).astype(np.int8)
+
+
+def _dense(ora, n, w, theta, sign, inv=False):
+    f = ora.butterfly_inv if inv else ora.butterfly_fwd
+    # column j of the matrix is F e_j; the oracle acts on rows of a batch
+    return f(np.eye(n), theta, sign, w).T
+
+
+# ------------------------------------------------------------------ fp16 rounding
+def test_f16_conversion_matches_numpy(ora):
+    """The oracle's own fp64 -> fp16 rounding agrees with numpy's correctly rounded
+    conversion on random values, exact ties, subnormals and the overflow edge."""
+    rng = np.random.default_rng(1)
+    vals = np.concatenate([
+        rng.standard_normal(3000) * 0.02, rng.standard_normal(1000) * 300.0,
+        rng.uniform(-1e-4, 1e-4, 1000), rng.uniform(-7e-8, 7e-8, 300),
+        # exact midpoints between neighbouring fp16 values (ties to even)
+        (np.arange(1024, 1100) + 0.5) * 2.0 ** -10, (np.arange(1, 60) + 0.5) * 2.0 ** -24,
+        [65504.0, 65519.0, 65519.999, 65520.0, 70000.0, -65520.0, 2.0 ** -24, 2.0 ** -25,
+         3 * 2.0 ** -26, 2.0 ** -14, 0.0, -0.0, 1.0 / 3.0],
+    ])
+    got = ora.f16_from_f64(vals)
+    want = vals.astype(np.float16).view(np.uint16)
+    assert np.array_equal(got, want)
+
+
+def test_f16_decode_all_bit_patterns(ora):
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    got = ora.f16_to_f64(bits)
+    want = bits.view(np.float16).astype(np.float64)
+    nan = np.isnan(want)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], want[~nan])
+
+
+# ------------------------------------------------------------------ P1: Theta = 0
+@pytest.mark.parametrize("n", [2, 4, 8, 16, 32, 64])
+def test_theta0_is_sylvester_hadamard(ora, n):
+    """F(0, s, n) = H_n diag(s) / sqrt(n) with H_n the Sylvester Hadamard matrix."""
+    rng = np.random.default_rng(n)
+    s = _rand_sign(rng, n)
+    M = _dense(ora, n, n, np.zeros((int(math.log2(n)), n // 2)), s)
+    want = scipy.linalg.hadamard(n) @ np.diag(s.astype(float)) / math.sqrt(n)
+    assert np.max(np.abs(M - want)) < 1e-14
+
+
+@pytest.mark.parametrize("n", [1024, 2048])
+def test_theta0_hadamard_spot(ora, n):
+    rng = np.random.default_rng(7)
+    s = _rand_sign(rng, n)
+    x = rng.standard_normal((3, n))
+    got = ora.butterfly_fwd(x, np.zeros((int(math.log2(n)), n // 2)), s, n)
+    want = (x * s) @ scipy.linalg.hadamard(n).T / math.sqrt(n)
+    assert np.max(np.abs(got - want)) < 1e-12
+
+
+def test_theta0_block_diagonal_hadamard(ora):
+    n, w = 64, 16
+    s = _rand_sign(np.random.default_rng(3), n)
+    M = _dense(ora, n, w, np.zeros((4, n // 2)), s)
+    want = np.kron(np.eye(n // w), scipy.linalg.hadamard(w)) @ np.diag(s.astype(float)) / 4.0
+    assert np.max(np.abs(M - want)) < 1e-14
+
+
+# ------------------------------------------------------------------ golden values
+def test_golden_butterfly(ora):
+    for (nw, th, sg, x, want) in read_golden("butterfly_examples.txt"):
+        n, w = int(nw[0]), int(nw[1])
+        theta = np.array([float(t) for t in th]).reshape(int(math.log2(w)), n // 2)
+        got = ora.butterfly_fwd(np.array([float(t) for t in x]), theta,
+                                np.array([int(t) for t in sg], np.int8), w)
+        assert np.allclose(got, [float(t) for t in want], rtol=0, atol=1e-15), (nw, got, want)
+
+
+# ------------------------------------------------------------------ P2: orthogonality
+@pytest.mark.parametrize("n,w,scale", [(4096, 4096, 0.05), (11008, 256, 0.05),
+                                       (2048, 512, 3.0), (28672, 4096, 0.05)])
+def test_orthogonal_norm_and_inverse(ora, n, w, scale):
+    rng = np.random.default_rng(n + w)
+    th, s = _rand_theta(rng, n, w, scale), _rand_sign(rng, n)
+    x = rng.standard_normal((2, n))
+    y = ora.butterfly_fwd(x, th, s, w)
+    assert np.allclose(np.linalg.norm(y, axis=1), np.linalg.norm(x, axis=1), rtol=1e-13, atol=0)
+    assert np.max(np.abs(ora.butterfly_inv(y, th, s, w) - x)) < 1e-12
+    assert np.max(np.abs(ora.butterfly_fwd(ora.butterfly_inv(x, th, s, w), th, s, w) - x)) < 1e-12
+
+
+@pytest.mark.parametrize("n,w", [(16, 16), (64, 64), (64, 8)])
+def test_dense_orthogonal_and_transpose(ora, n, w):
+    rng = np.random.default_rng(11)
+    th, s = _rand_theta(rng, n, w, 1.0), _rand_sign(rng, n)
+    M = _dense(ora, n, w, th, s)
+    assert np.max(np.abs(M.T @ M - np.eye(n))) < 1e-14
+    assert np.max(np.abs(_dense(ora, n, w, th, s, inv=True) - M.T)) < 1e-14
+
+
+# ------------------------------------------------------------------ structure of the stages
+def _stride_perm(n, w, t):
+    """Permutation matrix P that lists, block by block of 2^(t+1) coordinates, the
+    pairs (i, i + 2^t) next to each other (interleaving the two halves of the block)."""
+    h = 1 << t
+    order = []
+    for base in range(0, n, 2 * h):
+        for i in range(h):
+            order += [base + i, base + i + h]
+    P = np.zeros((n, n))
+    P[np.arange(n), order] = 1.0
+    return P
+
+
+def _page_block(theta):
+    """B(theta) = Q(theta) G_2: Givens rotation times the normalised Sylvester H_2."""
+    c, s = math.cos(theta), math.sin(theta)
+    Q = np.array([[c, -s], [s, c]])
+    G2 = np.array([[1.0, 1.0], [1.0, -1.0]]) / math.sqrt(2.0)
+    return Q @ G2
+
+
+def _page_butterfly(n, w, theta, sign):
+    """Dense F built from the pages' description: D first, then for t = 0..m-1 the
+    block-diagonal B_t conjugated by the stride permutation of stage t; pair c of
+    stage t takes theta[t][c]."""
+    m = int(math.log2(w))
+    F = np.diag(sign.astype(float))
+    for t in range(m):
+        P = _stride_perm(n, w, t)
+        Bt = scipy.linalg.block_diag(*[_page_block(theta[t][c]) for c in range(n // 2)])
+        F = P.T @ Bt @ P @ F
+    return F
+
+
+@pytest.mark.parametrize("n,w", [(8, 8), (16, 16), (32, 32), (32, 8), (64, 16)])
+def test_stages_match_stride_permutation_construction(ora, n, w):
+    rng = np.random.default_rng(n * 7 + w)
+    th, s = _rand_theta(rng, n, w, 1.5), _rand_sign(rng, n)
+    assert np.max(np.abs(_dense(ora, n, w, th, s) - _page_butterfly(n, w, th, s))) < 1e-13
+
+
+def test_single_angle_moves_only_its_pair(ora):
+    """Changing theta[t][p] alone changes the output exactly as the page block predicts."""
+    n = w = 16
+    rng = np.random.default_rng(5)
+    s = _rand_sign(rng, n)
+    base = np.zeros((4, n // 2))
+    for t in range(4):
+        for p in (0, 3, 7):
+            th = base.copy()
+            th[t, p] = 0.3
+            assert np.max(np.abs(_dense(ora, n, w, th, s) - _page_butterfly(n, w, th, s))) < 1e-14
+
+
+# ------------------------------------------------------------------ P6: block diagonal
+def test_block_diagonal_equals_independent_blocks(ora):
+    n, w = 11008, 256
+    rng = np.random.default_rng(9)
+    th, s = _rand_theta(rng, n, w, 0.05), _rand_sign(rng, n)
+    x = rng.standard_normal(n)
+    got = ora.butterfly_fwd(x, th, s, w)
+    for k in (0, 17, 42):
+        sl = slice(k * w, (k + 1) * w)
+        th_k = th[:, k * (w // 2):(k + 1) * (w // 2)]
+        assert np.max(np.abs(got[sl] - ora.butterfly_fwd(x[sl], th_k, s[sl], w))) < 1e-15
+
+
+# ------------------------------------------------------------------ theta = -pi/4: diagonal
+def test_theta_minus_quarter_pi_is_diagonal(ora):
+    """psi = 0 makes every block diag(1, -1): F = diag(s_i (-1)^popcount(i mod w))."""
+    n, w = 256, 64
+    s = _rand_sign(np.random.default_rng(2), n)
+    th = np.full((6, n // 2), -math.pi / 4)
+    x = np.random.default_rng(3).standard_normal(n)
+    par = np.array([(-1.0) ** bin(i % w).count("1") for i in range(n)])
+    assert np.max(np.abs(ora.butterfly_fwd(x, th, s, w) - s * par * x)) < 1e-15
+
+
+# ------------------------------------------------------------------ P3: exact change of basis
+@pytest.mark.parametrize("n_out,n_in,w_in,w_out", [(256, 512, 512, 256), (384, 256, 256, 128),
+                                                   (128, 1024, 64, 128)])
+def test_rotation_is_exact_change_of_basis(ora, n_out, n_in, w_in, w_out):
+    rng = np.random.default_rng(n_out + n_in)
+    W = rng.standard_normal((n_out, n_in)) * 0.02
+    thV, sV = _rand_theta(rng, n_in, w_in, 0.5), _rand_sign(rng, n_in)
+    thU, sU = _rand_theta(rng, n_out, w_out, 0.5), _rand_sign(rng, n_out)
+    Wr = ora.rotate_weights(W, thV, sV, w_in, thU, sU, w_out)
+    x = rng.standard_normal((3, n_in))
+    y = ora.dense_rotated_fwd(Wr, thV, sV, w_in, thU, sU, w_out, x)
+    want = x @ W.T
+    assert np.linalg.norm(y - want) / np.linalg.norm(want) < 1e-12
+    # and W' = U W V^T with V = F_V, U = F_U^T built from the pages' construction
+    if n_out <= 256 and n_in <= 512:
+        FV = _page_butterfly(n_in, w_in, thV, sV)
+        FU = _page_butterfly(n_out, w_out, thU, sU)
+        assert np.max(np.abs(Wr - FU.T @ W @ FV.T)) < 1e-13
+
+
+# ------------------------------------------------------------------ P4: quantizer
+def _deq(q, s16, z16, ora, group=64):
+    s = ora.f16_to_f64(s16).repeat(group, axis=1)
+    z = ora.f16_to_f64(z16).repeat(group, axis=1)
+    return s * q + z, s, z
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_quantizer_is_nearest_level(ora, bits):
+    rng = np.random.default_rng(bits)
+    W = rng.standard_normal((48, 512)) * 0.02
+    W[:, 5] *= 20.0
+    W[3, 64:128] = 0.125           # constant group -> scale 1
+    W[4, 128:192] = rng.standard_normal(64) * 1e-7   # tiny range
+    q, s16, z16 = ora.quantize(W, bits)
+    L = (1 << bits) - 1
+    assert q.max() <= L
+    mn = W.reshape(48, 8, 64).min(-1)
+    mx = W.reshape(48, 8, 64).max(-1)
+    want_z = mn.astype(np.float16).view(np.uint16)
+    want_s = ((mx - mn) / L).astype(np.float16).view(np.uint16)
+    want_s = np.where(want_s == 0, np.uint16(0x3C00), want_s)
+    assert np.array_equal(z16, want_z) and np.array_equal(s16, want_s)
+    deq, s, z = _deq(q, s16, z16, ora)
+    levels = s[..., None] * np.arange(L + 1) + z[..., None]
+    dist = np.abs(W[..., None] - levels)
+    best = dist.min(-1)
+    mine = np.abs(W - deq)
+    assert np.all(mine <= best * (1 + 1e-12) + 1e-300)
+    unclamped = (q > 0) & (q < L)
+    assert np.all(mine[unclamped] <= s[unclamped] / 2 * (1 + 1e-9))
+    ulp_z = np.abs(np.spacing(z.astype(np.float16)).astype(np.float64))
+    assert np.all(mine <= s / 2 * (1 + 1e-9) + ulp_z + 1e-300)
+
+
+def test_golden_quantize(ora):
+    for (bits, vals, sb, zb, codes) in read_golden("quantize_examples.txt"):
+        b = int(bits[0])
+        W = np.array([[float(v) for v in vals]])
+        assert W.shape == (1, 64)
+        q, s16, z16 = ora.quantize(W, b)
+        assert s16[0, 0] == int(sb[0], 16) and z16[0, 0] == int(zb[0], 16)
+        assert q[0].tolist() == [int(c) for c in codes]
+
+
+# ------------------------------------------------------------------ P5: packing
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_pack_roundtrip(ora, bits):
+    rng = np.random.default_rng(40 + bits)
+    q = rng.integers(0, 1 << bits, (12, 320)).astype(np.uint8)
+    p = ora.pack(q, bits)
+    assert p.size == 12 * 320 * bits // 8
+    assert np.array_equal(ora.unpack(p, 12, 320, bits), q)
+
+
+def test_golden_pack(ora):
+    for (bits, codes, want) in read_golden("pack_examples.txt"):
+        b = int(bits[0])
+        q = np.array([[int(c) for c in codes]], np.uint8)
+        assert q.shape == (1, 64)
+        assert ora.pack(q, b).tolist() == [int(h, 16) for h in want]
+
+
+# ------------------------------------------------------------------ P8: brute-force linear
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_linear_matches_dense_brute_force(ora, bits):
+    n_out, n_in, w_in, w_out = 64, 128, 64, 32
+    rng = np.random.default_rng(100 + bits)
+    W = rng.standard_normal((n_out, n_in)) * 0.02
+    thV, sV = _rand_theta(rng, n_in, w_in, 0.3), _rand_sign(rng, n_in)
+    thU, sU = _rand_theta(rng, n_out, w_out, 0.3), _rand_sign(rng, n_out)
+    lay, q, s16, z16, Wr = ora.prepare_layer(W, bits, w_in, w_out, thV, sV, thU, sU)
+    deq, _, _ = _deq(q, s16, z16, ora)
+    FV = _page_butterfly(n_in, w_in, thV, sV)
+    FU = _page_butterfly(n_out, w_out, thU, sU)
+    x = rng.standard_normal((4, n_in))
+    want = (FU @ deq @ FV @ x.T).T
+    got = ora.linear_fwd(lay, x)
+    assert np.max(np.abs(got - want)) < 1e-13 * np.max(np.abs(want))
+    # quantization error stays at the level the half-step bound allows
+    assert np.linalg.norm(got - x @ W.T) / np.linalg.norm(x @ W.T) < {2: 0.6, 3: 0.3, 4: 0.15}[bits]
+
+
+def test_linear_integer_special_case(ora):
+    """theta = -pi/4 (diagonal butterflies), scale 1, zero 0: y = D_U Q D_V x exactly."""
+    n_out, n_in = 64, 128
+    rng = np.random.default_rng(8)
+    q = rng.integers(0, 4, (n_out, n_in)).astype(np.uint8)
+    sz = np.zeros((n_out, n_in // 64, 2), np.uint16)
+    sz[..., 0] = 0x3C00
+    thV = np.full((7, n_in // 2), -math.pi / 4)
+    thU = np.full((6, n_out // 2), -math.pi / 4)
+    sV, sU = _rand_sign(rng, n_in), _rand_sign(rng, n_out)
+    lay = ora.Layer(n_in, n_out, 2, n_in, n_out, thV, sV, thU, sU, ora.pack(q, 2), sz)
+    x = rng.integers(-8, 9, (2, n_in)).astype(float)
+    dV = sV * np.array([(-1.0) ** bin(i).count("1") for i in range(n_in)])
+    dU = sU * np.array([(-1.0) ** bin(i).count("1") for i in range(n_out)])
+    want = ((q.astype(float) @ (x * dV).T).T) * dU
+    assert np.array_equal(ora.linear_fwd(lay, x), want)
+
+
+# ------------------------------------------------------------------ stack step
+def _tiny_stack(ora, n_layers, zero=(), seed=0):
+    hidden, ffn, nh, nkv, hd = 128, 192, 4, 2, 32
+    shapes = [(nh * hd, hidden), (nkv * hd, hidden), (nkv * hd, hidden), (hidden, nh * hd),
+              (ffn, hidden), (ffn, hidden), (hidden, ffn)]
+    rng = np.random.default_rng(seed)
+    layers = []
+    for l in range(n_layers):
+        for i, (n_out, n_in) in enumerate(shapes):
+            W = rng.standard_normal((n_out, n_in)) * 0.05
+            if i in zero:
+                W[:] = 0.0
+            w_in, w_out = (64 if n_in == ffn else n_in), (64 if n_out == ffn else n_out)
+            thV, sV = _rand_theta(rng, n_in, w_in, 0.05), _rand_sign(rng, n_in)
+            thU, sU = _rand_theta(rng, n_out, w_out, 0.05), _rand_sign(rng, n_out)
+            layers.append(ora.prepare_layer(W, 2, w_in, w_out, thV, sV, thU, sU)[0])
+    return layers, (hidden, ffn, nh, nkv, hd)
+
+
+def test_stack_zero_output_projections_is_identity(ora):
+    """With o_proj and down_proj weights all zero both residual branches vanish."""
+    layers, dims = _tiny_stack(ora, 2, zero=(3, 6))
+    x = np.random.default_rng(1).standard_normal((2, dims[0]))
+    assert np.array_equal(ora.stack_step(layers, *dims, x), x)
+
+
+def test_stack_q_k_do_not_reach_output(ora):
+    """A one-key attention returns its value: q_proj and k_proj cannot change the step."""
+    a, dims = _tiny_stack(ora, 1, seed=3)
+    b, _ = _tiny_stack(ora, 1, seed=4)
+    mixed = [b[0], b[1]] + a[2:]
+    x = np.random.default_rng(2).standard_normal((1, dims[0]))
+    assert np.array_equal(ora.stack_step(a, *dims, x), ora.stack_step(mixed, *dims, x))
+
+
+def test_stack_zero_up_kills_mlp(ora):
+    """silu(g) * 0 = 0: with up_proj zero the MLP branch is exactly zero."""
+    layers, dims = _tiny_stack(ora, 1, zero=(5,), seed=6)
+    ref, _ = _tiny_stack(ora, 1, zero=(5, 6), seed=6)
+    x = np.random.default_rng(7).standard_normal((1, dims[0]))
+    assert np.array_equal(ora.stack_step(layers, *dims, x), ora.stack_step(ref, *dims, x))
