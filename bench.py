@@ -1,0 +1,312 @@
+"""Benchmark: batch-1 decode through a Llama-2-7B-shaped stack of rotated 2-bit linears.
+
+One step = one decode token through 32 blocks of seven rotated low-bit linears
+(q/k/v/o 4096x4096, gate/up 11008x4096, down 4096x11008; 256-wide butterfly blocks
+on the 11008 side) with RMSNorm, residual adds, SiLU*up and the one-key attention
+stand-in between them -- every step of the hot path, in the library's kernels.
+Weights are random-initialised on the device (N(0, 0.02^2), 0.1% outlier columns x20)
+and rotated/quantized by the library; inputs are seeded N(0,1) bf16 vectors.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0). With N > 1 (torchrun) every rank runs an independent
+replica (the path has no exchange step); the time is the max over ranks.
+`--impl reference` times the fp64 CPU oracle on the host cores on a bounded sample of
+the same workload (one block of the stack per step), in the same metric.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+N_LAYERS = 32
+HIDDEN, FFN, NH, NKV, HD = 4096, 11008, 32, 32, 128
+BITS, GROUP, BATCH = 2, 64, 1
+WORKLOAD = 4
+METRIC = "rotated 2-bit linear: decode tokens/s (7B-shaped, batch 1) and HBM GB/s vs roofline"
+CONFIG_NAME = "llama2-7b-shaped 32-layer rotated 2-bit linear stack, batch-1 decode"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--layers", type=int, default=N_LAYERS)
+    ap.add_argument("--cpu-sample-layers", type=int, default=1)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def shapes():
+    from rotated_bit_matmul_b200 import synth
+    return synth.llama7b_linears()
+
+
+def algorithmic_bytes_per_step(n_layers, batch=BATCH, bits=BITS):
+    """Packed codes + fp16 scale/zero + fp32 activations in and out, per linear."""
+    tot = 0
+    for s in shapes():
+        tot += s.n_out * s.n_in * bits // 8 + s.n_out * (s.n_in // GROUP) * 4 + 4 * batch * (s.n_in + s.n_out)
+    return tot * n_layers
+
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks sampling
+class ClockSampler:
+    def __init__(self, index=0):
+        self.index = index
+        self.samples = []
+        self._stop = threading.Event()
+        self._th = None
+
+    def _run(self):
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                                     "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            return
+        try:
+            while not self._stop.is_set():
+                line = proc.stdout.readline()
+                if not line:
+                    break
+                self.samples.append([t.strip() for t in line.split(",")])
+        finally:
+            proc.terminate()
+
+    def __enter__(self):
+        self._th = threading.Thread(target=self._run, daemon=True)
+        self._th.start()
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        self._th.join(timeout=3)
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sm = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        mx = [float(s[2]) for s in self.samples if s[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for s in self.samples for i in range(4) if len(s) > 5 + i and s[5 + i] == "Active"})
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ CPU oracle sample
+def cpu_oracle_sample(sample_layers=1):
+    """Times the fp64 oracle on `sample_layers` blocks of the 7B stack (one token) and
+    scales to the 32-block step. Returns (tokens_per_s, seconds_per_block, threads)."""
+    import oracle
+    from rotated_bit_matmul_b200 import synth
+    threads = len(os.sched_getaffinity(0))
+    oracle.set_threads(threads)
+    lays = []
+    for l in range(sample_layers):
+        for i, s in enumerate(shapes()):
+            W = synth.weights(s.n_out, s.n_in, WORKLOAD, l, i)
+            thV, sV = synth.butterfly_params(s.n_in, s.w_in, WORKLOAD, l, i, "V")
+            thU, sU = synth.butterfly_params(s.n_out, s.w_out, WORKLOAD, l, i, "U")
+            lays.append(oracle.prepare_layer(W, BITS, s.w_in, s.w_out, thV, sV, thU, sU)[0])
+    x = synth.activations(BATCH, HIDDEN, WORKLOAD, 0).astype(np.float64)
+    t0 = time.perf_counter()
+    oracle.stack_step(lays, HIDDEN, FFN, NH, NKV, HD, x)
+    dt = time.perf_counter() - t0
+    per_block = dt / sample_layers
+    return 1.0 / (per_block * N_LAYERS), per_block, threads
+
+
+# ------------------------------------------------------------------ GPU path
+def build_stack(n_layers, device):
+    import torch
+    import rotated_bit_matmul_b200 as rb
+    from rotated_bit_matmul_b200 import synth
+    layers = []
+    for l in range(n_layers):
+        for i, s in enumerate(shapes()):
+            W = synth.device_weights(s.n_out, s.n_in, WORKLOAD, l, i, device=device)
+            thV, sV = synth.butterfly_params(s.n_in, s.w_in, WORKLOAD, l, i, "V")
+            thU, sU = synth.butterfly_params(s.n_out, s.w_out, WORKLOAD, l, i, "U")
+            thV, thU = torch.from_numpy(thV).to(device), torch.from_numpy(thU).to(device)
+            sV, sU = torch.from_numpy(sV).to(device), torch.from_numpy(sU).to(device)
+            Wr = rb.rotate_weights_device(W, thV, sV, s.w_in, thU, sU, s.w_out)
+            del W
+            codes, sz = rb.harp_quantize_weights(Wr, BITS, GROUP)
+            del Wr
+            layers.append(rb.HarpLayer(s.n_in, s.n_out, BITS, s.w_in, s.w_out, thV, sV, thU, sU, codes, sz))
+    torch.cuda.synchronize()
+    return rb.HarpStack(layers, HIDDEN, FFN, NH, NKV, HD)
+
+
+def launches_per_step(n_layers):
+    # one convert + per block: 2 RMSNorm, 7 x (input butterfly, GEMV, output butterfly),
+    # 2 residual adds, 1 SiLU*up (no repeat: 32 query heads over 32 kv heads) + one store
+    return 1 + n_layers * (2 + 7 * 3 + 2 + 1) + 1
+
+
+def run_ours(args, rank, world):
+    import torch
+    import torch.distributed as dist
+    from rotated_bit_matmul_b200 import synth
+    device = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(device)
+    stack = build_stack(args.layers, device)
+    K, Wm = args.steps, args.warmup
+    xs = torch.stack([torch.from_numpy(synth.activations(BATCH, HIDDEN, WORKLOAD, step=s)).to(torch.bfloat16)
+                      for s in range(K + Wm)]).to(device)
+    x_in = torch.empty((BATCH, HIDDEN), dtype=torch.bfloat16, device=device)
+    y = torch.empty((BATCH, HIDDEN), dtype=torch.float32, device=device)
+    ws = stack.workspace(BATCH)
+    stream = torch.cuda.Stream(device)
+
+    # warm-up (also first-use allocations), then capture one step into a CUDA graph
+    with torch.cuda.stream(stream):
+        for s in range(Wm):
+            x_in.copy_(xs[s])
+            stack.step(x_in, out=y, workspace=ws)
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        stack.step(x_in, out=y, workspace=ws)
+    stream.synchronize()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(device.index) as clk:
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for s in range(K):
+                x_in.copy_(xs[Wm + s], non_blocking=True)
+                g.replay()
+            e1.record(stream)
+        e1.synchronize()
+    torch.cuda.synchronize()
+    barrier()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / K
+    value = world * BATCH * K / (ms / 1e3)
+
+    # end to end through the public API with host buffers: pinned H2D of the step's
+    # input, the stack step, D2H of its output, every step
+    xh = torch.stack([torch.from_numpy(synth.activations(BATCH, HIDDEN, WORKLOAD, step=s)).to(torch.bfloat16)
+                      for s in range(K)]).pin_memory()
+    yh = torch.empty((K, BATCH, HIDDEN), dtype=torch.float32).pin_memory()
+    barrier()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for s in range(K):
+            x_in.copy_(xh[s], non_blocking=True)
+            stack.step(x_in, out=y, workspace=ws)
+            yh[s].copy_(y, non_blocking=True)
+        e1.record(stream)
+    e1.synchronize()
+    barrier()
+    ms_e2e = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms_e2e], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_e2e = float(t.item())
+    e2e = {"value": world * BATCH * K / (ms_e2e / 1e3), "unit": "tokens/s",
+           "h2d_bytes_per_step": int(xh[0].numel() * xh.element_size()),
+           "d2h_bytes_per_step": int(yh[0].numel() * yh.element_size())}
+
+    nbytes = algorithmic_bytes_per_step(args.layers)
+    peak, peak_kind = measured_peak()
+    achieved = nbytes / (ms_step * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": None,
+                "kernel": "whole decode step (graph of the step's kernels)", "peak_kind": peak_kind,
+                "algorithmic_bytes_per_step": nbytes}
+    del g
+    return dict(value=value, ms_step=ms_step, e2e=e2e, roofline=roofline, clocks=clk.summary(),
+                launches=launches_per_step(args.layers) * K)
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "gloo" if args.impl == "reference" else "nccl"
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+
+    config = {"workload": CONFIG_NAME, "layers": args.layers, "hidden": HIDDEN, "ffn": FFN, "bits": BITS,
+              "group": GROUP, "batch": BATCH, "global_batch": BATCH * world, "parallelism": f"replicas{world}",
+              "l2": "inputs larger than L2: each step streams ~2.03 GB of packed codes and scales (L2 126 MB)"}
+    base = {"metric": METRIC, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "data": "synthetic (seeded N(0,1) bf16 inputs; random-init N(0,0.02^2) weights with 0.1% outlier columns)",
+            "config": config}
+
+    if args.impl == "reference":
+        if rank == 0:
+            tps, per_block, threads = cpu_oracle_sample(args.cpu_sample_layers)
+            ms = per_block * N_LAYERS * 1e3
+            line = dict(base, impl="reference", value=tps, unit="tokens/s", ms_per_step=ms, dtype="f64",
+                        cpu_baseline={"value": tps, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                                      "sample": f"{args.cpu_sample_layers} of {N_LAYERS} blocks of one decode "
+                                                f"token per step, scaled to {N_LAYERS} blocks"},
+                        e2e={"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0})
+            line["steps"], line["warmup"] = 1, 0
+            print(json.dumps(line), flush=True)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+
+    r = run_ours(args, rank, world)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tps, per_block, threads = cpu_oracle_sample(args.cpu_sample_layers)
+        cpu = {"value": tps, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+               "sample": f"{args.cpu_sample_layers} of {N_LAYERS} blocks of one decode token, scaled to {N_LAYERS}"}
+    if rank == 0:
+        line = dict(base, value=r["value"], unit="tokens/s", ms_per_step=r["ms_step"],
+                    dtype="u2 codes x i16 activations -> i32 dot, f32 elsewhere", roofline=r["roofline"],
+                    cpu_baseline=cpu, e2e=r["e2e"], gpu_launches=r["launches"], clocks=r["clocks"])
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,162 @@
+/*
+ * harp.h -- C ABI of the B200 (sm_100a) rotated low-bit linear library.
+ *
+ * The method: "HARP: Hadamard-Preconditioned Adaptive Rotation Processor for
+ * Extreme LLM Quantization" (gist.science explanation of arXiv 2605.29843).
+ * A linear layer W (n_out x n_in) is stored as a low-bit quantization of the
+ * rotated matrix W' = U W V^T, where V and U^T are butterfly transforms:
+ *   F(theta, s, w) = S_{m-1} ... S_1 S_0 D,  m = log2(w),
+ *   D = diag(s), s_i in {+1,-1}; stage S_t pairs (i, i + 2^t) inside every w-wide
+ *   block with the 2x2 block Givens(theta) * H_2 = [[cos p, sin p], [sin p, -cos p]],
+ *   p = pi/4 + theta (Sec. 2.1 "Arquitetura Central": stride stages of block-diagonal
+ *   orthogonal B_t; Sec. 2.2: B = Q(theta) G_2, Theta = 0 gives the randomized
+ *   Hadamard transform). Pairs of stage t are numbered in increasing order of their
+ *   first index; theta is stored stage-major, [m][n/2] fp32.
+ *   n that is not a power of two uses w-wide blocks (block-diagonal butterfly).
+ * Online the layer computes y = U^T dequant(codes) V x = F_U(dequant(codes) F_V(x))
+ * with V = F(theta_V, s_V, w_in) and U^T = F(theta_U, s_U, w_out).
+ *
+ * Quantizer (a stand-in: the pages leave the codebook to the backend, Sec. 2.4):
+ * per output row and group of `group` = 64 consecutive columns of W',
+ * zero16 = fp16(min), scale16 = fp16((max-min)/(2^b-1)) (1 when that is 0),
+ * q = clamp(round_half_even((w - zero16)/scale16), 0, 2^b-1), dequant = scale16*q + zero16.
+ *
+ * Canonical layouts (device memory, row-major by output row, e = r*n_in + j):
+ *   codes, b = 2 or 4: code e in little-endian 32-bit word (e*b)/32, bits [(e*b)%32, +b);
+ *   codes, b = 3: a 2-bit plane of (q & 3) laid out as for b = 2 (n_out*n_in/4 bytes)
+ *                 followed by a 1-bit plane of (q >> 2): word e/32, bit e%32;
+ *   scale_zero: [n_out][n_in/group] half2, .x = scale16, .y = zero16.
+ *
+ * Conventions for every entry point:
+ *   - Pointers named "device" must be device memory of the current device; every
+ *     device pointer must be 16-byte aligned. `stream` is a cudaStream_t (0 = the
+ *     legacy default stream). All work is enqueued on `stream` and returns at once.
+ *   - Arguments are validated before anything is launched; on failure nothing is
+ *     launched, the call returns a non-zero status and harp_last_error() (a
+ *     thread-local string) says why. No C++ exception crosses this boundary.
+ *   - Device-side failures (a bounded wait that ran out, a failed bounds check) set
+ *     a per-device status word; harp_device_status() reads and clears it.
+ *   - Calls on different layer handles may run from different host threads.
+ */
+#ifndef HARP_H
+#define HARP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HARP_OK = 0,
+  HARP_ERR_INVALID_ARG = 1, /* bad size, alignment, null pointer, unsupported width */
+  HARP_ERR_UNSUPPORTED = 2, /* valid request this build does not implement */
+  HARP_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
+  HARP_ERR_WORKSPACE = 4,   /* workspace missing or smaller than the query returned */
+  HARP_ERR_TIMEOUT = 5,     /* a bounded device-side wait ran out (device status) */
+  HARP_ERR_DEVICE_CHECK = 6 /* a device-side bounds/consistency check failed */
+} harp_status;
+
+typedef enum { HARP_F32 = 0, HARP_BF16 = 1, HARP_F16 = 2 } harp_dtype;
+
+typedef struct harp_layer_s* harp_layer;
+typedef struct harp_stack_s* harp_stack;
+
+/* Thread-local description of the last failure on this host thread ("" if none). */
+const char* harp_last_error(void);
+
+/* Reads and clears the device status word of the current device (HARP_OK if clean).
+ * Synchronises `stream` first. */
+harp_status harp_device_status(void* stream);
+
+/* ---------------------------------------------------------------- butterfly
+ * y = F(theta, s, w) x for `batch` rows of n (row-major, contiguous).
+ * Sec. 2.1-2.2 of the HARP page: signs, then stages of stride 1, 2, ..., w/2.
+ *   n      : vector length, n % w == 0, n <= 2^30.
+ *   w      : block width, a power of two, 2 <= w <= 8192.
+ *   theta  : device fp32 [log2 w][n/2] angle offsets (the pi/4 is added inside).
+ *   sign   : device int8 [n], each +1 or -1.
+ *   x, y   : device, dtypes xt / yt (f32, bf16, f16); y may equal x when xt == yt.
+ * Arithmetic is fp32; sin/cos are evaluated in fp32 from pi/4 + theta.
+ */
+harp_status harp_butterfly_fwd(int64_t n, int w, int batch, const float* theta, const int8_t* sign,
+                               const void* x, harp_dtype xt, void* y, harp_dtype yt, void* stream);
+
+/* y = F(theta, s, w)^T x: the same stages in reverse order, then the signs
+ * (every 2x2 block is symmetric). Same arguments as harp_butterfly_fwd. */
+harp_status harp_butterfly_inv(int64_t n, int w, int batch, const float* theta, const int8_t* sign,
+                               const void* x, harp_dtype xt, void* y, harp_dtype yt, void* stream);
+
+/* ---------------------------------------------------------------- quantize
+ * Quantizes an already rotated matrix W' (device fp32 [n_out][n_in], row-major) into
+ * the canonical codes and scale_zero buffers (device, caller-owned, sizes
+ * n_out*n_in*bits/8 and n_out*(n_in/group)*4 bytes). bits in {2,3,4}, group == 64,
+ * n_in % 64 == 0. The arithmetic of the rule above is done in fp64 on the device, so
+ * the codes equal those of an fp64 evaluation of the same fp32 input.
+ */
+harp_status harp_quantize_weights(int64_t n_out, int64_t n_in, int bits, int group,
+                                  const float* W_rot, void* codes, void* scale_zero, void* stream);
+
+/* ---------------------------------------------------------------- layer
+ * Creates a layer handle.
+ *   n_in, n_out : multiples of 64, each <= 65536.
+ *   bits        : 2, 3 or 4.   group: 64.
+ *   w_in, w_out : butterfly block widths: powers of two, 64 <= w <= 8192, w | n.
+ *   theta_V, sign_V : device [log2 w_in][n_in/2] fp32, [n_in] int8 (input side V).
+ *   theta_U, sign_U : device [log2 w_out][n_out/2] fp32, [n_out] int8 (U^T side).
+ *   codes, scale_zero : device, canonical layout above.
+ * Ownership: the layer COPIES theta/sign (it stores cos/sin tables of pi/4 + theta in
+ * its own device memory) and BORROWS codes and scale_zero, which the caller keeps
+ * alive and unchanged until harp_destroy_layer. The copies are enqueued on `stream`.
+ */
+harp_status harp_create_layer(harp_layer* out, int64_t n_in, int64_t n_out, int bits, int group,
+                              int w_in, int w_out, const float* theta_V, const int8_t* sign_V,
+                              const float* theta_U, const int8_t* sign_U, const void* codes,
+                              const void* scale_zero, void* stream);
+
+/* Frees the layer's own device memory (synchronises the device first). Null is a no-op. */
+harp_status harp_destroy_layer(harp_layer layer);
+
+/* Bytes of device workspace harp_linear_fwd needs for `batch` rows (batch 1..256). */
+harp_status harp_linear_workspace_size(harp_layer layer, int batch, size_t* bytes);
+
+/* y = F_U(dequant(codes) F_V(x)) for `batch` rows.
+ *   x : device [batch][n_in] of dtype xt;  y : device [batch][n_out] of dtype yt.
+ *   workspace : device scratch of at least harp_linear_workspace_size bytes, 256-byte
+ *               aligned; its contents are overwritten. y must not alias x or workspace.
+ * Batches 1..8 run the CUDA-core dequant-GEMV (fp32 activations, exact integer dot
+ * products per group); 16..256 run the tcgen05 tensor-core path (bf16 operands, fp32
+ * accumulation) where built, else the GEMV path.
+ */
+harp_status harp_linear_fwd(harp_layer layer, int batch, const void* x, harp_dtype xt, void* y,
+                            harp_dtype yt, void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------- decoder stack
+ * A Llama-shaped stack of n_layers blocks, each with seven rotated linears in the
+ * order q, k, v, o, gate, up, down (layers[7*l + i]). One decode step computes, per
+ * block: n1 = rms(x); v = v_proj(n1) (q_proj and k_proj are evaluated too; a one-key
+ * attention returns its value); a = v repeated per key/value group (head h reads kv
+ * head h / (n_heads/n_kv_heads)); h = x + o_proj(a); n2 = rms(h);
+ * x' = h + down(silu(gate(n2)) * up(n2)); rms(u) = u / sqrt(mean(u^2) + eps).
+ * The stack borrows the layer handles (they must outlive it).
+ * Shapes: q n_heads*head_dim x hidden, k/v n_kv_heads*head_dim x hidden,
+ * o hidden x n_heads*head_dim, gate/up ffn x hidden, down hidden x ffn; the output-side
+ * block width of gate and up must equal the input-side block width of down.
+ */
+harp_status harp_stack_create(harp_stack* out, int n_layers, int hidden, int ffn, int n_heads,
+                              int n_kv_heads, int head_dim, float eps, const harp_layer* layers,
+                              void* stream);
+harp_status harp_stack_destroy(harp_stack stack);
+harp_status harp_stack_workspace_size(harp_stack stack, int batch, size_t* bytes);
+
+/* One decode step: out = stack(x). x, out: device [batch][hidden] of dtypes xt / ot
+ * (batch 1..256); out may equal x. workspace as for harp_linear_fwd. */
+harp_status harp_stack_step(harp_stack stack, int batch, const void* x, harp_dtype xt, void* out,
+                            harp_dtype ot, void* workspace, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HARP_H */

@@ -1,0 +1,204 @@
+"""B200 (sm_100a) rotated low-bit linear: HARP's inference hot path.
+
+"HARP: Hadamard-Preconditioned Adaptive Rotation Processor for Extreme LLM
+Quantization" wraps every linear layer in two butterfly transforms (log2 w stages
+of 2x2 Givens-times-Hadamard blocks after a random sign diagonal, initialised to the
+randomized Hadamard transform) around a low-bit quantized weight matrix:
+y = U^T dequant(Q(U W V^T)) V x, with V x and U^T applied online.
+
+This package is a thin torch-facing binding of libharp.so (C ABI in include/harp.h).
+The functions keep the C names; they marshal tensors into device pointers and the
+current CUDA stream and raise HarpError on a non-OK status. All arithmetic runs in
+the library's kernels; there is no Python or CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+
+from ._lib import (HARP_BF16, HARP_F16, HARP_F32, HarpError, call, load)  # noqa: F401
+
+__all__ = ["HarpError", "harp_butterfly_fwd", "harp_butterfly_inv", "harp_quantize_weights", "HarpLayer",
+           "HarpStack", "rotate_weights_device", "harp_device_status", "load"]
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _dt(t) -> int:
+    torch = _torch()
+    return {torch.float32: HARP_F32, torch.bfloat16: HARP_BF16, torch.float16: HARP_F16}[t.dtype]
+
+
+def _p(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _stream():
+    return ctypes.c_void_p(_torch().cuda.current_stream().cuda_stream)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("rotated_bit_matmul_b200 works on CUDA tensors only")
+
+
+def harp_device_status() -> None:
+    """Raises HarpError if a kernel reported a device-side failure (clears it)."""
+    call("harp_device_status", _stream())
+
+
+def _bfly(name, x, theta, sign, w, out_dtype=None, out=None):
+    torch = _torch()
+    _need_cuda(x, theta, sign)
+    x2 = x.reshape(-1, x.shape[-1]) if x.dim() > 1 else x.reshape(1, -1)
+    if not x2.is_contiguous():
+        x2 = x2.contiguous()
+    n = x2.shape[1]
+    if out is None:
+        out = torch.empty(x2.shape, dtype=out_dtype or x.dtype, device=x.device)
+    call(name, n, int(w), x2.shape[0], _p(theta), _p(sign), _p(x2), _dt(x2), _p(out), _dt(out), _stream())
+    return out.reshape(x.shape)
+
+
+def harp_butterfly_fwd(x, theta, sign, w, out_dtype=None, out=None):
+    """F(theta, s, w) x over the last dimension. theta fp32 [log2 w, n/2], sign int8 [n]."""
+    return _bfly("harp_butterfly_fwd", x, theta, sign, w, out_dtype, out)
+
+
+def harp_butterfly_inv(x, theta, sign, w, out_dtype=None, out=None):
+    """F(theta, s, w)^T x over the last dimension."""
+    return _bfly("harp_butterfly_inv", x, theta, sign, w, out_dtype, out)
+
+
+def harp_quantize_weights(W_rot, bits: int, group: int = 64):
+    """Quantizes a rotated fp32 [n_out, n_in] matrix; returns (codes uint8, scale_zero int32)."""
+    torch = _torch()
+    _need_cuda(W_rot)
+    W_rot = W_rot.contiguous()
+    n_out, n_in = W_rot.shape
+    codes = torch.empty(n_out * n_in * bits // 8, dtype=torch.uint8, device=W_rot.device)
+    sz = torch.empty(n_out * (n_in // group), dtype=torch.int32, device=W_rot.device)
+    call("harp_quantize_weights", n_out, n_in, int(bits), int(group), _p(W_rot), _p(codes), _p(sz), _stream())
+    return codes, sz
+
+
+def rotate_weights_device(W, theta_V, sign_V, w_in, theta_U, sign_U, w_out):
+    """W' = U W V^T on the device: rows through F_V, then columns through F_U^T."""
+    _need_cuda(W)
+    Wr = harp_butterfly_fwd(W.float().contiguous(), theta_V, sign_V, w_in)
+    Wt = Wr.t().contiguous()
+    harp_butterfly_inv(Wt, theta_U, sign_U, w_out, out=Wt)
+    return Wt.t().contiguous()
+
+
+class HarpLayer:
+    """A rotated low-bit linear on the device (wraps harp_create_layer)."""
+
+    def __init__(self, n_in, n_out, bits, w_in, w_out, theta_V, sign_V, theta_U, sign_U, codes, scale_zero,
+                 group=64):
+        _need_cuda(theta_V, sign_V, theta_U, sign_U, codes, scale_zero)
+        self.n_in, self.n_out, self.bits, self.group = int(n_in), int(n_out), int(bits), int(group)
+        self.w_in, self.w_out = int(w_in), int(w_out)
+        # the library borrows codes and scale_zero: keep them alive with the handle
+        self.codes, self.scale_zero = codes, scale_zero
+        h = ctypes.c_void_p()
+        call("harp_create_layer", ctypes.byref(h), self.n_in, self.n_out, self.bits, self.group, self.w_in,
+             self.w_out, _p(theta_V.contiguous()), _p(sign_V.contiguous()), _p(theta_U.contiguous()),
+             _p(sign_U.contiguous()), _p(codes), _p(scale_zero), _stream())
+        self.handle = h
+        self._ws = {}
+        self.device = codes.device
+
+    def workspace_bytes(self, batch: int) -> int:
+        n = ctypes.c_size_t()
+        call("harp_linear_workspace_size", self.handle, int(batch), ctypes.byref(n))
+        return n.value
+
+    def workspace(self, batch: int):
+        ws = self._ws.get(batch)
+        if ws is None:
+            ws = _torch().empty(max(self.workspace_bytes(batch), 256), dtype=_torch().uint8, device=self.device)
+            self._ws[batch] = ws
+        return ws
+
+    def __call__(self, x, out_dtype=None, out=None, workspace=None):
+        torch = _torch()
+        _need_cuda(x)
+        x2 = x.reshape(-1, self.n_in).contiguous()
+        if out is None:
+            out = torch.empty((x2.shape[0], self.n_out), dtype=out_dtype or x.dtype, device=x.device)
+        ws = workspace if workspace is not None else self.workspace(x2.shape[0])
+        call("harp_linear_fwd", self.handle, x2.shape[0], _p(x2), _dt(x2), _p(out), _dt(out), _p(ws),
+             ws.numel(), _stream())
+        return out
+
+    def close(self):
+        if getattr(self, "handle", None) is not None and self.handle.value:
+            call("harp_destroy_layer", self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class HarpStack:
+    """Llama-shaped decode stack of rotated linears (wraps harp_stack_create/step)."""
+
+    def __init__(self, layers, hidden, ffn, n_heads, n_kv_heads, head_dim, eps=1e-5):
+        self.layers = list(layers)
+        assert len(self.layers) % 7 == 0
+        arr = (ctypes.c_void_p * len(self.layers))(*[l.handle.value for l in self.layers])
+        h = ctypes.c_void_p()
+        call("harp_stack_create", ctypes.byref(h), len(self.layers) // 7, int(hidden), int(ffn), int(n_heads),
+             int(n_kv_heads), int(head_dim), ctypes.c_float(eps), arr, _stream())
+        self.handle = h
+        self.hidden = int(hidden)
+        self._ws = {}
+        self.device = self.layers[0].device
+
+    def workspace_bytes(self, batch: int) -> int:
+        n = ctypes.c_size_t()
+        call("harp_stack_workspace_size", self.handle, int(batch), ctypes.byref(n))
+        return n.value
+
+    def workspace(self, batch: int):
+        ws = self._ws.get(batch)
+        if ws is None:
+            ws = _torch().empty(self.workspace_bytes(batch), dtype=_torch().uint8, device=self.device)
+            self._ws[batch] = ws
+        return ws
+
+    def step(self, x, out_dtype=None, out=None, workspace=None):
+        torch = _torch()
+        _need_cuda(x)
+        x2 = x.reshape(-1, self.hidden).contiguous()
+        if out is None:
+            out = torch.empty(x2.shape, dtype=out_dtype or torch.float32, device=x.device)
+        ws = workspace if workspace is not None else self.workspace(x2.shape[0])
+        call("harp_stack_step", self.handle, x2.shape[0], _p(x2), _dt(x2), _p(out), _dt(out), _p(ws), ws.numel(),
+             _stream())
+        return out
+
+    def close(self):
+        if getattr(self, "handle", None) is not None and self.handle.value:
+            call("harp_stack_destroy", self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def log2i(w: int) -> int:
+    m = int(math.log2(w))
+    assert 1 << m == w
+    return m

@@ -1,0 +1,407 @@
+// C ABI of the rotated low-bit linear library: argument checks, layer handles,
+// workspace layout and kernel dispatch. Declarations and contracts: include/harp.h.
+#include <cudaTypedefs.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <string>
+
+#include "harp_internal.h"
+
+using namespace harp;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+harp_status fail(harp_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+harp_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(HARP_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+#define HARP_CUDA(call, what)                       \
+  do {                                              \
+    cudaError_t e_ = (call);                        \
+    if (e_ != cudaSuccess) return cuda_fail(e_, what); \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int log2_exact(int64_t w) {
+  if (w < 1) return -1;
+  int m = 0;
+  while ((int64_t(1) << m) < w) ++m;
+  return (int64_t(1) << m) == w ? m : -1;
+}
+
+bool valid_dtype(int dt) { return dt == HARP_F32 || dt == HARP_BF16 || dt == HARP_F16; }
+
+// ------------------------------------------------------------------ device status words
+std::mutex g_status_mu;
+int* g_status[64] = {nullptr};
+
+harp_status device_status_ptr(int** out) {
+  int dev = 0;
+  HARP_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(HARP_ERR_UNSUPPORTED, "device index %d >= 64", dev);
+  std::lock_guard<std::mutex> lk(g_status_mu);
+  if (!g_status[dev]) {
+    int* p = nullptr;
+    HARP_CUDA(cudaMalloc(&p, 4 * sizeof(int)), "cudaMalloc(status)");
+    HARP_CUDA(cudaMemset(p, 0, 4 * sizeof(int)), "cudaMemset(status)");
+    HARP_CUDA(cudaDeviceSynchronize(), "cudaDeviceSynchronize");
+    g_status[dev] = p;
+  }
+  *out = g_status[dev];
+  return HARP_OK;
+}
+
+// ------------------------------------------------------------------ tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D row-major tensor [rows][inner] of `esize`-byte elements, box 32 rows x 128 bytes,
+// 128-byte swizzle, zero fill out of bounds.
+harp_status make_tmap(CUtensorMap* tm, const void* base, CUtensorMapDataType dt, int esize, uint64_t inner,
+                      uint64_t rows, uint64_t row_bytes) {
+  auto fn = encode_fn();
+  if (!fn) return fail(HARP_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {(cuuint32_t)(128 / esize), 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(tm, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(HARP_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return HARP_OK;
+}
+
+harp_status check_bfly_args(int64_t n, int w, int batch, const float* theta, const int8_t* sign, const void* x,
+                            int xt, const void* y, int yt) {
+  if (n <= 0 || n > (int64_t(1) << 30)) return fail(HARP_ERR_INVALID_ARG, "butterfly: n=%lld out of range", (long long)n);
+  if (log2_exact(w) < 1 || w > kMaxW) return fail(HARP_ERR_INVALID_ARG, "butterfly: w=%d must be a power of two in [2, 8192]", w);
+  if (n % w) return fail(HARP_ERR_INVALID_ARG, "butterfly: w=%d does not divide n=%lld", w, (long long)n);
+  if (batch < 0 || batch > 65535) return fail(HARP_ERR_INVALID_ARG, "butterfly: batch=%d out of range", batch);
+  if (!valid_dtype(xt) || !valid_dtype(yt)) return fail(HARP_ERR_INVALID_ARG, "butterfly: unknown dtype");
+  if (!theta || !sign || !x || !y) return fail(HARP_ERR_INVALID_ARG, "butterfly: null pointer");
+  if (!aligned16(theta) || !aligned16(sign) || !aligned16(x) || !aligned16(y))
+    return fail(HARP_ERR_INVALID_ARG, "butterfly: device pointers must be 16-byte aligned");
+  if (x == y && xt != yt) return fail(HARP_ERR_INVALID_ARG, "butterfly: in-place needs equal dtypes");
+  return HARP_OK;
+}
+
+harp_status bfly_common(int64_t n, int w, int batch, const float* theta, const int8_t* sign, const void* x,
+                        harp_dtype xt, void* y, harp_dtype yt, void* stream, int inverse) {
+  harp_status st = check_bfly_args(n, w, batch, theta, sign, x, xt, y, yt);
+  if (st != HARP_OK) return st;
+  if (batch == 0) return HARP_OK;
+  int* status = nullptr;
+  if ((st = device_status_ptr(&status)) != HARP_OK) return st;
+  BflyParams p{};
+  p.n = n;
+  p.w = w;
+  p.m = log2_exact(w);
+  p.inverse = inverse;
+  p.theta = theta;
+  p.cs = nullptr;
+  p.sign = sign;
+  p.x = x;
+  p.xt = xt;
+  p.x_stride = n;
+  p.y = y;
+  p.yt = yt;
+  p.y_stride = n;
+  p.status = status;
+  HARP_CUDA(launch_butterfly(p, batch, static_cast<cudaStream_t>(stream)), "butterfly launch");
+  return HARP_OK;
+}
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+}  // namespace
+
+namespace harp {
+
+int xq_words_per_row(int64_t n_in, int bits) { return (int)(bits == 3 ? n_in : n_in / 2); }
+
+LinearWs linear_ws_layout(const Layer& L, int batch, void* base) {
+  LinearWs w{};
+  const int64_t ng = L.n_in / kGroup;
+  w.xq_stride = xq_words_per_row(L.n_in, L.bits);
+  w.g_stride = ng;
+  size_t off = 0;
+  const size_t o_xq = off;
+  off = align256(off + sizeof(int32_t) * (size_t)batch * (size_t)w.xq_stride);
+  const size_t o_xs = off;
+  off = align256(off + sizeof(float) * (size_t)batch * (size_t)ng);
+  const size_t o_sum = off;
+  off = align256(off + sizeof(float) * (size_t)batch * (size_t)ng);
+  const size_t o_z = off;
+  off = align256(off + sizeof(float) * (size_t)batch * (size_t)L.n_out);
+  w.bytes = off;
+  if (base) {
+    char* b = static_cast<char*>(base);
+    w.xq = reinterpret_cast<int32_t*>(b + o_xq);
+    w.xs = reinterpret_cast<float*>(b + o_xs);
+    w.xsum = reinterpret_cast<float*>(b + o_sum);
+    w.z = reinterpret_cast<float*>(b + o_z);
+  }
+  return w;
+}
+
+// Enqueues y = F_U(dequant(codes) F_V(x)) on st; arguments already validated.
+harp_status linear_forward(const Layer& L, int batch, const void* x, int xt, int64_t x_stride, void* y, int yt,
+                           int64_t y_stride, void* ws, cudaStream_t st) {
+  int* status = nullptr;
+  harp_status s = device_status_ptr(&status);
+  if (s != HARP_OK) return s;
+  LinearWs w = linear_ws_layout(L, batch, ws);
+
+  BflyParams pv{};
+  pv.n = L.n_in;
+  pv.w = L.w_in;
+  pv.m = L.m_in;
+  pv.inverse = 0;
+  pv.cs = L.csV;
+  pv.sign = L.sV;
+  pv.x = x;
+  pv.xt = xt;
+  pv.x_stride = x_stride;
+  pv.y = nullptr;
+  pv.xq = w.xq;
+  pv.xs = w.xs;
+  pv.xsum = w.xsum;
+  pv.bits = L.bits;
+  pv.xq_stride = w.xq_stride;
+  pv.g_stride = w.g_stride;
+  pv.status = status;
+  HARP_CUDA(launch_butterfly(pv, batch, st), "input butterfly launch");
+
+  for (int b0 = 0; b0 < batch; b0 += kMaxBatchGemv) {
+    GemvParams gp{};
+    gp.n_out = (int)L.n_out;
+    gp.n_in = (int)L.n_in;
+    gp.bits = L.bits;
+    gp.batch = batch - b0 < kMaxBatchGemv ? batch - b0 : kMaxBatchGemv;
+    gp.xq = w.xq + (int64_t)b0 * w.xq_stride;
+    gp.xq_stride = w.xq_stride;
+    gp.xs = w.xs + (int64_t)b0 * w.g_stride;
+    gp.xsum = w.xsum + (int64_t)b0 * w.g_stride;
+    gp.g_stride = w.g_stride;
+    gp.z = w.z + (int64_t)b0 * L.n_out;
+    gp.z_stride = L.n_out;
+    gp.status = status;
+    HARP_CUDA(launch_gemv(L, gp, st), "dequant-GEMV launch");
+  }
+
+  BflyParams pu{};
+  pu.n = L.n_out;
+  pu.w = L.w_out;
+  pu.m = L.m_out;
+  pu.inverse = 0;
+  pu.cs = L.csU;
+  pu.sign = L.sU;
+  pu.x = w.z;
+  pu.xt = DT_F32;
+  pu.x_stride = L.n_out;
+  pu.y = y;
+  pu.yt = yt;
+  pu.y_stride = y_stride;
+  pu.status = status;
+  HARP_CUDA(launch_butterfly(pu, batch, st), "output butterfly launch");
+  return HARP_OK;
+}
+
+harp_status device_status_for_kernels(int** out) { return device_status_ptr(out); }
+
+harp_status set_error(harp_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+}  // namespace harp
+
+extern "C" {
+
+const char* harp_last_error(void) { return g_last_error.c_str(); }
+
+harp_status harp_device_status(void* stream) {
+  int* status = nullptr;
+  harp_status st = device_status_ptr(&status);
+  if (st != HARP_OK) return st;
+  int host[2] = {0, 0};
+  HARP_CUDA(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)), "cudaStreamSynchronize");
+  HARP_CUDA(cudaMemcpy(host, status, sizeof host, cudaMemcpyDeviceToHost), "cudaMemcpy(status)");
+  if (host[0] == 0) return HARP_OK;
+  HARP_CUDA(cudaMemset(status, 0, 4 * sizeof(int)), "cudaMemset(status)");
+  HARP_CUDA(cudaDeviceSynchronize(), "cudaDeviceSynchronize");
+  return fail((harp_status)host[0], "device reported status %d at site %d", host[0], host[1]);
+}
+
+harp_status harp_butterfly_fwd(int64_t n, int w, int batch, const float* theta, const int8_t* sign, const void* x,
+                               harp_dtype xt, void* y, harp_dtype yt, void* stream) {
+  return bfly_common(n, w, batch, theta, sign, x, xt, y, yt, stream, 0);
+}
+
+harp_status harp_butterfly_inv(int64_t n, int w, int batch, const float* theta, const int8_t* sign, const void* x,
+                               harp_dtype xt, void* y, harp_dtype yt, void* stream) {
+  return bfly_common(n, w, batch, theta, sign, x, xt, y, yt, stream, 1);
+}
+
+harp_status harp_quantize_weights(int64_t n_out, int64_t n_in, int bits, int group, const float* W_rot, void* codes,
+                                  void* scale_zero, void* stream) {
+  if (bits < 2 || bits > 4) return fail(HARP_ERR_INVALID_ARG, "quantize: bits=%d not in {2,3,4}", bits);
+  if (group != kGroup) return fail(HARP_ERR_UNSUPPORTED, "quantize: group=%d (only 64 is supported)", group);
+  if (n_out <= 0 || n_in <= 0 || n_in % 64 || n_out > (int64_t(1) << 24) || n_in > (int64_t(1) << 24))
+    return fail(HARP_ERR_INVALID_ARG, "quantize: n_out=%lld n_in=%lld (need n_in %% 64 == 0)", (long long)n_out,
+                (long long)n_in);
+  if (!W_rot || !codes || !scale_zero) return fail(HARP_ERR_INVALID_ARG, "quantize: null pointer");
+  if (!aligned16(W_rot) || !aligned16(codes) || !aligned16(scale_zero))
+    return fail(HARP_ERR_INVALID_ARG, "quantize: device pointers must be 16-byte aligned");
+  HARP_CUDA(launch_quantize(n_out, n_in, bits, W_rot, codes, scale_zero, static_cast<cudaStream_t>(stream)),
+            "quantize launch");
+  return HARP_OK;
+}
+
+harp_status harp_create_layer(harp_layer* out, int64_t n_in, int64_t n_out, int bits, int group, int w_in,
+                              int w_out, const float* theta_V, const int8_t* sign_V, const float* theta_U,
+                              const int8_t* sign_U, const void* codes, const void* scale_zero, void* stream) {
+  if (!out) return fail(HARP_ERR_INVALID_ARG, "create_layer: null output handle");
+  *out = nullptr;
+  if (bits < 2 || bits > 4) return fail(HARP_ERR_INVALID_ARG, "create_layer: bits=%d not in {2,3,4}", bits);
+  if (group != kGroup) return fail(HARP_ERR_UNSUPPORTED, "create_layer: group=%d (only 64 is supported)", group);
+  if (n_in <= 0 || n_in % 256 || n_in > 65536)
+    return fail(HARP_ERR_INVALID_ARG, "create_layer: n_in=%lld must be a positive multiple of 256, <= 65536",
+                (long long)n_in);
+  if (n_out <= 0 || n_out > 65536) return fail(HARP_ERR_INVALID_ARG, "create_layer: n_out=%lld out of range", (long long)n_out);
+  const int m_in = log2_exact(w_in), m_out = log2_exact(w_out);
+  if (m_in < 6 || w_in > kMaxW || n_in % w_in)
+    return fail(HARP_ERR_INVALID_ARG, "create_layer: w_in=%d must be a power of two in [64, 8192] dividing n_in", w_in);
+  if (m_out < 1 || w_out > kMaxW || n_out % w_out)
+    return fail(HARP_ERR_INVALID_ARG, "create_layer: w_out=%d must be a power of two in [2, 8192] dividing n_out", w_out);
+  if (!theta_V || !sign_V || !theta_U || !sign_U || !codes || !scale_zero)
+    return fail(HARP_ERR_INVALID_ARG, "create_layer: null pointer");
+  if (!aligned16(theta_V) || !aligned16(sign_V) || !aligned16(theta_U) || !aligned16(sign_U) || !aligned16(codes) ||
+      !aligned16(scale_zero))
+    return fail(HARP_ERR_INVALID_ARG, "create_layer: device pointers must be 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  harp_layer_s* h = new (std::nothrow) harp_layer_s();
+  if (!h) return fail(HARP_ERR_INVALID_ARG, "create_layer: out of host memory");
+  Layer& L = h->L;
+  L.n_in = n_in;
+  L.n_out = n_out;
+  L.bits = bits;
+  L.group = group;
+  L.w_in = w_in;
+  L.w_out = w_out;
+  L.m_in = m_in;
+  L.m_out = m_out;
+  L.codes = codes;
+  L.scale_zero = scale_zero;
+  cudaGetDevice(&L.device);
+  const int64_t cnt_v = (int64_t)m_in * (n_in / 2), cnt_u = (int64_t)m_out * (n_out / 2);
+  auto cleanup = [&](harp_status s) {
+    cudaFree(L.csV);
+    cudaFree(L.csU);
+    cudaFree(L.sV);
+    cudaFree(L.sU);
+    delete h;
+    return s;
+  };
+  cudaError_t e;
+  if ((e = cudaMalloc(&L.csV, sizeof(float2) * cnt_v)) != cudaSuccess ||
+      (e = cudaMalloc(&L.csU, sizeof(float2) * cnt_u)) != cudaSuccess ||
+      (e = cudaMalloc(&L.sV, (size_t)n_in)) != cudaSuccess || (e = cudaMalloc(&L.sU, (size_t)n_out)) != cudaSuccess)
+    return cleanup(cuda_fail(e, "create_layer: cudaMalloc"));
+  if ((e = launch_cs_table(theta_V, cnt_v, L.csV, st)) != cudaSuccess ||
+      (e = launch_cs_table(theta_U, cnt_u, L.csU, st)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(L.sV, sign_V, (size_t)n_in, cudaMemcpyDeviceToDevice, st)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(L.sU, sign_U, (size_t)n_out, cudaMemcpyDeviceToDevice, st)) != cudaSuccess)
+    return cleanup(cuda_fail(e, "create_layer: copies"));
+  const int pb = bits == 4 ? 4 : 2;  // bits of the (first) code plane
+  harp_status s =
+      make_tmap(&L.tm_codes, codes, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, (uint64_t)n_in * pb / 64, (uint64_t)n_out,
+                (uint64_t)n_in * pb / 8);
+  if (s == HARP_OK && bits == 3)
+    s = make_tmap(&L.tm_hi, static_cast<const char*>(codes) + n_out * n_in / 4, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8,
+                  (uint64_t)n_in / 64, (uint64_t)n_out, (uint64_t)n_in / 8);
+  if (s == HARP_OK && bits != 3) L.tm_hi = L.tm_codes;
+  if (s == HARP_OK)
+    s = make_tmap(&L.tm_sz, scale_zero, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, (uint64_t)n_in / 64, (uint64_t)n_out,
+                  (uint64_t)n_in / 16);
+  if (s != HARP_OK) return cleanup(s);
+  *out = h;
+  return HARP_OK;
+}
+
+harp_status harp_destroy_layer(harp_layer layer) {
+  if (!layer) return HARP_OK;
+  int prev = 0;
+  cudaGetDevice(&prev);
+  cudaSetDevice(layer->L.device);
+  cudaDeviceSynchronize();
+  cudaFree(layer->L.csV);
+  cudaFree(layer->L.csU);
+  cudaFree(layer->L.sV);
+  cudaFree(layer->L.sU);
+  cudaSetDevice(prev);
+  delete layer;
+  return HARP_OK;
+}
+
+harp_status harp_linear_workspace_size(harp_layer layer, int batch, size_t* bytes) {
+  if (!layer || !bytes) return fail(HARP_ERR_INVALID_ARG, "linear_workspace_size: null pointer");
+  if (batch < 1 || batch > 256) return fail(HARP_ERR_INVALID_ARG, "linear_workspace_size: batch=%d not in [1,256]", batch);
+  *bytes = linear_ws_layout(layer->L, batch, nullptr).bytes;
+  return HARP_OK;
+}
+
+harp_status harp_linear_fwd(harp_layer layer, int batch, const void* x, harp_dtype xt, void* y, harp_dtype yt,
+                            void* workspace, size_t ws_bytes, void* stream) {
+  if (!layer) return fail(HARP_ERR_INVALID_ARG, "linear_fwd: null layer");
+  if (batch < 1 || batch > 256) return fail(HARP_ERR_INVALID_ARG, "linear_fwd: batch=%d not in [1,256]", batch);
+  if (!valid_dtype(xt) || !valid_dtype(yt)) return fail(HARP_ERR_INVALID_ARG, "linear_fwd: unknown dtype");
+  if (!x || !y) return fail(HARP_ERR_INVALID_ARG, "linear_fwd: null pointer");
+  if (!aligned16(x) || !aligned16(y)) return fail(HARP_ERR_INVALID_ARG, "linear_fwd: pointers must be 16-byte aligned");
+  if (x == y) return fail(HARP_ERR_INVALID_ARG, "linear_fwd: y must not alias x");
+  const size_t need = linear_ws_layout(layer->L, batch, nullptr).bytes;
+  if (!workspace || ws_bytes < need)
+    return fail(HARP_ERR_WORKSPACE, "linear_fwd: workspace of %zu bytes needed, %zu given", need, ws_bytes);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(HARP_ERR_INVALID_ARG, "linear_fwd: workspace must be 256-byte aligned");
+  int dev = 0;
+  HARP_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  if (dev != layer->L.device) return fail(HARP_ERR_INVALID_ARG, "linear_fwd: layer lives on device %d, current is %d", layer->L.device, dev);
+  return linear_forward(layer->L, batch, x, xt, layer->L.n_in, y, yt, layer->L.n_out, workspace,
+                        static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,101 @@
+// Internal declarations of the rotated low-bit linear library (host + device).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/harp.h"
+
+namespace harp {
+
+enum { DT_F32 = 0, DT_BF16 = 1, DT_F16 = 2 };
+
+constexpr int kGroup = 64;       // quantization group (columns)
+constexpr int kMaxBatchGemv = 8; // batch rows the CUDA-core GEMV handles per launch
+constexpr int kMaxW = 8192;      // widest butterfly block held by one CTA
+
+// Butterfly launch description. One CTA transforms one w-wide block of one row.
+struct BflyParams {
+  int64_t n;
+  int w, m, inverse;
+  const float* theta;  // [m][n/2] angle offsets (pi/4 added in-kernel) or null when cs is set
+  const float2* cs;    // [m][n/2] (cos, sin) of pi/4 + theta, or null
+  const int8_t* sign;  // [n]
+  const void* x;
+  int xt;
+  int64_t x_stride;    // elements between rows
+  void* y;             // may be null when only the prep outputs are wanted
+  int yt;
+  int64_t y_stride;
+  // Optional epilogue producing the GEMV operand (null xq disables it):
+  int32_t* xq;         // int16 pairs in dp2a order, xq_stride words per row
+  float* xs;           // per group 2^-e (the int16 scale), g_stride per row
+  float* xsum;         // per group fp32 sum of the transformed values
+  int bits;
+  int64_t xq_stride, g_stride;
+  int* status;
+};
+
+// Dequant-GEMV launch description (codes come through the layer's tensor maps).
+struct GemvParams {
+  int n_out, n_in, bits, batch;
+  const int32_t* xq;
+  int64_t xq_stride;
+  const float* xs;
+  const float* xsum;
+  int64_t g_stride;
+  float* z;
+  int64_t z_stride;
+  int* status;
+};
+
+struct Layer {
+  int64_t n_in, n_out;
+  int bits, group, w_in, w_out, m_in, m_out;
+  float2* csV;   // [m_in][n_in/2]
+  float2* csU;   // [m_out][n_out/2]
+  int8_t* sV;
+  int8_t* sU;
+  const void* codes;
+  const void* scale_zero;
+  CUtensorMap tm_codes;  // 2-bit/4-bit codes, or the 2-bit plane of 3-bit codes
+  CUtensorMap tm_hi;     // 1-bit plane of 3-bit codes (unused otherwise)
+  CUtensorMap tm_sz;     // scale_zero as uint32 [n_out][n_in/64]
+  int device;
+};
+
+// Workspace carve-up for a linear forward with `batch` rows.
+struct LinearWs {
+  int32_t* xq;
+  float* xs;
+  float* xsum;
+  float* z;
+  int64_t xq_stride, g_stride;
+  size_t bytes;
+};
+
+LinearWs linear_ws_layout(const Layer& L, int batch, void* base);
+int xq_words_per_row(int64_t n_in, int bits);
+
+cudaError_t launch_butterfly(const BflyParams& p, int batch, cudaStream_t st);
+cudaError_t launch_gemv(const Layer& L, const GemvParams& p, cudaStream_t st);
+cudaError_t launch_quantize(int64_t n_out, int64_t n_in, int bits, const float* W, void* codes,
+                            void* scale_zero, cudaStream_t st);
+cudaError_t launch_cs_table(const float* theta, int64_t count, float2* cs, cudaStream_t st);
+
+// Records a printf-style message as the thread's last error and returns `st`.
+harp_status set_error(harp_status st, const char* fmt, ...);
+// Per-device status word the kernels report failures into (allocated on first use,
+// which therefore must not happen inside a stream capture).
+harp_status device_status_for_kernels(int** out);
+// Enqueues y = F_U(dequant(codes) F_V(x)) for validated arguments.
+harp_status linear_forward(const Layer& L, int batch, const void* x, int xt, int64_t x_stride, void* y, int yt,
+                           int64_t y_stride, void* ws, cudaStream_t st);
+
+}  // namespace harp
+
+struct harp_layer_s {
+  harp::Layer L;
+};

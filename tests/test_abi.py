@@ -1,0 +1,103 @@
+"""CPU checks of the C ABI: the library loads, exports every entry point include/harp.h
+declares, and rejects bad arguments with a status (validation runs before any CUDA
+call, so none of these touch a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "harp.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(harp_[a-z_0-9]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from rotated_bit_matmul_b200 import build_lib, _lib
+    build_lib.build()
+    return _lib.load()
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = _declared()
+    assert "harp_linear_fwd" in names and "harp_create_layer" in names
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_binding_signatures_cover_header():
+    from rotated_bit_matmul_b200 import _lib
+    assert sorted(_lib.SIGNATURES) == _declared()
+
+
+FAKE = ctypes.c_void_p(1 << 20)       # aligned, never dereferenced: validation fails first
+MIS = ctypes.c_void_p((1 << 20) + 4)  # misaligned
+
+
+@pytest.mark.parametrize("n,w,batch,x,err", [
+    (1024, 3, 1, FAKE, 1),       # w not a power of two
+    (1024, 16384, 1, FAKE, 1),   # w too wide
+    (1000, 16, 1, FAKE, 1),      # w does not divide n
+    (1024, 1024, -1, FAKE, 1),   # negative batch
+    (1024, 1024, 1, MIS, 1),     # misaligned pointer
+    (1024, 1024, 1, None, 1),    # null pointer
+])
+def test_butterfly_rejects_bad_arguments(lib, n, w, batch, x, err):
+    st = lib.harp_butterfly_fwd(n, w, batch, FAKE, FAKE, x, 0, FAKE, 0, None)
+    assert st == err
+    assert lib.harp_last_error()
+
+
+def test_butterfly_inplace_dtype_mismatch(lib):
+    assert lib.harp_butterfly_inv(1024, 1024, 1, FAKE, FAKE, FAKE, 0, FAKE, 1, None) == 1
+
+
+@pytest.mark.parametrize("args,err", [
+    ((4096, 4096, 5, 64), 1),    # bits out of range
+    ((4096, 4096, 2, 32), 2),    # unsupported group
+    ((4096, 100, 2, 64), 1),     # n_in not a multiple of 64
+])
+def test_quantize_rejects_bad_arguments(lib, args, err):
+    assert lib.harp_quantize_weights(*args, FAKE, FAKE, FAKE, None) == err
+
+
+@pytest.mark.parametrize("n_in,n_out,bits,w_in,w_out,err", [
+    (4096, 4096, 1, 4096, 4096, 1),    # bits
+    (4000, 4096, 2, 4096, 4096, 1),    # n_in not a multiple of 256
+    (4096, 4096, 2, 32, 4096, 1),      # w_in below 64
+    (4096, 4096, 2, 4096, 3000, 1),    # w_out not a power of two
+    (11008, 4096, 2, 4096, 4096, 1),   # w_in does not divide n_in
+    (4096, 4096, 2, 16384, 4096, 1),   # w_in too wide
+])
+def test_create_layer_rejects_bad_arguments(lib, n_in, n_out, bits, w_in, w_out, err):
+    h = ctypes.c_void_p()
+    st = lib.harp_create_layer(ctypes.byref(h), n_in, n_out, bits, 64, w_in, w_out, FAKE, FAKE, FAKE, FAKE, FAKE,
+                               FAKE, None)
+    assert st == err and not h.value
+
+
+def test_null_handles(lib):
+    n = ctypes.c_size_t()
+    assert lib.harp_linear_workspace_size(None, 1, ctypes.byref(n)) == 1
+    assert lib.harp_linear_fwd(None, 1, FAKE, 0, FAKE, 0, FAKE, 1 << 20, None) == 1
+    assert lib.harp_destroy_layer(None) == 0
+    assert lib.harp_stack_destroy(None) == 0
+    assert lib.harp_stack_step(None, 1, FAKE, 0, FAKE, 0, FAKE, 1 << 20, None) == 1
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    from rotated_bit_matmul_b200 import _lib
+    with pytest.raises(ImportError):
+        saved = _lib._lib
+        _lib._lib = None
+        try:
+            _lib.load(str(tmp_path / "missing.so"))
+        finally:
+            _lib._lib = saved

@@ -1,0 +1,240 @@
+"""GPU parity: the sm_100a kernels, called through the C ABI, against the fp64 oracle
+on identical seeded inputs (codes and parameters produced by the oracle).
+
+Gates: relative L2 <= 2e-3 on the fp32-accumulate GEMV path (the figure the
+library's contract states for that path); butterflies alone <= 5e-6 (pure fp32
+arithmetic, ~13 stages); integer special cases and the quantizer's codes must match
+bit for bit.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+from harp_cases import device_layer, oracle_layer, rel_l2
+from rotated_bit_matmul_b200 import synth
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+GATE = 2e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from rotated_bit_matmul_b200 import build_lib, _lib
+    build_lib.build()
+    _lib.load()
+    yield
+    import rotated_bit_matmul_b200 as rb
+    torch.cuda.synchronize()
+    rb.harp_device_status()
+
+
+def _dev(a, dt):
+    return torch.from_numpy(np.ascontiguousarray(a)).to("cuda", dtype=dt)
+
+
+# ------------------------------------------------------------------ butterflies
+BFLY_CASES = [(1024, 1024, 1), (4096, 4096, 3), (11008, 256, 2), (8192, 8192, 1), (28672, 4096, 1),
+              (96, 32, 5), (6, 2, 2), (64, 64, 4), (2048, 128, 7)]
+
+
+@pytest.mark.parametrize("n,w,batch", BFLY_CASES)
+@pytest.mark.parametrize("inverse", [False, True])
+def test_butterfly_matches_oracle(n, w, batch, inverse):
+    import rotated_bit_matmul_b200 as rb
+    rng = np.random.default_rng(n + w + batch)
+    theta = rng.uniform(-0.05, 0.05, (int(math.log2(w)), n // 2)).astype(np.float32)
+    sign = (rng.integers(0, 2, n) * 2 - 1).astype(np.int8)
+    x = rng.standard_normal((batch, n)).astype(np.float32)
+    f = rb.harp_butterfly_inv if inverse else rb.harp_butterfly_fwd
+    got = f(_dev(x, torch.float32), _dev(theta, torch.float32), _dev(sign, torch.int8), w).cpu().numpy()
+    want = (oracle.butterfly_inv if inverse else oracle.butterfly_fwd)(x, theta, sign, w)
+    assert rel_l2(got, want) < 5e-6
+
+
+@pytest.mark.parametrize("xdt,ydt,gate", [("bfloat16", "float32", 5e-6), ("float32", "bfloat16", GATE),
+                                          ("float16", "float16", GATE)])
+def test_butterfly_dtypes_and_inplace(xdt, ydt, gate):
+    import rotated_bit_matmul_b200 as rb
+    n, w = 4096, 4096
+    rng = np.random.default_rng(5)
+    theta = rng.uniform(-0.05, 0.05, (12, n // 2)).astype(np.float32)
+    sign = (rng.integers(0, 2, n) * 2 - 1).astype(np.int8)
+    xd = _dev(rng.standard_normal((2, n)).astype(np.float32), getattr(torch, xdt))
+    xh = xd.float().cpu().numpy()
+    got = rb.harp_butterfly_fwd(xd, _dev(theta, torch.float32), _dev(sign, torch.int8), w,
+                                out_dtype=getattr(torch, ydt))
+    want = oracle.butterfly_fwd(xh, theta, sign, w)
+    assert rel_l2(got.float().cpu().numpy(), want) < gate
+    if xdt == ydt:  # in place
+        rb.harp_butterfly_fwd(xd, _dev(theta, torch.float32), _dev(sign, torch.int8), w, out=xd)
+        assert rel_l2(xd.float().cpu().numpy(), want) < gate
+
+
+def test_butterfly_theta0_is_hadamard():
+    import scipy.linalg
+    import rotated_bit_matmul_b200 as rb
+    n = 1024
+    sign = (np.random.default_rng(1).integers(0, 2, n) * 2 - 1).astype(np.int8)
+    x = np.eye(n, dtype=np.float32)[:64]
+    got = rb.harp_butterfly_fwd(_dev(x, torch.float32), torch.zeros((10, n // 2), device="cuda"),
+                                _dev(sign, torch.int8), n).cpu().numpy()
+    want = (scipy.linalg.hadamard(n) @ np.diag(sign.astype(float)) / 32.0).T[:64]
+    assert np.max(np.abs(got - want)) < 1e-6
+
+
+# ------------------------------------------------------------------ quantizer
+@pytest.mark.parametrize("bits", [2, 3, 4])
+@pytest.mark.parametrize("n_out,n_in", [(256, 4096), (100, 11008), (7, 64)])
+def test_quantize_matches_oracle_codes(bits, n_out, n_in):
+    import rotated_bit_matmul_b200 as rb
+    W = synth.weights(n_out, n_in, 2, 0, 4)
+    Wr32 = W.astype(np.float32)  # any fp32 matrix: both sides quantize the same values
+    Wr32[0, :64] = 0.37           # a constant group (scale forced to 1)
+    q, s16, z16 = oracle.quantize(Wr32.astype(np.float64), bits)
+    codes, sz = rb.harp_quantize_weights(_dev(Wr32, torch.float32), bits)
+    want_codes = oracle.pack(q, bits)
+    got_codes = codes.cpu().numpy()
+    got_q = oracle.unpack(got_codes, n_out, n_in, bits)
+    match = float(np.mean(got_q == q))
+    assert match >= 0.9999, match
+    assert np.array_equal(got_codes, want_codes)
+    got_sz = sz.cpu().numpy().view(np.uint16).reshape(n_out, n_in // 64, 2)
+    assert np.array_equal(got_sz[..., 0], s16) and np.array_equal(got_sz[..., 1], z16)
+
+
+# ------------------------------------------------------------------ linear
+def _linear_check(case, batch, xdt=torch.bfloat16, ydt=torch.float32, workload=2, gate=GATE):
+    x = synth.activations(batch, case["n_in"], workload, step=batch, bf16=(xdt == torch.bfloat16))
+    L = device_layer(case)
+    got = L(_dev(x, xdt), out_dtype=ydt).float().cpu().numpy()
+    want = oracle.linear_fwd(case["lay"], x.astype(np.float64))
+    err = rel_l2(got, want)
+    L.close()
+    assert err < gate, err
+    return err
+
+
+def test_config1_single_layer_fp32():
+    case = oracle_layer(1024, 1024, 1024, 1024, 2, workload=1)
+    _linear_check(case, 1, xdt=torch.float32, workload=1)
+
+
+@pytest.mark.parametrize("shape", synth.llama7b_linears(), ids=lambda s: s.name)
+def test_config2_llama7b_linears(shape):
+    case = oracle_layer(shape.n_out, shape.n_in, shape.w_in, shape.w_out, 2, linear=synth.LINEAR_NAMES.index(shape.name))
+    _linear_check(case, 1)
+
+
+@pytest.mark.parametrize("bits", [3, 4])
+@pytest.mark.parametrize("n_out,n_in,w_in,w_out", [(4096, 4096, 4096, 4096), (11008, 4096, 4096, 256),
+                                                   (4096, 11008, 256, 4096)])
+def test_bits_3_4(bits, n_out, n_in, w_in, w_out):
+    case = oracle_layer(n_out, n_in, w_in, w_out, bits, workload=5)
+    _linear_check(case, 1, workload=5)
+
+
+@pytest.mark.parametrize("batch", [2, 4, 8, 16, 64])
+def test_batch_sweep_4096(batch):
+    case = oracle_layer(4096, 4096, 4096, 4096, 2, workload=3)
+    _linear_check(case, batch, workload=3)
+
+
+@pytest.mark.parametrize("batch", [4, 16])
+def test_batch_sweep_11008(batch):
+    case = oracle_layer(11008, 4096, 4096, 256, 2, workload=3, linear=4)
+    _linear_check(case, batch, workload=3)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_ragged_shapes(bits):
+    """n_out = 200 (not a multiple of the 32-row tiles), n_in = 768 (a ragged last chunk)."""
+    case = oracle_layer(200, 768, 256, 8, bits, workload=9)
+    _linear_check(case, 3, workload=9)
+
+
+@pytest.mark.parametrize("ydt", [torch.bfloat16, torch.float16])
+def test_output_dtypes(ydt):
+    case = oracle_layer(1024, 2048, 1024, 512, 2, workload=8)
+    _linear_check(case, 2, ydt=ydt, gate=4e-3)
+
+
+def test_70b_shapes_one_each():
+    for sh in synth.llama70b_linears()[:3] + synth.llama70b_linears()[6:]:
+        case = oracle_layer(sh.n_out, sh.n_in, sh.w_in, sh.w_out, 2, workload=5, linear=synth.LINEAR_NAMES.index(sh.name))
+        _linear_check(case, 1, workload=5)
+
+
+def test_integer_special_case_bit_exact():
+    """theta = -pi/4 makes both butterflies diagonal +-1; with scale 1, zero 0 and small
+    integer inputs every step is exact, so y = D_U Q D_V x must come out bit for bit."""
+    import rotated_bit_matmul_b200 as rb
+    n_out, n_in = 384, 1024
+    rng = np.random.default_rng(3)
+    q = rng.integers(0, 4, (n_out, n_in)).astype(np.uint8)
+    sz = np.zeros((n_out, n_in // 64, 2), np.uint16)
+    sz[..., 0] = 0x3C00
+    qpi = np.float32(-np.pi / 4)
+    thV = np.full((10, n_in // 2), qpi, np.float32)
+    thU = np.full((7, n_out // 2), qpi, np.float32)
+    sV = (rng.integers(0, 2, n_in) * 2 - 1).astype(np.int8)
+    sU = (rng.integers(0, 2, n_out) * 2 - 1).astype(np.int8)
+    L = rb.HarpLayer(n_in, n_out, 2, 1024, 128, _dev(thV, torch.float32), _dev(sV, torch.int8),
+                     _dev(thU, torch.float32), _dev(sU, torch.int8), _dev(oracle.pack(q, 2), torch.uint8),
+                     _dev(sz.reshape(-1).view(np.int32), torch.int32))
+    x = rng.integers(-8, 9, (2, n_in)).astype(np.float32)
+    got = L(_dev(x, torch.float32)).cpu().numpy()
+    dV = sV * np.array([(-1.0) ** bin(i % 1024).count("1") for i in range(n_in)])
+    dU = sU * np.array([(-1.0) ** bin(i % 128).count("1") for i in range(n_out)])
+    want = (q.astype(np.float64) @ (x * dV).T).T * dU
+    assert np.array_equal(got.astype(np.float64), want)
+
+
+def test_workspace_errors():
+    import rotated_bit_matmul_b200 as rb
+    case = oracle_layer(256, 512, 512, 256, 2, workload=9)
+    L = device_layer(case)
+    x = torch.zeros((1, 512), device="cuda")
+    with pytest.raises(rb.HarpError) as e:
+        L(x, workspace=torch.empty(16, dtype=torch.uint8, device="cuda"))
+    assert e.value.status == 4
+    L.close()
+
+
+# ------------------------------------------------------------------ stack
+def _stack_case(n_layers, dims, workload, wide_ffn_block):
+    hidden, ffn, nh, nkv, hd = dims
+    dq, dkv = nh * hd, nkv * hd
+    shapes = [(dq, hidden), (dkv, hidden), (dkv, hidden), (hidden, dq), (ffn, hidden), (ffn, hidden), (hidden, ffn)]
+    cases = []
+    for l in range(n_layers):
+        for i, (n_out, n_in) in enumerate(shapes):
+            w_in = wide_ffn_block if n_in == ffn else n_in
+            w_out = wide_ffn_block if n_out == ffn else n_out
+            cases.append(oracle_layer(n_out, n_in, min(w_in, 8192), min(w_out, 8192), 2, workload, l, i))
+    return cases
+
+
+@pytest.mark.parametrize("dims,n_layers,block,batch", [
+    ((256, 768, 4, 2, 64), 2, 256, 1),
+    ((256, 768, 4, 2, 64), 2, 256, 3),
+    ((4096, 11008, 32, 32, 128), 1, 256, 1),
+])
+def test_stack_matches_oracle(dims, n_layers, block, batch):
+    import rotated_bit_matmul_b200 as rb
+    cases = _stack_case(n_layers, dims, 4, block)
+    layers = [device_layer(c) for c in cases]
+    S = rb.HarpStack(layers, *dims)
+    x = synth.activations(batch, dims[0], 4, step=0)
+    got = S.step(_dev(x, torch.bfloat16)).cpu().numpy()
+    want = oracle.stack_step([c["lay"] for c in cases], *dims, x.astype(np.float64))
+    err = rel_l2(got, want)
+    S.close()
+    for l in layers:
+        l.close()
+    assert err < GATE, err
