@@ -132,6 +132,25 @@ harp_status harp_linear_workspace_size(harp_layer layer, int batch, size_t* byte
 harp_status harp_linear_fwd(harp_layer layer, int batch, const void* x, harp_dtype xt, void* y,
                             harp_dtype yt, void* workspace, size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------- linear, no allocation
+ * harp_linear_fwd for callers that cannot allocate device memory: code that runs inside
+ * another framework's memory pool, real-time paths where an allocation may block or
+ * fail, and hosts that hand the library only pre-registered buffers. The paper has no
+ * counterpart; this is a library convenience. Its scratch is a 2 MiB array in the
+ * library's device image, which every GPU that loads the library holds until exit.
+ *   x, y  : as for harp_linear_fwd (caller-owned device memory); no workspace argument.
+ *   Fails with HARP_ERR_WORKSPACE when the layer and batch need more than 2 MiB of
+ *   scratch (harp_linear_workspace_size says how much).
+ *   The first call on a device looks up the array's device address; make that first
+ *   call before any stream capture. All calls on a device share the array and it keeps
+ *   the last call's contents (nothing in it must start at zero): calls that overlap on
+ *   the GPU (other streams, other host threads) race, so serialise them.
+ *   Allocates nothing (no cudaMalloc, cudaFree or allocating library routine); for the
+ *   same reason a device-side wait that runs out ends the kernel without a status report.
+ */
+harp_status harp_linear_fwd_static(harp_layer layer, int batch, const void* x, harp_dtype xt, void* y,
+                                   harp_dtype yt, void* stream);
+
 /* ---------------------------------------------------------------- decoder stack
  * A Llama-shaped stack of n_layers blocks, each with seven rotated linears in the
  * order q, k, v, o, gate, up, down (layers[7*l + i]). One decode step computes, per

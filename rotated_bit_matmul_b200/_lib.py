@@ -34,6 +34,7 @@ SIGNATURES = {
     "harp_destroy_layer": (_I, [_P]),
     "harp_linear_workspace_size": (_I, [_P, _I, ctypes.POINTER(_SZ)]),
     "harp_linear_fwd": (_I, [_P, _I, _P, _I, _P, _I, _P, _SZ, _P]),
+    "harp_linear_fwd_static": (_I, [_P, _I, _P, _I, _P, _I, _P]),
     "harp_stack_create": (_I, [ctypes.POINTER(_P), _I, _I, _I, _I, _I, _I, ctypes.c_float, ctypes.POINTER(_P), _P]),
     "harp_stack_destroy": (_I, [_P]),
     "harp_stack_workspace_size": (_I, [_P, _I, ctypes.POINTER(_SZ)]),
