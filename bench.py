@@ -163,7 +163,9 @@ def build_stack(n_layers, device):
     return rb.HarpStack(layers, HIDDEN, FFN, NH, NKV, HD)
 
 
-def launches_per_step(n_layers):
+def launches_per_step(n_layers, fused):
+    if fused:
+        return 1  # the fused decode-step kernel (its counter reset is a cudaMemsetAsync)
     # one convert + per block: 2 RMSNorm, 7 x (input butterfly, GEMV, output butterfly),
     # 2 residual adds, 1 SiLU*up (no repeat: 32 query heads over 32 kv heads) + one store
     return 1 + n_layers * (2 + 7 * 3 + 2 + 1) + 1
@@ -193,6 +195,11 @@ def run_ours(args, rank, world):
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream):
         stack.step(x_in, out=y, workspace=ws)
+    stream.synchronize()
+    with torch.cuda.stream(stream):  # the first replays upload the graph: keep them untimed
+        for s in range(max(Wm, 3)):
+            x_in.copy_(xs[s])
+            g.replay()
     stream.synchronize()
 
     def barrier():
@@ -248,13 +255,14 @@ def run_ours(args, rank, world):
     nbytes = algorithmic_bytes_per_step(args.layers)
     peak, peak_kind = measured_peak()
     achieved = nbytes / (ms_step * 1e-3) / 1e9
+    fused = stack.uses_fused_step(BATCH)
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": None,
-                "kernel": "whole decode step (graph of the step's kernels)", "peak_kind": peak_kind,
-                "algorithmic_bytes_per_step": nbytes}
+                "kernel": "decode_kernel (one launch per step)" if fused else "whole decode step (graph of kernels)",
+                "peak_kind": peak_kind, "algorithmic_bytes_per_step": nbytes}
     del g
     return dict(value=value, ms_step=ms_step, e2e=e2e, roofline=roofline, clocks=clk.summary(),
-                launches=launches_per_step(args.layers) * K)
+                launches=launches_per_step(args.layers, fused) * K, fused=fused)
 
 
 def main():

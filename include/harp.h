@@ -169,6 +169,12 @@ harp_status harp_stack_create(harp_stack* out, int n_layers, int hidden, int ffn
 harp_status harp_stack_destroy(harp_stack stack);
 harp_status harp_stack_workspace_size(harp_stack stack, int batch, size_t* bytes);
 
+/* 1 when harp_stack_step with this batch runs the fused single-kernel decode step
+ * (batch 1, hidden a power of two in [4096, 8192], n_heads*head_dim == hidden, single-block
+ * q/k/v/o/down butterflies, gate/up output blocks 64..512 wide, one bit width), else 0
+ * (the step then runs one launch sequence per linear). */
+int harp_stack_uses_fused_step(harp_stack stack, int batch);
+
 /* One decode step: out = stack(x). x, out: device [batch][hidden] of dtypes xt / ot
  * (batch 1..256); out may equal x. workspace as for harp_linear_fwd. */
 harp_status harp_stack_step(harp_stack stack, int batch, const void* x, harp_dtype xt, void* out,

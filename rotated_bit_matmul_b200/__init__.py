@@ -168,6 +168,10 @@ class HarpStack:
         call("harp_stack_workspace_size", self.handle, int(batch), ctypes.byref(n))
         return n.value
 
+    def uses_fused_step(self, batch: int = 1) -> bool:
+        """True when a step of this batch runs the single-kernel fused decode path."""
+        return bool(load().harp_stack_uses_fused_step(self.handle, int(batch)))
+
     def workspace(self, batch: int):
         ws = self._ws.get(batch)
         if ws is None:

@@ -39,6 +39,7 @@ SIGNATURES = {
     "harp_stack_destroy": (_I, [_P]),
     "harp_stack_workspace_size": (_I, [_P, _I, ctypes.POINTER(_SZ)]),
     "harp_stack_step": (_I, [_P, _I, _P, _I, _P, _I, _P, _SZ, _P]),
+    "harp_stack_uses_fused_step": (_I, [_P, _I]),
 }
 
 

@@ -7,122 +7,301 @@
 // Forward: signs, then stages of stride 1, 2, ..., w/2. Transpose: stages in
 // reverse, then signs (each 2x2 block is symmetric).
 //
-// One CTA owns one w-wide block (w <= 8192, 32 KB of fp32 in shared memory) of one
-// row and runs all log2(w) stages there; the optional epilogue turns the result
-// into the operand the dequant-GEMV reads (int16 values in dp2a pair order, one
-// power-of-two scale and one fp32 sum per group of 64).
+// Work split. A w-wide block is held by a thread-block cluster of C CTAs (C = 8 for
+// w >= 4096, 4 for 2048, 2 for 1024, else 1), E = w / C elements each:
+//   layout A: CTA r holds the contiguous chunk [r E, (r+1) E) -> stages 0 .. e-1
+//             (e = log2 E) are local;
+//   layout B: CTA r holds, for every chunk j, the run [j E + r E/C, j E + (r+1) E/C)
+//             -> the remaining log2 C stages (which pair chunk j with j + 2^d) are local.
+// Switching layouts is one gather through distributed shared memory between two
+// cluster barriers. Each CTA first prefetches exactly its slice of the per-stage
+// parameters (cos/sin pairs of the layer, or raw theta for the stand-alone API) with
+// bulk copies into shared memory, so no stage waits on global memory.
+// The forward epilogue can also emit the GEMV operand: per group of 64 outputs an
+// int16 copy in dp2a pair order, the power-of-two scale and the fp32 group sum.
 #include "common.cuh"
 
 namespace harp {
 
-// Position (int16 index inside the group's 32-word block) of column j (0..63) of a
-// group in the dp2a pair order the GEMV expects for its code format.
-__device__ __forceinline__ int xq_pos_lo(int bits, int j) {
-  if (bits == 4) {
-    const int c = j >> 3, r = j & 7;
-    return (c * 4 + (r & 1) * 2 + (r >> 2)) * 2 + ((r >> 1) & 1);
-  }
-  const int c = j >> 4, r = j & 15, m = r & 3, q = r >> 2;  // 2-bit codes / 2-bit plane
-  return (c * 8 + 2 * m + (q >> 1)) * 2 + (q & 1);
-}
-__device__ __forceinline__ int xq_pos_hi(int j) {  // 1-bit plane of 3-bit codes
-  const int c = j >> 5, r = j & 31, m = r & 7, q = r >> 3;
-  return (c * 16 + 2 * m + (q >> 1)) * 2 + (q & 1);
+namespace {
+
+constexpr int kBflyThreads = 256;
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
 }
 
-__global__ void __launch_bounds__(512) bfly_kernel(BflyParams p) {
-  extern __shared__ float sx[];
-  const int w = p.w, m = p.m;
-  const int64_t k = blockIdx.x, row = blockIdx.y;
-  const int64_t base = k * w;
-  const int nthr = blockDim.x, tid = threadIdx.x;
-  const int64_t half_n = p.n >> 1;
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ float ld_dsmem(const float* local, uint32_t cta) {
+  uint32_t ra;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(local)), "r"(cta));
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(ra) : "memory");
+  return v;
+}
+
+struct Geom {
+  int C, lc, E, e, run;  // cluster size, log2 C, elements per CTA, log2 E, E / C
+};
+
+__device__ __forceinline__ Geom geom(int w, int m, int C) {
+  Geom g;
+  g.C = C;
+  g.lc = 31 - __clz(C);
+  g.E = w / C;
+  g.e = m - g.lc;
+  g.run = g.E / C;
+  return g;
+}
+
+// one stage on the layout-A buffer: local pairs (i, i + 2^t), parameter slot q
+template <bool CS>
+__device__ __forceinline__ void stage_a(float* x, const void* tab, int t, int E, int tid, int nthr) {
+  const int h = 1 << t;
   const float kQuarterPi = 0.785398163397448309616f;
-
-  for (int i = tid; i < w; i += nthr) {
-    float v = load_act(p.x, row * p.x_stride + base + i, p.xt);
-    if (!p.inverse) v *= (float)p.sign[base + i];
-    sx[i] = v;
+  for (int q = tid; q < (E >> 1); q += nthr) {
+    const int i = ((q >> t) << (t + 1)) | (q & (h - 1));
+    float c, s;
+    if (CS) {
+      const float2 v = static_cast<const float2*>(tab)[q];
+      c = v.x;
+      s = v.y;
+    } else {
+      sincosf(kQuarterPi + static_cast<const float*>(tab)[q], &s, &c);
+    }
+    const float a = x[i], b = x[i + h];
+    x[i] = fmaf(c, a, s * b);
+    x[i + h] = fmaf(s, a, -c * b);
   }
-  __syncthreads();
+}
 
-  for (int s = 0; s < m; ++s) {
-    const int t = p.inverse ? (m - 1 - s) : s;
-    const int h = 1 << t;
-    const int64_t off = (int64_t)t * half_n + k * (w >> 1);
-    for (int q = tid; q < (w >> 1); q += nthr) {
-      const int i = ((q >> t) << (t + 1)) | (q & (h - 1));
-      float c, sn;
-      if (p.cs) {
-        const float2 v = p.cs[off + q];
-        c = v.x;
-        sn = v.y;
-      } else {
-        sincosf(kQuarterPi + p.theta[off + q], &sn, &c);
+// one stage on the layout-B buffer: runs j and j + 2^d (bit d of j clear), same offset
+template <bool CS>
+__device__ __forceinline__ void stage_b(float* x, const void* tab, int d, int run, int E, int tid, int nthr) {
+  const float kQuarterPi = 0.785398163397448309616f;
+  for (int q = tid; q < (E >> 1); q += nthr) {
+    const int jj = q / run, ii = q - jj * run;
+    const int j = ((jj >> d) << (d + 1)) | (jj & ((1 << d) - 1));
+    float c, s;
+    if (CS) {
+      const float2 v = static_cast<const float2*>(tab)[q];
+      c = v.x;
+      s = v.y;
+    } else {
+      sincosf(kQuarterPi + static_cast<const float*>(tab)[q], &s, &c);
+    }
+    float* pa = x + j * run + ii;
+    float* pb = pa + (run << d);
+    const float a = *pa, b = *pb;
+    *pa = fmaf(c, a, s * b);
+    *pb = fmaf(s, a, -c * b);
+  }
+}
+
+template <bool CS>
+__global__ void __launch_bounds__(kBflyThreads) bfly_kernel(BflyParams p, int C) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  const Geom g = geom(p.w, p.m, C);
+  const int w = p.w, m = p.m, E = g.E, run = g.run;
+  const int tid = threadIdx.x, nthr = blockDim.x;
+  const uint32_t r = C > 1 ? cluster_rank() : 0;
+  const int64_t blk = blockIdx.x / C, row = blockIdx.y;
+  const int64_t base = blk * w;
+  const int64_t half_n = p.n >> 1;
+  constexpr int esz = CS ? 8 : 4;
+
+  float* xa = reinterpret_cast<float*>(sm);
+  float* xb = xa + E;
+  uint8_t* tab = reinterpret_cast<uint8_t*>(xb + E);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(tab + (size_t)m * (E >> 1) * esz);
+  const void* gtab = CS ? static_cast<const void*>(p.cs) : static_cast<const void*>(p.theta);
+
+  // ---- prefetch this CTA's parameter slice: stage t occupies E/2 entries. Bulk copies
+  // need 16-byte aligned sources, destinations and sizes; tiny widths use plain loads.
+  const bool use_bulk = (((E >> 1) * esz) % 16 == 0) && ((half_n * esz) % 16 == 0) &&
+                        (((w >> 1) * esz) % 16 == 0) && (C == 1 || (run * esz) % 16 == 0);
+  if (!use_bulk) {
+    for (int t = 0; t < m; ++t) {
+      const uint8_t* src_stage = static_cast<const uint8_t*>(gtab) + ((int64_t)t * half_n + blk * (w >> 1)) * esz;
+      uint8_t* dst = tab + (size_t)t * (E >> 1) * esz;
+      for (int q = tid; q < (E >> 1); q += nthr) {
+        int64_t src_q;
+        if (t < g.e) {
+          src_q = (int64_t)r * (E >> 1) + q;
+        } else {
+          const int d = t - g.e, jj = q / run, ii = q - jj * run;
+          const int j = ((jj >> d) << (d + 1)) | (jj & ((1 << d) - 1));
+          src_q = (int64_t)(j >> (d + 1)) * (1 << t) + (int64_t)E * (j & ((1 << d) - 1)) + (int64_t)r * run + ii;
+        }
+        for (int b = 0; b < esz; b += 4)
+          *reinterpret_cast<uint32_t*>(dst + (size_t)q * esz + b) =
+              *reinterpret_cast<const uint32_t*>(src_stage + src_q * esz + b);
       }
-      const float a = sx[i], b = sx[i + h];
-      sx[i] = fmaf(c, a, sn * b);
-      sx[i + h] = fmaf(sn, a, -c * b);
+    }
+  } else if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(bar, (uint32_t)(m * (E >> 1) * esz));
+    for (int t = 0; t < m; ++t) {
+      const uint8_t* src_stage = static_cast<const uint8_t*>(gtab) + ((int64_t)t * half_n + blk * (w >> 1)) * esz;
+      uint8_t* dst = tab + (size_t)t * (E >> 1) * esz;
+      if (t < g.e) {
+        bulk_g2s(dst, src_stage + (int64_t)r * (E >> 1) * esz, (uint32_t)((E >> 1) * esz), bar);
+      } else {
+        const int d = t - g.e;
+        for (int jj = 0; jj < (C >> 1); ++jj) {
+          const int j = ((jj >> d) << (d + 1)) | (jj & ((1 << d) - 1));
+          const int64_t pbase = (int64_t)(j >> (d + 1)) * (1 << t) + (int64_t)E * (j & ((1 << d) - 1)) + (int64_t)r * run;
+          bulk_g2s(dst + (size_t)jj * run * esz, src_stage + pbase * esz, (uint32_t)(run * esz), bar);
+        }
+      }
+    }
+  }
+
+  if (!p.inverse) {
+    // ---- load chunk r (layout A), signs first
+    for (int i = tid; i < E; i += nthr) {
+      const int64_t gi = base + (int64_t)r * E + i;
+      xa[i] = load_act(p.x, row * p.x_stride + gi, p.xt) * (float)p.sign[gi];
     }
     __syncthreads();
-  }
-
-  if (p.inverse)
-    for (int i = tid; i < w; i += nthr) sx[i] *= (float)p.sign[base + i];
-  if (p.inverse) __syncthreads();
-
-  if (p.y)
-    for (int i = tid; i < w; i += nthr) store_act(p.y, row * p.y_stride + base + i, p.yt, sx[i]);
-
-  if (p.xq) {
-    // Per group of 64: e = 15 - E with max|v| = f 2^E, f in [0.5, 1), so that
-    // max|v| 2^e < 2^15; int16 value = rint(v 2^e) (clamped to +-32767).
-    const int lane = tid & 31, warp = tid >> 5, nwarps = nthr >> 5;
-    int16_t* xq16 = reinterpret_cast<int16_t*>(p.xq + row * p.xq_stride);
-    for (int g = warp; g < (w >> 6); g += nwarps) {
-      const float v0 = sx[g * 64 + 2 * lane], v1 = sx[g * 64 + 2 * lane + 1];
-      float amax = fmaxf(fabsf(v0), fabsf(v1));
-      float sum = v0 + v1;
-      const bool bad = __any_sync(0xffffffffu, !(isfinite(v0) && isfinite(v1)));
+    if (use_bulk) mbar_wait(bar, 0, p.status, 10);
+    for (int t = 0; t < g.e; ++t) {
+      stage_a<CS>(xa, tab + (size_t)t * (E >> 1) * esz, t, E, tid, nthr);
+      __syncthreads();
+    }
+    float* out = xa;
+    if (C > 1) {
+      cluster_sync();
+      for (int L = tid; L < E; L += nthr) {
+        const int j = L / run, ii = L - j * run;
+        xb[L] = ld_dsmem(xa + r * run + ii, (uint32_t)j);
+      }
+      cluster_sync();  // every peer has finished reading this CTA's chunk
+      for (int d = 0; d < g.lc; ++d) {
+        stage_b<CS>(xb, tab + (size_t)(g.e + d) * (E >> 1) * esz, d, run, E, tid, nthr);
+        __syncthreads();
+      }
+      out = xb;
+    }
+    // local index L <-> global element: layout A: r E + L; layout B: j E + r run + ii
+    auto gidx = [&](int L) -> int64_t {
+      if (C == 1) return base + L;
+      const int j = L / run, ii = L - j * run;
+      return base + (int64_t)j * E + (int64_t)r * run + ii;
+    };
+    if (p.y)
+      for (int L = tid; L < E; L += nthr) store_act(p.y, row * p.y_stride + gidx(L), p.yt, out[L]);
+    if (p.xq) {
+      // groups of 64 consecutive outputs (runs are >= 64 long): int16 at scale 2^e with
+      // max|v| 2^e < 2^15 (e = 15 - E', max|v| = f 2^E', f in [0.5, 1))
+      const int lane = tid & 31, warp = tid >> 5, nwarps = nthr >> 5;
+      int16_t* xq16 = reinterpret_cast<int16_t*>(p.xq + row * p.xq_stride);
+      for (int gl = warp; gl < (E >> 6); gl += nwarps) {
+        const float v0 = out[gl * 64 + 2 * lane], v1 = out[gl * 64 + 2 * lane + 1];
+        float amax = fmaxf(fabsf(v0), fabsf(v1));
+        float sum = v0 + v1;
+        const bool bad = __any_sync(0xffffffffu, !(isfinite(v0) && isfinite(v1)));
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        for (int o = 16; o > 0; o >>= 1) {
+          amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+          sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        }
+        int ex = 0;
+        if (amax > 0.f && !bad) {
+          int E2;
+          frexpf(amax, &E2);
+          ex = min(max(15 - E2, -126), 126);
+        }
+        const float sc = ldexpf(1.f, ex);
+        const int q0 = max(-32767, min(32767, __float2int_rn(v0 * sc)));
+        const int q1 = max(-32767, min(32767, __float2int_rn(v1 * sc)));
+        const int64_t gg = gidx(gl * 64) >> 6;  // global group index
+        int16_t* grp = xq16 + gg * 64;
+        grp[xq_pos_lo(p.bits, 2 * lane)] = (int16_t)q0;
+        grp[xq_pos_lo(p.bits, 2 * lane + 1)] = (int16_t)q1;
+        if (p.bits == 3) {
+          int16_t* hi = xq16 + p.n + gg * 64;  // the 1-bit-plane order follows n int16 values
+          hi[xq_pos_hi(2 * lane)] = (int16_t)q0;
+          hi[xq_pos_hi(2 * lane + 1)] = (int16_t)q1;
+        }
+        if (lane == 0) {
+          p.xs[row * p.g_stride + gg] = bad ? __int_as_float(0x7fc00000) : ldexpf(1.f, -ex);
+          p.xsum[row * p.g_stride + gg] = bad ? __int_as_float(0x7fc00000) : sum;
+        }
       }
-      int e = 0;
-      if (amax > 0.f && !bad) {
-        int E;
-        frexpf(amax, &E);
-        e = min(max(15 - E, -126), 126);
+    }
+  } else {
+    // ---- transpose: high stages first (layout B), then the local ones (layout A)
+    float* cur = xa;
+    if (C > 1) {
+      for (int L = tid; L < E; L += nthr) {
+        const int j = L / run, ii = L - j * run;
+        xb[L] = load_act(p.x, row * p.x_stride + base + (int64_t)j * E + (int64_t)r * run + ii, p.xt);
       }
-      const float sc = ldexpf(1.f, e);
-      const int q0 = max(-32767, min(32767, __float2int_rn(v0 * sc)));
-      const int q1 = max(-32767, min(32767, __float2int_rn(v1 * sc)));
-      const int64_t gg = k * (w >> 6) + g;
-      int16_t* grp = xq16 + gg * 64;
-      grp[xq_pos_lo(p.bits, 2 * lane)] = (int16_t)q0;
-      grp[xq_pos_lo(p.bits, 2 * lane + 1)] = (int16_t)q1;
-      if (p.bits == 3) {
-        int16_t* hi = xq16 + p.n + gg * 64;  // hi-plane order starts after n int16 values
-        hi[xq_pos_hi(2 * lane)] = (int16_t)q0;
-        hi[xq_pos_hi(2 * lane + 1)] = (int16_t)q1;
+      __syncthreads();
+      if (use_bulk) mbar_wait(bar, 0, p.status, 11);
+      for (int d = g.lc - 1; d >= 0; --d) {
+        stage_b<CS>(xb, tab + (size_t)(g.e + d) * (E >> 1) * esz, d, run, E, tid, nthr);
+        __syncthreads();
       }
-      if (lane == 0) {
-        p.xs[row * p.g_stride + gg] = bad ? __int_as_float(0x7fc00000) : ldexpf(1.f, -e);
-        p.xsum[row * p.g_stride + gg] = bad ? __int_as_float(0x7fc00000) : sum;
+      cluster_sync();
+      for (int u = tid; u < E; u += nthr) {
+        const int q = u / run;  // owner CTA of chunk-r element u in layout B
+        xa[u] = ld_dsmem(xb + r * run + (u - q * run), (uint32_t)q);
       }
+      cluster_sync();
+    } else {
+      for (int i = tid; i < E; i += nthr) xa[i] = load_act(p.x, row * p.x_stride + base + i, p.xt);
+      __syncthreads();
+      if (use_bulk) mbar_wait(bar, 0, p.status, 11);
+    }
+    for (int t = g.e - 1; t >= 0; --t) {
+      stage_a<CS>(cur, tab + (size_t)t * (E >> 1) * esz, t, E, tid, nthr);
+      __syncthreads();
+    }
+    for (int i = tid; i < E; i += nthr) {
+      const int64_t gi = base + (int64_t)r * E + i;
+      store_act(p.y, row * p.y_stride + gi, p.yt, cur[i] * (float)p.sign[gi]);
     }
   }
 }
+
+int cluster_for(int w) { return w >= 4096 ? 8 : (w == 2048 ? 4 : (w == 1024 ? 2 : 1)); }
+
+}  // namespace
 
 cudaError_t launch_butterfly(const BflyParams& p, int batch, cudaStream_t st) {
   if (batch <= 0) return cudaSuccess;
-  const int threads = p.w >= 1024 ? 512 : (p.w >= 64 ? p.w / 2 : 32);
-  const size_t smem = sizeof(float) * (size_t)p.w;
-  // at most 32 KB of dynamic shared memory: below the default 48 KB limit
-  dim3 grid((unsigned)(p.n / p.w), (unsigned)batch);
-  bfly_kernel<<<grid, threads, smem, st>>>(p);
-  return cudaGetLastError();
+  const int C = cluster_for(p.w);
+  const int E = p.w / C;
+  const bool cs = p.cs != nullptr;
+  const size_t smem = sizeof(float) * 2 * (size_t)E + (size_t)p.m * (E / 2) * (cs ? 8 : 4) + 16;
+  int threads = E / 2 < kBflyThreads ? E / 2 : kBflyThreads;
+  if (threads < 32) threads = 32;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((p.n / p.w) * C), (unsigned)batch, 1);
+  cfg.blockDim = dim3((unsigned)threads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cs ? cudaFuncSetAttribute(bfly_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
+                       : cudaFuncSetAttribute(bfly_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  return cs ? cudaLaunchKernelEx(&cfg, bfly_kernel<true>, p, C) : cudaLaunchKernelEx(&cfg, bfly_kernel<false>, p, C);
 }
 
 // cos/sin tables of pi/4 + theta, computed once per layer in fp32.

@@ -95,6 +95,14 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, uint64_
       : "memory");
 }
 
+// 1-D bulk copy global -> shared (16-byte aligned addresses, size a multiple of 16)
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
 __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
 }
@@ -119,6 +127,21 @@ __device__ __forceinline__ int4 ldg_nc_v4(const int4* p) {
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "l"(p));
   return v;
+}
+
+// Position (int16 index inside the group's 32-word block) of column j (0..63) of a
+// group in the dp2a pair order the GEMV expects for its code format.
+__device__ __forceinline__ int xq_pos_lo(int bits, int j) {
+  if (bits == 4) {
+    const int c = j >> 3, r = j & 7;
+    return (c * 4 + (r & 1) * 2 + (r >> 2)) * 2 + ((r >> 1) & 1);
+  }
+  const int c = j >> 4, r = j & 15, m = r & 3, q = r >> 2;  // 2-bit codes / 2-bit plane
+  return (c * 8 + 2 * m + (q >> 1)) * 2 + (q & 1);
+}
+__device__ __forceinline__ int xq_pos_hi(int j) {  // 1-bit plane of 3-bit codes
+  const int c = j >> 5, r = j & 31, m = r & 7, q = r >> 3;
+  return (c * 16 + 2 * m + (q >> 1)) * 2 + (q & 1);
 }
 
 // ------------------------------------------------------------------ programmatic dependent launch

@@ -1,0 +1,56 @@
+// Fused batch-1 decode step: shared host/device declarations.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace harp {
+namespace dec {
+
+constexpr int kC = 8;                // CTAs per cluster
+constexpr int kCW = 16;              // consumer warps per CTA
+constexpr int kNT = 32 * kCW;        // consumer threads
+constexpr int kThreads = kNT + 32;   // + one producer warp
+constexpr int kMaxClusters = 64;
+
+// One linear as the fused kernel sees it (device array, 64-byte aligned for the maps).
+struct alignas(64) Lin {
+  CUtensorMap tm_codes, tm_hi, tm_sz;
+  const float2* csV;
+  const float2* csU;
+  const int8_t* sV;
+  const int8_t* sU;
+  int n_in, n_out, w_in, w_out, m_in, m_out, pad0, pad1;
+};
+
+struct Params {
+  const Lin* lin;  // [L][7]: q, k, v, o, gate, up, down
+  int L, hidden, ffn, n_heads, n_kv, head_dim, rep, bits;
+  float eps;
+  int G;           // clusters in the grid
+  int E;           // hidden / kC
+  int m_hidden;    // log2(hidden)
+  const void* x_in;
+  int xt;
+  void* y_out;
+  int yt;
+  float *zq, *zk, *qout, *kout;  // [L][dq], [L][dkv]
+  float *zv, *zo, *zg, *zu, *zd;
+  int32_t* xq_down;
+  float* xs_down;
+  float* xsum_down;
+  unsigned* counters;  // [L][5], zero at launch
+  int* status;
+  int ring_stages, tab_bytes, xq_bytes;
+  int asg_qkv[kMaxClusters], idx_qkv[kMaxClusters], cnt_qkv[3];
+  int asg_gu[kMaxClusters], idx_gu[kMaxClusters], cnt_gu[2];
+};
+
+cudaError_t launch(const Params& p, cudaStream_t st);
+size_t smem_for(const Params& p);
+int stage_bytes_for(int bits);
+cudaError_t max_clusters(const Params& p, int* out);
+
+}  // namespace dec
+}  // namespace harp

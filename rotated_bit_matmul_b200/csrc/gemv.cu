@@ -14,97 +14,17 @@
 // a ring of shared-memory stages guarded by mbarriers; consumer warps own one output
 // row per lane and split each stage's groups between them. Every CTA gets a
 // contiguous, balanced range of output rows; the grid is one CTA per SM.
-#include "common.cuh"
+#include "gemv_core.cuh"
 
 namespace harp {
 
 namespace {
 
+using namespace gemv_core;
+
 constexpr int kConsumerWarps = 8;
 constexpr int kThreads = 32 * (1 + kConsumerWarps);
-constexpr int kStages = 6;
-constexpr int kSlab = 32 * 128;  // one TMA box: 32 rows x 128 bytes
-
-template <int BITS>
-struct Geo {
-  static constexpr int kChunkCols = BITS == 4 ? 1024 : 2048;  // columns per stage
-  static constexpr int kChunkGroups = kChunkCols / 64;
-  static constexpr int kGroupsPerSlab = BITS == 4 ? 4 : 8;       // codes (or 2-bit plane)
-  static constexpr int kCodeSlabs = kChunkGroups / kGroupsPerSlab;
-  static constexpr int kHiSlabs = BITS == 3 ? kChunkGroups / 16 : 0;  // 1-bit plane
-  static constexpr int kStageBytes = (kCodeSlabs + kHiSlabs + 1) * kSlab;
-};
-
-// Address of the 16-byte chunk `c` (0..7) of `row` inside a 128B-swizzled box.
-__device__ __forceinline__ const uint8_t* swz(const uint8_t* slab, int row, int c) {
-  return slab + row * 128 + ((c ^ (row & 7)) << 4);
-}
-
-template <int BITS>
-__device__ __forceinline__ int group_dot(const uint8_t* codes_slabs, const uint8_t* hi_slabs, int lane,
-                                         int gl, const int4* __restrict__ xg, const int4* __restrict__ xgh) {
-  if constexpr (BITS == 2 || BITS == 3) {
-    const uint4 cw = *reinterpret_cast<const uint4*>(swz(codes_slabs + (gl >> 3) * kSlab, lane, gl & 7));
-    const uint32_t wv[4] = {cw.x, cw.y, cw.z, cw.w};
-    int a0 = 0, a1 = 0, a2 = 0, a3 = 0;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int4 xa = ldg_nc_v4(xg + 2 * k), xb = ldg_nc_v4(xg + 2 * k + 1);
-      const uint32_t w = wv[k];
-      const uint32_t m0 = w & 0x03030303u, m1 = w & 0x0C0C0C0Cu, m2 = w & 0x30303030u, m3 = w & 0xC0C0C0C0u;
-      a0 = dp2a_lo(xa.x, m0, a0);
-      a0 = dp2a_hi(xa.y, m0, a0);
-      a1 = dp2a_lo(xa.z, m1, a1);
-      a1 = dp2a_hi(xa.w, m1, a1);
-      a2 = dp2a_lo(xb.x, m2, a2);
-      a2 = dp2a_hi(xb.y, m2, a2);
-      a3 = dp2a_lo(xb.z, m3, a3);
-      a3 = dp2a_hi(xb.w, m3, a3);
-    }
-    int acc = a0 + (a1 >> 2) + (a2 >> 4) + (a3 >> 6);
-    if constexpr (BITS == 3) {
-      const int gh = gl & 15;
-      const uint2 hw = *reinterpret_cast<const uint2*>(swz(hi_slabs + (gl >> 4) * kSlab, lane, gh >> 1) + (gh & 1) * 8);
-      const uint32_t hv[2] = {hw.x, hw.y};
-      int h = 0;
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-#pragma unroll
-        for (int mm = 0; mm < 8; mm += 2) {
-          const int4 xa = ldg_nc_v4(xgh + 4 * k + mm / 2);
-          const uint32_t ma = hv[k] & (0x01010101u << mm), mb = hv[k] & (0x01010101u << (mm + 1));
-          int ha = 0, hb = 0;
-          ha = dp2a_lo(xa.x, ma, ha);
-          ha = dp2a_hi(xa.y, ma, ha);
-          hb = dp2a_lo(xa.z, mb, hb);
-          hb = dp2a_hi(xa.w, mb, hb);
-          h += (ha >> mm) + (hb >> (mm + 1));
-        }
-      }
-      acc += 4 * h;
-    }
-    return acc;
-  } else {  // 4-bit: two 16-byte chunks per group, 8 codes per word
-    const uint8_t* slab = codes_slabs + (gl >> 2) * kSlab;
-    const int c0 = (gl & 3) * 2;
-    const uint4 ca = *reinterpret_cast<const uint4*>(swz(slab, lane, c0));
-    const uint4 cb = *reinterpret_cast<const uint4*>(swz(slab, lane, c0 + 1));
-    const uint32_t wv[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
-    int lo = 0, hi = 0;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int4 xa = ldg_nc_v4(xg + k);
-      const uint32_t ml = wv[k] & 0x0F0F0F0Fu, mh = wv[k] & 0xF0F0F0F0u;
-      lo = dp2a_lo(xa.x, ml, lo);
-      lo = dp2a_hi(xa.y, ml, lo);
-      hi = dp2a_lo(xa.z, mh, hi);
-      hi = dp2a_hi(xa.w, mh, hi);
-    }
-    return lo + (hi >> 4);
-  }
-}
-
-template <int BITS>
+template <int BITS, bool XS>
 __global__ void __launch_bounds__(kThreads, 1)
     gemv_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_hi,
                 const __grid_constant__ CUtensorMap tm_sz, GemvParams p) {
@@ -112,9 +32,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smem;
-  uint64_t* full = reinterpret_cast<uint64_t*>(ring + kStages * G::kStageBytes);
-  uint64_t* empty = full + kStages;
-  float* red = reinterpret_cast<float*>(empty + kStages);  // [kConsumerWarps][kMaxBatchGemv][32]
+  uint64_t* full = reinterpret_cast<uint64_t*>(ring + G::kStages * G::kStageBytes);
+  uint64_t* empty = full + G::kStages;
+  uint64_t* xbar = empty + G::kStages;
+  float* red = reinterpret_cast<float*>(xbar + 2);  // [kConsumerWarps][kMaxBatchGemv][32]
+  // staged activation operand (XS): per batch row xq (xq_stride words), xs and xsum (g_stride each)
+  uint8_t* xstage = reinterpret_cast<uint8_t*>(red + kConsumerWarps * kMaxBatchGemv * 32);
+  const int64_t xrow_bytes = 4 * (p.xq_stride + 2 * p.g_stride);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r0 = (int)(((int64_t)p.n_out * blockIdx.x) / gridDim.x);
@@ -126,10 +50,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nstages = nsub * nchunks;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < G::kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kConsumerWarps);
     }
+    mbar_init(xbar, 1);
     fence_mbar_init();
   }
   __syncthreads();
@@ -141,9 +66,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tm_codes);
       tma_prefetch_desc(&tm_sz);
       if (BITS == 3) tma_prefetch_desc(&tm_hi);
+      if constexpr (XS) {
+        mbar_arrive_expect_tx(xbar, (uint32_t)(xrow_bytes * p.batch));
+        for (int b = 0; b < p.batch; ++b) {
+          uint8_t* dst = xstage + b * xrow_bytes;
+          bulk_g2s(dst, p.xq + b * p.xq_stride, (uint32_t)(4 * p.xq_stride), xbar);
+          bulk_g2s(dst + 4 * p.xq_stride, p.xs + b * p.g_stride, (uint32_t)(4 * p.g_stride), xbar);
+          bulk_g2s(dst + 4 * (p.xq_stride + p.g_stride), p.xsum + b * p.g_stride, (uint32_t)(4 * p.g_stride), xbar);
+        }
+      }
       for (int k = 0; k < nstages; ++k) {
-        const int slot = k % kStages;
-        if (k >= kStages && !mbar_wait(&empty[slot], ((k / kStages) - 1) & 1, p.status, 1)) break;
+        const int slot = k % G::kStages;
+        if (k >= G::kStages && !mbar_wait(&empty[slot], ((k / G::kStages) - 1) & 1, p.status, 1)) break;
         const int sub = k / nchunks, ch = k % nchunks;
         const int row0 = r0 + (int)(((int64_t)nrows * sub) / nsub);
         const int g0 = ch * G::kChunkGroups;
@@ -170,10 +104,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
   for (int b = 0; b < kMaxBatchGemv; ++b) zacc[b] = 0.f;
   bool ok = true;
+  if constexpr (XS) ok = mbar_wait(xbar, 0, p.status, 3);
 
   for (int k = 0; k < nstages && ok; ++k) {
-    const int slot = k % kStages;
-    if (!mbar_wait(&full[slot], (k / kStages) & 1, p.status, 2)) {
+    const int slot = k % G::kStages;
+    if (!mbar_wait(&full[slot], (k / G::kStages) & 1, p.status, 2)) {
       ok = false;
       break;
     }
@@ -193,10 +128,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int b = 0; b < kMaxBatchGemv; ++b) {
         if (b < p.batch) {
-          const int4* xg = reinterpret_cast<const int4*>(p.xq + b * p.xq_stride + (int64_t)g * 32);
-          const int4* xgh = reinterpret_cast<const int4*>(p.xq + b * p.xq_stride + p.n_in / 2 + (int64_t)g * 32);
-          const int acc = group_dot<BITS>(st, st + G::kCodeSlabs * kSlab, lane, gl, xg, xgh);
-          const float xs = p.xs[b * p.g_stride + g], xsum = p.xsum[b * p.g_stride + g];
+          const int32_t* xqb;
+          float xs, xsum;
+          if constexpr (XS) {
+            const uint8_t* row = xstage + b * xrow_bytes;
+            xqb = reinterpret_cast<const int32_t*>(row);
+            xs = reinterpret_cast<const float*>(row + 4 * p.xq_stride)[g];
+            xsum = reinterpret_cast<const float*>(row + 4 * (p.xq_stride + p.g_stride))[g];
+          } else {
+            xqb = p.xq + b * p.xq_stride;
+            xs = p.xs[b * p.g_stride + g];
+            xsum = p.xsum[b * p.g_stride + g];
+          }
+          const int4* xg = reinterpret_cast<const int4*>(xqb + (int64_t)g * 32);
+          const int4* xgh = reinterpret_cast<const int4*>(xqb + p.n_in / 2 + (int64_t)g * 32);
+          const int acc = group_dot<BITS, XS>(st, st + G::kCodeSlabs * kSlab, lane, gl, xg, xgh);
           zacc[b] = fmaf(s16, (float)acc * xs, fmaf(z16, xsum, zacc[b]));
         }
       }
@@ -223,28 +169,41 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int BITS>
-cudaError_t launch_bits(const Layer& L, const GemvParams& p, cudaStream_t st) {
+template <int BITS, bool XS>
+cudaError_t launch_bits(const Layer& L, const GemvParams& p, cudaStream_t st, int dev, int nsm) {
   using G = Geo<BITS>;
-  const size_t smem = 1024 + (size_t)kStages * G::kStageBytes + 2 * kStages * sizeof(uint64_t) +
+  const size_t xbytes = XS ? (size_t)4 * (p.xq_stride + 2 * p.g_stride) * p.batch : 0;
+  const size_t base = 1024 + (size_t)G::kStages * G::kStageBytes + (2 * G::kStages + 2) * sizeof(uint64_t) +
                       sizeof(float) * kConsumerWarps * kMaxBatchGemv * 32;
-  int dev = 0, nsm = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-  if (e != cudaSuccess) return e;
+  const size_t smem = base + xbytes;
+  const size_t smem_max = base + (XS ? kXStageMax : 0);
   static bool attr_done[64] = {false};  // the attribute is per device; set it once each
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!attr_done[dev]) {
-    e = cudaFuncSetAttribute(gemv_kernel<BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<BITS, XS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem_max);
     if (e != cudaSuccess) return e;
     attr_done[dev] = true;
   }
   // one CTA per SM, but never fewer than ~8 rows per CTA
   int grid = nsm;
   if (p.n_out < 8 * grid) grid = (p.n_out + 7) / 8;
-  gemv_kernel<BITS><<<grid, kThreads, smem, st>>>(L.tm_codes, L.tm_hi, L.tm_sz, p);
+  gemv_kernel<BITS, XS><<<grid, kThreads, smem, st>>>(L.tm_codes, L.tm_hi, L.tm_sz, p);
   return cudaGetLastError();
+}
+
+template <int BITS>
+cudaError_t launch_bits(const Layer& L, const GemvParams& p, cudaStream_t st) {
+  int dev = 0, nsm = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  const int64_t xbytes = 4 * (p.xq_stride + 2 * p.g_stride) * (int64_t)p.batch;
+  // bulk copies need 16-byte multiples: xq rows are n_in/2 or n_in words, xs/xsum rows n_in/64 floats
+  const bool aligned = (p.g_stride % 4 == 0) && (p.xq_stride % 4 == 0);
+  if (xbytes <= kXStageMax && aligned) return launch_bits<BITS, true>(L, p, st, dev, nsm);
+  return launch_bits<BITS, false>(L, p, st, dev, nsm);
 }
 
 }  // namespace

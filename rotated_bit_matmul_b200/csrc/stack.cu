@@ -1,12 +1,14 @@
 // Llama-shaped decoder stack whose seven linears per block are rotated low-bit
 // layers: RMSNorm, residual adds, SiLU * up, and the key/value-group broadcast of a
 // one-key attention (its output is the value), around harp linear forwards.
+#include <algorithm>
 #include <cstring>
 #include <new>
 #include <string>
 #include <vector>
 
 #include "common.cuh"
+#include "decode.h"
 
 using namespace harp;
 
@@ -15,6 +17,11 @@ struct harp_stack_s {
   float eps;
   std::vector<harp_layer> layers;
   int device;
+  // fused batch-1 decode step (null when this stack's shapes are outside its domain)
+  bool fused = false;
+  dec::Lin* d_lin = nullptr;
+  dec::Params fp{};
+  std::string fused_why;
 };
 
 namespace {
@@ -104,6 +111,191 @@ StackWs stack_ws(const harp_stack_s* S, int batch, void* base) {
 
 harp_status sfail(harp_status s, const std::string& msg) { return set_error(s, "%s", msg.c_str()); }
 
+// ---------------------------------------------------------------- fused decode step
+struct FusedWs {
+  size_t bytes;
+};
+
+// carves the fused kernel's buffers out of `base` (or just sizes them when base is null)
+size_t fused_ws(const harp_stack_s* S, dec::Params* p, void* base) {
+  const size_t L = S->n_layers, dq = (size_t)S->n_heads * S->head_dim, dkv = (size_t)S->n_kv_heads * S->head_dim;
+  const size_t H = S->hidden, F = S->ffn;
+  const int bits = S->layers[0]->L.bits;
+  const size_t words = bits == 3 ? F : F / 2, ngf = F / 64;
+  size_t off = 0;
+  auto take = [&](size_t bytes) -> char* {
+    char* r = base ? static_cast<char*>(base) + off : nullptr;
+    off = a256(off + bytes);
+    return r;
+  };
+  char* zq = take(4 * L * dq);
+  char* zk = take(4 * L * dkv);
+  char* qo = take(4 * L * dq);
+  char* ko = take(4 * L * dkv);
+  char* zv = take(4 * dkv);
+  char* zo = take(4 * H);
+  char* zg = take(4 * F);
+  char* zu = take(4 * F);
+  char* zd = take(4 * H);
+  char* xq = take(4 * words);
+  char* xs = take(4 * ngf);
+  char* xsum = take(4 * ngf);
+  char* cnt = take(4 * 5 * L);
+  if (p && base) {
+    p->zq = reinterpret_cast<float*>(zq);
+    p->zk = reinterpret_cast<float*>(zk);
+    p->qout = reinterpret_cast<float*>(qo);
+    p->kout = reinterpret_cast<float*>(ko);
+    p->zv = reinterpret_cast<float*>(zv);
+    p->zo = reinterpret_cast<float*>(zo);
+    p->zg = reinterpret_cast<float*>(zg);
+    p->zu = reinterpret_cast<float*>(zu);
+    p->zd = reinterpret_cast<float*>(zd);
+    p->xq_down = reinterpret_cast<int32_t*>(xq);
+    p->xs_down = reinterpret_cast<float*>(xs);
+    p->xsum_down = reinterpret_cast<float*>(xsum);
+    p->counters = reinterpret_cast<unsigned*>(cnt);
+  }
+  return off;
+}
+
+int ilog2(int v) {
+  int m = 0;
+  while ((1 << m) < v) ++m;
+  return m;
+}
+
+// proportional split of G clusters over linears of n_k rows (each >= 1), largest remainder
+void assign(int G, const int* rows, int k, int* asg, int* idx, int* cnt) {
+  long long tot = 0;
+  for (int i = 0; i < k; ++i) tot += rows[i];
+  int given = 0;
+  double rem[3];
+  for (int i = 0; i < k; ++i) {
+    const double share = (double)G * rows[i] / (double)tot;
+    cnt[i] = (int)share < 1 ? 1 : (int)share;
+    rem[i] = share - cnt[i];
+    given += cnt[i];
+  }
+  while (given < G) {
+    int best = 0;
+    for (int i = 1; i < k; ++i)
+      if (rem[i] > rem[best]) best = i;
+    cnt[best] += 1;
+    rem[best] -= 1.0;
+    ++given;
+  }
+  while (given > G) {
+    int best = -1;
+    for (int i = 0; i < k; ++i)
+      if (cnt[i] > 1 && (best < 0 || rem[i] < rem[best])) best = i;
+    cnt[best] -= 1;
+    rem[best] += 1.0;
+    --given;
+  }
+  int c = 0;
+  for (int i = 0; i < k; ++i)
+    for (int j = 0; j < cnt[i]; ++j, ++c) {
+      asg[c] = i;
+      idx[c] = j;
+    }
+}
+
+// Decides whether the fused kernel covers this stack and prepares its constant state.
+void setup_fused(harp_stack_s* S) {
+  S->fused = false;
+  auto no = [&](const std::string& why) { S->fused_why = why; };
+  const int H = S->hidden, F = S->ffn, dq = S->n_heads * S->head_dim, dkv = S->n_kv_heads * S->head_dim;
+  const int bits = S->layers[0]->L.bits;
+  if (H < 4096 || H > kMaxW || (H & (H - 1))) return no("hidden must be a power of two in [4096, 8192]");
+  if (dq != H) return no("n_heads * head_dim must equal hidden");
+  if (dkv < 256 || dkv > H || (dkv & (dkv - 1))) return no("n_kv_heads * head_dim must be a power of two in [256, hidden]");
+  const int wb = S->layers[4]->L.w_out;
+  if (wb < 64 || wb > 512) return no("gate/up output blocks must be 64..512 wide");
+  for (int l = 0; l < S->n_layers; ++l) {
+    const Layer* L[7];
+    for (int i = 0; i < 7; ++i) L[i] = &S->layers[7 * l + i]->L;
+    for (int i = 0; i < 7; ++i)
+      if (L[i]->bits != bits) return no("all linears must share one bit width");
+    for (int i = 0; i < 3; ++i)
+      if (L[i]->w_in != H) return no("q/k/v input butterflies must be hidden-wide");
+    if (L[0]->w_out != dq || L[1]->w_out != dkv || L[2]->w_out != dkv) return no("q/k/v output butterflies must be single blocks");
+    if (L[3]->w_in != H || L[3]->w_out != H) return no("o butterflies must be hidden-wide");
+    if (L[4]->w_in != H || L[5]->w_in != H) return no("gate/up input butterflies must be hidden-wide");
+    if (L[4]->w_out != wb || L[5]->w_out != wb || L[6]->w_in != wb) return no("gate/up output and down input blocks must match");
+    if (L[6]->w_out != H) return no("down output butterfly must be hidden-wide");
+  }
+  dec::Params& p = S->fp;
+  p = dec::Params{};
+  p.L = S->n_layers;
+  p.hidden = H;
+  p.ffn = F;
+  p.n_heads = S->n_heads;
+  p.n_kv = S->n_kv_heads;
+  p.head_dim = S->head_dim;
+  p.rep = S->n_heads / S->n_kv_heads;
+  p.bits = bits;
+  p.eps = S->eps;
+  p.E = H / dec::kC;
+  p.m_hidden = ilog2(H);
+  // shared-memory budget: tables of the largest chain, operand of the widest input
+  auto tb = [](int w) { return 8 * ilog2(w) * (w / dec::kC / 2); };
+  int tab = 2 * tb(H);
+  tab = std::max(tab, tb(dkv) + tb(H));
+  const int wbm = ilog2(wb);
+  p.tab_bytes = std::max(tab, 3 * 4 * wb * wbm);
+  auto xqb = [&](int n) { return 4 * ((bits == 3 ? n : n / 2) + 2 * (n / 64)); };
+  p.xq_bytes = (std::max(xqb(H), xqb(F)) + 15) & ~15;  // keeps the mbarriers after it 8-byte aligned
+  int optin = 0;
+  cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, S->device);
+  const int stage = dec::stage_bytes_for(bits);
+  p.ring_stages = 1;
+  const size_t fixed = dec::smem_for(p) - (size_t)stage;
+  p.ring_stages = (int)((optin - (long long)fixed) / stage);
+  if (p.ring_stages < 2) return no("not enough shared memory for the weight ring");
+  if (p.ring_stages > 16) p.ring_stages = 16;
+  int G = 0;
+  cudaError_t e = dec::max_clusters(p, &G);
+  if (e != cudaSuccess || G < 1) return no(std::string("cluster occupancy query failed: ") + cudaGetErrorString(e));
+  if (G > dec::kMaxClusters) G = dec::kMaxClusters;
+  const int nblocks = F / wb;
+  // P7: block CTAs come first, the last two clusters apply F_U_q / F_U_k
+  while (G > 3 && nblocks > (G - 2) * dec::kC) --G;
+  if (G < 3 || nblocks > (G - 2) * dec::kC) return no("too few co-resident clusters");
+  p.G = G;
+  const int rq[3] = {dq, dkv, dkv}, rg[2] = {F, F};
+  assign(G, rq, 3, p.asg_qkv, p.idx_qkv, p.cnt_qkv);
+  assign(G, rg, 2, p.asg_gu, p.idx_gu, p.cnt_gu);
+  // device copy of the per-linear descriptors
+  std::vector<dec::Lin> h(7 * (size_t)S->n_layers);
+  for (size_t i = 0; i < h.size(); ++i) {
+    const Layer& L = S->layers[i]->L;
+    dec::Lin& d = h[i];
+    memset(&d, 0, sizeof d);
+    d.tm_codes = L.tm_codes;
+    d.tm_hi = L.tm_hi;
+    d.tm_sz = L.tm_sz;
+    d.csV = L.csV;
+    d.csU = L.csU;
+    d.sV = L.sV;
+    d.sU = L.sU;
+    d.n_in = (int)L.n_in;
+    d.n_out = (int)L.n_out;
+    d.w_in = L.w_in;
+    d.w_out = L.w_out;
+    d.m_in = L.m_in;
+    d.m_out = L.m_out;
+  }
+  if (cudaMalloc(&S->d_lin, sizeof(dec::Lin) * h.size()) != cudaSuccess) return no("cudaMalloc failed");
+  if (cudaMemcpy(S->d_lin, h.data(), sizeof(dec::Lin) * h.size(), cudaMemcpyHostToDevice) != cudaSuccess) {
+    cudaFree(S->d_lin);
+    S->d_lin = nullptr;
+    return no("cudaMemcpy failed");
+  }
+  p.lin = S->d_lin;
+  S->fused = true;
+}
+
 }  // namespace
 
 extern "C" {
@@ -138,19 +330,33 @@ harp_status harp_stack_create(harp_stack* out, int n_layers, int hidden, int ffn
   S->eps = eps;
   S->layers.assign(layers, layers + 7 * (size_t)n_layers);
   cudaGetDevice(&S->device);
+  setup_fused(S);
+  cudaGetLastError();  // a refused fused set-up is not an error of this call
   *out = S;
   return HARP_OK;
 }
 
 harp_status harp_stack_destroy(harp_stack stack) {
+  if (!stack) return HARP_OK;
+  if (stack->d_lin) {
+    int prev = 0;
+    cudaGetDevice(&prev);
+    cudaSetDevice(stack->device);
+    cudaDeviceSynchronize();
+    cudaFree(stack->d_lin);
+    cudaSetDevice(prev);
+  }
   delete stack;
   return HARP_OK;
 }
+
+int harp_stack_uses_fused_step(harp_stack stack, int batch) { return stack && stack->fused && batch == 1; }
 
 harp_status harp_stack_workspace_size(harp_stack stack, int batch, size_t* bytes) {
   if (!stack || !bytes) return sfail(HARP_ERR_INVALID_ARG, "stack_workspace_size: null pointer");
   if (batch < 1 || batch > 256) return sfail(HARP_ERR_INVALID_ARG, "stack_workspace_size: batch out of range");
   *bytes = stack_ws(stack, batch, nullptr).bytes;
+  if (stack->fused && batch == 1) *bytes = std::max(*bytes, fused_ws(stack, nullptr, nullptr));
   return HARP_OK;
 }
 
@@ -159,11 +365,29 @@ harp_status harp_stack_step(harp_stack S, int batch, const void* x, harp_dtype x
   if (!S || !x || !out) return sfail(HARP_ERR_INVALID_ARG, "stack_step: null pointer");
   if (batch < 1 || batch > 256) return sfail(HARP_ERR_INVALID_ARG, "stack_step: batch out of range");
   if (xt < 0 || xt > 2 || ot < 0 || ot > 2) return sfail(HARP_ERR_INVALID_ARG, "stack_step: unknown dtype");
-  const size_t need = stack_ws(S, batch, nullptr).bytes;
+  size_t need = stack_ws(S, batch, nullptr).bytes;
+  const bool fused = S->fused && batch == 1;
+  if (fused) need = std::max(need, fused_ws(S, nullptr, nullptr));
   if (!workspace || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return sfail(HARP_ERR_WORKSPACE, "stack_step: workspace of " + std::to_string(need) +
                                          " bytes (256-byte aligned) needed");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (fused) {
+    int* status = nullptr;
+    harp_status hs = device_status_for_kernels(&status);
+    if (hs != HARP_OK) return hs;
+    dec::Params p = S->fp;
+    fused_ws(S, &p, workspace);
+    p.x_in = x;
+    p.xt = xt;
+    p.y_out = out;
+    p.yt = ot;
+    p.status = status;
+    cudaError_t e = cudaMemsetAsync(p.counters, 0, sizeof(unsigned) * 5 * (size_t)S->n_layers, st);
+    if (e == cudaSuccess) e = dec::launch(p, st);
+    if (e != cudaSuccess) return sfail(HARP_ERR_CUDA, std::string("fused decode step: ") + cudaGetErrorString(e));
+    return HARP_OK;
+  }
   StackWs w = stack_ws(S, batch, workspace);
   const int64_t B = batch, H = S->hidden, F = S->ffn;
   const int64_t dq = (int64_t)S->n_heads * S->head_dim, dkv = (int64_t)S->n_kv_heads * S->head_dim;

@@ -238,3 +238,37 @@ def test_stack_matches_oracle(dims, n_layers, block, batch):
     for l in layers:
         l.close()
     assert err < GATE, err
+
+
+# ------------------------------------------------------------------ fused decode step
+@pytest.mark.parametrize("n_layers,bits", [(2, 2), (1, 3), (1, 4)])
+def test_fused_decode_step_matches_oracle(n_layers, bits):
+    """The single-kernel batch-1 decode step on 7B-wide blocks against the oracle."""
+    import rotated_bit_matmul_b200 as rb
+    dims = (4096, 11008, 32, 32, 128)
+    hidden, ffn = dims[0], dims[1]
+    shapes = [(4096, hidden), (4096, hidden), (4096, hidden), (hidden, 4096), (ffn, hidden), (ffn, hidden),
+              (hidden, ffn)]
+    cases = []
+    for l in range(n_layers):
+        for i, (n_out, n_in) in enumerate(shapes):
+            w_in = 256 if n_in == ffn else n_in
+            w_out = 256 if n_out == ffn else n_out
+            cases.append(oracle_layer(n_out, n_in, w_in, w_out, bits, 6, l, i))
+    layers = [device_layer(c) for c in cases]
+    S = rb.HarpStack(layers, *dims)
+    assert S.uses_fused_step(1)
+    x = synth.activations(1, hidden, 6, step=3)
+    got = S.step(_dev(x, torch.bfloat16)).cpu().numpy()
+    torch.cuda.synchronize()
+    rb.harp_device_status()
+    want = oracle.stack_step([c["lay"] for c in cases], *dims, x.astype(np.float64))
+    err = rel_l2(got, want)
+    # the same step through the per-linear path (batch 2 with a duplicated row)
+    got2 = S.step(_dev(np.concatenate([x, x]), torch.bfloat16)).cpu().numpy()
+    S.close()
+    for l in layers:
+        l.close()
+    assert err < GATE, err
+    assert rel_l2(got2[0], want[0]) < GATE
+    assert rel_l2(got, got2[:1]) < 1e-4
