@@ -213,12 +213,8 @@ __global__ void __launch_bounds__(kBflyThreads) bfly_kernel(BflyParams p, int C)
           sum += __shfl_xor_sync(0xffffffffu, sum, o);
         }
         int ex = 0;
-        if (amax > 0.f && !bad) {
-          int E2;
-          frexpf(amax, &E2);
-          ex = min(max(15 - E2, -126), 126);
-        }
-        const float sc = ldexpf(1.f, ex);
+        if (amax > 0.f && !bad) ex = group_exponent(amax);
+        const float sc = pow2f(ex);
         const int q0 = max(-32767, min(32767, __float2int_rn(v0 * sc)));
         const int q1 = max(-32767, min(32767, __float2int_rn(v1 * sc)));
         const int64_t gg = gidx(gl * 64) >> 6;  // global group index
@@ -231,7 +227,7 @@ __global__ void __launch_bounds__(kBflyThreads) bfly_kernel(BflyParams p, int C)
           hi[xq_pos_hi(2 * lane + 1)] = (int16_t)q1;
         }
         if (lane == 0) {
-          p.xs[row * p.g_stride + gg] = bad ? __int_as_float(0x7fc00000) : ldexpf(1.f, -ex);
+          p.xs[row * p.g_stride + gg] = bad ? __int_as_float(0x7fc00000) : pow2f(-ex);
           p.xsum[row * p.g_stride + gg] = bad ? __int_as_float(0x7fc00000) : sum;
         }
       }

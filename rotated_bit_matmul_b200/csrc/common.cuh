@@ -144,6 +144,17 @@ __device__ __forceinline__ int xq_pos_hi(int j) {  // 1-bit plane of 3-bit codes
   return (c * 16 + 2 * m + (q >> 1)) * 2 + (q & 1);
 }
 
+// Scale exponent of a group of the GEMV operand: the e in [-126, 126] with
+// max|v| * 2^e in [2^14, 2^15), i.e. 15 - E for max|v| = f 2^E, f in [0.5, 1), read straight
+// from the exponent field (a denormal maximum takes the largest scale, 126).
+__device__ __forceinline__ int group_exponent(float amax) {
+  const int field = (int)((__float_as_uint(amax) >> 23) & 0xffu);
+  const int E = field == 0 ? -126 : field - 126;
+  return min(max(15 - E, -126), 126);
+}
+// 2^e for e in [-126, 127], exact
+__device__ __forceinline__ float pow2f(int e) { return __int_as_float((e + 127) << 23); }
+
 // ------------------------------------------------------------------ programmatic dependent launch
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" :::); }

@@ -11,7 +11,7 @@ namespace dec {
 constexpr int kC = 8;                // CTAs per cluster
 constexpr int kCW = 16;              // consumer warps per CTA
 constexpr int kNT = 32 * kCW;        // consumer threads
-constexpr int kThreads = kNT + 32;   // + one producer warp
+constexpr int kThreads = kNT + 64;   // + a weight-ring producer warp and a table producer warp
 constexpr int kMaxClusters = 64;
 
 // One linear as the fused kernel sees it (device array, 64-byte aligned for the maps).
@@ -35,8 +35,10 @@ struct Params {
   int xt;
   void* y_out;
   int yt;
-  float *zq, *zk, *qout, *kout;  // [L][dq], [L][dkv]
-  float *zv, *zo, *zg, *zu, *zd;
+  // split-K partial sums of every GEMV, [nk][n_out] (q and k kept per block: [L][nk][n])
+  float *zpq, *zpk, *zpv, *zpo, *zpg, *zpu, *zpd;
+  int nk_h, nk_f;      // column chunks of a hidden-wide / ffn-wide input
+  float *qout, *kout;  // F_U of q and k per block, [L][dq], [L][dkv]
   int32_t* xq_down;
   float* xs_down;
   float* xsum_down;
@@ -50,6 +52,7 @@ struct Params {
 cudaError_t launch(const Params& p, cudaStream_t st);
 size_t smem_for(const Params& p);
 int stage_bytes_for(int bits);
+int chunk_cols_for(int bits);
 cudaError_t max_clusters(const Params& p, int* out);
 
 }  // namespace dec

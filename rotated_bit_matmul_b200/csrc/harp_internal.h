@@ -6,7 +6,7 @@
 #include <stddef.h>
 #include <stdint.h>
 
-#include "../../include/harp.h"
+#include "harp.h"
 
 namespace harp {
 

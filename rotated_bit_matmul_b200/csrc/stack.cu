@@ -121,6 +121,8 @@ size_t fused_ws(const harp_stack_s* S, dec::Params* p, void* base) {
   const size_t L = S->n_layers, dq = (size_t)S->n_heads * S->head_dim, dkv = (size_t)S->n_kv_heads * S->head_dim;
   const size_t H = S->hidden, F = S->ffn;
   const int bits = S->layers[0]->L.bits;
+  const size_t kc = (size_t)dec::chunk_cols_for(bits);
+  const size_t nkh = (H + kc - 1) / kc, nkf = (F + kc - 1) / kc;
   const size_t words = bits == 3 ? F : F / 2, ngf = F / 64;
   size_t off = 0;
   auto take = [&](size_t bytes) -> char* {
@@ -128,29 +130,33 @@ size_t fused_ws(const harp_stack_s* S, dec::Params* p, void* base) {
     off = a256(off + bytes);
     return r;
   };
-  char* zq = take(4 * L * dq);
-  char* zk = take(4 * L * dkv);
+  char* zpq = take(4 * L * nkh * dq);
+  char* zpk = take(4 * L * nkh * dkv);
   char* qo = take(4 * L * dq);
   char* ko = take(4 * L * dkv);
-  char* zv = take(4 * dkv);
-  char* zo = take(4 * H);
-  char* zg = take(4 * F);
-  char* zu = take(4 * F);
-  char* zd = take(4 * H);
+  char* zpv = take(4 * nkh * dkv);
+  char* zpo = take(4 * nkh * H);
+  char* zpg = take(4 * nkh * F);
+  char* zpu = take(4 * nkh * F);
+  char* zpd = take(4 * nkf * H);
   char* xq = take(4 * words);
   char* xs = take(4 * ngf);
   char* xsum = take(4 * ngf);
   char* cnt = take(4 * 5 * L);
+  if (p) {
+    p->nk_h = (int)nkh;
+    p->nk_f = (int)nkf;
+  }
   if (p && base) {
-    p->zq = reinterpret_cast<float*>(zq);
-    p->zk = reinterpret_cast<float*>(zk);
+    p->zpq = reinterpret_cast<float*>(zpq);
+    p->zpk = reinterpret_cast<float*>(zpk);
     p->qout = reinterpret_cast<float*>(qo);
     p->kout = reinterpret_cast<float*>(ko);
-    p->zv = reinterpret_cast<float*>(zv);
-    p->zo = reinterpret_cast<float*>(zo);
-    p->zg = reinterpret_cast<float*>(zg);
-    p->zu = reinterpret_cast<float*>(zu);
-    p->zd = reinterpret_cast<float*>(zd);
+    p->zpv = reinterpret_cast<float*>(zpv);
+    p->zpo = reinterpret_cast<float*>(zpo);
+    p->zpg = reinterpret_cast<float*>(zpg);
+    p->zpu = reinterpret_cast<float*>(zpu);
+    p->zpd = reinterpret_cast<float*>(zpd);
     p->xq_down = reinterpret_cast<int32_t*>(xq);
     p->xs_down = reinterpret_cast<float*>(xs);
     p->xsum_down = reinterpret_cast<float*>(xsum);
@@ -248,12 +254,10 @@ void setup_fused(harp_stack_s* S) {
   p.xq_bytes = (std::max(xqb(H), xqb(F)) + 15) & ~15;  // keeps the mbarriers after it 8-byte aligned
   int optin = 0;
   cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, S->device);
-  const int stage = dec::stage_bytes_for(bits);
-  p.ring_stages = 1;
-  const size_t fixed = dec::smem_for(p) - (size_t)stage;
-  p.ring_stages = (int)((optin - (long long)fixed) / stage);
+  // as many ring stages as fit (each also carries its reduction scratch and barriers)
+  p.ring_stages = 16;
+  while (p.ring_stages >= 2 && dec::smem_for(p) > (size_t)optin) --p.ring_stages;
   if (p.ring_stages < 2) return no("not enough shared memory for the weight ring");
-  if (p.ring_stages > 16) p.ring_stages = 16;
   int G = 0;
   cudaError_t e = dec::max_clusters(p, &G);
   if (e != cudaSuccess || G < 1) return no(std::string("cluster occupancy query failed: ") + cudaGetErrorString(e));
