@@ -62,6 +62,26 @@ def algorithmic_bytes_per_step(n_layers, batch=BATCH, bits=BITS):
     return tot * n_layers
 
 
+# DRAM bytes (read + write) of one fused decode launch per transformer block, from the
+# ncu capture summarised in profiles/decode_kernel_llama2-7b_2bit_batch1.md (4-block
+# case, 270.77 MB per launch, scaled by blocks), and a hash of the kernel's sources at
+# capture time: the figure is reported only while those sources are unchanged.
+TRAFFIC_PER_BLOCK = {"bytes": 270_773_760 // 4, "sources_sha256_16": "960232bf36427e64"}
+KERNEL_SOURCES = ("decode.cu", "decode.h", "common.cuh", "gemv_core.cuh")
+
+
+def traffic_per_step(n_layers):
+    import hashlib
+    csrc = os.path.join(ROOT, "rotated_bit_matmul_b200", "csrc")
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    if h.hexdigest()[:16] != TRAFFIC_PER_BLOCK["sources_sha256_16"]:
+        return None
+    return TRAFFIC_PER_BLOCK["bytes"] * n_layers
+
+
 def measured_peak():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -119,13 +139,9 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ CPU oracle sample
-def cpu_oracle_sample(sample_layers=1):
-    """Times the fp64 oracle on `sample_layers` blocks of the 7B stack (one token) and
-    scales to the 32-block step. Returns (tokens_per_s, seconds_per_block, threads)."""
+def _oracle_block(sample_layers):
     import oracle
     from rotated_bit_matmul_b200 import synth
-    threads = len(os.sched_getaffinity(0))
-    oracle.set_threads(threads)
     lays = []
     for l in range(sample_layers):
         for i, s in enumerate(shapes()):
@@ -133,12 +149,30 @@ def cpu_oracle_sample(sample_layers=1):
             thV, sV = synth.butterfly_params(s.n_in, s.w_in, WORKLOAD, l, i, "V")
             thU, sU = synth.butterfly_params(s.n_out, s.w_out, WORKLOAD, l, i, "U")
             lays.append(oracle.prepare_layer(W, BITS, s.w_in, s.w_out, thV, sV, thU, sU)[0])
-    x = synth.activations(BATCH, HIDDEN, WORKLOAD, 0).astype(np.float64)
-    t0 = time.perf_counter()
-    oracle.stack_step(lays, HIDDEN, FFN, NH, NKV, HD, x)
-    dt = time.perf_counter() - t0
-    per_block = dt / sample_layers
-    return 1.0 / (per_block * N_LAYERS), per_block, threads
+    return lays
+
+
+def cpu_oracle_sample(sample_layers=1, min_seconds=10.0, steps=None, warmup=0):
+    """Times the fp64 oracle on `sample_layers` blocks of the 7B stack for one token per
+    pass and scales to the 32-block step. Without `steps` it repeats passes until
+    `min_seconds` of CPU work have been timed; with `steps` it runs `warmup` untimed and
+    `steps` timed passes. Returns (tokens_per_s, seconds_per_block, threads, passes)."""
+    import oracle
+    from rotated_bit_matmul_b200 import synth
+    threads = len(os.sched_getaffinity(0))
+    oracle.set_threads(threads)
+    lays = _oracle_block(sample_layers)
+    for w in range(warmup):
+        oracle.stack_step(lays, HIDDEN, FFN, NH, NKV, HD, synth.activations(BATCH, HIDDEN, WORKLOAD, step=w).astype(np.float64))
+    passes, dt = 0, 0.0
+    while (steps is not None and passes < steps) or (steps is None and (passes == 0 or dt < min_seconds)):
+        x = synth.activations(BATCH, HIDDEN, WORKLOAD, step=warmup + passes).astype(np.float64)
+        t0 = time.perf_counter()
+        oracle.stack_step(lays, HIDDEN, FFN, NH, NKV, HD, x)
+        dt += time.perf_counter() - t0
+        passes += 1
+    per_block = dt / (passes * sample_layers)
+    return 1.0 / (per_block * N_LAYERS), per_block, threads, passes
 
 
 # ------------------------------------------------------------------ GPU path
@@ -171,11 +205,10 @@ def launches_per_step(n_layers, fused):
     return 1 + n_layers * (2 + 7 * 3 + 2 + 1) + 1
 
 
-def run_ours(args, rank, world):
+def run_ours(args, rk):
     import torch
-    import torch.distributed as dist
-    from rotated_bit_matmul_b200 import synth
-    device = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    from rotated_bit_matmul_b200 import replicas, synth
+    device = torch.device("cuda", rk.local_rank)
     torch.cuda.set_device(device)
     stack = build_stack(args.layers, device)
     K, Wm = args.steps, args.warmup
@@ -202,12 +235,8 @@ def run_ours(args, rank, world):
             g.replay()
     stream.synchronize()
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
+    replicas.barrier(rk)
     torch.cuda.synchronize()
     with ClockSampler(device.index) as clk:
         with torch.cuda.stream(stream):
@@ -218,21 +247,17 @@ def run_ours(args, rank, world):
             e1.record(stream)
         e1.synchronize()
     torch.cuda.synchronize()
-    barrier()
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    replicas.barrier(rk)
+    ms = replicas.max_over_ranks(rk, e0.elapsed_time(e1), device)
     ms_step = ms / K
-    value = world * BATCH * K / (ms / 1e3)
+    value = replicas.whole_job_rate(rk, BATCH * K, ms)
 
     # end to end through the public API with host buffers: pinned H2D of the step's
     # input, the stack step, D2H of its output, every step
     xh = torch.stack([torch.from_numpy(synth.activations(BATCH, HIDDEN, WORKLOAD, step=s)).to(torch.bfloat16)
                       for s in range(K)]).pin_memory()
     yh = torch.empty((K, BATCH, HIDDEN), dtype=torch.float32).pin_memory()
-    barrier()
+    replicas.barrier(rk)
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):
         e0.record(stream)
@@ -242,13 +267,9 @@ def run_ours(args, rank, world):
             yh[s].copy_(y, non_blocking=True)
         e1.record(stream)
     e1.synchronize()
-    barrier()
-    ms_e2e = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms_e2e], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = float(t.item())
-    e2e = {"value": world * BATCH * K / (ms_e2e / 1e3), "unit": "tokens/s",
+    replicas.barrier(rk)
+    ms_e2e = replicas.max_over_ranks(rk, e0.elapsed_time(e1), device)
+    e2e = {"value": replicas.whole_job_rate(rk, BATCH * K, ms_e2e), "unit": "tokens/s",
            "h2d_bytes_per_step": int(xh[0].numel() * xh.element_size()),
            "d2h_bytes_per_step": int(yh[0].numel() * yh.element_size())}
 
@@ -257,7 +278,7 @@ def run_ours(args, rank, world):
     achieved = nbytes / (ms_step * 1e-3) / 1e9
     fused = stack.uses_fused_step(BATCH)
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": None,
+                "frac": round(achieved / peak, 4), "traffic": traffic_per_step(args.layers) if fused else None,
                 "kernel": "decode_kernel (one launch per step)" if fused else "whole decode step (graph of kernels)",
                 "peak_kind": peak_kind, "algorithmic_bytes_per_step": nbytes}
     del g
@@ -267,13 +288,11 @@ def run_ours(args, rank, world):
 
 def main():
     args = parse()
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        backend = "gloo" if args.impl == "reference" else "nccl"
-        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    from rotated_bit_matmul_b200 import replicas
+    rk = replicas.from_env()
+    # the reference arm is the CPU oracle: its ranks meet over gloo
+    replicas.init(rk, "gloo" if args.impl == "reference" else "nccl")
+    world = rk.world
 
     config = {"workload": CONFIG_NAME, "layers": args.layers, "hidden": HIDDEN, "ffn": FFN, "bits": BITS,
               "group": GROUP, "batch": BATCH, "global_batch": BATCH * world, "parallelism": f"replicas{world}",
@@ -284,36 +303,33 @@ def main():
             "config": config}
 
     if args.impl == "reference":
-        if rank == 0:
-            tps, per_block, threads = cpu_oracle_sample(args.cpu_sample_layers)
+        # rank 0 alone times the oracle; the other ranks leave without work
+        if rk.rank == 0:
+            tps, per_block, threads, passes = cpu_oracle_sample(args.cpu_sample_layers, steps=args.steps,
+                                                                warmup=args.warmup)
             ms = per_block * N_LAYERS * 1e3
             line = dict(base, impl="reference", value=tps, unit="tokens/s", ms_per_step=ms, dtype="f64",
                         cpu_baseline={"value": tps, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                                      "sample": f"{args.cpu_sample_layers} of {N_LAYERS} blocks of one decode "
-                                                f"token per step, scaled to {N_LAYERS} blocks"},
+                                      "sample": f"each step: {args.cpu_sample_layers} of {N_LAYERS} blocks of one "
+                                                f"decode token, scaled to {N_LAYERS} blocks"},
                         e2e={"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0})
-            line["steps"], line["warmup"] = 1, 0
             print(json.dumps(line), flush=True)
-        if world > 1:
-            import torch.distributed as dist
-            dist.destroy_process_group()
+        replicas.finish(rk)
         return
 
-    r = run_ours(args, rank, world)
+    r = run_ours(args, rk)
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tps, per_block, threads = cpu_oracle_sample(args.cpu_sample_layers)
+    if rk.rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tps, per_block, threads, passes = cpu_oracle_sample(args.cpu_sample_layers)
         cpu = {"value": tps, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-               "sample": f"{args.cpu_sample_layers} of {N_LAYERS} blocks of one decode token, scaled to {N_LAYERS}"}
-    if rank == 0:
+               "sample": f"{passes} passes of {args.cpu_sample_layers} of {N_LAYERS} blocks of one decode token "
+                         f"(about 10 s of CPU work), scaled to {N_LAYERS} blocks"}
+    if rk.rank == 0:
         line = dict(base, value=r["value"], unit="tokens/s", ms_per_step=r["ms_step"],
                     dtype="u2 codes x i16 activations -> i32 dot, f32 elsewhere", roofline=r["roofline"],
                     cpu_baseline=cpu, e2e=r["e2e"], gpu_launches=r["launches"], clocks=r["clocks"])
         print(json.dumps(line), flush=True)
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-        dist.destroy_process_group()
+    replicas.finish(rk)
 
 
 if __name__ == "__main__":
