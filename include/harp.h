@@ -118,16 +118,23 @@ harp_status harp_create_layer(harp_layer* out, int64_t n_in, int64_t n_out, int 
 /* Frees the layer's own device memory (synchronises the device first). Null is a no-op. */
 harp_status harp_destroy_layer(harp_layer layer);
 
-/* Bytes of device workspace harp_linear_fwd needs for `batch` rows (batch 1..256). */
+/* Bytes of device workspace harp_linear_fwd needs for `batch` rows (batch 1..65535). */
 harp_status harp_linear_workspace_size(harp_layer layer, int batch, size_t* bytes);
 
 /* y = F_U(dequant(codes) F_V(x)) for `batch` rows.
  *   x : device [batch][n_in] of dtype xt;  y : device [batch][n_out] of dtype yt.
  *   workspace : device scratch of at least harp_linear_workspace_size bytes, 256-byte
  *               aligned; its contents are overwritten. y must not alias x or workspace.
- * Batches 1..8 run the CUDA-core dequant-GEMV (fp32 activations, exact integer dot
- * products per group); 16..256 run the tcgen05 tensor-core path (bf16 operands, fp32
- * accumulation) where built, else the GEMV path.
+ * Batches 1..15 run the CUDA-core dequant-GEMV: the transformed activations as int16 with
+ * a power-of-two scale per 64-column group, and exact integer dot products per group,
+ * in passes of 8 rows.
+ * Batches 16..65535 run the tcgen05 tensor-core path:
+ *   - the transformed activations as fp16 with a power-of-two scale per row, and the
+ *     weights as fp16 s*q;
+ *   - fp32 accumulation in tensor memory;
+ *   - the zero term m * (group sum) as one more K block;
+ *   - in chunks of 256 rows.
+ * Both paths take the same workspace call; its size depends on the path.
  */
 harp_status harp_linear_fwd(harp_layer layer, int batch, const void* x, harp_dtype xt, void* y,
                             harp_dtype yt, void* workspace, size_t ws_bytes, void* stream);

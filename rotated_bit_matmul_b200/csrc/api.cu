@@ -10,6 +10,7 @@
 #include <string>
 
 #include "harp_internal.h"
+#include "mma.h"
 
 using namespace harp;
 
@@ -86,16 +87,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // 128-byte swizzle, zero fill out of bounds.
 harp_status make_tmap(CUtensorMap* tm, const void* base, CUtensorMapDataType dt, int esize, uint64_t inner,
                       uint64_t rows, uint64_t row_bytes) {
-  auto fn = encode_fn();
-  if (!fn) return fail(HARP_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
-  cuuint64_t dims[2] = {inner, rows};
-  cuuint64_t strides[1] = {row_bytes};
-  cuuint32_t box[2] = {(cuuint32_t)(128 / esize), 32};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(tm, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return fail(HARP_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  if (!encode_fn()) return fail(HARP_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  if (!harp::encode_map_2d(tm, dt, base, inner, rows, row_bytes, (uint32_t)(128 / esize), 32,
+                           CU_TENSOR_MAP_SWIZZLE_128B))
+    return fail(HARP_ERR_CUDA, "cuTensorMapEncodeTiled failed");
   return HARP_OK;
 }
 
@@ -145,30 +140,45 @@ size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 namespace harp {
 
+bool encode_map_2d(CUtensorMap* tm, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t rows,
+                   uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(tm, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int xq_words_per_row(int64_t n_in, int bits) { return (int)(bits == 3 ? n_in : n_in / 2); }
 
 LinearWs linear_ws_layout(const Layer& L, int batch, void* base) {
   LinearWs w{};
   const int64_t ng = L.n_in / kGroup;
-  w.xq_stride = xq_words_per_row(L.n_in, L.bits);
-  w.g_stride = ng;
   size_t off = 0;
-  const size_t o_xq = off;
-  off = align256(off + sizeof(int32_t) * (size_t)batch * (size_t)w.xq_stride);
-  const size_t o_xs = off;
-  off = align256(off + sizeof(float) * (size_t)batch * (size_t)ng);
-  const size_t o_sum = off;
-  off = align256(off + sizeof(float) * (size_t)batch * (size_t)ng);
-  const size_t o_z = off;
-  off = align256(off + sizeof(float) * (size_t)batch * (size_t)L.n_out);
-  w.bytes = off;
-  if (base) {
-    char* b = static_cast<char*>(base);
-    w.xq = reinterpret_cast<int32_t*>(b + o_xq);
-    w.xs = reinterpret_cast<float*>(b + o_xs);
-    w.xsum = reinterpret_cast<float*>(b + o_sum);
-    w.z = reinterpret_cast<float*>(b + o_z);
+  char* b = static_cast<char*>(base);
+  auto carve = [&](size_t bytes) -> void* {
+    const size_t o = off;
+    off = align256(off + bytes);
+    return b ? b + o : nullptr;
+  };
+  if (batch >= kMinBatchMma) {
+    w.x16_ld = mma::x16_ld(L.n_in);
+    w.xf = static_cast<float*>(carve(sizeof(float) * (size_t)batch * (size_t)L.n_in));
+    w.x16 = carve(2 * (size_t)batch * (size_t)w.x16_ld);
+    w.rowscale = static_cast<float*>(carve(sizeof(float) * (size_t)batch));
+    w.zpart = static_cast<float*>(carve(sizeof(float) * (size_t)L.msplits * (size_t)batch * (size_t)L.n_out));
+  } else {
+    w.xq_stride = xq_words_per_row(L.n_in, L.bits);
+    w.g_stride = ng;
+    w.xq = static_cast<int32_t*>(carve(sizeof(int32_t) * (size_t)batch * (size_t)w.xq_stride));
+    w.xs = static_cast<float*>(carve(sizeof(float) * (size_t)batch * (size_t)ng));
+    w.xsum = static_cast<float*>(carve(sizeof(float) * (size_t)batch * (size_t)ng));
+    w.z = static_cast<float*>(carve(sizeof(float) * (size_t)batch * (size_t)L.n_out));
   }
+  w.bytes = off;
   return w;
 }
 
@@ -178,7 +188,13 @@ harp_status linear_forward(const Layer& L, int batch, const void* x, int xt, int
   int* status = nullptr;
   harp_status s = device_status_ptr(&status);
   if (s != HARP_OK) return s;
+  return linear_forward_status(L, batch, x, xt, x_stride, y, yt, y_stride, ws, st, status);
+}
+
+harp_status linear_forward_status(const Layer& L, int batch, const void* x, int xt, int64_t x_stride, void* y,
+                                  int yt, int64_t y_stride, void* ws, cudaStream_t st, int* status) {
   LinearWs w = linear_ws_layout(L, batch, ws);
+  const bool tc = batch >= kMinBatchMma;
 
   BflyParams pv{};
   pv.n = L.n_in;
@@ -190,31 +206,49 @@ harp_status linear_forward(const Layer& L, int batch, const void* x, int xt, int
   pv.x = x;
   pv.xt = xt;
   pv.x_stride = x_stride;
-  pv.y = nullptr;
-  pv.xq = w.xq;
-  pv.xs = w.xs;
-  pv.xsum = w.xsum;
-  pv.bits = L.bits;
-  pv.xq_stride = w.xq_stride;
-  pv.g_stride = w.g_stride;
   pv.status = status;
-  HARP_CUDA(launch_butterfly(pv, batch, st), "input butterfly launch");
+  if (tc) {
+    // x~ in fp32, then the fp16 operand with its group sums
+    pv.y = w.xf;
+    pv.yt = DT_F32;
+    pv.y_stride = L.n_in;
+    HARP_CUDA(launch_butterfly(pv, batch, st), "input butterfly launch");
+    HARP_CUDA(mma::launch_x16_prep(w.xf, L.n_in, L.bits, batch, static_cast<__half*>(w.x16), w.rowscale, status, st),
+              "operand prep launch");
+    mma::Call c{};
+    c.x16 = static_cast<const __half*>(w.x16);
+    c.ld = w.x16_ld;
+    c.rowscale = w.rowscale;
+    c.zpart = w.zpart;
+    c.batch = batch;
+    c.status = status;
+    HARP_CUDA(mma::launch(L, c, st), "dequant-MMA launch");
+  } else {
+    pv.y = nullptr;
+    pv.xq = w.xq;
+    pv.xs = w.xs;
+    pv.xsum = w.xsum;
+    pv.bits = L.bits;
+    pv.xq_stride = w.xq_stride;
+    pv.g_stride = w.g_stride;
+    HARP_CUDA(launch_butterfly(pv, batch, st), "input butterfly launch");
 
-  for (int b0 = 0; b0 < batch; b0 += kMaxBatchGemv) {
-    GemvParams gp{};
-    gp.n_out = (int)L.n_out;
-    gp.n_in = (int)L.n_in;
-    gp.bits = L.bits;
-    gp.batch = batch - b0 < kMaxBatchGemv ? batch - b0 : kMaxBatchGemv;
-    gp.xq = w.xq + (int64_t)b0 * w.xq_stride;
-    gp.xq_stride = w.xq_stride;
-    gp.xs = w.xs + (int64_t)b0 * w.g_stride;
-    gp.xsum = w.xsum + (int64_t)b0 * w.g_stride;
-    gp.g_stride = w.g_stride;
-    gp.z = w.z + (int64_t)b0 * L.n_out;
-    gp.z_stride = L.n_out;
-    gp.status = status;
-    HARP_CUDA(launch_gemv(L, gp, st), "dequant-GEMV launch");
+    for (int b0 = 0; b0 < batch; b0 += kMaxBatchGemv) {
+      GemvParams gp{};
+      gp.n_out = (int)L.n_out;
+      gp.n_in = (int)L.n_in;
+      gp.bits = L.bits;
+      gp.batch = batch - b0 < kMaxBatchGemv ? batch - b0 : kMaxBatchGemv;
+      gp.xq = w.xq + (int64_t)b0 * w.xq_stride;
+      gp.xq_stride = w.xq_stride;
+      gp.xs = w.xs + (int64_t)b0 * w.g_stride;
+      gp.xsum = w.xsum + (int64_t)b0 * w.g_stride;
+      gp.g_stride = w.g_stride;
+      gp.z = w.z + (int64_t)b0 * L.n_out;
+      gp.z_stride = L.n_out;
+      gp.status = status;
+      HARP_CUDA(launch_gemv(L, gp, st), "dequant-GEMV launch");
+    }
   }
 
   BflyParams pu{};
@@ -224,9 +258,11 @@ harp_status linear_forward(const Layer& L, int batch, const void* x, int xt, int
   pu.inverse = 0;
   pu.cs = L.csU;
   pu.sign = L.sU;
-  pu.x = w.z;
+  pu.x = tc ? w.zpart : w.z;
   pu.xt = DT_F32;
   pu.x_stride = L.n_out;
+  pu.nsum = tc ? L.msplits : 1;
+  pu.sum_stride = (int64_t)batch * L.n_out;
   pu.y = y;
   pu.yt = yt;
   pu.y_stride = y_stride;
@@ -358,6 +394,22 @@ harp_status harp_create_layer(harp_layer* out, int64_t n_in, int64_t n_out, int 
     s = make_tmap(&L.tm_sz, scale_zero, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, (uint64_t)n_in / 64, (uint64_t)n_out,
                   (uint64_t)n_in / 16);
   if (s != HARP_OK) return cleanup(s);
+  // tensor-core path: one group of codes, a split's scale_zero / 1-bit plane per 128 rows
+  const mma::Split sp = mma::choose_split(n_out, n_in, bits);
+  L.msplits = sp.splits;
+  L.mgs = sp.gs;
+  const uint64_t rb = (uint64_t)n_in * pb / 8;  // bytes per row of the (first) code plane
+  bool mok = encode_map_2d(&L.tm_mcodes, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, rb, (uint64_t)n_out, rb,
+                           (uint32_t)(64 * pb / 8), mma::kBM, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+             encode_map_2d(&L.tm_msz, CU_TENSOR_MAP_DATA_TYPE_UINT32, scale_zero, (uint64_t)n_in / 64,
+                           (uint64_t)n_out, (uint64_t)n_in / 16, (uint32_t)sp.gs, mma::kBM,
+                           CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (mok && bits == 3)
+    mok = encode_map_2d(&L.tm_mhi, CU_TENSOR_MAP_DATA_TYPE_UINT8, static_cast<const char*>(codes) + n_out * n_in / 4,
+                        (uint64_t)n_in / 8, (uint64_t)n_out, (uint64_t)n_in / 8, (uint32_t)(8 * sp.gs), mma::kBM,
+                        CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (mok && bits != 3) L.tm_mhi = L.tm_msz;
+  if (!mok) return cleanup(fail(HARP_ERR_CUDA, "create_layer: tensor maps of the tensor-core path"));
   *out = h;
   return HARP_OK;
 }
@@ -379,7 +431,8 @@ harp_status harp_destroy_layer(harp_layer layer) {
 
 harp_status harp_linear_workspace_size(harp_layer layer, int batch, size_t* bytes) {
   if (!layer || !bytes) return fail(HARP_ERR_INVALID_ARG, "linear_workspace_size: null pointer");
-  if (batch < 1 || batch > 256) return fail(HARP_ERR_INVALID_ARG, "linear_workspace_size: batch=%d not in [1,256]", batch);
+  if (batch < 1 || batch > kMaxBatch)
+    return fail(HARP_ERR_INVALID_ARG, "linear_workspace_size: batch=%d not in [1,%d]", batch, kMaxBatch);
   *bytes = linear_ws_layout(layer->L, batch, nullptr).bytes;
   return HARP_OK;
 }
@@ -387,7 +440,8 @@ harp_status harp_linear_workspace_size(harp_layer layer, int batch, size_t* byte
 harp_status harp_linear_fwd(harp_layer layer, int batch, const void* x, harp_dtype xt, void* y, harp_dtype yt,
                             void* workspace, size_t ws_bytes, void* stream) {
   if (!layer) return fail(HARP_ERR_INVALID_ARG, "linear_fwd: null layer");
-  if (batch < 1 || batch > 256) return fail(HARP_ERR_INVALID_ARG, "linear_fwd: batch=%d not in [1,256]", batch);
+  if (batch < 1 || batch > kMaxBatch)
+    return fail(HARP_ERR_INVALID_ARG, "linear_fwd: batch=%d not in [1,%d]", batch, kMaxBatch);
   if (!valid_dtype(xt) || !valid_dtype(yt)) return fail(HARP_ERR_INVALID_ARG, "linear_fwd: unknown dtype");
   if (!x || !y) return fail(HARP_ERR_INVALID_ARG, "linear_fwd: null pointer");
   if (!aligned16(x) || !aligned16(y)) return fail(HARP_ERR_INVALID_ARG, "linear_fwd: pointers must be 16-byte aligned");

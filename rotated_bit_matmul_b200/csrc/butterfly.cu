@@ -167,7 +167,9 @@ __global__ void __launch_bounds__(kBflyThreads) bfly_kernel(BflyParams p, int C)
     // ---- load chunk r (layout A), signs first
     for (int i = tid; i < E; i += nthr) {
       const int64_t gi = base + (int64_t)r * E + i;
-      xa[i] = load_act(p.x, row * p.x_stride + gi, p.xt) * (float)p.sign[gi];
+      float v = load_act(p.x, row * p.x_stride + gi, p.xt);
+      for (int k = 1; k < p.nsum; ++k) v += load_act(p.x, k * p.sum_stride + row * p.x_stride + gi, p.xt);
+      xa[i] = v * (float)p.sign[gi];
     }
     __syncthreads();
     if (use_bulk) mbar_wait(bar, 0, p.status, 10);

@@ -64,6 +64,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try_wait, but a thread that finds the phase incomplete may sleep up to
+// `hint_ns` (it wakes when the phase completes) instead of returning at once.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
@@ -84,6 +96,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
   }
   report(status, 5 /* HARP_ERR_TIMEOUT */, where);
   return false;
+}
+
+// Bounded wait for one thread of a warp (the others meet it at __syncwarp): sleeps in
+// slices of up to 0.2 ms, gives up after `limit_ns` like mbar_wait.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, int* status, int where,
+                                                uint64_t limit_ns = 1000000000ull) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait_sleep(bar, parity, 200000u))
+    if (globaltimer_ns() - t0 > limit_ns) {
+      report(status, 5 /* HARP_ERR_TIMEOUT */, where);
+      return false;
+    }
+  return true;
 }
 
 // ------------------------------------------------------------------ TMA (no multicast)

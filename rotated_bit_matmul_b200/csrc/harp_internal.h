@@ -15,6 +15,8 @@ enum { DT_F32 = 0, DT_BF16 = 1, DT_F16 = 2 };
 constexpr int kGroup = 64;       // quantization group (columns)
 constexpr int kMaxBatchGemv = 8; // batch rows the CUDA-core GEMV handles per launch
 constexpr int kMaxW = 8192;      // widest butterfly block held by one CTA
+constexpr int kMinBatchMma = 16; // token batches from here on take the tensor-core path
+constexpr int kMaxBatch = 65535; // token rows per harp_linear_fwd call (a grid dimension)
 
 // Butterfly launch description. One CTA transforms one w-wide block of one row.
 struct BflyParams {
@@ -35,6 +37,8 @@ struct BflyParams {
   float* xsum;         // per group fp32 sum of the transformed values
   int bits;
   int64_t xq_stride, g_stride;
+  int nsum;            // forward input: sum of nsum fp32 partial arrays sum_stride apart (<= 1: one)
+  int64_t sum_stride;
   int* status;
 };
 
@@ -63,16 +67,26 @@ struct Layer {
   CUtensorMap tm_codes;  // 2-bit/4-bit codes, or the 2-bit plane of 3-bit codes
   CUtensorMap tm_hi;     // 1-bit plane of 3-bit codes (unused otherwise)
   CUtensorMap tm_sz;     // scale_zero as uint32 [n_out][n_in/64]
+  // tensor-core path (token batches >= kMinBatchMma): 128-row boxes of one group's codes,
+  // of a split's scale_zero and of a split's 1-bit plane (3-bit codes)
+  CUtensorMap tm_mcodes, tm_msz, tm_mhi;
+  int msplits, mgs;      // input-group splits per 128-row tile and groups per split
   int device;
 };
 
-// Workspace carve-up for a linear forward with `batch` rows.
+// Workspace carve-up for a linear forward with `batch` rows. Below kMinBatchMma rows
+// (GEMV): xq, xs, xsum, z. From kMinBatchMma rows (tensor cores): xf, x16, rowscale, zpart.
 struct LinearWs {
   int32_t* xq;
   float* xs;
   float* xsum;
   float* z;
   int64_t xq_stride, g_stride;
+  float* xf;          // [batch][n_in] transformed input
+  void* x16;          // [batch][x16_ld] fp16 operand + group sums
+  float* rowscale;    // [batch]
+  float* zpart;       // [msplits][batch][n_out]
+  int64_t x16_ld;
   size_t bytes;
 };
 
@@ -85,6 +99,11 @@ cudaError_t launch_quantize(int64_t n_out, int64_t n_in, int bits, const float* 
                             void* scale_zero, cudaStream_t st);
 cudaError_t launch_cs_table(const float* theta, int64_t count, float2* cs, cudaStream_t st);
 
+// 2-D tiled tensor map over a row-major [rows][inner] array; false if the driver
+// entry point is missing or rejects the arguments.
+bool encode_map_2d(CUtensorMap* tm, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t rows,
+                   uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw);
+
 // Records a printf-style message as the thread's last error and returns `st`.
 harp_status set_error(harp_status st, const char* fmt, ...);
 // Per-device status word the kernels report failures into (allocated on first use,
@@ -93,6 +112,9 @@ harp_status device_status_for_kernels(int** out);
 // Enqueues y = F_U(dequant(codes) F_V(x)) for validated arguments.
 harp_status linear_forward(const Layer& L, int batch, const void* x, int xt, int64_t x_stride, void* y, int yt,
                            int64_t y_stride, void* ws, cudaStream_t st);
+// The same with an explicit status word (null: device-side failures are not recorded).
+harp_status linear_forward_status(const Layer& L, int batch, const void* x, int xt, int64_t x_stride, void* y,
+                                  int yt, int64_t y_stride, void* ws, cudaStream_t st, int* status);
 
 }  // namespace harp
 

@@ -1,0 +1,478 @@
+// Dequant -> tcgen05 tensor-core contraction of the rotated low-bit linear for token
+// batches of 16 and more (HARP: "rotated, quantized linear y = U^T deq(Q(U W V^T)) V x").
+//
+// One CTA owns a tile of 128 weight rows, up to 256 tokens and one split of the input
+// groups:
+// * warp 0 streams, with TMA and no multicast, into a shared-memory ring:
+//   * the packed codes of one 64-column group per stage;
+//   * the matching 64 columns of the fp16 token operand.
+// * warps 2..9 expand the codes to fp16 s*q in the 128-byte-swizzled K-major layout
+//   that the tensor core reads.
+// * one lane of warp 1 issues tcgen05.mma kind::f16 (M = 128, N = tokens, K = 16) into a
+//   tensor-memory accumulator. It commits each stage back to the ring.
+// * warps 2..9 then read the accumulator with tcgen05.ld and store the split's fp32
+//   partial sums. The output butterfly adds the splits in a fixed order.
+//
+// Zero term. deq(q) = s q + m for each (row, group), so
+//   z = sum_j (s q_j) x_j + sum_g m_g X_g,
+// where X_g is a group sum of the operand. The second sum runs on the tensor core as one
+// extra K block per split, the first stage of the ring:
+// * the weight side holds the split's m values (fp16, exactly as stored);
+// * the token side holds the group sums, which the operand prep appends after the n_in
+//   columns.
+// Hoisting m leaves one packed FMA per pair of weights: fma(1024 + q, s, -1024 s) rounds
+// q s once.
+#include "common.cuh"
+#include "mma.h"
+
+#include <algorithm>
+
+namespace harp {
+namespace mma {
+namespace {
+
+// ------------------------------------------------------------------ tcgen05 / proxy helpers
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of 128 bytes,
+// 8-row groups 1024 bytes apart (start address 16-byte units, version 1, layout 2).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3fffu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// Instruction descriptor of kind::f16: fp32 accumulator, A = B = fp16, both K-major,
+// N >> 3 in bits 17..22, M >> 4 in bits 24..28.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N) {
+  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_f16(uint32_t tmem_d, uint64_t ad, uint64_t bd, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(ad), "l"(bd), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+// Arrives on `bar` once every tcgen05.mma this thread issued before has completed.
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {  // whole warp
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)), "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {  // whole warp
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// 8 consecutive accumulator columns of this thread's lane (whole warp).
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
+  uint32_t r0, r1, r2, r3, r4, r5, r6, r7;
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3), "=r"(r4), "=r"(r5), "=r"(r6), "=r"(r7)
+               : "r"(taddr)
+               : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+  v[0] = __uint_as_float(r0); v[1] = __uint_as_float(r1); v[2] = __uint_as_float(r2); v[3] = __uint_as_float(r3);
+  v[4] = __uint_as_float(r4); v[5] = __uint_as_float(r5); v[6] = __uint_as_float(r6); v[7] = __uint_as_float(r7);
+}
+
+__device__ __forceinline__ void st_shared_v4(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(smem_u32(p)), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+
+__device__ __forceinline__ uint32_t h2u(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+__device__ __forceinline__ __half2 u2h(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
+
+// fp16 (q_lo, q_hi) * s, rounded once, from t = (1024 + q_lo, 1024 + q_hi) as fp16 bits.
+// The fast form needs -1024 s finite in fp16 (|s| < 64); larger scales take two steps.
+__device__ __forceinline__ uint32_t scale_pair(uint32_t t, __half2 s2, __half2 c2, bool fast) {
+  if (fast) return h2u(__hfma2(u2h(t), s2, c2));
+  return h2u(__hmul2(__hsub2(u2h(t), __half2half2(__float2half(1024.f))), s2));
+}
+
+constexpr int kMaxStages = 8;
+
+struct Params {
+  CUtensorMap tm_codes;  // codes (2-bit plane of 3-bit codes) as bytes, box {cb, 128}
+  CUtensorMap tm_sz;     // scale_zero as uint32, box {gs, 128}
+  CUtensorMap tm_hi;     // 1-bit plane of 3-bit codes as bytes, box {8 gs, 128}
+  CUtensorMap tm_x;      // fp16 operand [batch][ld], box {64, N}, 128-byte swizzle
+  int n_out, n_in, G, gs, N, stages, batch, ncols;
+  const float* rowscale;
+  float* zpart;
+  int* status;
+};
+
+template <int BITS>
+struct Geo {
+  static constexpr int kCodeBytes = BITS == 4 ? 32 : 16;  // bytes of one row's group in the code tile
+  static constexpr int kA = kBM * 128;                     // dequantized weight tile (16 KB)
+};
+
+// Dynamic shared memory: [ring: stages x (A 16 KB | X N*128 | codes 128*cb)] [sz 128*gs*4]
+// [hi 128*gs*8] [barriers]; the ring starts 1024-byte aligned (swizzle atoms).
+template <int BITS>
+__host__ __device__ inline int stage_bytes(int N) {
+  return Geo<BITS>::kA + N * 128 + kBM * Geo<BITS>::kCodeBytes;
+}
+template <int BITS>
+__host__ __device__ inline int fixed_bytes(int gs) {
+  return kBM * gs * 4 + (BITS == 3 ? kBM * gs * 8 : 0) + 256 + 1024;  // + barriers + alignment slack
+}
+
+template <int BITS>
+__global__ void __launch_bounds__(kThreads, 1) mma_kernel(const __grid_constant__ Params p) {
+  using Gm = Geo<BITS>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int SB = stage_bytes<BITS>(p.N);
+  const int ST = p.stages;
+  uint8_t* ring = base;
+  uint32_t* sz_s = reinterpret_cast<uint32_t*>(ring + (size_t)ST * SB);
+  uint8_t* hi_s = reinterpret_cast<uint8_t*>(sz_s + kBM * p.gs);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(hi_s + (BITS == 3 ? kBM * p.gs * 8 : 0));
+  uint64_t* full = bars;                    // [ST] TMA landed (codes + operand)
+  uint64_t* afull = bars + kMaxStages;      // [ST] dequantized tile written
+  uint64_t* empty = bars + 2 * kMaxStages;  // [ST] MMAs of the stage completed
+  uint64_t* pre = bars + 3 * kMaxStages;    // scale/zero (and hi plane) of the split landed
+  uint64_t* accb = pre + 1;                 // accumulator complete
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(accb + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tile = blockIdx.x, split = blockIdx.y, b0 = blockIdx.z * kMaxN;
+  const int g0 = split * p.gs;
+  const int ngs = min(p.gs, p.G - g0);  // groups of this split
+  const int nst = 1 + ngs;              // the zero block, then one stage per group
+  const int row0 = tile * kBM;
+
+  if (tid == 0) {
+    for (int i = 0; i < ST; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&afull[i], kDqWarps);
+      mbar_init(&empty[i], 1);
+    }
+    mbar_init(pre, 1);
+    mbar_init(accb, 1);
+    fence_mbar_init();
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) tmem_alloc(tslot, (uint32_t)p.ncols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+
+  if (warp == 0) {
+    // ---------------- producer (lane 0 issues; the warp stays converged around it)
+    if (lane == 0) {
+      tma_prefetch_desc(&p.tm_codes);
+      tma_prefetch_desc(&p.tm_x);
+      mbar_arrive_expect_tx(pre, (uint32_t)(kBM * p.gs * 4 + (BITS == 3 ? kBM * p.gs * 8 : 0)));
+      tma_load_2d(sz_s, &p.tm_sz, pre, g0, row0);
+      if (BITS == 3) tma_load_2d(hi_s, &p.tm_hi, pre, g0 * 8, row0);
+      int k = 0;
+      for (; k < nst; ++k) {
+        const int slot = k % ST;
+        if (k >= ST && !mbar_wait_sleep(&empty[slot], ((k / ST) - 1) & 1, p.status, 80)) break;
+        uint8_t* st = ring + (size_t)slot * SB;
+        uint8_t* X = st + Gm::kA;
+        uint8_t* C = X + p.N * 128;
+        if (k == 0) {
+          mbar_arrive_expect_tx(&full[slot], (uint32_t)(p.N * 128));
+          tma_load_2d(X, &p.tm_x, &full[slot], p.n_in + g0, b0);
+        } else {
+          const int g = g0 + k - 1;
+          mbar_arrive_expect_tx(&full[slot], (uint32_t)(p.N * 128 + kBM * Gm::kCodeBytes));
+          tma_load_2d(C, &p.tm_codes, &full[slot], g * Gm::kCodeBytes, row0);
+          tma_load_2d(X, &p.tm_x, &full[slot], g * 64, b0);
+        }
+      }
+      // copies still in flight land before the CTA may leave
+      mbar_wait(pre, 0, p.status, 81);
+      for (int q = max(0, k - ST); q < k; ++q) mbar_wait(&full[q % ST], (q / ST) & 1, p.status, 82);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_f16(kBM, p.N);
+      for (int k = 0; k < nst; ++k) {
+        const int slot = k % ST, ph = (k / ST) & 1;
+        if (!mbar_wait_sleep(&full[slot], ph, p.status, 83) || !mbar_wait_sleep(&afull[slot], ph, p.status, 84)) break;
+        tc_fence_after();
+        const uint32_t a = smem_u32(ring + (size_t)slot * SB);
+        const uint32_t x = a + Gm::kA;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_f16(tmem, sw128_desc(a + 32 * kk), sw128_desc(x + 32 * kk), idesc, (k | kk) != 0);
+        mma_commit(&empty[slot]);
+      }
+      mma_commit(accb);  // also when stopped early: arrives once the issued MMAs are done
+      mbar_wait(accb, 0, p.status, 85);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- dequant, then epilogue (256 threads: row m, half h of each group)
+    const int t = tid - 64, m = t & (kBM - 1), h = t >> 7;
+    const int sw = m & 7;
+    // lane 0 of each warp waits and the warp meets it at __syncwarp, which orders the
+    // landed tile before the other lanes' reads (a few pollers, not 256, on each barrier)
+    auto warp_wait = [&](uint64_t* bar, uint32_t ph, int where) -> bool {
+      int w = 1;
+      if (lane == 0) w = mbar_wait_sleep(bar, ph, p.status, where);
+      return __shfl_sync(0xffffffffu, w, 0) != 0;
+    };
+    bool ok = warp_wait(pre, 0, 86);
+    for (int k = 0; ok && k < nst; ++k) {
+      const int slot = k % ST, ph = (k / ST) & 1;
+      if (!warp_wait(&full[slot], ph, 87)) {
+        ok = false;
+        break;
+      }
+      uint8_t* st = ring + (size_t)slot * SB;
+      uint8_t* arow = st + (m >> 3) * 1024 + sw * 128;
+      if (k == 0) {
+        // zero block: column j < ngs holds m of group g0 + j, the rest 0
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int j0 = 32 * h + 8 * c + 2 * e;
+            const uint32_t lo = j0 < ngs ? (sz_s[m * p.gs + j0] >> 16) : 0u;
+            const uint32_t hi = j0 + 1 < ngs ? (sz_s[m * p.gs + j0 + 1] >> 16) : 0u;
+            o[e] = lo | (hi << 16);
+          }
+          st_shared_v4(arow + (((4 * h + c) ^ sw) << 4), o[0], o[1], o[2], o[3]);
+        }
+      } else {
+        const int gl = k - 1;
+        const uint32_t szw = sz_s[m * p.gs + gl];
+        const __half s = __ushort_as_half((unsigned short)(szw & 0xffffu));
+        const __half2 s2 = __half2half2(s);
+        const bool fast = fabsf(__half2float(s)) < 32.f;
+        const __half2 c2 = __half2half2(fast ? __hmul(s, __float2half(-1024.f)) : __float2half(0.f));
+        const uint8_t* C = st + Gm::kA + p.N * 128;
+        if (BITS == 4) {
+          const uint4 cw = *reinterpret_cast<const uint4*>(C + m * 32 + 16 * h);
+          const uint32_t wv[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            uint32_t o[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              o[i] = scale_pair(((wv[u] >> (4 * i)) & 0x000F000Fu) | 0x64006400u, s2, c2, fast);
+            st_shared_v4(arow + (((4 * h + u) ^ sw) << 4), o[0], o[1], o[2], o[3]);
+          }
+        } else {
+          const uint2 cw = *reinterpret_cast<const uint2*>(C + m * 16 + 8 * h);
+          uint32_t hw = 0;
+          if (BITS == 3) hw = reinterpret_cast<const uint32_t*>(hi_s + (m * p.gs + gl) * 8)[h];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const uint32_t w = u ? cw.y : cw.x;
+            // hi bits of codes 16u+i and 16u+8+i moved to bits i and 16+i, then up by 2
+            const uint32_t y2 = BITS == 3 ? (__byte_perm(hw, 0u, u ? 0x4342u : 0x4140u) << 2) : 0u;
+            uint32_t o[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              uint32_t tq = ((w >> (2 * i)) & 0x00030003u) | 0x64006400u;
+              if (BITS == 3) tq |= (y2 >> i) & 0x00040004u;
+              o[i] = scale_pair(tq, s2, c2, fast);
+            }
+            st_shared_v4(arow + (((4 * h + 2 * u) ^ sw) << 4), o[0], o[1], o[2], o[3]);
+            st_shared_v4(arow + (((4 * h + 2 * u + 1) ^ sw) << 4), o[4], o[5], o[6], o[7]);
+          }
+        }
+      }
+      fence_proxy_async_smem();  // generic-proxy stores -> visible to the tensor core
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&afull[slot]);
+    }
+    // ---------------- epilogue: accumulator lanes 32 (warp % 4) .. +31, half of the columns
+    if (ok && warp_wait(accb, 0, 88)) {
+      tc_fence_after();
+      const int q = warp & 3, ch = (warp - 2) >> 2;
+      const int r = row0 + 32 * q + lane;
+      const int half = p.N >> 1;
+      float* zp = p.zpart + (int64_t)split * p.batch * p.n_out;
+      for (int c0 = ch * half; c0 < (ch + 1) * half; c0 += 8) {
+        float v[8];
+        tmem_ld8(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int b = b0 + c0 + j;
+          if (b < p.batch && r < p.n_out) zp[(int64_t)b * p.n_out + r] = v[j] * p.rowscale[b];
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, (uint32_t)p.ncols);
+  }
+}
+
+// ------------------------------------------------------------------ fp16 operand prep
+// One CTA per token row: max |v| -> scale 2^e with max |v| 2^e in [256, 512) (so the group
+// sums stay below 2^15), then the scaled values in pair order and the group sums.
+template <int BITS>
+__global__ void __launch_bounds__(256) x16_prep_kernel(const float* __restrict__ xt, int n_in, int64_t ld,
+                                                       __half* __restrict__ x16, float* __restrict__ rowscale) {
+  __shared__ float red[8];
+  __shared__ int bad_s;
+  const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const float* x = xt + (int64_t)b * n_in;
+  float amax = 0.f;
+  int bad = 0;
+  for (int j = tid; j < n_in; j += 256) {
+    const float v = x[j];
+    bad |= !isfinite(v);
+    amax = fmaxf(amax, fabsf(v));
+  }
+  bad = __any_sync(0xffffffffu, bad);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if (tid == 0) bad_s = 0;
+  __syncthreads();
+  if (lane == 0) {
+    red[warp] = amax;
+    if (bad) bad_s = 1;
+  }
+  __syncthreads();
+  amax = red[0];
+  for (int i = 1; i < 8; ++i) amax = fmaxf(amax, red[i]);
+  int e = 0;
+  if (amax > 0.f) {
+    const int field = (int)((__float_as_uint(amax) >> 23) & 0xffu);
+    const int E = field == 0 ? -127 : field - 127;  // amax in [2^E, 2^(E+1))
+    e = min(max(8 - E, -126), 126);
+  }
+  const float sc = pow2f(e);
+  __half* out = x16 + (int64_t)b * ld;
+  const int G = n_in / 64;
+  for (int g = warp; g < G; g += 8) {
+    const int j0 = g * 64 + 2 * lane;
+    const float v0 = x[j0] * sc, v1 = x[j0 + 1] * sc;
+    float s = v0 + v1;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    const int jj[2] = {2 * lane, 2 * lane + 1};
+    const float vv[2] = {v0, v1};
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int j = jj[k];
+      int pos;
+      if (BITS == 4) {
+        const int c = j >> 3, i = j & 7;
+        pos = 8 * c + (i < 4 ? 2 * i : 2 * (i - 4) + 1);
+      } else {
+        const int c = j >> 4, i = j & 15;
+        pos = 16 * c + (i < 8 ? 2 * i : 2 * (i - 8) + 1);
+      }
+      out[g * 64 + pos] = __float2half_rn(vv[k]);
+    }
+    if (lane == 0) out[n_in + g] = __float2half_rn(s);
+  }
+  for (int64_t j = n_in + G + tid; j < ld; j += 256) out[j] = __float2half_rn(0.f);
+  if (tid == 0) rowscale[b] = bad_s ? __int_as_float(0x7fc00000) : pow2f(-e);
+}
+
+}  // namespace
+
+int64_t x16_ld(int64_t n_in) { return n_in + ((n_in / 64 + 63) / 64) * 64; }
+
+Split choose_split(int64_t n_out, int64_t n_in, int bits) {
+  const int tiles = (int)((n_out + kBM - 1) / kBM);
+  const int G = (int)(n_in / 64);
+  const int gmax = bits == 3 ? 32 : kMaxGs;  // the 1-bit plane box holds 8 bytes per group
+  // gs is a multiple of 8 so that every split's first group sum (fp16 column n_in + g0)
+  // starts a TMA box on a 16-byte boundary
+  int s = std::max(1, (148 + tiles - 1) / tiles);
+  int gs = (G + s - 1) / s;
+  gs = std::min(gmax, std::max(8, (gs + 7) / 8 * 8));
+  s = (G + gs - 1) / gs;
+  return Split{s, gs};
+}
+
+cudaError_t launch_x16_prep(const float* xt, int64_t n_in, int bits, int batch, __half* x16, float* rowscale,
+                            int* status, cudaStream_t st) {
+  (void)status;
+  const int64_t ld = x16_ld(n_in);
+  if (bits == 4)
+    x16_prep_kernel<4><<<batch, 256, 0, st>>>(xt, (int)n_in, ld, x16, rowscale);
+  else
+    x16_prep_kernel<2><<<batch, 256, 0, st>>>(xt, (int)n_in, ld, x16, rowscale);
+  return cudaGetLastError();
+}
+
+template <int BITS>
+static cudaError_t launch_t(const Layer& L, const Call& c, cudaStream_t st) {
+  Params p{};
+  p.tm_codes = L.tm_mcodes;
+  p.tm_sz = L.tm_msz;
+  p.tm_hi = L.tm_mhi;
+  p.n_out = (int)L.n_out;
+  p.n_in = (int)L.n_in;
+  p.G = (int)(L.n_in / 64);
+  p.gs = L.mgs;
+  p.batch = c.batch;
+  const int n16 = (std::min(c.batch, kMaxN) + 15) / 16 * 16;
+  p.N = n16;
+  p.ncols = 32;
+  while (p.ncols < p.N) p.ncols <<= 1;
+  p.rowscale = c.rowscale;
+  p.zpart = c.zpart;
+  p.status = c.status;
+
+  int dev = 0, optin = 0, sm_smem = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  cudaDeviceGetAttribute(&sm_smem, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+  const int SB = stage_bytes<BITS>(p.N), FB = fixed_bytes<BITS>(p.gs);
+  p.stages = std::min(kMaxStages, (optin - FB) / SB);
+  if (p.stages < 2) return cudaErrorInvalidConfiguration;
+  int smem = FB + p.stages * SB;
+  // tensor memory: CTAs resident on one SM must fit in its 512 columns
+  const int max_ctas = 512 / p.ncols;
+  const int per_cta_floor = sm_smem / (max_ctas + 1) + 1;  // more than this keeps <= max_ctas per SM
+  if ((sm_smem / (smem + 1024)) > max_ctas) smem = std::max(smem, per_cta_floor);
+  static bool attr_done[64] = {false};  // the attribute is per device; set it once each
+  if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+    const cudaError_t e = cudaFuncSetAttribute(mma_kernel<BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+    if (e != cudaSuccess) return e;
+    attr_done[dev] = true;
+  }
+
+  // operand tensor map: fp16 [batch][ld], box {64, N}, 128-byte swizzle
+  if (!encode_map_2d(&p.tm_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, c.x16, (uint64_t)c.ld, (uint64_t)c.batch,
+                     (uint64_t)c.ld * 2, 64, (uint32_t)p.N, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  const int tiles = (p.n_out + kBM - 1) / kBM;
+  const int splits = (p.G + p.gs - 1) / p.gs;
+  const int chunks = (c.batch + kMaxN - 1) / kMaxN;
+  mma_kernel<BITS><<<dim3(tiles, splits, chunks), kThreads, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch(const Layer& L, const Call& c, cudaStream_t st) {
+  if (L.bits == 2) return launch_t<2>(L, c, st);
+  if (L.bits == 3) return launch_t<3>(L, c, st);
+  return launch_t<4>(L, c, st);
+}
+
+}  // namespace mma
+}  // namespace harp

@@ -80,58 +80,8 @@ extern "C" harp_status harp_linear_fwd_static(harp_layer layer, int batch, const
   harp_status s = scratch_address(&base);
   if (s != HARP_OK) return s;
   int* status = nullptr;  // see the note on device status above
-  LinearWs w = linear_ws_layout(L, batch, base);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-
-  BflyParams pv{};
-  pv.n = L.n_in;
-  pv.w = L.w_in;
-  pv.m = L.m_in;
-  pv.cs = L.csV;
-  pv.sign = L.sV;
-  pv.x = x;
-  pv.xt = xt;
-  pv.x_stride = L.n_in;
-  pv.xq = w.xq;
-  pv.xs = w.xs;
-  pv.xsum = w.xsum;
-  pv.bits = L.bits;
-  pv.xq_stride = w.xq_stride;
-  pv.g_stride = w.g_stride;
-  pv.status = status;
-  if ((e = launch_butterfly(pv, batch, st)) != cudaSuccess)
-    return set_error(HARP_ERR_CUDA, "linear_fwd_static: input butterfly: %s", cudaGetErrorString(e));
-  for (int b0 = 0; b0 < batch; b0 += kMaxBatchGemv) {
-    GemvParams gp{};
-    gp.n_out = (int)L.n_out;
-    gp.n_in = (int)L.n_in;
-    gp.bits = L.bits;
-    gp.batch = batch - b0 < kMaxBatchGemv ? batch - b0 : kMaxBatchGemv;
-    gp.xq = w.xq + (int64_t)b0 * w.xq_stride;
-    gp.xq_stride = w.xq_stride;
-    gp.xs = w.xs + (int64_t)b0 * w.g_stride;
-    gp.xsum = w.xsum + (int64_t)b0 * w.g_stride;
-    gp.g_stride = w.g_stride;
-    gp.z = w.z + (int64_t)b0 * L.n_out;
-    gp.z_stride = L.n_out;
-    gp.status = status;
-    if ((e = launch_gemv(L, gp, st)) != cudaSuccess)
-      return set_error(HARP_ERR_CUDA, "linear_fwd_static: GEMV: %s", cudaGetErrorString(e));
-  }
-  BflyParams pu{};
-  pu.n = L.n_out;
-  pu.w = L.w_out;
-  pu.m = L.m_out;
-  pu.cs = L.csU;
-  pu.sign = L.sU;
-  pu.x = w.z;
-  pu.xt = DT_F32;
-  pu.x_stride = L.n_out;
-  pu.y = y;
-  pu.yt = yt;
-  pu.y_stride = L.n_out;
-  pu.status = status;
-  if ((e = launch_butterfly(pu, batch, st)) != cudaSuccess)
-    return set_error(HARP_ERR_CUDA, "linear_fwd_static: output butterfly: %s", cudaGetErrorString(e));
+  harp_status r = linear_forward_status(L, batch, x, xt, L.n_in, y, yt, L.n_out, base,
+                                        static_cast<cudaStream_t>(stream), status);
+  if (r != HARP_OK) return set_error(r, "linear_fwd_static: %s", harp_last_error());
   return HARP_OK;
 }
