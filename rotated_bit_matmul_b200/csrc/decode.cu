@@ -603,7 +603,7 @@ __device__ __forceinline__ bool run_units(const Params& p, Smem& s, const Range&
       const uint8_t* szs = st + (Gm::kCodeSlabs + Gm::kHiSlabs) * kSlab;
       for (int gl = warp; gl < gc; gl += kCW) {
         const int gg = g0 + gl;
-        const uint32_t szw = *reinterpret_cast<const uint32_t*>(swz(szs, lane, gl >> 2) + (gl & 3) * 4);
+        const uint32_t szw = sz_word(szs, lane, gl);
         const float s16 = __half2float(__ushort_as_half((unsigned short)(szw & 0xffffu)));
         const float z16 = __half2float(__ushort_as_half((unsigned short)(szw >> 16)));
         const int4* xg = reinterpret_cast<const int4*>(s.xq + (int64_t)gg * 32);
@@ -718,7 +718,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 const int cslabs = (gc + Gm::kGroupsPerSlab - 1) / Gm::kGroupsPerSlab;
                 const int hslabs = BITS == 3 ? (gc + 15) / 16 : 0;
                 uint8_t* st = s.ring + (size_t)slot * Gm::kStageBytes;
-                mbar_arrive_expect_tx(&s.full[slot], (uint32_t)((cslabs + hslabs + 1) * kSlab));
+                mbar_arrive_expect_tx(&s.full[slot], (uint32_t)((cslabs + hslabs + (gc + 31) / 32) * kSlab));
                 const int code_x0 = g0 * (BITS == 4 ? 32 : 16) / 8;
                 for (int q = 0; q < cslabs; ++q)
                   tma_load_2d(st + q * kSlab, &g.L->tm_codes, &s.full[slot], code_x0 + q * 16, tile * 32);
@@ -726,7 +726,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                   for (int q = 0; q < hslabs; ++q)
                     tma_load_2d(st + (Gm::kCodeSlabs + q) * kSlab, &g.L->tm_hi, &s.full[slot], g0 + q * 16,
                                 tile * 32);
-                tma_load_2d(st + (Gm::kCodeSlabs + Gm::kHiSlabs) * kSlab, &g.L->tm_sz, &s.full[slot], g0, tile * 32);
+                for (int q = 0; q < (gc + 31) / 32; ++q)
+                  tma_load_2d(st + (Gm::kCodeSlabs + Gm::kHiSlabs + q) * kSlab, &g.L->tm_sz, &s.full[slot],
+                              g0 + q * 32, tile * 32);
               }
             }
             ok = __shfl_sync(0xffffffffu, go, 0) != 0;

@@ -85,14 +85,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int cslabs = (gc + G::kGroupsPerSlab - 1) / G::kGroupsPerSlab;
         const int hslabs = BITS == 3 ? (gc + 15) / 16 : 0;
         uint8_t* st = ring + slot * G::kStageBytes;
-        mbar_arrive_expect_tx(&full[slot], (uint32_t)((cslabs + hslabs + 1) * kSlab));
+        mbar_arrive_expect_tx(&full[slot], (uint32_t)((cslabs + hslabs + (gc + 31) / 32) * kSlab));
         // x coordinates are in 8-byte units; every one is a multiple of 16 (128-byte slabs)
         const int code_x0 = g0 * (BITS == 4 ? 32 : 16) / 8;  // 16 or 32 code bytes per group
         for (int s = 0; s < cslabs; ++s) tma_load_2d(st + s * kSlab, &tm_codes, &full[slot], code_x0 + s * 16, row0);
         if (BITS == 3)
           for (int s = 0; s < hslabs; ++s)
             tma_load_2d(st + (G::kCodeSlabs + s) * kSlab, &tm_hi, &full[slot], g0 + s * 16, row0);
-        tma_load_2d(st + (G::kCodeSlabs + G::kHiSlabs) * kSlab, &tm_sz, &full[slot], g0, row0);
+        for (int s = 0; s < (gc + 31) / 32; ++s)
+          tma_load_2d(st + (G::kCodeSlabs + G::kHiSlabs + s) * kSlab, &tm_sz, &full[slot], g0 + s * 32, row0);
       }
     }
     return;
@@ -122,7 +123,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     for (int gl = cw; gl < gc; gl += kConsumerWarps) {
       const int g = g0 + gl;
-      const uint32_t szw = *reinterpret_cast<const uint32_t*>(swz(szs, lane, gl >> 2) + (gl & 3) * 4);
+      const uint32_t szw = sz_word(szs, lane, gl);
       const float s16 = __half2float(__ushort_as_half((unsigned short)(szw & 0xffffu)));
       const float z16 = __half2float(__ushort_as_half((unsigned short)(szw >> 16)));
 #pragma unroll

@@ -11,20 +11,30 @@ namespace gemv_core {
 constexpr int kSlab = 32 * 128;  // one TMA box: 32 rows x 128 bytes
 constexpr int kXStageMax = 64 * 1024;  // activation operand staged in shared memory up to this size
 
+// One ring stage holds one unit of work: 32 rows x one chunk of input columns. Chunks of
+// 4096 columns (2048 for 4-bit codes) make stages of 36-56 KB, which keeps the number of
+// per-unit hand-offs low; TMA rings sustain only a few million stages per second per SM.
 template <int BITS>
 struct Geo {
-  static constexpr int kChunkCols = BITS == 4 ? 1024 : 2048;  // columns per stage
+  static constexpr int kChunkCols = BITS == 4 ? 2048 : 4096;  // columns per stage
   static constexpr int kChunkGroups = kChunkCols / 64;
   static constexpr int kGroupsPerSlab = BITS == 4 ? 4 : 8;       // codes (or 2-bit plane)
   static constexpr int kCodeSlabs = kChunkGroups / kGroupsPerSlab;
   static constexpr int kHiSlabs = BITS == 3 ? kChunkGroups / 16 : 0;  // 1-bit plane
-  static constexpr int kStageBytes = (kCodeSlabs + kHiSlabs + 1) * kSlab;
-  static constexpr int kStages = BITS == 3 ? 4 : 6;
+  static constexpr int kSzSlabs = kChunkGroups / 32;                  // scale/zero, 32 groups per box
+  static constexpr int kStageBytes = (kCodeSlabs + kHiSlabs + kSzSlabs) * kSlab;
+  static constexpr int kStages = BITS == 3 ? 2 : (BITS == 2 ? 3 : 4);  // stand-alone GEMV ring (<= 160 KB)
 };
+
 
 // Address of the 16-byte chunk `c` (0..7) of `row` inside a 128B-swizzled box.
 __device__ __forceinline__ const uint8_t* swz(const uint8_t* slab, int row, int c) {
   return slab + row * 128 + ((c ^ (row & 7)) << 4);
+}
+
+// scale_zero word of group gl (of the chunk) for `row`, from the stage's scale/zero boxes
+__device__ __forceinline__ uint32_t sz_word(const uint8_t* szs, int row, int gl) {
+  return *reinterpret_cast<const uint32_t*>(swz(szs + (gl >> 5) * kSlab, row, (gl >> 2) & 7) + (gl & 3) * 4);
 }
 
 template <bool XS>
