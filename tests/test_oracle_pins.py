@@ -363,3 +363,68 @@ def test_stack_zero_up_kills_mlp(ora):
     ref, _ = _tiny_stack(ora, 1, zero=(5, 6), seed=6)
     x = np.random.default_rng(7).standard_normal((1, dims[0]))
     assert np.array_equal(ora.stack_step(layers, *dims, x), ora.stack_step(ref, *dims, x))
+
+
+def _sparse_exact_layer(ora, n_out, n_in, w_in, w_out, entries, rng):
+    """A layer whose dequantized rotated matrix is exactly known: theta = -pi/4 makes both
+    butterflies diagonal (+-1, see test_linear_integer_special_case), scale 1 and zero 0
+    make dequant(q) = q, and `entries` maps output row i -> (input column j, code value).
+    Returns the oracle layer and the effective dense matrix D_U Q D_V."""
+    q = np.zeros((n_out, n_in), np.uint8)
+    for i, (j, v) in entries.items():
+        q[i, j] = v
+    sz = np.zeros((n_out, n_in // 64, 2), np.uint16)
+    sz[..., 0] = 0x3C00  # fp16 1.0
+    mV, mU = int(math.log2(w_in)), int(math.log2(w_out))
+    thV = np.full((mV, n_in // 2), -math.pi / 4)
+    thU = np.full((mU, n_out // 2), -math.pi / 4)
+    sV, sU = _rand_sign(rng, n_in), _rand_sign(rng, n_out)
+    dV = sV * np.array([(-1.0) ** bin(i % w_in).count("1") for i in range(n_in)])
+    dU = sU * np.array([(-1.0) ** bin(i % w_out).count("1") for i in range(n_out)])
+    lay = ora.Layer(n_in, n_out, 2, w_in, w_out, thV, sV, thU, sU, ora.pack(q, 2), sz)
+    return lay, dU[:, None] * q.astype(float) * dV[None, :]
+
+
+def test_stack_glue_closed_form(ora):
+    """Every linear is a sparse exact map and the input a constant vector, so each glue
+    step reduces to a scalar closed form:
+    - RMSNorm of c*1 is c / sqrt(c^2 + eps) per element;
+    - the one-key attention copies kv head h // rep into query head h;
+    - SiLU(g) = g / (1 + e^-g) gates the up value.
+    A swapped gate/up, a sigmoid in place of SiLU, eps outside the root, a missing residual
+    or the kv groups taken modulo instead of by division each change the result."""
+    hidden, ffn, nh, nkv, hd = 128, 192, 4, 2, 32
+    dq, dkv, rep = nh * hd, nkv * hd, nh // nkv
+    eps, c = 1e-5, 0.75
+    rng = np.random.default_rng(21)
+    # q, k: anything (a one-key attention ignores them)
+    lq, _ = _sparse_exact_layer(ora, dq, hidden, hidden, dq, {0: (1, 1)}, rng)
+    lk, _ = _sparse_exact_layer(ora, dkv, hidden, hidden, dkv, {0: (2, 3)}, rng)
+    # v: kv head 1, dim 5 <- input 7 (code 2); o: output 9 <- query head 2, dim 5 (code 3);
+    # head 2 reads kv head 2 // rep = 1 (2 % rep would be kv head 0, which is all zero)
+    lv, Mv = _sparse_exact_layer(ora, dkv, hidden, hidden, dkv, {32 + 5: (7, 2)}, rng)
+    lo, Mo = _sparse_exact_layer(ora, hidden, dq, dq, hidden, {9: (2 * hd + 5, 3)}, rng)
+    # gate/up rows 10 and 70 read inputs 9 and 40; down output 20 <- ffn rows 10 and 70
+    lg, Mg = _sparse_exact_layer(ora, ffn, hidden, hidden, 64, {10: (9, 1), 70: (40, 2)}, rng)
+    lu, Mu = _sparse_exact_layer(ora, ffn, hidden, hidden, 64, {10: (40, 3), 70: (9, 1)}, rng)
+    ld, Md = _sparse_exact_layer(ora, hidden, ffn, 64, hidden, {20: (10, 1), 21: (70, 2)}, rng)
+    x = np.full((1, hidden), c)
+    got = ora.stack_step([lq, lk, lv, lo, lg, lu, ld], hidden, ffn, nh, nkv, hd, x, eps=eps)
+
+    a1 = c / math.sqrt(c * c + eps)                      # RMSNorm of a constant vector
+    v = Mv[32 + 5, 7] * a1                               # the only nonzero of v
+    # query head 2 reads kv head 2 // rep = 1: its dim 5 carries v
+    o9 = Mo[9, 2 * hd + 5] * v
+    h1 = np.full(hidden, c)
+    h1[9] += o9
+    r2 = 1.0 / math.sqrt(float(np.mean(h1 * h1)) + eps)
+    n9, n40 = h1[9] * r2, h1[40] * r2
+    g10, g70 = Mg[10, 9] * n9, Mg[70, 40] * n40
+    u10, u70 = Mu[10, 40] * n40, Mu[70, 9] * n9
+    silu = lambda t: t / (1.0 + math.exp(-t))
+    m10, m70 = silu(g10) * u10, silu(g70) * u70
+    want = h1.copy()
+    want[20] += Md[20, 10] * m10
+    want[21] += Md[21, 70] * m70
+    assert np.max(np.abs(got[0] - want)) < 1e-13
+    assert o9 != 0 and m10 != 0 and m70 != 0  # the case exercises every branch
