@@ -172,3 +172,15 @@ def test_stack_batch16():
     err = rel_l2(got, want)
     print(f"stack batch 16 rel-L2 {err:.3e}")
     assert err < GATE, err
+
+
+@pytest.mark.parametrize("bits", [3, 4])
+@pytest.mark.parametrize("batch", [1, 16])
+@pytest.mark.parametrize("name", ["k", "down"])
+def test_70b_shapes_bits_3_4(name, batch, bits):
+    """Llama-70B shapes at 3 and 4 bits, one token (dequant-GEMV) and 16 tokens
+    (tensor cores): k_proj (1024 x 8192, a narrow output) and down_proj (8192 x 28672,
+    block-diagonal 4096-wide input butterflies)."""
+    sh = next(s for s in synth.llama70b_linears() if s.name == name)
+    case = oracle_layer(sh.n_out, sh.n_in, sh.w_in, sh.w_out, bits, workload=5, linear=synth.LINEAR_NAMES.index(name))
+    _check(case, batch, 5)
