@@ -35,6 +35,9 @@ BITS, GROUP, BATCH = 2, 64, 1
 WORKLOAD = 4
 METRIC = "rotated 2-bit linear: decode tokens/s (7B-shaped, batch 1) and HBM GB/s vs roofline"
 CONFIG_NAME = "llama2-7b-shaped 32-layer rotated 2-bit linear stack, batch-1 decode"
+# with --rht every butterfly is the fixed randomized Hadamard transform (Theta = 0): the
+# baseline the HARP pages compare against (same codes budget, no learned angles)
+CONFIG_NAME_RHT = "llama2-7b-shaped 32-layer 2-bit linear stack with fixed randomized Hadamard rotations, batch-1 decode"
 
 
 def parse():
@@ -46,6 +49,8 @@ def parse():
     ap.add_argument("--layers", type=int, default=N_LAYERS)
     ap.add_argument("--cpu-sample-layers", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--rht", action="store_true",
+                    help="fixed randomized Hadamard rotations (Theta = 0) instead of the learned-angle butterflies")
     return ap.parse_args()
 
 
@@ -139,7 +144,7 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ CPU oracle sample
-def _oracle_block(sample_layers):
+def _oracle_block(sample_layers, rht=False):
     import oracle
     from rotated_bit_matmul_b200 import synth
     lays = []
@@ -148,11 +153,13 @@ def _oracle_block(sample_layers):
             W = synth.weights(s.n_out, s.n_in, WORKLOAD, l, i)
             thV, sV = synth.butterfly_params(s.n_in, s.w_in, WORKLOAD, l, i, "V")
             thU, sU = synth.butterfly_params(s.n_out, s.w_out, WORKLOAD, l, i, "U")
+            if rht:
+                thV, thU = np.zeros_like(thV), np.zeros_like(thU)
             lays.append(oracle.prepare_layer(W, BITS, s.w_in, s.w_out, thV, sV, thU, sU)[0])
     return lays
 
 
-def cpu_oracle_sample(sample_layers=1, min_seconds=10.0, steps=None, warmup=0):
+def cpu_oracle_sample(sample_layers=1, min_seconds=10.0, steps=None, warmup=0, rht=False):
     """Times the fp64 oracle on `sample_layers` blocks of the 7B stack for one token per
     pass and scales to the 32-block step. Without `steps` it repeats passes until
     `min_seconds` of CPU work have been timed; with `steps` it runs `warmup` untimed and
@@ -161,7 +168,7 @@ def cpu_oracle_sample(sample_layers=1, min_seconds=10.0, steps=None, warmup=0):
     from rotated_bit_matmul_b200 import synth
     threads = len(os.sched_getaffinity(0))
     oracle.set_threads(threads)
-    lays = _oracle_block(sample_layers)
+    lays = _oracle_block(sample_layers, rht)
     for w in range(warmup):
         oracle.stack_step(lays, HIDDEN, FFN, NH, NKV, HD, synth.activations(BATCH, HIDDEN, WORKLOAD, step=w).astype(np.float64))
     passes, dt = 0, 0.0
@@ -176,7 +183,7 @@ def cpu_oracle_sample(sample_layers=1, min_seconds=10.0, steps=None, warmup=0):
 
 
 # ------------------------------------------------------------------ GPU path
-def build_stack(n_layers, device):
+def build_stack(n_layers, device, rht=False):
     import torch
     import rotated_bit_matmul_b200 as rb
     from rotated_bit_matmul_b200 import synth
@@ -187,6 +194,8 @@ def build_stack(n_layers, device):
             thV, sV = synth.butterfly_params(s.n_in, s.w_in, WORKLOAD, l, i, "V")
             thU, sU = synth.butterfly_params(s.n_out, s.w_out, WORKLOAD, l, i, "U")
             thV, thU = torch.from_numpy(thV).to(device), torch.from_numpy(thU).to(device)
+            if rht:  # Theta = 0 on both sides: no angles reach the library
+                thV = thU = None
             sV, sU = torch.from_numpy(sV).to(device), torch.from_numpy(sU).to(device)
             Wr = rb.rotate_weights_device(W, thV, sV, s.w_in, thU, sU, s.w_out)
             del W
@@ -210,7 +219,7 @@ def run_ours(args, rk):
     from rotated_bit_matmul_b200 import replicas, synth
     device = torch.device("cuda", rk.local_rank)
     torch.cuda.set_device(device)
-    stack = build_stack(args.layers, device)
+    stack = build_stack(args.layers, device, args.rht)
     K, Wm = args.steps, args.warmup
     xs = torch.stack([torch.from_numpy(synth.activations(BATCH, HIDDEN, WORKLOAD, step=s)).to(torch.bfloat16)
                       for s in range(K + Wm)]).to(device)
@@ -278,7 +287,7 @@ def run_ours(args, rk):
     achieved = nbytes / (ms_step * 1e-3) / 1e9
     fused = stack.uses_fused_step(BATCH)
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": traffic_per_step(args.layers) if fused else None,
+                "frac": round(achieved / peak, 4), "traffic": traffic_per_step(args.layers) if fused and not args.rht else None,
                 "kernel": "decode_kernel (one launch per step)" if fused else "whole decode step (graph of kernels)",
                 "peak_kind": peak_kind, "algorithmic_bytes_per_step": nbytes}
     del g
@@ -294,7 +303,7 @@ def main():
     replicas.init(rk, "gloo" if args.impl == "reference" else "nccl")
     world = rk.world
 
-    config = {"workload": CONFIG_NAME, "layers": args.layers, "hidden": HIDDEN, "ffn": FFN, "bits": BITS,
+    config = {"workload": CONFIG_NAME_RHT if args.rht else CONFIG_NAME, "layers": args.layers, "hidden": HIDDEN, "ffn": FFN, "bits": BITS,
               "group": GROUP, "batch": BATCH, "global_batch": BATCH * world, "parallelism": f"replicas{world}",
               "l2": "inputs larger than L2: each step streams ~2.03 GB of packed codes and scales (L2 126 MB)"}
     base = {"metric": METRIC, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -306,7 +315,7 @@ def main():
         # rank 0 alone times the oracle; the other ranks leave without work
         if rk.rank == 0:
             tps, per_block, threads, passes = cpu_oracle_sample(args.cpu_sample_layers, steps=args.steps,
-                                                                warmup=args.warmup)
+                                                                warmup=args.warmup, rht=args.rht)
             ms = per_block * N_LAYERS * 1e3
             line = dict(base, impl="reference", value=tps, unit="tokens/s", ms_per_step=ms, dtype="f64",
                         cpu_baseline={"value": tps, "unit": "tokens/s", "cores": threads, "kind": "oracle",
@@ -320,7 +329,7 @@ def main():
     r = run_ours(args, rk)
     cpu = None
     if rk.rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tps, per_block, threads, passes = cpu_oracle_sample(args.cpu_sample_layers)
+        tps, per_block, threads, passes = cpu_oracle_sample(args.cpu_sample_layers, rht=args.rht)
         cpu = {"value": tps, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                "sample": f"{passes} passes of {args.cpu_sample_layers} of {N_LAYERS} blocks of one decode token "
                          f"(about 10 s of CPU work), scaled to {N_LAYERS} blocks"}

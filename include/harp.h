@@ -75,7 +75,9 @@ harp_status harp_device_status(void* stream);
  * Sec. 2.1-2.2 of the HARP page: signs, then stages of stride 1, 2, ..., w/2.
  *   n      : vector length, n % w == 0, n <= 2^30.
  *   w      : block width, a power of two, 2 <= w <= 8192.
- *   theta  : device fp32 [log2 w][n/2] angle offsets (the pi/4 is added inside).
+ *   theta  : device fp32 [log2 w][n/2] angle offsets (the pi/4 is added inside), or
+ *            NULL for Theta == 0: the fixed randomized Hadamard transform H_w D / sqrt(w)
+ *            per block (every 2x2 block [[1, 1], [1, -1]] / sqrt 2; no angles are read).
  *   sign   : device int8 [n], each +1 or -1.
  *   x, y   : device, dtypes xt / yt (f32, bf16, f16); y may equal x when xt == yt.
  * Arithmetic is fp32; sin/cos are evaluated in fp32 from pi/4 + theta.
@@ -105,6 +107,9 @@ harp_status harp_quantize_weights(int64_t n_out, int64_t n_in, int bits, int gro
  *   w_in, w_out : butterfly block widths: powers of two, 64 <= w <= 8192, w | n.
  *   theta_V, sign_V : device [log2 w_in][n_in/2] fp32, [n_in] int8 (input side V).
  *   theta_U, sign_U : device [log2 w_out][n_out/2] fp32, [n_out] int8 (U^T side).
+ *   A NULL theta_V or theta_U makes that side the fixed randomized Hadamard transform
+ *   (Theta == 0, "RHT"): its kernels use the constant 1/sqrt 2 blocks and load no
+ *   per-stage parameters. The codes must then come from a W' rotated with Theta == 0.
  *   codes, scale_zero : device, canonical layout above.
  * Ownership: the layer COPIES theta/sign (it stores cos/sin tables of pi/4 + theta in
  * its own device memory) and BORROWS codes and scale_zero, which the caller keeps

@@ -36,6 +36,10 @@ def _p(t):
     return ctypes.c_void_p(t.data_ptr()) if t is not None else None
 
 
+def _contig(t):
+    return t.contiguous() if t is not None else None
+
+
 def _stream():
     return ctypes.c_void_p(_torch().cuda.current_stream().cuda_stream)
 
@@ -65,7 +69,8 @@ def _bfly(name, x, theta, sign, w, out_dtype=None, out=None):
 
 
 def harp_butterfly_fwd(x, theta, sign, w, out_dtype=None, out=None):
-    """F(theta, s, w) x over the last dimension. theta fp32 [log2 w, n/2], sign int8 [n]."""
+    """F(theta, s, w) x over the last dimension. theta fp32 [log2 w, n/2] (None: Theta = 0,
+    the fixed randomized Hadamard transform), sign int8 [n]."""
     return _bfly("harp_butterfly_fwd", x, theta, sign, w, out_dtype, out)
 
 
@@ -96,7 +101,8 @@ def rotate_weights_device(W, theta_V, sign_V, w_in, theta_U, sign_U, w_out):
 
 
 class HarpLayer:
-    """A rotated low-bit linear on the device (wraps harp_create_layer)."""
+    """A rotated low-bit linear on the device (wraps harp_create_layer). theta_V or theta_U
+    None makes that side the fixed randomized Hadamard transform (Theta = 0)."""
 
     def __init__(self, n_in, n_out, bits, w_in, w_out, theta_V, sign_V, theta_U, sign_U, codes, scale_zero,
                  group=64):
@@ -107,7 +113,7 @@ class HarpLayer:
         self.codes, self.scale_zero = codes, scale_zero
         h = ctypes.c_void_p()
         call("harp_create_layer", ctypes.byref(h), self.n_in, self.n_out, self.bits, self.group, self.w_in,
-             self.w_out, _p(theta_V.contiguous()), _p(sign_V.contiguous()), _p(theta_U.contiguous()),
+             self.w_out, _p(_contig(theta_V)), _p(sign_V.contiguous()), _p(_contig(theta_U)),
              _p(sign_U.contiguous()), _p(codes), _p(scale_zero), _stream())
         self.handle = h
         self._ws = {}

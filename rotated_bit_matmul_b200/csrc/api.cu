@@ -101,8 +101,8 @@ harp_status check_bfly_args(int64_t n, int w, int batch, const float* theta, con
   if (n % w) return fail(HARP_ERR_INVALID_ARG, "butterfly: w=%d does not divide n=%lld", w, (long long)n);
   if (batch < 0 || batch > 65535) return fail(HARP_ERR_INVALID_ARG, "butterfly: batch=%d out of range", batch);
   if (!valid_dtype(xt) || !valid_dtype(yt)) return fail(HARP_ERR_INVALID_ARG, "butterfly: unknown dtype");
-  if (!theta || !sign || !x || !y) return fail(HARP_ERR_INVALID_ARG, "butterfly: null pointer");
-  if (!aligned16(theta) || !aligned16(sign) || !aligned16(x) || !aligned16(y))
+  if (!sign || !x || !y) return fail(HARP_ERR_INVALID_ARG, "butterfly: null pointer");
+  if ((theta && !aligned16(theta)) || !aligned16(sign) || !aligned16(x) || !aligned16(y))
     return fail(HARP_ERR_INVALID_ARG, "butterfly: device pointers must be 16-byte aligned");
   if (x == y && xt != yt) return fail(HARP_ERR_INVALID_ARG, "butterfly: in-place needs equal dtypes");
   return HARP_OK;
@@ -343,10 +343,9 @@ harp_status harp_create_layer(harp_layer* out, int64_t n_in, int64_t n_out, int 
     return fail(HARP_ERR_INVALID_ARG, "create_layer: w_in=%d must be a power of two in [64, 8192] dividing n_in", w_in);
   if (m_out < 1 || w_out > kMaxW || n_out % w_out)
     return fail(HARP_ERR_INVALID_ARG, "create_layer: w_out=%d must be a power of two in [2, 8192] dividing n_out", w_out);
-  if (!theta_V || !sign_V || !theta_U || !sign_U || !codes || !scale_zero)
-    return fail(HARP_ERR_INVALID_ARG, "create_layer: null pointer");
-  if (!aligned16(theta_V) || !aligned16(sign_V) || !aligned16(theta_U) || !aligned16(sign_U) || !aligned16(codes) ||
-      !aligned16(scale_zero))
+  if (!sign_V || !sign_U || !codes || !scale_zero) return fail(HARP_ERR_INVALID_ARG, "create_layer: null pointer");
+  if ((theta_V && !aligned16(theta_V)) || !aligned16(sign_V) || (theta_U && !aligned16(theta_U)) ||
+      !aligned16(sign_U) || !aligned16(codes) || !aligned16(scale_zero))
     return fail(HARP_ERR_INVALID_ARG, "create_layer: device pointers must be 16-byte aligned");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   harp_layer_s* h = new (std::nothrow) harp_layer_s();
@@ -373,12 +372,13 @@ harp_status harp_create_layer(harp_layer* out, int64_t n_in, int64_t n_out, int 
     return s;
   };
   cudaError_t e;
-  if ((e = cudaMalloc(&L.csV, sizeof(float2) * cnt_v)) != cudaSuccess ||
-      (e = cudaMalloc(&L.csU, sizeof(float2) * cnt_u)) != cudaSuccess ||
+  // a side with a null theta is the fixed randomized Hadamard transform: no table
+  if ((theta_V && (e = cudaMalloc(&L.csV, sizeof(float2) * cnt_v)) != cudaSuccess) ||
+      (theta_U && (e = cudaMalloc(&L.csU, sizeof(float2) * cnt_u)) != cudaSuccess) ||
       (e = cudaMalloc(&L.sV, (size_t)n_in)) != cudaSuccess || (e = cudaMalloc(&L.sU, (size_t)n_out)) != cudaSuccess)
     return cleanup(cuda_fail(e, "create_layer: cudaMalloc"));
-  if ((e = launch_cs_table(theta_V, cnt_v, L.csV, st)) != cudaSuccess ||
-      (e = launch_cs_table(theta_U, cnt_u, L.csU, st)) != cudaSuccess ||
+  if ((theta_V && (e = launch_cs_table(theta_V, cnt_v, L.csV, st)) != cudaSuccess) ||
+      (theta_U && (e = launch_cs_table(theta_U, cnt_u, L.csU, st)) != cudaSuccess) ||
       (e = cudaMemcpyAsync(L.sV, sign_V, (size_t)n_in, cudaMemcpyDeviceToDevice, st)) != cudaSuccess ||
       (e = cudaMemcpyAsync(L.sU, sign_U, (size_t)n_out, cudaMemcpyDeviceToDevice, st)) != cudaSuccess)
     return cleanup(cuda_fail(e, "create_layer: copies"));

@@ -26,6 +26,7 @@ namespace harp {
 namespace {
 
 constexpr int kBflyThreads = 256;
+constexpr float kRsqrt2 = 0.70710678118654752440f;  // cos(pi/4) = sin(pi/4)
 
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
@@ -67,7 +68,9 @@ __device__ __forceinline__ void stage_a(float* x, const void* tab, int t, int E,
   for (int q = tid; q < (E >> 1); q += nthr) {
     const int i = ((q >> t) << (t + 1)) | (q & (h - 1));
     float c, s;
-    if (CS) {
+    if (!tab) {
+      c = s = kRsqrt2;  // Theta == 0: the randomized Hadamard transform
+    } else if (CS) {
       const float2 v = static_cast<const float2*>(tab)[q];
       c = v.x;
       s = v.y;
@@ -88,7 +91,9 @@ __device__ __forceinline__ void stage_b(float* x, const void* tab, int d, int ru
     const int jj = q / run, ii = q - jj * run;
     const int j = ((jj >> d) << (d + 1)) | (jj & ((1 << d) - 1));
     float c, s;
-    if (CS) {
+    if (!tab) {
+      c = s = kRsqrt2;
+    } else if (CS) {
       const float2 v = static_cast<const float2*>(tab)[q];
       c = v.x;
       s = v.y;
@@ -120,12 +125,16 @@ __global__ void __launch_bounds__(kBflyThreads) bfly_kernel(BflyParams p, int C)
   uint8_t* tab = reinterpret_cast<uint8_t*>(xb + E);
   uint64_t* bar = reinterpret_cast<uint64_t*>(tab + (size_t)m * (E >> 1) * esz);
   const void* gtab = CS ? static_cast<const void*>(p.cs) : static_cast<const void*>(p.theta);
+  const bool rht = gtab == nullptr;  // Theta == 0: no per-stage parameters to load
+  const uint8_t* stab = rht ? nullptr : tab;
 
   // ---- prefetch this CTA's parameter slice: stage t occupies E/2 entries. Bulk copies
   // need 16-byte aligned sources, destinations and sizes; tiny widths use plain loads.
-  const bool use_bulk = (((E >> 1) * esz) % 16 == 0) && ((half_n * esz) % 16 == 0) &&
+  const bool use_bulk = !rht && (((E >> 1) * esz) % 16 == 0) && ((half_n * esz) % 16 == 0) &&
                         (((w >> 1) * esz) % 16 == 0) && (C == 1 || (run * esz) % 16 == 0);
-  if (!use_bulk) {
+  if (rht) {
+    // nothing to prefetch
+  } else if (!use_bulk) {
     for (int t = 0; t < m; ++t) {
       const uint8_t* src_stage = static_cast<const uint8_t*>(gtab) + ((int64_t)t * half_n + blk * (w >> 1)) * esz;
       uint8_t* dst = tab + (size_t)t * (E >> 1) * esz;
@@ -174,7 +183,7 @@ __global__ void __launch_bounds__(kBflyThreads) bfly_kernel(BflyParams p, int C)
     __syncthreads();
     if (use_bulk) mbar_wait(bar, 0, p.status, 10);
     for (int t = 0; t < g.e; ++t) {
-      stage_a<CS>(xa, tab + (size_t)t * (E >> 1) * esz, t, E, tid, nthr);
+      stage_a<CS>(xa, stab ? stab + (size_t)t * (E >> 1) * esz : nullptr, t, E, tid, nthr);
       __syncthreads();
     }
     float* out = xa;
@@ -186,7 +195,7 @@ __global__ void __launch_bounds__(kBflyThreads) bfly_kernel(BflyParams p, int C)
       }
       cluster_sync();  // every peer has finished reading this CTA's chunk
       for (int d = 0; d < g.lc; ++d) {
-        stage_b<CS>(xb, tab + (size_t)(g.e + d) * (E >> 1) * esz, d, run, E, tid, nthr);
+        stage_b<CS>(xb, stab ? stab + (size_t)(g.e + d) * (E >> 1) * esz : nullptr, d, run, E, tid, nthr);
         __syncthreads();
       }
       out = xb;
@@ -245,7 +254,7 @@ __global__ void __launch_bounds__(kBflyThreads) bfly_kernel(BflyParams p, int C)
       __syncthreads();
       if (use_bulk) mbar_wait(bar, 0, p.status, 11);
       for (int d = g.lc - 1; d >= 0; --d) {
-        stage_b<CS>(xb, tab + (size_t)(g.e + d) * (E >> 1) * esz, d, run, E, tid, nthr);
+        stage_b<CS>(xb, stab ? stab + (size_t)(g.e + d) * (E >> 1) * esz : nullptr, d, run, E, tid, nthr);
         __syncthreads();
       }
       cluster_sync();
@@ -260,7 +269,7 @@ __global__ void __launch_bounds__(kBflyThreads) bfly_kernel(BflyParams p, int C)
       if (use_bulk) mbar_wait(bar, 0, p.status, 11);
     }
     for (int t = g.e - 1; t >= 0; --t) {
-      stage_a<CS>(cur, tab + (size_t)t * (E >> 1) * esz, t, E, tid, nthr);
+      stage_a<CS>(cur, stab ? stab + (size_t)t * (E >> 1) * esz : nullptr, t, E, tid, nthr);
       __syncthreads();
     }
     for (int i = tid; i < E; i += nthr) {

@@ -235,6 +235,7 @@ __device__ __forceinline__ uint32_t load_table_cluster(float2* dst, const float2
                                        uint64_t* bar) {
   const int E = w / kC, e = m - 3, run = E / kC;
   const int64_t half_n = n >> 1;
+  if (!cs) return (uint32_t)(8 * m * (E >> 1));  // Theta == 0: nothing to copy, same layout
   for (int t = 0; t < m; ++t) {
     const float2* src = cs + (int64_t)t * half_n + (int64_t)blk * (w >> 1);
     float2* d = dst + (size_t)t * (E >> 1);
@@ -254,17 +255,24 @@ __device__ __forceinline__ uint32_t load_table_cluster(float2* dst, const float2
 
 // the whole block `blk` of width w held by one CTA: one run of w/2 pairs per stage
 __device__ __forceinline__ uint32_t load_table_local(float2* dst, const float2* cs, int64_t n, int w, int m, int blk, uint64_t* bar) {
+  if (!cs) return (uint32_t)(4 * w * m);
   for (int t = 0; t < m; ++t)
     bulk_g2s(dst + (size_t)t * (w >> 1), cs + (int64_t)t * (n >> 1) + (int64_t)blk * (w >> 1), (uint32_t)(4 * w), bar);
   return (uint32_t)(4 * w * m);
 }
 
 __device__ __forceinline__ uint32_t table_bytes_cluster(int w, int m) { return (uint32_t)(8 * m * (w / kC / 2)); }
+// bytes a table load actually transfers (none for a Theta == 0 side)
+__device__ __forceinline__ uint32_t copied_bytes_cluster(const float2* cs, int w, int m) {
+  return cs ? table_bytes_cluster(w, m) : 0u;
+}
 
 // P7 roles: block CTAs, and the clusters applying F_U_q / F_U_k
 __device__ __forceinline__ int qk_cluster(const Params& p, int which) { return p.G - 1 - which; }
 
 // ------------------------------------------------------------------ butterfly stages
+constexpr float kRsqrt2 = 0.70710678118654752440f;  // cos(pi/4) = sin(pi/4): the Theta == 0 block
+
 __device__ __forceinline__ void rot(float& a, float& b, float2 cs) {
   const float x = a, y = b;
   a = fmaf(cs.x, x, cs.y * y);
@@ -273,7 +281,8 @@ __device__ __forceinline__ void rot(float& a, float& b, float2 cs) {
 
 // NS stages t .. t+NS-1 (pairs (i, i + 2^s)) on a buffer of E elements, 2^NS values per
 // thread held in registers; table row s (E/2 pairs, pair numbered by first index).
-template <int NS>
+// HAD: every block is the Theta == 0 block [[1, 1], [1, -1]] / sqrt 2 (no table read).
+template <int NS, bool HAD>
 __device__ __forceinline__ void round_a(float* x, const float2* tab, int t, int E, int ct) {
   constexpr int P = 1 << NS;
   const int nthr = E / P, h = 1 << t;
@@ -291,7 +300,7 @@ __device__ __forceinline__ void round_a(float* x, const float2* tab, int t, int 
         if (k & (1 << s)) continue;
         const int i = base + k * h;
         const int q = ((i >> (ts + 1)) << ts) | (i & (hs - 1));
-        rot(v[k], v[k + (1 << s)], tt[q]);
+        rot(v[k], v[k + (1 << s)], HAD ? make_float2(kRsqrt2, kRsqrt2) : tt[q]);
       }
     }
 #pragma unroll
@@ -301,18 +310,20 @@ __device__ __forceinline__ void round_a(float* x, const float2* tab, int t, int 
 }
 
 // layout-A stages t0 .. t1-1, three per shared-memory round
+template <bool HAD>
 __device__ __forceinline__ void stages_a(float* x, const float2* tab, int t0, int t1, int E, int ct) {
   int t = t0;
   while (t1 - t >= 3) {
-    round_a<3>(x, tab, t, E, ct);
+    round_a<3, HAD>(x, tab, t, E, ct);
     t += 3;
   }
-  if (t1 - t == 2) round_a<2>(x, tab, t, E, ct);
-  if (t1 - t == 1) round_a<1>(x, tab, t, E, ct);
+  if (t1 - t == 2) round_a<2, HAD>(x, tab, t, E, ct);
+  if (t1 - t == 1) round_a<1, HAD>(x, tab, t, E, ct);
 }
 
 // the three layout-B stages (runs j and j + 2^d, same offset), one round: thread T holds
 // the 8 values {j run + T}; table rows e, e+1, e+2 numbered jj run + T
+template <bool HAD>
 __device__ __forceinline__ void stages_b(float* x, const float2* tab, int e, int E, int ct) {
   const int run = E / kC;
   if (ct < run) {
@@ -326,7 +337,7 @@ __device__ __forceinline__ void stages_b(float* x, const float2* tab, int e, int
       for (int j = 0; j < kC; ++j) {
         if (j & (1 << d)) continue;
         const int jj = ((j >> (d + 1)) << d) | (j & ((1 << d) - 1));
-        rot(v[j], v[j + (1 << d)], tt[jj * run + ct]);
+        rot(v[j], v[j + (1 << d)], HAD ? make_float2(kRsqrt2, kRsqrt2) : tt[jj * run + ct]);
       }
     }
 #pragma unroll
@@ -447,6 +458,7 @@ __device__ __forceinline__ float zsum(const float* zp, int nk, int n, int i) {
 
 // ------------------------------------------------------------------ chains (cluster-collective)
 // residual chain: [res += F_U(z)] ; n = rms(res) ; x~ = F_V(n) ; operand
+template <bool HAD>
 __device__ __forceinline__ bool chain_residual(const Params& p, Smem& s, Xchg& X, const Lin* U, const float* zp, int nk,
                                const Lin* V, bool first, uint32_t r, int ct, const float2* tabU,
                                const float2* tabV) {
@@ -459,10 +471,10 @@ __device__ __forceinline__ bool chain_residual(const Params& p, Smem& s, Xchg& X
       s.xa[i] = zsum(zp, nk, W, gi) * (float)s.sgn[i];
     }
     cbar();
-    stages_a(s.xa, tabU, 0, e, E, ct);
+    stages_a<HAD>(s.xa, tabU, 0, e, E, ct);
     push_a_to_b(s.xa, s.xb, E, r, ct);
     if (!exchange(s, X, ct, p.status, 41)) return false;
-    stages_b(s.xb, tabU, e, E, ct);
+    stages_b<HAD>(s.xb, tabU, e, E, ct);
     for (int L = ct; L < E; L += kNT) s.res[L] += s.xb[L];
   }
   if (!V) {
@@ -489,26 +501,28 @@ __device__ __forceinline__ bool chain_residual(const Params& p, Smem& s, Xchg& X
   const float inv = 1.0f / sqrtf(t / (float)W + p.eps);
   for (int i = ct; i < E; i += kNT) s.xa[i] *= inv * (float)s.sgn[kSgnSlot + i];
   cbar();
-  stages_a(s.xa, tabV, 0, e, E, ct);
+  stages_a<HAD>(s.xa, tabV, 0, e, E, ct);
   push_a_to_b(s.xa, s.xb, E, r, ct);
   if (!exchange(s, X, ct, p.status, 43)) return false;
-  stages_b(s.xb, tabV, e, E, ct);
+  stages_b<HAD>(s.xb, tabV, e, E, ct);
   return prep_and_broadcast(s, X, s.xb, V->n_in, p.bits, E, r, ct, p.status);
 }
 
 // attention chain: v = F_U_v(z_v); a = v broadcast per KV group; x~ = F_V_o(a); operand
+template <bool HAD>
 __device__ __forceinline__ bool chain_attn(const Params& p, Smem& s, Xchg& X, const Lin* Lv, const Lin* Lo, uint32_t r, int ct,
                            const float2* tabU, const float2* tabV) {
   const int Wu = Lv->w_out, Eu = Wu / kC, eu = Lv->m_out - 3;
+
   for (int i = ct; i < Eu; i += kNT) {
     const int gi = (int)r * Eu + i;
     s.xa[i] = zsum(p.zpv, p.nk_h, Wu, gi) * (float)s.sgn[i];
   }
   cbar();
-  stages_a(s.xa, tabU, 0, eu, Eu, ct);
+  stages_a<HAD>(s.xa, tabU, 0, eu, Eu, ct);
   push_a_to_b(s.xa, s.xb, Eu, r, ct);
   if (!exchange(s, X, ct, p.status, 44)) return false;
-  stages_b(s.xb, tabU, eu, Eu, ct);
+  stages_b<HAD>(s.xb, tabU, eu, Eu, ct);
   // push every v value to the layout-A owners of the query-head elements that copy it
   const int Eo = p.E, eo = p.m_hidden - 3, hd = p.head_dim, rep = p.rep;
   for (int L = ct; L < Eu; L += kNT) {
@@ -521,26 +535,28 @@ __device__ __forceinline__ bool chain_attn(const Params& p, Smem& s, Xchg& X, co
   if (!exchange(s, X, ct, p.status, 45)) return false;
   for (int i = ct; i < Eo; i += kNT) s.xa[i] *= (float)s.sgn[kSgnSlot + i];
   cbar();
-  stages_a(s.xa, tabV, 0, eo, Eo, ct);
+  stages_a<HAD>(s.xa, tabV, 0, eo, Eo, ct);
   push_a_to_b(s.xa, s.xb, Eo, r, ct);
   if (!exchange(s, X, ct, p.status, 46)) return false;
-  stages_b(s.xb, tabV, eo, Eo, ct);
+  stages_b<HAD>(s.xb, tabV, eo, Eo, ct);
   return prep_and_broadcast(s, X, s.xb, Lo->n_in, p.bits, Eo, r, ct, p.status);
 }
 
 // F_U of a q or k GEMV output (cluster-distributed), written to out[gidx]
+template <bool HAD>
 __device__ __forceinline__ bool chain_out_only(const Params& p, Smem& s, Xchg& X, const Lin* Lq, const float* zp, float* out,
                                uint32_t r, int ct, const float2* tab) {
   const int W = Lq->w_out, E = W / kC, e = Lq->m_out - 3;
+
   for (int i = ct; i < E; i += kNT) {
     const int gi = (int)r * E + i;
     s.xa[i] = zsum(zp, p.nk_h, W, gi) * (float)s.sgn[i];
   }
   cbar();
-  stages_a(s.xa, tab, 0, e, E, ct);
+  stages_a<HAD>(s.xa, tab, 0, e, E, ct);
   push_a_to_b(s.xa, s.xb, E, r, ct);
   if (!exchange(s, X, ct, p.status, 47)) return false;
-  stages_b(s.xb, tab, e, E, ct);
+  stages_b<HAD>(s.xb, tab, e, E, ct);
   for (int L = ct; L < E; L += kNT) out[gidx_b(L, E, r)] = s.xb[L];
   cbar();
   return true;
@@ -548,6 +564,7 @@ __device__ __forceinline__ bool chain_out_only(const Params& p, Smem& s, Xchg& X
 
 // one whole MLP block (width <= 512) in one CTA: F_U_gate, F_U_up, silu*up, F_V_down,
 // operand of the down projection for this block (to global)
+template <bool HAD>
 __device__ __forceinline__ void block_chain(const Params& p, Smem& s, const Lin* Lg, const Lin* Lu, const Lin* Ld, int blk, int ct,
                             const float2* tab) {
   const int wb = Lg->w_out, mb = Lg->m_out, F = p.ffn;
@@ -557,14 +574,14 @@ __device__ __forceinline__ void block_chain(const Params& p, Smem& s, const Lin*
     s.xb[i] = zsum(p.zpu, p.nk_h, F, base + i) * (float)s.sgn[kSgnSlot + i];
   }
   cbar();
-  stages_a(s.xa, tab, 0, mb, wb, ct);
-  stages_a(s.xb, tab + (size_t)mb * (wb >> 1), 0, mb, wb, ct);
+  stages_a<HAD>(s.xa, tab, 0, mb, wb, ct);
+  stages_a<HAD>(s.xb, tab + (size_t)mb * (wb >> 1), 0, mb, wb, ct);
   for (int i = ct; i < wb; i += kNT) {
     const float g = s.xa[i];
     s.xa[i] = g / (1.0f + expf(-g)) * s.xb[i] * (float)s.sgn[2 * kSgnSlot + i];
   }
   cbar();
-  stages_a(s.xa, tab + (size_t)2 * mb * (wb >> 1), 0, mb, wb, ct);
+  stages_a<HAD>(s.xa, tab + (size_t)2 * mb * (wb >> 1), 0, mb, wb, ct);
   const int n_in = Ld->n_in;
   int16_t* xq16 = reinterpret_cast<int16_t*>(p.xq_down);
   const int warp = ct >> 5, lane = ct & 31;
@@ -668,7 +685,9 @@ __device__ __noinline__ bool grid_barrier(const Params& p, int idx, int ct) {
 }
 
 // ------------------------------------------------------------------ the kernel
-template <int BITS>
+// HAD: every butterfly of the stack is the fixed randomized Hadamard transform (Theta == 0,
+// no cos/sin tables); the learned-angle instantiation keeps its rounds free of that case.
+template <int BITS, bool HAD>
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_constant__ Params p) {
   using Gm = Geo<BITS>;
   Smem s = carve(p, Gm::kStageBytes);
@@ -759,9 +778,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         if (!(ok = begin())) break;
         if (lane == 0) {
           uint32_t bytes = 0;
-          if (prev) bytes += table_bytes_cluster(prev[6].w_out, prev[6].m_out);
+          if (prev) bytes += copied_bytes_cluster(prev[6].csU, prev[6].w_out, prev[6].m_out);
           const Lin* V = l < L ? lin + p.asg_qkv[c] : nullptr;
-          if (V) bytes += table_bytes_cluster(V->w_in, V->m_in);
+          if (V) bytes += copied_bytes_cluster(V->csV, V->w_in, V->m_in);
           const int Eh = p.E;
           if (prev) bytes += Eh;
           if (V) bytes += Eh;
@@ -781,7 +800,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         if (lane == 0) {
           const uint32_t b0 = table_bytes_cluster(lin[2].w_out, lin[2].m_out);
           const int Eu = lin[2].w_out / kC, Eo = lin[3].w_in / kC;
-          mbar_arrive_expect_tx(s.tab_full, b0 + table_bytes_cluster(lin[3].w_in, lin[3].m_in) + Eu + Eo);
+          mbar_arrive_expect_tx(s.tab_full, copied_bytes_cluster(lin[2].csU, lin[2].w_out, lin[2].m_out) +
+                                                copied_bytes_cluster(lin[3].csV, lin[3].w_in, lin[3].m_in) + Eu + Eo);
           load_table_cluster(s.tab, lin[2].csU, lin[2].n_out, lin[2].w_out, lin[2].m_out, 0, (int)r, s.tab_full);
           load_table_cluster(s.tab + b0 / 8, lin[3].csV, lin[3].n_in, lin[3].w_in, lin[3].m_in, 0, (int)r, s.tab_full);
           bulk_g2s(s.sgn, lin[2].sU + (int64_t)r * Eu, (uint32_t)Eu, s.tab_full);
@@ -794,7 +814,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
           const Lin* V = lin + 4 + p.asg_gu[c];
           const uint32_t b0 = table_bytes_cluster(lin[3].w_out, lin[3].m_out);
           const int Eh = p.E;
-          mbar_arrive_expect_tx(s.tab_full, b0 + table_bytes_cluster(V->w_in, V->m_in) + 2 * Eh);
+          mbar_arrive_expect_tx(s.tab_full, copied_bytes_cluster(lin[3].csU, lin[3].w_out, lin[3].m_out) +
+                                                copied_bytes_cluster(V->csV, V->w_in, V->m_in) + 2 * Eh);
           load_table_cluster(s.tab, lin[3].csU, lin[3].n_out, lin[3].w_out, lin[3].m_out, 0, (int)r, s.tab_full);
           load_table_cluster(s.tab + b0 / 8, V->csV, V->n_in, V->w_in, V->m_in, 0, (int)r, s.tab_full);
           bulk_g2s(s.sgn, lin[3].sU + (int64_t)r * Eh, (uint32_t)Eh, s.tab_full);
@@ -807,10 +828,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
           uint32_t bytes = 0;
           const int wb = lin[4].w_out, mb = lin[4].m_out;
           const int blk = t_cta;  // at most one MLP block per CTA (checked at set-up)
-          if (blk < nblocks) bytes += 3 * 4 * wb * mb + 3 * wb;
+          if (blk < nblocks)
+            bytes += (lin[4].csU ? 4 * wb * mb : 0) + (lin[5].csU ? 4 * wb * mb : 0) + (lin[6].csV ? 4 * wb * mb : 0) +
+                     3 * wb;
           const int qk = c == qk_cluster(p, 0) ? 0 : (c == qk_cluster(p, 1) ? 1 : -1);
           const int Eq = qk >= 0 ? lin[qk].w_out / kC : 0;
-          if (qk >= 0) bytes += table_bytes_cluster(lin[qk].w_out, lin[qk].m_out) + Eq;
+          if (qk >= 0) bytes += copied_bytes_cluster(lin[qk].csU, lin[qk].w_out, lin[qk].m_out) + Eq;
           mbar_arrive_expect_tx(s.tab_full, bytes);
           if (blk < nblocks) {
             uint32_t off = 0;
@@ -855,7 +878,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     {
       const float2* tU = s.tab;
       const float2* tV = prev ? s.tab + table_bytes_cluster(prev[6].w_out, prev[6].m_out) / 8 : s.tab;
-      ok = chain_residual(p, s, X, prev ? prev + 6 : nullptr, p.zpd, p.nk_f, lin + p.asg_qkv[c], l == 0, r, ct, tU,
+      ok = chain_residual<HAD>(p, s, X, prev ? prev + 6 : nullptr, p.zpd, p.nk_f, lin + p.asg_qkv[c], l == 0, r, ct, tU,
                           tV);
     }
     tab_release();
@@ -865,7 +888,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     if (!(ok = grid_barrier(p, l * 5 + 0, ct))) break;
     // P3
     if (!(ok = tab_acquire())) break;
-    ok = chain_attn(p, s, X, lin + 2, lin + 3, r, ct, s.tab,
+    ok = chain_attn<HAD>(p, s, X, lin + 2, lin + 3, r, ct, s.tab,
                     s.tab + table_bytes_cluster(lin[2].w_out, lin[2].m_out) / 8);
     tab_release();
     if (!ok) break;
@@ -874,7 +897,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     if (!(ok = grid_barrier(p, l * 5 + 1, ct))) break;
     // P5
     if (!(ok = tab_acquire())) break;
-    ok = chain_residual(p, s, X, lin + 3, p.zpo, p.nk_h, lin + 4 + p.asg_gu[c], false, r, ct, s.tab,
+    ok = chain_residual<HAD>(p, s, X, lin + 3, p.zpo, p.nk_h, lin + 4 + p.asg_gu[c], false, r, ct, s.tab,
                         s.tab + table_bytes_cluster(lin[3].w_out, lin[3].m_out) / 8);
     tab_release();
     if (!ok) break;
@@ -884,13 +907,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     // P7
     if (!(ok = tab_acquire())) break;
     {
-      if (t_cta < nblocks) block_chain(p, s, lin + 4, lin + 5, lin + 6, t_cta, ct, s.tab);
+      if (t_cta < nblocks) block_chain<HAD>(p, s, lin + 4, lin + 5, lin + 6, t_cta, ct, s.tab);
       const int qk = c == qk_cluster(p, 0) ? 0 : (c == qk_cluster(p, 1) ? 1 : -1);
       if (qk >= 0) {
         float* out = qk == 0 ? p.qout + (int64_t)l * lin[0].n_out : p.kout + (int64_t)l * lin[1].n_out;
         const float* zp = qk == 0 ? p.zpq + (int64_t)l * p.nk_h * lin[0].n_out
                                   : p.zpk + (int64_t)l * p.nk_h * lin[1].n_out;
-        ok = chain_out_only(p, s, X, lin + qk, zp, out, r, ct, s.tab);
+        ok = chain_out_only<HAD>(p, s, X, lin + qk, zp, out, r, ct, s.tab);
       }
     }
     tab_release();
@@ -916,7 +939,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   // final: out = h_{L-1} + F_U_down(z_down)
   if (ok && (ok = tab_acquire())) {
     const Lin* last = p.lin + 7 * (L - 1);
-    ok = chain_residual(p, s, X, last + 6, p.zpd, p.nk_f, nullptr, false, r, ct, s.tab, s.tab);
+    ok = chain_residual<HAD>(p, s, X, last + 6, p.zpd, p.nk_f, nullptr, false, r, ct, s.tab, s.tab);
     if (ok && c == 0)
       for (int L2 = ct; L2 < p.E; L2 += kNT) store_act(p.y_out, gidx_b(L2, p.E, r), p.yt, s.res[L2]);
     tab_release();
@@ -933,14 +956,16 @@ size_t smem_bytes(const Params& p) {
 }
 
 template <int BITS>
-const void* kernel_ptr() {
-  return reinterpret_cast<const void*>(decode_kernel<BITS>);
+const void* kernel_ptr(bool had) {
+  return had ? reinterpret_cast<const void*>(decode_kernel<BITS, true>)
+             : reinterpret_cast<const void*>(decode_kernel<BITS, false>);
 }
 
 template <int BITS>
 cudaError_t launch_bits(const Params& p, cudaStream_t st) {
   const size_t smem = smem_bytes<BITS>(p);
-  cudaError_t e = cudaFuncSetAttribute(decode_kernel<BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(kernel_ptr<BITS>(p.had != 0), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(p.G * kC), 1, 1);
@@ -954,7 +979,8 @@ cudaError_t launch_bits(const Params& p, cudaStream_t st) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_kernel<BITS>, p);
+  return p.had ? cudaLaunchKernelEx(&cfg, decode_kernel<BITS, true>, p)
+               : cudaLaunchKernelEx(&cfg, decode_kernel<BITS, false>, p);
 }
 
 cudaError_t launch(const Params& p, cudaStream_t st) {
@@ -983,7 +1009,8 @@ int chunk_cols_for(int bits) {
 }
 
 cudaError_t max_clusters(const Params& p, int* out) {
-  const void* fn = p.bits == 2 ? kernel_ptr<2>() : (p.bits == 3 ? kernel_ptr<3>() : kernel_ptr<4>());
+  const bool had = p.had != 0;
+  const void* fn = p.bits == 2 ? kernel_ptr<2>(had) : (p.bits == 3 ? kernel_ptr<3>(had) : kernel_ptr<4>(had));
   const size_t smem = smem_for(p);
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

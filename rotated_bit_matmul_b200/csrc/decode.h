@@ -44,6 +44,7 @@ struct Params {
   float* xsum_down;
   unsigned* counters;  // [L][5], zero at launch
   int* status;
+  int had;  // every butterfly is Theta == 0 (the fixed randomized Hadamard transform)
   int ring_stages, tab_bytes, xq_bytes;
   int asg_qkv[kMaxClusters], idx_qkv[kMaxClusters], cnt_qkv[3];
   int asg_gu[kMaxClusters], idx_gu[kMaxClusters], cnt_gu[2];

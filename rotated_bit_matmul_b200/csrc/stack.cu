@@ -231,8 +231,17 @@ void setup_fused(harp_stack_s* S) {
     if (L[4]->w_out != wb || L[5]->w_out != wb || L[6]->w_in != wb) return no("gate/up output and down input blocks must match");
     if (L[6]->w_out != H) return no("down output butterfly must be hidden-wide");
   }
+  // every butterfly learned (cos/sin tables) or every one Theta == 0: one kernel
+  // instantiation per case, so neither pays for the other in its rotation rounds
+  bool any_learned = false, any_fixed = false;
+  for (const harp_layer l : S->layers) {
+    any_learned |= l->L.csV != nullptr || l->L.csU != nullptr;
+    any_fixed |= l->L.csV == nullptr || l->L.csU == nullptr;
+  }
+  if (any_learned && any_fixed) return no("mixing learned and Theta = 0 butterflies is not fused");
   dec::Params& p = S->fp;
   p = dec::Params{};
+  p.had = any_fixed ? 1 : 0;
   p.L = S->n_layers;
   p.hidden = H;
   p.ffn = F;
