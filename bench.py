@@ -71,7 +71,7 @@ def algorithmic_bytes_per_step(n_layers, batch=BATCH, bits=BITS):
 # ncu capture summarised in profiles/decode_kernel_llama2-7b_2bit_batch1.md (4-block
 # case, 271.64 MB per launch, scaled by blocks), and a hash of the kernel's sources at
 # capture time: the figure is reported only while those sources are unchanged.
-TRAFFIC_PER_BLOCK = {"bytes": 271_644_160 // 4, "sources_sha256_16": "0e560bffa6d2c883"}
+TRAFFIC_PER_BLOCK = {"bytes": 271_644_160 // 4, "sources_sha256_16": "53b216f27efb691e"}
 KERNEL_SOURCES = ("decode.cu", "decode.h", "common.cuh", "gemv_core.cuh")
 
 

@@ -181,8 +181,4 @@ __device__ __forceinline__ int group_exponent(float amax) {
 // 2^e for e in [-126, 127], exact
 __device__ __forceinline__ float pow2f(int e) { return __int_as_float((e + 127) << 23); }
 
-// ------------------------------------------------------------------ programmatic dependent launch
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" :::); }
-
 }  // namespace harp

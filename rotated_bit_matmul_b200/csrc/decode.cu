@@ -1000,10 +1000,6 @@ size_t smem_for(const Params& p) {
   }
 }
 
-int stage_bytes_for(int bits) {
-  return bits == 2 ? Geo<2>::kStageBytes : (bits == 3 ? Geo<3>::kStageBytes : Geo<4>::kStageBytes);
-}
-
 int chunk_cols_for(int bits) {
   return bits == 2 ? Geo<2>::kChunkCols : (bits == 3 ? Geo<3>::kChunkCols : Geo<4>::kChunkCols);
 }

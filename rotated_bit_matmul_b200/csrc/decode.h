@@ -52,7 +52,6 @@ struct Params {
 
 cudaError_t launch(const Params& p, cudaStream_t st);
 size_t smem_for(const Params& p);
-int stage_bytes_for(int bits);
 int chunk_cols_for(int bits);
 cudaError_t max_clusters(const Params& p, int* out);
 
