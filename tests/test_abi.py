@@ -101,3 +101,24 @@ def test_binding_fails_loudly_without_library(tmp_path):
             _lib.load(str(tmp_path / "missing.so"))
         finally:
             _lib._lib = saved
+
+
+def _no_gpu():
+    import torch
+    if torch.cuda.is_available():
+        # on a GPU the calls below would reach the device with placeholder pointers
+        pytest.skip("needs a machine without a CUDA device")
+
+
+def test_null_theta_passes_validation(lib):
+    """A null theta selects the fixed randomized Hadamard transform (Theta = 0): argument
+    checks accept it, and without a GPU the calls fail only at the first CUDA call
+    (HARP_ERR_CUDA), not as HARP_ERR_INVALID_ARG."""
+    _no_gpu()
+    h = ctypes.c_void_p()
+    st = lib.harp_create_layer(ctypes.byref(h), 4096, 4096, 2, 64, 4096, 4096, None, FAKE, None, FAKE, FAKE,
+                               FAKE, None)
+    assert st == 3 and not h.value, lib.harp_last_error()
+    assert lib.harp_butterfly_fwd(4096, 4096, 1, None, FAKE, FAKE, 0, FAKE, 0, None) == 3
+    # a null sign vector is still an error
+    assert lib.harp_butterfly_fwd(4096, 4096, 1, None, None, FAKE, 0, FAKE, 0, None) == 1
