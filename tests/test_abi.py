@@ -122,3 +122,9 @@ def test_null_theta_passes_validation(lib):
     assert lib.harp_butterfly_fwd(4096, 4096, 1, None, FAKE, FAKE, 0, FAKE, 0, None) == 3
     # a null sign vector is still an error
     assert lib.harp_butterfly_fwd(4096, 4096, 1, None, None, FAKE, 0, FAKE, 0, None) == 1
+
+
+def test_empty_batch_is_a_no_op(lib):
+    """batch 0 is valid for the butterflies and returns before any launch."""
+    assert lib.harp_butterfly_fwd(4096, 4096, 0, FAKE, FAKE, FAKE, 0, FAKE, 0, None) == 0
+    assert lib.harp_butterfly_inv(4096, 4096, 0, None, FAKE, FAKE, 0, FAKE, 0, None) == 0
