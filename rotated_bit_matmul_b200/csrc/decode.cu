@@ -594,22 +594,29 @@ __device__ __forceinline__ void block_chain(const Params& p, Smem& s, const Lin*
 }
 
 // ------------------------------------------------------------------ GEMV (consumer side)
-// Warps move through the CTA's units on their own; the last warp to finish a unit
-// reduces the 16 per-warp partial rows and writes the unit's partial sums.
+// The 16 consumer warps form two halves that take alternate units of the CTA's range,
+// so two units are in flight and each warp covers 8 groups of a unit; the last warp of a
+// half to finish a unit reduces its 8 per-warp partial rows and writes the unit's sums.
+constexpr int kHalf = kCW / 2;
+
 template <int BITS>
 __device__ __forceinline__ bool run_units(const Params& p, Smem& s, const Range& g, uint32_t& kring, int ct) {
   using Gm = Geo<BITS>;
   const int warp = ct >> 5, lane = ct & 31;
+  const int hv = warp / kHalf, hw = warp - hv * kHalf;  // half, warp within the half
   const int n_out = g.L->n_out, n_in = g.L->n_in, ngroups = n_in / 64;
   const int words = BITS == 3 ? n_in : n_in / 2;
   const float* xsA = reinterpret_cast<const float*>(s.xq + words);
   const float* xsumA = xsA + ngroups;
+  const int nu = g.u1 - g.u0;
   bool ok = true;
-  for (int u = g.u0; u < g.u1; ++u, ++kring) {
-    const int slot = kring % p.ring_stages;
+  for (int i = hv; i < nu; i += 2) {
+    const uint32_t kr = kring + (uint32_t)i;
+    const int slot = kr % p.ring_stages;
+    const int u = g.u0 + i;
     if (ok) {
       int w = 1;
-      if (lane == 0) w = wait_phase<false>(&s.full[slot], (kring / p.ring_stages) & 1, p.status, 50);
+      if (lane == 0) w = wait_phase<false>(&s.full[slot], (kr / p.ring_stages) & 1, p.status, 50);
       ok = __shfl_sync(0xffffffffu, w, 0) != 0;
     }
     const int tile = u / g.nk, kc = u - tile * g.nk, row0 = tile * 32;
@@ -618,7 +625,7 @@ __device__ __forceinline__ bool run_units(const Params& p, Smem& s, const Range&
     if (ok) {
       const uint8_t* st = s.ring + (size_t)slot * Gm::kStageBytes;
       const uint8_t* szs = st + (Gm::kCodeSlabs + Gm::kHiSlabs) * kSlab;
-      for (int gl = warp; gl < gc; gl += kCW) {
+      for (int gl = hw; gl < gc; gl += kHalf) {
         const int gg = g0 + gl;
         const uint32_t szw = sz_word(szs, lane, gl);
         const float s16 = __half2float(__ushort_as_half((unsigned short)(szw & 0xffffu)));
@@ -630,19 +637,19 @@ __device__ __forceinline__ bool run_units(const Params& p, Smem& s, const Range&
       }
     }
     float* red = s.red + (size_t)slot * kCW * 32;
-    red[warp * 32 + lane] = zacc;
+    red[hw * 32 + lane] = zacc;
     __syncwarp();
     int last = 0;
     if (lane == 0) {
       __threadfence_block();
-      last = atomicAdd(&s.ucnt[slot], 1) == kCW - 1;
+      last = atomicAdd(&s.ucnt[slot], 1) == kHalf - 1;
     }
     last = __shfl_sync(0xffffffffu, last, 0);
     if (last) {
       __threadfence_block();
       float t = 0.f;
 #pragma unroll
-      for (int w = 0; w < kCW; ++w) t += red[w * 32 + lane];
+      for (int w = 0; w < kHalf; ++w) t += red[w * 32 + lane];
       if (ok && row0 + lane < n_out) g.zp[(int64_t)kc * n_out + row0 + lane] = t;
       __syncwarp();
       if (lane == 0) s.ucnt[slot] = 0;
@@ -650,6 +657,7 @@ __device__ __forceinline__ bool run_units(const Params& p, Smem& s, const Range&
     __syncwarp();
     if (lane == 0) mbar_arrive(&s.empty[slot]);
   }
+  kring += (uint32_t)nu;
   return cbar_and(ok);
 }
 
@@ -699,7 +707,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   if (tid == 0) {
     for (int i = 0; i < p.ring_stages; ++i) {
       mbar_init(&s.full[i], 1);
-      mbar_init(&s.empty[i], kCW);
+      mbar_init(&s.empty[i], kHalf);  // the 8 warps of the half that consumed the unit
       s.ucnt[i] = 0;
     }
     mbar_init(s.tab_full, 1);
