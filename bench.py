@@ -69,9 +69,9 @@ def algorithmic_bytes_per_step(n_layers, batch=BATCH, bits=BITS):
 
 # DRAM bytes (read + write) of one fused decode launch per transformer block, from the
 # ncu capture summarised in profiles/decode_kernel_llama2-7b_2bit_batch1.md (4-block
-# case, 271.64 MB per launch, scaled by blocks), and a hash of the kernel's sources at
+# case, 271.18 MB per launch, scaled by blocks), and a hash of the kernel's sources at
 # capture time: the figure is reported only while those sources are unchanged.
-TRAFFIC_PER_BLOCK = {"bytes": 271_644_160 // 4, "sources_sha256_16": "53b216f27efb691e"}
+TRAFFIC_PER_BLOCK = {"bytes": 271_180_032 // 4, "sources_sha256_16": "a6dd0b2573c588ba"}
 KERNEL_SOURCES = ("decode.cu", "decode.h", "common.cuh", "gemv_core.cuh")
 
 
