@@ -61,6 +61,7 @@ def lib():
         L.ora_f16_to_f64.argtypes = [ctypes.c_uint16]
         L.ora_f16_to_f64.restype = ctypes.c_double
         L.ora_set_threads.argtypes = [_int]
+        L.ora_calib_error.argtypes = [_i64, _i64, _int, _int, _i64, _i64, _dp, _i8p, _dp, _i8p, _dp, _dp, _dp]
         L.ora_get_threads.restype = _int
         _lib = L
     return _lib
@@ -242,3 +243,16 @@ def stack_step(layers, hidden, ffn, n_heads, n_kv_heads, head_dim, x, eps=1e-5):
     _check(lib().ora_stack_step(len(layers) // 7, arr, hidden, ffn, n_heads, n_kv_heads, head_dim,
                                 float(eps), x2.shape[0], _d(x2), _d(out)), "stack")
     return out.reshape(-1) if one else out
+
+
+def calib_error(W, bits, w_in, w_out, thV, sV, thU, sU, h=None, group=64):
+    """Calibration forward: L = sum_rj h_j (W - U^T deq(Q(U W V^T)) V)_rj^2 (h None: 1)."""
+    W = _f64(W)
+    n_out, n_in = W.shape
+    thV, thU, sV, sU = _f64(thV), _f64(thU), _i8(sV), _i8(sU)
+    hh = _f64(h) if h is not None else None
+    out = ctypes.c_double()
+    _check(lib().ora_calib_error(n_out, n_in, int(bits), int(group), int(w_in), int(w_out), _d(thV),
+                                 sV.ctypes.data_as(_i8p), _d(thU), sU.ctypes.data_as(_i8p), _d(W),
+                                 _d(hh) if hh is not None else None, ctypes.byref(out)), "calib_error")
+    return out.value

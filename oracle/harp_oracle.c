@@ -413,3 +413,75 @@ done:
   free(h); free(nrm); free(q); free(k); free(v); free(a); free(o); free(g); free(u);
   return rc;
 }
+
+/* ------------------------------------------------------------------ calibration forward
+ * The reconstruction error that a calibration of the angles reduces (the page's
+ * adaptation of each layer's rotation to its quantizer, Sec. 2.2 and 3): rotate,
+ * quantize and dequantize in the rotated coordinates, rotate back, and weigh the error
+ * of every input column by h_j (the diagonal of a Hessian proxy X^T X; h NULL: all 1):
+ *   W' = U W V^T,   W^ = U^T deq(Q(W')) V,   L = sum_{r,j} h_j (W_rj - W^_rj)^2.
+ * W^ is formed by undoing the rotation's two passes: every column through F_U (= U^T),
+ * every row through F_V^T. The sum runs row by row in index order.
+ */
+int ora_calib_error(int64_t n_out, int64_t n_in, int bits, int group, int64_t w_in, int64_t w_out,
+                    const double* thV, const int8_t* sV, const double* thU, const int8_t* sU,
+                    const double* W, const double* h, double* out) {
+  if (bits < 2 || bits > 4 || group < 1 || n_in % group) return ORA_EINVAL;
+  const size_t nw = (size_t)n_out * (size_t)n_in;
+  const int64_t ng = n_in / group;
+  double* Wd = (double*)malloc(sizeof(double) * nw);
+  uint8_t* q = (uint8_t*)malloc(nw);
+  uint16_t* s16 = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)n_out * (size_t)ng);
+  uint16_t* z16 = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)n_out * (size_t)ng);
+  double* rowsum = (double*)malloc(sizeof(double) * (size_t)n_out);
+  int rc = ORA_OK;
+  if (!Wd || !q || !s16 || !z16 || !rowsum) { rc = ORA_EINVAL; goto done; }
+  memcpy(Wd, W, sizeof(double) * nw);
+  if ((rc = ora_rotate_weights(n_out, n_in, w_in, w_out, thV, sV, thU, sU, Wd))) goto done;
+  if ((rc = ora_quantize(n_out, n_in, bits, group, Wd, q, s16, z16))) goto done;
+  for (int64_t r = 0; r < n_out; ++r)
+    for (int64_t j = 0; j < n_in; ++j) {
+      const int64_t g = r * ng + j / group;
+      Wd[r * n_in + j] = ora_f16_to_f64(s16[g]) * (double)q[r * n_in + j] + ora_f16_to_f64(z16[g]);
+    }
+  /* columns through F_U = U^T */
+  {
+    int bad = 0;
+#pragma omp parallel
+    {
+      double* col = (double*)malloc(sizeof(double) * (size_t)n_out);
+      if (!col) {
+#pragma omp atomic write
+        bad = 1;
+      } else {
+#pragma omp for schedule(static)
+        for (int64_t j = 0; j < n_in; ++j) {
+          for (int64_t r = 0; r < n_out; ++r) col[r] = Wd[r * n_in + j];
+          ora_butterfly_fwd(n_out, w_out, 1, thU, sU, col);
+          for (int64_t r = 0; r < n_out; ++r) Wd[r * n_in + j] = col[r];
+        }
+        free(col);
+      }
+    }
+    if (bad) { rc = ORA_EINVAL; goto done; }
+  }
+  /* rows through F_V^T */
+  if ((rc = ora_butterfly_inv(n_in, w_in, n_out, thV, sV, Wd))) goto done;
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < n_out; ++r) {
+    double acc = 0.0;
+    for (int64_t j = 0; j < n_in; ++j) {
+      const double d = W[r * n_in + j] - Wd[r * n_in + j];
+      acc += (h ? h[j] : 1.0) * d * d;
+    }
+    rowsum[r] = acc;
+  }
+  {
+    double tot = 0.0;
+    for (int64_t r = 0; r < n_out; ++r) tot += rowsum[r];
+    *out = tot;
+  }
+done:
+  free(Wd); free(q); free(s16); free(z16); free(rowsum);
+  return rc;
+}

@@ -428,3 +428,55 @@ def test_stack_glue_closed_form(ora):
     want[21] += Md[21, 70] * m70
     assert np.max(np.abs(got[0] - want)) < 1e-13
     assert o9 != 0 and m10 != 0 and m70 != 0  # the case exercises every branch
+
+
+# ------------------------------------------------------------------ calibration forward
+def _calib_case(seed, n_out=128, n_in=256, w_in=128, w_out=64, bits=2):
+    rng = np.random.default_rng(seed)
+    W = rng.standard_normal((n_out, n_in)) * 0.02
+    W[:, 7] *= 20.0  # an outlier input column, as in the workloads
+    thV, thU = _rand_theta(rng, n_in, w_in, 0.05), _rand_theta(rng, n_out, w_out, 0.05)
+    sV, sU = _rand_sign(rng, n_in), _rand_sign(rng, n_out)
+    return W, bits, w_in, w_out, thV, sV, thU, sU
+
+
+def test_calib_error_unweighted_is_the_rotated_quantization_error(ora):
+    """The butterflies are orthogonal, so with h = 1 the error in the original coordinates
+    equals the quantization error of W' itself: sum (W' - deq(Q(W')))^2, formed here from
+    rotate_weights and quantize without any inverse rotation."""
+    W, bits, w_in, w_out, thV, sV, thU, sU = _calib_case(1)
+    Wr = ora.rotate_weights(W, thV, sV, w_in, thU, sU, w_out)
+    q, s16, z16 = ora.quantize(Wr, bits)
+    s = np.repeat(s16.view(np.float16).astype(np.float64), 64, axis=1)
+    z = np.repeat(z16.view(np.float16).astype(np.float64), 64, axis=1)
+    want = float(np.sum((Wr - (s * q + z)) ** 2))
+    got = ora.calib_error(W, bits, w_in, w_out, thV, sV, thU, sU)
+    assert abs(got - want) <= 1e-10 * want
+
+
+def test_calib_error_single_column_matches_the_linear(ora):
+    """h = e_j keeps only column j: W^ e_j is the dequantized layer applied to e_j, which
+    linear_fwd computes on its own path (F_U(deq . F_V(x)) with codes unpacked on the fly)."""
+    W, bits, w_in, w_out, thV, sV, thU, sU = _calib_case(2)
+    lay = ora.prepare_layer(W, bits, w_in, w_out, thV, sV, thU, sU)[0]
+    for j in (0, 7, 200):
+        e = np.zeros(W.shape[1])
+        e[j] = 1.0
+        col = ora.linear_fwd(lay, e)
+        want = float(np.sum((W[:, j] - col) ** 2))
+        got = ora.calib_error(W, bits, w_in, w_out, thV, sV, thU, sU, h=e)
+        assert abs(got - want) <= 1e-10 * max(want, 1e-30)
+
+
+def test_calib_error_weights_and_degenerate_cases(ora):
+    """Linear and nonnegative in h; zero for W = 0 (every group constant, exact); more
+    bits reduce the error."""
+    W, bits, w_in, w_out, thV, sV, thU, sU = _calib_case(3)
+    rng = np.random.default_rng(4)
+    h = rng.uniform(0.1, 5.0, W.shape[1])
+    L1 = ora.calib_error(W, bits, w_in, w_out, thV, sV, thU, sU, h=h)
+    L3 = ora.calib_error(W, bits, w_in, w_out, thV, sV, thU, sU, h=3.0 * h)
+    assert L1 > 0 and abs(L3 - 3.0 * L1) <= 1e-10 * L3
+    assert ora.calib_error(np.zeros_like(W), bits, w_in, w_out, thV, sV, thU, sU) == 0.0
+    errs = [ora.calib_error(W, b, w_in, w_out, thV, sV, thU, sU) for b in (2, 3, 4)]
+    assert errs[0] > errs[1] > errs[2]
