@@ -100,6 +100,34 @@ harp_status harp_butterfly_inv(int64_t n, int w, int batch, const float* theta, 
 harp_status harp_quantize_weights(int64_t n_out, int64_t n_in, int bits, int group,
                                   const float* W_rot, void* codes, void* scale_zero, void* stream);
 
+/* ---------------------------------------------------------------- calibration
+ * The reconstruction error that adapting the rotations reduces (HARP page, Sec. 2.2 and
+ * Sec. 3: the angles of each layer are fitted to its quantizer):
+ *   W' = U W V^T,  W^ = U^T deq(Q(W')) V,  *err = sum_{r,j} h_j (W_rj - W^_rj)^2
+ * with U = F(theta_U, sign_U, w_out)^T and V = F(theta_V, sign_V, w_in), Q and deq the
+ * quantizer above (codes and their fp16 scale and zero, exactly as the linear uses them).
+ *   n_out, n_in : n_in % 256 == 0, n_out % 32 == 0, each < 65536 (each side is the other
+ *                 side's butterfly batch).
+ *   bits, group : {2, 3, 4}, 64.    w_in, w_out: butterfly widths dividing n_in, n_out.
+ *   W           : device fp32 [n_out][n_in], row-major, not modified.
+ *   theta_V/U   : device fp32 [log2 w][n/2] or NULL (Theta = 0); sign_V/U device int8 [n].
+ *   h           : device fp32 [n_in] per-input-column weights (e.g. the diagonal of the
+ *                 calibration inputs' second moment), or NULL for all ones.
+ *   err         : device fp64 scalar, written on `stream` (8-byte aligned).
+ *   workspace   : device, 256-byte aligned, >= harp_calib_workspace_size bytes
+ *                 (2 fp32 copies of W plus the codes); overwritten.
+ * Rotations run in fp32 on the library's butterfly kernels; the squared differences and
+ * their sum are fp64, summed in a fixed order (the result is reproducible run to run).
+ * Pointers must be 16-byte aligned. Errors: HARP_ERR_INVALID_ARG for sizes, widths,
+ * null or misaligned pointers; HARP_ERR_WORKSPACE; HARP_ERR_CUDA on a launch failure.
+ */
+harp_status harp_calib_workspace_size(int64_t n_out, int64_t n_in, int bits, size_t* bytes);
+
+harp_status harp_calib_error(int64_t n_out, int64_t n_in, int bits, int group, int w_in, int w_out,
+                             const float* W, const float* theta_V, const int8_t* sign_V,
+                             const float* theta_U, const int8_t* sign_U, const float* h, double* err,
+                             void* workspace, size_t ws_bytes, void* stream);
+
 /* ---------------------------------------------------------------- layer
  * Creates a layer handle.
  *   n_in, n_out : multiples of 64, each <= 65536.

@@ -19,7 +19,7 @@ import math
 from ._lib import (HARP_BF16, HARP_F16, HARP_F32, HarpError, call, load)  # noqa: F401
 
 __all__ = ["HarpError", "harp_butterfly_fwd", "harp_butterfly_inv", "harp_quantize_weights", "HarpLayer",
-           "HarpStack", "rotate_weights_device", "harp_device_status", "load"]
+           "HarpStack", "rotate_weights_device", "harp_calib_error", "harp_device_status", "load"]
 
 
 def _torch():
@@ -98,6 +98,25 @@ def rotate_weights_device(W, theta_V, sign_V, w_in, theta_U, sign_U, w_out):
     Wt = Wr.t().contiguous()
     harp_butterfly_inv(Wt, theta_U, sign_U, w_out, out=Wt)
     return Wt.t().contiguous()
+
+
+def harp_calib_error(W, bits, w_in, w_out, theta_V, sign_V, theta_U, sign_U, h=None, group=64, out=None):
+    """Calibration forward: sum_rj h_j (W - U^T deq(Q(U W V^T)) V)_rj^2 as a device fp64
+    scalar tensor (h None: all ones). theta None: that side is Theta = 0."""
+    torch = _torch()
+    _need_cuda(W, theta_V, sign_V, theta_U, sign_U, h)
+    W = W.float().contiguous()
+    n_out, n_in = W.shape
+    n = ctypes.c_size_t()
+    call("harp_calib_workspace_size", n_out, n_in, int(bits), ctypes.byref(n))
+    ws = torch.empty(n.value, dtype=torch.uint8, device=W.device)
+    if out is None:
+        out = torch.empty((), dtype=torch.float64, device=W.device)
+    hh = h.float().contiguous() if h is not None else None
+    call("harp_calib_error", n_out, n_in, int(bits), int(group), int(w_in), int(w_out), _p(W), _p(_contig(theta_V)),
+         _p(sign_V.contiguous()), _p(_contig(theta_U)), _p(sign_U.contiguous()), _p(hh), _p(out), _p(ws),
+         ws.numel(), _stream())
+    return out
 
 
 class HarpLayer:

@@ -128,3 +128,34 @@ def test_empty_batch_is_a_no_op(lib):
     """batch 0 is valid for the butterflies and returns before any launch."""
     assert lib.harp_butterfly_fwd(4096, 4096, 0, FAKE, FAKE, FAKE, 0, FAKE, 0, None) == 0
     assert lib.harp_butterfly_inv(4096, 4096, 0, None, FAKE, FAKE, 0, FAKE, 0, None) == 0
+
+
+def test_calib_workspace_size(lib):
+    """Two fp32 copies of W, the packed codes, scale/zero words and one fp64 per row."""
+    n = ctypes.c_size_t()
+    assert lib.harp_calib_workspace_size(4096, 4096, 2, ctypes.byref(n)) == 0
+    assert n.value == 2 * 4 * 4096 * 4096 + 4096 * 4096 * 2 // 8 + 4096 * 64 * 4 + 8 * 4096
+    assert lib.harp_calib_workspace_size(4096, 4096, 5, ctypes.byref(n)) == 1
+    assert lib.harp_calib_workspace_size(4096, 4096, 2, None) == 1
+
+
+@pytest.mark.parametrize("n_out,n_in,bits,group,w_in,w_out,ws,err", [
+    (4096, 4096, 2, 64, 4096, 4096, 1 << 20, 4),    # workspace too small
+    (4096, 4096, 2, 32, 4096, 4096, 1 << 40, 2),    # unsupported group
+    (4096, 4000, 2, 64, 4096, 4096, 1 << 40, 1),    # n_in not a multiple of 256
+    (4000, 4096, 2, 64, 4096, 4096, 1 << 40, 1),    # n_out not a multiple of 32
+    (65536, 4096, 2, 64, 4096, 4096, 1 << 40, 1),   # n_out is a butterfly batch: < 65536
+    (4096, 4096, 2, 64, 3000, 4096, 1 << 40, 1),    # w_in not a power of two
+    (4096, 11008, 2, 64, 4096, 4096, 1 << 40, 1),   # w_in does not divide n_in
+])
+def test_calib_rejects_bad_arguments(lib, n_out, n_in, bits, group, w_in, w_out, ws, err):
+    st = lib.harp_calib_error(n_out, n_in, bits, group, w_in, w_out, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE,
+                              FAKE, ws, None)
+    assert st == err, lib.harp_last_error()
+
+
+def test_calib_rejects_misaligned_pointers(lib):
+    assert lib.harp_calib_error(4096, 4096, 2, 64, 4096, 4096, MIS, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE,
+                                1 << 40, None) == 1
+    assert lib.harp_calib_error(4096, 4096, 2, 64, 4096, 4096, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, FAKE,
+                                1 << 40, None) == 1
