@@ -61,7 +61,8 @@ def lib():
         L.ora_f16_to_f64.argtypes = [ctypes.c_uint16]
         L.ora_f16_to_f64.restype = ctypes.c_double
         L.ora_set_threads.argtypes = [_int]
-        L.ora_calib_error.argtypes = [_i64, _i64, _int, _int, _i64, _i64, _dp, _i8p, _dp, _i8p, _dp, _dp, _dp]
+        L.ora_calib_fit.argtypes = [_i64, _i64, _int, _int, _i64, _i64, _dp, _i8p, _dp, _i8p, _dp, _dp,
+                                    ctypes.c_double, _dp, _dp, _dp]
         L.ora_get_threads.restype = _int
         _lib = L
     return _lib
@@ -245,14 +246,22 @@ def stack_step(layers, hidden, ffn, n_heads, n_kv_heads, head_dim, x, eps=1e-5):
     return out.reshape(-1) if one else out
 
 
-def calib_error(W, bits, w_in, w_out, thV, sV, thU, sU, h=None, group=64):
-    """Calibration forward: L = sum_rj h_j (W - U^T deq(Q(U W V^T)) V)_rj^2 (h None: 1)."""
+def calib_fit(W, bits, w_in, w_out, thV, sV, thU, sU, H=None, lambda_bd=0.0, grad=False, group=64):
+    """The page's per-layer fitting loss L_fit = L_diag + lambda_bd R_bd (HARP Sec. 2.3).
+
+    H: the input-side Hessian proxy [n_in, n_in] (None: identity). Returns
+    (L_fit, L_diag, R_bd), and with grad=True also (dL_fit/dtheta_V, dL_fit/dtheta_U)
+    with the code target held constant."""
     W = _f64(W)
     n_out, n_in = W.shape
     thV, thU, sV, sU = _f64(thV), _f64(thU), _i8(sV), _i8(sU)
-    hh = _f64(h) if h is not None else None
-    out = ctypes.c_double()
-    _check(lib().ora_calib_error(n_out, n_in, int(bits), int(group), int(w_in), int(w_out), _d(thV),
-                                 sV.ctypes.data_as(_i8p), _d(thU), sU.ctypes.data_as(_i8p), _d(W),
-                                 _d(hh) if hh is not None else None, ctypes.byref(out)), "calib_error")
-    return out.value
+    HH = _f64(H) if H is not None else None
+    out = np.zeros(3)
+    gV = np.zeros_like(thV) if grad else None
+    gU = np.zeros_like(thU) if grad else None
+    _check(lib().ora_calib_fit(n_out, n_in, int(bits), int(group), int(w_in), int(w_out), _d(thV),
+                               sV.ctypes.data_as(_i8p), _d(thU), sU.ctypes.data_as(_i8p), _d(W),
+                               _d(HH) if HH is not None else None, float(lambda_bd), _d(out),
+                               _d(gV) if grad else None, _d(gU) if grad else None), "calib_fit")
+    loss = (float(out[0]), float(out[1]), float(out[2]))
+    return (loss, gV, gU) if grad else loss

@@ -414,74 +414,219 @@ done:
   return rc;
 }
 
-/* ------------------------------------------------------------------ calibration forward
- * The reconstruction error that a calibration of the angles reduces (the page's
- * adaptation of each layer's rotation to its quantizer, Sec. 2.2 and 3): rotate,
- * quantize and dequantize in the rotated coordinates, rotate back, and weigh the error
- * of every input column by h_j (the diagonal of a Hessian proxy X^T X; h NULL: all 1):
- *   W' = U W V^T,   W^ = U^T deq(Q(W')) V,   L = sum_{r,j} h_j (W_rj - W^_rj)^2.
- * W^ is formed by undoing the rotation's two passes: every column through F_U (= U^T),
- * every row through F_V^T. The sum runs row by row in index order.
+/* ------------------------------------------------------------------ calibration objective
+ * The per-layer fitting loss of the HARP page, Sec. 2.3 (Objetivo de Otimizacao):
+ *   L_fit(Theta) = L_diag(Theta) + lambda_bd * R_bd(Theta_V).
+ * H is the input-side Hessian proxy [n_in][n_in] (symmetric; NULL: the identity). In the
+ * rotated coordinates the layer sees inputs V x, so its proxy there is H' = V H V^T.
+ *   L_diag = sum_{r,j} d_j (W'_rj - T_rj)^2,   d = diag(H'),
+ *            W' = U W V^T and T = deq(Q(W')) its blockwise code target;
+ *   R_bd   = sum of H'_ij^2 over i, j in different quantizer groups (floor(i / group)).
+ * The gradient treats T as a constant (the page stops gradients through the discrete
+ * code assignment) and is taken with respect to the angle offsets theta of both
+ * butterflies, through W' (U and V), d (V) and R_bd (V).
+ *
+ * Backward through one 2x2 block: the stage maps (a, b) to (u, v) = (c a + s b, s a - c b)
+ * with c = cos p, s = sin p, p = pi/4 + theta. Its derivative in p is (-v, u), so
+ * dL/dtheta = g_v u - g_u v from the block's outputs and their gradients alone, and
+ * since the block is its own inverse, (a, b) and (g_a, g_b) are the block applied to
+ * (u, v) and (g_u, g_v).
  */
-int ora_calib_error(int64_t n_out, int64_t n_in, int bits, int group, int64_t w_in, int64_t w_out,
-                    const double* thV, const int8_t* sV, const double* thU, const int8_t* sU,
-                    const double* W, const double* h, double* out) {
+typedef struct {
+  int64_t n, w;
+  int m;
+  double* c; /* [m][n/2] cos(pi/4 + theta), then sin */
+  double* s;
+} ora_tab;
+
+static int ora_tab_make(ora_tab* T, int64_t n, int64_t w, const double* theta) {
+  T->n = n;
+  T->w = w;
+  T->m = ora_check_bfly(n, w);
+  T->c = T->s = NULL;
+  if (T->m < 1) return ORA_EINVAL;
+  const size_t k = (size_t)T->m * (size_t)(n / 2);
+  T->c = (double*)malloc(sizeof(double) * k);
+  T->s = (double*)malloc(sizeof(double) * k);
+  if (!T->c || !T->s) return ORA_EINVAL;
+  for (size_t i = 0; i < k; ++i) {
+    const double psi = ORA_PI / 4.0 + theta[i];
+    T->c[i] = cos(psi);
+    T->s[i] = sin(psi);
+  }
+  return ORA_OK;
+}
+
+static void ora_tab_free(ora_tab* T) { free(T->c); free(T->s); }
+
+/* One stage t of one w-wide block k, run backwards on a row: y holds the stage's
+ * outputs and becomes its inputs, g likewise for the gradients; dth gets the angle
+ * gradients of the stage's pairs. */
+static void ora_stage_back(const ora_tab* T, int t, int64_t k, double* y, double* g, double* dth) {
+  const int64_t h = (int64_t)1 << t, w = T->w;
+  for (int64_t i = k * w; i < (k + 1) * w; ++i) {
+    const int64_t il = i - k * w;
+    if (il & h) continue;
+    const int64_t p = (int64_t)t * (T->n / 2) + k * (w / 2) + ((il >> (t + 1)) << t) + (il & (h - 1));
+    const double c = T->c[p], s = T->s[p];
+    const double u = y[i], v = y[i + h], gu = g[i], gv = g[i + h];
+    dth[p] += gv * u - gu * v;
+    y[i] = c * u + s * v;
+    y[i + h] = s * u - c * v;
+    g[i] = c * gu + s * gv;
+    g[i + h] = s * gu - c * gv;
+  }
+}
+
+/* Backward of `batch` rows that went through F (inverse = 0) or F^T (inverse = 1):
+ * y: the rows' outputs, replaced by their inputs; g: dL/dy, replaced by dL/dx;
+ * dth [m][n/2] += dL/dtheta. Blocks are independent (disjoint pairs) and run in
+ * parallel; rows run in index order, so every angle's sum has one fixed order. */
+static void ora_bfly_back(const ora_tab* T, int64_t batch, const int8_t* sign, int inverse, double* y, double* g,
+                          double* dth) {
+  const int64_t n = T->n, nb = n / T->w;
+#pragma omp parallel for schedule(static)
+  for (int64_t k = 0; k < nb; ++k) {
+    for (int64_t r = 0; r < batch; ++r) {
+      double* yr = y + r * n;
+      double* gr = g + r * n;
+      if (inverse) { /* F^T = D S_0 ... S_{m-1}: undo D, then S_0 first */
+        for (int64_t i = k * T->w; i < (k + 1) * T->w; ++i) { yr[i] *= (double)sign[i]; gr[i] *= (double)sign[i]; }
+        for (int t = 0; t < T->m; ++t) ora_stage_back(T, t, k, yr, gr, dth);
+      } else { /* F = S_{m-1} ... S_0 D: S_{m-1} first, then D */
+        for (int t = T->m - 1; t >= 0; --t) ora_stage_back(T, t, k, yr, gr, dth);
+        for (int64_t i = k * T->w; i < (k + 1) * T->w; ++i) { yr[i] *= (double)sign[i]; gr[i] *= (double)sign[i]; }
+      }
+    }
+  }
+}
+
+static void ora_transpose(int64_t R, int64_t C, const double* in, double* out) {
+#pragma omp parallel for schedule(static)
+  for (int64_t c = 0; c < C; ++c)
+    for (int64_t r = 0; r < R; ++r) out[c * R + r] = in[r * C + c];
+}
+
+/* out[0] = L_fit, out[1] = L_diag, out[2] = R_bd. gV [log2 w_in][n_in/2] and
+ * gU [log2 w_out][n_out/2] receive dL_fit/dtheta when non-NULL. */
+int ora_calib_fit(int64_t n_out, int64_t n_in, int bits, int group, int64_t w_in, int64_t w_out,
+                  const double* thV, const int8_t* sV, const double* thU, const int8_t* sU, const double* W,
+                  const double* H, double lambda_bd, double* out, double* gV, double* gU) {
   if (bits < 2 || bits > 4 || group < 1 || n_in % group) return ORA_EINVAL;
-  const size_t nw = (size_t)n_out * (size_t)n_in;
+  const int mi = ora_check_bfly(n_in, w_in), mo = ora_check_bfly(n_out, w_out);
+  if (mi < 1 || mo < 1) return ORA_EINVAL;
+  const size_t nw = (size_t)n_out * (size_t)n_in, nh = (size_t)n_in * (size_t)n_in;
   const int64_t ng = n_in / group;
-  double* Wd = (double*)malloc(sizeof(double) * nw);
-  uint8_t* q = (uint8_t*)malloc(nw);
-  uint16_t* s16 = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)n_out * (size_t)ng);
-  uint16_t* z16 = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)n_out * (size_t)ng);
-  double* rowsum = (double*)malloc(sizeof(double) * (size_t)n_out);
+  const int grad = gV || gU;
+  double *Wr = NULL, *E = NULL, *A = NULL, *Hp = NULL, *Hq = NULL, *K = NULL, *d = NULL, *e = NULL, *row = NULL;
+  uint8_t* q = NULL;
+  uint16_t *s16 = NULL, *z16 = NULL;
+  ora_tab TV = {0}, TU = {0};
   int rc = ORA_OK;
-  if (!Wd || !q || !s16 || !z16 || !rowsum) { rc = ORA_EINVAL; goto done; }
-  memcpy(Wd, W, sizeof(double) * nw);
-  if ((rc = ora_rotate_weights(n_out, n_in, w_in, w_out, thV, sV, thU, sU, Wd))) goto done;
-  if ((rc = ora_quantize(n_out, n_in, bits, group, Wd, q, s16, z16))) goto done;
+  Wr = (double*)malloc(sizeof(double) * nw);
+  E = (double*)malloc(sizeof(double) * nw);
+  q = (uint8_t*)malloc(nw);
+  s16 = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)n_out * (size_t)ng);
+  z16 = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)n_out * (size_t)ng);
+  d = (double*)malloc(sizeof(double) * (size_t)n_in);
+  e = (double*)malloc(sizeof(double) * (size_t)n_in);
+  row = (double*)malloc(sizeof(double) * (size_t)n_out);
+  if (!Wr || !E || !q || !s16 || !z16 || !d || !e || !row) { rc = ORA_EINVAL; goto done; }
+
+  /* W', its code target T and the residual E = W' - T */
+  memcpy(Wr, W, sizeof(double) * nw);
+  if ((rc = ora_rotate_weights(n_out, n_in, w_in, w_out, thV, sV, thU, sU, Wr))) goto done;
+  if ((rc = ora_quantize(n_out, n_in, bits, group, Wr, q, s16, z16))) goto done;
   for (int64_t r = 0; r < n_out; ++r)
     for (int64_t j = 0; j < n_in; ++j) {
       const int64_t g = r * ng + j / group;
-      Wd[r * n_in + j] = ora_f16_to_f64(s16[g]) * (double)q[r * n_in + j] + ora_f16_to_f64(z16[g]);
+      E[r * n_in + j] = Wr[r * n_in + j] - (ora_f16_to_f64(s16[g]) * (double)q[r * n_in + j] + ora_f16_to_f64(z16[g]));
     }
-  /* columns through F_U = U^T */
+
+  /* H' = V H V^T: rows of H through F_V give B = H V^T; rows of B^T through F_V give H' */
+  if (H) {
+    Hp = (double*)malloc(sizeof(double) * nh);
+    Hq = (double*)malloc(sizeof(double) * nh);
+    if (!Hp || !Hq) { rc = ORA_EINVAL; goto done; }
+    memcpy(Hp, H, sizeof(double) * nh);
+    if ((rc = ora_butterfly_fwd(n_in, w_in, n_in, thV, sV, Hp))) goto done;
+    ora_transpose(n_in, n_in, Hp, Hq);
+    if ((rc = ora_butterfly_fwd(n_in, w_in, n_in, thV, sV, Hq))) goto done;
+    for (int64_t j = 0; j < n_in; ++j) d[j] = Hq[j * n_in + j];
+  } else {
+    for (int64_t j = 0; j < n_in; ++j) d[j] = 1.0;
+  }
+
+  /* the loss, summed row by row in index order */
   {
-    int bad = 0;
-#pragma omp parallel
-    {
-      double* col = (double*)malloc(sizeof(double) * (size_t)n_out);
-      if (!col) {
-#pragma omp atomic write
-        bad = 1;
-      } else {
-#pragma omp for schedule(static)
-        for (int64_t j = 0; j < n_in; ++j) {
-          for (int64_t r = 0; r < n_out; ++r) col[r] = Wd[r * n_in + j];
-          ora_butterfly_fwd(n_out, w_out, 1, thU, sU, col);
-          for (int64_t r = 0; r < n_out; ++r) Wd[r * n_in + j] = col[r];
-        }
-        free(col);
+    double Ld = 0.0, Rb = 0.0;
+    for (int64_t r = 0; r < n_out; ++r) {
+      double acc = 0.0;
+      for (int64_t j = 0; j < n_in; ++j) acc += d[j] * E[r * n_in + j] * E[r * n_in + j];
+      Ld += acc;
+    }
+    if (H)
+      for (int64_t i = 0; i < n_in; ++i) {
+        double acc = 0.0;
+        for (int64_t j = 0; j < n_in; ++j)
+          if (i / group != j / group) acc += Hq[i * n_in + j] * Hq[i * n_in + j];
+        Rb += acc;
       }
-    }
-    if (bad) { rc = ORA_EINVAL; goto done; }
+    out[0] = Ld + lambda_bd * Rb;
+    out[1] = Ld;
+    out[2] = Rb;
   }
-  /* rows through F_V^T */
-  if ((rc = ora_butterfly_inv(n_in, w_in, n_out, thV, sV, Wd))) goto done;
-#pragma omp parallel for schedule(static)
-  for (int64_t r = 0; r < n_out; ++r) {
+  if (!grad) goto done;
+
+  if ((rc = ora_tab_make(&TV, n_in, w_in, thV)) || (rc = ora_tab_make(&TU, n_out, w_out, thU))) goto done;
+  double* dV = (double*)calloc((size_t)mi * (size_t)(n_in / 2), sizeof(double));
+  double* dU = (double*)calloc((size_t)mo * (size_t)(n_out / 2), sizeof(double));
+  A = (double*)malloc(sizeof(double) * nw);
+  if (!dV || !dU || !A) { free(dV); free(dU); rc = ORA_EINVAL; goto done; }
+
+  /* dL_diag/dW' = 2 d_j E_rj (T constant); e_j = sum_r E_rj^2 = dL_diag/dd_j */
+  for (int64_t j = 0; j < n_in; ++j) {
     double acc = 0.0;
-    for (int64_t j = 0; j < n_in; ++j) {
-      const double d = W[r * n_in + j] - Wd[r * n_in + j];
-      acc += (h ? h[j] : 1.0) * d * d;
-    }
-    rowsum[r] = acc;
+    for (int64_t r = 0; r < n_out; ++r) acc += E[r * n_in + j] * E[r * n_in + j];
+    e[j] = acc;
   }
-  {
-    double tot = 0.0;
-    for (int64_t r = 0; r < n_out; ++r) tot += rowsum[r];
-    *out = tot;
+  for (int64_t r = 0; r < n_out; ++r)
+    for (int64_t j = 0; j < n_in; ++j) E[r * n_in + j] *= 2.0 * d[j];
+
+  /* columns: W'_{:,j} = F_U^T A_{:,j}; back through it, one column at a time */
+  for (int64_t j = 0; j < n_in; ++j) {
+    double* gcol = A; /* scratch: the column's gradient, then written back into E */
+    for (int64_t r = 0; r < n_out; ++r) { row[r] = Wr[r * n_in + j]; gcol[r] = E[r * n_in + j]; }
+    ora_bfly_back(&TU, 1, sU, 1, row, gcol, dU);
+    for (int64_t r = 0; r < n_out; ++r) E[r * n_in + j] = gcol[r];
   }
+  /* rows: A_r = F_V W_r (recomputed), back through F_V with dL/dA in E */
+  memcpy(A, W, sizeof(double) * nw);
+  if ((rc = ora_butterfly_fwd(n_in, w_in, n_out, thV, sV, A))) { free(dV); free(dU); goto done; }
+  ora_bfly_back(&TV, n_out, sV, 0, A, E, dV);
+
+  if (H) {
+    /* dL/dH' = 2 lambda_bd H' (off-group entries) + diag(e) */
+    K = (double*)malloc(sizeof(double) * nh);
+    if (!K) { free(dV); free(dU); rc = ORA_EINVAL; goto done; }
+    for (int64_t i = 0; i < n_in; ++i)
+      for (int64_t j = 0; j < n_in; ++j)
+        K[i * n_in + j] = (i / group != j / group ? 2.0 * lambda_bd * Hq[i * n_in + j] : 0.0) + (i == j ? e[i] : 0.0);
+    /* second pass: rows of H' came from rows of B^T; Hq becomes B^T, K its gradient */
+    ora_bfly_back(&TV, n_in, sV, 0, Hq, K, dV);
+    /* first pass: rows of B came from rows of H */
+    ora_transpose(n_in, n_in, Hq, Hp);
+    ora_transpose(n_in, n_in, K, Hq);
+    ora_bfly_back(&TV, n_in, sV, 0, Hp, Hq, dV);
+  }
+  if (gV) memcpy(gV, dV, sizeof(double) * (size_t)mi * (size_t)(n_in / 2));
+  if (gU) memcpy(gU, dU, sizeof(double) * (size_t)mo * (size_t)(n_out / 2));
+  free(dV);
+  free(dU);
 done:
-  free(Wd); free(q); free(s16); free(z16); free(rowsum);
+  free(Wr); free(E); free(A); free(Hp); free(Hq); free(K); free(d); free(e); free(row);
+  free(q); free(s16); free(z16);
+  ora_tab_free(&TV);
+  ora_tab_free(&TU);
   return rc;
 }

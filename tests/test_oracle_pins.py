@@ -430,7 +430,7 @@ def test_stack_glue_closed_form(ora):
     assert o9 != 0 and m10 != 0 and m70 != 0  # the case exercises every branch
 
 
-# ------------------------------------------------------------------ calibration forward
+# ------------------------------------------------------------------ calibration objective
 def _calib_case(seed, n_out=128, n_in=256, w_in=128, w_out=64, bits=2):
     rng = np.random.default_rng(seed)
     W = rng.standard_normal((n_out, n_in)) * 0.02
@@ -440,43 +440,126 @@ def _calib_case(seed, n_out=128, n_in=256, w_in=128, w_out=64, bits=2):
     return W, bits, w_in, w_out, thV, sV, thU, sU
 
 
-def test_calib_error_unweighted_is_the_rotated_quantization_error(ora):
-    """The butterflies are orthogonal, so with h = 1 the error in the original coordinates
-    equals the quantization error of W' itself: sum (W' - deq(Q(W')))^2, formed here from
-    rotate_weights and quantize without any inverse rotation."""
+def _spd(rng, n):
+    """A Hessian proxy X^T X / N of heavy-tailed activations with two outlier channels."""
+    X = rng.standard_t(4, size=(3 * n, n))
+    X[:, 3] *= 8.0
+    X[:, n - 5] *= 5.0
+    return X.T @ X / X.shape[0]
+
+
+def _off_group(M, group=64):
+    n = M.shape[0]
+    blk = np.arange(n) // group
+    return float(np.sum(np.where(blk[:, None] != blk[None, :], M * M, 0.0)))
+
+
+def test_calib_identity_hessian_is_the_rotated_quantization_error(ora):
+    """H = I: d = 1 and R_bd = 0, so L_diag is the quantization error of W' itself,
+    formed here from rotate_weights and quantize."""
     W, bits, w_in, w_out, thV, sV, thU, sU = _calib_case(1)
     Wr = ora.rotate_weights(W, thV, sV, w_in, thU, sU, w_out)
     q, s16, z16 = ora.quantize(Wr, bits)
     s = np.repeat(s16.view(np.float16).astype(np.float64), 64, axis=1)
     z = np.repeat(z16.view(np.float16).astype(np.float64), 64, axis=1)
     want = float(np.sum((Wr - (s * q + z)) ** 2))
-    got = ora.calib_error(W, bits, w_in, w_out, thV, sV, thU, sU)
-    assert abs(got - want) <= 1e-10 * want
+    Lf, Ld, Rb = ora.calib_fit(W, bits, w_in, w_out, thV, sV, thU, sU, lambda_bd=7.0)
+    assert abs(Ld - want) <= 1e-10 * want and Rb == 0.0 and Lf == Ld
+    Lf2, Ld2, Rb2 = ora.calib_fit(W, bits, w_in, w_out, thV, sV, thU, sU, H=np.eye(W.shape[1]), lambda_bd=7.0)
+    assert abs(Ld2 - want) <= 1e-10 * want and Rb2 < 1e-24
 
 
-def test_calib_error_single_column_matches_the_linear(ora):
-    """h = e_j keeps only column j: W^ e_j is the dequantized layer applied to e_j, which
-    linear_fwd computes on its own path (F_U(deq . F_V(x)) with codes unpacked on the fly)."""
+def test_calib_identity_hessian_matches_the_linear(ora):
+    """The butterflies are orthogonal, so with H = I L_diag is also ||W - W^||_F^2 with W^
+    the dequantized layer: its columns are linear_fwd of the unit vectors, on the linear's
+    own path (F_U(deq . F_V(x)), codes unpacked on the fly)."""
     W, bits, w_in, w_out, thV, sV, thU, sU = _calib_case(2)
     lay = ora.prepare_layer(W, bits, w_in, w_out, thV, sV, thU, sU)[0]
-    for j in (0, 7, 200):
-        e = np.zeros(W.shape[1])
-        e[j] = 1.0
-        col = ora.linear_fwd(lay, e)
-        want = float(np.sum((W[:, j] - col) ** 2))
-        got = ora.calib_error(W, bits, w_in, w_out, thV, sV, thU, sU, h=e)
-        assert abs(got - want) <= 1e-10 * max(want, 1e-30)
+    What = ora.linear_fwd(lay, np.eye(W.shape[1])).T
+    want = float(np.sum((W - What) ** 2))
+    got = ora.calib_fit(W, bits, w_in, w_out, thV, sV, thU, sU)[1]
+    assert abs(got - want) <= 1e-9 * want
 
 
-def test_calib_error_weights_and_degenerate_cases(ora):
-    """Linear and nonnegative in h; zero for W = 0 (every group constant, exact); more
-    bits reduce the error."""
-    W, bits, w_in, w_out, thV, sV, thU, sU = _calib_case(3)
-    rng = np.random.default_rng(4)
-    h = rng.uniform(0.1, 5.0, W.shape[1])
-    L1 = ora.calib_error(W, bits, w_in, w_out, thV, sV, thU, sU, h=h)
-    L3 = ora.calib_error(W, bits, w_in, w_out, thV, sV, thU, sU, h=3.0 * h)
-    assert L1 > 0 and abs(L3 - 3.0 * L1) <= 1e-10 * L3
-    assert ora.calib_error(np.zeros_like(W), bits, w_in, w_out, thV, sV, thU, sU) == 0.0
-    errs = [ora.calib_error(W, b, w_in, w_out, thV, sV, thU, sU) for b in (2, 3, 4)]
+def test_calib_diagonal_weight_under_the_hadamard_transform(ora):
+    """Theta_V = 0 and w_in = n_in make V a signed Sylvester Hadamard matrix / sqrt(n), all
+    of whose entries square to 1/n: for H = diag(a), every d_j = mean(a), so L_diag is
+    mean(a) times the unweighted error."""
+    W, bits, _, w_out, _, sV, thU, sU = _calib_case(3)
+    n_in = W.shape[1]
+    zero = np.zeros((int(np.log2(n_in)), n_in // 2))
+    a = np.random.default_rng(5).uniform(0.1, 9.0, n_in)
+    L1 = ora.calib_fit(W, bits, n_in, w_out, zero, sV, thU, sU)[1]
+    La = ora.calib_fit(W, bits, n_in, w_out, zero, sV, thU, sU, H=np.diag(a))[1]
+    assert abs(La - a.mean() * L1) <= 1e-10 * La
+
+
+def test_calib_block_penalty_invariants(ora):
+    """R_bd(c I) = 0 for any rotation (V V^T = I); R_bd is quadratic and L_diag linear in H;
+    with butterfly blocks inside the 64-column groups (w_in = 32) V mixes only within a
+    group, so R_bd equals the off-group energy of H itself."""
+    rng = np.random.default_rng(6)
+    W, bits, w_in, w_out, thV, sV, thU, sU = _calib_case(4)
+    n_in = W.shape[1]
+    H = _spd(rng, n_in)
+    assert ora.calib_fit(W, bits, w_in, w_out, thV, sV, thU, sU, H=3.0 * np.eye(n_in))[2] < 1e-20
+    _, Ld1, Rb1 = ora.calib_fit(W, bits, w_in, w_out, thV, sV, thU, sU, H=H)
+    _, Ld2, Rb2 = ora.calib_fit(W, bits, w_in, w_out, thV, sV, thU, sU, H=2.0 * H)
+    assert Rb1 > 0 and abs(Rb2 - 4.0 * Rb1) <= 1e-10 * Rb2 and abs(Ld2 - 2.0 * Ld1) <= 1e-10 * Ld2
+    th32 = _rand_theta(rng, n_in, 32, 0.3)
+    Rb = ora.calib_fit(W, bits, 32, w_out, th32, sV, thU, sU, H=H)[2]
+    want = _off_group(H)
+    assert abs(Rb - want) <= 1e-10 * want
+    # and a 128-wide V does move energy across groups
+    assert abs(Rb1 - want) > 1e-3 * want
+
+
+@pytest.mark.parametrize("theta_scale", [0.0, 0.05])
+def test_calib_gradient_matches_finite_differences(ora, theta_scale):
+    """dL_fit/dtheta against central differences of the loss with the code target frozen,
+    written densely here: V, U as matrices (butterflies of the unit vectors),
+    W' = U W V^T, H' = V H V^T, L = sum d_j (W' - T)^2 + lambda sum_off H'^2. Checked along
+    random directions and on single angles of both butterflies, at the Hadamard start
+    (Theta = 0) and away from it."""
+    rng = np.random.default_rng(7)
+    n_out, n_in, w_in, w_out, bits, lam = 64, 256, 128, 32, 2, 0.3  # V blocks span two groups
+    W = rng.standard_normal((n_out, n_in)) * 0.02
+    W[:, 9] *= 15.0
+    thV = _rand_theta(rng, n_in, w_in, theta_scale)
+    thU = _rand_theta(rng, n_out, w_out, theta_scale)
+    sV, sU = _rand_sign(rng, n_in), _rand_sign(rng, n_out)
+    H = _spd(rng, n_in)
+    (Lf, Ld, Rb), gV, gU = ora.calib_fit(W, bits, w_in, w_out, thV, sV, thU, sU, H=H, lambda_bd=lam, grad=True)
+    Wr = ora.rotate_weights(W, thV, sV, w_in, thU, sU, w_out)
+    q, s16, z16 = ora.quantize(Wr, bits)
+    T = np.repeat(s16.view(np.float16).astype(np.float64), 64, axis=1) * q + \
+        np.repeat(z16.view(np.float16).astype(np.float64), 64, axis=1)
+
+    def loss(tV, tU):
+        V = _dense(ora, n_in, w_in, tV, sV)
+        U = _dense(ora, n_out, w_out, tU, sU).T
+        Wp = U @ W @ V.T
+        Hp = V @ H @ V.T
+        return float(np.sum(np.diag(Hp)[None, :] * (Wp - T) ** 2)) + lam * _off_group(Hp)
+
+    assert abs(loss(thV, thU) - Lf) <= 1e-10 * Lf
+    eps = 1e-5
+    for k in range(3):
+        dV, dU = rng.standard_normal(thV.shape), rng.standard_normal(thU.shape)
+        fd = (loss(thV + eps * dV, thU + eps * dU) - loss(thV - eps * dV, thU - eps * dU)) / (2 * eps)
+        an = float(np.sum(gV * dV) + np.sum(gU * dU))
+        assert abs(fd - an) <= 1e-6 * max(abs(an), 1e-3), (k, fd, an)
+    for (side, t, p) in [("V", 0, 3), ("V", 5, 40), ("U", 0, 1), ("U", 4, 17)]:
+        dV, dU = np.zeros_like(thV), np.zeros_like(thU)
+        (dV if side == "V" else dU)[t, p] = 1.0
+        fd = (loss(thV + eps * dV, thU + eps * dU) - loss(thV - eps * dV, thU - eps * dU)) / (2 * eps)
+        an = float((gV if side == "V" else gU)[t, p])
+        assert abs(fd - an) <= 1e-6 * max(abs(an), 1e-2), (side, t, p, fd, an)
+
+
+def test_calib_degenerate_cases(ora):
+    """Zero for W = 0 with H = I (every group constant, exact); more bits reduce L_diag."""
+    W, bits, w_in, w_out, thV, sV, thU, sU = _calib_case(8)
+    assert ora.calib_fit(np.zeros_like(W), bits, w_in, w_out, thV, sV, thU, sU) == (0.0, 0.0, 0.0)
+    errs = [ora.calib_fit(W, b, w_in, w_out, thV, sV, thU, sU)[1] for b in (2, 3, 4)]
     assert errs[0] > errs[1] > errs[2]
