@@ -101,32 +101,47 @@ harp_status harp_quantize_weights(int64_t n_out, int64_t n_in, int bits, int gro
                                   const float* W_rot, void* codes, void* scale_zero, void* stream);
 
 /* ---------------------------------------------------------------- calibration
- * The reconstruction error that adapting the rotations reduces (HARP page, Sec. 2.2 and
- * Sec. 3: the angles of each layer are fitted to its quantizer):
- *   W' = U W V^T,  W^ = U^T deq(Q(W')) V,  *err = sum_{r,j} h_j (W_rj - W^_rj)^2
- * with U = F(theta_U, sign_U, w_out)^T and V = F(theta_V, sign_V, w_in), Q and deq the
- * quantizer above (codes and their fp16 scale and zero, exactly as the linear uses them).
+ * The per-layer fitting loss that calibration minimises over the angles (HARP page,
+ * Sec. 2.3, Objetivo de Otimizacao), and its gradient:
+ *   W' = U W V^T,  T = deq(Q(W')),  H' = V H V^T,  d = diag(H')
+ *   L_diag = sum_{r,j} d_j (W'_rj - T_rj)^2
+ *   R_bd   = sum of H'_ij^2 over i, j in different 64-column quantizer groups
+ *   L_fit  = L_diag + lambda_bd * R_bd
+ * Here V = F(theta_V, sign_V, w_in) and U = F(theta_U, sign_U, w_out)^T. Q and deq are the
+ * quantizer above: the codes and their fp16 scale and zero, exactly as the linear stores
+ * them. The gradient holds T constant (no gradient through the code assignment).
  *   n_out, n_in : n_in % 256 == 0, n_out % 32 == 0, each < 65536 (each side is the other
  *                 side's butterfly batch).
  *   bits, group : {2, 3, 4}, 64.    w_in, w_out: butterfly widths dividing n_in, n_out.
  *   W           : device fp32 [n_out][n_in], row-major, not modified.
- *   theta_V/U   : device fp32 [log2 w][n/2] or NULL (Theta = 0); sign_V/U device int8 [n].
- *   h           : device fp32 [n_in] per-input-column weights (e.g. the diagonal of the
- *                 calibration inputs' second moment), or NULL for all ones.
- *   err         : device fp64 scalar, written on `stream` (8-byte aligned).
- *   workspace   : device, 256-byte aligned, >= harp_calib_workspace_size bytes
- *                 (2 fp32 copies of W plus the codes); overwritten.
- * Rotations run in fp32 on the library's butterfly kernels; the squared differences and
- * their sum are fp64, summed in a fixed order (the result is reproducible run to run).
- * Pointers must be 16-byte aligned. Errors: HARP_ERR_INVALID_ARG for sizes, widths,
- * null or misaligned pointers; HARP_ERR_WORKSPACE; HARP_ERR_CUDA on a launch failure.
+ *   theta_V/U   : device fp32 [log2 w][n/2] angle offsets, or NULL for Theta = 0.
+ *   sign_V/U    : device int8 [n].
+ *   H           : device fp32 [n_in][n_in] symmetric Hessian proxy of the layer's inputs
+ *                 (e.g. X^T X / N), or NULL for the identity (then d = 1 and R_bd = 0).
+ *   lambda_bd   : >= 0.
+ *   loss        : device fp64 [3] = {L_fit, L_diag, R_bd}, written on `stream`.
+ *   grad_theta_V/U : device fp32, shaped like theta, receive dL_fit/dtheta; NULL skips
+ *                 that side (both NULL: no backward pass). A NULL theta still gets its
+ *                 gradient at Theta = 0, where calibration starts.
+ *   workspace   : device, 256-byte aligned, at least harp_calib_workspace_size bytes for
+ *                 the same sizes, with_hessian = (H != NULL) and with_grad; overwritten.
+ *                 Roughly 3 fp32 copies of W, plus 3 of H when H is given.
+ * Rotations and the backward stages run in fp32. Sums of squares and the angle-gradient
+ * sums are fp64 and run in a fixed order, so a call repeats its results exactly.
+ * Pointers must be 16-byte aligned (loss 8).
+ * Errors:
+ *   HARP_ERR_INVALID_ARG for sizes, widths, a negative lambda, null or misaligned pointers;
+ *   HARP_ERR_WORKSPACE;
+ *   HARP_ERR_CUDA on a launch failure.
  */
-harp_status harp_calib_workspace_size(int64_t n_out, int64_t n_in, int bits, size_t* bytes);
+harp_status harp_calib_workspace_size(int64_t n_out, int64_t n_in, int bits, int w_in, int w_out,
+                                      int with_hessian, int with_grad, size_t* bytes);
 
-harp_status harp_calib_error(int64_t n_out, int64_t n_in, int bits, int group, int w_in, int w_out,
-                             const float* W, const float* theta_V, const int8_t* sign_V,
-                             const float* theta_U, const int8_t* sign_U, const float* h, double* err,
-                             void* workspace, size_t ws_bytes, void* stream);
+harp_status harp_calib_fit(int64_t n_out, int64_t n_in, int bits, int group, int w_in, int w_out,
+                           const float* W, const float* theta_V, const int8_t* sign_V,
+                           const float* theta_U, const int8_t* sign_U, const float* H, double lambda_bd,
+                           double* loss, float* grad_theta_V, float* grad_theta_U, void* workspace,
+                           size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------- layer
  * Creates a layer handle.

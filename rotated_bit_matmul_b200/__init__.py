@@ -19,7 +19,7 @@ import math
 from ._lib import (HARP_BF16, HARP_F16, HARP_F32, HarpError, call, load)  # noqa: F401
 
 __all__ = ["HarpError", "harp_butterfly_fwd", "harp_butterfly_inv", "harp_quantize_weights", "HarpLayer",
-           "HarpStack", "rotate_weights_device", "harp_calib_error", "harp_device_status", "load"]
+           "HarpStack", "rotate_weights_device", "harp_calib_fit", "harp_device_status", "load"]
 
 
 def _torch():
@@ -100,23 +100,29 @@ def rotate_weights_device(W, theta_V, sign_V, w_in, theta_U, sign_U, w_out):
     return Wt.t().contiguous()
 
 
-def harp_calib_error(W, bits, w_in, w_out, theta_V, sign_V, theta_U, sign_U, h=None, group=64, out=None):
-    """Calibration forward: sum_rj h_j (W - U^T deq(Q(U W V^T)) V)_rj^2 as a device fp64
-    scalar tensor (h None: all ones). theta None: that side is Theta = 0."""
+def harp_calib_fit(W, bits, w_in, w_out, theta_V, sign_V, theta_U, sign_U, H=None, lambda_bd=0.0, grad=False,
+                   group=64):
+    """The per-layer fitting loss L_fit = L_diag + lambda_bd R_bd (wraps harp_calib_fit).
+
+    Returns a device fp64 tensor [L_fit, L_diag, R_bd]; with grad=True also the fp32
+    gradients in theta_V and theta_U (shaped [log2 w, n/2]). theta None: Theta = 0.
+    H: the fp32 [n_in, n_in] input Hessian proxy, or None for the identity."""
     torch = _torch()
-    _need_cuda(W, theta_V, sign_V, theta_U, sign_U, h)
+    _need_cuda(W, theta_V, sign_V, theta_U, sign_U, H)
     W = W.float().contiguous()
     n_out, n_in = W.shape
+    Hc = H.float().contiguous() if H is not None else None
     n = ctypes.c_size_t()
-    call("harp_calib_workspace_size", n_out, n_in, int(bits), ctypes.byref(n))
+    call("harp_calib_workspace_size", n_out, n_in, int(bits), int(w_in), int(w_out), int(H is not None), int(grad),
+         ctypes.byref(n))
     ws = torch.empty(n.value, dtype=torch.uint8, device=W.device)
-    if out is None:
-        out = torch.empty((), dtype=torch.float64, device=W.device)
-    hh = h.float().contiguous() if h is not None else None
-    call("harp_calib_error", n_out, n_in, int(bits), int(group), int(w_in), int(w_out), _p(W), _p(_contig(theta_V)),
-         _p(sign_V.contiguous()), _p(_contig(theta_U)), _p(sign_U.contiguous()), _p(hh), _p(out), _p(ws),
-         ws.numel(), _stream())
-    return out
+    loss = torch.empty(3, dtype=torch.float64, device=W.device)
+    gV = torch.empty((log2i(w_in), n_in // 2), dtype=torch.float32, device=W.device) if grad else None
+    gU = torch.empty((log2i(w_out), n_out // 2), dtype=torch.float32, device=W.device) if grad else None
+    call("harp_calib_fit", n_out, n_in, int(bits), int(group), int(w_in), int(w_out), _p(W), _p(_contig(theta_V)),
+         _p(sign_V.contiguous()), _p(_contig(theta_U)), _p(sign_U.contiguous()), _p(Hc), float(lambda_bd), _p(loss),
+         _p(gV), _p(gU), _p(ws), ws.numel(), _stream())
+    return (loss, gV, gU) if grad else loss
 
 
 class HarpLayer:

@@ -7,13 +7,16 @@ sides of every parity test start from identical numbers.
 
 Seeds: ``numpy.random.default_rng([workload, layer, linear, role])``.
   workload: 1 single 1024x1024 layer, 2 the seven 7B decoder-layer linears,
-            3 the batch sweep, 4 the 32-layer 7B stack, 5 the 80-layer 70B stack.
+            3 the batch sweep, 4 the 32-layer 7B stack, 5 the 80-layer 70B stack,
+            11 the calibration-objective cases.
   linear:   0 q, 1 k, 2 v, 3 o, 4 gate, 5 up, 6 down, 7 = the step input.
-  role:     0 W, 1 outlier columns, 2 theta_V, 3 s_V, 4 theta_U, 5 s_U, 6 x.
+  role:     0 W, 1 outlier columns, 2 theta_V, 3 s_V, 4 theta_U, 5 s_U, 6 x,
+            7 calibration inputs.
 Weights ~ N(0, 0.02^2) with a seeded set of outlier input columns scaled by 20;
 theta ~ U(-0.05, 0.05) per pair and stage (the pi/4 Hadamard angle is added by
 the method, not here); signs are Rademacher; activations ~ N(0, 1), rounded to
-bf16 where the workload says bf16.
+bf16 where the workload says bf16. Calibration inputs (the samples a layer's Hessian
+proxy X^T X / N is formed from) are N(0, 1) with the layer's outlier channels x10.
 """
 from __future__ import annotations
 
@@ -21,7 +24,7 @@ from dataclasses import dataclass
 
 import numpy as np
 
-ROLE_W, ROLE_OUTLIER, ROLE_THETA_V, ROLE_SIGN_V, ROLE_THETA_U, ROLE_SIGN_U, ROLE_X = range(7)
+ROLE_W, ROLE_OUTLIER, ROLE_THETA_V, ROLE_SIGN_V, ROLE_THETA_U, ROLE_SIGN_U, ROLE_X, ROLE_CALIB_X = range(8)
 LINEAR_NAMES = ("q", "k", "v", "o", "gate", "up", "down")
 INPUT_SLOT = 7
 
@@ -87,6 +90,13 @@ def butterfly_params(n: int, w: int, workload: int, layer: int, linear: int, sid
     theta = rng(workload, layer, linear, rt).uniform(-0.05, 0.05, size=(m, n // 2)).astype(np.float32)
     sign = (rng(workload, layer, linear, rs).integers(0, 2, size=n, dtype=np.int8) * 2 - 1).astype(np.int8)
     return theta, sign
+
+
+def calibration_inputs(n_samples: int, n_in: int, workload: int, layer: int, linear: int) -> np.ndarray:
+    """fp32 [n_samples, n_in] layer inputs: N(0, 1) with the outlier channels scaled x10."""
+    X = rng(workload, layer, linear, ROLE_CALIB_X).standard_normal((n_samples, n_in), dtype=np.float32)
+    X[:, outlier_columns(n_in, workload, layer, linear)] *= np.float32(10.0)
+    return X
 
 
 def round_to_bf16(x: np.ndarray) -> np.ndarray:

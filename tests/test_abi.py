@@ -131,12 +131,25 @@ def test_empty_batch_is_a_no_op(lib):
 
 
 def test_calib_workspace_size(lib):
-    """Two fp32 copies of W, the packed codes, scale/zero words and one fp64 per row."""
+    """Without a Hessian proxy or gradient: two fp32 copies of W, the packed codes, the
+    scale/zero words and per-column fp32/fp64 vectors; each extra adds its buffers."""
     n = ctypes.c_size_t()
-    assert lib.harp_calib_workspace_size(4096, 4096, 2, ctypes.byref(n)) == 0
-    assert n.value == 2 * 4 * 4096 * 4096 + 4096 * 4096 * 2 // 8 + 4096 * 64 * 4 + 8 * 4096
-    assert lib.harp_calib_workspace_size(4096, 4096, 5, ctypes.byref(n)) == 1
-    assert lib.harp_calib_workspace_size(4096, 4096, 2, None) == 1
+    assert lib.harp_calib_workspace_size(4096, 4096, 2, 4096, 4096, 0, 0, ctypes.byref(n)) == 0
+    base = n.value
+    nw = 4096 * 4096
+    assert base >= 2 * 4 * nw + nw * 2 // 8 + 4096 * 64 * 4 and base < 2 * 4 * nw + nw // 4 + (8 << 20)
+    assert lib.harp_calib_workspace_size(4096, 4096, 2, 4096, 4096, 1, 0, ctypes.byref(n)) == 0
+    assert n.value - base == 2 * 4 * 4096 * 4096
+    assert lib.harp_calib_workspace_size(4096, 4096, 2, 4096, 4096, 1, 1, ctypes.byref(n)) == 0
+    assert n.value > base + 4 * 4 * nw
+    assert lib.harp_calib_workspace_size(4096, 4096, 5, 4096, 4096, 0, 0, ctypes.byref(n)) == 1
+    assert lib.harp_calib_workspace_size(4096, 4096, 2, 4096, 3000, 0, 0, ctypes.byref(n)) == 1
+    assert lib.harp_calib_workspace_size(4096, 4096, 2, 4096, 4096, 0, 0, None) == 1
+
+
+def _calib(lib, n_out, n_in, bits, group, w_in, w_out, W=FAKE, H=None, lam=0.0, loss=FAKE, ws=1 << 40):
+    return lib.harp_calib_fit(n_out, n_in, bits, group, w_in, w_out, W, FAKE, FAKE, FAKE, FAKE, H, lam, loss, None,
+                              None, FAKE, ws, None)
 
 
 @pytest.mark.parametrize("n_out,n_in,bits,group,w_in,w_out,ws,err", [
@@ -149,13 +162,12 @@ def test_calib_workspace_size(lib):
     (4096, 11008, 2, 64, 4096, 4096, 1 << 40, 1),   # w_in does not divide n_in
 ])
 def test_calib_rejects_bad_arguments(lib, n_out, n_in, bits, group, w_in, w_out, ws, err):
-    st = lib.harp_calib_error(n_out, n_in, bits, group, w_in, w_out, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE,
-                              FAKE, ws, None)
+    st = _calib(lib, n_out, n_in, bits, group, w_in, w_out, ws=ws)
     assert st == err, lib.harp_last_error()
 
 
-def test_calib_rejects_misaligned_pointers(lib):
-    assert lib.harp_calib_error(4096, 4096, 2, 64, 4096, 4096, MIS, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE,
-                                1 << 40, None) == 1
-    assert lib.harp_calib_error(4096, 4096, 2, 64, 4096, 4096, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, FAKE,
-                                1 << 40, None) == 1
+def test_calib_rejects_misaligned_pointers_and_negative_lambda(lib):
+    assert _calib(lib, 4096, 4096, 2, 64, 4096, 4096, W=MIS) == 1
+    assert _calib(lib, 4096, 4096, 2, 64, 4096, 4096, H=MIS) == 1
+    assert _calib(lib, 4096, 4096, 2, 64, 4096, 4096, loss=None) == 1
+    assert _calib(lib, 4096, 4096, 2, 64, 4096, 4096, lam=-1.0) == 1
