@@ -61,6 +61,7 @@ def lib():
         L.ora_f16_to_f64.argtypes = [ctypes.c_uint16]
         L.ora_f16_to_f64.restype = ctypes.c_double
         L.ora_set_threads.argtypes = [_int]
+        L.ora_quantize_angles.argtypes = [_i64, _i64, _dp, _i8p, ctypes.POINTER(ctypes.c_float)]
         L.ora_calib_fit.argtypes = [_i64, _i64, _int, _int, _i64, _i64, _dp, _i8p, _dp, _i8p, _dp, _dp,
                                     ctypes.c_double, _dp, _dp, _dp]
         L.ora_get_threads.restype = _int
@@ -244,6 +245,23 @@ def stack_step(layers, hidden, ffn, n_heads, n_kv_heads, head_dim, x, eps=1e-5):
     _check(lib().ora_stack_step(len(layers) // 7, arr, hidden, ffn, n_heads, n_kv_heads, head_dim,
                                 float(eps), x2.shape[0], _d(x2), _d(out)), "stack")
     return out.reshape(-1) if one else out
+
+
+def quantize_angles(theta):
+    """int8 angle storage: (q int8 [m, n/2], delta fp32 [m]) with one symmetric step per
+    stage, delta_t = fp32(max |theta_t| / 127), q = RNE(theta / delta_t) clamped to +-127."""
+    th = _f64(theta)
+    m, half = th.shape
+    q = np.zeros((m, half), np.int8)
+    d = np.zeros(m, np.float32)
+    _check(lib().ora_quantize_angles(m, half, _d(th), q.ctypes.data_as(_i8p),
+                                     d.ctypes.data_as(ctypes.POINTER(ctypes.c_float))), "quantize_angles")
+    return q, d
+
+
+def dequantize_angles(q, delta):
+    """theta^ = delta_t * q_tp in fp64 (the angles a layer stored in int8 applies)."""
+    return np.asarray(delta, np.float64)[:, None] * np.asarray(q, np.float64)
 
 
 def calib_fit(W, bits, w_in, w_out, thV, sV, thU, sU, H=None, lambda_bd=0.0, grad=False, group=64):

@@ -414,6 +414,33 @@ done:
   return rc;
 }
 
+/* ------------------------------------------------------------------ int8 angles
+ * The HARP page stores its parameters in int8 (Sec. 2.4, Armazenamento; Sec. 4, 2.00 ->
+ * 2.05 bits per parameter at 2 bits). The format is this library's reading:
+ * every stage t of a butterfly has one symmetric step, and the angle offsets become
+ *   delta_t = fp32(max_p |theta_tp| / 127),
+ *   q_tp    = clamp(round_half_even(theta_tp / delta_t), -127, 127)   (0 when delta_t = 0),
+ *   theta^  = delta_t * q_tp.
+ * A layer stored this way is the layer built from theta^: W' is rotated with theta^.
+ */
+int ora_quantize_angles(int64_t m, int64_t half, const double* theta, int8_t* q, float* delta) {
+  if (m < 1 || half < 1) return ORA_EINVAL;
+  for (int64_t t = 0; t < m; ++t) {
+    const double* th = theta + t * half;
+    double mx = 0.0;
+    for (int64_t p = 0; p < half; ++p) mx = fabs(th[p]) > mx ? fabs(th[p]) : mx;
+    const float d = (float)(mx / 127.0);
+    delta[t] = d;
+    for (int64_t p = 0; p < half; ++p) {
+      double v = d > 0.0f ? rint(th[p] / (double)d) : 0.0;
+      if (v > 127.0) v = 127.0;
+      if (v < -127.0) v = -127.0;
+      q[t * half + p] = (int8_t)v;
+    }
+  }
+  return ORA_OK;
+}
+
 /* ------------------------------------------------------------------ calibration objective
  * The per-layer fitting loss of the HARP page, Sec. 2.3 (Objetivo de Otimizacao):
  *   L_fit(Theta) = L_diag(Theta) + lambda_bd * R_bd(Theta_V).

@@ -563,3 +563,52 @@ def test_calib_degenerate_cases(ora):
     assert ora.calib_fit(np.zeros_like(W), bits, w_in, w_out, thV, sV, thU, sU) == (0.0, 0.0, 0.0)
     errs = [ora.calib_fit(W, b, w_in, w_out, thV, sV, thU, sU)[1] for b in (2, 3, 4)]
     assert errs[0] > errs[1] > errs[2]
+
+
+# ------------------------------------------------------------------ int8 angles
+def test_angle_q8_hand_example(ora):
+    """Hand-computed: stage 0 has max |theta| = 0.127, so delta = fp32(0.001), and
+    0.127 -> 127, -0.0636 -> -63.6 -> -64, 0.001 -> 0.99999995 -> 1, 0 -> 0. An all-zero
+    stage has delta 0 and codes 0."""
+    th = np.array([[0.127, -0.0636, 0.001, 0.0], [0.0, 0.0, 0.0, 0.0]])
+    q, d = ora.quantize_angles(th)
+    assert q.tolist() == [[127, -64, 1, 0], [0, 0, 0, 0]]
+    assert d[0] == np.float32(0.001) and d[1] == 0.0
+
+
+def test_angle_q8_is_the_nearest_code(ora):
+    """Brute force over all 255 codes of each stage's step: the chosen code is the nearest
+    (ties to even), so |theta^ - theta| <= delta / 2, and the largest angle of a stage
+    reaches +-127."""
+    rng = np.random.default_rng(21)
+    th = rng.uniform(-0.05, 0.05, (6, 96)) * rng.uniform(0.1, 3.0, (6, 1))
+    th[2, 5] = 0.0
+    th[3] = np.round(th[3] * 1e3) / 1e3  # many values on exact grid points
+    q, d = ora.quantize_angles(th)
+    codes = np.arange(-127, 128, dtype=np.float64)
+    for t in range(th.shape[0]):
+        dist = np.abs(th[t][:, None] - float(d[t]) * codes[None, :])
+        best = dist.min(axis=1)
+        mine = np.abs(th[t] - float(d[t]) * q[t])
+        assert np.all(mine <= best + 1e-18)
+        assert np.all(mine <= float(d[t]) / 2 * (1 + 1e-12))
+        assert np.abs(q[t]).max() == 127
+    assert np.array_equal(ora.dequantize_angles(q, d), d.astype(np.float64)[:, None] * q)
+
+
+def test_angle_q8_butterfly_error_bound(ora):
+    """Each 2x2 block moves by at most |d theta| in operator norm (its derivative in the
+    angle is orthogonal), so ||F(theta^) x - F(theta) x|| <= sum_t max_p |d theta_tp| ||x||,
+    and with the nearest code that is at most sum_t delta_t / 2."""
+    rng = np.random.default_rng(22)
+    n, w = 1024, 1024
+    th = _rand_theta(rng, n, w, 0.05)
+    s = _rand_sign(rng, n)
+    q, d = ora.quantize_angles(th)
+    thq = ora.dequantize_angles(q, d)
+    x = rng.standard_normal((4, n))
+    diff = np.linalg.norm(ora.butterfly_fwd(x, thq, s, w) - ora.butterfly_fwd(x, th, s, w), axis=1)
+    bound = np.abs(thq - th).max(axis=1).sum()
+    assert np.all(diff <= bound * np.linalg.norm(x, axis=1) * (1 + 1e-9))
+    assert bound <= d.astype(np.float64).sum() / 2 * (1 + 1e-12)
+    assert diff.max() > 0
