@@ -38,6 +38,9 @@ CONFIG_NAME = "llama2-7b-shaped 32-layer rotated 2-bit linear stack, batch-1 dec
 # with --rht every butterfly is the fixed randomized Hadamard transform (Theta = 0): the
 # baseline the HARP pages compare against (same codes budget, no learned angles)
 CONFIG_NAME_RHT = "llama2-7b-shaped 32-layer 2-bit linear stack with fixed randomized Hadamard rotations, batch-1 decode"
+# with --int8-angles every butterfly keeps its angles in int8 (one step per stage), as the
+# HARP pages' storage option; the layers are built from the dequantized angles
+CONFIG_NAME_Q8 = "llama2-7b-shaped 32-layer rotated 2-bit linear stack with int8 butterfly angles, batch-1 decode"
 
 
 def parse():
@@ -51,7 +54,12 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--rht", action="store_true",
                     help="fixed randomized Hadamard rotations (Theta = 0) instead of the learned-angle butterflies")
-    return ap.parse_args()
+    ap.add_argument("--int8-angles", action="store_true",
+                    help="learned angles stored in int8 with a per-stage step (decoded in the kernels)")
+    args = ap.parse_args()
+    if args.rht and args.int8_angles:
+        ap.error("--rht and --int8-angles exclude each other")
+    return args
 
 
 def shapes():
@@ -144,7 +152,7 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ CPU oracle sample
-def _oracle_block(sample_layers, rht=False):
+def _oracle_block(sample_layers, rht=False, q8=False):
     import oracle
     from rotated_bit_matmul_b200 import synth
     lays = []
@@ -155,11 +163,14 @@ def _oracle_block(sample_layers, rht=False):
             thU, sU = synth.butterfly_params(s.n_out, s.w_out, WORKLOAD, l, i, "U")
             if rht:
                 thV, thU = np.zeros_like(thV), np.zeros_like(thU)
+            if q8:
+                thV = oracle.dequantize_angles(*oracle.quantize_angles(thV))
+                thU = oracle.dequantize_angles(*oracle.quantize_angles(thU))
             lays.append(oracle.prepare_layer(W, BITS, s.w_in, s.w_out, thV, sV, thU, sU)[0])
     return lays
 
 
-def cpu_oracle_sample(sample_layers=1, min_seconds=10.0, steps=None, warmup=0, rht=False):
+def cpu_oracle_sample(sample_layers=1, min_seconds=10.0, steps=None, warmup=0, rht=False, q8=False):
     """Times the fp64 oracle on `sample_layers` blocks of the 7B stack for one token per
     pass and scales to the 32-block step. Without `steps` it repeats passes until
     `min_seconds` of CPU work have been timed; with `steps` it runs `warmup` untimed and
@@ -168,7 +179,7 @@ def cpu_oracle_sample(sample_layers=1, min_seconds=10.0, steps=None, warmup=0, r
     from rotated_bit_matmul_b200 import synth
     threads = len(os.sched_getaffinity(0))
     oracle.set_threads(threads)
-    lays = _oracle_block(sample_layers, rht)
+    lays = _oracle_block(sample_layers, rht, q8)
     for w in range(warmup):
         oracle.stack_step(lays, HIDDEN, FFN, NH, NKV, HD, synth.activations(BATCH, HIDDEN, WORKLOAD, step=w).astype(np.float64))
     passes, dt = 0, 0.0
@@ -183,7 +194,7 @@ def cpu_oracle_sample(sample_layers=1, min_seconds=10.0, steps=None, warmup=0, r
 
 
 # ------------------------------------------------------------------ GPU path
-def build_stack(n_layers, device, rht=False):
+def build_stack(n_layers, device, rht=False, q8=False):
     import torch
     import rotated_bit_matmul_b200 as rb
     from rotated_bit_matmul_b200 import synth
@@ -197,11 +208,19 @@ def build_stack(n_layers, device, rht=False):
             if rht:  # Theta = 0 on both sides: no angles reach the library
                 thV = thU = None
             sV, sU = torch.from_numpy(sV).to(device), torch.from_numpy(sU).to(device)
+            if q8:  # int8 angles; W is rotated with the angles they stand for
+                qV, dV = rb.harp_quantize_angles(thV)
+                qU, dU = rb.harp_quantize_angles(thU)
+                thV, thU = dV[:, None] * qV.float(), dU[:, None] * qU.float()
             Wr = rb.rotate_weights_device(W, thV, sV, s.w_in, thU, sU, s.w_out)
             del W
             codes, sz = rb.harp_quantize_weights(Wr, BITS, GROUP)
             del Wr
-            layers.append(rb.HarpLayer(s.n_in, s.n_out, BITS, s.w_in, s.w_out, thV, sV, thU, sU, codes, sz))
+            if q8:
+                layers.append(rb.HarpLayer.int8_angles(s.n_in, s.n_out, BITS, s.w_in, s.w_out, qV, dV, sV, qU, dU, sU,
+                                                       codes, sz))
+            else:
+                layers.append(rb.HarpLayer(s.n_in, s.n_out, BITS, s.w_in, s.w_out, thV, sV, thU, sU, codes, sz))
     torch.cuda.synchronize()
     return rb.HarpStack(layers, HIDDEN, FFN, NH, NKV, HD)
 
@@ -219,7 +238,7 @@ def run_ours(args, rk):
     from rotated_bit_matmul_b200 import replicas, synth
     device = torch.device("cuda", rk.local_rank)
     torch.cuda.set_device(device)
-    stack = build_stack(args.layers, device, args.rht)
+    stack = build_stack(args.layers, device, args.rht, args.int8_angles)
     K, Wm = args.steps, args.warmup
     xs = torch.stack([torch.from_numpy(synth.activations(BATCH, HIDDEN, WORKLOAD, step=s)).to(torch.bfloat16)
                       for s in range(K + Wm)]).to(device)
@@ -287,7 +306,7 @@ def run_ours(args, rk):
     achieved = nbytes / (ms_step * 1e-3) / 1e9
     fused = stack.uses_fused_step(BATCH)
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": traffic_per_step(args.layers) if fused and not args.rht else None,
+                "frac": round(achieved / peak, 4), "traffic": traffic_per_step(args.layers) if fused and not (args.rht or args.int8_angles) else None,
                 "kernel": "decode_kernel (one launch per step)" if fused else "whole decode step (graph of kernels)",
                 "peak_kind": peak_kind, "algorithmic_bytes_per_step": nbytes}
     del g
@@ -303,7 +322,8 @@ def main():
     replicas.init(rk, "gloo" if args.impl == "reference" else "nccl")
     world = rk.world
 
-    config = {"workload": CONFIG_NAME_RHT if args.rht else CONFIG_NAME, "layers": args.layers, "hidden": HIDDEN, "ffn": FFN, "bits": BITS,
+    workload = CONFIG_NAME_RHT if args.rht else (CONFIG_NAME_Q8 if args.int8_angles else CONFIG_NAME)
+    config = {"workload": workload, "layers": args.layers, "hidden": HIDDEN, "ffn": FFN, "bits": BITS,
               "group": GROUP, "batch": BATCH, "global_batch": BATCH * world, "parallelism": f"replicas{world}",
               "l2": "inputs larger than L2: each step streams ~2.03 GB of packed codes and scales (L2 126 MB)"}
     base = {"metric": METRIC, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -315,7 +335,8 @@ def main():
         # rank 0 alone times the oracle; the other ranks leave without work
         if rk.rank == 0:
             tps, per_block, threads, passes = cpu_oracle_sample(args.cpu_sample_layers, steps=args.steps,
-                                                                warmup=args.warmup, rht=args.rht)
+                                                                warmup=args.warmup, rht=args.rht,
+                                                                q8=args.int8_angles)
             ms = per_block * N_LAYERS * 1e3
             line = dict(base, impl="reference", value=tps, unit="tokens/s", ms_per_step=ms, dtype="f64",
                         cpu_baseline={"value": tps, "unit": "tokens/s", "cores": threads, "kind": "oracle",
@@ -329,7 +350,7 @@ def main():
     r = run_ours(args, rk)
     cpu = None
     if rk.rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tps, per_block, threads, passes = cpu_oracle_sample(args.cpu_sample_layers, rht=args.rht)
+        tps, per_block, threads, passes = cpu_oracle_sample(args.cpu_sample_layers, rht=args.rht, q8=args.int8_angles)
         cpu = {"value": tps, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                "sample": f"{passes} passes of {args.cpu_sample_layers} of {N_LAYERS} blocks of one decode token "
                          f"(about 10 s of CPU work), scaled to {N_LAYERS} blocks"}

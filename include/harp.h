@@ -100,6 +100,35 @@ harp_status harp_butterfly_inv(int64_t n, int w, int batch, const float* theta, 
 harp_status harp_quantize_weights(int64_t n_out, int64_t n_in, int bits, int group,
                                   const float* W_rot, void* codes, void* scale_zero, void* stream);
 
+/* ---------------------------------------------------------------- int8 angles
+ * The HARP page stores its parameters in int8 (Sec. 2.4, Armazenamento, and Sec. 4:
+ * 2.00 -> 2.05 bits per parameter at 2 bits); the format is this library's:
+ * one symmetric step per butterfly stage,
+ *   delta_t = fp32(max_p |theta_tp| / 127),
+ *   q_tp    = clamp(round_half_even(theta_tp / delta_t), -127, 127)   (0 when delta_t = 0),
+ * and the layer applies theta^ = delta_t * q_tp. The codes and steps are computed in fp64
+ * from the fp32 angles, so they equal those of an fp64 evaluation exactly.
+ *   m      : stages, 1..16.    half_n: pairs per stage (n/2).
+ *   theta  : device fp32 [m][half_n], finite.
+ *   q      : device int8 [m][half_n] (out).    delta: device fp32 [m] (out).
+ * All pointers 16-byte aligned. */
+harp_status harp_quantize_angles(int m, int64_t half_n, const float* theta, int8_t* q, float* delta,
+                                 void* stream);
+
+/* A layer whose butterflies keep their angles in int8: the same as harp_create_layer, with
+ * each side's theta replaced by (q [log2 w][n/2] int8, delta [log2 w] fp32) from
+ * harp_quantize_angles. The layer copies both (1 byte per angle plus a 64-byte head), and
+ * its kernels evaluate cos/sin of pi/4 + delta_t q as they rotate, instead of reading
+ * 8-byte (cos, sin) pairs. codes/scale_zero must come from W rotated with the dequantized
+ * angles theta^ (the exact change of basis holds for theta^, not theta). q NULL makes that
+ * side Theta = 0 (delta ignored). The fused decode step runs when every butterfly of a
+ * stack uses int8 angles, like when all use fp32 angles or all are Theta = 0. */
+harp_status harp_create_layer_q8(harp_layer* out, int64_t n_in, int64_t n_out, int bits, int group,
+                                 int w_in, int w_out, const int8_t* q_V, const float* delta_V,
+                                 const int8_t* sign_V, const int8_t* q_U, const float* delta_U,
+                                 const int8_t* sign_U, const void* codes, const void* scale_zero,
+                                 void* stream);
+
 /* ---------------------------------------------------------------- calibration
  * The per-layer fitting loss that calibration minimises over the angles (HARP page,
  * Sec. 2.3, Objetivo de Otimizacao), and its gradient:

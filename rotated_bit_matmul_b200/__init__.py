@@ -19,7 +19,7 @@ import math
 from ._lib import (HARP_BF16, HARP_F16, HARP_F32, HarpError, call, load)  # noqa: F401
 
 __all__ = ["HarpError", "harp_butterfly_fwd", "harp_butterfly_inv", "harp_quantize_weights", "HarpLayer",
-           "HarpStack", "rotate_weights_device", "harp_calib_fit", "harp_device_status", "load"]
+           "HarpStack", "rotate_weights_device", "harp_quantize_angles", "harp_calib_fit", "harp_device_status", "load"]
 
 
 def _torch():
@@ -91,6 +91,19 @@ def harp_quantize_weights(W_rot, bits: int, group: int = 64):
     return codes, sz
 
 
+def harp_quantize_angles(theta):
+    """int8 storage of a butterfly's angle offsets theta fp32 [m, n/2]: returns (q int8
+    [m, n/2], delta fp32 [m]) with delta_t = max |theta_t| / 127 and q = RNE(theta / delta_t)."""
+    torch = _torch()
+    _need_cuda(theta)
+    th = theta.float().contiguous()
+    m, half = th.shape
+    q = torch.empty((m, half), dtype=torch.int8, device=th.device)
+    d = torch.empty(max(m, 4), dtype=torch.float32, device=th.device)  # 16-byte allocation
+    call("harp_quantize_angles", int(m), int(half), _p(th), _p(q), _p(d), _stream())
+    return q, d[:m]
+
+
 def rotate_weights_device(W, theta_V, sign_V, w_in, theta_U, sign_U, w_out):
     """W' = U W V^T on the device: rows through F_V, then columns through F_U^T."""
     _need_cuda(W)
@@ -132,15 +145,35 @@ class HarpLayer:
     def __init__(self, n_in, n_out, bits, w_in, w_out, theta_V, sign_V, theta_U, sign_U, codes, scale_zero,
                  group=64):
         _need_cuda(theta_V, sign_V, theta_U, sign_U, codes, scale_zero)
-        self.n_in, self.n_out, self.bits, self.group = int(n_in), int(n_out), int(bits), int(group)
-        self.w_in, self.w_out = int(w_in), int(w_out)
-        # the library borrows codes and scale_zero: keep them alive with the handle
-        self.codes, self.scale_zero = codes, scale_zero
+        self._fields(n_in, n_out, bits, w_in, w_out, codes, scale_zero, group)
         h = ctypes.c_void_p()
         call("harp_create_layer", ctypes.byref(h), self.n_in, self.n_out, self.bits, self.group, self.w_in,
              self.w_out, _p(_contig(theta_V)), _p(sign_V.contiguous()), _p(_contig(theta_U)),
              _p(sign_U.contiguous()), _p(codes), _p(scale_zero), _stream())
         self.handle = h
+
+    @classmethod
+    def int8_angles(cls, n_in, n_out, bits, w_in, w_out, q_V, delta_V, sign_V, q_U, delta_U, sign_U, codes,
+                    scale_zero, group=64):
+        """A layer keeping its angles in int8 (wraps harp_create_layer_q8): q int8
+        [log2 w, n/2] and delta fp32 [log2 w] per side, as harp_quantize_angles returns
+        them; q None makes that side Theta = 0."""
+        _need_cuda(q_V, delta_V, sign_V, q_U, delta_U, sign_U, codes, scale_zero)
+        self = cls.__new__(cls)
+        self._fields(n_in, n_out, bits, w_in, w_out, codes, scale_zero, group)
+        h = ctypes.c_void_p()
+        call("harp_create_layer_q8", ctypes.byref(h), self.n_in, self.n_out, self.bits, self.group, self.w_in,
+             self.w_out, _p(_contig(q_V)), _p(_contig(delta_V)), _p(sign_V.contiguous()), _p(_contig(q_U)),
+             _p(_contig(delta_U)), _p(sign_U.contiguous()), _p(codes), _p(scale_zero), _stream())
+        self.handle = h
+        return self
+
+    def _fields(self, n_in, n_out, bits, w_in, w_out, codes, scale_zero, group):
+        self.handle = None
+        self.n_in, self.n_out, self.bits, self.group = int(n_in), int(n_out), int(bits), int(group)
+        self.w_in, self.w_out = int(w_in), int(w_out)
+        # the library borrows codes and scale_zero: keep them alive with the handle
+        self.codes, self.scale_zero = codes, scale_zero
         self._ws = {}
         self.device = codes.device
 

@@ -40,6 +40,9 @@ SIGNATURES = {
     "harp_stack_workspace_size": (_I, [_P, _I, ctypes.POINTER(_SZ)]),
     "harp_stack_step": (_I, [_P, _I, _P, _I, _P, _I, _P, _SZ, _P]),
     "harp_stack_uses_fused_step": (_I, [_P, _I]),
+    "harp_quantize_angles": (_I, [_I, _I64, _P, _P, _P, _P]),
+    "harp_create_layer_q8": (_I, [ctypes.POINTER(_P), _I64, _I64, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P,
+                                  _P]),
     "harp_calib_workspace_size": (_I, [_I64, _I64, _I, _I, _I, _I, _I, ctypes.POINTER(_SZ)]),
     "harp_calib_fit": (_I, [_I64, _I64, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, ctypes.c_double, _P, _P, _P, _P,
                             _SZ, _P]),

@@ -202,6 +202,7 @@ harp_status linear_forward_status(const Layer& L, int batch, const void* x, int 
   pv.m = L.m_in;
   pv.inverse = 0;
   pv.cs = L.csV;
+  pv.q8 = L.q8V;
   pv.sign = L.sV;
   pv.x = x;
   pv.xt = xt;
@@ -257,6 +258,7 @@ harp_status linear_forward_status(const Layer& L, int batch, const void* x, int 
   pu.m = L.m_out;
   pu.inverse = 0;
   pu.cs = L.csU;
+  pu.q8 = L.q8U;
   pu.sign = L.sU;
   pu.x = tc ? w.zpart : w.z;
   pu.xt = DT_F32;
@@ -327,9 +329,19 @@ harp_status harp_quantize_weights(int64_t n_out, int64_t n_in, int bits, int gro
   return HARP_OK;
 }
 
-harp_status harp_create_layer(harp_layer* out, int64_t n_in, int64_t n_out, int bits, int group, int w_in,
-                              int w_out, const float* theta_V, const int8_t* sign_V, const float* theta_U,
-                              const int8_t* sign_U, const void* codes, const void* scale_zero, void* stream) {
+namespace {
+
+// One side's angles: raw theta (cos/sin tables are built), int8 codes with their steps
+// (copied into the layer's int8 storage), or neither (Theta = 0).
+struct SideAngles {
+  const float* theta;
+  const int8_t* q8;
+  const float* delta;
+};
+
+harp_status create_layer_impl(harp_layer* out, int64_t n_in, int64_t n_out, int bits, int group, int w_in, int w_out,
+                              SideAngles av, const int8_t* sign_V, SideAngles au, const int8_t* sign_U,
+                              const void* codes, const void* scale_zero, void* stream) {
   if (!out) return fail(HARP_ERR_INVALID_ARG, "create_layer: null output handle");
   *out = nullptr;
   if (bits < 2 || bits > 4) return fail(HARP_ERR_INVALID_ARG, "create_layer: bits=%d not in {2,3,4}", bits);
@@ -344,8 +356,13 @@ harp_status harp_create_layer(harp_layer* out, int64_t n_in, int64_t n_out, int 
   if (m_out < 1 || w_out > kMaxW || n_out % w_out)
     return fail(HARP_ERR_INVALID_ARG, "create_layer: w_out=%d must be a power of two in [2, 8192] dividing n_out", w_out);
   if (!sign_V || !sign_U || !codes || !scale_zero) return fail(HARP_ERR_INVALID_ARG, "create_layer: null pointer");
+  const float* theta_V = av.theta;
+  const float* theta_U = au.theta;
+  if ((av.q8 && !av.delta) || (au.q8 && !au.delta))
+    return fail(HARP_ERR_INVALID_ARG, "create_layer_q8: int8 angles need their per-stage steps");
   if ((theta_V && !aligned16(theta_V)) || !aligned16(sign_V) || (theta_U && !aligned16(theta_U)) ||
-      !aligned16(sign_U) || !aligned16(codes) || !aligned16(scale_zero))
+      !aligned16(sign_U) || !aligned16(codes) || !aligned16(scale_zero) || (av.q8 && !aligned16(av.q8)) ||
+      (au.q8 && !aligned16(au.q8)) || (av.delta && !aligned16(av.delta)) || (au.delta && !aligned16(au.delta)))
     return fail(HARP_ERR_INVALID_ARG, "create_layer: device pointers must be 16-byte aligned");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   harp_layer_s* h = new (std::nothrow) harp_layer_s();
@@ -366,6 +383,8 @@ harp_status harp_create_layer(harp_layer* out, int64_t n_in, int64_t n_out, int 
   auto cleanup = [&](harp_status s) {
     cudaFree(L.csV);
     cudaFree(L.csU);
+    cudaFree(L.q8V);
+    cudaFree(L.q8U);
     cudaFree(L.sV);
     cudaFree(L.sU);
     delete h;
@@ -382,6 +401,17 @@ harp_status harp_create_layer(harp_layer* out, int64_t n_in, int64_t n_out, int 
       (e = cudaMemcpyAsync(L.sV, sign_V, (size_t)n_in, cudaMemcpyDeviceToDevice, st)) != cudaSuccess ||
       (e = cudaMemcpyAsync(L.sU, sign_U, (size_t)n_out, cudaMemcpyDeviceToDevice, st)) != cudaSuccess)
     return cleanup(cuda_fail(e, "create_layer: copies"));
+  // int8 angles: a zeroed 64-byte head with the m fp32 steps, then the codes
+  auto q8_side = [&](const SideAngles& a, int m, int64_t cnt, uint8_t** dst) -> cudaError_t {
+    if (!a.q8) return cudaSuccess;
+    cudaError_t r = cudaMalloc(dst, (size_t)kQ8Head + (size_t)cnt);
+    if (r == cudaSuccess) r = cudaMemsetAsync(*dst, 0, kQ8Head, st);
+    if (r == cudaSuccess) r = cudaMemcpyAsync(*dst, a.delta, sizeof(float) * (size_t)m, cudaMemcpyDeviceToDevice, st);
+    if (r == cudaSuccess) r = cudaMemcpyAsync(*dst + kQ8Head, a.q8, (size_t)cnt, cudaMemcpyDeviceToDevice, st);
+    return r;
+  };
+  if ((e = q8_side(av, m_in, cnt_v, &L.q8V)) != cudaSuccess || (e = q8_side(au, m_out, cnt_u, &L.q8U)) != cudaSuccess)
+    return cleanup(cuda_fail(e, "create_layer_q8: int8 angle storage"));
   const int pb = bits == 4 ? 4 : 2;  // bits of the (first) code plane
   harp_status s =
       make_tmap(&L.tm_codes, codes, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, (uint64_t)n_in * pb / 64, (uint64_t)n_out,
@@ -414,6 +444,34 @@ harp_status harp_create_layer(harp_layer* out, int64_t n_in, int64_t n_out, int 
   return HARP_OK;
 }
 
+}  // namespace
+
+harp_status harp_create_layer(harp_layer* out, int64_t n_in, int64_t n_out, int bits, int group, int w_in,
+                              int w_out, const float* theta_V, const int8_t* sign_V, const float* theta_U,
+                              const int8_t* sign_U, const void* codes, const void* scale_zero, void* stream) {
+  return create_layer_impl(out, n_in, n_out, bits, group, w_in, w_out, SideAngles{theta_V, nullptr, nullptr}, sign_V,
+                           SideAngles{theta_U, nullptr, nullptr}, sign_U, codes, scale_zero, stream);
+}
+
+harp_status harp_create_layer_q8(harp_layer* out, int64_t n_in, int64_t n_out, int bits, int group, int w_in,
+                                 int w_out, const int8_t* q_V, const float* delta_V, const int8_t* sign_V,
+                                 const int8_t* q_U, const float* delta_U, const int8_t* sign_U, const void* codes,
+                                 const void* scale_zero, void* stream) {
+  return create_layer_impl(out, n_in, n_out, bits, group, w_in, w_out, SideAngles{nullptr, q_V, delta_V}, sign_V,
+                           SideAngles{nullptr, q_U, delta_U}, sign_U, codes, scale_zero, stream);
+}
+
+harp_status harp_quantize_angles(int m, int64_t half_n, const float* theta, int8_t* q, float* delta, void* stream) {
+  if (m < 1 || m > 16 || half_n < 1 || half_n > (int64_t(1) << 29))
+    return fail(HARP_ERR_INVALID_ARG, "quantize_angles: m=%d or half_n=%lld out of range", m, (long long)half_n);
+  if (!theta || !q || !delta) return fail(HARP_ERR_INVALID_ARG, "quantize_angles: null pointer");
+  if (!aligned16(theta) || !aligned16(q) || !aligned16(delta))
+    return fail(HARP_ERR_INVALID_ARG, "quantize_angles: device pointers must be 16-byte aligned");
+  HARP_CUDA(launch_quantize_angles(m, half_n, theta, q, delta, static_cast<cudaStream_t>(stream)),
+            "quantize_angles launch");
+  return HARP_OK;
+}
+
 harp_status harp_destroy_layer(harp_layer layer) {
   if (!layer) return HARP_OK;
   int prev = 0;
@@ -422,6 +480,8 @@ harp_status harp_destroy_layer(harp_layer layer) {
   cudaDeviceSynchronize();
   cudaFree(layer->L.csV);
   cudaFree(layer->L.csU);
+  cudaFree(layer->L.q8V);
+  cudaFree(layer->L.q8U);
   cudaFree(layer->L.sV);
   cudaFree(layer->L.sU);
   cudaSetDevice(prev);

@@ -15,8 +15,10 @@
 //             -> the remaining log2 C stages (which pair chunk j with j + 2^d) are local.
 // Switching layouts is one gather through distributed shared memory between two
 // cluster barriers. Each CTA first prefetches exactly its slice of the per-stage
-// parameters (cos/sin pairs of the layer, or raw theta for the stand-alone API) with
-// bulk copies into shared memory, so no stage waits on global memory.
+// parameters with bulk copies into shared memory, so no stage waits on global memory.
+// The parameters come in one of three forms (TM): raw theta (the stand-alone API),
+// the layer's cos/sin pairs, or the layer's int8 angles, whose (cos, sin) of
+// pi/4 + delta_t q are evaluated as each rotation needs them.
 // The forward epilogue can also emit the GEMV operand: per group of 64 outputs an
 // int16 copy in dp2a pair order, the power-of-two scale and the fp32 group sum.
 #include "common.cuh"
@@ -60,23 +62,33 @@ __device__ __forceinline__ Geom geom(int w, int m, int C) {
   return g;
 }
 
-// one stage on the layout-A buffer: local pairs (i, i + 2^t), parameter slot q
-template <bool CS>
-__device__ __forceinline__ void stage_a(float* x, const void* tab, int t, int E, int tid, int nthr) {
-  const int h = 1 << t;
+enum { kTabTheta = 0, kTabCS = 1, kTabQ8 = 2 };
+
+// (cos, sin) of pi/4 + theta for parameter slot q of a stage's table (sc: the int8 step)
+template <int TM>
+__device__ __forceinline__ void coef(const void* tab, int q, float sc, float& c, float& s) {
   const float kQuarterPi = 0.785398163397448309616f;
+  if (!tab) {
+    c = s = kRsqrt2;  // Theta == 0: the randomized Hadamard transform
+  } else if (TM == kTabCS) {
+    const float2 v = static_cast<const float2*>(tab)[q];
+    c = v.x;
+    s = v.y;
+  } else if (TM == kTabQ8) {
+    sincosf(fmaf(sc, (float)static_cast<const int8_t*>(tab)[q], kQuarterPi), &s, &c);
+  } else {
+    sincosf(kQuarterPi + static_cast<const float*>(tab)[q], &s, &c);
+  }
+}
+
+// one stage on the layout-A buffer: local pairs (i, i + 2^t), parameter slot q
+template <int TM>
+__device__ __forceinline__ void stage_a(float* x, const void* tab, float sc, int t, int E, int tid, int nthr) {
+  const int h = 1 << t;
   for (int q = tid; q < (E >> 1); q += nthr) {
     const int i = ((q >> t) << (t + 1)) | (q & (h - 1));
     float c, s;
-    if (!tab) {
-      c = s = kRsqrt2;  // Theta == 0: the randomized Hadamard transform
-    } else if (CS) {
-      const float2 v = static_cast<const float2*>(tab)[q];
-      c = v.x;
-      s = v.y;
-    } else {
-      sincosf(kQuarterPi + static_cast<const float*>(tab)[q], &s, &c);
-    }
+    coef<TM>(tab, q, sc, c, s);
     const float a = x[i], b = x[i + h];
     x[i] = fmaf(c, a, s * b);
     x[i + h] = fmaf(s, a, -c * b);
@@ -84,22 +96,13 @@ __device__ __forceinline__ void stage_a(float* x, const void* tab, int t, int E,
 }
 
 // one stage on the layout-B buffer: runs j and j + 2^d (bit d of j clear), same offset
-template <bool CS>
-__device__ __forceinline__ void stage_b(float* x, const void* tab, int d, int run, int E, int tid, int nthr) {
-  const float kQuarterPi = 0.785398163397448309616f;
+template <int TM>
+__device__ __forceinline__ void stage_b(float* x, const void* tab, float sc, int d, int run, int E, int tid, int nthr) {
   for (int q = tid; q < (E >> 1); q += nthr) {
     const int jj = q / run, ii = q - jj * run;
     const int j = ((jj >> d) << (d + 1)) | (jj & ((1 << d) - 1));
     float c, s;
-    if (!tab) {
-      c = s = kRsqrt2;
-    } else if (CS) {
-      const float2 v = static_cast<const float2*>(tab)[q];
-      c = v.x;
-      s = v.y;
-    } else {
-      sincosf(kQuarterPi + static_cast<const float*>(tab)[q], &s, &c);
-    }
+    coef<TM>(tab, q, sc, c, s);
     float* pa = x + j * run + ii;
     float* pb = pa + (run << d);
     const float a = *pa, b = *pb;
@@ -108,7 +111,7 @@ __device__ __forceinline__ void stage_b(float* x, const void* tab, int d, int ru
   }
 }
 
-template <bool CS>
+template <int TM>
 __global__ void __launch_bounds__(kBflyThreads) bfly_kernel(BflyParams p, int C) {
   extern __shared__ __align__(16) uint8_t sm[];
   const Geom g = geom(p.w, p.m, C);
@@ -118,15 +121,20 @@ __global__ void __launch_bounds__(kBflyThreads) bfly_kernel(BflyParams p, int C)
   const int64_t blk = blockIdx.x / C, row = blockIdx.y;
   const int64_t base = blk * w;
   const int64_t half_n = p.n >> 1;
-  constexpr int esz = CS ? 8 : 4;
+  constexpr int esz = TM == kTabCS ? 8 : (TM == kTabQ8 ? 1 : 4);
 
   float* xa = reinterpret_cast<float*>(sm);
   float* xb = xa + E;
   uint8_t* tab = reinterpret_cast<uint8_t*>(xb + E);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(tab + (size_t)m * (E >> 1) * esz);
-  const void* gtab = CS ? static_cast<const void*>(p.cs) : static_cast<const void*>(p.theta);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(tab + (((size_t)m * (E >> 1) * esz + 7) & ~size_t(7)));
+  const void* gtab = TM == kTabCS   ? static_cast<const void*>(p.cs)
+                     : TM == kTabQ8 ? static_cast<const void*>(p.q8 ? p.q8 + kQ8Head : nullptr)
+                                    : static_cast<const void*>(p.theta);
   const bool rht = gtab == nullptr;  // Theta == 0: no per-stage parameters to load
   const uint8_t* stab = rht ? nullptr : tab;
+  // int8 angles: stage t's step, read where the stage starts (uniform, cached)
+  const float* steps = TM == kTabQ8 && !rht ? reinterpret_cast<const float*>(p.q8) : nullptr;
+  auto step_of = [&](int t) -> float { return steps ? __ldg(steps + t) : 0.f; };
 
   // ---- prefetch this CTA's parameter slice: stage t occupies E/2 entries. Bulk copies
   // need 16-byte aligned sources, destinations and sizes; tiny widths use plain loads.
@@ -147,9 +155,12 @@ __global__ void __launch_bounds__(kBflyThreads) bfly_kernel(BflyParams p, int C)
           const int j = ((jj >> d) << (d + 1)) | (jj & ((1 << d) - 1));
           src_q = (int64_t)(j >> (d + 1)) * (1 << t) + (int64_t)E * (j & ((1 << d) - 1)) + (int64_t)r * run + ii;
         }
-        for (int b = 0; b < esz; b += 4)
-          *reinterpret_cast<uint32_t*>(dst + (size_t)q * esz + b) =
-              *reinterpret_cast<const uint32_t*>(src_stage + src_q * esz + b);
+        if (esz == 1)
+          dst[q] = src_stage[src_q];
+        else
+          for (int b = 0; b < esz; b += 4)
+            *reinterpret_cast<uint32_t*>(dst + (size_t)q * esz + b) =
+                *reinterpret_cast<const uint32_t*>(src_stage + src_q * esz + b);
       }
     }
   } else if (tid == 0) {
@@ -183,7 +194,7 @@ __global__ void __launch_bounds__(kBflyThreads) bfly_kernel(BflyParams p, int C)
     __syncthreads();
     if (use_bulk) mbar_wait(bar, 0, p.status, 10);
     for (int t = 0; t < g.e; ++t) {
-      stage_a<CS>(xa, stab ? stab + (size_t)t * (E >> 1) * esz : nullptr, t, E, tid, nthr);
+      stage_a<TM>(xa, stab ? stab + (size_t)t * (E >> 1) * esz : nullptr, step_of(t), t, E, tid, nthr);
       __syncthreads();
     }
     float* out = xa;
@@ -195,7 +206,8 @@ __global__ void __launch_bounds__(kBflyThreads) bfly_kernel(BflyParams p, int C)
       }
       cluster_sync();  // every peer has finished reading this CTA's chunk
       for (int d = 0; d < g.lc; ++d) {
-        stage_b<CS>(xb, stab ? stab + (size_t)(g.e + d) * (E >> 1) * esz : nullptr, d, run, E, tid, nthr);
+        stage_b<TM>(xb, stab ? stab + (size_t)(g.e + d) * (E >> 1) * esz : nullptr, step_of(g.e + d), d, run, E, tid,
+                    nthr);
         __syncthreads();
       }
       out = xb;
@@ -254,7 +266,8 @@ __global__ void __launch_bounds__(kBflyThreads) bfly_kernel(BflyParams p, int C)
       __syncthreads();
       if (use_bulk) mbar_wait(bar, 0, p.status, 11);
       for (int d = g.lc - 1; d >= 0; --d) {
-        stage_b<CS>(xb, stab ? stab + (size_t)(g.e + d) * (E >> 1) * esz : nullptr, d, run, E, tid, nthr);
+        stage_b<TM>(xb, stab ? stab + (size_t)(g.e + d) * (E >> 1) * esz : nullptr, step_of(g.e + d), d, run, E, tid,
+                    nthr);
         __syncthreads();
       }
       cluster_sync();
@@ -269,7 +282,7 @@ __global__ void __launch_bounds__(kBflyThreads) bfly_kernel(BflyParams p, int C)
       if (use_bulk) mbar_wait(bar, 0, p.status, 11);
     }
     for (int t = g.e - 1; t >= 0; --t) {
-      stage_a<CS>(cur, stab ? stab + (size_t)t * (E >> 1) * esz : nullptr, t, E, tid, nthr);
+      stage_a<TM>(cur, stab ? stab + (size_t)t * (E >> 1) * esz : nullptr, step_of(t), t, E, tid, nthr);
       __syncthreads();
     }
     for (int i = tid; i < E; i += nthr) {
@@ -287,8 +300,11 @@ cudaError_t launch_butterfly(const BflyParams& p, int batch, cudaStream_t st) {
   if (batch <= 0) return cudaSuccess;
   const int C = cluster_for(p.w);
   const int E = p.w / C;
-  const bool cs = p.cs != nullptr;
-  const size_t smem = sizeof(float) * 2 * (size_t)E + (size_t)p.m * (E / 2) * (cs ? 8 : 4) + 16;
+  const int tm = p.q8 ? kTabQ8 : (p.cs ? kTabCS : kTabTheta);
+  const int esz = tm == kTabCS ? 8 : (tm == kTabQ8 ? 1 : 4);
+  // the parameter table is followed by the mbarrier, which wants 8-byte alignment
+  const size_t tab_bytes = ((size_t)p.m * (E / 2) * esz + 7) & ~size_t(7);
+  const size_t smem = sizeof(float) * 2 * (size_t)E + tab_bytes + 16;
   int threads = E / 2 < kBflyThreads ? E / 2 : kBflyThreads;
   if (threads < 32) threads = 32;
   cudaLaunchConfig_t cfg = {};
@@ -303,12 +319,16 @@ cudaError_t launch_butterfly(const BflyParams& p, int batch, cudaStream_t st) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  const void* fn = tm == kTabQ8   ? reinterpret_cast<const void*>(bfly_kernel<kTabQ8>)
+                   : tm == kTabCS ? reinterpret_cast<const void*>(bfly_kernel<kTabCS>)
+                                  : reinterpret_cast<const void*>(bfly_kernel<kTabTheta>);
   if (smem > 48 * 1024) {
-    cudaError_t e = cs ? cudaFuncSetAttribute(bfly_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
-                       : cudaFuncSetAttribute(bfly_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  return cs ? cudaLaunchKernelEx(&cfg, bfly_kernel<true>, p, C) : cudaLaunchKernelEx(&cfg, bfly_kernel<false>, p, C);
+  if (tm == kTabQ8) return cudaLaunchKernelEx(&cfg, bfly_kernel<kTabQ8>, p, C);
+  if (tm == kTabCS) return cudaLaunchKernelEx(&cfg, bfly_kernel<kTabCS>, p, C);
+  return cudaLaunchKernelEx(&cfg, bfly_kernel<kTabTheta>, p, C);
 }
 
 // cos/sin tables of pi/4 + theta, computed once per layer in fp32.
@@ -327,6 +347,43 @@ cudaError_t launch_cs_table(const float* theta, int64_t count, float2* cs, cudaS
   const int threads = 256;
   const int64_t blocks = (count + threads - 1) / threads;
   cs_table_kernel<<<(unsigned)(blocks < 4096 ? blocks : 4096), threads, 0, st>>>(theta, count, cs);
+  return cudaGetLastError();
+}
+
+// int8 angle storage, one CTA per stage: delta_t = fp32(max |theta_t| / 127) and
+// q = round-half-even(theta / delta_t) evaluated in fp64 (the inputs are fp32, so the
+// quotient is exact before rounding), clamped to +-127; q = 0 when delta_t = 0.
+__global__ void __launch_bounds__(256) quantize_angles_kernel(const float* __restrict__ theta, int64_t half_n,
+                                                              int8_t* __restrict__ q, float* __restrict__ delta) {
+  __shared__ float red[8];
+  __shared__ float dsh;
+  const int t = blockIdx.x, tid = threadIdx.x;
+  const float* th = theta + (int64_t)t * half_n;
+  float mx = 0.f;
+  for (int64_t i = tid; i < half_n; i += 256) mx = fmaxf(mx, fabsf(th[i]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if ((tid & 31) == 0) red[tid >> 5] = mx;
+  __syncthreads();
+  if (tid == 0) {
+    float m = 0.f;
+    for (int k = 0; k < 8; ++k) m = fmaxf(m, red[k]);
+    dsh = (float)((double)m / 127.0);
+    delta[t] = dsh;
+  }
+  __syncthreads();
+  const double d = (double)dsh;
+  for (int64_t i = tid; i < half_n; i += 256) {
+    double v = d > 0.0 ? rint((double)th[i] / d) : 0.0;
+    v = fmin(fmax(v, -127.0), 127.0);
+    q[(int64_t)t * half_n + i] = (int8_t)(int)v;
+  }
+}
+
+cudaError_t launch_quantize_angles(int m, int64_t half_n, const float* theta, int8_t* q, float* delta,
+                                   cudaStream_t st) {
+  if (m <= 0 || half_n <= 0) return cudaSuccess;
+  quantize_angles_kernel<<<(unsigned)m, 256, 0, st>>>(theta, half_n, q, delta);
   return cudaGetLastError();
 }
 

@@ -18,9 +18,11 @@
 //    thread, three stages per shared-memory round trip), the cross-CTA stages reached
 //    by pushing data into the peers' shared memory and one cluster barrier (8
 //    parallel release-arrives, acquire on the own barrier). A second producer warp
-//    prefetches every chain's cos/sin tables with bulk copies. When every butterfly of
-//    the stack has Theta == 0 (the fixed randomized Hadamard transform) a separate
-//    instantiation uses the constant 1/sqrt 2 blocks and no tables are loaded.
+//    prefetches every chain's angle tables with bulk copies. The kernel is instantiated
+//    per form of the angles (TM): (cos, sin) fp32 pairs, 8 bytes per rotation; int8
+//    angles, 1 byte per rotation plus one step per stage, whose cos/sin are evaluated as
+//    the rotation runs; or Theta == 0 everywhere (the fixed randomized Hadamard
+//    transform), where the constant 1/sqrt 2 blocks need no table at all.
 //  * Grid-wide barriers (release/acquire counters) only where a whole output vector
 //    is needed: after q/k/v, o, gate/up, the MLP blocks, and down.
 //
@@ -147,7 +149,7 @@ constexpr int kSgnSlot = 1024;  // bytes per prefetched sign slice (>= the wides
 
 struct Smem {
   uint8_t* ring;
-  float2* tab;
+  uint8_t* tab;
   int8_t* sgn;  // 4 slots of kSgnSlot: the sign slices of the current chain's butterflies
   float *xa, *xb, *res, *ss, *red;
   int* ucnt;
@@ -161,7 +163,7 @@ __device__ __forceinline__ Smem carve(const Params& p, int stage_bytes) {
   Smem s;
   s.ring = b;
   b += (size_t)p.ring_stages * stage_bytes;
-  s.tab = reinterpret_cast<float2*>(b);
+  s.tab = b;
   b += p.tab_bytes;
   s.sgn = reinterpret_cast<int8_t*>(b);
   b += 4 * kSgnSlot;
@@ -231,42 +233,70 @@ __device__ __forceinline__ Range units(const Params& p, int l, int ph, int c, in
 }
 
 // ------------------------------------------------------------------ table loads (producer warp 1)
+// Table of one butterfly in shared memory: stage t holds the parameters of the CTA's
+// rotations in stage order, E/2 entries of 8 bytes (cos, sin) or 1 byte (int8 angle);
+// int8 tables start with the 64-byte head of per-stage steps.
+template <int TM>
+__device__ __forceinline__ constexpr int tab_esz() { return TM == kTmQ8 ? 1 : 8; }
+template <int TM>
+__device__ __forceinline__ constexpr int tab_head() { return TM == kTmQ8 ? kQ8Head : 0; }
+
+template <int TM>
+__device__ __forceinline__ uint32_t table_bytes_cluster(int w, int m) {
+  return (uint32_t)(tab_head<TM>() + tab_esz<TM>() * m * (w / kC / 2));
+}
+template <int TM>
+__device__ __forceinline__ uint32_t table_bytes_local(int w, int m) {
+  return (uint32_t)(tab_head<TM>() + tab_esz<TM>() * m * (w / 2));
+}
+// bytes a table load actually transfers (none for Theta == 0)
+template <int TM>
+__device__ __forceinline__ uint32_t copied_bytes_cluster(const uint8_t* src, int w, int m) {
+  return TM == kTmHad || !src ? 0u : table_bytes_cluster<TM>(w, m);
+}
+template <int TM>
+__device__ __forceinline__ uint32_t copied_bytes_local(const uint8_t* src, int w, int m) {
+  return TM == kTmHad || !src ? 0u : table_bytes_local<TM>(w, m);
+}
+
 // Per-CTA slice of a cluster-distributed butterfly (width w, C = 8): stage t < e is the
 // contiguous run of the CTA's chunk; stage t >= e is C/2 runs of `run` pairs.
-__device__ __forceinline__ uint32_t load_table_cluster(float2* dst, const float2* cs, int64_t n, int w, int m, int blk, int r,
-                                       uint64_t* bar) {
+template <int TM>
+__device__ __forceinline__ uint32_t load_table_cluster(uint8_t* dst, const uint8_t* src, int64_t n, int w, int m,
+                                                       int blk, int r, uint64_t* bar) {
+  constexpr int esz = tab_esz<TM>(), head = tab_head<TM>();
   const int E = w / kC, e = m - 3, run = E / kC;
   const int64_t half_n = n >> 1;
-  if (!cs) return (uint32_t)(8 * m * (E >> 1));  // Theta == 0: nothing to copy, same layout
+  if (TM == kTmHad || !src) return table_bytes_cluster<TM>(w, m);  // nothing to copy, same layout
+  if (head) bulk_g2s(dst, src, (uint32_t)head, bar);
   for (int t = 0; t < m; ++t) {
-    const float2* src = cs + (int64_t)t * half_n + (int64_t)blk * (w >> 1);
-    float2* d = dst + (size_t)t * (E >> 1);
+    const uint8_t* st = src + head + ((int64_t)t * half_n + (int64_t)blk * (w >> 1)) * esz;
+    uint8_t* d = dst + head + (size_t)t * (E >> 1) * esz;
     if (t < e) {
-      bulk_g2s(d, src + (int64_t)r * (E >> 1), (uint32_t)(8 * (E >> 1)), bar);
+      bulk_g2s(d, st + (int64_t)r * (E >> 1) * esz, (uint32_t)(esz * (E >> 1)), bar);
     } else {
       const int dd = t - e;
       for (int jj = 0; jj < (kC >> 1); ++jj) {
         const int j = ((jj >> dd) << (dd + 1)) | (jj & ((1 << dd) - 1));
         const int64_t pb = (int64_t)(j >> (dd + 1)) * (1 << t) + (int64_t)E * (j & ((1 << dd) - 1)) + (int64_t)r * run;
-        bulk_g2s(d + jj * run, src + pb, (uint32_t)(8 * run), bar);
+        bulk_g2s(d + (size_t)jj * run * esz, st + pb * esz, (uint32_t)(esz * run), bar);
       }
     }
   }
-  return (uint32_t)(8 * m * (E >> 1));
+  return table_bytes_cluster<TM>(w, m);
 }
 
 // the whole block `blk` of width w held by one CTA: one run of w/2 pairs per stage
-__device__ __forceinline__ uint32_t load_table_local(float2* dst, const float2* cs, int64_t n, int w, int m, int blk, uint64_t* bar) {
-  if (!cs) return (uint32_t)(4 * w * m);
+template <int TM>
+__device__ __forceinline__ uint32_t load_table_local(uint8_t* dst, const uint8_t* src, int64_t n, int w, int m, int blk,
+                                                     uint64_t* bar) {
+  constexpr int esz = tab_esz<TM>(), head = tab_head<TM>();
+  if (TM == kTmHad || !src) return table_bytes_local<TM>(w, m);
+  if (head) bulk_g2s(dst, src, (uint32_t)head, bar);
   for (int t = 0; t < m; ++t)
-    bulk_g2s(dst + (size_t)t * (w >> 1), cs + (int64_t)t * (n >> 1) + (int64_t)blk * (w >> 1), (uint32_t)(4 * w), bar);
-  return (uint32_t)(4 * w * m);
-}
-
-__device__ __forceinline__ uint32_t table_bytes_cluster(int w, int m) { return (uint32_t)(8 * m * (w / kC / 2)); }
-// bytes a table load actually transfers (none for a Theta == 0 side)
-__device__ __forceinline__ uint32_t copied_bytes_cluster(const float2* cs, int w, int m) {
-  return cs ? table_bytes_cluster(w, m) : 0u;
+    bulk_g2s(dst + head + (size_t)t * (w >> 1) * esz, src + head + ((int64_t)t * (n >> 1) + (int64_t)blk * (w >> 1)) * esz,
+             (uint32_t)(esz * (w >> 1)), bar);
+  return table_bytes_local<TM>(w, m);
 }
 
 // P7 roles: block CTAs, and the clusters applying F_U_q / F_U_k
@@ -274,6 +304,34 @@ __device__ __forceinline__ int qk_cluster(const Params& p, int which) { return p
 
 // ------------------------------------------------------------------ butterfly stages
 constexpr float kRsqrt2 = 0.70710678118654752440f;  // cos(pi/4) = sin(pi/4): the Theta == 0 block
+
+// One stage's row of a table of E/2 entries per stage: (cos, sin) pairs, or int8 angles
+// with the stage's step.
+struct StageTab {
+  const float2* cs;
+  const int8_t* q8;
+  float step;
+};
+
+template <int TM>
+__device__ __forceinline__ StageTab stage_tab(const uint8_t* tab, int ts, int E) {
+  StageTab r;
+  r.cs = reinterpret_cast<const float2*>(tab) + (size_t)ts * (E >> 1);
+  r.q8 = reinterpret_cast<const int8_t*>(tab + kQ8Head) + (size_t)ts * (E >> 1);
+  r.step = TM == kTmQ8 ? reinterpret_cast<const float*>(tab)[ts] : 0.f;
+  return r;
+}
+
+// (cos, sin) of rotation q of a stage. int8 angles take the fast sine/cosine unit:
+// pi/4 + delta_t q lies within a few tenths of pi/4.
+template <int TM>
+__device__ __forceinline__ float2 coef(const StageTab& st, int q) {
+  if (TM == kTmHad) return make_float2(kRsqrt2, kRsqrt2);
+  if (TM == kTmCS) return st.cs[q];
+  float s, c;
+  __sincosf(fmaf(st.step, (float)st.q8[q], 0.785398163397448309616f), &s, &c);
+  return make_float2(c, s);
+}
 
 __device__ __forceinline__ void rot(float& a, float& b, float2 cs) {
   const float x = a, y = b;
@@ -283,9 +341,9 @@ __device__ __forceinline__ void rot(float& a, float& b, float2 cs) {
 
 // NS stages t .. t+NS-1 (pairs (i, i + 2^s)) on a buffer of E elements, 2^NS values per
 // thread held in registers; table row s (E/2 pairs, pair numbered by first index).
-// HAD: every block is the Theta == 0 block [[1, 1], [1, -1]] / sqrt 2 (no table read).
-template <int NS, bool HAD>
-__device__ __forceinline__ void round_a(float* x, const float2* tab, int t, int E, int ct) {
+// TM == kTmHad: every block is the Theta == 0 block [[1, 1], [1, -1]] / sqrt 2 (no table read).
+template <int NS, int TM>
+__device__ __forceinline__ void round_a(float* x, const uint8_t* tab, int t, int E, int ct) {
   constexpr int P = 1 << NS;
   const int nthr = E / P, h = 1 << t;
   if (ct < nthr) {
@@ -296,13 +354,13 @@ __device__ __forceinline__ void round_a(float* x, const float2* tab, int t, int 
 #pragma unroll
     for (int s = 0; s < NS; ++s) {
       const int ts = t + s, hs = 1 << ts;
-      const float2* tt = tab + (size_t)ts * (E >> 1);
+      const StageTab st = stage_tab<TM>(tab, ts, E);
 #pragma unroll
       for (int k = 0; k < P; ++k) {
         if (k & (1 << s)) continue;
         const int i = base + k * h;
         const int q = ((i >> (ts + 1)) << ts) | (i & (hs - 1));
-        rot(v[k], v[k + (1 << s)], HAD ? make_float2(kRsqrt2, kRsqrt2) : tt[q]);
+        rot(v[k], v[k + (1 << s)], coef<TM>(st, q));
       }
     }
 #pragma unroll
@@ -312,21 +370,21 @@ __device__ __forceinline__ void round_a(float* x, const float2* tab, int t, int 
 }
 
 // layout-A stages t0 .. t1-1, three per shared-memory round
-template <bool HAD>
-__device__ __forceinline__ void stages_a(float* x, const float2* tab, int t0, int t1, int E, int ct) {
+template <int TM>
+__device__ __forceinline__ void stages_a(float* x, const uint8_t* tab, int t0, int t1, int E, int ct) {
   int t = t0;
   while (t1 - t >= 3) {
-    round_a<3, HAD>(x, tab, t, E, ct);
+    round_a<3, TM>(x, tab, t, E, ct);
     t += 3;
   }
-  if (t1 - t == 2) round_a<2, HAD>(x, tab, t, E, ct);
-  if (t1 - t == 1) round_a<1, HAD>(x, tab, t, E, ct);
+  if (t1 - t == 2) round_a<2, TM>(x, tab, t, E, ct);
+  if (t1 - t == 1) round_a<1, TM>(x, tab, t, E, ct);
 }
 
 // the three layout-B stages (runs j and j + 2^d, same offset), one round: thread T holds
 // the 8 values {j run + T}; table rows e, e+1, e+2 numbered jj run + T
-template <bool HAD>
-__device__ __forceinline__ void stages_b(float* x, const float2* tab, int e, int E, int ct) {
+template <int TM>
+__device__ __forceinline__ void stages_b(float* x, const uint8_t* tab, int e, int E, int ct) {
   const int run = E / kC;
   if (ct < run) {
     float v[kC];
@@ -334,12 +392,12 @@ __device__ __forceinline__ void stages_b(float* x, const float2* tab, int e, int
     for (int j = 0; j < kC; ++j) v[j] = x[j * run + ct];
 #pragma unroll
     for (int d = 0; d < 3; ++d) {
-      const float2* tt = tab + (size_t)(e + d) * (E >> 1);
+      const StageTab st = stage_tab<TM>(tab, e + d, E);
 #pragma unroll
       for (int j = 0; j < kC; ++j) {
         if (j & (1 << d)) continue;
         const int jj = ((j >> (d + 1)) << d) | (j & ((1 << d) - 1));
-        rot(v[j], v[j + (1 << d)], HAD ? make_float2(kRsqrt2, kRsqrt2) : tt[jj * run + ct]);
+        rot(v[j], v[j + (1 << d)], coef<TM>(st, jj * run + ct));
       }
     }
 #pragma unroll
@@ -460,10 +518,10 @@ __device__ __forceinline__ float zsum(const float* zp, int nk, int n, int i) {
 
 // ------------------------------------------------------------------ chains (cluster-collective)
 // residual chain: [res += F_U(z)] ; n = rms(res) ; x~ = F_V(n) ; operand
-template <bool HAD>
+template <int TM>
 __device__ __forceinline__ bool chain_residual(const Params& p, Smem& s, Xchg& X, const Lin* U, const float* zp, int nk,
-                               const Lin* V, bool first, uint32_t r, int ct, const float2* tabU,
-                               const float2* tabV) {
+                               const Lin* V, bool first, uint32_t r, int ct, const uint8_t* tabU,
+                               const uint8_t* tabV) {
   const int W = p.hidden, E = p.E, e = p.m_hidden - 3;
   if (first) {
     for (int L = ct; L < E; L += kNT) s.res[L] = load_act(p.x_in, gidx_b(L, E, r), p.xt);
@@ -473,10 +531,10 @@ __device__ __forceinline__ bool chain_residual(const Params& p, Smem& s, Xchg& X
       s.xa[i] = zsum(zp, nk, W, gi) * (float)s.sgn[i];
     }
     cbar();
-    stages_a<HAD>(s.xa, tabU, 0, e, E, ct);
+    stages_a<TM>(s.xa, tabU, 0, e, E, ct);
     push_a_to_b(s.xa, s.xb, E, r, ct);
     if (!exchange(s, X, ct, p.status, 41)) return false;
-    stages_b<HAD>(s.xb, tabU, e, E, ct);
+    stages_b<TM>(s.xb, tabU, e, E, ct);
     for (int L = ct; L < E; L += kNT) s.res[L] += s.xb[L];
   }
   if (!V) {
@@ -503,17 +561,17 @@ __device__ __forceinline__ bool chain_residual(const Params& p, Smem& s, Xchg& X
   const float inv = 1.0f / sqrtf(t / (float)W + p.eps);
   for (int i = ct; i < E; i += kNT) s.xa[i] *= inv * (float)s.sgn[kSgnSlot + i];
   cbar();
-  stages_a<HAD>(s.xa, tabV, 0, e, E, ct);
+  stages_a<TM>(s.xa, tabV, 0, e, E, ct);
   push_a_to_b(s.xa, s.xb, E, r, ct);
   if (!exchange(s, X, ct, p.status, 43)) return false;
-  stages_b<HAD>(s.xb, tabV, e, E, ct);
+  stages_b<TM>(s.xb, tabV, e, E, ct);
   return prep_and_broadcast(s, X, s.xb, V->n_in, p.bits, E, r, ct, p.status);
 }
 
 // attention chain: v = F_U_v(z_v); a = v broadcast per KV group; x~ = F_V_o(a); operand
-template <bool HAD>
+template <int TM>
 __device__ __forceinline__ bool chain_attn(const Params& p, Smem& s, Xchg& X, const Lin* Lv, const Lin* Lo, uint32_t r, int ct,
-                           const float2* tabU, const float2* tabV) {
+                           const uint8_t* tabU, const uint8_t* tabV) {
   const int Wu = Lv->w_out, Eu = Wu / kC, eu = Lv->m_out - 3;
 
   for (int i = ct; i < Eu; i += kNT) {
@@ -521,10 +579,10 @@ __device__ __forceinline__ bool chain_attn(const Params& p, Smem& s, Xchg& X, co
     s.xa[i] = zsum(p.zpv, p.nk_h, Wu, gi) * (float)s.sgn[i];
   }
   cbar();
-  stages_a<HAD>(s.xa, tabU, 0, eu, Eu, ct);
+  stages_a<TM>(s.xa, tabU, 0, eu, Eu, ct);
   push_a_to_b(s.xa, s.xb, Eu, r, ct);
   if (!exchange(s, X, ct, p.status, 44)) return false;
-  stages_b<HAD>(s.xb, tabU, eu, Eu, ct);
+  stages_b<TM>(s.xb, tabU, eu, Eu, ct);
   // push every v value to the layout-A owners of the query-head elements that copy it
   const int Eo = p.E, eo = p.m_hidden - 3, hd = p.head_dim, rep = p.rep;
   for (int L = ct; L < Eu; L += kNT) {
@@ -537,17 +595,17 @@ __device__ __forceinline__ bool chain_attn(const Params& p, Smem& s, Xchg& X, co
   if (!exchange(s, X, ct, p.status, 45)) return false;
   for (int i = ct; i < Eo; i += kNT) s.xa[i] *= (float)s.sgn[kSgnSlot + i];
   cbar();
-  stages_a<HAD>(s.xa, tabV, 0, eo, Eo, ct);
+  stages_a<TM>(s.xa, tabV, 0, eo, Eo, ct);
   push_a_to_b(s.xa, s.xb, Eo, r, ct);
   if (!exchange(s, X, ct, p.status, 46)) return false;
-  stages_b<HAD>(s.xb, tabV, eo, Eo, ct);
+  stages_b<TM>(s.xb, tabV, eo, Eo, ct);
   return prep_and_broadcast(s, X, s.xb, Lo->n_in, p.bits, Eo, r, ct, p.status);
 }
 
 // F_U of a q or k GEMV output (cluster-distributed), written to out[gidx]
-template <bool HAD>
+template <int TM>
 __device__ __forceinline__ bool chain_out_only(const Params& p, Smem& s, Xchg& X, const Lin* Lq, const float* zp, float* out,
-                               uint32_t r, int ct, const float2* tab) {
+                               uint32_t r, int ct, const uint8_t* tab) {
   const int W = Lq->w_out, E = W / kC, e = Lq->m_out - 3;
 
   for (int i = ct; i < E; i += kNT) {
@@ -555,10 +613,10 @@ __device__ __forceinline__ bool chain_out_only(const Params& p, Smem& s, Xchg& X
     s.xa[i] = zsum(zp, p.nk_h, W, gi) * (float)s.sgn[i];
   }
   cbar();
-  stages_a<HAD>(s.xa, tab, 0, e, E, ct);
+  stages_a<TM>(s.xa, tab, 0, e, E, ct);
   push_a_to_b(s.xa, s.xb, E, r, ct);
   if (!exchange(s, X, ct, p.status, 47)) return false;
-  stages_b<HAD>(s.xb, tab, e, E, ct);
+  stages_b<TM>(s.xb, tab, e, E, ct);
   for (int L = ct; L < E; L += kNT) out[gidx_b(L, E, r)] = s.xb[L];
   cbar();
   return true;
@@ -566,9 +624,9 @@ __device__ __forceinline__ bool chain_out_only(const Params& p, Smem& s, Xchg& X
 
 // one whole MLP block (width <= 512) in one CTA: F_U_gate, F_U_up, silu*up, F_V_down,
 // operand of the down projection for this block (to global)
-template <bool HAD>
+template <int TM>
 __device__ __forceinline__ void block_chain(const Params& p, Smem& s, const Lin* Lg, const Lin* Lu, const Lin* Ld, int blk, int ct,
-                            const float2* tab) {
+                            const uint8_t* tab) {
   const int wb = Lg->w_out, mb = Lg->m_out, F = p.ffn;
   const int base = blk * wb;
   for (int i = ct; i < wb; i += kNT) {
@@ -576,14 +634,14 @@ __device__ __forceinline__ void block_chain(const Params& p, Smem& s, const Lin*
     s.xb[i] = zsum(p.zpu, p.nk_h, F, base + i) * (float)s.sgn[kSgnSlot + i];
   }
   cbar();
-  stages_a<HAD>(s.xa, tab, 0, mb, wb, ct);
-  stages_a<HAD>(s.xb, tab + (size_t)mb * (wb >> 1), 0, mb, wb, ct);
+  stages_a<TM>(s.xa, tab, 0, mb, wb, ct);
+  stages_a<TM>(s.xb, tab + table_bytes_local<TM>(wb, mb), 0, mb, wb, ct);
   for (int i = ct; i < wb; i += kNT) {
     const float g = s.xa[i];
     s.xa[i] = g / (1.0f + expf(-g)) * s.xb[i] * (float)s.sgn[2 * kSgnSlot + i];
   }
   cbar();
-  stages_a<HAD>(s.xa, tab + (size_t)2 * mb * (wb >> 1), 0, mb, wb, ct);
+  stages_a<TM>(s.xa, tab + 2 * table_bytes_local<TM>(wb, mb), 0, mb, wb, ct);
   const int n_in = Ld->n_in;
   int16_t* xq16 = reinterpret_cast<int16_t*>(p.xq_down);
   const int warp = ct >> 5, lane = ct & 31;
@@ -695,9 +753,9 @@ __device__ __noinline__ bool grid_barrier(const Params& p, int idx, int ct) {
 }
 
 // ------------------------------------------------------------------ the kernel
-// HAD: every butterfly of the stack is the fixed randomized Hadamard transform (Theta == 0,
-// no cos/sin tables); the learned-angle instantiation keeps its rounds free of that case.
-template <int BITS, bool HAD>
+// TM: how every butterfly of the stack keeps its angles (kTmCS, kTmHad, kTmQ8); each form
+// has its own instantiation, so no rotation round branches on it.
+template <int BITS, int TM>
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_constant__ Params p) {
   using Gm = Geo<BITS>;
   Smem s = carve(p, Gm::kStageBytes);
@@ -788,18 +846,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         if (!(ok = begin())) break;
         if (lane == 0) {
           uint32_t bytes = 0;
-          if (prev) bytes += copied_bytes_cluster(prev[6].csU, prev[6].w_out, prev[6].m_out);
+          if (prev) bytes += copied_bytes_cluster<TM>(prev[6].tU, prev[6].w_out, prev[6].m_out);
           const Lin* V = l < L ? lin + p.asg_qkv[c] : nullptr;
-          if (V) bytes += copied_bytes_cluster(V->csV, V->w_in, V->m_in);
+          if (V) bytes += copied_bytes_cluster<TM>(V->tV, V->w_in, V->m_in);
           const int Eh = p.E;
           if (prev) bytes += Eh;
           if (V) bytes += Eh;
           mbar_arrive_expect_tx(s.tab_full, bytes);
           uint32_t off = 0;
           if (prev)
-            off += load_table_cluster(s.tab, prev[6].csU, prev[6].n_out, prev[6].w_out, prev[6].m_out, 0, (int)r,
+            off += load_table_cluster<TM>(s.tab, prev[6].tU, prev[6].n_out, prev[6].w_out, prev[6].m_out, 0, (int)r,
                                       s.tab_full);
-          if (V) load_table_cluster(s.tab + off / 8, V->csV, V->n_in, V->w_in, V->m_in, 0, (int)r, s.tab_full);
+          if (V) load_table_cluster<TM>(s.tab + off, V->tV, V->n_in, V->w_in, V->m_in, 0, (int)r, s.tab_full);
           if (prev) bulk_g2s(s.sgn, prev[6].sU + (int64_t)r * Eh, (uint32_t)Eh, s.tab_full);
           if (V) bulk_g2s(s.sgn + kSgnSlot, V->sV + (int64_t)r * Eh, (uint32_t)Eh, s.tab_full);
         }
@@ -808,12 +866,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         // P3
         if (!(ok = begin())) break;
         if (lane == 0) {
-          const uint32_t b0 = table_bytes_cluster(lin[2].w_out, lin[2].m_out);
+          const uint32_t b0 = table_bytes_cluster<TM>(lin[2].w_out, lin[2].m_out);
           const int Eu = lin[2].w_out / kC, Eo = lin[3].w_in / kC;
-          mbar_arrive_expect_tx(s.tab_full, copied_bytes_cluster(lin[2].csU, lin[2].w_out, lin[2].m_out) +
-                                                copied_bytes_cluster(lin[3].csV, lin[3].w_in, lin[3].m_in) + Eu + Eo);
-          load_table_cluster(s.tab, lin[2].csU, lin[2].n_out, lin[2].w_out, lin[2].m_out, 0, (int)r, s.tab_full);
-          load_table_cluster(s.tab + b0 / 8, lin[3].csV, lin[3].n_in, lin[3].w_in, lin[3].m_in, 0, (int)r, s.tab_full);
+          mbar_arrive_expect_tx(s.tab_full, copied_bytes_cluster<TM>(lin[2].tU, lin[2].w_out, lin[2].m_out) +
+                                                copied_bytes_cluster<TM>(lin[3].tV, lin[3].w_in, lin[3].m_in) + Eu + Eo);
+          load_table_cluster<TM>(s.tab, lin[2].tU, lin[2].n_out, lin[2].w_out, lin[2].m_out, 0, (int)r, s.tab_full);
+          load_table_cluster<TM>(s.tab + b0, lin[3].tV, lin[3].n_in, lin[3].w_in, lin[3].m_in, 0, (int)r, s.tab_full);
           bulk_g2s(s.sgn, lin[2].sU + (int64_t)r * Eu, (uint32_t)Eu, s.tab_full);
           bulk_g2s(s.sgn + kSgnSlot, lin[3].sV + (int64_t)r * Eo, (uint32_t)Eo, s.tab_full);
         }
@@ -822,12 +880,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         if (!(ok = begin())) break;
         if (lane == 0) {
           const Lin* V = lin + 4 + p.asg_gu[c];
-          const uint32_t b0 = table_bytes_cluster(lin[3].w_out, lin[3].m_out);
+          const uint32_t b0 = table_bytes_cluster<TM>(lin[3].w_out, lin[3].m_out);
           const int Eh = p.E;
-          mbar_arrive_expect_tx(s.tab_full, copied_bytes_cluster(lin[3].csU, lin[3].w_out, lin[3].m_out) +
-                                                copied_bytes_cluster(V->csV, V->w_in, V->m_in) + 2 * Eh);
-          load_table_cluster(s.tab, lin[3].csU, lin[3].n_out, lin[3].w_out, lin[3].m_out, 0, (int)r, s.tab_full);
-          load_table_cluster(s.tab + b0 / 8, V->csV, V->n_in, V->w_in, V->m_in, 0, (int)r, s.tab_full);
+          mbar_arrive_expect_tx(s.tab_full, copied_bytes_cluster<TM>(lin[3].tU, lin[3].w_out, lin[3].m_out) +
+                                                copied_bytes_cluster<TM>(V->tV, V->w_in, V->m_in) + 2 * Eh);
+          load_table_cluster<TM>(s.tab, lin[3].tU, lin[3].n_out, lin[3].w_out, lin[3].m_out, 0, (int)r, s.tab_full);
+          load_table_cluster<TM>(s.tab + b0, V->tV, V->n_in, V->w_in, V->m_in, 0, (int)r, s.tab_full);
           bulk_g2s(s.sgn, lin[3].sU + (int64_t)r * Eh, (uint32_t)Eh, s.tab_full);
           bulk_g2s(s.sgn + kSgnSlot, V->sV + (int64_t)r * Eh, (uint32_t)Eh, s.tab_full);
         }
@@ -839,23 +897,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
           const int wb = lin[4].w_out, mb = lin[4].m_out;
           const int blk = t_cta;  // at most one MLP block per CTA (checked at set-up)
           if (blk < nblocks)
-            bytes += (lin[4].csU ? 4 * wb * mb : 0) + (lin[5].csU ? 4 * wb * mb : 0) + (lin[6].csV ? 4 * wb * mb : 0) +
-                     3 * wb;
+            bytes += copied_bytes_local<TM>(lin[4].tU, wb, mb) + copied_bytes_local<TM>(lin[5].tU, wb, mb) +
+                     copied_bytes_local<TM>(lin[6].tV, wb, mb) + 3 * wb;
           const int qk = c == qk_cluster(p, 0) ? 0 : (c == qk_cluster(p, 1) ? 1 : -1);
           const int Eq = qk >= 0 ? lin[qk].w_out / kC : 0;
-          if (qk >= 0) bytes += copied_bytes_cluster(lin[qk].csU, lin[qk].w_out, lin[qk].m_out) + Eq;
+          if (qk >= 0) bytes += copied_bytes_cluster<TM>(lin[qk].tU, lin[qk].w_out, lin[qk].m_out) + Eq;
           mbar_arrive_expect_tx(s.tab_full, bytes);
           if (blk < nblocks) {
             uint32_t off = 0;
-            off += load_table_local(s.tab + off / 8, lin[4].csU, lin[4].n_out, wb, mb, blk, s.tab_full);
-            off += load_table_local(s.tab + off / 8, lin[5].csU, lin[5].n_out, wb, mb, blk, s.tab_full);
-            load_table_local(s.tab + off / 8, lin[6].csV, lin[6].n_in, wb, mb, blk, s.tab_full);
+            off += load_table_local<TM>(s.tab + off, lin[4].tU, lin[4].n_out, wb, mb, blk, s.tab_full);
+            off += load_table_local<TM>(s.tab + off, lin[5].tU, lin[5].n_out, wb, mb, blk, s.tab_full);
+            load_table_local<TM>(s.tab + off, lin[6].tV, lin[6].n_in, wb, mb, blk, s.tab_full);
             bulk_g2s(s.sgn, lin[4].sU + (int64_t)blk * wb, (uint32_t)wb, s.tab_full);
             bulk_g2s(s.sgn + kSgnSlot, lin[5].sU + (int64_t)blk * wb, (uint32_t)wb, s.tab_full);
             bulk_g2s(s.sgn + 2 * kSgnSlot, lin[6].sV + (int64_t)blk * wb, (uint32_t)wb, s.tab_full);
           }
           if (qk >= 0) {
-            load_table_cluster(s.tab, lin[qk].csU, lin[qk].n_out, lin[qk].w_out, lin[qk].m_out, 0, (int)r, s.tab_full);
+            load_table_cluster<TM>(s.tab, lin[qk].tU, lin[qk].n_out, lin[qk].w_out, lin[qk].m_out, 0, (int)r, s.tab_full);
             bulk_g2s(s.sgn, lin[qk].sU + (int64_t)r * Eq, (uint32_t)Eq, s.tab_full);
           }
         }
@@ -886,9 +944,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     // P1
     if (!(ok = tab_acquire())) break;
     {
-      const float2* tU = s.tab;
-      const float2* tV = prev ? s.tab + table_bytes_cluster(prev[6].w_out, prev[6].m_out) / 8 : s.tab;
-      ok = chain_residual<HAD>(p, s, X, prev ? prev + 6 : nullptr, p.zpd, p.nk_f, lin + p.asg_qkv[c], l == 0, r, ct, tU,
+      const uint8_t* tU = s.tab;
+      const uint8_t* tV = prev ? s.tab + table_bytes_cluster<TM>(prev[6].w_out, prev[6].m_out) : s.tab;
+      ok = chain_residual<TM>(p, s, X, prev ? prev + 6 : nullptr, p.zpd, p.nk_f, lin + p.asg_qkv[c], l == 0, r, ct, tU,
                           tV);
     }
     tab_release();
@@ -898,8 +956,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     if (!(ok = grid_barrier(p, l * 5 + 0, ct))) break;
     // P3
     if (!(ok = tab_acquire())) break;
-    ok = chain_attn<HAD>(p, s, X, lin + 2, lin + 3, r, ct, s.tab,
-                    s.tab + table_bytes_cluster(lin[2].w_out, lin[2].m_out) / 8);
+    ok = chain_attn<TM>(p, s, X, lin + 2, lin + 3, r, ct, s.tab,
+                    s.tab + table_bytes_cluster<TM>(lin[2].w_out, lin[2].m_out));
     tab_release();
     if (!ok) break;
     // P4
@@ -907,8 +965,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     if (!(ok = grid_barrier(p, l * 5 + 1, ct))) break;
     // P5
     if (!(ok = tab_acquire())) break;
-    ok = chain_residual<HAD>(p, s, X, lin + 3, p.zpo, p.nk_h, lin + 4 + p.asg_gu[c], false, r, ct, s.tab,
-                        s.tab + table_bytes_cluster(lin[3].w_out, lin[3].m_out) / 8);
+    ok = chain_residual<TM>(p, s, X, lin + 3, p.zpo, p.nk_h, lin + 4 + p.asg_gu[c], false, r, ct, s.tab,
+                        s.tab + table_bytes_cluster<TM>(lin[3].w_out, lin[3].m_out));
     tab_release();
     if (!ok) break;
     // P6
@@ -917,13 +975,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     // P7
     if (!(ok = tab_acquire())) break;
     {
-      if (t_cta < nblocks) block_chain<HAD>(p, s, lin + 4, lin + 5, lin + 6, t_cta, ct, s.tab);
+      if (t_cta < nblocks) block_chain<TM>(p, s, lin + 4, lin + 5, lin + 6, t_cta, ct, s.tab);
       const int qk = c == qk_cluster(p, 0) ? 0 : (c == qk_cluster(p, 1) ? 1 : -1);
       if (qk >= 0) {
         float* out = qk == 0 ? p.qout + (int64_t)l * lin[0].n_out : p.kout + (int64_t)l * lin[1].n_out;
         const float* zp = qk == 0 ? p.zpq + (int64_t)l * p.nk_h * lin[0].n_out
                                   : p.zpk + (int64_t)l * p.nk_h * lin[1].n_out;
-        ok = chain_out_only<HAD>(p, s, X, lin + qk, zp, out, r, ct, s.tab);
+        ok = chain_out_only<TM>(p, s, X, lin + qk, zp, out, r, ct, s.tab);
       }
     }
     tab_release();
@@ -949,7 +1007,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   // final: out = h_{L-1} + F_U_down(z_down)
   if (ok && (ok = tab_acquire())) {
     const Lin* last = p.lin + 7 * (L - 1);
-    ok = chain_residual<HAD>(p, s, X, last + 6, p.zpd, p.nk_f, nullptr, false, r, ct, s.tab, s.tab);
+    ok = chain_residual<TM>(p, s, X, last + 6, p.zpd, p.nk_f, nullptr, false, r, ct, s.tab, s.tab);
     if (ok && c == 0)
       for (int L2 = ct; L2 < p.E; L2 += kNT) store_act(p.y_out, gidx_b(L2, p.E, r), p.yt, s.res[L2]);
     tab_release();
@@ -966,15 +1024,16 @@ size_t smem_bytes(const Params& p) {
 }
 
 template <int BITS>
-const void* kernel_ptr(bool had) {
-  return had ? reinterpret_cast<const void*>(decode_kernel<BITS, true>)
-             : reinterpret_cast<const void*>(decode_kernel<BITS, false>);
+const void* kernel_ptr(int tm) {
+  return tm == kTmHad  ? reinterpret_cast<const void*>(decode_kernel<BITS, kTmHad>)
+         : tm == kTmQ8 ? reinterpret_cast<const void*>(decode_kernel<BITS, kTmQ8>)
+                       : reinterpret_cast<const void*>(decode_kernel<BITS, kTmCS>);
 }
 
 template <int BITS>
 cudaError_t launch_bits(const Params& p, cudaStream_t st) {
   const size_t smem = smem_bytes<BITS>(p);
-  cudaError_t e = cudaFuncSetAttribute(kernel_ptr<BITS>(p.had != 0), cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(kernel_ptr<BITS>(p.tm), cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -989,8 +1048,9 @@ cudaError_t launch_bits(const Params& p, cudaStream_t st) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return p.had ? cudaLaunchKernelEx(&cfg, decode_kernel<BITS, true>, p)
-               : cudaLaunchKernelEx(&cfg, decode_kernel<BITS, false>, p);
+  if (p.tm == kTmHad) return cudaLaunchKernelEx(&cfg, decode_kernel<BITS, kTmHad>, p);
+  if (p.tm == kTmQ8) return cudaLaunchKernelEx(&cfg, decode_kernel<BITS, kTmQ8>, p);
+  return cudaLaunchKernelEx(&cfg, decode_kernel<BITS, kTmCS>, p);
 }
 
 cudaError_t launch(const Params& p, cudaStream_t st) {
@@ -1015,8 +1075,7 @@ int chunk_cols_for(int bits) {
 }
 
 cudaError_t max_clusters(const Params& p, int* out) {
-  const bool had = p.had != 0;
-  const void* fn = p.bits == 2 ? kernel_ptr<2>(had) : (p.bits == 3 ? kernel_ptr<3>(had) : kernel_ptr<4>(had));
+  const void* fn = p.bits == 2 ? kernel_ptr<2>(p.tm) : (p.bits == 3 ? kernel_ptr<3>(p.tm) : kernel_ptr<4>(p.tm));
   const size_t smem = smem_for(p);
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

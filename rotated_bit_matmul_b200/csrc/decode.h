@@ -14,11 +14,16 @@ constexpr int kNT = 32 * kCW;        // consumer threads
 constexpr int kThreads = kNT + 64;   // + a weight-ring producer warp and a table producer warp
 constexpr int kMaxClusters = 64;
 
+// How the butterflies of a fused stack keep their angles (one kernel instantiation each):
+// kTmCS (cos, sin) fp32 pairs per rotation; kTmHad every butterfly Theta == 0 (no
+// parameters); kTmQ8 int8 angles with a per-stage step (a 64-byte head, then the codes).
+enum { kTmCS = 0, kTmHad = 1, kTmQ8 = 2 };
+
 // One linear as the fused kernel sees it (device array, 64-byte aligned for the maps).
 struct alignas(64) Lin {
   CUtensorMap tm_codes, tm_hi, tm_sz;
-  const float2* csV;
-  const float2* csU;
+  const uint8_t* tV;  // input-side angle storage in the stack's form (see kTm*), or null
+  const uint8_t* tU;  // output-side angle storage
   const int8_t* sV;
   const int8_t* sU;
   int n_in, n_out, w_in, w_out, m_in, m_out, pad0, pad1;
@@ -44,7 +49,7 @@ struct Params {
   float* xsum_down;
   unsigned* counters;  // [L][5], zero at launch
   int* status;
-  int had;  // every butterfly is Theta == 0 (the fixed randomized Hadamard transform)
+  int tm;   // kTmCS, kTmHad or kTmQ8: how every butterfly of the stack keeps its angles
   int ring_stages, tab_bytes, xq_bytes;
   int asg_qkv[kMaxClusters], idx_qkv[kMaxClusters], cnt_qkv[3];
   int asg_gu[kMaxClusters], idx_gu[kMaxClusters], cnt_gu[2];

@@ -17,6 +17,9 @@ constexpr int kMaxBatchGemv = 8; // batch rows the CUDA-core GEMV handles per la
 constexpr int kMaxW = 8192;      // widest butterfly block held by one CTA
 constexpr int kMinBatchMma = 16; // token batches from here on take the tensor-core path
 constexpr int kMaxBatch = 65535; // token rows per harp_linear_fwd call (a grid dimension)
+// int8 angle storage of one butterfly: a 64-byte head holding the fp32 step delta_t of
+// every stage (up to 16; log2 8192 = 13), then the codes int8 [m][n/2].
+constexpr int kQ8Head = 64;
 
 // Butterfly launch description. One CTA transforms one w-wide block of one row.
 struct BflyParams {
@@ -24,6 +27,7 @@ struct BflyParams {
   int w, m, inverse;
   const float* theta;  // [m][n/2] angle offsets (pi/4 added in-kernel) or null when cs is set
   const float2* cs;    // [m][n/2] (cos, sin) of pi/4 + theta, or null
+  const uint8_t* q8;   // int8 angles (kQ8Head bytes of fp32 steps, then int8 [m][n/2]), or null
   const int8_t* sign;  // [n]
   const void* x;
   int xt;
@@ -60,6 +64,8 @@ struct Layer {
   int bits, group, w_in, w_out, m_in, m_out;
   float2* csV;   // [m_in][n_in/2]
   float2* csU;   // [m_out][n_out/2]
+  uint8_t* q8V;  // int8 angle storage of the input side (kQ8Head + m_in * n_in/2 bytes), or null
+  uint8_t* q8U;  // int8 angle storage of the output side, or null
   int8_t* sV;
   int8_t* sU;
   const void* codes;
@@ -98,6 +104,8 @@ cudaError_t launch_gemv(const Layer& L, const GemvParams& p, cudaStream_t st);
 cudaError_t launch_quantize(int64_t n_out, int64_t n_in, int bits, const float* W, void* codes,
                             void* scale_zero, cudaStream_t st);
 cudaError_t launch_cs_table(const float* theta, int64_t count, float2* cs, cudaStream_t st);
+cudaError_t launch_quantize_angles(int m, int64_t half_n, const float* theta, int8_t* q, float* delta,
+                                   cudaStream_t st);
 
 // 2-D tiled tensor map over a row-major [rows][inner] array; false if the driver
 // entry point is missing or rejects the arguments.

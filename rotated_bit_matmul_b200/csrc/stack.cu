@@ -231,17 +231,37 @@ void setup_fused(harp_stack_s* S) {
     if (L[4]->w_out != wb || L[5]->w_out != wb || L[6]->w_in != wb) return no("gate/up output and down input blocks must match");
     if (L[6]->w_out != H) return no("down output butterfly must be hidden-wide");
   }
-  // every butterfly learned (cos/sin tables) or every one Theta == 0: one kernel
-  // instantiation per case, so neither pays for the other in its rotation rounds
-  bool any_learned = false, any_fixed = false;
+  // every butterfly in one form: fp32 angles (cos/sin tables), int8 angles, or Theta == 0.
+  // One kernel instantiation per form, so none pays for another in its rotation rounds.
+  int n_cs = 0, n_q8 = 0, n_had = 0;
   for (const harp_layer l : S->layers) {
-    any_learned |= l->L.csV != nullptr || l->L.csU != nullptr;
-    any_fixed |= l->L.csV == nullptr || l->L.csU == nullptr;
+    const Layer& L = l->L;
+    for (int side = 0; side < 2; ++side) {
+      const bool q8 = side ? L.q8U != nullptr : L.q8V != nullptr;
+      const bool cs = side ? L.csU != nullptr : L.csV != nullptr;
+      n_q8 += q8;
+      n_cs += cs && !q8;
+      n_had += !cs && !q8;
+    }
   }
-  if (any_learned && any_fixed) return no("mixing learned and Theta = 0 butterflies is not fused");
+  int tm = dec::kTmCS;
+  if (n_had && !n_cs && !n_q8)
+    tm = dec::kTmHad;
+  else if (n_q8 && !n_cs && !n_had)
+    tm = dec::kTmQ8;
+  else if (n_q8 || n_had)
+    return no("butterflies with fp32 angles, int8 angles and Theta = 0 are not fused together");
+  if (tm == dec::kTmQ8) {
+    // int8 slices are copied with 16-byte bulk copies: per-CTA runs of w/64 angles
+    for (int w : {H, dq, dkv})
+      if (w % 1024) return no("int8 angles need butterflies of widths that are multiples of 1024");
+    if (wb % 32) return no("int8 angles need MLP blocks of a multiple of 32");
+    for (const harp_layer l : S->layers)
+      if ((l->L.n_in / 2) % 16 || (l->L.n_out / 2) % 16) return no("int8 angles need n_in, n_out multiples of 32");
+  }
   dec::Params& p = S->fp;
   p = dec::Params{};
-  p.had = any_fixed ? 1 : 0;
+  p.tm = tm;
   p.L = S->n_layers;
   p.hidden = H;
   p.ffn = F;
@@ -254,11 +274,14 @@ void setup_fused(harp_stack_s* S) {
   p.E = H / dec::kC;
   p.m_hidden = ilog2(H);
   // shared-memory budget: tables of the largest chain, operand of the widest input
-  auto tb = [](int w) { return 8 * ilog2(w) * (w / dec::kC / 2); };
+  const int esz = tm == dec::kTmQ8 ? 1 : 8, head = tm == dec::kTmQ8 ? kQ8Head : 0;
+  auto tb = [&](int w) { return head + esz * ilog2(w) * (w / dec::kC / 2); };
   int tab = 2 * tb(H);
   tab = std::max(tab, tb(dkv) + tb(H));
+  tab = std::max(tab, tb(dq));
   const int wbm = ilog2(wb);
-  p.tab_bytes = std::max(tab, 3 * 4 * wb * wbm);
+  tab = std::max(tab, 3 * (head + esz * wbm * (wb / 2)));
+  p.tab_bytes = (tab + 15) & ~15;  // the sign slices after it take 16-byte bulk copies
   auto xqb = [&](int n) { return 4 * ((bits == 3 ? n : n / 2) + 2 * (n / 64)); };
   p.xq_bytes = (std::max(xqb(H), xqb(F)) + 15) & ~15;  // keeps the mbarriers after it 8-byte aligned
   int optin = 0;
@@ -288,8 +311,8 @@ void setup_fused(harp_stack_s* S) {
     d.tm_codes = L.tm_codes;
     d.tm_hi = L.tm_hi;
     d.tm_sz = L.tm_sz;
-    d.csV = L.csV;
-    d.csU = L.csU;
+    d.tV = L.q8V ? L.q8V : reinterpret_cast<const uint8_t*>(L.csV);
+    d.tU = L.q8U ? L.q8U : reinterpret_cast<const uint8_t*>(L.csU);
     d.sV = L.sV;
     d.sU = L.sU;
     d.n_in = (int)L.n_in;

@@ -8,7 +8,7 @@ sides of every parity test start from identical numbers.
 Seeds: ``numpy.random.default_rng([workload, layer, linear, role])``.
   workload: 1 single 1024x1024 layer, 2 the seven 7B decoder-layer linears,
             3 the batch sweep, 4 the 32-layer 7B stack, 5 the 80-layer 70B stack,
-            11 the calibration-objective cases.
+            11 the calibration-objective cases, 12 the int8-angle cases.
   linear:   0 q, 1 k, 2 v, 3 o, 4 gate, 5 up, 6 down, 7 = the step input.
   role:     0 W, 1 outlier columns, 2 theta_V, 3 s_V, 4 theta_U, 5 s_U, 6 x,
             7 calibration inputs.
