@@ -76,14 +76,16 @@ def algorithmic_bytes_per_step(n_layers, batch=BATCH, bits=BITS):
 
 
 # DRAM bytes (read + write) of one fused decode launch per transformer block, from the
-# ncu capture summarised in profiles/decode_kernel_llama2-7b_2bit_batch1.md (4-block
-# case, 271.18 MB per launch, scaled by blocks), and a hash of the kernel's sources at
-# capture time: the figure is reported only while those sources are unchanged.
-TRAFFIC_PER_BLOCK = {"bytes": 271_180_032 // 4, "sources_sha256_16": "9fd516eaca1dd9d2"}
+# ncu captures summarised in profiles/decode_kernel_llama2-7b_2bit_batch1.md (4-block
+# case, scaled by blocks): 270.97 MB per launch with fp32 cos/sin tables, 258.86 MB with
+# int8 angles. With them, a hash of the kernel's sources at capture time: the figures are
+# reported only while those sources are unchanged.
+TRAFFIC_PER_BLOCK = {"bytes": {"fp32": 270_965_248 // 4, "int8": 258_862_848 // 4},
+                     "sources_sha256_16": "a7a80626b48c905c"}
 KERNEL_SOURCES = ("decode.cu", "decode.h", "common.cuh", "gemv_core.cuh")
 
 
-def traffic_per_step(n_layers):
+def traffic_per_step(n_layers, angles="fp32"):
     import hashlib
     csrc = os.path.join(ROOT, "rotated_bit_matmul_b200", "csrc")
     h = hashlib.sha256()
@@ -92,7 +94,7 @@ def traffic_per_step(n_layers):
             h.update(fh.read())
     if h.hexdigest()[:16] != TRAFFIC_PER_BLOCK["sources_sha256_16"]:
         return None
-    return TRAFFIC_PER_BLOCK["bytes"] * n_layers
+    return TRAFFIC_PER_BLOCK["bytes"][angles] * n_layers
 
 
 def measured_peak():
@@ -306,7 +308,8 @@ def run_ours(args, rk):
     achieved = nbytes / (ms_step * 1e-3) / 1e9
     fused = stack.uses_fused_step(BATCH)
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": traffic_per_step(args.layers) if fused and not (args.rht or args.int8_angles) else None,
+                "frac": round(achieved / peak, 4), "traffic": (traffic_per_step(args.layers, "int8" if args.int8_angles else "fp32")
+                            if fused and not args.rht else None),
                 "kernel": "decode_kernel (one launch per step)" if fused else "whole decode step (graph of kernels)",
                 "peak_kind": peak_kind, "algorithmic_bytes_per_step": nbytes}
     del g
