@@ -61,6 +61,9 @@ def lib():
         L.ora_f16_to_f64.argtypes = [ctypes.c_uint16]
         L.ora_f16_to_f64.restype = ctypes.c_double
         L.ora_set_threads.argtypes = [_int]
+        L.ora_mr_mixer.argtypes = [_int, _dp, _dp]
+        L.ora_cayley.argtypes = [_int, _dp, _dp]
+        L.ora_mr_butterfly.argtypes = [_i64, _int, ctypes.POINTER(ctypes.c_int), _dp, _i8p, _dp, _int, _i64, _dp]
         L.ora_quantize_angles.argtypes = [_i64, _i64, _dp, _i8p, ctypes.POINTER(ctypes.c_float)]
         L.ora_calib_fit.argtypes = [_i64, _i64, _int, _int, _i64, _i64, _dp, _i8p, _dp, _i8p, _dp, _dp,
                                     ctypes.c_double, _dp, _dp, _dp]
@@ -245,6 +248,62 @@ def stack_step(layers, hidden, ffn, n_heads, n_kv_heads, head_dim, x, eps=1e-5):
     _check(lib().ora_stack_step(len(layers) // 7, arr, hidden, ffn, n_heads, n_kv_heads, head_dim,
                                 float(eps), x2.shape[0], _d(x2), _d(out)), "stack")
     return out.reshape(-1) if one else out
+
+
+def mr_param_count(b: int) -> int:
+    """Parameters of one b x b block: 1 angle for b = 2, b(b-1)/2 Cayley parameters above."""
+    return 1 if b == 2 else b * (b - 1) // 2
+
+
+def mr_theta_size(radices) -> int:
+    d = int(np.prod(radices))
+    return sum((d // b) * mr_param_count(b) for b in radices)
+
+
+def mr_mixer(b, M=None):
+    """G_b: Sylvester H_b / sqrt(b) for powers of two, else the positive-diagonal QR factor
+    of the fixed Gaussian M (HARP Sec. 2.2, base mixer)."""
+    G = np.zeros((b, b))
+    MM = _f64(M) if M is not None else None
+    _check(lib().ora_mr_mixer(int(b), _d(MM) if MM is not None else None, _d(G)), "mr_mixer")
+    return G
+
+
+def cayley(theta, b):
+    """(I - A)(I + A)^-1 for the skew-symmetric A of the b(b-1)/2 parameters (upper triangle,
+    row by row)."""
+    th = _f64(theta).reshape(-1)
+    assert th.size == b * (b - 1) // 2
+    Q = np.zeros((b, b))
+    _check(lib().ora_cayley(int(b), _d(th), _d(Q)), "cayley")
+    return Q
+
+
+def _mr(x, radices, theta, sign, gauss, inverse):
+    v = np.array(x, dtype=np.float64, copy=True, order="C")
+    d = v.shape[-1]
+    r = (ctypes.c_int * len(radices))(*[int(b) for b in radices])
+    th = _f64(theta).reshape(-1)
+    assert th.size == mr_theta_size(radices)
+    g = None
+    if gauss is not None:
+        g = np.concatenate([np.zeros(b * b) if m is None else _f64(m).reshape(-1) for b, m in zip(radices, gauss)])
+    sg = _i8(sign)
+    _check(lib().ora_mr_butterfly(d, len(radices), r, _d(th), sg.ctypes.data_as(_i8p), _d(g) if g is not None else None,
+                                  int(inverse), v.size // d, _d(v)), "mr_butterfly")
+    return v
+
+
+def mr_butterfly_fwd(x, radices, theta, sign, gauss=None):
+    """Mixed-radix F(theta, s, b) x over the last dimension (HARP Sec. 2.1): signs, then stage
+    t = 0..m-1 mixing the b_t coordinates that differ in mixed-radix digit t. gauss: one
+    b_t x b_t Gaussian per stage (None entries for powers of two)."""
+    return _mr(x, radices, theta, sign, gauss, False)
+
+
+def mr_butterfly_inv(x, radices, theta, sign, gauss=None):
+    """F^T x: the stage transposes from t = m-1 down to 0, then the signs."""
+    return _mr(x, radices, theta, sign, gauss, True)
 
 
 def quantize_angles(theta):

@@ -414,6 +414,194 @@ done:
   return rc;
 }
 
+/* ------------------------------------------------------------------ mixed-radix schedules
+ * HARP page, Sec. 2.1 (Suporte a Misto-Raiz) and Sec. 2.2: for d = b_0 b_1 ... b_{m-1},
+ * stage t applies a block-diagonal orthogonal matrix to groups of b_t coordinates that
+ * stride permutations bring together. Read here as mixed-radix digits:
+ *   stride s_t = b_0 ... b_{t-1}; index i has digit i_t = (i / s_t) mod b_t;
+ *   group c of stage t is the b_t indices base_c + j s_t (j = 0..b_t-1) that share every
+ *   other digit, groups numbered in increasing order of base_c:
+ *   base_c = (c mod s_t) + (c div s_t) s_t b_t.
+ * With every b_t = 2 this is the radix-2 butterfly above (pairs (i, i + 2^t)).
+ * Block B_{t,c} = Q_{t,c}(theta) G_{b_t}:
+ *   b = 2: the Givens block of the radix-2 butterfly, one angle offset;
+ *   b > 2: Q = (I - A)(I + A)^-1 (the Cayley map) of the skew-symmetric A whose strict upper
+ *          triangle holds the b(b-1)/2 parameters row by row (A_ij = theta, A_ji = -theta);
+ *          G_b = H_b / sqrt(b) (Sylvester) when b is a power of two, else the orthogonal
+ *          factor of the QR factorisation of a fixed Gaussian matrix M_b, with R's diagonal
+ *          made positive (which makes the factor unique).
+ * theta: stage after stage, group after group, the group's parameters in the order above.
+ * F = B_{m-1} ... B_0 D (signs first); F^T applies B_t^T from t = m-1 down to 0, then D.
+ */
+static int ora_mr_params(int b) { return b == 2 ? 1 : b * (b - 1) / 2; }
+
+static int ora_is_pow2(int b) { return b >= 1 && (b & (b - 1)) == 0; }
+
+/* G_b [b][b]: Sylvester H_b / sqrt(b), or the Q factor of M (row-major b x b) by modified
+ * Gram-Schmidt on its columns, each column orthogonalised twice, R's diagonal positive. */
+int ora_mr_mixer(int b, const double* M, double* G) {
+  if (b < 2) return ORA_EINVAL;
+  if (ora_is_pow2(b)) {
+    const double sc = 1.0 / sqrt((double)b);
+    for (int i = 0; i < b; ++i)
+      for (int j = 0; j < b; ++j) G[i * b + j] = (__builtin_popcount((unsigned)(i & j)) & 1) ? -sc : sc;
+    return ORA_OK;
+  }
+  if (!M) return ORA_EINVAL;
+  double* q = (double*)malloc(sizeof(double) * (size_t)b);
+  if (!q) return ORA_EINVAL;
+  for (int j = 0; j < b; ++j) {
+    for (int i = 0; i < b; ++i) q[i] = M[i * b + j];
+    for (int pass = 0; pass < 2; ++pass)
+      for (int k = 0; k < j; ++k) {
+        double dot = 0.0;
+        for (int i = 0; i < b; ++i) dot += G[i * b + k] * q[i];
+        for (int i = 0; i < b; ++i) q[i] -= dot * G[i * b + k];
+      }
+    double nrm = 0.0;
+    for (int i = 0; i < b; ++i) nrm += q[i] * q[i];
+    nrm = sqrt(nrm);
+    if (!(nrm > 0.0)) { free(q); return ORA_EINVAL; }
+    for (int i = 0; i < b; ++i) G[i * b + j] = q[i] / nrm;
+  }
+  free(q);
+  return ORA_OK;
+}
+
+/* Q = (I - A)(I + A)^-1 for the skew-symmetric A of the b(b-1)/2 parameters th;
+ * (I + A) is inverted by Gauss-Jordan elimination with partial pivoting. */
+int ora_cayley(int b, const double* th, double* Q) {
+  if (b < 2) return ORA_EINVAL;
+  const size_t bb = (size_t)b * (size_t)b;
+  double* A = (double*)calloc(bb, sizeof(double));
+  double* P = (double*)malloc(sizeof(double) * bb);   /* I + A, reduced in place */
+  double* X = (double*)malloc(sizeof(double) * bb);   /* becomes (I + A)^-1 */
+  if (!A || !P || !X) { free(A); free(P); free(X); return ORA_EINVAL; }
+  int k = 0;
+  for (int i = 0; i < b; ++i)
+    for (int j = i + 1; j < b; ++j, ++k) {
+      A[i * b + j] = th[k];
+      A[j * b + i] = -th[k];
+    }
+  for (int i = 0; i < b; ++i)
+    for (int j = 0; j < b; ++j) {
+      P[i * b + j] = (i == j ? 1.0 : 0.0) + A[i * b + j];
+      X[i * b + j] = i == j ? 1.0 : 0.0;
+    }
+  for (int col = 0; col < b; ++col) {
+    int piv = col;
+    for (int r = col + 1; r < b; ++r)
+      if (fabs(P[r * b + col]) > fabs(P[piv * b + col])) piv = r;
+    if (piv != col)
+      for (int j = 0; j < b; ++j) {
+        double t = P[col * b + j]; P[col * b + j] = P[piv * b + j]; P[piv * b + j] = t;
+        t = X[col * b + j]; X[col * b + j] = X[piv * b + j]; X[piv * b + j] = t;
+      }
+    const double dv = P[col * b + col];
+    for (int j = 0; j < b; ++j) { P[col * b + j] /= dv; X[col * b + j] /= dv; }
+    for (int r = 0; r < b; ++r) {
+      if (r == col) continue;
+      const double f = P[r * b + col];
+      if (f == 0.0) continue;
+      for (int j = 0; j < b; ++j) { P[r * b + j] -= f * P[col * b + j]; X[r * b + j] -= f * X[col * b + j]; }
+    }
+  }
+  for (int i = 0; i < b; ++i)
+    for (int j = 0; j < b; ++j) {
+      double acc = 0.0;
+      for (int l = 0; l < b; ++l) acc += ((i == l ? 1.0 : 0.0) - A[i * b + l]) * X[l * b + j];
+      Q[i * b + j] = acc;
+    }
+  free(A); free(P); free(X);
+  return ORA_OK;
+}
+
+/* The stage blocks B_{t,c} [groups][b][b] of one stage (b = 2 included, as a 2 x 2 matrix). */
+static int ora_mr_stage_blocks(int64_t d, int b, const double* th, const double* M, double* Bs) {
+  const int64_t groups = d / b;
+  const size_t bb = (size_t)b * (size_t)b;
+  if (b == 2) {
+    for (int64_t c = 0; c < groups; ++c) {
+      const double psi = ORA_PI / 4.0 + th[c], cs = cos(psi), sn = sin(psi);
+      double* B = Bs + (size_t)c * 4;
+      B[0] = cs; B[1] = sn; B[2] = sn; B[3] = -cs;
+    }
+    return ORA_OK;
+  }
+  double* G = (double*)malloc(sizeof(double) * bb);
+  double* Q = (double*)malloc(sizeof(double) * bb);
+  int rc = (G && Q) ? ora_mr_mixer(b, M, G) : ORA_EINVAL;
+  for (int64_t c = 0; c < groups && rc == ORA_OK; ++c) {
+    rc = ora_cayley(b, th + (size_t)c * (size_t)ora_mr_params(b), Q);
+    double* B = Bs + (size_t)c * bb;
+    for (int i = 0; i < b && rc == ORA_OK; ++i)
+      for (int j = 0; j < b; ++j) {
+        double acc = 0.0;
+        for (int l = 0; l < b; ++l) acc += Q[i * b + l] * G[l * b + j];
+        B[i * b + j] = acc;
+      }
+  }
+  free(G); free(Q);
+  return rc;
+}
+
+/* x [batch][d] in place. radix [m]; theta: every stage's parameters, stage after stage;
+ * gauss: every stage's b_t x b_t Gaussian, stage after stage (read only for radices that
+ * are not powers of two; may be NULL when there are none). */
+int ora_mr_butterfly(int64_t d, int m, const int* radix, const double* theta, const int8_t* sign,
+                     const double* gauss, int inverse, int64_t batch, double* x) {
+  if (m < 1 || d < 2 || batch < 0) return ORA_EINVAL;
+  int64_t prod = 1;
+  for (int t = 0; t < m; ++t) {
+    if (radix[t] < 2 || radix[t] > 256) return ORA_EINVAL;
+    prod *= radix[t];
+  }
+  if (prod != d) return ORA_EINVAL;
+  double** blocks = (double**)calloc((size_t)m, sizeof(double*));
+  if (!blocks) return ORA_EINVAL;
+  int rc = ORA_OK;
+  size_t toff = 0, goff = 0;
+  for (int t = 0; t < m && rc == ORA_OK; ++t) {
+    const int b = radix[t];
+    blocks[t] = (double*)malloc(sizeof(double) * (size_t)(d / b) * (size_t)b * (size_t)b);
+    if (!blocks[t]) { rc = ORA_EINVAL; break; }
+    rc = ora_mr_stage_blocks(d, b, theta + toff, gauss ? gauss + goff : NULL, blocks[t]);
+    toff += (size_t)(d / b) * (size_t)ora_mr_params(b);
+    goff += (size_t)b * (size_t)b;
+  }
+  if (rc == ORA_OK) {
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < batch; ++r) {
+      double* v = x + r * d;
+      double tmp[256], out[256];
+      if (!inverse)
+        for (int64_t i = 0; i < d; ++i) v[i] *= (double)sign[i];
+      for (int step = 0; step < m; ++step) {
+        const int t = inverse ? m - 1 - step : step;
+        const int b = radix[t];
+        int64_t st = 1;
+        for (int k = 0; k < t; ++k) st *= radix[k];
+        for (int64_t c = 0; c < d / b; ++c) {
+          const int64_t base = (c % st) + (c / st) * st * b;
+          const double* B = blocks[t] + (size_t)c * (size_t)b * (size_t)b;
+          for (int j = 0; j < b; ++j) tmp[j] = v[base + j * st];
+          for (int i = 0; i < b; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < b; ++j) acc += (inverse ? B[j * b + i] : B[i * b + j]) * tmp[j];
+            out[i] = acc;
+          }
+          for (int i = 0; i < b; ++i) v[base + i * st] = out[i];
+        }
+      }
+      if (inverse)
+        for (int64_t i = 0; i < d; ++i) v[i] *= (double)sign[i];
+    }
+  }
+  for (int t = 0; t < m; ++t) free(blocks[t]);
+  free(blocks);
+  return rc;
+}
+
 /* ------------------------------------------------------------------ int8 angles
  * The HARP page stores its parameters in int8 (Sec. 2.4, Armazenamento; Sec. 4, 2.00 ->
  * 2.05 bits per parameter at 2 bits). The format is this library's reading:

@@ -612,3 +612,140 @@ def test_angle_q8_butterfly_error_bound(ora):
     assert np.all(diff <= bound * np.linalg.norm(x, axis=1) * (1 + 1e-9))
     assert bound <= d.astype(np.float64).sum() / 2 * (1 + 1e-12)
     assert diff.max() > 0
+
+
+# ------------------------------------------------------------------ mixed-radix schedules
+def _mr_theta(rng, radices, scale):
+    return rng.uniform(-scale, scale, oracle_mr_size(radices))
+
+
+def oracle_mr_size(radices):
+    d = int(np.prod(radices))
+    return sum((d // b) * (1 if b == 2 else b * (b - 1) // 2) for b in radices)
+
+
+def _gauss(rng, radices):
+    return [None if (b & (b - 1)) == 0 else rng.standard_normal((b, b)) for b in radices]
+
+
+def _mr_dense(ora, radices, theta, sign, gauss=None, inverse=False):
+    d = int(np.prod(radices))
+    f = ora.mr_butterfly_inv if inverse else ora.mr_butterfly_fwd
+    return f(np.eye(d), radices, theta, sign, gauss).T
+
+
+def test_mr_all_radix2_is_the_butterfly(ora):
+    """Every b_t = 2: the mixed-radix schedule is the radix-2 butterfly, parameters in the
+    same stage-major, pair-numbered order."""
+    rng = np.random.default_rng(31)
+    d = 256
+    th = _rand_theta(rng, d, d, 0.3)
+    s = _rand_sign(rng, d)
+    x = rng.standard_normal((3, d))
+    rad = [2] * 8
+    assert np.allclose(ora.mr_butterfly_fwd(x, rad, th.reshape(-1), s), ora.butterfly_fwd(x, th, s, d), atol=1e-13)
+    assert np.allclose(ora.mr_butterfly_inv(x, rad, th.reshape(-1), s), ora.butterfly_inv(x, th, s, d), atol=1e-13)
+
+
+@pytest.mark.parametrize("radices", [(8, 8), (4, 2, 8), (16, 4), (2, 32), (64,)])
+def test_mr_hadamard_start_power_of_two(ora, radices):
+    """Theta = 0 with power-of-two radices: every block is a Sylvester H_b / sqrt(b) and
+    their Kronecker product over the digits is H_d (Sec. 2.2: HARP starts at the fixed
+    randomized Hadamard transform)."""
+    from scipy.linalg import hadamard
+    rng = np.random.default_rng(32)
+    d = int(np.prod(radices))
+    s = _rand_sign(rng, d)
+    F = _mr_dense(ora, radices, np.zeros(oracle_mr_size(radices)), s)
+    assert np.allclose(F, hadamard(d) * s[None, :] / np.sqrt(d), atol=1e-13)
+
+
+def test_mr_hadamard_start_kronecker_with_odd_radices(ora):
+    """Theta = 0, schedule (3, 4, 5): stage t mixes digit t (stride b_0...b_{t-1}), so F is
+    kron(G_5, G_4, G_3) D with the slowest digit's mixer leftmost."""
+    rng = np.random.default_rng(33)
+    rad = (3, 4, 5)
+    g = _gauss(rng, rad)
+    s = _rand_sign(rng, 60)
+    F = _mr_dense(ora, rad, np.zeros(oracle_mr_size(rad)), s, g)
+    G3, G4, G5 = ora.mr_mixer(3, g[0]), ora.mr_mixer(4), ora.mr_mixer(5, g[2])
+    assert np.allclose(F, np.kron(G5, np.kron(G4, G3)) * s[None, :], atol=1e-13)
+
+
+def test_mr_stages_as_stride_permutations(ora):
+    """The page's construction written independently with numpy axes: index i is the array
+    position (i_{m-1}, ..., i_0) of a C-ordered tensor; stage t moves axis m-1-t last (the
+    stride permutation), applies block c = B_{t,c} to row c of the remaining axes in C order,
+    and moves the axis back. Blocks from cayley() and mr_mixer()."""
+    rng = np.random.default_rng(34)
+    rad = (3, 2, 4, 5)
+    d = int(np.prod(rad))
+    th = _mr_theta(rng, rad, 0.4)
+    g = _gauss(rng, rad)
+    s = _rand_sign(rng, d)
+    x = rng.standard_normal(d)
+    v = (x * s).reshape(tuple(reversed(rad)))
+    off = 0
+    for t, b in enumerate(rad):
+        ax = len(rad) - 1 - t
+        rows = np.moveaxis(v, ax, -1).reshape(-1, b)
+        out = np.empty_like(rows)
+        for c in range(rows.shape[0]):
+            if b == 2:
+                p = np.pi / 4 + th[off + c]
+                B = np.array([[np.cos(p), np.sin(p)], [np.sin(p), -np.cos(p)]])
+            else:
+                k = b * (b - 1) // 2
+                B = ora.cayley(th[off + c * k: off + (c + 1) * k], b) @ ora.mr_mixer(b, g[t])
+            out[c] = B @ rows[c]
+        off += (d // b) * (1 if b == 2 else b * (b - 1) // 2)
+        shape = list(np.moveaxis(v, ax, -1).shape)
+        v = np.moveaxis(out.reshape(shape), -1, ax)
+    assert np.allclose(ora.mr_butterfly_fwd(x, rad, th, s, g), v.reshape(-1), atol=1e-13)
+
+
+def test_cayley_closed_forms(ora):
+    """Q(0) = I; for b = 2, A = [[0, a], [-a, 0]] gives [[1 - a^2, -2a], [2a, 1 - a^2]] / (1 + a^2);
+    Q is orthogonal with det +1; Q(-theta) = Q(theta)^T."""
+    assert np.allclose(ora.cayley(np.zeros(10), 5), np.eye(5), atol=0)
+    a = 0.37
+    want = np.array([[1 - a * a, -2 * a], [2 * a, 1 - a * a]]) / (1 + a * a)
+    assert np.allclose(ora.cayley([a], 2), want, atol=1e-15)
+    rng = np.random.default_rng(35)
+    for b in (3, 5, 8, 43):
+        th = rng.uniform(-0.8, 0.8, b * (b - 1) // 2)
+        Q = ora.cayley(th, b)
+        assert np.allclose(Q.T @ Q, np.eye(b), atol=1e-12)
+        assert abs(np.linalg.det(Q) - 1.0) < 1e-10
+        assert np.allclose(ora.cayley(-th, b), Q.T, atol=1e-12)
+
+
+def test_mr_mixer_properties(ora):
+    """Powers of two: H_b / sqrt(b). Otherwise G is orthogonal and G^T M is upper triangular
+    with a positive diagonal, which fixes G uniquely for an invertible M."""
+    from scipy.linalg import hadamard
+    for b in (2, 4, 16):
+        assert np.allclose(ora.mr_mixer(b), hadamard(b) / np.sqrt(b), atol=1e-15)
+    rng = np.random.default_rng(36)
+    for b in (3, 5, 7, 43):
+        M = rng.standard_normal((b, b))
+        G = ora.mr_mixer(b, M)
+        assert np.allclose(G.T @ G, np.eye(b), atol=1e-12)
+        R = G.T @ M
+        assert np.allclose(np.tril(R, -1), 0.0, atol=1e-11)
+        assert np.all(np.diag(R) > 0)
+
+
+@pytest.mark.parametrize("radices", [(8, 8, 8, 5, 2), (2, 2, 2, 2, 2, 2, 2, 2, 43)])
+def test_mr_orthogonal_at_page_sizes(ora, radices):
+    """The page's example schedule for d = 5120 (8, 8, 8, 5, 2), and 11008 = 2^8 43: norms are
+    kept and F^T undoes F, for random angles."""
+    rng = np.random.default_rng(37)
+    d = int(np.prod(radices))
+    th = _mr_theta(rng, radices, 0.2)
+    g = _gauss(rng, radices)
+    s = _rand_sign(rng, d)
+    x = rng.standard_normal((2, d))
+    y = ora.mr_butterfly_fwd(x, radices, th, s, g)
+    assert np.allclose(np.linalg.norm(y, axis=1), np.linalg.norm(x, axis=1), rtol=1e-12)
+    assert np.allclose(ora.mr_butterfly_inv(y, radices, th, s, g), x, atol=1e-12)
