@@ -100,6 +100,40 @@ harp_status harp_butterfly_inv(int64_t n, int w, int batch, const float* theta, 
 harp_status harp_quantize_weights(int64_t n_out, int64_t n_in, int bits, int group,
                                   const float* W_rot, void* codes, void* scale_zero, void* stream);
 
+/* ---------------------------------------------------------------- mixed-radix schedules
+ * HARP page, Sec. 2.1 (Suporte a Misto-Raiz) and 2.2: for d = b_0 b_1 ... b_{m-1} the
+ * rotation is signs, then stages t = 0..m-1, stage t mixing the b_t coordinates that differ
+ * only in mixed-radix digit t (stride b_0 ... b_{t-1}; group c starts at
+ * (c mod s_t) + (c div s_t) s_t b_t) with B_{t,c} = Q_{t,c}(theta) G_{b_t}:
+ *   b = 2: the Givens block of the radix-2 butterfly (one angle offset, pi/4 added inside);
+ *   b > 2: Q = (I - A)(I + A)^-1 (Cayley) of the skew-symmetric A whose strict upper
+ *          triangle holds the group's b(b-1)/2 parameters row by row; G_b = H_b / sqrt(b)
+ *          (Sylvester) for powers of two, else the orthogonal factor of the QR
+ *          factorisation of the stage's fixed Gaussian matrix, R's diagonal positive.
+ * With every b_t = 2 this is harp_butterfly_fwd with w = d.
+ * A plan computes every block once (fp64, stored fp32) and owns them.
+ *   d      : 2..16384, the product of the radices.    m: 1..32 stages.
+ *   radix  : HOST int [m], each in [2, 64].
+ *   theta  : device fp32, stage after stage, group after group, the group's parameters.
+ *   sign   : device int8 [d] (copied).
+ *   gauss  : device fp32, one b_t x b_t row-major matrix per stage, stage after stage
+ *            (entries of power-of-two stages are not read); NULL when every radix is a
+ *            power of two. The pages give no seed for it: it is the caller's input.
+ * Synchronises `stream` (the set-up is checked before returning). Errors:
+ * HARP_ERR_INVALID_ARG (sizes, radices, pointers, a singular Gaussian), HARP_ERR_CUDA. */
+typedef struct harp_mr_plan_s* harp_mr_plan;
+harp_status harp_mr_plan_create(harp_mr_plan* out, int64_t d, int m, const int* radix, const float* theta,
+                                const int8_t* sign, const float* gauss, void* stream);
+harp_status harp_mr_plan_destroy(harp_mr_plan plan);
+
+/* y = F x (fwd) or F^T x (inv: the stage transposes from t = m-1 down to 0, then the signs)
+ * for `batch` rows of d, row-major; dtypes f32/bf16/f16; y may equal x when xt == yt;
+ * pointers 16-byte aligned. Arithmetic is fp32. */
+harp_status harp_mr_butterfly_fwd(harp_mr_plan plan, int batch, const void* x, harp_dtype xt, void* y,
+                                  harp_dtype yt, void* stream);
+harp_status harp_mr_butterfly_inv(harp_mr_plan plan, int batch, const void* x, harp_dtype xt, void* y,
+                                  harp_dtype yt, void* stream);
+
 /* ---------------------------------------------------------------- int8 angles
  * The HARP page stores its parameters in int8 (Sec. 2.4, Armazenamento, and Sec. 4:
  * 2.00 -> 2.05 bits per parameter at 2 bits); the format is this library's:

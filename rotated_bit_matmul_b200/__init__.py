@@ -19,7 +19,7 @@ import math
 from ._lib import (HARP_BF16, HARP_F16, HARP_F32, HarpError, call, load)  # noqa: F401
 
 __all__ = ["HarpError", "harp_butterfly_fwd", "harp_butterfly_inv", "harp_quantize_weights", "HarpLayer",
-           "HarpStack", "rotate_weights_device", "harp_quantize_angles", "harp_calib_fit", "harp_device_status", "load"]
+           "HarpStack", "HarpMixedRadix", "rotate_weights_device", "harp_quantize_angles", "harp_calib_fit", "harp_device_status", "load"]
 
 
 def _torch():
@@ -203,6 +203,55 @@ class HarpLayer:
     def close(self):
         if getattr(self, "handle", None) is not None and self.handle.value:
             call("harp_destroy_layer", self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class HarpMixedRadix:
+    """A mixed-radix butterfly (wraps harp_mr_plan_*): d = prod(radices), stage t mixing the
+    coordinates that differ in mixed-radix digit t with Q(theta) G_b blocks (Givens for
+    b = 2, Cayley times the base mixer above). theta: fp32, stage after stage, group after
+    group; gauss: one b x b fp32 Gaussian per stage (None when every radix is a power of two)."""
+
+    def __init__(self, radices, theta, sign, gauss=None):
+        _need_cuda(theta, sign, gauss)
+        self.radices = [int(b) for b in radices]
+        self.d = int(math.prod(self.radices))
+        want = sum((self.d // b) * (1 if b == 2 else b * (b - 1) // 2) for b in self.radices)
+        if theta.numel() != want:
+            raise ValueError(f"theta has {theta.numel()} parameters, the schedule needs {want}")
+        if gauss is not None and gauss.numel() != sum(b * b for b in self.radices):
+            raise ValueError("gauss needs one b x b matrix per stage")
+        r = (ctypes.c_int * len(self.radices))(*self.radices)
+        h = ctypes.c_void_p()
+        self.handle = None
+        call("harp_mr_plan_create", ctypes.byref(h), self.d, len(self.radices), r, _p(theta.float().contiguous()),
+             _p(sign.contiguous()), _p(gauss.float().contiguous() if gauss is not None else None), _stream())
+        self.handle = h
+
+    def _apply(self, name, x, out_dtype, out):
+        torch = _torch()
+        _need_cuda(x)
+        x2 = x.reshape(-1, self.d).contiguous()
+        if out is None:
+            out = torch.empty(x2.shape, dtype=out_dtype or x.dtype, device=x.device)
+        call(name, self.handle, x2.shape[0], _p(x2), _dt(x2), _p(out), _dt(out), _stream())
+        return out.reshape(x.shape)
+
+    def fwd(self, x, out_dtype=None, out=None):
+        return self._apply("harp_mr_butterfly_fwd", x, out_dtype, out)
+
+    def inv(self, x, out_dtype=None, out=None):
+        return self._apply("harp_mr_butterfly_inv", x, out_dtype, out)
+
+    def close(self):
+        if getattr(self, "handle", None) is not None and self.handle.value:
+            call("harp_mr_plan_destroy", self.handle)
             self.handle = None
 
     def __del__(self):

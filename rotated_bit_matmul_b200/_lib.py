@@ -40,6 +40,10 @@ SIGNATURES = {
     "harp_stack_workspace_size": (_I, [_P, _I, ctypes.POINTER(_SZ)]),
     "harp_stack_step": (_I, [_P, _I, _P, _I, _P, _I, _P, _SZ, _P]),
     "harp_stack_uses_fused_step": (_I, [_P, _I]),
+    "harp_mr_plan_create": (_I, [ctypes.POINTER(_P), _I64, _I, ctypes.POINTER(ctypes.c_int), _P, _P, _P, _P]),
+    "harp_mr_plan_destroy": (_I, [_P]),
+    "harp_mr_butterfly_fwd": (_I, [_P, _I, _P, _I, _P, _I, _P]),
+    "harp_mr_butterfly_inv": (_I, [_P, _I, _P, _I, _P, _I, _P]),
     "harp_quantize_angles": (_I, [_I, _I64, _P, _P, _P, _P]),
     "harp_create_layer_q8": (_I, [ctypes.POINTER(_P), _I64, _I64, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P,
                                   _P]),

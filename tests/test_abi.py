@@ -171,3 +171,22 @@ def test_calib_rejects_misaligned_pointers_and_negative_lambda(lib):
     assert _calib(lib, 4096, 4096, 2, 64, 4096, 4096, H=MIS) == 1
     assert _calib(lib, 4096, 4096, 2, 64, 4096, 4096, loss=None) == 1
     assert _calib(lib, 4096, 4096, 2, 64, 4096, 4096, lam=-1.0) == 1
+
+
+def test_mr_plan_rejects_bad_arguments(lib):
+    """Validation of the mixed-radix plan happens before any CUDA call."""
+    h = ctypes.c_void_p()
+
+    def create(d, radices, gauss=None, theta=FAKE):
+        r = (ctypes.c_int * len(radices))(*radices)
+        return lib.harp_mr_plan_create(ctypes.byref(h), d, len(radices), r, theta, FAKE, gauss, None)
+
+    assert create(60, [3, 4, 5]) == 1            # odd radices without their Gaussian
+    assert create(64, [8, 4]) == 1               # radices do not multiply to d
+    assert create(128, [2, 64, 1]) == 1          # radix below 2
+    assert create(16384 * 2, [128, 256]) == 1    # d too large, radices too large
+    assert create(64, [8, 8], theta=MIS) == 1    # misaligned theta
+    assert create(64, [8, 8], theta=None) == 1   # null theta
+    assert not h.value
+    assert lib.harp_mr_plan_destroy(None) == 0
+    assert lib.harp_mr_butterfly_fwd(None, 1, FAKE, 0, FAKE, 0, None) == 1
