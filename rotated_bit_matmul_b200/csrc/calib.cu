@@ -380,12 +380,9 @@ cudaError_t rows(const float* x, float* y, int64_t n, int w, int64_t batch, cons
 // Backward through `batch` rows of a butterfly, adding dL/dtheta into gacc (fp64).
 cudaError_t rows_back(float* y, float* g, int64_t n, int w, int64_t batch, const float* theta, const int8_t* sign,
                       int inverse, float* part, double* gacc, cudaStream_t st) {
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(bfly_back_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kBackSmem);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  // the opt-in is per device and cheap to repeat, so it is set on every call
+  cudaError_t e = cudaFuncSetAttribute(bfly_back_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kBackSmem);
+  if (e != cudaSuccess) return e;
   BackParams p{};
   p.n = n;
   p.w = w;
@@ -401,7 +398,7 @@ cudaError_t rows_back(float* y, float* g, int64_t n, int w, int64_t batch, const
   p.R = back_rows(w);
   p.part = part;
   const int64_t np = (int64_t)p.m * (n / 2);
-  cudaError_t e = cudaMemsetAsync(part, 0, sizeof(float) * (size_t)nch * (size_t)np, st);
+  e = cudaMemsetAsync(part, 0, sizeof(float) * (size_t)nch * (size_t)np, st);
   if (e != cudaSuccess) return e;
   const size_t smem = sizeof(float) * 2 * (size_t)p.R * (size_t)w;
   bfly_back_kernel<<<dim3((unsigned)(n / w), (unsigned)nch), kBackThreads, smem, st>>>(p);
