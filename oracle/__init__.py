@@ -306,6 +306,52 @@ def mr_butterfly_inv(x, radices, theta, sign, gauss=None):
     return _mr(x, radices, theta, sign, gauss, True)
 
 
+class MixedRadixSide:
+    """One side of a linear with a mixed-radix butterfly: radices, parameters (stage after
+    stage), signs and one Gaussian per stage (None for powers of two)."""
+
+    def __init__(self, radices, theta, sign, gauss=None):
+        self.radices = [int(b) for b in radices]
+        self.theta = _f64(theta).reshape(-1)
+        self.sign = _i8(sign)
+        self.gauss = gauss
+
+    def fwd(self, x):
+        return mr_butterfly_fwd(x, self.radices, self.theta, self.sign, self.gauss)
+
+    def inv(self, x):
+        return mr_butterfly_inv(x, self.radices, self.theta, self.sign, self.gauss)
+
+
+def mr_rotate_weights(W, V: MixedRadixSide, U: MixedRadixSide):
+    """W' = U W V^T with V = F_V and U = F_U^T: rows through F_V, then columns through F_U^T."""
+    Wr = V.fwd(_f64(W))
+    return np.ascontiguousarray(U.inv(np.ascontiguousarray(Wr.T)).T)
+
+
+def mr_prepare_layer(W, bits, V: MixedRadixSide, U: MixedRadixSide, group=64):
+    """Rotate with mixed-radix sides, quantize and pack; returns (layer dict, W')."""
+    Wr = mr_rotate_weights(W, V, U)
+    q, s, z = quantize(Wr, bits, group)
+    return dict(V=V, U=U, bits=int(bits), group=int(group), packed=pack(q, bits), sz=scale_zero(s, z),
+                n_out=Wr.shape[0], n_in=Wr.shape[1]), Wr
+
+
+def mr_linear_fwd(layer, x):
+    """y = F_U(deq(codes) F_V(x)) for a mixed-radix layer: the codes are unpacked, each
+    dequantized to scale16 q + zero16 of its group, and applied as a dense matrix."""
+    x = _f64(x)
+    one = x.ndim == 1
+    x2 = x.reshape(1, -1) if one else x
+    n_out, n_in, g = layer["n_out"], layer["n_in"], layer["group"]
+    q = unpack(layer["packed"], n_out, n_in, layer["bits"]).astype(np.float64)
+    sz = np.asarray(layer["sz"], np.uint16).reshape(n_out, n_in // g, 2)
+    s = np.repeat(f16_to_f64(sz[:, :, 0]), g, axis=1)
+    z = np.repeat(f16_to_f64(sz[:, :, 1]), g, axis=1)
+    y = layer["U"].fwd((layer["V"].fwd(x2)) @ (s * q + z).T)
+    return y.reshape(-1) if one else y
+
+
 def quantize_angles(theta):
     """int8 angle storage: (q int8 [m, n/2], delta fp32 [m]) with one symmetric step per
     stage, delta_t = fp32(max |theta_t| / 127), q = RNE(theta / delta_t) clamped to +-127."""

@@ -749,3 +749,51 @@ def test_mr_orthogonal_at_page_sizes(ora, radices):
     y = ora.mr_butterfly_fwd(x, radices, th, s, g)
     assert np.allclose(np.linalg.norm(y, axis=1), np.linalg.norm(x, axis=1), rtol=1e-12)
     assert np.allclose(ora.mr_butterfly_inv(y, radices, th, s, g), x, atol=1e-12)
+
+
+def _mr_side(ora, rng, radices, scale=0.2):
+    d = int(np.prod(radices))
+    return ora.MixedRadixSide(radices, rng.uniform(-scale, scale, oracle_mr_size(radices)), _rand_sign(rng, d),
+                              _gauss(rng, radices))
+
+
+def test_mr_linear_exact_change_of_basis(ora):
+    """Sec. 5 with mixed-radix sides: F_U(W' F_V x) = W x for the unquantized W' = U W V^T,
+    with odd radices on both sides (n_in = 192 = 3 4 16, n_out = 40 = 5 8)."""
+    rng = np.random.default_rng(41)
+    V, U = _mr_side(ora, rng, (3, 4, 16)), _mr_side(ora, rng, (5, 8))
+    W = rng.standard_normal((40, 192))
+    Wr = ora.mr_rotate_weights(W, V, U)
+    x = rng.standard_normal((3, 192))
+    assert np.allclose(U.fwd(V.fwd(x) @ Wr.T), x @ W.T, atol=1e-12)
+
+
+def test_mr_linear_all_radix2_is_the_linear(ora):
+    """All-radix-2 sides: the mixed-radix layer is the radix-2 layer of the same angles,
+    codes and output."""
+    rng = np.random.default_rng(42)
+    n_in, n_out = 256, 128
+    thV, thU = _rand_theta(rng, n_in, n_in, 0.05), _rand_theta(rng, n_out, n_out, 0.05)
+    sV, sU = _rand_sign(rng, n_in), _rand_sign(rng, n_out)
+    W = rng.standard_normal((n_out, n_in)) * 0.02
+    V = ora.MixedRadixSide([2] * 8, thV.reshape(-1), sV)
+    U = ora.MixedRadixSide([2] * 7, thU.reshape(-1), sU)
+    mr, _ = ora.mr_prepare_layer(W, 2, V, U)
+    lay = ora.prepare_layer(W, 2, n_in, n_out, thV, sV, thU, sU)[0]
+    assert np.array_equal(mr["packed"], lay.packed) and np.array_equal(mr["sz"], lay.sz)
+    x = rng.standard_normal((2, n_in))
+    assert np.allclose(ora.mr_linear_fwd(mr, x), ora.linear_fwd(lay, x), atol=1e-12)
+
+
+def test_mr_linear_dequantizes_its_own_codes(ora):
+    """The mixed-radix linear applies exactly scale16 q + zero16 of quantize()'s output,
+    through its packed codes and scale/zero words."""
+    rng = np.random.default_rng(43)
+    V, U = _mr_side(ora, rng, (3, 64)), _mr_side(ora, rng, (5, 8))
+    W = rng.standard_normal((40, 192)) * 0.02
+    mr, Wr = ora.mr_prepare_layer(W, 3, V, U)
+    q, s16, z16 = ora.quantize(Wr, 3)
+    deq = np.repeat(s16.view(np.float16).astype(np.float64), 64, axis=1) * q + \
+        np.repeat(z16.view(np.float16).astype(np.float64), 64, axis=1)
+    x = rng.standard_normal((2, 192))
+    assert np.allclose(ora.mr_linear_fwd(mr, x), U.fwd(V.fwd(x) @ deq.T), atol=1e-12)
