@@ -51,7 +51,7 @@ extern "C" {
 typedef enum {
   HARP_OK = 0,
   HARP_ERR_INVALID_ARG = 1, /* bad size, alignment, null pointer, unsupported width */
-  HARP_ERR_UNSUPPORTED = 2, /* valid request this build does not implement */
+  HARP_ERR_UNSUPPORTED = 2, /* a valid request the library does not implement */
   HARP_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
   HARP_ERR_WORKSPACE = 4,   /* workspace missing or smaller than the query returned */
   HARP_ERR_TIMEOUT = 5,     /* a bounded device-side wait ran out (device status) */
