@@ -346,8 +346,9 @@ def mr_linear_fwd(layer, x):
     n_out, n_in, g = layer["n_out"], layer["n_in"], layer["group"]
     q = unpack(layer["packed"], n_out, n_in, layer["bits"]).astype(np.float64)
     sz = np.asarray(layer["sz"], np.uint16).reshape(n_out, n_in // g, 2)
-    s = np.repeat(f16_to_f64(sz[:, :, 0]), g, axis=1)
-    z = np.repeat(f16_to_f64(sz[:, :, 1]), g, axis=1)
+    # fp16 -> fp64 is exact; numpy's conversion serves as the library step
+    s = np.repeat(np.ascontiguousarray(sz[:, :, 0]).view(np.float16).astype(np.float64), g, axis=1)
+    z = np.repeat(np.ascontiguousarray(sz[:, :, 1]).view(np.float16).astype(np.float64), g, axis=1)
     y = layer["U"].fwd((layer["V"].fwd(x2)) @ (s * q + z).T)
     return y.reshape(-1) if one else y
 
