@@ -75,9 +75,9 @@ def algorithmic_bytes_per_step(n_layers, batch=BATCH, bits=BITS):
     return tot * n_layers
 
 
-# DRAM bytes (read + write) of one fused decode launch per transformer block, from the
-# ncu captures summarised in profiles/decode_kernel_llama2-7b_2bit_batch1.md (4-block
-# case, scaled by blocks): 270.97 MB per launch with fp32 cos/sin tables, 258.86 MB with
+# DRAM bytes (read + write) of one fused decode launch per transformer block, from an
+# ncu capture of the 4-block stack (dram__bytes_read.sum + dram__bytes_write.sum, scaled
+# by blocks): 270.97 MB per launch with fp32 cos/sin tables, 258.86 MB with
 # int8 angles. With them, a hash of the kernel's sources at capture time: the figures are
 # reported only while those sources are unchanged.
 TRAFFIC_PER_BLOCK = {"bytes": {"fp32": 270_965_248 // 4, "int8": 258_862_848 // 4},

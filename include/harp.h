@@ -70,6 +70,20 @@ const char* harp_last_error(void);
  * Synchronises `stream` first. */
 harp_status harp_device_status(void* stream);
 
+/* Testing hook for the failure paths; everything is off by default and the paper has no
+ * counterpart. It applies process-wide to launches made after it:
+ *   wait_limit_us   : > 0 bounds the device-side waits of harp_linear_fwd's dequant-GEMV and of
+ *                     the fused decode step by that many microseconds (0 restores the default,
+ *                     about 1-2 s);
+ *   gemv_skip_stage : >= 0 makes the first CTA of the dequant-GEMV skip issuing that stage of
+ *                     its weight ring, so its consumers' wait runs out (-1: off);
+ *   decode_barrier  : >= 0 raises the arrival target of that grid barrier of the fused decode
+ *                     step (index 5 * block + phase) by one, so no CTA passes it (-1: off).
+ * A wait that runs out records HARP_ERR_TIMEOUT and its site in the device status word and
+ * ends the kernel after waiting (bounded) for its copies in flight; no GPU fault is raised.
+ * Returns HARP_ERR_INVALID_ARG for negative values other than -1. */
+harp_status harp_test_set_faults(int wait_limit_us, int gemv_skip_stage, int decode_barrier);
+
 /* ---------------------------------------------------------------- butterfly
  * y = F(theta, s, w) x for `batch` rows of n (row-major, contiguous).
  * Sec. 2.1-2.2 of the HARP page: signs, then stages of stride 1, 2, ..., w/2.
@@ -259,8 +273,12 @@ harp_status harp_linear_fwd(harp_layer layer, int batch, const void* x, harp_dty
  *   x, y  : as for harp_linear_fwd (caller-owned device memory); no workspace argument.
  *   Fails with HARP_ERR_WORKSPACE when the layer and batch need more than 2 MiB of
  *   scratch (harp_linear_workspace_size says how much).
- *   The first call on a device looks up the array's device address; make that first
- *   call before any stream capture. All calls on a device share the array and it keeps
+ *   The first call on a device looks up the array's device address; under CUDA's lazy
+ *   module loading that lookup also loads the part of the library holding the array, so
+ *   the 2 MiB are taken from the device at that first call. Make that first call before
+ *   any stream capture; later calls take no device memory. Batches as for
+ *   harp_linear_fwd (1..65535), as far as their scratch fits. All calls on a device
+ *   share the array and it keeps
  *   the last call's contents (nothing in it must start at zero): calls that overlap on
  *   the GPU (other streams, other host threads) race, so serialise them.
  *   Allocates nothing (no cudaMalloc, cudaFree or allocating library routine); for the

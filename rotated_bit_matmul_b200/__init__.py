@@ -19,7 +19,8 @@ import math
 from ._lib import (HARP_BF16, HARP_F16, HARP_F32, HarpError, call, load)  # noqa: F401
 
 __all__ = ["HarpError", "harp_butterfly_fwd", "harp_butterfly_inv", "harp_quantize_weights", "HarpLayer",
-           "HarpStack", "HarpMixedRadix", "rotate_weights_device", "harp_quantize_angles", "harp_calib_fit", "harp_device_status", "load"]
+           "HarpStack", "HarpMixedRadix", "rotate_weights_device", "harp_quantize_angles", "harp_calib_fit", "harp_device_status",
+           "harp_test_set_faults", "load"]
 
 
 def _torch():
@@ -53,6 +54,13 @@ def _need_cuda(*ts):
 def harp_device_status() -> None:
     """Raises HarpError if a kernel reported a device-side failure (clears it)."""
     call("harp_device_status", _stream())
+
+
+def harp_test_set_faults(wait_limit_us: int = 0, gemv_skip_stage: int = -1, decode_barrier: int = -1) -> None:
+    """Testing hook for the failure paths (process-wide; the defaults switch it off): a short
+    bound on device-side waits, a weight-ring stage the dequant-GEMV's first CTA never
+    issues, a grid barrier of the fused decode step that can never complete."""
+    call("harp_test_set_faults", int(wait_limit_us), int(gemv_skip_stage), int(decode_barrier))
 
 
 def _bfly(name, x, theta, sign, w, out_dtype=None, out=None):

@@ -27,6 +27,7 @@ _SZ = ctypes.c_size_t
 SIGNATURES = {
     "harp_last_error": (ctypes.c_char_p, []),
     "harp_device_status": (_I, [_P]),
+    "harp_test_set_faults": (_I, [_I, _I, _I]),
     "harp_butterfly_fwd": (_I, [_I64, _I, _I, _P, _P, _P, _I, _P, _I, _P]),
     "harp_butterfly_inv": (_I, [_I64, _I, _I, _P, _P, _P, _I, _P, _I, _P]),
     "harp_quantize_weights": (_I, [_I64, _I64, _I, _I, _P, _P, _P, _P]),

@@ -2,6 +2,7 @@
 // workspace layout and kernel dispatch. Declarations and contracts: include/harp.h.
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -236,6 +237,9 @@ harp_status linear_forward_status(const Layer& L, int batch, const void* x, int 
 
     for (int b0 = 0; b0 < batch; b0 += kMaxBatchGemv) {
       GemvParams gp{};
+      const TestHooks th = test_hooks();
+      gp.wait_ns = th.wait_ns;
+      gp.skip_stage = th.gemv_skip_stage;
       gp.n_out = (int)L.n_out;
       gp.n_in = (int)L.n_in;
       gp.bits = L.bits;
@@ -275,6 +279,24 @@ harp_status linear_forward_status(const Layer& L, int batch, const void* x, int 
 
 harp_status device_status_for_kernels(int** out) { return device_status_ptr(out); }
 
+namespace {
+std::atomic<uint64_t> g_hook_wait_ns{0};
+std::atomic<long long> g_hook_wait_cycles{0};
+std::atomic<int> g_hook_gemv_skip{-1};
+std::atomic<int> g_hook_barrier_extra{-1};
+}  // namespace
+
+TestHooks test_hooks() {
+  TestHooks h;
+  const uint64_t ns = g_hook_wait_ns.load();
+  const long long cyc = g_hook_wait_cycles.load();
+  h.wait_ns = ns ? ns : 1000000000ull;         // 1 s of wall time
+  h.wait_cycles = cyc ? cyc : 4000000000ll;    // about 2 s of SM clock at 1.97 GHz
+  h.gemv_skip_stage = g_hook_gemv_skip.load();
+  h.decode_barrier_extra = g_hook_barrier_extra.load();
+  return h;
+}
+
 harp_status set_error(harp_status st, const char* fmt, ...) {
   char buf[512];
   va_list ap;
@@ -290,6 +312,17 @@ harp_status set_error(harp_status st, const char* fmt, ...) {
 extern "C" {
 
 const char* harp_last_error(void) { return g_last_error.c_str(); }
+
+harp_status harp_test_set_faults(int wait_limit_us, int gemv_skip_stage, int decode_barrier) {
+  if (wait_limit_us < 0 || gemv_skip_stage < -1 || decode_barrier < -1)
+    return fail(HARP_ERR_INVALID_ARG, "test_set_faults: negative limit or index");
+  g_hook_wait_ns.store((uint64_t)wait_limit_us * 1000ull);
+  // the fused step counts SM clock cycles: 2 per nanosecond covers clocks up to 2 GHz
+  g_hook_wait_cycles.store((long long)wait_limit_us * 2000ll);
+  g_hook_gemv_skip.store(gemv_skip_stage);
+  g_hook_barrier_extra.store(decode_barrier);
+  return HARP_OK;
+}
 
 harp_status harp_device_status(void* stream) {
   int* status = nullptr;

@@ -140,6 +140,7 @@ __global__ void __launch_bounds__(kBflyThreads) bfly_kernel(BflyParams p, int C)
   // need 16-byte aligned sources, destinations and sizes; tiny widths use plain loads.
   const bool use_bulk = !rht && (((E >> 1) * esz) % 16 == 0) && ((half_n * esz) % 16 == 0) &&
                         (((w >> 1) * esz) % 16 == 0) && (C == 1 || (run * esz) % 16 == 0);
+  bool ok = true;  // false once a bounded wait has run out
   if (rht) {
     // nothing to prefetch
   } else if (!use_bulk) {
@@ -192,24 +193,29 @@ __global__ void __launch_bounds__(kBflyThreads) bfly_kernel(BflyParams p, int C)
       xa[i] = v * (float)p.sign[gi];
     }
     __syncthreads();
-    if (use_bulk) mbar_wait(bar, 0, p.status, 10);
-    for (int t = 0; t < g.e; ++t) {
-      stage_a<TM>(xa, stab ? stab + (size_t)t * (E >> 1) * esz : nullptr, step_of(t), t, E, tid, nthr);
-      __syncthreads();
-    }
+    // a parameter copy that never lands ends this CTA's work (the status word says where);
+    // the cluster barriers the peers expect are still taken
+    if (use_bulk) ok = __syncthreads_and(mbar_wait(bar, 0, p.status, 10)) != 0;
+    if (ok)
+      for (int t = 0; t < g.e; ++t) {
+        stage_a<TM>(xa, stab ? stab + (size_t)t * (E >> 1) * esz : nullptr, step_of(t), t, E, tid, nthr);
+        __syncthreads();
+      }
     float* out = xa;
     if (C > 1) {
       cluster_sync();
-      for (int L = tid; L < E; L += nthr) {
-        const int j = L / run, ii = L - j * run;
-        xb[L] = ld_dsmem(xa + r * run + ii, (uint32_t)j);
-      }
+      if (ok)
+        for (int L = tid; L < E; L += nthr) {
+          const int j = L / run, ii = L - j * run;
+          xb[L] = ld_dsmem(xa + r * run + ii, (uint32_t)j);
+        }
       cluster_sync();  // every peer has finished reading this CTA's chunk
-      for (int d = 0; d < g.lc; ++d) {
-        stage_b<TM>(xb, stab ? stab + (size_t)(g.e + d) * (E >> 1) * esz : nullptr, step_of(g.e + d), d, run, E, tid,
-                    nthr);
-        __syncthreads();
-      }
+      if (ok)
+        for (int d = 0; d < g.lc; ++d) {
+          stage_b<TM>(xb, stab ? stab + (size_t)(g.e + d) * (E >> 1) * esz : nullptr, step_of(g.e + d), d, run, E,
+                      tid, nthr);
+          __syncthreads();
+        }
       out = xb;
     }
     // local index L <-> global element: layout A: r E + L; layout B: j E + r run + ii
@@ -218,9 +224,9 @@ __global__ void __launch_bounds__(kBflyThreads) bfly_kernel(BflyParams p, int C)
       const int j = L / run, ii = L - j * run;
       return base + (int64_t)j * E + (int64_t)r * run + ii;
     };
-    if (p.y)
+    if (ok && p.y)
       for (int L = tid; L < E; L += nthr) store_act(p.y, row * p.y_stride + gidx(L), p.yt, out[L]);
-    if (p.xq) {
+    if (ok && p.xq) {
       // groups of 64 consecutive outputs (runs are >= 64 long): int16 at scale 2^e with
       // max|v| 2^e < 2^15 (e = 15 - E', max|v| = f 2^E', f in [0.5, 1))
       const int lane = tid & 31, warp = tid >> 5, nwarps = nthr >> 5;
@@ -264,32 +270,39 @@ __global__ void __launch_bounds__(kBflyThreads) bfly_kernel(BflyParams p, int C)
         xb[L] = load_act(p.x, row * p.x_stride + base + (int64_t)j * E + (int64_t)r * run + ii, p.xt);
       }
       __syncthreads();
-      if (use_bulk) mbar_wait(bar, 0, p.status, 11);
-      for (int d = g.lc - 1; d >= 0; --d) {
-        stage_b<TM>(xb, stab ? stab + (size_t)(g.e + d) * (E >> 1) * esz : nullptr, step_of(g.e + d), d, run, E, tid,
-                    nthr);
-        __syncthreads();
-      }
+      if (use_bulk) ok = __syncthreads_and(mbar_wait(bar, 0, p.status, 11)) != 0;
+      if (ok)
+        for (int d = g.lc - 1; d >= 0; --d) {
+          stage_b<TM>(xb, stab ? stab + (size_t)(g.e + d) * (E >> 1) * esz : nullptr, step_of(g.e + d), d, run, E,
+                      tid, nthr);
+          __syncthreads();
+        }
       cluster_sync();
-      for (int u = tid; u < E; u += nthr) {
-        const int q = u / run;  // owner CTA of chunk-r element u in layout B
-        xa[u] = ld_dsmem(xb + r * run + (u - q * run), (uint32_t)q);
-      }
+      if (ok)
+        for (int u = tid; u < E; u += nthr) {
+          const int q = u / run;  // owner CTA of chunk-r element u in layout B
+          xa[u] = ld_dsmem(xb + r * run + (u - q * run), (uint32_t)q);
+        }
       cluster_sync();
     } else {
       for (int i = tid; i < E; i += nthr) xa[i] = load_act(p.x, row * p.x_stride + base + i, p.xt);
       __syncthreads();
-      if (use_bulk) mbar_wait(bar, 0, p.status, 11);
+      if (use_bulk) ok = __syncthreads_and(mbar_wait(bar, 0, p.status, 11)) != 0;
     }
-    for (int t = g.e - 1; t >= 0; --t) {
-      stage_a<TM>(cur, stab ? stab + (size_t)t * (E >> 1) * esz : nullptr, step_of(t), t, E, tid, nthr);
-      __syncthreads();
-    }
-    for (int i = tid; i < E; i += nthr) {
-      const int64_t gi = base + (int64_t)r * E + i;
-      store_act(p.y, row * p.y_stride + gi, p.yt, cur[i] * (float)p.sign[gi]);
+    if (ok) {
+      for (int t = g.e - 1; t >= 0; --t) {
+        stage_a<TM>(cur, stab ? stab + (size_t)t * (E >> 1) * esz : nullptr, step_of(t), t, E, tid, nthr);
+        __syncthreads();
+      }
+      for (int i = tid; i < E; i += nthr) {
+        const int64_t gi = base + (int64_t)r * E + i;
+        store_act(p.y, row * p.y_stride + gi, p.yt, cur[i] * (float)p.sign[gi]);
+      }
     }
   }
+  // after a time-out the parameter copy may still be writing into this CTA's shared
+  // memory: give it one more bounded wait before the CTA exits
+  if (!ok && tid == 0) mbar_wait(bar, 0, nullptr, 12);
 }
 
 int cluster_for(int w) { return w >= 4096 ? 8 : (w == 2048 ? 4 : (w == 1024 ? 2 : 1)); }

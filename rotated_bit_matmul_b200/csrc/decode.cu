@@ -96,8 +96,9 @@ __device__ __forceinline__ bool try_wait_cluster(uint64_t* bar, uint32_t parity)
 __device__ __forceinline__ bool aborted(const int* status) { return *(volatile const int*)status != 0; }
 
 // Wait bounds are counted in SM clock cycles (clock64 is cheap to read, the global
-// timer is not): 4e9 cycles is about 2 s at the B200's top clock, longer when slower.
-constexpr long long kWaitCycles = 4000000000ll;
+// timer is not): by default 4e9 cycles, about 2 s at the B200's top clock, longer when
+// slower. The launch sets it (Params::wait_cycles) into this CTA-wide copy.
+__shared__ long long s_wait_cycles;
 constexpr long long kAbortCheckCycles = 40000;  // start reading the shared abort word after ~20 us
 
 // bounded wait on a local mbarrier phase; false on time-out or abort. SLEEP (the
@@ -114,7 +115,7 @@ __device__ __noinline__ bool wait_phase(uint64_t* bar, uint32_t parity, int* sta
     }
     const long long dt = clock64() - t0;
     if (dt > kAbortCheckCycles && aborted(status)) return false;
-    if (dt > kWaitCycles) {
+    if (dt > s_wait_cycles) {
       report(status, 5, where);
       return false;
     }
@@ -729,7 +730,7 @@ __device__ __noinline__ bool grid_barrier(const Params& p, int idx, int ct) {
     unsigned* c = p.counters + idx;
     __threadfence();
     asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(c) : "memory");
-    const unsigned target = (unsigned)(p.G * kC);
+    const unsigned target = (unsigned)(p.G * kC) + (idx == p.barrier_extra ? 1u : 0u);  // + testing hook
     const long long t0 = clock64();
     for (uint32_t it = 0;; ++it) {
       unsigned v;
@@ -741,7 +742,7 @@ __device__ __noinline__ bool grid_barrier(const Params& p, int idx, int ct) {
           mine = false;
           break;
         }
-        if (dt > kWaitCycles) {
+        if (dt > s_wait_cycles) {
           report(p.status, 5, 60 + (idx % 5));
           mine = false;
           break;
@@ -765,6 +766,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   const int t_cta = c * kC + (int)r;
 
   if (tid == 0) {
+    s_wait_cycles = p.wait_cycles;
     for (int i = 0; i < p.ring_stages; ++i) {
       mbar_init(&s.full[i], 1);
       mbar_init(&s.empty[i], kHalf);  // the 8 warps of the half that consumed the unit

@@ -49,6 +49,8 @@ struct Params {
   float* xsum_down;
   unsigned* counters;  // [L][5], zero at launch
   int* status;
+  long long wait_cycles;  // bound of every wait, in SM clock cycles
+  int barrier_extra;      // testing hook: grid barrier whose target is raised by one (-1: none)
   int tm;   // kTmCS, kTmHad or kTmQ8: how every butterfly of the stack keeps its angles
   int ring_stages, tab_bytes, xq_bytes;
   int asg_qkv[kMaxClusters], idx_qkv[kMaxClusters], cnt_qkv[3];

@@ -75,9 +75,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           bulk_g2s(dst + 4 * (p.xq_stride + p.g_stride), p.xsum + b * p.g_stride, (uint32_t)(4 * p.g_stride), xbar);
         }
       }
-      for (int k = 0; k < nstages; ++k) {
+      int k = 0;
+      for (; k < nstages; ++k) {
         const int slot = k % G::kStages;
-        if (k >= G::kStages && !mbar_wait(&empty[slot], ((k / G::kStages) - 1) & 1, p.status, 1)) break;
+        if (k >= G::kStages && !mbar_wait(&empty[slot], ((k / G::kStages) - 1) & 1, p.status, 1, p.wait_ns)) break;
+        if (k == p.skip_stage && blockIdx.x == 0) continue;  // testing hook: this stage never lands
         const int sub = k / nchunks, ch = k % nchunks;
         const int row0 = r0 + (int)(((int64_t)nrows * sub) / nsub);
         const int g0 = ch * G::kChunkGroups;
@@ -95,6 +97,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < (gc + 31) / 32; ++s)
           tma_load_2d(st + (G::kCodeSlabs + G::kHiSlabs + s) * kSlab, &tm_sz, &full[slot], g0 + s * 32, row0);
       }
+      // the CTA must not exit while copies are still writing into its shared memory: wait
+      // (bounded) for the stages issued last, which the consumers may have left behind
+      const int nlast = k < G::kStages ? k : G::kStages;
+      for (int q = k - nlast; q < k; ++q)
+        if (!(q == p.skip_stage && blockIdx.x == 0))
+          mbar_wait(&full[q % G::kStages], (q / G::kStages) & 1, nullptr, 4, p.wait_ns);
     }
     return;
   }
@@ -105,11 +113,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
   for (int b = 0; b < kMaxBatchGemv; ++b) zacc[b] = 0.f;
   bool ok = true;
-  if constexpr (XS) ok = mbar_wait(xbar, 0, p.status, 3);
+  if constexpr (XS) ok = mbar_wait(xbar, 0, p.status, 3, p.wait_ns);
 
   for (int k = 0; k < nstages && ok; ++k) {
     const int slot = k % G::kStages;
-    if (!mbar_wait(&full[slot], (k / G::kStages) & 1, p.status, 2)) {
+    if (!mbar_wait(&full[slot], (k / G::kStages) & 1, p.status, 2, p.wait_ns)) {
       ok = false;
       break;
     }

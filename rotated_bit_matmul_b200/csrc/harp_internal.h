@@ -46,8 +46,23 @@ struct BflyParams {
   int* status;
 };
 
+// Testing hooks (harp_test_set_faults): off by default. wait_ns bounds every mbarrier
+// wait of the stand-alone kernels, wait_cycles every wait of the fused decode step
+// (SM clock cycles); gemv_skip_stage >= 0 makes the stand-alone GEMV's producer in CTA 0
+// skip that ring stage; decode_barrier_extra raises the target of one grid barrier of the
+// fused step (its index, or -1) by one, so that barrier can never complete.
+struct TestHooks {
+  uint64_t wait_ns;
+  long long wait_cycles;
+  int gemv_skip_stage;
+  int decode_barrier_extra;
+};
+TestHooks test_hooks();
+
 // Dequant-GEMV launch description (codes come through the layer's tensor maps).
 struct GemvParams {
+  uint64_t wait_ns;     // bound of every mbarrier wait
+  int skip_stage;       // testing hook: ring stage CTA 0's producer does not issue (-1: none)
   int n_out, n_in, bits, batch;
   const int32_t* xq;
   int64_t xq_stride;

@@ -419,6 +419,9 @@ harp_status harp_stack_step(harp_stack S, int batch, const void* x, harp_dtype x
     p.y_out = out;
     p.yt = ot;
     p.status = status;
+    const TestHooks th = test_hooks();
+    p.wait_cycles = th.wait_cycles;
+    p.barrier_extra = th.decode_barrier_extra;
     cudaError_t e = cudaMemsetAsync(p.counters, 0, sizeof(unsigned) * 5 * (size_t)S->n_layers, st);
     if (e == cudaSuccess) e = dec::launch(p, st);
     if (e != cudaSuccess) return sfail(HARP_ERR_CUDA, std::string("fused decode step: ") + cudaGetErrorString(e));

@@ -11,8 +11,12 @@
 //
 // Properties the caller must know:
 //   - The first call on a device looks up the array's device address
-//     (cudaGetSymbolAddress) with that device current; make that first call before
-//     any stream capture. Later calls on the device do no set-up.
+//     (cudaGetSymbolAddress) with that device current. With CUDA's lazy module
+//     loading that lookup is also what loads the part of the library image holding
+//     the array, so the array's 2 MiB are taken from the device at that first call
+//     (by the driver, not by an allocation call of this library). Make that first call
+//     before any stream capture, and at a point where taking 2 MiB is acceptable.
+//     Later calls on the device do no set-up and take no device memory.
 //   - Requests whose scratch would exceed 2 MiB are rejected (HARP_ERR_WORKSPACE).
 //   - All calls on a device share the one array, which keeps what the last call
 //     wrote. Nothing in it has to start at zero (every byte is written before it is
@@ -58,7 +62,8 @@ using namespace harp;
 extern "C" harp_status harp_linear_fwd_static(harp_layer layer, int batch, const void* x, harp_dtype xt, void* y,
                                               harp_dtype yt, void* stream) {
   if (!layer) return set_error(HARP_ERR_INVALID_ARG, "linear_fwd_static: null layer");
-  if (batch < 1 || batch > 256) return set_error(HARP_ERR_INVALID_ARG, "linear_fwd_static: batch=%d not in [1,256]", batch);
+  if (batch < 1 || batch > kMaxBatch)
+    return set_error(HARP_ERR_INVALID_ARG, "linear_fwd_static: batch=%d not in [1,%d]", batch, kMaxBatch);
   if (xt < HARP_F32 || xt > HARP_F16 || yt < HARP_F32 || yt > HARP_F16)
     return set_error(HARP_ERR_INVALID_ARG, "linear_fwd_static: unknown dtype");
   if (!x || !y) return set_error(HARP_ERR_INVALID_ARG, "linear_fwd_static: null pointer");

@@ -190,3 +190,12 @@ def test_mr_plan_rejects_bad_arguments(lib):
     assert not h.value
     assert lib.harp_mr_plan_destroy(None) == 0
     assert lib.harp_mr_butterfly_fwd(None, 1, FAKE, 0, FAKE, 0, None) == 1
+
+
+def test_fault_hook_validates_and_switches_off(lib):
+    """The testing hook of the failure paths takes no CUDA call: bad values are refused and
+    the defaults switch it off again."""
+    assert lib.harp_test_set_faults(-1, -1, -1) == 1
+    assert lib.harp_test_set_faults(0, -2, -1) == 1
+    assert lib.harp_test_set_faults(1000, 0, 3) == 0
+    assert lib.harp_test_set_faults(0, -1, -1) == 0

@@ -52,6 +52,40 @@ def test_static_scratch_matches_workspace_entry_point(lib):
     L.close()
 
 
+def test_static_scratch_tensor_core_path(lib):
+    """16 tokens take the tcgen05 path; a 4096 x 4096 layer needs about 1.4 MiB of its
+    scratch, which fits the array. Two calls in a row, each equal to harp_linear_fwd."""
+    case = oracle_layer(4096, 4096, 4096, 4096, 2, workload=3)
+    L = device_layer(case)
+    assert L.workspace_bytes(16) <= (2 << 20)
+    for call in range(2):
+        x = torch.from_numpy(synth.activations(16, 4096, 3, step=200 + call)).to("cuda", torch.bfloat16)
+        want = L(x, out_dtype=torch.float32)
+        got = torch.full((16, 4096), float("nan"), device="cuda")
+        assert _static_call(lib, L, x, got) == 0, lib.harp_last_error()
+        torch.cuda.synchronize()
+        err = rel_l2(got.cpu().numpy(), want.cpu().numpy())
+        assert err < GATE, (call, err)
+    L.close()
+
+
+def test_static_scratch_takes_no_device_memory_after_the_first_call(lib):
+    """After the first call (which may load the library part holding the array), further
+    calls leave the device's free memory exactly as it was."""
+    case = oracle_layer(1024, 2048, 2048, 1024, 2, workload=8)
+    L = device_layer(case)
+    x = torch.from_numpy(synth.activations(2, 2048, 8, step=5)).to("cuda", torch.bfloat16)
+    y = torch.empty((2, 1024), device="cuda")
+    assert _static_call(lib, L, x, y) == 0, lib.harp_last_error()
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    for _ in range(3):
+        assert _static_call(lib, L, x, y) == 0, lib.harp_last_error()
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free0
+    L.close()
+
+
 def test_static_scratch_rejects_oversize(lib):
     import rotated_bit_matmul_b200 as rb
     n_out, n_in, batch = 65536, 4096, 16   # z alone needs 16 * 65536 * 4 bytes = 4 MiB
