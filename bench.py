@@ -56,6 +56,12 @@ def parse():
                     help="fixed randomized Hadamard rotations (Theta = 0) instead of the learned-angle butterflies")
     ap.add_argument("--int8-angles", action="store_true",
                     help="learned angles stored in int8 with a per-stage step (decoded in the kernels)")
+    ap.add_argument("--config", type=int, default=4, choices=[1, 2, 3, 4, 5],
+                    help="4 (default): the 7B 32-block decode stack; 1: one 1024x1024 layer; 2: the seven 7B "
+                         "linears; 3: the batch sweep; 5: the 70B 80-block stack at 2/3/4 bits, batch 1 and 16. "
+                         "Configs other than 4 print one JSON line per measured cell")
+    ap.add_argument("--distinct-blocks", type=int, default=8,
+                    help="config 5: distinct seeded blocks cycled over the 80 layers")
     args = ap.parse_args()
     if args.rht and args.int8_angles:
         ap.error("--rht and --int8-angles exclude each other")
@@ -95,6 +101,15 @@ def traffic_per_step(n_layers, angles="fp32"):
     if h.hexdigest()[:16] != TRAFFIC_PER_BLOCK["sources_sha256_16"]:
         return None
     return TRAFFIC_PER_BLOCK["bytes"][angles] * n_layers
+
+
+def measured_tc_peak():
+    """Dense bf16 tensor-core TFLOP/s from MEASURED_PEAKS.json (burst), else the fallback."""
+    try:
+        d = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+        return float(d["bf16_tflops"])
+    except Exception:
+        return 1590.0
 
 
 def measured_peak():
@@ -317,8 +332,189 @@ def run_ours(args, rk):
                 launches=launches_per_step(args.layers, fused) * K, fused=fused)
 
 
+# ------------------------------------------------------------------ configs 1, 2, 3, 5
+def _line(metric, value, unit, higher, config, roofline, cpu=None, launches=None, clocks=None, dtype=None, extra=None):
+    d = {"metric": metric, "value": value, "unit": unit, "n_gpus": 1, "higher_is_better": higher,
+         "scaling": "weak", "vs_baseline": None, "dtype": dtype or "u2/u3/u4 codes x i16 or f16 activations",
+         "data": "synthetic (seeded N(0,1) activations; random-init N(0,0.02^2) weights with 0.1% outlier columns)",
+         "config": config, "roofline": roofline, "cpu_baseline": cpu, "gpu_launches": launches, "clocks": clocks}
+    if extra:
+        d.update(extra)
+    print(json.dumps(d), flush=True)
+
+
+def _oracle_linear_us(n_out, n_in, w_in, w_out, bits, batch, threads, seconds=10.0):
+    """Times oracle.linear_fwd on one seeded layer (host-prepared) for about `seconds`."""
+    import oracle
+    from rotated_bit_matmul_b200 import synth
+    oracle.set_threads(threads)
+    W = synth.weights(n_out, n_in, 1, 0, 0)
+    thV, sV = synth.butterfly_params(n_in, w_in, 1, 0, 0, "V")
+    thU, sU = synth.butterfly_params(n_out, w_out, 1, 0, 0, "U")
+    lay = oracle.prepare_layer(W, bits, w_in, w_out, thV, sV, thU, sU)[0]
+    x = synth.activations(batch, n_in, 1, step=0, bf16=False).astype(np.float64)
+    n, t0 = 0, time.perf_counter()
+    while n == 0 or time.perf_counter() - t0 < seconds:
+        oracle.linear_fwd(lay, x)
+        n += 1
+    return (time.perf_counter() - t0) / n * 1e6, n
+
+
+def run_linear_configs(args):
+    """Configs 1-3: single rotated linears through harp_linear_fwd, graph-replayed over
+    enough distinct layers that each call streams its weights from HBM (cold L2)."""
+    import torch
+    from rotated_bit_matmul_b200 import linear_timing as lt
+    peak, peak_kind = measured_peak()
+    tc_peak = measured_tc_peak()
+    threads = len(os.sched_getaffinity(0))
+    if args.config == 1:
+        with ClockSampler(0) as clk:
+            r = lt.time_shape(1024, 1024, 1024, 1024, 2, [1], xdtype=torch.float32, min_layers=64)[0]
+        us = r["us_per_call"]
+        cpu = None
+        if not args.no_cpu_baseline:
+            o_us, n = _oracle_linear_us(1024, 1024, 1024, 1024, 2, 1, threads)
+            o1, n1 = _oracle_linear_us(1024, 1024, 1024, 1024, 2, 1, 1, seconds=5.0)
+            cpu = {"value": round(o_us, 1), "unit": "us/call", "cores": threads, "kind": "oracle",
+                   "sample": f"{n} calls of the whole layer on {threads} threads; 1 thread: {o1:.1f} us ({n1} calls)"}
+        ach = r["alg_bytes"] / us / 1e3
+        _line("single 1024x1024 rotated 2-bit linear, batch 1: latency per call", us, "us/call", False,
+              {"workload": "config 1: one 1024x1024 rotated 2-bit linear, fp32 x [1,1024], w 1024 both sides",
+               "distinct_layers": r["layers"], "l2": "each call reads another of the layer copies (cold L2)"},
+              {"bound": "hbm", "achieved": round(ach, 1), "peak": peak, "unit": "GB/s", "frac": round(ach / peak, 4),
+               "traffic": None, "peak_kind": peak_kind, "algorithmic_bytes_per_call": r["alg_bytes"],
+               "kernel": "whole harp_linear_fwd (3 launches)"},
+              cpu=cpu, launches=3, clocks=clk.summary(), dtype="u2 codes x i16 activations -> i32 dot")
+        return
+    shapes = lt.SHAPES if args.config == 2 else lt.SHAPES[:2]
+    batches = [1] if args.config == 2 else [1, 4, 16, 64, 256]
+    names = {0: "q/k/v/o 4096x4096", 1: "gate/up 11008x4096", 2: "down 4096x11008"}
+    mult = {0: 4, 1: 2, 2: 1}
+    total_us, total_bytes = 0.0, 0
+    for i, shp in enumerate(shapes):
+        with ClockSampler(0) as clk:
+            rows = lt.time_shape(*shp, 2, batches)
+        for r in rows:
+            us, B = r["us_per_call"], r["batch"]
+            ach = r["alg_bytes"] / us / 1e3
+            tf = r["tflops"]
+            bound = "tensor" if B >= 64 else "hbm"
+            roof = {"bound": bound, "achieved": round(ach, 1) if bound == "hbm" else tf,
+                    "peak": peak if bound == "hbm" else tc_peak, "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
+                    "frac": round((ach / peak) if bound == "hbm" else (tf / tc_peak), 4), "traffic": None,
+                    "hbm_frac": round(ach / peak, 4), "tensor_frac": round(tf / tc_peak, 4),
+                    "algorithmic_bytes_per_call": r["alg_bytes"], "peak_kind": peak_kind,
+                    "kernel": "whole harp_linear_fwd: " + ("GEMV path" if B < 16 else "tcgen05 path")}
+            _line(f"rotated 2-bit linear {names[i]}, batch {B}: time per call", us, "us/call", False,
+                  {"workload": f"config {args.config}: {names[i]} rotated 2-bit linear, bf16 x [{B},{shp[1]}]",
+                   "batch": B, "distinct_layers": r["layers"], "l2": "cold L2: distinct layer copies per call"},
+                  roof, launches=3 if B < 16 else 4, clocks=clk.summary())
+            if args.config == 2:
+                total_us += mult[i] * us
+                total_bytes += mult[i] * r["alg_bytes"]
+    if args.config == 2:
+        ach = total_bytes / total_us / 1e3
+        _line("the seven linears of a 7B-shaped block, batch 1: time per block", round(total_us, 2), "us/block",
+              False, {"workload": "config 2: q/k/v/o 4096x4096, gate/up 11008x4096, down 4096x11008, batch 1",
+                      "sum_of": "4 x q/k/v/o + 2 x gate/up + 1 x down calls"},
+              {"bound": "hbm", "achieved": round(ach, 1), "peak": peak, "unit": "GB/s", "frac": round(ach / peak, 4),
+               "traffic": None, "peak_kind": peak_kind, "kernel": "21 launches (3 per linear)"},
+              launches=21)
+
+
+def run_70b(args):
+    """Config 5: the Llama-70B-shaped 80-block stack at 2, 3 and 4 bits, batch 1 and 16.
+    Weights of `--distinct-blocks` seeded blocks are drawn on the device, rotated once and
+    quantized at each bit width; the 80 layers cycle through them, so every step streams
+    all 80 blocks' codes (a block is 0.27-0.48 GB, and the same weights come back only
+    after distinct_blocks - 1 other blocks, far more than the 126 MB L2)."""
+    import torch
+    import rotated_bit_matmul_b200 as rb
+    from rotated_bit_matmul_b200 import synth
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    hidden, ffn, nh, nkv, hd = synth.STACK_DIMS["70b"]
+    shapes = synth.llama70b_linears()
+    nl = 80
+    D = max(1, min(args.distinct_blocks, nl))
+    per_bits = {b: [] for b in (2, 3, 4)}  # bits -> list over distinct blocks of 7 HarpLayers
+    for d in range(D):
+        blk = {b: [] for b in per_bits}
+        for i, s in enumerate(shapes):
+            W = synth.device_weights(s.n_out, s.n_in, 5, d, i, device=dev)
+            thV, sV = synth.butterfly_params(s.n_in, s.w_in, 5, d, i, "V")
+            thU, sU = synth.butterfly_params(s.n_out, s.w_out, 5, d, i, "U")
+            thV, thU = torch.from_numpy(thV).to(dev), torch.from_numpy(thU).to(dev)
+            sV, sU = torch.from_numpy(sV).to(dev), torch.from_numpy(sU).to(dev)
+            Wr = rb.rotate_weights_device(W, thV, sV, s.w_in, thU, sU, s.w_out)
+            del W
+            for b in per_bits:
+                codes, sz = rb.harp_quantize_weights(Wr, b, GROUP)
+                blk[b].append(rb.HarpLayer(s.n_in, s.n_out, b, s.w_in, s.w_out, thV, sV, thU, sU, codes, sz))
+            del Wr
+        for b in per_bits:
+            per_bits[b].append(blk[b])
+    torch.cuda.synchronize()
+    peak, peak_kind = measured_peak()
+    K, Wm = args.steps, args.warmup
+    for bits, blocks in per_bits.items():
+        handles = [blocks[l % D][i] for l in range(nl) for i in range(7)]
+        S = rb.HarpStack(handles, hidden, ffn, nh, nkv, hd)
+        for B in (1, 16):
+            wbytes = sum(s.n_out * s.n_in * bits // 8 + s.n_out * (s.n_in // GROUP) * 4 for s in shapes) * nl
+            abytes = sum(4 * B * (s.n_in + s.n_out) for s in shapes) * nl
+            xs = torch.from_numpy(synth.activations(B, hidden, 5, step=0)).to(dev, torch.bfloat16)
+            y = torch.empty((B, hidden), dtype=torch.float32, device=dev)
+            ws = S.workspace(B)
+            st = torch.cuda.Stream(dev)
+            with torch.cuda.stream(st):
+                for _ in range(Wm):
+                    S.step(xs, out=y, workspace=ws)
+            st.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=st):
+                S.step(xs, out=y, workspace=ws)
+            with torch.cuda.stream(st):
+                for _ in range(3):
+                    g.replay()
+            st.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with ClockSampler(0) as clk:
+                with torch.cuda.stream(st):
+                    e0.record(st)
+                    for _ in range(K):
+                        g.replay()
+                    e1.record(st)
+                e1.synchronize()
+            ms = e0.elapsed_time(e1) / K
+            del g
+            ach = (wbytes + abytes) / (ms * 1e-3) / 1e9
+            fused = S.uses_fused_step(B)
+            _line(f"rotated {bits}-bit linear stack, Llama-70B-shaped, batch {B}: decode tokens/s", B / (ms * 1e-3),
+                  "tokens/s", True,
+                  {"workload": f"config 5: Llama-70B-shaped 80-block rotated {bits}-bit linear stack, batch-{B} decode",
+                   "layers": nl, "distinct_blocks": D, "hidden": hidden, "ffn": ffn, "bits": bits, "batch": B,
+                   "l2": "inputs larger than L2"},
+                  {"bound": "hbm", "achieved": round(ach, 1), "peak": peak, "unit": "GB/s", "frac": round(ach / peak, 4),
+                   "traffic": None, "peak_kind": peak_kind, "algorithmic_bytes_per_step": wbytes + abytes,
+                   "kernel": "fused decode step" if fused else "per-linear path (graph of kernels)"},
+                  launches=None, clocks=clk.summary(), extra={"ms_per_step": ms, "steps": K, "warmup": Wm})
+        S.close()
+    for blocks in per_bits.values():
+        for blk in blocks:
+            for L in blk:
+                L.close()
+
+
 def main():
     args = parse()
+    if args.config != 4 and args.impl == "ours":
+        if args.config == 5:
+            run_70b(args)
+        else:
+            run_linear_configs(args)
+        return
     from rotated_bit_matmul_b200 import replicas
     rk = replicas.from_env()
     # the reference arm is the CPU oracle: its ranks meet over gloo

@@ -233,14 +233,54 @@ __device__ __forceinline__ Range units(const Params& p, int l, int ph, int c, in
   return g;
 }
 
+// Cursor over a CTA's units in consumer order (block, phase, unit), used to run the L2
+// prefetch ahead of the ring.
+struct UnitCursor {
+  int l, ph, u;
+  Range g;
+  template <int BITS>
+  __device__ __forceinline__ void normalize(const Params& p, int c, int r) {
+    while (l < p.L && u >= g.u1) {
+      if (++ph == 4) {
+        ph = 0;
+        ++l;
+      }
+      if (l >= p.L) return;
+      g = units<BITS>(p, l, ph, c, r);
+      u = g.u0;
+    }
+  }
+  template <int BITS>
+  __device__ __forceinline__ void next(const Params& p, int c, int r) {
+    ++u;
+    normalize<BITS>(p, c, r);
+  }
+};
+
+// the boxes of one unit, as the ring loads them, requested into L2
+template <int BITS>
+__device__ __forceinline__ void prefetch_unit(const Range& g, int u) {
+  using Gm = Geo<BITS>;
+  const int ngroups = g.L->n_in / 64;
+  const int tile = u / g.nk, kc = u - tile * g.nk;
+  const int g0 = kc * Gm::kChunkGroups, gc = min(Gm::kChunkGroups, ngroups - g0);
+  const int cslabs = (gc + Gm::kGroupsPerSlab - 1) / Gm::kGroupsPerSlab;
+  const int code_x0 = g0 * (BITS == 4 ? 32 : 16) / 8;
+  for (int q = 0; q < cslabs; ++q) tma_prefetch_l2_2d(&g.L->tm_codes, code_x0 + q * 16, tile * 32);
+  if (BITS == 3)
+    for (int q = 0; q < (gc + 15) / 16; ++q) tma_prefetch_l2_2d(&g.L->tm_hi, g0 + q * 16, tile * 32);
+  for (int q = 0; q < (gc + 31) / 32; ++q) tma_prefetch_l2_2d(&g.L->tm_sz, g0 + q * 32, tile * 32);
+}
+
 // ------------------------------------------------------------------ table loads (producer warp 1)
-// Table of one butterfly in shared memory: stage t holds the parameters of the CTA's
-// rotations in stage order, E/2 entries of 8 bytes (cos, sin) or 1 byte (int8 angle);
-// int8 tables start with the 64-byte head of per-stage steps.
+// Table of one butterfly in shared memory: stage t holds the (cos, sin) pairs of the
+// CTA's rotations in stage order, E/2 entries of 8 bytes. fp32 tables are copied as they
+// are; int8 angles are expanded into pairs by the producer warp as it stages them, so the
+// activation chains read the same table format whatever the layer keeps in memory.
 template <int TM>
-__device__ __forceinline__ constexpr int tab_esz() { return TM == kTmQ8 ? 1 : 8; }
+__device__ __forceinline__ constexpr int tab_esz() { return 8; }
 template <int TM>
-__device__ __forceinline__ constexpr int tab_head() { return TM == kTmQ8 ? kQ8Head : 0; }
+__device__ __forceinline__ constexpr int tab_head() { return 0; }
 
 template <int TM>
 __device__ __forceinline__ uint32_t table_bytes_cluster(int w, int m) {
@@ -250,14 +290,65 @@ template <int TM>
 __device__ __forceinline__ uint32_t table_bytes_local(int w, int m) {
   return (uint32_t)(tab_head<TM>() + tab_esz<TM>() * m * (w / 2));
 }
-// bytes a table load actually transfers (none for Theta == 0)
+// bytes a table load transfers by bulk copy (fp32 tables only: none for Theta == 0, and
+// int8 angles are expanded by the warp's own loads)
 template <int TM>
 __device__ __forceinline__ uint32_t copied_bytes_cluster(const uint8_t* src, int w, int m) {
-  return TM == kTmHad || !src ? 0u : table_bytes_cluster<TM>(w, m);
+  return TM != kTmCS || !src ? 0u : table_bytes_cluster<TM>(w, m);
 }
 template <int TM>
 __device__ __forceinline__ uint32_t copied_bytes_local(const uint8_t* src, int w, int m) {
-  return TM == kTmHad || !src ? 0u : table_bytes_local<TM>(w, m);
+  return TM != kTmCS || !src ? 0u : table_bytes_local<TM>(w, m);
+}
+
+// pair index, in the stage's full row, of entry q of the CTA's slice of a
+// cluster-distributed stage t (the order load_table_cluster copies them in)
+__device__ __forceinline__ int64_t slice_pair(int t, int q, int E, int e, int r) {
+  if (t < e) return (int64_t)r * (E >> 1) + q;
+  const int run = E / kC, dd = t - e, jj = q / run, ii = q - jj * run;
+  const int j = ((jj >> dd) << (dd + 1)) | (jj & ((1 << dd) - 1));
+  return (int64_t)(j >> (dd + 1)) * (1 << t) + (int64_t)E * (j & ((1 << dd) - 1)) + (int64_t)r * run + ii;
+}
+
+// int8 angles -> (cos, sin) of pi/4 + delta_t q for the CTA's slice (all 32 lanes of the
+// producer warp; the fast sine/cosine unit, about 5e-7 absolute error near pi/4)
+__device__ __noinline__ void expand_cluster(uint8_t* dst, const uint8_t* q8, int64_t n, int w, int m, int r,
+                                            int lane) {
+  if (!q8) return;
+  const int E = w / kC, e = m - 3;
+  const int64_t half_n = n >> 1;
+  const float* steps = reinterpret_cast<const float*>(q8);
+  const int8_t* codes = reinterpret_cast<const int8_t*>(q8 + kQ8Head);
+  float2* out = reinterpret_cast<float2*>(dst);
+  for (int t = 0; t < m; ++t) {
+    const float st = __ldg(steps + t);
+    for (int q = lane; q < (E >> 1); q += 32) {
+      float sn, cs;
+      __sincosf(fmaf(st, (float)__ldg(codes + (int64_t)t * half_n + slice_pair(t, q, E, e, r)),
+                     0.785398163397448309616f),
+                &sn, &cs);
+      out[(size_t)t * (E >> 1) + q] = make_float2(cs, sn);
+    }
+  }
+}
+
+// the same for block `blk` of width w held whole by one CTA
+__device__ __noinline__ void expand_local(uint8_t* dst, const uint8_t* q8, int64_t n, int w, int m, int blk,
+                                          int lane) {
+  if (!q8) return;
+  const float* steps = reinterpret_cast<const float*>(q8);
+  const int8_t* codes = reinterpret_cast<const int8_t*>(q8 + kQ8Head);
+  float2* out = reinterpret_cast<float2*>(dst);
+  for (int t = 0; t < m; ++t) {
+    const float st = __ldg(steps + t);
+    for (int q = lane; q < (w >> 1); q += 32) {
+      float sn, cs;
+      __sincosf(fmaf(st, (float)__ldg(codes + (int64_t)t * (n >> 1) + (int64_t)blk * (w >> 1) + q),
+                     0.785398163397448309616f),
+                &sn, &cs);
+      out[(size_t)t * (w >> 1) + q] = make_float2(cs, sn);
+    }
+  }
 }
 
 // Per-CTA slice of a cluster-distributed butterfly (width w, C = 8): stage t < e is the
@@ -268,7 +359,7 @@ __device__ __forceinline__ uint32_t load_table_cluster(uint8_t* dst, const uint8
   constexpr int esz = tab_esz<TM>(), head = tab_head<TM>();
   const int E = w / kC, e = m - 3, run = E / kC;
   const int64_t half_n = n >> 1;
-  if (TM == kTmHad || !src) return table_bytes_cluster<TM>(w, m);  // nothing to copy, same layout
+  if (TM != kTmCS || !src) return table_bytes_cluster<TM>(w, m);  // nothing to copy, same layout
   if (head) bulk_g2s(dst, src, (uint32_t)head, bar);
   for (int t = 0; t < m; ++t) {
     const uint8_t* st = src + head + ((int64_t)t * half_n + (int64_t)blk * (w >> 1)) * esz;
@@ -292,7 +383,7 @@ template <int TM>
 __device__ __forceinline__ uint32_t load_table_local(uint8_t* dst, const uint8_t* src, int64_t n, int w, int m, int blk,
                                                      uint64_t* bar) {
   constexpr int esz = tab_esz<TM>(), head = tab_head<TM>();
-  if (TM == kTmHad || !src) return table_bytes_local<TM>(w, m);
+  if (TM != kTmCS || !src) return table_bytes_local<TM>(w, m);
   if (head) bulk_g2s(dst, src, (uint32_t)head, bar);
   for (int t = 0; t < m; ++t)
     bulk_g2s(dst + head + (size_t)t * (w >> 1) * esz, src + head + ((int64_t)t * (n >> 1) + (int64_t)blk * (w >> 1)) * esz,
@@ -759,6 +850,8 @@ __device__ __noinline__ bool grid_barrier(const Params& p, int idx, int ct) {
 template <int BITS, int TM>
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_constant__ Params p) {
   using Gm = Geo<BITS>;
+  // the form the consumers read the staged tables in: int8 angles arrive expanded
+  constexpr int TC = TM == kTmQ8 ? kTmCS : TM;
   Smem s = carve(p, Gm::kStageBytes);
   const uint32_t r = cta_rank();
   const int c = (int)cluster_id_x();
@@ -787,7 +880,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     // never diverges around a blocking wait); lane 0 waits and issues, the others follow.
     const int pw = (tid - kNT) >> 5, lane = tid & 31;
     if (pw == 0) {
-      // ---------------- weight ring: every unit of the step, in consumer order
+      // ---------------- weight ring: every unit of the step, in consumer order. A second
+      // cursor runs p.pf_dist units ahead and asks for those units' boxes to be brought
+      // into L2, so HBM keeps streaming while the activation chains run and the ring's
+      // copies are served from L2.
+      UnitCursor pf;
+      pf.l = 0;
+      pf.ph = 0;
+      pf.g = units<BITS>(p, 0, 0, c, (int)r);
+      pf.u = pf.g.u0;
+      pf.normalize<BITS>(p, c, (int)r);
+      if (lane == 0)
+        for (int d = 0; d < p.pf_dist && pf.l < L; ++d) {
+          prefetch_unit<BITS>(pf.g, pf.u);
+          pf.next<BITS>(p, c, (int)r);
+        }
       uint32_t k = 0;
       bool ok = true;
       for (int l = 0; l < L && ok; ++l)
@@ -797,6 +904,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
           for (int u = g.u0; u < g.u1; ++u) {
             const int slot = k % p.ring_stages;
             int go = 1;
+            if (lane == 0 && pf.l < L) {
+              prefetch_unit<BITS>(pf.g, pf.u);
+              pf.next<BITS>(p, c, (int)r);
+            }
             if (lane == 0) {
               if (k >= (uint32_t)p.ring_stages &&
                   !wait_phase<false, true>(&s.empty[slot], ((k / p.ring_stages) - 1) & 1, p.status, 51)) {
@@ -836,6 +947,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       // ---------------- tables: one set per chain slot, in consumer order
       uint32_t slot = 0;
       bool ok = true;
+      // fp32 tables: the bulk copies' bytes complete the slot. int8 angles: the bytes
+      // announced are the signs'; the warp expands the angles into (cos, sin) pairs, then
+      // lane 0's arrival completes the slot together with those copies.
+      auto announce = [&](uint32_t bytes) {
+        if (TM == kTmQ8) mbar_expect_tx(s.tab_full, bytes);
+        else mbar_arrive_expect_tx(s.tab_full, bytes);
+      };
+      auto finish = [&]() {
+        if (TM == kTmQ8) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(s.tab_full);
+        }
+      };
       auto begin = [&]() -> bool {
         int go = 1;
         if (lane == 0 && slot > 0 && !wait_phase<false, true>(s.tab_empty, (slot - 1) & 1, p.status, 53)) go = 0;
@@ -854,7 +978,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
           const int Eh = p.E;
           if (prev) bytes += Eh;
           if (V) bytes += Eh;
-          mbar_arrive_expect_tx(s.tab_full, bytes);
+          announce(bytes);
           uint32_t off = 0;
           if (prev)
             off += load_table_cluster<TM>(s.tab, prev[6].tU, prev[6].n_out, prev[6].w_out, prev[6].m_out, 0, (int)r,
@@ -863,6 +987,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
           if (prev) bulk_g2s(s.sgn, prev[6].sU + (int64_t)r * Eh, (uint32_t)Eh, s.tab_full);
           if (V) bulk_g2s(s.sgn + kSgnSlot, V->sV + (int64_t)r * Eh, (uint32_t)Eh, s.tab_full);
         }
+        if (TM == kTmQ8) {
+          const Lin* V = l < L ? lin + p.asg_qkv[c] : nullptr;
+          uint32_t off = 0;
+          if (prev) {
+            expand_cluster(s.tab, prev[6].tU, prev[6].n_out, prev[6].w_out, prev[6].m_out, (int)r, lane);
+            off = table_bytes_cluster<TM>(prev[6].w_out, prev[6].m_out);
+          }
+          if (V) expand_cluster(s.tab + off, V->tV, V->n_in, V->w_in, V->m_in, (int)r, lane);
+        }
+        finish();
         ++slot;
         if (l == L) break;
         // P3
@@ -870,13 +1004,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         if (lane == 0) {
           const uint32_t b0 = table_bytes_cluster<TM>(lin[2].w_out, lin[2].m_out);
           const int Eu = lin[2].w_out / kC, Eo = lin[3].w_in / kC;
-          mbar_arrive_expect_tx(s.tab_full, copied_bytes_cluster<TM>(lin[2].tU, lin[2].w_out, lin[2].m_out) +
-                                                copied_bytes_cluster<TM>(lin[3].tV, lin[3].w_in, lin[3].m_in) + Eu + Eo);
+          announce(copied_bytes_cluster<TM>(lin[2].tU, lin[2].w_out, lin[2].m_out) +
+                   copied_bytes_cluster<TM>(lin[3].tV, lin[3].w_in, lin[3].m_in) + Eu + Eo);
           load_table_cluster<TM>(s.tab, lin[2].tU, lin[2].n_out, lin[2].w_out, lin[2].m_out, 0, (int)r, s.tab_full);
           load_table_cluster<TM>(s.tab + b0, lin[3].tV, lin[3].n_in, lin[3].w_in, lin[3].m_in, 0, (int)r, s.tab_full);
           bulk_g2s(s.sgn, lin[2].sU + (int64_t)r * Eu, (uint32_t)Eu, s.tab_full);
           bulk_g2s(s.sgn + kSgnSlot, lin[3].sV + (int64_t)r * Eo, (uint32_t)Eo, s.tab_full);
         }
+        if (TM == kTmQ8) {
+          expand_cluster(s.tab, lin[2].tU, lin[2].n_out, lin[2].w_out, lin[2].m_out, (int)r, lane);
+          expand_cluster(s.tab + table_bytes_cluster<TM>(lin[2].w_out, lin[2].m_out), lin[3].tV, lin[3].n_in,
+                         lin[3].w_in, lin[3].m_in, (int)r, lane);
+        }
+        finish();
         ++slot;
         // P5
         if (!(ok = begin())) break;
@@ -884,13 +1024,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
           const Lin* V = lin + 4 + p.asg_gu[c];
           const uint32_t b0 = table_bytes_cluster<TM>(lin[3].w_out, lin[3].m_out);
           const int Eh = p.E;
-          mbar_arrive_expect_tx(s.tab_full, copied_bytes_cluster<TM>(lin[3].tU, lin[3].w_out, lin[3].m_out) +
-                                                copied_bytes_cluster<TM>(V->tV, V->w_in, V->m_in) + 2 * Eh);
+          announce(copied_bytes_cluster<TM>(lin[3].tU, lin[3].w_out, lin[3].m_out) +
+                   copied_bytes_cluster<TM>(V->tV, V->w_in, V->m_in) + 2 * Eh);
           load_table_cluster<TM>(s.tab, lin[3].tU, lin[3].n_out, lin[3].w_out, lin[3].m_out, 0, (int)r, s.tab_full);
           load_table_cluster<TM>(s.tab + b0, V->tV, V->n_in, V->w_in, V->m_in, 0, (int)r, s.tab_full);
           bulk_g2s(s.sgn, lin[3].sU + (int64_t)r * Eh, (uint32_t)Eh, s.tab_full);
           bulk_g2s(s.sgn + kSgnSlot, V->sV + (int64_t)r * Eh, (uint32_t)Eh, s.tab_full);
         }
+        if (TM == kTmQ8) {
+          const Lin* V = lin + 4 + p.asg_gu[c];
+          expand_cluster(s.tab, lin[3].tU, lin[3].n_out, lin[3].w_out, lin[3].m_out, (int)r, lane);
+          expand_cluster(s.tab + table_bytes_cluster<TM>(lin[3].w_out, lin[3].m_out), V->tV, V->n_in, V->w_in,
+                         V->m_in, (int)r, lane);
+        }
+        finish();
         ++slot;
         // P7: this CTA's MLP blocks, or F_U_q / F_U_k for the two q/k clusters
         if (!(ok = begin())) break;
@@ -904,7 +1051,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
           const int qk = c == qk_cluster(p, 0) ? 0 : (c == qk_cluster(p, 1) ? 1 : -1);
           const int Eq = qk >= 0 ? lin[qk].w_out / kC : 0;
           if (qk >= 0) bytes += copied_bytes_cluster<TM>(lin[qk].tU, lin[qk].w_out, lin[qk].m_out) + Eq;
-          mbar_arrive_expect_tx(s.tab_full, bytes);
+          announce(bytes);
           if (blk < nblocks) {
             uint32_t off = 0;
             off += load_table_local<TM>(s.tab + off, lin[4].tU, lin[4].n_out, wb, mb, blk, s.tab_full);
@@ -919,6 +1066,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             bulk_g2s(s.sgn, lin[qk].sU + (int64_t)r * Eq, (uint32_t)Eq, s.tab_full);
           }
         }
+        if (TM == kTmQ8) {
+          const int wb = lin[4].w_out, mb = lin[4].m_out, blk = t_cta;
+          if (blk < nblocks) {
+            const uint32_t tb = table_bytes_local<TM>(wb, mb);
+            expand_local(s.tab, lin[4].tU, lin[4].n_out, wb, mb, blk, lane);
+            expand_local(s.tab + tb, lin[5].tU, lin[5].n_out, wb, mb, blk, lane);
+            expand_local(s.tab + 2 * tb, lin[6].tV, lin[6].n_in, wb, mb, blk, lane);
+          }
+          const int qk = c == qk_cluster(p, 0) ? 0 : (c == qk_cluster(p, 1) ? 1 : -1);
+          if (qk >= 0) expand_cluster(s.tab, lin[qk].tU, lin[qk].n_out, lin[qk].w_out, lin[qk].m_out, (int)r, lane);
+        }
+        finish();
         ++slot;
       }
       if (lane == 0 && slot > 0) wait_phase<false, true>(s.tab_full, (slot - 1) & 1, p.status, 54);
@@ -947,8 +1106,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     if (!(ok = tab_acquire())) break;
     {
       const uint8_t* tU = s.tab;
-      const uint8_t* tV = prev ? s.tab + table_bytes_cluster<TM>(prev[6].w_out, prev[6].m_out) : s.tab;
-      ok = chain_residual<TM>(p, s, X, prev ? prev + 6 : nullptr, p.zpd, p.nk_f, lin + p.asg_qkv[c], l == 0, r, ct, tU,
+      const uint8_t* tV = prev ? s.tab + table_bytes_cluster<TC>(prev[6].w_out, prev[6].m_out) : s.tab;
+      ok = chain_residual<TC>(p, s, X, prev ? prev + 6 : nullptr, p.zpd, p.nk_f, lin + p.asg_qkv[c], l == 0, r, ct, tU,
                           tV);
     }
     tab_release();
@@ -958,8 +1117,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     if (!(ok = grid_barrier(p, l * 5 + 0, ct))) break;
     // P3
     if (!(ok = tab_acquire())) break;
-    ok = chain_attn<TM>(p, s, X, lin + 2, lin + 3, r, ct, s.tab,
-                    s.tab + table_bytes_cluster<TM>(lin[2].w_out, lin[2].m_out));
+    ok = chain_attn<TC>(p, s, X, lin + 2, lin + 3, r, ct, s.tab,
+                    s.tab + table_bytes_cluster<TC>(lin[2].w_out, lin[2].m_out));
     tab_release();
     if (!ok) break;
     // P4
@@ -967,8 +1126,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     if (!(ok = grid_barrier(p, l * 5 + 1, ct))) break;
     // P5
     if (!(ok = tab_acquire())) break;
-    ok = chain_residual<TM>(p, s, X, lin + 3, p.zpo, p.nk_h, lin + 4 + p.asg_gu[c], false, r, ct, s.tab,
-                        s.tab + table_bytes_cluster<TM>(lin[3].w_out, lin[3].m_out));
+    ok = chain_residual<TC>(p, s, X, lin + 3, p.zpo, p.nk_h, lin + 4 + p.asg_gu[c], false, r, ct, s.tab,
+                        s.tab + table_bytes_cluster<TC>(lin[3].w_out, lin[3].m_out));
     tab_release();
     if (!ok) break;
     // P6
@@ -977,13 +1136,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     // P7
     if (!(ok = tab_acquire())) break;
     {
-      if (t_cta < nblocks) block_chain<TM>(p, s, lin + 4, lin + 5, lin + 6, t_cta, ct, s.tab);
+      if (t_cta < nblocks) block_chain<TC>(p, s, lin + 4, lin + 5, lin + 6, t_cta, ct, s.tab);
       const int qk = c == qk_cluster(p, 0) ? 0 : (c == qk_cluster(p, 1) ? 1 : -1);
       if (qk >= 0) {
         float* out = qk == 0 ? p.qout + (int64_t)l * lin[0].n_out : p.kout + (int64_t)l * lin[1].n_out;
         const float* zp = qk == 0 ? p.zpq + (int64_t)l * p.nk_h * lin[0].n_out
                                   : p.zpk + (int64_t)l * p.nk_h * lin[1].n_out;
-        ok = chain_out_only<TM>(p, s, X, lin + qk, zp, out, r, ct, s.tab);
+        ok = chain_out_only<TC>(p, s, X, lin + qk, zp, out, r, ct, s.tab);
       }
     }
     tab_release();
@@ -1009,7 +1168,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   // final: out = h_{L-1} + F_U_down(z_down)
   if (ok && (ok = tab_acquire())) {
     const Lin* last = p.lin + 7 * (L - 1);
-    ok = chain_residual<TM>(p, s, X, last + 6, p.zpd, p.nk_f, nullptr, false, r, ct, s.tab, s.tab);
+    ok = chain_residual<TC>(p, s, X, last + 6, p.zpd, p.nk_f, nullptr, false, r, ct, s.tab, s.tab);
     if (ok && c == 0)
       for (int L2 = ct; L2 < p.E; L2 += kNT) store_act(p.y_out, gidx_b(L2, p.E, r), p.yt, s.res[L2]);
     tab_release();

@@ -53,6 +53,7 @@ struct Params {
   int barrier_extra;      // testing hook: grid barrier whose target is raised by one (-1: none)
   int tm;   // kTmCS, kTmHad or kTmQ8: how every butterfly of the stack keeps its angles
   int ring_stages, tab_bytes, xq_bytes;
+  int pf_dist;  // units the L2 prefetch runs ahead of the ring (0: none)
   int asg_qkv[kMaxClusters], idx_qkv[kMaxClusters], cnt_qkv[3];
   int asg_gu[kMaxClusters], idx_gu[kMaxClusters], cnt_gu[2];
 };

@@ -2,6 +2,7 @@
 // layers: RMSNorm, residual adds, SiLU * up, and the key/value-group broadcast of a
 // one-key attention (its output is the value), around harp linear forwards.
 #include <algorithm>
+#include <cstdlib>
 #include <cstring>
 #include <new>
 #include <string>
@@ -251,14 +252,6 @@ void setup_fused(harp_stack_s* S) {
     tm = dec::kTmQ8;
   else if (n_q8 || n_had)
     return no("butterflies with fp32 angles, int8 angles and Theta = 0 are not fused together");
-  if (tm == dec::kTmQ8) {
-    // int8 slices are copied with 16-byte bulk copies: per-CTA runs of w/64 angles
-    for (int w : {H, dq, dkv})
-      if (w % 1024) return no("int8 angles need butterflies of widths that are multiples of 1024");
-    if (wb % 32) return no("int8 angles need MLP blocks of a multiple of 32");
-    for (const harp_layer l : S->layers)
-      if ((l->L.n_in / 2) % 16 || (l->L.n_out / 2) % 16) return no("int8 angles need n_in, n_out multiples of 32");
-  }
   dec::Params& p = S->fp;
   p = dec::Params{};
   p.tm = tm;
@@ -274,7 +267,8 @@ void setup_fused(harp_stack_s* S) {
   p.E = H / dec::kC;
   p.m_hidden = ilog2(H);
   // shared-memory budget: tables of the largest chain, operand of the widest input
-  const int esz = tm == dec::kTmQ8 ? 1 : 8, head = tm == dec::kTmQ8 ? kQ8Head : 0;
+  // tables are staged as (cos, sin) pairs whatever the layer keeps (int8 angles are expanded)
+  const int esz = 8, head = 0;
   auto tb = [&](int w) { return head + esz * ilog2(w) * (w / dec::kC / 2); };
   int tab = 2 * tb(H);
   tab = std::max(tab, tb(dkv) + tb(H));
@@ -290,6 +284,9 @@ void setup_fused(harp_stack_s* S) {
   p.ring_stages = 16;
   while (p.ring_stages >= 2 && dec::smem_for(p) > (size_t)optin) --p.ring_stages;
   if (p.ring_stages < 2) return no("not enough shared memory for the weight ring");
+  // L2 prefetch distance: HARP_PF_DIST overrides (a tuning knob), else 16 units
+  p.pf_dist = 16;
+  if (const char* e = getenv("HARP_PF_DIST")) p.pf_dist = std::max(0, atoi(e));
   int G = 0;
   cudaError_t e = dec::max_clusters(p, &G);
   if (e != cudaSuccess || G < 1) return no(std::string("cluster occupancy query failed: ") + cudaGetErrorString(e));

@@ -37,14 +37,15 @@ def _layers(n_out, n_in, w_in, w_out, bits, count, device):
             for _ in range(count)]
 
 
-def time_shape(n_out, n_in, w_in, w_out, bits, batches, reps=10, device="cuda"):
+def time_shape(n_out, n_in, w_in, w_out, bits, batches, reps=10, device="cuda", xdtype=None, min_layers=4):
     import torch
+    xdtype = xdtype or torch.bfloat16
     wbytes = n_out * n_in * bits // 8 + n_out * (n_in // 64) * 4
-    count = max(4, int(np.ceil(1.5 * L2_BYTES / wbytes)))
+    count = max(min_layers, int(np.ceil(1.5 * L2_BYTES / wbytes)))
     layers = _layers(n_out, n_in, w_in, w_out, bits, count, device)
     out = []
     for batch in batches:
-        x = torch.randn(batch, n_in, device=device).to(torch.bfloat16)
+        x = torch.randn(batch, n_in, device=device).to(xdtype)
         y = torch.empty(batch, n_out, device=device)
         ws = layers[0].workspace(batch)
         st = torch.cuda.Stream(device)
@@ -69,8 +70,11 @@ def time_shape(n_out, n_in, w_in, w_out, bits, batches, reps=10, device="cuda"):
                 e1.synchronize()
                 ts.append(e0.elapsed_time(e1) / count)
         us = float(np.median(ts)) * 1e3
-        out.append(dict(n_out=n_out, n_in=n_in, bits=bits, batch=batch, layers=count, us_per_call=round(us, 2),
-                        weight_gbs=round(wbytes / us / 1e3, 1), tflops=round(2 * n_out * n_in * batch / us / 1e6, 2)))
+        abytes = x.element_size() * batch * n_in + 4 * batch * n_out  # activations in and out
+        out.append(dict(n_out=n_out, n_in=n_in, bits=bits, batch=batch, layers=count, us_per_call=round(us, 3),
+                        weight_gbs=round(wbytes / us / 1e3, 1), alg_bytes=wbytes + abytes,
+                        alg_gbs=round((wbytes + abytes) / us / 1e3, 1),
+                        tflops=round(2 * n_out * n_in * batch / us / 1e6, 2)))
         del g
     for L in layers:
         L.close()

@@ -189,24 +189,45 @@ def test_70b_shapes_bits_3_4(name, batch, bits):
     _check(case, batch, 5)
 
 
-def test_70b_block_stack_batch_1_and_16():
+def _70b_block_cases(bits_list, workload=11):
+    """Oracle layers of one Llama-70B-shaped block at several bit widths: each linear's W is
+    drawn and rotated once (the expensive fp64 part), then quantized per bit width."""
+    shapes = synth.llama70b_linears()
+    out = {b: [] for b in bits_list}
+    for i, s in enumerate(shapes):
+        W = synth.weights(s.n_out, s.n_in, workload, 0, i)
+        thV, sV = synth.butterfly_params(s.n_in, s.w_in, workload, 0, i, "V")
+        thU, sU = synth.butterfly_params(s.n_out, s.w_out, workload, 0, i, "U")
+        Wr = oracle.rotate_weights(W, thV, sV, s.w_in, thU, sU, s.w_out)
+        del W
+        for b in bits_list:
+            q, s16, z16 = oracle.quantize(Wr, b)
+            lay = oracle.Layer(s.n_in, s.n_out, b, s.w_in, s.w_out, thV, sV, thU, sU, oracle.pack(q, b),
+                               oracle.scale_zero(s16, z16))
+            out[b].append(dict(lay=lay, thV=thV, sV=sV, thU=thU, sU=sU, n_in=s.n_in, n_out=s.n_out, w_in=s.w_in,
+                               w_out=s.w_out, bits=b))
+        del Wr
+    return out
+
+
+def test_70b_block_stack_bits_2_3_4_batch_1_and_16():
     """One Llama-70B-shaped block (hidden 8192, FFN 28672 in 4096-wide butterfly blocks,
-    64 query heads and 8 KV heads of 128), 2-bit, one decode step at 1 token (per-linear
-    GEMV path; KV heads broadcast x8) and at 16 tokens (tensor-core path)."""
+    64 query heads and 8 KV heads of 128) at 2, 3 and 4 bits, one decode step at 1 token
+    (KV heads broadcast x8) and at 16 tokens (tensor-core path)."""
     import rotated_bit_matmul_b200 as rb
     dims = (8192, 28672, 64, 8, 128)
-    shapes = synth.llama70b_linears()
-    cases = [oracle_layer(s.n_out, s.n_in, s.w_in, s.w_out, 2, 11, 0, i) for i, s in enumerate(shapes)]
-    layers = [device_layer(c) for c in cases]
-    S = rb.HarpStack(layers, *dims)
-    for batch in (1, 16):
-        x = synth.activations(batch, dims[0], 11, step=batch)
-        got = S.step(_dev(x, torch.bfloat16)).cpu().numpy()
-        torch.cuda.synchronize()
-        want = oracle.stack_step([c["lay"] for c in cases], *dims, x.astype(np.float64))
-        err = rel_l2(got, want)
-        print(f"70B block batch {batch} rel-L2 {err:.3e}")
-        assert err < (GATE if batch < 16 else TC_STACK_GATE), (batch, err)
-    S.close()
-    for L in layers:
-        L.close()
+    per_bits = _70b_block_cases((2, 3, 4))
+    for bits, cases in per_bits.items():
+        layers = [device_layer(c) for c in cases]
+        S = rb.HarpStack(layers, *dims)
+        for batch in (1, 16):
+            x = synth.activations(batch, dims[0], 11, step=batch)
+            got = S.step(_dev(x, torch.bfloat16)).cpu().numpy()
+            torch.cuda.synchronize()
+            want = oracle.stack_step([c["lay"] for c in cases], *dims, x.astype(np.float64))
+            err = rel_l2(got, want)
+            print(f"70B block {bits}-bit batch {batch} rel-L2 {err:.3e}")
+            assert err < (GATE if batch < 16 else TC_STACK_GATE), (bits, batch, err)
+        S.close()
+        for L in layers:
+            L.close()

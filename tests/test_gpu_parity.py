@@ -116,7 +116,15 @@ def _linear_check(case, batch, xdt=torch.bfloat16, ydt=torch.float32, workload=2
     want = oracle.linear_fwd(case["lay"], x.astype(np.float64))
     err = rel_l2(got, want)
     L.close()
+    # the worst token row, and the worst 32-row output tile of it (a few wrong rows of an
+    # 11008-row output barely move the whole-tensor figure)
+    rows = max(rel_l2(got[b], want[b]) for b in range(batch))
+    n_out = want.shape[1]
+    tiles = max(rel_l2(got[b, t:t + 32], want[b, t:t + 32]) for b in range(batch) for t in range(0, n_out, 32))
+    print(f"n_out={n_out} batch={batch}: rel-L2 {err:.3e}, worst row {rows:.3e}, worst 32-row tile {tiles:.3e}")
     assert err < gate, err
+    assert rows < 2 * gate, rows
+    assert tiles < 10 * gate, tiles
     return err
 
 
