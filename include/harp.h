@@ -148,6 +148,23 @@ harp_status harp_mr_butterfly_fwd(harp_mr_plan plan, int batch, const void* x, h
 harp_status harp_mr_butterfly_inv(harp_mr_plan plan, int batch, const void* x, harp_dtype xt, void* y,
                                   harp_dtype yt, void* stream);
 
+/* A layer whose two sides are mixed-radix butterflies (HARP page, Sec. 2.1, Suporte a
+ * Misto-Raiz): y = F_U(dequant(codes) F_V(x)) with F_V the plan V's forward transform and
+ * F_U the plan U's. For a width such as 11008 = 2^8 * 43 this mixes all coordinates, where a
+ * radix-2 layer uses independent 256-wide blocks. codes/scale_zero must come from
+ * W' = F_U^T W F_V^T rotated with the same plans (canonical layouts as for harp_create_layer).
+ *   n_in  : a multiple of 256, <= 16384, equal to V's length;  n_out: <= 16384, U's length.
+ *   V, U  : plans of harp_mr_plan_create on the current device. BORROWED, like codes and
+ *           scale_zero: keep all four alive and unchanged until harp_destroy_layer.
+ * harp_linear_fwd runs the plans' transforms (fp32) around the same dequant-GEMV (1..15
+ * tokens; the transformed input is brought to the int16 group operand) or tcgen05 path (16+
+ * tokens; the split partials are summed before the output transform). Stacks of such layers
+ * take the per-linear path. Errors: HARP_ERR_INVALID_ARG (sizes, lengths, pointers, device),
+ * HARP_ERR_UNSUPPORTED (group), HARP_ERR_CUDA. */
+harp_status harp_create_layer_mr(harp_layer* out, int64_t n_in, int64_t n_out, int bits, int group,
+                                 harp_mr_plan V, harp_mr_plan U, const void* codes, const void* scale_zero,
+                                 void* stream);
+
 /* ---------------------------------------------------------------- int8 angles
  * The HARP page stores its parameters in int8 (Sec. 2.4, Armazenamento, and Sec. 4:
  * 2.00 -> 2.05 bits per parameter at 2 bits); the format is this library's:

@@ -176,6 +176,21 @@ class HarpLayer:
         self.handle = h
         return self
 
+    @classmethod
+    def mixed_radix(cls, V, U, bits, codes, scale_zero, group=64):
+        """A layer whose sides are mixed-radix butterflies (wraps harp_create_layer_mr): V and U
+        are HarpMixedRadix plans of lengths n_in and n_out; the layer borrows them (they must
+        outlive it) as it borrows codes and scale_zero."""
+        _need_cuda(codes, scale_zero)
+        self = cls.__new__(cls)
+        self._fields(V.d, U.d, bits, 0, 0, codes, scale_zero, group)
+        self._plans = (V, U)
+        h = ctypes.c_void_p()
+        call("harp_create_layer_mr", ctypes.byref(h), self.n_in, self.n_out, self.bits, self.group, V.handle,
+             U.handle, _p(codes), _p(scale_zero), _stream())
+        self.handle = h
+        return self
+
     def _fields(self, n_in, n_out, bits, w_in, w_out, codes, scale_zero, group):
         self.handle = None
         self.n_in, self.n_out, self.bits, self.group = int(n_in), int(n_out), int(bits), int(group)

@@ -46,6 +46,7 @@ SIGNATURES = {
     "harp_mr_butterfly_fwd": (_I, [_P, _I, _P, _I, _P, _I, _P]),
     "harp_mr_butterfly_inv": (_I, [_P, _I, _P, _I, _P, _I, _P]),
     "harp_quantize_angles": (_I, [_I, _I64, _P, _P, _P, _P]),
+    "harp_create_layer_mr": (_I, [ctypes.POINTER(_P), _I64, _I64, _I, _I, _P, _P, _P, _P, _P]),
     "harp_create_layer_q8": (_I, [ctypes.POINTER(_P), _I64, _I64, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P,
                                   _P]),
     "harp_calib_workspace_size": (_I, [_I64, _I64, _I, _I, _I, _I, _I, ctypes.POINTER(_SZ)]),

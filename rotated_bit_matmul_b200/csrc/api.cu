@@ -171,7 +171,9 @@ LinearWs linear_ws_layout(const Layer& L, int batch, void* base) {
     w.x16 = carve(2 * (size_t)batch * (size_t)w.x16_ld);
     w.rowscale = static_cast<float*>(carve(sizeof(float) * (size_t)batch));
     w.zpart = static_cast<float*>(carve(sizeof(float) * (size_t)L.msplits * (size_t)batch * (size_t)L.n_out));
+    if (L.mrU) w.zmr = static_cast<float*>(carve(sizeof(float) * (size_t)batch * (size_t)L.n_out));
   } else {
+    if (L.mrV) w.xmr = static_cast<float*>(carve(sizeof(float) * (size_t)batch * (size_t)L.n_in));
     w.xq_stride = xq_words_per_row(L.n_in, L.bits);
     w.g_stride = ng;
     w.xq = static_cast<int32_t*>(carve(sizeof(int32_t) * (size_t)batch * (size_t)w.xq_stride));
@@ -192,8 +194,61 @@ harp_status linear_forward(const Layer& L, int batch, const void* x, int xt, int
   return linear_forward_status(L, batch, x, xt, x_stride, y, yt, y_stride, ws, st, status);
 }
 
+// y = F_U(dequant(codes) F_V(x)) with mixed-radix sides: the plans' transforms around
+// the radix-2 layers' GEMV (operand prepared from the fp32 transform) or tensor-core
+// contraction (split partials summed before the output transform)
+static harp_status mr_linear_forward(const Layer& L, int batch, const void* x, int xt, int64_t x_stride, void* y,
+                                     int yt, int64_t y_stride, void* ws, cudaStream_t st, int* status) {
+  if (x_stride != L.n_in || y_stride != L.n_out)
+    return fail(HARP_ERR_UNSUPPORTED, "mixed-radix linear: rows must be contiguous");
+  LinearWs w = linear_ws_layout(L, batch, ws);
+  const float* z = nullptr;
+  if (batch >= kMinBatchMma) {
+    HARP_CUDA(launch_mr(L.mrV, 0, batch, x, xt, w.xf, DT_F32, st), "input transform launch");
+    HARP_CUDA(mma::launch_x16_prep(w.xf, L.n_in, L.bits, batch, static_cast<__half*>(w.x16), w.rowscale, status, st),
+              "operand prep launch");
+    mma::Call c{};
+    c.x16 = static_cast<const __half*>(w.x16);
+    c.ld = w.x16_ld;
+    c.rowscale = w.rowscale;
+    c.zpart = w.zpart;
+    c.batch = batch;
+    c.status = status;
+    HARP_CUDA(mma::launch(L, c, st), "dequant-MMA launch");
+    HARP_CUDA(launch_sum_splits(w.zpart, L.msplits, (int64_t)batch * L.n_out, w.zmr, st), "split sum launch");
+    z = w.zmr;
+  } else {
+    HARP_CUDA(launch_mr(L.mrV, 0, batch, x, xt, w.xmr, DT_F32, st), "input transform launch");
+    HARP_CUDA(launch_operand_prep(w.xmr, L.n_in, L.bits, batch, w.xq, w.xq_stride, w.xs, w.xsum, w.g_stride, st),
+              "operand prep launch");
+    for (int b0 = 0; b0 < batch; b0 += kMaxBatchGemv) {
+      GemvParams gp{};
+      const TestHooks th = test_hooks();
+      gp.wait_ns = th.wait_ns;
+      gp.skip_stage = th.gemv_skip_stage;
+      gp.n_out = (int)L.n_out;
+      gp.n_in = (int)L.n_in;
+      gp.bits = L.bits;
+      gp.batch = batch - b0 < kMaxBatchGemv ? batch - b0 : kMaxBatchGemv;
+      gp.xq = w.xq + (int64_t)b0 * w.xq_stride;
+      gp.xq_stride = w.xq_stride;
+      gp.xs = w.xs + (int64_t)b0 * w.g_stride;
+      gp.xsum = w.xsum + (int64_t)b0 * w.g_stride;
+      gp.g_stride = w.g_stride;
+      gp.z = w.z + (int64_t)b0 * L.n_out;
+      gp.z_stride = L.n_out;
+      gp.status = status;
+      HARP_CUDA(launch_gemv(L, gp, st), "dequant-GEMV launch");
+    }
+    z = w.z;
+  }
+  HARP_CUDA(launch_mr(L.mrU, 0, batch, z, DT_F32, y, yt, st), "output transform launch");
+  return HARP_OK;
+}
+
 harp_status linear_forward_status(const Layer& L, int batch, const void* x, int xt, int64_t x_stride, void* y,
                                   int yt, int64_t y_stride, void* ws, cudaStream_t st, int* status) {
+  if (L.mrV) return mr_linear_forward(L, batch, x, xt, x_stride, y, yt, y_stride, ws, st, status);
   LinearWs w = linear_ws_layout(L, batch, ws);
   const bool tc = batch >= kMinBatchMma;
 
@@ -364,6 +419,8 @@ harp_status harp_quantize_weights(int64_t n_out, int64_t n_in, int bits, int gro
 
 namespace {
 
+harp_status layer_maps(Layer& L);
+
 // One side's angles: raw theta (cos/sin tables are built), int8 codes with their steps
 // (copied into the layer's int8 storage), or neither (Theta = 0).
 struct SideAngles {
@@ -445,6 +502,22 @@ harp_status create_layer_impl(harp_layer* out, int64_t n_in, int64_t n_out, int 
   };
   if ((e = q8_side(av, m_in, cnt_v, &L.q8V)) != cudaSuccess || (e = q8_side(au, m_out, cnt_u, &L.q8U)) != cudaSuccess)
     return cleanup(cuda_fail(e, "create_layer_q8: int8 angle storage"));
+  harp_status s = layer_maps(L);
+  if (s != HARP_OK) return cleanup(s);
+  *out = h;
+  return HARP_OK;
+}
+
+}  // namespace
+
+namespace {
+// TMA descriptors of a layer's codes and scale/zero (GEMV and tensor-core boxes) and the
+// tensor-core split of its input groups
+harp_status layer_maps(Layer& L) {
+  const int64_t n_in = L.n_in, n_out = L.n_out;
+  const int bits = L.bits;
+  const void* codes = L.codes;
+  const void* scale_zero = L.scale_zero;
   const int pb = bits == 4 ? 4 : 2;  // bits of the (first) code plane
   harp_status s =
       make_tmap(&L.tm_codes, codes, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, (uint64_t)n_in * pb / 64, (uint64_t)n_out,
@@ -456,7 +529,7 @@ harp_status create_layer_impl(harp_layer* out, int64_t n_in, int64_t n_out, int 
   if (s == HARP_OK)
     s = make_tmap(&L.tm_sz, scale_zero, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, (uint64_t)n_in / 64, (uint64_t)n_out,
                   (uint64_t)n_in / 16);
-  if (s != HARP_OK) return cleanup(s);
+  if (s != HARP_OK) return s;
   // tensor-core path: one group of codes, a split's scale_zero / 1-bit plane per 128 rows
   const mma::Split sp = mma::choose_split(n_out, n_in, bits);
   L.msplits = sp.splits;
@@ -472,8 +545,7 @@ harp_status create_layer_impl(harp_layer* out, int64_t n_in, int64_t n_out, int 
                         (uint64_t)n_in / 8, (uint64_t)n_out, (uint64_t)n_in / 8, (uint32_t)(8 * sp.gs), mma::kBM,
                         CU_TENSOR_MAP_SWIZZLE_NONE);
   if (mok && bits != 3) L.tm_mhi = L.tm_msz;
-  if (!mok) return cleanup(fail(HARP_ERR_CUDA, "create_layer: tensor maps of the tensor-core path"));
-  *out = h;
+  if (!mok) return fail(HARP_ERR_CUDA, "create_layer: tensor maps of the tensor-core path");
   return HARP_OK;
 }
 
@@ -492,6 +564,50 @@ harp_status harp_create_layer_q8(harp_layer* out, int64_t n_in, int64_t n_out, i
                                  const void* scale_zero, void* stream) {
   return create_layer_impl(out, n_in, n_out, bits, group, w_in, w_out, SideAngles{nullptr, q_V, delta_V}, sign_V,
                            SideAngles{nullptr, q_U, delta_U}, sign_U, codes, scale_zero, stream);
+}
+
+harp_status harp_create_layer_mr(harp_layer* out, int64_t n_in, int64_t n_out, int bits, int group, harp_mr_plan V,
+                                 harp_mr_plan U, const void* codes, const void* scale_zero, void* stream) {
+  (void)stream;
+  if (!out) return fail(HARP_ERR_INVALID_ARG, "create_layer_mr: null output handle");
+  *out = nullptr;
+  if (bits < 2 || bits > 4) return fail(HARP_ERR_INVALID_ARG, "create_layer_mr: bits=%d not in {2,3,4}", bits);
+  if (group != kGroup) return fail(HARP_ERR_UNSUPPORTED, "create_layer_mr: group=%d (only 64 is supported)", group);
+  if (!V || !U || !codes || !scale_zero) return fail(HARP_ERR_INVALID_ARG, "create_layer_mr: null pointer");
+  if (n_in <= 0 || n_in % 256 || n_in > 16384)
+    return fail(HARP_ERR_INVALID_ARG, "create_layer_mr: n_in=%lld must be a positive multiple of 256, <= 16384",
+                (long long)n_in);
+  if (n_out <= 0 || n_out > 16384)
+    return fail(HARP_ERR_INVALID_ARG, "create_layer_mr: n_out=%lld not in [1, 16384]", (long long)n_out);
+  if (mr_plan_d(V) != n_in || mr_plan_d(U) != n_out)
+    return fail(HARP_ERR_INVALID_ARG, "create_layer_mr: the plans' lengths must be n_in and n_out");
+  if (!aligned16(codes) || !aligned16(scale_zero))
+    return fail(HARP_ERR_INVALID_ARG, "create_layer_mr: device pointers must be 16-byte aligned");
+  int dev = 0;
+  HARP_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  if (mr_plan_device(V) != dev || mr_plan_device(U) != dev)
+    return fail(HARP_ERR_INVALID_ARG, "create_layer_mr: the plans live on another device");
+  harp_layer_s* h = new (std::nothrow) harp_layer_s();
+  if (!h) return fail(HARP_ERR_INVALID_ARG, "create_layer_mr: out of host memory");
+  Layer& L = h->L;
+  L.n_in = n_in;
+  L.n_out = n_out;
+  L.bits = bits;
+  L.group = group;
+  L.mrV = V;
+  L.mrU = U;
+  L.codes = codes;
+  L.scale_zero = scale_zero;
+  L.device = dev;
+  // no radix-2 butterfly: the fused decode step and the radix-2 kernels never take this layer
+  L.w_in = L.w_out = 0;
+  const harp_status s = layer_maps(L);
+  if (s != HARP_OK) {
+    delete h;
+    return s;
+  }
+  *out = h;
+  return HARP_OK;
 }
 
 harp_status harp_quantize_angles(int m, int64_t half_n, const float* theta, int8_t* q, float* delta, void* stream) {

@@ -192,4 +192,36 @@ __device__ __forceinline__ int group_exponent(float amax) {
 // 2^e for e in [-126, 127], exact
 __device__ __forceinline__ float pow2f(int e) { return __int_as_float((e + 127) << 23); }
 
+// int16 GEMV operand of one group of 64 values v[0..63] (one warp): the values at scale
+// 2^e with max |v| 2^e in [2^14, 2^15), in dp2a pair order (and the 1-bit-plane order for
+// 3-bit codes); lane 0 writes the scale 2^-e and the fp32 group sum. A non-finite value
+// makes the group's scale and sum NaN.
+__device__ __forceinline__ void prep_group(const float* v, int bits, int16_t* grp, int16_t* grp_hi, float* xs,
+                                           float* xsum, int lane) {
+  const float v0 = v[2 * lane], v1 = v[2 * lane + 1];
+  float amax = fmaxf(fabsf(v0), fabsf(v1));
+  float sum = v0 + v1;
+  const bool bad = __any_sync(0xffffffffu, !(isfinite(v0) && isfinite(v1)));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  }
+  int ex = 0;
+  if (amax > 0.f && !bad) ex = group_exponent(amax);
+  const float sc = pow2f(ex);
+  const int q0 = max(-32767, min(32767, __float2int_rn(v0 * sc)));
+  const int q1 = max(-32767, min(32767, __float2int_rn(v1 * sc)));
+  grp[xq_pos_lo(bits, 2 * lane)] = (int16_t)q0;
+  grp[xq_pos_lo(bits, 2 * lane + 1)] = (int16_t)q1;
+  if (bits == 3) {
+    grp_hi[xq_pos_hi(2 * lane)] = (int16_t)q0;
+    grp_hi[xq_pos_hi(2 * lane + 1)] = (int16_t)q1;
+  }
+  if (lane == 0) {
+    *xs = bad ? __int_as_float(0x7fc00000) : pow2f(-ex);
+    *xsum = bad ? __int_as_float(0x7fc00000) : sum;
+  }
+}
+
 }  // namespace harp

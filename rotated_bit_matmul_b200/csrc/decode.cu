@@ -8,23 +8,31 @@
 //  * Weights never depend on activations, so a producer warp per CTA streams that
 //    CTA's share of every GEMV of the step, in order, with 2-D TMA tile loads (no
 //    multicast) into a ring of shared-memory stages, while the activation chain runs.
-//    A GEMV is cut into units of 32 output rows x one column chunk (split-K); each
-//    unit's partial sums go to a buffer the next chain adds up in a fixed order. The
-//    16 consumer warps form two halves that take alternate units, without any
-//    CTA-wide barrier: the last warp of a half to finish a unit reduces it.
+//    A second cursor runs ahead of the ring and asks for the boxes of later units in L2
+//    (bulk tensor prefetch), so HBM keeps streaming while the chains run. A GEMV is cut
+//    into units of 32 output rows x 2048 input columns (split-K); each unit's partial
+//    sums go to a buffer the next chain adds up in a fixed order. The 16 consumer warps
+//    form two halves that take alternate units; the last warp of a half to finish a
+//    unit reduces it.
 //  * CTAs form clusters of 8. Each cluster computes the activation chain between two
-//    GEMVs itself (redundantly with the other clusters): a w-wide butterfly spread
-//    over its 8 CTAs (w/8 elements each), local stages register-blocked (8 values per
-//    thread, three stages per shared-memory round trip), the cross-CTA stages reached
-//    by pushing data into the peers' shared memory and one cluster barrier (8
-//    parallel release-arrives, acquire on the own barrier). A second producer warp
-//    prefetches every chain's angle tables with bulk copies. The kernel is instantiated
-//    per form of the angles (TM): (cos, sin) fp32 pairs, 8 bytes per rotation; int8
-//    angles, 1 byte per rotation plus one step per stage, whose cos/sin are evaluated as
-//    the rotation runs; or Theta == 0 everywhere (the fixed randomized Hadamard
-//    transform), where the constant 1/sqrt 2 blocks need no table at all.
-//  * Grid-wide barriers (release/acquire counters) only where a whole output vector
-//    is needed: after q/k/v, o, gate/up, the MLP blocks, and down.
+//    GEMVs itself (redundantly with the other clusters): a w-wide butterfly is spread
+//    over the 8 CTAs, w/8 elements each. Every consumer thread holds one (two when
+//    w = 8192) elements. Stages of stride below 32 are warp shuffles; one transpose
+//    through shared memory turns the next five stride bits into lane bits; the last
+//    three stages (the CTA bits) follow one exchange: every CTA stores its elements
+//    straight into the owners' shared memory with st.async, whose completion is
+//    counted in bytes on the receiver's mbarrier (data and signal in one). Exchanges
+//    alternate between two receive buffers and two mbarriers, so a CTA that runs one
+//    exchange ahead never writes into data a peer is still reading.
+//  * Every thread fetches the (cos, sin) pairs of its own rotations from the layer's
+//    tables in L2 (int8 angles: the code, decoded as it rotates) when the chain starts,
+//    together with the GEMV outputs it needs; no table is staged in shared memory, which
+//    leaves it to the weight ring. Theta == 0 (the fixed randomized Hadamard transform)
+//    needs no fetch at all.
+//  * The residual stream lives in registers, in the layout the last butterfly stage
+//    leaves it in.
+//  * Grid-wide barriers (release/acquire counters) only where a whole output vector is
+//    needed: after q/k/v, o, gate/up, the MLP blocks, and down.
 //
 // Per block l (Sec. 2.1-2.2 and 5 of the HARP page for the butterflies; the glue is the
 // stack definition of include/harp.h):
@@ -35,15 +43,16 @@
 //   P4 GEMV o                                   -> grid barrier
 //   P5 chain: h_l = x_l + F_U_o(z_o), rms, F_V of gate or up, operand
 //   P6 GEMV gate or up                          -> grid barrier
-//   P7 per MLP block (one CTA each): F_U_gate, F_U_up, silu*up, F_V_down, operand to
-//      global; two otherwise idle clusters apply F_U_q and F_U_k of this block
-//                                               -> grid barrier
+//   P7 MLP blocks (one CTA each up to 512 wide, one cluster each from 2048): F_U_gate,
+//      F_U_up, silu*up, F_V_down, operand to global; the two last clusters apply F_U_q
+//      and F_U_k of this block                  -> grid barrier
 //   P8 GEMV down                                -> grid barrier
 // and after the last block: out = h_{L-1} + F_U_down(z_down).
 //
-// Every wait is bounded (about 2 s of SM clock) and checks a shared abort word, and every
-// outcome that decides control flow is made uniform across the consumer threads, so a
-// failure anywhere ends the kernel with HARP_ERR_TIMEOUT instead of a hang.
+// Every wait is bounded (about 2 s of SM clock unless the testing hook shortens it) and
+// checks a shared abort word, and every outcome that decides control flow is made
+// uniform across the consumer threads, so a failure anywhere ends the kernel with
+// HARP_ERR_TIMEOUT instead of a hang.
 #include "decode.h"
 #include "gemv_core.cuh"
 
@@ -51,6 +60,20 @@ namespace harp {
 namespace dec {
 
 using namespace gemv_core;
+
+// ------------------------------------------------------------------ GEMV unit geometry
+// 32 output rows x 2048 input columns per unit and ring stage (20 / 28 / 36 KB of codes
+// and scale/zero at 2 / 3 / 4 bits).
+template <int BITS>
+struct FGeo {
+  static constexpr int kChunkCols = 2048;
+  static constexpr int kChunkGroups = kChunkCols / 64;
+  static constexpr int kGroupsPerSlab = BITS == 4 ? 4 : 8;
+  static constexpr int kCodeSlabs = kChunkGroups / kGroupsPerSlab;
+  static constexpr int kHiSlabs = BITS == 3 ? kChunkGroups / 16 : 0;
+  static constexpr int kSzSlabs = 1;
+  static constexpr int kStageBytes = (kCodeSlabs + kHiSlabs + kSzSlabs) * kSlab;
+};
 
 // ------------------------------------------------------------------ small device helpers
 __device__ __forceinline__ uint32_t cta_rank() {
@@ -63,7 +86,7 @@ __device__ __forceinline__ uint32_t cluster_id_x() {
   asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
   return r;
 }
-// not the .aligned form: the producer warps reach the final barrier at other times
+// not the .aligned form: the producer warp reaches the final barrier at another time
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
 }
@@ -72,16 +95,18 @@ __device__ __forceinline__ uint32_t peer_addr(const void* local, uint32_t cta) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(local)), "r"(cta));
   return ra;
 }
-__device__ __forceinline__ void st_peer4(void* local, uint32_t cta, float4 v) {
-  asm volatile("st.shared::cluster.v4.f32 [%0], {%1,%2,%3,%4};" ::"r"(peer_addr(local, cta)), "f"(v.x), "f"(v.y),
-               "f"(v.z), "f"(v.w)
+// stores into CTA `cta`'s copy of `local_dst`; the receiver's copy of `local_bar` counts the bytes
+__device__ __forceinline__ void st_async_f32(float* local_dst, uint64_t* local_bar, uint32_t cta, float v) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(
+                   peer_addr(local_dst, cta)),
+               "r"(__float_as_uint(v)), "r"(peer_addr(local_bar, cta))
                : "memory");
 }
-__device__ __forceinline__ void st_peer(void* local, uint32_t cta, float v) {
-  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(peer_addr(local, cta)), "f"(v) : "memory");
-}
-__device__ __forceinline__ void arrive_remote(uint64_t* bar, uint32_t cta) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(peer_addr(bar, cta)) : "memory");
+__device__ __forceinline__ void st_async_v4(void* local_dst, uint64_t* local_bar, uint32_t cta, int4 v) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                   peer_addr(local_dst, cta)),
+               "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(peer_addr(local_bar, cta))
+               : "memory");
 }
 __device__ __forceinline__ bool try_wait_cluster(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
@@ -101,10 +126,10 @@ __device__ __forceinline__ bool aborted(const int* status) { return *(volatile c
 __shared__ long long s_wait_cycles;
 constexpr long long kAbortCheckCycles = 40000;  // start reading the shared abort word after ~20 us
 
-// bounded wait on a local mbarrier phase; false on time-out or abort. SLEEP (the
-// producer warps) backs off between polls so that a waiting producer leaves its issue
-// slots to the consumer warps sharing its scheduler.
-template <bool CLUSTER, bool SLEEP = false>
+// bounded wait on a local mbarrier phase; false on time-out, or on abort when ABORT.
+// SLEEP (the producer warp) backs off between polls so that a waiting producer leaves
+// its issue slots to the consumer warps sharing its scheduler.
+template <bool CLUSTER, bool SLEEP = false, bool ABORT = true>
 __device__ __noinline__ bool wait_phase(uint64_t* bar, uint32_t parity, int* status, int where) {
   if (CLUSTER ? try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
@@ -114,7 +139,7 @@ __device__ __noinline__ bool wait_phase(uint64_t* bar, uint32_t parity, int* sta
       if (SLEEP) __nanosleep(128);
     }
     const long long dt = clock64() - t0;
-    if (dt > kAbortCheckCycles && aborted(status)) return false;
+    if (ABORT && dt > kAbortCheckCycles && aborted(status)) return false;
     if (dt > s_wait_cycles) {
       report(status, 5, where);
       return false;
@@ -137,25 +162,31 @@ __device__ __forceinline__ bool cbar_and(bool v) {
       : "memory");
   return out != 0;
 }
-
-template <bool CLUSTER>
-__device__ __forceinline__ bool wait_uniform(uint64_t* bar, uint32_t parity, int* status, int where, int ct) {
-  bool mine = true;
-  if (ct == 0) mine = wait_phase<CLUSTER>(bar, parity, status, where);
-  return cbar_and(mine);
+// sum of an int over the consumer threads
+__device__ __forceinline__ int cbar_sum(int v, int* scratch, int ct) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if ((ct & 31) == 0) scratch[ct >> 5] = v;
+  cbar();
+  int t = 0;
+#pragma unroll
+  for (int w = 0; w < kCW; ++w) t += scratch[w];
+  cbar();
+  return t;
 }
 
 // ------------------------------------------------------------------ shared memory carve-up
-constexpr int kSgnSlot = 1024;  // bytes per prefetched sign slice (>= the widest per-CTA chunk)
+constexpr int kRxFloats = 8 * (128 + 4);  // a layout-B vector of the widest chunk (runs of 128, padded)
 
 struct Smem {
   uint8_t* ring;
-  uint8_t* tab;
-  int8_t* sgn;  // 4 slots of kSgnSlot: the sign slices of the current chain's butterflies
-  float *xa, *xb, *res, *ss, *red;
-  int* ucnt;
-  int32_t* xq;  // local GEMV operand: xq words, then xs [ng], then xsum [ng]
-  uint64_t *full, *empty, *tab_full, *tab_empty, *xchg;
+  float* T;        // local transposes and operand staging (kRxFloats)
+  float* rx[2];    // receive buffers of alternate exchanges (kRxFloats each)
+  float* misc;     // [0, 8) rms partials by source CTA, [8, 24) per-warp scratch
+  int32_t* xq;     // GEMV operand: xq words, then xs [ng], then xsum [ng]
+  float* red;      // GEMV reduction scratch: ring_stages x 16 warps x 32 lanes
+  int* ucnt;       // per ring stage: warps of the half done with the unit
+  uint64_t *full, *empty, *xbar;
 };
 
 __device__ __forceinline__ Smem carve(const Params& p, int stage_bytes) {
@@ -164,18 +195,14 @@ __device__ __forceinline__ Smem carve(const Params& p, int stage_bytes) {
   Smem s;
   s.ring = b;
   b += (size_t)p.ring_stages * stage_bytes;
-  s.tab = b;
-  b += p.tab_bytes;
-  s.sgn = reinterpret_cast<int8_t*>(b);
-  b += 4 * kSgnSlot;
-  s.xa = reinterpret_cast<float*>(b);
-  b += 4 * p.E;
-  s.xb = reinterpret_cast<float*>(b);
-  b += 4 * p.E;
-  s.res = reinterpret_cast<float*>(b);
-  b += 4 * p.E;
-  s.ss = reinterpret_cast<float*>(b);
-  b += 4 * 16;
+  s.T = reinterpret_cast<float*>(b);
+  b += 4 * kRxFloats;
+  s.rx[0] = reinterpret_cast<float*>(b);
+  b += 4 * kRxFloats;
+  s.rx[1] = reinterpret_cast<float*>(b);
+  b += 4 * kRxFloats;
+  s.misc = reinterpret_cast<float*>(b);
+  b += 4 * 32;
   s.red = reinterpret_cast<float*>(b);
   b += (size_t)4 * kCW * 32 * p.ring_stages;
   s.ucnt = reinterpret_cast<int*>(b);
@@ -184,14 +211,572 @@ __device__ __forceinline__ Smem carve(const Params& p, int stage_bytes) {
   b += p.xq_bytes;
   s.full = reinterpret_cast<uint64_t*>(b);
   s.empty = s.full + p.ring_stages;
-  s.tab_full = s.empty + p.ring_stages;
-  s.tab_empty = s.tab_full + 1;
-  s.xchg = s.tab_empty + 1;
+  s.xbar = s.empty + p.ring_stages;
   return s;
 }
 
+// ------------------------------------------------------------------ cluster exchanges
+// Exchange k (the same sequence in every CTA of the cluster) lands in rx[k & 1] and is
+// counted on xbar[k & 1]. A CTA pushes exchange k + 1 only after it has read what
+// exchange k delivered (xch_begin starts with a consumer barrier), and it can run at most
+// one exchange ahead of any peer (completing exchange k needs every peer's exchange-k
+// data), so exchange k + 2 never overwrites data a peer has not read.
+struct Xch {
+  uint32_t k = 0;
+};
+
+__device__ __forceinline__ uint32_t xb_of(const Xch& x) { return x.k & 1; }
+
+// opens exchange x.k: this CTA will receive rx_bytes from its peers
+__device__ __forceinline__ void xch_begin(Smem& s, const Xch& x, uint32_t rx_bytes, int ct) {
+  cbar();
+  if (ct == 0) mbar_arrive_expect_tx(&s.xbar[xb_of(x)], rx_bytes);
+}
+
+__device__ __forceinline__ bool xch_end(Smem& s, Xch& x, int* status, int where, int ct) {
+  bool mine = true;
+  if (ct == 0) mine = wait_phase<true>(&s.xbar[xb_of(x)], (x.k >> 1) & 1, status, where);
+  ++x.k;
+  return cbar_and(mine);
+}
+
+// a float for element slot `idx` of CTA `dst`'s receive buffer of this exchange
+__device__ __forceinline__ void put(Smem& s, const Xch& x, uint32_t me, uint32_t dst, int idx, float v) {
+  float* buf = s.rx[xb_of(x)] + idx;
+  if (dst == me) *buf = v;
+  else st_async_f32(buf, &s.xbar[xb_of(x)], dst, v);
+}
+
+// ------------------------------------------------------------------ element maps
+// A butterfly whose CTA share is E = 2^EB elements (a w = 8E wide block spread over the
+// cluster, or a whole block of w = E in one CTA):
+//   phase 1: thread ct holds e = s * 512 + ct: stages 0..4 pair lanes (shuffles);
+//   phase 2: after a transpose, lane bits 0..L2-1 hold e bits 5..5+L2-1, so stages 5..EB-1
+//            pair lanes again; e bits 0..4 come from the remaining lane bits, the warp
+//            and the slot s;
+//   layout B (cluster butterflies): CTA r holds, for every CTA index j, the run
+//            [j E + r run, +run), run = E/8: thread ct holds j = lane & 7 and the offset
+//            ii = (lane >> 3) | (warp << 2) | (s << 6), so the three cross-CTA stages pair
+//            lanes 1, 2 and 4 apart.
+// s < P = max(1, E / 512) slots per thread; threads from min(E, 512) on hold nothing.
+template <int EB>
+struct Map {
+  static constexpr int E = 1 << EB;
+  static constexpr int P = E > kNT ? E / kNT : 1;
+  static constexpr int NT = E < kNT ? E : kNT;
+  static constexpr int L2 = EB - 5 < 5 ? EB - 5 : 5;
+  static constexpr int RUN = E / kC;
+  static constexpr int RB = EB - 3;
+  static constexpr int PAD = RUN + 4;  // run stride in the layout-B buffer: a warp's reads hit 32 banks
+  __device__ static int e1(int ct, int s) { return s * kNT + ct; }
+  __device__ static int e2(int ct, int s) {
+    if constexpr (EB <= 5) {
+      return e1(ct, s);
+    } else {
+      const int lane = ct & 31, warp = ct >> 5;
+      return ((lane & ((1 << L2) - 1)) << 5) | (((lane >> L2) | (warp << (5 - L2)) | (s << (9 - L2))) & 31);
+    }
+  }
+  __device__ static int bj(int ct) { return ct & 7; }
+  __device__ static int bii(int ct, int s) { return ((ct & 31) >> 3) | ((ct >> 5) << 2) | (s << 6); }
+  __device__ static int idx_b(int j, int ii) { return j * PAD + ii; }
+};
+
+// layout-A buffer index: xor swizzle keeps a warp's phase-1 and phase-2 accesses on
+// (nearly) distinct banks
+__device__ __forceinline__ int idx_a(int e) { return e ^ ((e >> 5) & 31); }
+
+// pair number of element g in stage t (pairs numbered by their first index)
+__device__ __forceinline__ int64_t pair_of(int64_t g, int t) {
+  return ((g >> (t + 1)) << t) | (g & ((int64_t(1) << t) - 1));
+}
+
+// ------------------------------------------------------------------ rotation coefficients
+// What a thread keeps in registers per rotation: the (cos, sin) pair, the angle pi/4 +
+// delta_t q of an int8 layer (decoded by the fast sine/cosine unit when the stage runs),
+// or nothing for Theta == 0.
+template <int TM>
+struct Cf {
+  float2 v;
+};
+template <>
+struct Cf<kTmQ8> {
+  float psi;
+};
+template <>
+struct Cf<kTmHad> {};
+
+constexpr float kQuarterPi = 0.785398163397448309616f;
+constexpr float kRsqrt2 = 0.70710678118654752440f;  // cos(pi/4) = sin(pi/4): the Theta == 0 block
+
+// tab: the side's angle storage (float2 [m][n/2], or int8 after a 64-byte head of steps)
+template <int TM>
+__device__ __forceinline__ Cf<TM> fetch_cf(const uint8_t* tab, int64_t half_n, int t, int64_t q) {
+  Cf<TM> c;
+  if constexpr (TM == kTmCS) {
+    c.v = __ldg(reinterpret_cast<const float2*>(tab) + (int64_t)t * half_n + q);
+  } else if constexpr (TM == kTmQ8) {
+    const float step = __ldg(reinterpret_cast<const float*>(tab) + t);
+    const int8_t code = __ldg(reinterpret_cast<const int8_t*>(tab + kQ8Head) + (int64_t)t * half_n + q);
+    c.psi = fmaf(step, (float)code, kQuarterPi);
+  }
+  return c;
+}
+
+template <int TM>
+__device__ __forceinline__ float2 cs_of(const Cf<TM>& c) {
+  if constexpr (TM == kTmCS) {
+    return c.v;
+  } else if constexpr (TM == kTmQ8) {
+    float sn, co;
+    __sincosf(c.psi, &sn, &co);
+    return make_float2(co, sn);
+  } else {
+    return make_float2(kRsqrt2, kRsqrt2);
+  }
+}
+
+// one 2x2 block [[c, s], [s, -c]] applied to the pair (a, b) held by two lanes: the lane
+// holding a (upper = false) gets c a + s b, the lane holding b gets s a - c b
+template <int TM>
+__device__ __forceinline__ float rot_lane(float v, int lanes, bool upper, const Cf<TM>& cf) {
+  const float p = __shfl_xor_sync(0xffffffffu, v, lanes);
+  const float2 cs = cs_of<TM>(cf);
+  return fmaf(upper ? -cs.x : cs.x, v, cs.y * p);
+}
+
+// ------------------------------------------------------------------ butterfly engines
+// Cluster-distributed F(theta, s, w) over one w = 8E wide block (block `blk` of the side's
+// n-vector). fetch() loads the thread's coefficients; run() takes the signed input in
+// phase-1 order and leaves the output in layout B.
+template <int EB, int TM>
+struct ClusterBfly {
+  using M = Map<EB>;
+  static constexpr int NS = EB + 3;
+  Cf<TM> cf[NS][M::P];
+
+  __device__ __forceinline__ void fetch(const uint8_t* tab, int64_t half_n, int64_t blk, uint32_t r, int ct) {
+    if constexpr (TM != kTmHad) {
+      if (ct >= M::NT) return;
+      const int64_t base = blk * (int64_t)(kC * M::E);
+#pragma unroll
+      for (int s = 0; s < M::P; ++s) {
+        const int64_t g1 = base + (int64_t)r * M::E + M::e1(ct, s);
+        const int64_t g2 = base + (int64_t)r * M::E + M::e2(ct, s);
+        const int64_t gb = base + (int64_t)M::bj(ct) * M::E + (int64_t)r * M::RUN + M::bii(ct, s);
+#pragma unroll
+        for (int t = 0; t < NS; ++t)
+          cf[t][s] = fetch_cf<TM>(tab, half_n, t, pair_of(t < 5 ? g1 : (t < EB ? g2 : gb), t));
+      }
+    }
+  }
+
+  // v: this CTA's chunk in phase-1 order, signs applied. Returns with v in layout B.
+  __device__ __forceinline__ bool run(float (&v)[2], Smem& sm, Xch& x, uint32_t r, int ct, int* status,
+                                      int where) {
+    const bool act = ct < M::NT;
+    if (act) {
+#pragma unroll
+      for (int t = 0; t < (EB < 5 ? EB : 5); ++t)
+#pragma unroll
+        for (int s = 0; s < M::P; ++s) v[s] = rot_lane<TM>(v[s], 1 << t, (M::e1(ct, s) >> t) & 1, cf[t][s]);
+    }
+    if constexpr (EB > 5) {
+      cbar();  // earlier readers of T are done
+      if (act)
+#pragma unroll
+        for (int s = 0; s < M::P; ++s) sm.T[idx_a(M::e1(ct, s))] = v[s];
+      cbar();
+      if (act) {
+#pragma unroll
+        for (int s = 0; s < M::P; ++s) v[s] = sm.T[idx_a(M::e2(ct, s))];
+#pragma unroll
+        for (int t = 5; t < EB; ++t)
+#pragma unroll
+          for (int s = 0; s < M::P; ++s)
+            v[s] = rot_lane<TM>(v[s], 1 << (t - 5), (M::e2(ct, s) >> t) & 1, cf[t][s]);
+      }
+    }
+    // layout A -> B: element e goes to CTA e / run, slot (j = r, ii = e mod run)
+    xch_begin(sm, x, 4u * M::RUN * (kC - 1), ct);
+    if (act)
+#pragma unroll
+      for (int s = 0; s < M::P; ++s) {
+        const int e = M::e2(ct, s);
+        put(sm, x, r, (uint32_t)(e >> M::RB), M::idx_b((int)r, e & (M::RUN - 1)), v[s]);
+      }
+    const float* rx = sm.rx[xb_of(x)];
+    const bool ok = xch_end(sm, x, status, where, ct);
+    if (act) {
+#pragma unroll
+      for (int s = 0; s < M::P; ++s) v[s] = rx[M::idx_b(M::bj(ct), M::bii(ct, s))];
+#pragma unroll
+      for (int d = 0; d < 3; ++d)
+#pragma unroll
+        for (int s = 0; s < M::P; ++s) v[s] = rot_lane<TM>(v[s], 1 << d, (M::bj(ct) >> d) & 1, cf[EB + d][s]);
+    }
+    return ok;
+  }
+
+  // global (within the block) element index of slot s in layout B
+  __device__ __forceinline__ static int gb(uint32_t r, int ct, int s) {
+    return M::bj(ct) * M::E + (int)r * M::RUN + M::bii(ct, s);
+  }
+  __device__ __forceinline__ static int ga(uint32_t r, int ct, int s) { return (int)r * M::E + M::e1(ct, s); }
+};
+
+// A whole w = 2^EB block (EB <= 9) in one CTA: phase-1 input, phase-2 output.
+template <int EB, int TM>
+struct LocalBfly {
+  using M = Map<EB>;
+  Cf<TM> cf[EB];
+
+  __device__ __forceinline__ void fetch(const uint8_t* tab, int64_t half_n, int64_t blk, int ct) {
+    if constexpr (TM != kTmHad) {
+      if (ct >= M::NT) return;
+      const int64_t base = blk * (int64_t)M::E;
+#pragma unroll
+      for (int t = 0; t < EB; ++t)
+        cf[t] = fetch_cf<TM>(tab, half_n, t, pair_of(base + (t < 5 ? M::e1(ct, 0) : M::e2(ct, 0)), t));
+    }
+  }
+
+  __device__ __forceinline__ void run(float& v, Smem& sm, int ct) {
+    const bool act = ct < M::NT;
+    if (act)
+#pragma unroll
+      for (int t = 0; t < (EB < 5 ? EB : 5); ++t) v = rot_lane<TM>(v, 1 << t, (M::e1(ct, 0) >> t) & 1, cf[t]);
+    if constexpr (EB > 5) {
+      cbar();
+      if (act) sm.T[idx_a(M::e1(ct, 0))] = v;
+      cbar();
+      if (act) {
+        v = sm.T[idx_a(M::e2(ct, 0))];
+#pragma unroll
+        for (int t = 5; t < EB; ++t) v = rot_lane<TM>(v, 1 << (t - 5), (M::e2(ct, 0) >> t) & 1, cf[t]);
+      }
+    }
+  }
+};
+
+// ------------------------------------------------------------------ GEMV operand
+// x~ of a hidden-wide input in layout B (runs of >= 64): the CTA's groups into its own
+// operand buffer, then to every peer's (one exchange)
+template <int EB>
+__device__ bool prep_broadcast(const float (&v)[2], int n_in, int bits, Smem& sm, Xch& x, uint32_t r, int ct,
+                               int* status) {
+  using M = Map<EB>;
+  static_assert(M::RUN >= 64, "operand groups must lie inside one run");
+  constexpr int GPR = M::RUN / 64, NGL = M::E / 64;  // groups per run, groups of this CTA
+  const int warp = ct >> 5, lane = ct & 31;
+  const int words = bits == 3 ? n_in : n_in / 2, ng = n_in / 64;
+  int16_t* xq16 = reinterpret_cast<int16_t*>(sm.xq);
+  float* xsA = reinterpret_cast<float*>(sm.xq + words);
+  float* xsumA = xsA + ng;
+  cbar();
+  if (ct < M::NT)
+#pragma unroll
+    for (int s = 0; s < M::P; ++s) sm.T[M::idx_b(M::bj(ct), M::bii(ct, s))] = v[s];
+  cbar();
+  if (warp < NGL) {
+    const int j = warp / GPR, kk = warp - j * GPR;
+    const int G = (j * M::E + (int)r * M::RUN + 64 * kk) >> 6;
+    prep_group(sm.T + j * M::PAD + 64 * kk, bits, xq16 + (int64_t)G * 64, xq16 + n_in + (int64_t)G * 64, xsA + G,
+               xsumA + G, lane);
+  }
+  const int planes = bits == 3 ? 2 : 1;
+  xch_begin(sm, x, (uint32_t)((kC - 1) * NGL * (128 * planes + 8)), ct);  // starts with a barrier: prep is done
+  uint64_t* bar = &sm.xbar[xb_of(x)];
+  // 8 int4 per group and plane, to the 7 peers
+  for (int it = ct; it < NGL * planes * 8 * (kC - 1); it += kNT) {
+    const int qi = it % (kC - 1), rest = it / (kC - 1);
+    const int part = rest & 7, pl = (rest >> 3) % planes, lg = (rest >> 3) / planes;
+    const uint32_t q = (uint32_t)(qi < (int)r ? qi : qi + 1);
+    const int j = lg / GPR, kk = lg - j * GPR;
+    const int G = (j * M::E + (int)r * M::RUN + 64 * kk) >> 6;
+    const int word = pl * (n_in / 2) + G * 32 + part * 4;
+    st_async_v4(sm.xq + word, bar, q, *reinterpret_cast<const int4*>(sm.xq + word));
+  }
+  for (int it = ct; it < NGL * (kC - 1); it += kNT) {
+    const int qi = it % (kC - 1), lg = it / (kC - 1);
+    const uint32_t q = (uint32_t)(qi < (int)r ? qi : qi + 1);
+    const int j = lg / GPR, kk = lg - j * GPR;
+    const int G = (j * M::E + (int)r * M::RUN + 64 * kk) >> 6;
+    st_async_f32(xsA + G, bar, q, xsA[G]);
+    st_async_f32(xsumA + G, bar, q, xsumA[G]);
+  }
+  return xch_end(sm, x, status, 40, ct);
+}
+
+// sum of the split-K partials of element i (fixed order)
+__device__ __forceinline__ float zsum(const float* zp, int nk, int64_t n, int64_t i) {
+  float t = __ldcg(zp + i);
+  for (int k = 1; k < nk; ++k) t += __ldcg(zp + (int64_t)k * n + i);
+  return t;
+}
+
+// ------------------------------------------------------------------ chains (cluster-collective)
+// Residual chain: [res += F_U(z)] ; n = rms(res) ; x~ = F_V(n) ; operand. EB: log2 of the
+// hidden-wide chunk (hidden / 8). U null: res is the step's input; V null: the final step.
+template <int EB, int TM>
+__device__ __noinline__ bool chain_residual(const Params& p, Smem& sm, Xch& x, float (&res)[2], const Lin* U,
+                                            const float* zp, int nk, const Lin* V, uint32_t r, int ct) {
+  using M = Map<EB>;
+  using BF = ClusterBfly<EB, TM>;
+  const bool act = ct < M::NT;
+  bool ok = true;
+  if (!U) {
+    if (act)
+#pragma unroll
+      for (int s = 0; s < M::P; ++s) res[s] = load_act(p.x_in, BF::gb(r, ct, s), p.xt);
+  } else {
+    BF fu;
+    fu.fetch(U->tU, (int64_t)U->n_out / 2, 0, r, ct);
+    float v[2] = {0.f, 0.f};
+    if (act)
+#pragma unroll
+      for (int s = 0; s < M::P; ++s) {
+        const int g = BF::ga(r, ct, s);
+        v[s] = zsum(zp, nk, U->n_out, g) * (float)__ldg(U->sU + g);
+      }
+    ok = fu.run(v, sm, x, r, ct, p.status, 41);
+    if (act)
+#pragma unroll
+      for (int s = 0; s < M::P; ++s) res[s] += v[s];
+  }
+  if (!V || !ok) return ok;
+  BF fv;
+  fv.fetch(V->tV, (int64_t)V->n_in / 2, 0, r, ct);
+  // sum of squares: warps, then the CTA (fixed order), then to every peer's slot r along
+  // with the residual values each peer holds in layout A for F_V
+  float acc = 0.f;
+  if (act)
+#pragma unroll
+    for (int s = 0; s < M::P; ++s) acc = fmaf(res[s], res[s], acc);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if ((ct & 31) == 0) sm.misc[8 + (ct >> 5)] = acc;
+  xch_begin(sm, x, 4u * M::RUN * (kC - 1) + 4u * (kC - 1), ct);
+  if (ct == 0) {
+    float t = 0.f;
+    for (int w = 0; w < kCW; ++w) t += sm.misc[8 + w];
+    for (uint32_t q = 0; q < kC; ++q)
+      if (q == r) sm.misc[r] = t;
+      else st_async_f32(sm.misc + r, &sm.xbar[xb_of(x)], q, t);
+  }
+  if (act)
+#pragma unroll
+    for (int s = 0; s < M::P; ++s) {
+      const int j = M::bj(ct), ii = M::bii(ct, s);
+      put(sm, x, r, (uint32_t)j, idx_a((int)r * M::RUN + ii), res[s]);
+    }
+  const float* rx = sm.rx[xb_of(x)];
+  if (!(ok = xch_end(sm, x, p.status, 42, ct))) return false;
+  float tot = 0.f;
+  for (int q = 0; q < kC; ++q) tot += sm.misc[q];
+  const float inv = 1.0f / sqrtf(tot / (float)p.hidden + p.eps);
+  float v[2] = {0.f, 0.f};
+  if (act)
+#pragma unroll
+    for (int s = 0; s < M::P; ++s) {
+      const int e = M::e1(ct, s);
+      v[s] = rx[idx_a(e)] * inv * (float)__ldg(V->sV + (int)r * M::E + e);
+    }
+  if (!(ok = fv.run(v, sm, x, r, ct, p.status, 43))) return false;
+  return prep_broadcast<EB>(v, V->n_in, p.bits, sm, x, r, ct, p.status);
+}
+
+// attention chain: v = F_U_v(z_v); a = v repeated per KV group; x~ = F_V_o(a); operand.
+// EBU: log2 of the v chunk (dkv / 8), EB: of the hidden chunk.
+template <int EBU, int EB, int TM>
+__device__ __noinline__ bool chain_attn(const Params& p, Smem& sm, Xch& x, const Lin* Lv, const Lin* Lo, uint32_t r,
+                                        int ct) {
+  using MU = Map<EBU>;
+  using M = Map<EB>;
+  ClusterBfly<EBU, TM> fu;
+  fu.fetch(Lv->tU, (int64_t)Lv->n_out / 2, 0, r, ct);
+  float v[2] = {0.f, 0.f};
+  if (ct < MU::NT)
+#pragma unroll
+    for (int s = 0; s < MU::P; ++s) {
+      const int g = ClusterBfly<EBU, TM>::ga(r, ct, s);
+      v[s] = zsum(p.zpv, p.nk_h, Lv->n_out, g) * (float)__ldg(Lv->sU + g);
+    }
+  if (!fu.run(v, sm, x, r, ct, p.status, 44)) return false;
+  ClusterBfly<EB, TM> fv;
+  fv.fetch(Lo->tV, (int64_t)Lo->n_in / 2, 0, r, ct);
+  // every v value to the layout-A owners of the query-head elements that copy it
+  const int hd = p.head_dim, rep = p.rep;
+  int self = 0;
+  if (ct < MU::NT)
+#pragma unroll
+    for (int s = 0; s < MU::P; ++s) {
+      const int gv = ClusterBfly<EBU, TM>::gb(r, ct, s), kvh = gv / hd, d = gv - kvh * hd;
+      for (int h = kvh * rep; h < (kvh + 1) * rep; ++h) self += ((h * hd + d) >> EB) == (int)r;
+    }
+  self = cbar_sum(self, reinterpret_cast<int*>(sm.misc + 8), ct);
+  xch_begin(sm, x, 4u * (uint32_t)(M::E - self), ct);
+  if (ct < MU::NT)
+#pragma unroll
+    for (int s = 0; s < MU::P; ++s) {
+      const int gv = ClusterBfly<EBU, TM>::gb(r, ct, s), kvh = gv / hd, d = gv - kvh * hd;
+      for (int h = kvh * rep; h < (kvh + 1) * rep; ++h) {
+        const int ga = h * hd + d;
+        put(sm, x, r, (uint32_t)(ga >> EB), idx_a(ga & (M::E - 1)), v[s]);
+      }
+    }
+  const float* rx = sm.rx[xb_of(x)];
+  if (!xch_end(sm, x, p.status, 45, ct)) return false;
+  float w[2] = {0.f, 0.f};
+  if (ct < M::NT)
+#pragma unroll
+    for (int s = 0; s < M::P; ++s) {
+      const int e = M::e1(ct, s);
+      w[s] = rx[idx_a(e)] * (float)__ldg(Lo->sV + (int)r * M::E + e);
+    }
+  if (!fv.run(w, sm, x, r, ct, p.status, 46)) return false;
+  return prep_broadcast<EB>(w, Lo->n_in, p.bits, sm, x, r, ct, p.status);
+}
+
+// F_U of a q or k GEMV output (cluster-distributed), written to out[g]
+template <int EB, int TM>
+__device__ __noinline__ bool chain_out_only(const Params& p, Smem& sm, Xch& x, const Lin* Lq, const float* zp,
+                                            float* out, uint32_t r, int ct) {
+  using M = Map<EB>;
+  using BF = ClusterBfly<EB, TM>;
+  BF fu;
+  fu.fetch(Lq->tU, (int64_t)Lq->n_out / 2, 0, r, ct);
+  float v[2] = {0.f, 0.f};
+  if (ct < M::NT)
+#pragma unroll
+    for (int s = 0; s < M::P; ++s) {
+      const int g = BF::ga(r, ct, s);
+      v[s] = zsum(zp, p.nk_h, Lq->n_out, g) * (float)__ldg(Lq->sU + g);
+    }
+  const bool ok = fu.run(v, sm, x, r, ct, p.status, 47);
+  if (ok && ct < M::NT)
+#pragma unroll
+    for (int s = 0; s < M::P; ++s) out[BF::gb(r, ct, s)] = v[s];
+  return ok;
+}
+
+__device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
+
+// One MLP block of width 2^EB <= 512 in one CTA: F_U_gate, F_U_up, silu * up, F_V_down,
+// operand of the down projection for this block (to global)
+template <int EB, int TM>
+__device__ __noinline__ void mlp_block_local(const Params& p, Smem& sm, const Lin* Lg, const Lin* Lu, const Lin* Ld,
+                                             int blk, int ct) {
+  using M = Map<EB>;
+  LocalBfly<EB, TM> fg, fu, fd;
+  fg.fetch(Lg->tU, (int64_t)Lg->n_out / 2, blk, ct);
+  fu.fetch(Lu->tU, (int64_t)Lu->n_out / 2, blk, ct);
+  fd.fetch(Ld->tV, (int64_t)Ld->n_in / 2, blk, ct);
+  const bool act = ct < M::NT;
+  const int64_t base = (int64_t)blk * M::E;
+  float vg = 0.f, vu = 0.f;
+  if (act) {
+    const int64_t g = base + M::e1(ct, 0);
+    vg = zsum(p.zpg, p.nk_h, Lg->n_out, g) * (float)__ldg(Lg->sU + g);
+    vu = zsum(p.zpu, p.nk_h, Lu->n_out, g) * (float)__ldg(Lu->sU + g);
+  }
+  fg.run(vg, sm, ct);
+  fu.run(vu, sm, ct);
+  // both in phase-2 order; F_V_down starts from phase-1 order
+  float h = 0.f;
+  if (act) {
+    const int64_t g = base + M::e2(ct, 0);
+    h = silu(vg) * vu * (float)__ldg(Ld->sV + g);
+  }
+  cbar();
+  if (act) sm.T[idx_a(M::e2(ct, 0))] = h;
+  cbar();
+  if (act) h = sm.T[idx_a(M::e1(ct, 0))];
+  fd.run(h, sm, ct);
+  cbar();
+  if (act) sm.T[M::e2(ct, 0)] = h;  // natural order for the groups
+  cbar();
+  const int warp = ct >> 5, lane = ct & 31, n_in = Ld->n_in;
+  int16_t* xq16 = reinterpret_cast<int16_t*>(p.xq_down);
+  if (warp < (M::E >> 6)) {
+    const int G = (int)(base >> 6) + warp;
+    prep_group(sm.T + 64 * warp, p.bits, xq16 + (int64_t)G * 64, xq16 + n_in + (int64_t)G * 64, p.xs_down + G,
+               p.xsum_down + G, lane);
+  }
+}
+
+// One MLP block of width 8 * 2^EB (>= 2048) on one cluster: the same steps, each
+// butterfly spread over the cluster; the operand groups go to global from layout B.
+template <int EB, int TM>
+__device__ __noinline__ bool mlp_block_cluster(const Params& p, Smem& sm, Xch& x, const Lin* Lg, const Lin* Lu,
+                                               const Lin* Ld, int blk, uint32_t r, int ct) {
+  using M = Map<EB>;
+  using BF = ClusterBfly<EB, TM>;
+  static_assert(M::RUN >= 64, "operand groups must lie inside one run");
+  constexpr int W = kC * M::E;
+  const bool act = ct < M::NT;
+  const int64_t base = (int64_t)blk * W;
+  float vg[2] = {0.f, 0.f}, vu[2] = {0.f, 0.f};
+  {
+    BF fg;
+    fg.fetch(Lg->tU, (int64_t)Lg->n_out / 2, blk, r, ct);
+    if (act)
+#pragma unroll
+      for (int s = 0; s < M::P; ++s) {
+        const int64_t g = base + BF::ga(r, ct, s);
+        vg[s] = zsum(p.zpg, p.nk_h, Lg->n_out, g) * (float)__ldg(Lg->sU + g);
+      }
+    if (!fg.run(vg, sm, x, r, ct, p.status, 48)) return false;
+  }
+  {
+    BF fu;
+    fu.fetch(Lu->tU, (int64_t)Lu->n_out / 2, blk, r, ct);
+    if (act)
+#pragma unroll
+      for (int s = 0; s < M::P; ++s) {
+        const int64_t g = base + BF::ga(r, ct, s);
+        vu[s] = zsum(p.zpu, p.nk_h, Lu->n_out, g) * (float)__ldg(Lu->sU + g);
+      }
+    if (!fu.run(vu, sm, x, r, ct, p.status, 49)) return false;
+  }
+  BF fd;
+  fd.fetch(Ld->tV, (int64_t)Ld->n_in / 2, blk, r, ct);
+  // h = silu(gate) * up in layout B, to the layout-A owners
+  xch_begin(sm, x, 4u * M::RUN * (kC - 1), ct);
+  if (act)
+#pragma unroll
+    for (int s = 0; s < M::P; ++s)
+      put(sm, x, r, (uint32_t)M::bj(ct), idx_a((int)r * M::RUN + M::bii(ct, s)), silu(vg[s]) * vu[s]);
+  const float* rx = sm.rx[xb_of(x)];
+  if (!xch_end(sm, x, p.status, 50, ct)) return false;
+  float v[2] = {0.f, 0.f};
+  if (act)
+#pragma unroll
+    for (int s = 0; s < M::P; ++s) {
+      const int e = M::e1(ct, s);
+      v[s] = rx[idx_a(e)] * (float)__ldg(Ld->sV + base + (int)r * M::E + e);
+    }
+  if (!fd.run(v, sm, x, r, ct, p.status, 51)) return false;
+  // groups of 64 inside the runs, to the global down operand
+  constexpr int GPR = M::RUN / 64, NGL = M::E / 64;
+  cbar();
+  if (act)
+#pragma unroll
+    for (int s = 0; s < M::P; ++s) sm.T[M::idx_b(M::bj(ct), M::bii(ct, s))] = v[s];
+  cbar();
+  const int warp = ct >> 5, lane = ct & 31, n_in = Ld->n_in;
+  int16_t* xq16 = reinterpret_cast<int16_t*>(p.xq_down);
+  if (warp < NGL) {
+    const int j = warp / GPR, kk = warp - j * GPR;
+    const int G = (int)((base + j * M::E + (int)r * M::RUN + 64 * kk) >> 6);
+    prep_group(sm.T + j * M::PAD + 64 * kk, p.bits, xq16 + (int64_t)G * 64, xq16 + n_in + (int64_t)G * 64,
+               p.xs_down + G, p.xsum_down + G, lane);
+  }
+  return true;
+}
+
 // ------------------------------------------------------------------ GEMV work units
-// A unit is 32 output rows x one column chunk of one linear: exactly one ring stage.
+// A unit is 32 output rows x one 2048-column chunk of one linear: exactly one ring stage.
 struct Range {
   const Lin* L;
   float* zp;  // partial sums [nk][n_out]
@@ -226,7 +811,7 @@ __device__ __forceinline__ Range units(const Params& p, int l, int ph, int c, in
     parts = p.G * kC;
     g.zp = ph == 1 ? p.zpo : p.zpd;
   }
-  g.nk = (g.L->n_in + Geo<BITS>::kChunkCols - 1) / Geo<BITS>::kChunkCols;
+  g.nk = (g.L->n_in + FGeo<BITS>::kChunkCols - 1) / FGeo<BITS>::kChunkCols;
   const int U = ((g.L->n_out + 31) / 32) * g.nk;
   g.u0 = split(U, i, parts);
   g.u1 = split(U, i + 1, parts);
@@ -260,7 +845,7 @@ struct UnitCursor {
 // the boxes of one unit, as the ring loads them, requested into L2
 template <int BITS>
 __device__ __forceinline__ void prefetch_unit(const Range& g, int u) {
-  using Gm = Geo<BITS>;
+  using Gm = FGeo<BITS>;
   const int ngroups = g.L->n_in / 64;
   const int tile = u / g.nk, kc = u - tile * g.nk;
   const int g0 = kc * Gm::kChunkGroups, gc = min(Gm::kChunkGroups, ngroups - g0);
@@ -272,488 +857,15 @@ __device__ __forceinline__ void prefetch_unit(const Range& g, int u) {
   for (int q = 0; q < (gc + 31) / 32; ++q) tma_prefetch_l2_2d(&g.L->tm_sz, g0 + q * 32, tile * 32);
 }
 
-// ------------------------------------------------------------------ table loads (producer warp 1)
-// Table of one butterfly in shared memory: stage t holds the (cos, sin) pairs of the
-// CTA's rotations in stage order, E/2 entries of 8 bytes. fp32 tables are copied as they
-// are; int8 angles are expanded into pairs by the producer warp as it stages them, so the
-// activation chains read the same table format whatever the layer keeps in memory.
-template <int TM>
-__device__ __forceinline__ constexpr int tab_esz() { return 8; }
-template <int TM>
-__device__ __forceinline__ constexpr int tab_head() { return 0; }
-
-template <int TM>
-__device__ __forceinline__ uint32_t table_bytes_cluster(int w, int m) {
-  return (uint32_t)(tab_head<TM>() + tab_esz<TM>() * m * (w / kC / 2));
-}
-template <int TM>
-__device__ __forceinline__ uint32_t table_bytes_local(int w, int m) {
-  return (uint32_t)(tab_head<TM>() + tab_esz<TM>() * m * (w / 2));
-}
-// bytes a table load transfers by bulk copy (fp32 tables only: none for Theta == 0, and
-// int8 angles are expanded by the warp's own loads)
-template <int TM>
-__device__ __forceinline__ uint32_t copied_bytes_cluster(const uint8_t* src, int w, int m) {
-  return TM != kTmCS || !src ? 0u : table_bytes_cluster<TM>(w, m);
-}
-template <int TM>
-__device__ __forceinline__ uint32_t copied_bytes_local(const uint8_t* src, int w, int m) {
-  return TM != kTmCS || !src ? 0u : table_bytes_local<TM>(w, m);
-}
-
-// pair index, in the stage's full row, of entry q of the CTA's slice of a
-// cluster-distributed stage t (the order load_table_cluster copies them in)
-__device__ __forceinline__ int64_t slice_pair(int t, int q, int E, int e, int r) {
-  if (t < e) return (int64_t)r * (E >> 1) + q;
-  const int run = E / kC, dd = t - e, jj = q / run, ii = q - jj * run;
-  const int j = ((jj >> dd) << (dd + 1)) | (jj & ((1 << dd) - 1));
-  return (int64_t)(j >> (dd + 1)) * (1 << t) + (int64_t)E * (j & ((1 << dd) - 1)) + (int64_t)r * run + ii;
-}
-
-// int8 angles -> (cos, sin) of pi/4 + delta_t q for the CTA's slice (all 32 lanes of the
-// producer warp; the fast sine/cosine unit, about 5e-7 absolute error near pi/4)
-__device__ __noinline__ void expand_cluster(uint8_t* dst, const uint8_t* q8, int64_t n, int w, int m, int r,
-                                            int lane) {
-  if (!q8) return;
-  const int E = w / kC, e = m - 3;
-  const int64_t half_n = n >> 1;
-  const float* steps = reinterpret_cast<const float*>(q8);
-  const int8_t* codes = reinterpret_cast<const int8_t*>(q8 + kQ8Head);
-  float2* out = reinterpret_cast<float2*>(dst);
-  for (int t = 0; t < m; ++t) {
-    const float st = __ldg(steps + t);
-    for (int q = lane; q < (E >> 1); q += 32) {
-      float sn, cs;
-      __sincosf(fmaf(st, (float)__ldg(codes + (int64_t)t * half_n + slice_pair(t, q, E, e, r)),
-                     0.785398163397448309616f),
-                &sn, &cs);
-      out[(size_t)t * (E >> 1) + q] = make_float2(cs, sn);
-    }
-  }
-}
-
-// the same for block `blk` of width w held whole by one CTA
-__device__ __noinline__ void expand_local(uint8_t* dst, const uint8_t* q8, int64_t n, int w, int m, int blk,
-                                          int lane) {
-  if (!q8) return;
-  const float* steps = reinterpret_cast<const float*>(q8);
-  const int8_t* codes = reinterpret_cast<const int8_t*>(q8 + kQ8Head);
-  float2* out = reinterpret_cast<float2*>(dst);
-  for (int t = 0; t < m; ++t) {
-    const float st = __ldg(steps + t);
-    for (int q = lane; q < (w >> 1); q += 32) {
-      float sn, cs;
-      __sincosf(fmaf(st, (float)__ldg(codes + (int64_t)t * (n >> 1) + (int64_t)blk * (w >> 1) + q),
-                     0.785398163397448309616f),
-                &sn, &cs);
-      out[(size_t)t * (w >> 1) + q] = make_float2(cs, sn);
-    }
-  }
-}
-
-// Per-CTA slice of a cluster-distributed butterfly (width w, C = 8): stage t < e is the
-// contiguous run of the CTA's chunk; stage t >= e is C/2 runs of `run` pairs.
-template <int TM>
-__device__ __forceinline__ uint32_t load_table_cluster(uint8_t* dst, const uint8_t* src, int64_t n, int w, int m,
-                                                       int blk, int r, uint64_t* bar) {
-  constexpr int esz = tab_esz<TM>(), head = tab_head<TM>();
-  const int E = w / kC, e = m - 3, run = E / kC;
-  const int64_t half_n = n >> 1;
-  if (TM != kTmCS || !src) return table_bytes_cluster<TM>(w, m);  // nothing to copy, same layout
-  if (head) bulk_g2s(dst, src, (uint32_t)head, bar);
-  for (int t = 0; t < m; ++t) {
-    const uint8_t* st = src + head + ((int64_t)t * half_n + (int64_t)blk * (w >> 1)) * esz;
-    uint8_t* d = dst + head + (size_t)t * (E >> 1) * esz;
-    if (t < e) {
-      bulk_g2s(d, st + (int64_t)r * (E >> 1) * esz, (uint32_t)(esz * (E >> 1)), bar);
-    } else {
-      const int dd = t - e;
-      for (int jj = 0; jj < (kC >> 1); ++jj) {
-        const int j = ((jj >> dd) << (dd + 1)) | (jj & ((1 << dd) - 1));
-        const int64_t pb = (int64_t)(j >> (dd + 1)) * (1 << t) + (int64_t)E * (j & ((1 << dd) - 1)) + (int64_t)r * run;
-        bulk_g2s(d + (size_t)jj * run * esz, st + pb * esz, (uint32_t)(esz * run), bar);
-      }
-    }
-  }
-  return table_bytes_cluster<TM>(w, m);
-}
-
-// the whole block `blk` of width w held by one CTA: one run of w/2 pairs per stage
-template <int TM>
-__device__ __forceinline__ uint32_t load_table_local(uint8_t* dst, const uint8_t* src, int64_t n, int w, int m, int blk,
-                                                     uint64_t* bar) {
-  constexpr int esz = tab_esz<TM>(), head = tab_head<TM>();
-  if (TM != kTmCS || !src) return table_bytes_local<TM>(w, m);
-  if (head) bulk_g2s(dst, src, (uint32_t)head, bar);
-  for (int t = 0; t < m; ++t)
-    bulk_g2s(dst + head + (size_t)t * (w >> 1) * esz, src + head + ((int64_t)t * (n >> 1) + (int64_t)blk * (w >> 1)) * esz,
-             (uint32_t)(esz * (w >> 1)), bar);
-  return table_bytes_local<TM>(w, m);
-}
-
-// P7 roles: block CTAs, and the clusters applying F_U_q / F_U_k
-__device__ __forceinline__ int qk_cluster(const Params& p, int which) { return p.G - 1 - which; }
-
-// ------------------------------------------------------------------ butterfly stages
-constexpr float kRsqrt2 = 0.70710678118654752440f;  // cos(pi/4) = sin(pi/4): the Theta == 0 block
-
-// One stage's row of a table of E/2 entries per stage: (cos, sin) pairs, or int8 angles
-// with the stage's step.
-struct StageTab {
-  const float2* cs;
-  const int8_t* q8;
-  float step;
-};
-
-template <int TM>
-__device__ __forceinline__ StageTab stage_tab(const uint8_t* tab, int ts, int E) {
-  StageTab r;
-  r.cs = reinterpret_cast<const float2*>(tab) + (size_t)ts * (E >> 1);
-  r.q8 = reinterpret_cast<const int8_t*>(tab + kQ8Head) + (size_t)ts * (E >> 1);
-  r.step = TM == kTmQ8 ? reinterpret_cast<const float*>(tab)[ts] : 0.f;
-  return r;
-}
-
-// (cos, sin) of rotation q of a stage. int8 angles take the fast sine/cosine unit:
-// pi/4 + delta_t q lies within a few tenths of pi/4.
-template <int TM>
-__device__ __forceinline__ float2 coef(const StageTab& st, int q) {
-  if (TM == kTmHad) return make_float2(kRsqrt2, kRsqrt2);
-  if (TM == kTmCS) return st.cs[q];
-  float s, c;
-  __sincosf(fmaf(st.step, (float)st.q8[q], 0.785398163397448309616f), &s, &c);
-  return make_float2(c, s);
-}
-
-__device__ __forceinline__ void rot(float& a, float& b, float2 cs) {
-  const float x = a, y = b;
-  a = fmaf(cs.x, x, cs.y * y);
-  b = fmaf(cs.y, x, -cs.x * y);
-}
-
-// NS stages t .. t+NS-1 (pairs (i, i + 2^s)) on a buffer of E elements, 2^NS values per
-// thread held in registers; table row s (E/2 pairs, pair numbered by first index).
-// TM == kTmHad: every block is the Theta == 0 block [[1, 1], [1, -1]] / sqrt 2 (no table read).
-template <int NS, int TM>
-__device__ __forceinline__ void round_a(float* x, const uint8_t* tab, int t, int E, int ct) {
-  constexpr int P = 1 << NS;
-  const int nthr = E / P, h = 1 << t;
-  if (ct < nthr) {
-    const int base = ((ct >> t) << (t + NS)) | (ct & (h - 1));
-    float v[P];
-#pragma unroll
-    for (int k = 0; k < P; ++k) v[k] = x[base + k * h];
-#pragma unroll
-    for (int s = 0; s < NS; ++s) {
-      const int ts = t + s, hs = 1 << ts;
-      const StageTab st = stage_tab<TM>(tab, ts, E);
-#pragma unroll
-      for (int k = 0; k < P; ++k) {
-        if (k & (1 << s)) continue;
-        const int i = base + k * h;
-        const int q = ((i >> (ts + 1)) << ts) | (i & (hs - 1));
-        rot(v[k], v[k + (1 << s)], coef<TM>(st, q));
-      }
-    }
-#pragma unroll
-    for (int k = 0; k < P; ++k) x[base + k * h] = v[k];
-  }
-  cbar();
-}
-
-// layout-A stages t0 .. t1-1, three per shared-memory round
-template <int TM>
-__device__ __forceinline__ void stages_a(float* x, const uint8_t* tab, int t0, int t1, int E, int ct) {
-  int t = t0;
-  while (t1 - t >= 3) {
-    round_a<3, TM>(x, tab, t, E, ct);
-    t += 3;
-  }
-  if (t1 - t == 2) round_a<2, TM>(x, tab, t, E, ct);
-  if (t1 - t == 1) round_a<1, TM>(x, tab, t, E, ct);
-}
-
-// the three layout-B stages (runs j and j + 2^d, same offset), one round: thread T holds
-// the 8 values {j run + T}; table rows e, e+1, e+2 numbered jj run + T
-template <int TM>
-__device__ __forceinline__ void stages_b(float* x, const uint8_t* tab, int e, int E, int ct) {
-  const int run = E / kC;
-  if (ct < run) {
-    float v[kC];
-#pragma unroll
-    for (int j = 0; j < kC; ++j) v[j] = x[j * run + ct];
-#pragma unroll
-    for (int d = 0; d < 3; ++d) {
-      const StageTab st = stage_tab<TM>(tab, e + d, E);
-#pragma unroll
-      for (int j = 0; j < kC; ++j) {
-        if (j & (1 << d)) continue;
-        const int jj = ((j >> (d + 1)) << d) | (j & ((1 << d) - 1));
-        rot(v[j], v[j + (1 << d)], coef<TM>(st, jj * run + ct));
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < kC; ++j) x[j * run + ct] = v[j];
-  }
-  cbar();
-}
-
-// ------------------------------------------------------------------ cluster data movement
-struct Xchg {
-  uint32_t phase = 0;
-};
-
-// Cluster-wide exchange point among the consumer threads of the 8 CTAs: everything this
-// CTA pushed into its peers before it is visible to them after it.
-__device__ __forceinline__ bool exchange(Smem& s, Xchg& x, int ct, int* status, int where) {
-  cbar();
-  if (ct < kC) arrive_remote(s.xchg, (uint32_t)ct);
-  bool mine = true;
-  if (ct == 0) mine = wait_phase<true>(s.xchg, x.phase, status, where);
-  x.phase ^= 1;
-  return cbar_and(mine);
-}
-
-// layout A (own chunk) -> layout B: run q of my chunk goes to CTA q at offset r*run
-__device__ void push_a_to_b(const float* src, float* dst, int E, uint32_t r, int ct) {
-  const int run = E / kC;
-  for (int v = ct; v < (E >> 2); v += kNT) {
-    const int i = v * 4, q = i / run, ii = i - q * run;
-    st_peer4(dst + r * run + ii, (uint32_t)q, *reinterpret_cast<const float4*>(src + i));
-  }
-}
-
-// layout B -> layout A: my run j goes to CTA j at offset r*run
-__device__ void push_b_to_a(const float* src, float* dst, int E, uint32_t r, int ct) {
-  const int run = E / kC;
-  for (int v = ct; v < (E >> 2); v += kNT) {
-    const int L = v * 4, j = L / run, ii = L - j * run;
-    st_peer4(dst + r * run + ii, (uint32_t)j, *reinterpret_cast<const float4*>(src + L));
-  }
-}
-
-// global element index of local position L in layout B (width kC*E, CTA rank r)
-__device__ __forceinline__ int gidx_b(int L, int E, uint32_t r) {
-  const int run = E / kC, j = L / run, ii = L - j * run;
-  return j * E + (int)r * run + ii;
-}
-
-// int16 GEMV operand of one group of 64 values (one warp); lane 0 writes xs and xsum
-__device__ __forceinline__ void prep_group(const float* v, int bits, int16_t* grp, int16_t* grp_hi, float* xs,
-                                           float* xsum, int lane) {
-  const float v0 = v[2 * lane], v1 = v[2 * lane + 1];
-  float amax = fmaxf(fabsf(v0), fabsf(v1));
-  float sum = v0 + v1;
-  const bool bad = __any_sync(0xffffffffu, !(isfinite(v0) && isfinite(v1)));
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  }
-  int ex = 0;
-  if (amax > 0.f && !bad) ex = group_exponent(amax);
-  const float sc = pow2f(ex);
-  const int q0 = max(-32767, min(32767, __float2int_rn(v0 * sc)));
-  const int q1 = max(-32767, min(32767, __float2int_rn(v1 * sc)));
-  grp[xq_pos_lo(bits, 2 * lane)] = (int16_t)q0;
-  grp[xq_pos_lo(bits, 2 * lane + 1)] = (int16_t)q1;
-  if (bits == 3) {
-    grp_hi[xq_pos_hi(2 * lane)] = (int16_t)q0;
-    grp_hi[xq_pos_hi(2 * lane + 1)] = (int16_t)q1;
-  }
-  if (lane == 0) {
-    *xs = bad ? __int_as_float(0x7fc00000) : pow2f(-ex);
-    *xsum = bad ? __int_as_float(0x7fc00000) : sum;
-  }
-}
-
-// operand of a hidden-wide input held in layout B: prep the CTA's own groups into its
-// local operand buffer and push them into every peer's buffer, then exchange
-__device__ __forceinline__ bool prep_and_broadcast(Smem& s, Xchg& X, const float* xb, int n_in, int bits, int E, uint32_t r, int ct,
-                                   int* status) {
-  const int ng = n_in / 64;
-  int16_t* xq16 = reinterpret_cast<int16_t*>(s.xq);
-  const int words = bits == 3 ? n_in : n_in / 2;
-  float* xsA = reinterpret_cast<float*>(s.xq + words);
-  float* xsumA = xsA + ng;
-  const int warp = ct >> 5, lane = ct & 31, ngl = E >> 6;
-  for (int gl = warp; gl < ngl; gl += kCW) {
-    const int g = gidx_b(gl * 64, E, r) >> 6;
-    prep_group(xb + gl * 64, bits, xq16 + (int64_t)g * 64, xq16 + n_in + (int64_t)g * 64, xsA + g, xsumA + g, lane);
-  }
-  cbar();
-  // 8 float4 per group (16 with the 1-bit-plane order), to the 7 peers
-  const int per = bits == 3 ? 16 : 8;
-  for (int it = ct; it < ngl * per * kC; it += kNT) {
-    const int q = it % kC, rest = it / kC, part = rest % per, gl = rest / per;
-    if (q == (int)r) continue;
-    const int g = gidx_b(gl * 64, E, r) >> 6;
-    const int word = part < 8 ? g * 32 + part * 4 : n_in / 2 + g * 32 + (part - 8) * 4;
-    st_peer4(s.xq + word, (uint32_t)q, *reinterpret_cast<const float4*>(s.xq + word));
-  }
-  for (int it = ct; it < ngl * kC; it += kNT) {
-    const int q = it % kC, gl = it / kC;
-    if (q == (int)r) continue;
-    const int g = gidx_b(gl * 64, E, r) >> 6;
-    st_peer(xsA + g, (uint32_t)q, xsA[g]);
-    st_peer(xsumA + g, (uint32_t)q, xsumA[g]);
-  }
-  return exchange(s, X, ct, status, 40);
-}
-
-// sum of the split-K partials of element i (fixed order)
-__device__ __forceinline__ float zsum(const float* zp, int nk, int n, int i) {
-  float t = __ldcg(zp + i);
-  for (int k = 1; k < nk; ++k) t += __ldcg(zp + (int64_t)k * n + i);
-  return t;
-}
-
-// ------------------------------------------------------------------ chains (cluster-collective)
-// residual chain: [res += F_U(z)] ; n = rms(res) ; x~ = F_V(n) ; operand
-template <int TM>
-__device__ __forceinline__ bool chain_residual(const Params& p, Smem& s, Xchg& X, const Lin* U, const float* zp, int nk,
-                               const Lin* V, bool first, uint32_t r, int ct, const uint8_t* tabU,
-                               const uint8_t* tabV) {
-  const int W = p.hidden, E = p.E, e = p.m_hidden - 3;
-  if (first) {
-    for (int L = ct; L < E; L += kNT) s.res[L] = load_act(p.x_in, gidx_b(L, E, r), p.xt);
-  } else {
-    for (int i = ct; i < E; i += kNT) {
-      const int gi = (int)r * E + i;
-      s.xa[i] = zsum(zp, nk, W, gi) * (float)s.sgn[i];
-    }
-    cbar();
-    stages_a<TM>(s.xa, tabU, 0, e, E, ct);
-    push_a_to_b(s.xa, s.xb, E, r, ct);
-    if (!exchange(s, X, ct, p.status, 41)) return false;
-    stages_b<TM>(s.xb, tabU, e, E, ct);
-    for (int L = ct; L < E; L += kNT) s.res[L] += s.xb[L];
-  }
-  if (!V) {
-    cbar();
-    return true;  // final step: no input butterfly
-  }
-  // sum of squares of this CTA's share (fixed-order tree) pushed to every peer's slot r,
-  // together with the residual values each peer needs for its layout-A chunk
-  float acc = 0.f;
-  for (int L = ct; L < E; L += kNT) acc = fmaf(s.res[L], s.res[L], acc);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-  if ((ct & 31) == 0) s.red[ct >> 5] = acc;
-  cbar();
-  if (ct < kC) {
-    float t = 0.f;
-    for (int w = 0; w < kCW; ++w) t += s.red[w];
-    st_peer(s.ss + r, (uint32_t)ct, t);
-  }
-  push_b_to_a(s.res, s.xa, E, r, ct);
-  if (!exchange(s, X, ct, p.status, 42)) return false;
-  float t = 0.f;
-  for (int q = 0; q < kC; ++q) t += s.ss[q];
-  const float inv = 1.0f / sqrtf(t / (float)W + p.eps);
-  for (int i = ct; i < E; i += kNT) s.xa[i] *= inv * (float)s.sgn[kSgnSlot + i];
-  cbar();
-  stages_a<TM>(s.xa, tabV, 0, e, E, ct);
-  push_a_to_b(s.xa, s.xb, E, r, ct);
-  if (!exchange(s, X, ct, p.status, 43)) return false;
-  stages_b<TM>(s.xb, tabV, e, E, ct);
-  return prep_and_broadcast(s, X, s.xb, V->n_in, p.bits, E, r, ct, p.status);
-}
-
-// attention chain: v = F_U_v(z_v); a = v broadcast per KV group; x~ = F_V_o(a); operand
-template <int TM>
-__device__ __forceinline__ bool chain_attn(const Params& p, Smem& s, Xchg& X, const Lin* Lv, const Lin* Lo, uint32_t r, int ct,
-                           const uint8_t* tabU, const uint8_t* tabV) {
-  const int Wu = Lv->w_out, Eu = Wu / kC, eu = Lv->m_out - 3;
-
-  for (int i = ct; i < Eu; i += kNT) {
-    const int gi = (int)r * Eu + i;
-    s.xa[i] = zsum(p.zpv, p.nk_h, Wu, gi) * (float)s.sgn[i];
-  }
-  cbar();
-  stages_a<TM>(s.xa, tabU, 0, eu, Eu, ct);
-  push_a_to_b(s.xa, s.xb, Eu, r, ct);
-  if (!exchange(s, X, ct, p.status, 44)) return false;
-  stages_b<TM>(s.xb, tabU, eu, Eu, ct);
-  // push every v value to the layout-A owners of the query-head elements that copy it
-  const int Eo = p.E, eo = p.m_hidden - 3, hd = p.head_dim, rep = p.rep;
-  for (int L = ct; L < Eu; L += kNT) {
-    const int gv = gidx_b(L, Eu, r), kvh = gv / hd, d = gv - kvh * hd;
-    for (int h = kvh * rep; h < (kvh + 1) * rep; ++h) {
-      const int ga = h * hd + d;
-      st_peer(s.xa + (ga % Eo), (uint32_t)(ga / Eo), s.xb[L]);
-    }
-  }
-  if (!exchange(s, X, ct, p.status, 45)) return false;
-  for (int i = ct; i < Eo; i += kNT) s.xa[i] *= (float)s.sgn[kSgnSlot + i];
-  cbar();
-  stages_a<TM>(s.xa, tabV, 0, eo, Eo, ct);
-  push_a_to_b(s.xa, s.xb, Eo, r, ct);
-  if (!exchange(s, X, ct, p.status, 46)) return false;
-  stages_b<TM>(s.xb, tabV, eo, Eo, ct);
-  return prep_and_broadcast(s, X, s.xb, Lo->n_in, p.bits, Eo, r, ct, p.status);
-}
-
-// F_U of a q or k GEMV output (cluster-distributed), written to out[gidx]
-template <int TM>
-__device__ __forceinline__ bool chain_out_only(const Params& p, Smem& s, Xchg& X, const Lin* Lq, const float* zp, float* out,
-                               uint32_t r, int ct, const uint8_t* tab) {
-  const int W = Lq->w_out, E = W / kC, e = Lq->m_out - 3;
-
-  for (int i = ct; i < E; i += kNT) {
-    const int gi = (int)r * E + i;
-    s.xa[i] = zsum(zp, p.nk_h, W, gi) * (float)s.sgn[i];
-  }
-  cbar();
-  stages_a<TM>(s.xa, tab, 0, e, E, ct);
-  push_a_to_b(s.xa, s.xb, E, r, ct);
-  if (!exchange(s, X, ct, p.status, 47)) return false;
-  stages_b<TM>(s.xb, tab, e, E, ct);
-  for (int L = ct; L < E; L += kNT) out[gidx_b(L, E, r)] = s.xb[L];
-  cbar();
-  return true;
-}
-
-// one whole MLP block (width <= 512) in one CTA: F_U_gate, F_U_up, silu*up, F_V_down,
-// operand of the down projection for this block (to global)
-template <int TM>
-__device__ __forceinline__ void block_chain(const Params& p, Smem& s, const Lin* Lg, const Lin* Lu, const Lin* Ld, int blk, int ct,
-                            const uint8_t* tab) {
-  const int wb = Lg->w_out, mb = Lg->m_out, F = p.ffn;
-  const int base = blk * wb;
-  for (int i = ct; i < wb; i += kNT) {
-    s.xa[i] = zsum(p.zpg, p.nk_h, F, base + i) * (float)s.sgn[i];
-    s.xb[i] = zsum(p.zpu, p.nk_h, F, base + i) * (float)s.sgn[kSgnSlot + i];
-  }
-  cbar();
-  stages_a<TM>(s.xa, tab, 0, mb, wb, ct);
-  stages_a<TM>(s.xb, tab + table_bytes_local<TM>(wb, mb), 0, mb, wb, ct);
-  for (int i = ct; i < wb; i += kNT) {
-    const float g = s.xa[i];
-    s.xa[i] = g / (1.0f + expf(-g)) * s.xb[i] * (float)s.sgn[2 * kSgnSlot + i];
-  }
-  cbar();
-  stages_a<TM>(s.xa, tab + 2 * table_bytes_local<TM>(wb, mb), 0, mb, wb, ct);
-  const int n_in = Ld->n_in;
-  int16_t* xq16 = reinterpret_cast<int16_t*>(p.xq_down);
-  const int warp = ct >> 5, lane = ct & 31;
-  for (int gl = warp; gl < (wb >> 6); gl += kCW) {
-    const int g = (base >> 6) + gl;
-    prep_group(s.xa + gl * 64, p.bits, xq16 + (int64_t)g * 64, xq16 + n_in + (int64_t)g * 64, p.xs_down + g,
-               p.xsum_down + g, lane);
-  }
-  cbar();
-}
-
 // ------------------------------------------------------------------ GEMV (consumer side)
 // The 16 consumer warps form two halves that take alternate units of the CTA's range,
-// so two units are in flight and each warp covers 8 groups of a unit; the last warp of a
+// so two units are in flight and each warp covers 4 groups of a unit; the last warp of a
 // half to finish a unit reduces its 8 per-warp partial rows and writes the unit's sums.
 constexpr int kHalf = kCW / 2;
 
 template <int BITS>
 __device__ __forceinline__ bool run_units(const Params& p, Smem& s, const Range& g, uint32_t& kring, int ct) {
-  using Gm = Geo<BITS>;
+  using Gm = FGeo<BITS>;
   const int warp = ct >> 5, lane = ct & 31;
   const int hv = warp / kHalf, hw = warp - hv * kHalf;  // half, warp within the half
   const int n_out = g.L->n_out, n_in = g.L->n_in, ngroups = n_in / 64;
@@ -768,7 +880,7 @@ __device__ __forceinline__ bool run_units(const Params& p, Smem& s, const Range&
     const int u = g.u0 + i;
     if (ok) {
       int w = 1;
-      if (lane == 0) w = wait_phase<false>(&s.full[slot], (kr / p.ring_stages) & 1, p.status, 50);
+      if (lane == 0) w = wait_phase<false>(&s.full[slot], (kr / p.ring_stages) & 1, p.status, 52);
       ok = __shfl_sync(0xffffffffu, w, 0) != 0;
     }
     const int tile = u / g.nk, kc = u - tile * g.nk, row0 = tile * 32;
@@ -844,19 +956,78 @@ __device__ __noinline__ bool grid_barrier(const Params& p, int idx, int ct) {
   return cbar_and(mine);
 }
 
+// ------------------------------------------------------------------ chain dispatch
+// the widths come from the stack's shapes at run time; each width has its instantiation
+template <int TM>
+__device__ __forceinline__ bool residual_any(const Params& p, Smem& sm, Xch& x, float (&res)[2], const Lin* U,
+                                             const float* zp, int nk, const Lin* V, uint32_t r, int ct) {
+  return p.eb_h == 10 ? chain_residual<10, TM>(p, sm, x, res, U, zp, nk, V, r, ct)
+                      : chain_residual<9, TM>(p, sm, x, res, U, zp, nk, V, r, ct);
+}
+
+template <int TM, int EB>
+__device__ __forceinline__ bool attn_eb(const Params& p, Smem& sm, Xch& x, const Lin* Lv, const Lin* Lo, uint32_t r,
+                                        int ct) {
+  switch (p.eb_kv) {
+    case 5: return chain_attn<5, EB, TM>(p, sm, x, Lv, Lo, r, ct);
+    case 6: return chain_attn<6, EB, TM>(p, sm, x, Lv, Lo, r, ct);
+    case 7: return chain_attn<7, EB, TM>(p, sm, x, Lv, Lo, r, ct);
+    case 8: return chain_attn<8, EB, TM>(p, sm, x, Lv, Lo, r, ct);
+    case 9: return chain_attn<9, EB, TM>(p, sm, x, Lv, Lo, r, ct);
+    default: return chain_attn<10, EB, TM>(p, sm, x, Lv, Lo, r, ct);
+  }
+}
+
+template <int TM>
+__device__ __forceinline__ bool out_only_any(const Params& p, Smem& sm, Xch& x, int eb, const Lin* Lq,
+                                             const float* zp, float* out, uint32_t r, int ct) {
+  switch (eb) {
+    case 5: return chain_out_only<5, TM>(p, sm, x, Lq, zp, out, r, ct);
+    case 6: return chain_out_only<6, TM>(p, sm, x, Lq, zp, out, r, ct);
+    case 7: return chain_out_only<7, TM>(p, sm, x, Lq, zp, out, r, ct);
+    case 8: return chain_out_only<8, TM>(p, sm, x, Lq, zp, out, r, ct);
+    case 9: return chain_out_only<9, TM>(p, sm, x, Lq, zp, out, r, ct);
+    default: return chain_out_only<10, TM>(p, sm, x, Lq, zp, out, r, ct);
+  }
+}
+
+// MLP blocks of phase P7: eb_blk = log2(block width); <= 9: one CTA per block, else one
+// cluster per block (4096 or 8192 wide: log2 of the per-CTA share = eb_blk - 3)
+template <int TM>
+__device__ __forceinline__ bool mlp_any(const Params& p, Smem& sm, Xch& x, const Lin* lin, int c, uint32_t r,
+                                        int ct) {
+  const int t_cta = c * kC + (int)r;
+  switch (p.eb_blk) {
+    case 6:
+      if (t_cta < p.nblocks) mlp_block_local<6, TM>(p, sm, lin + 4, lin + 5, lin + 6, t_cta, ct);
+      return true;
+    case 7:
+      if (t_cta < p.nblocks) mlp_block_local<7, TM>(p, sm, lin + 4, lin + 5, lin + 6, t_cta, ct);
+      return true;
+    case 8:
+      if (t_cta < p.nblocks) mlp_block_local<8, TM>(p, sm, lin + 4, lin + 5, lin + 6, t_cta, ct);
+      return true;
+    case 9:
+      if (t_cta < p.nblocks) mlp_block_local<9, TM>(p, sm, lin + 4, lin + 5, lin + 6, t_cta, ct);
+      return true;
+    case 12: return c < p.nblocks ? mlp_block_cluster<9, TM>(p, sm, x, lin + 4, lin + 5, lin + 6, c, r, ct) : true;
+    default: return c < p.nblocks ? mlp_block_cluster<10, TM>(p, sm, x, lin + 4, lin + 5, lin + 6, c, r, ct) : true;
+  }
+}
+
+// P7 roles: MLP-block CTAs or clusters first, the last two clusters apply F_U_q / F_U_k
+__device__ __forceinline__ int qk_cluster(const Params& p, int which) { return p.G - 1 - which; }
+
 // ------------------------------------------------------------------ the kernel
 // TM: how every butterfly of the stack keeps its angles (kTmCS, kTmHad, kTmQ8); each form
-// has its own instantiation, so no rotation round branches on it.
+// has its own instantiation, so no rotation branches on it.
 template <int BITS, int TM>
-__global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_constant__ Params p) {
-  using Gm = Geo<BITS>;
-  // the form the consumers read the staged tables in: int8 angles arrive expanded
-  constexpr int TC = TM == kTmQ8 ? kTmCS : TM;
+__global__ void __maxnreg__(120) decode_kernel(const __grid_constant__ Params p) {
+  using Gm = FGeo<BITS>;
   Smem s = carve(p, Gm::kStageBytes);
   const uint32_t r = cta_rank();
   const int c = (int)cluster_id_x();
   const int tid = threadIdx.x;
-  const int t_cta = c * kC + (int)r;
 
   if (tid == 0) {
     s_wait_cycles = p.wait_cycles;
@@ -865,288 +1036,124 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       mbar_init(&s.empty[i], kHalf);  // the 8 warps of the half that consumed the unit
       s.ucnt[i] = 0;
     }
-    mbar_init(s.tab_full, 1);
-    mbar_init(s.tab_empty, 1);
-    mbar_init(s.xchg, kC);
+    mbar_init(&s.xbar[0], 1);
+    mbar_init(&s.xbar[1], 1);
     fence_mbar_init();
   }
-  cluster_sync_all();  // every CTA's barriers exist before any remote arrive
+  cluster_sync_all();  // every CTA's barriers exist before any remote store signals one
 
   const int L = p.L;
-  const int nblocks = p.ffn / p.lin[4].w_out;  // MLP blocks of the gate/up output side
 
   if (tid >= kNT) {
-    // Two producer warps. Every lane of a producer warp runs the same loop (so the warp
-    // never diverges around a blocking wait); lane 0 waits and issues, the others follow.
-    const int pw = (tid - kNT) >> 5, lane = tid & 31;
-    if (pw == 0) {
-      // ---------------- weight ring: every unit of the step, in consumer order. A second
-      // cursor runs p.pf_dist units ahead and asks for those units' boxes to be brought
-      // into L2, so HBM keeps streaming while the activation chains run and the ring's
-      // copies are served from L2.
-      UnitCursor pf;
-      pf.l = 0;
-      pf.ph = 0;
-      pf.g = units<BITS>(p, 0, 0, c, (int)r);
-      pf.u = pf.g.u0;
-      pf.normalize<BITS>(p, c, (int)r);
-      if (lane == 0)
-        for (int d = 0; d < p.pf_dist && pf.l < L; ++d) {
-          prefetch_unit<BITS>(pf.g, pf.u);
-          pf.next<BITS>(p, c, (int)r);
-        }
-      uint32_t k = 0;
-      bool ok = true;
-      for (int l = 0; l < L && ok; ++l)
-        for (int ph = 0; ph < 4 && ok; ++ph) {
-          const Range g = units<BITS>(p, l, ph, c, (int)r);
-          const int ngroups = g.L->n_in / 64;
-          for (int u = g.u0; u < g.u1; ++u) {
-            const int slot = k % p.ring_stages;
-            int go = 1;
-            if (lane == 0 && pf.l < L) {
+    // ---------------- producer warp: the weight ring, every unit of the step in consumer
+    // order. Every lane runs the same loop (the warp never diverges around a blocking
+    // wait); lane 0 waits and issues. A second cursor runs p.pf_dist units ahead and asks
+    // for those units' boxes in L2, so HBM keeps streaming while the chains run and the
+    // ring's copies are served from L2.
+    const int lane = tid & 31;
+    UnitCursor pf;
+    pf.l = 0;
+    pf.ph = 0;
+    pf.g = units<BITS>(p, 0, 0, c, (int)r);
+    pf.u = pf.g.u0;
+    pf.normalize<BITS>(p, c, (int)r);
+    if (lane == 0)
+      for (int d = 0; d < p.pf_dist && pf.l < L; ++d) {
+        prefetch_unit<BITS>(pf.g, pf.u);
+        pf.next<BITS>(p, c, (int)r);
+      }
+    uint32_t k = 0;
+    bool ok = true;
+    for (int l = 0; l < L && ok; ++l)
+      for (int ph = 0; ph < 4 && ok; ++ph) {
+        const Range g = units<BITS>(p, l, ph, c, (int)r);
+        const int ngroups = g.L->n_in / 64;
+        for (int u = g.u0; u < g.u1; ++u) {
+          const int slot = k % p.ring_stages;
+          int go = 1;
+          if (lane == 0) {
+            if (pf.l < L) {
               prefetch_unit<BITS>(pf.g, pf.u);
               pf.next<BITS>(p, c, (int)r);
             }
-            if (lane == 0) {
-              if (k >= (uint32_t)p.ring_stages &&
-                  !wait_phase<false, true>(&s.empty[slot], ((k / p.ring_stages) - 1) & 1, p.status, 51)) {
-                go = 0;
-              } else {
-                const int tile = u / g.nk, kc = u - tile * g.nk;
-                const int g0 = kc * Gm::kChunkGroups, gc = min(Gm::kChunkGroups, ngroups - g0);
-                const int cslabs = (gc + Gm::kGroupsPerSlab - 1) / Gm::kGroupsPerSlab;
-                const int hslabs = BITS == 3 ? (gc + 15) / 16 : 0;
-                uint8_t* st = s.ring + (size_t)slot * Gm::kStageBytes;
-                mbar_arrive_expect_tx(&s.full[slot], (uint32_t)((cslabs + hslabs + (gc + 31) / 32) * kSlab));
-                const int code_x0 = g0 * (BITS == 4 ? 32 : 16) / 8;
-                for (int q = 0; q < cslabs; ++q)
-                  tma_load_2d(st + q * kSlab, &g.L->tm_codes, &s.full[slot], code_x0 + q * 16, tile * 32);
-                if (BITS == 3)
-                  for (int q = 0; q < hslabs; ++q)
-                    tma_load_2d(st + (Gm::kCodeSlabs + q) * kSlab, &g.L->tm_hi, &s.full[slot], g0 + q * 16,
-                                tile * 32);
-                for (int q = 0; q < (gc + 31) / 32; ++q)
-                  tma_load_2d(st + (Gm::kCodeSlabs + Gm::kHiSlabs + q) * kSlab, &g.L->tm_sz, &s.full[slot],
-                              g0 + q * 32, tile * 32);
-              }
+            if (k >= (uint32_t)p.ring_stages &&
+                !wait_phase<false, true>(&s.empty[slot], ((k / p.ring_stages) - 1) & 1, p.status, 53)) {
+              go = 0;
+            } else {
+              const int tile = u / g.nk, kc = u - tile * g.nk;
+              const int g0 = kc * Gm::kChunkGroups, gc = min(Gm::kChunkGroups, ngroups - g0);
+              const int cslabs = (gc + Gm::kGroupsPerSlab - 1) / Gm::kGroupsPerSlab;
+              const int hslabs = BITS == 3 ? (gc + 15) / 16 : 0;
+              uint8_t* st = s.ring + (size_t)slot * Gm::kStageBytes;
+              mbar_arrive_expect_tx(&s.full[slot], (uint32_t)((cslabs + hslabs + (gc + 31) / 32) * kSlab));
+              const int code_x0 = g0 * (BITS == 4 ? 32 : 16) / 8;
+              for (int q = 0; q < cslabs; ++q)
+                tma_load_2d(st + q * kSlab, &g.L->tm_codes, &s.full[slot], code_x0 + q * 16, tile * 32);
+              if (BITS == 3)
+                for (int q = 0; q < hslabs; ++q)
+                  tma_load_2d(st + (Gm::kCodeSlabs + q) * kSlab, &g.L->tm_hi, &s.full[slot], g0 + q * 16, tile * 32);
+              for (int q = 0; q < (gc + 31) / 32; ++q)
+                tma_load_2d(st + (Gm::kCodeSlabs + Gm::kHiSlabs + q) * kSlab, &g.L->tm_sz, &s.full[slot],
+                            g0 + q * 32, tile * 32);
             }
-            ok = __shfl_sync(0xffffffffu, go, 0) != 0;
-            if (!ok) break;
-            ++k;  // k counts the stages issued so far
           }
+          ok = __shfl_sync(0xffffffffu, go, 0) != 0;
+          if (!ok) break;
+          ++k;  // k counts the stages issued so far
         }
-      // drain: wait for the copies still in flight before the CTA may exit
-      if (lane == 0) {
-        const uint32_t nwait = k < (uint32_t)p.ring_stages ? k : (uint32_t)p.ring_stages;
-        for (uint32_t q = k - nwait; q < k; ++q)
-          wait_phase<false, true>(&s.full[q % p.ring_stages], (q / p.ring_stages) & 1, p.status, 52);
       }
-      __syncwarp();
-    } else {
-      // ---------------- tables: one set per chain slot, in consumer order
-      uint32_t slot = 0;
-      bool ok = true;
-      // fp32 tables: the bulk copies' bytes complete the slot. int8 angles: the bytes
-      // announced are the signs'; the warp expands the angles into (cos, sin) pairs, then
-      // lane 0's arrival completes the slot together with those copies.
-      auto announce = [&](uint32_t bytes) {
-        if (TM == kTmQ8) mbar_expect_tx(s.tab_full, bytes);
-        else mbar_arrive_expect_tx(s.tab_full, bytes);
-      };
-      auto finish = [&]() {
-        if (TM == kTmQ8) {
-          __syncwarp();
-          if (lane == 0) mbar_arrive(s.tab_full);
-        }
-      };
-      auto begin = [&]() -> bool {
-        int go = 1;
-        if (lane == 0 && slot > 0 && !wait_phase<false, true>(s.tab_empty, (slot - 1) & 1, p.status, 53)) go = 0;
-        return __shfl_sync(0xffffffffu, go, 0) != 0;
-      };
-      for (int l = 0; l <= L && ok; ++l) {
-        const Lin* lin = p.lin + 7 * l;
-        const Lin* prev = l > 0 ? p.lin + 7 * (l - 1) : nullptr;
-        // P1 (or the final step when l == L)
-        if (!(ok = begin())) break;
-        if (lane == 0) {
-          uint32_t bytes = 0;
-          if (prev) bytes += copied_bytes_cluster<TM>(prev[6].tU, prev[6].w_out, prev[6].m_out);
-          const Lin* V = l < L ? lin + p.asg_qkv[c] : nullptr;
-          if (V) bytes += copied_bytes_cluster<TM>(V->tV, V->w_in, V->m_in);
-          const int Eh = p.E;
-          if (prev) bytes += Eh;
-          if (V) bytes += Eh;
-          announce(bytes);
-          uint32_t off = 0;
-          if (prev)
-            off += load_table_cluster<TM>(s.tab, prev[6].tU, prev[6].n_out, prev[6].w_out, prev[6].m_out, 0, (int)r,
-                                      s.tab_full);
-          if (V) load_table_cluster<TM>(s.tab + off, V->tV, V->n_in, V->w_in, V->m_in, 0, (int)r, s.tab_full);
-          if (prev) bulk_g2s(s.sgn, prev[6].sU + (int64_t)r * Eh, (uint32_t)Eh, s.tab_full);
-          if (V) bulk_g2s(s.sgn + kSgnSlot, V->sV + (int64_t)r * Eh, (uint32_t)Eh, s.tab_full);
-        }
-        if (TM == kTmQ8) {
-          const Lin* V = l < L ? lin + p.asg_qkv[c] : nullptr;
-          uint32_t off = 0;
-          if (prev) {
-            expand_cluster(s.tab, prev[6].tU, prev[6].n_out, prev[6].w_out, prev[6].m_out, (int)r, lane);
-            off = table_bytes_cluster<TM>(prev[6].w_out, prev[6].m_out);
-          }
-          if (V) expand_cluster(s.tab + off, V->tV, V->n_in, V->w_in, V->m_in, (int)r, lane);
-        }
-        finish();
-        ++slot;
-        if (l == L) break;
-        // P3
-        if (!(ok = begin())) break;
-        if (lane == 0) {
-          const uint32_t b0 = table_bytes_cluster<TM>(lin[2].w_out, lin[2].m_out);
-          const int Eu = lin[2].w_out / kC, Eo = lin[3].w_in / kC;
-          announce(copied_bytes_cluster<TM>(lin[2].tU, lin[2].w_out, lin[2].m_out) +
-                   copied_bytes_cluster<TM>(lin[3].tV, lin[3].w_in, lin[3].m_in) + Eu + Eo);
-          load_table_cluster<TM>(s.tab, lin[2].tU, lin[2].n_out, lin[2].w_out, lin[2].m_out, 0, (int)r, s.tab_full);
-          load_table_cluster<TM>(s.tab + b0, lin[3].tV, lin[3].n_in, lin[3].w_in, lin[3].m_in, 0, (int)r, s.tab_full);
-          bulk_g2s(s.sgn, lin[2].sU + (int64_t)r * Eu, (uint32_t)Eu, s.tab_full);
-          bulk_g2s(s.sgn + kSgnSlot, lin[3].sV + (int64_t)r * Eo, (uint32_t)Eo, s.tab_full);
-        }
-        if (TM == kTmQ8) {
-          expand_cluster(s.tab, lin[2].tU, lin[2].n_out, lin[2].w_out, lin[2].m_out, (int)r, lane);
-          expand_cluster(s.tab + table_bytes_cluster<TM>(lin[2].w_out, lin[2].m_out), lin[3].tV, lin[3].n_in,
-                         lin[3].w_in, lin[3].m_in, (int)r, lane);
-        }
-        finish();
-        ++slot;
-        // P5
-        if (!(ok = begin())) break;
-        if (lane == 0) {
-          const Lin* V = lin + 4 + p.asg_gu[c];
-          const uint32_t b0 = table_bytes_cluster<TM>(lin[3].w_out, lin[3].m_out);
-          const int Eh = p.E;
-          announce(copied_bytes_cluster<TM>(lin[3].tU, lin[3].w_out, lin[3].m_out) +
-                   copied_bytes_cluster<TM>(V->tV, V->w_in, V->m_in) + 2 * Eh);
-          load_table_cluster<TM>(s.tab, lin[3].tU, lin[3].n_out, lin[3].w_out, lin[3].m_out, 0, (int)r, s.tab_full);
-          load_table_cluster<TM>(s.tab + b0, V->tV, V->n_in, V->w_in, V->m_in, 0, (int)r, s.tab_full);
-          bulk_g2s(s.sgn, lin[3].sU + (int64_t)r * Eh, (uint32_t)Eh, s.tab_full);
-          bulk_g2s(s.sgn + kSgnSlot, V->sV + (int64_t)r * Eh, (uint32_t)Eh, s.tab_full);
-        }
-        if (TM == kTmQ8) {
-          const Lin* V = lin + 4 + p.asg_gu[c];
-          expand_cluster(s.tab, lin[3].tU, lin[3].n_out, lin[3].w_out, lin[3].m_out, (int)r, lane);
-          expand_cluster(s.tab + table_bytes_cluster<TM>(lin[3].w_out, lin[3].m_out), V->tV, V->n_in, V->w_in,
-                         V->m_in, (int)r, lane);
-        }
-        finish();
-        ++slot;
-        // P7: this CTA's MLP blocks, or F_U_q / F_U_k for the two q/k clusters
-        if (!(ok = begin())) break;
-        if (lane == 0) {
-          uint32_t bytes = 0;
-          const int wb = lin[4].w_out, mb = lin[4].m_out;
-          const int blk = t_cta;  // at most one MLP block per CTA (checked at set-up)
-          if (blk < nblocks)
-            bytes += copied_bytes_local<TM>(lin[4].tU, wb, mb) + copied_bytes_local<TM>(lin[5].tU, wb, mb) +
-                     copied_bytes_local<TM>(lin[6].tV, wb, mb) + 3 * wb;
-          const int qk = c == qk_cluster(p, 0) ? 0 : (c == qk_cluster(p, 1) ? 1 : -1);
-          const int Eq = qk >= 0 ? lin[qk].w_out / kC : 0;
-          if (qk >= 0) bytes += copied_bytes_cluster<TM>(lin[qk].tU, lin[qk].w_out, lin[qk].m_out) + Eq;
-          announce(bytes);
-          if (blk < nblocks) {
-            uint32_t off = 0;
-            off += load_table_local<TM>(s.tab + off, lin[4].tU, lin[4].n_out, wb, mb, blk, s.tab_full);
-            off += load_table_local<TM>(s.tab + off, lin[5].tU, lin[5].n_out, wb, mb, blk, s.tab_full);
-            load_table_local<TM>(s.tab + off, lin[6].tV, lin[6].n_in, wb, mb, blk, s.tab_full);
-            bulk_g2s(s.sgn, lin[4].sU + (int64_t)blk * wb, (uint32_t)wb, s.tab_full);
-            bulk_g2s(s.sgn + kSgnSlot, lin[5].sU + (int64_t)blk * wb, (uint32_t)wb, s.tab_full);
-            bulk_g2s(s.sgn + 2 * kSgnSlot, lin[6].sV + (int64_t)blk * wb, (uint32_t)wb, s.tab_full);
-          }
-          if (qk >= 0) {
-            load_table_cluster<TM>(s.tab, lin[qk].tU, lin[qk].n_out, lin[qk].w_out, lin[qk].m_out, 0, (int)r, s.tab_full);
-            bulk_g2s(s.sgn, lin[qk].sU + (int64_t)r * Eq, (uint32_t)Eq, s.tab_full);
-          }
-        }
-        if (TM == kTmQ8) {
-          const int wb = lin[4].w_out, mb = lin[4].m_out, blk = t_cta;
-          if (blk < nblocks) {
-            const uint32_t tb = table_bytes_local<TM>(wb, mb);
-            expand_local(s.tab, lin[4].tU, lin[4].n_out, wb, mb, blk, lane);
-            expand_local(s.tab + tb, lin[5].tU, lin[5].n_out, wb, mb, blk, lane);
-            expand_local(s.tab + 2 * tb, lin[6].tV, lin[6].n_in, wb, mb, blk, lane);
-          }
-          const int qk = c == qk_cluster(p, 0) ? 0 : (c == qk_cluster(p, 1) ? 1 : -1);
-          if (qk >= 0) expand_cluster(s.tab, lin[qk].tU, lin[qk].n_out, lin[qk].w_out, lin[qk].m_out, (int)r, lane);
-        }
-        finish();
-        ++slot;
-      }
-      if (lane == 0 && slot > 0) wait_phase<false, true>(s.tab_full, (slot - 1) & 1, p.status, 54);
-      __syncwarp();
+    // drain: the copies still in flight must land before the CTA may exit (bounded, and
+    // not cut short by the abort word: these are this CTA's own copies)
+    if (lane == 0) {
+      const uint32_t nwait = k < (uint32_t)p.ring_stages ? k : (uint32_t)p.ring_stages;
+      for (uint32_t q = k - nwait; q < k; ++q)
+        wait_phase<false, true, false>(&s.full[q % p.ring_stages], (q / p.ring_stages) & 1, p.status, 54);
     }
+    __syncwarp();
     cluster_sync_all();
     return;
   }
 
   // ---------------- consumers
   const int ct = tid;
-  uint32_t kring = 0, tslot = 0;
-  Xchg X;
+  uint32_t kring = 0;
+  Xch X;
+  float res[2] = {0.f, 0.f};  // the residual stream, this CTA's layout-B share
   bool ok = true;
-  auto tab_acquire = [&]() -> bool { return wait_uniform<false>(s.tab_full, tslot & 1, p.status, 55, ct); };
-  auto tab_release = [&]() {
-    cbar();
-    if (ct == 0) mbar_arrive(s.tab_empty);
-    ++tslot;
-  };
 
   for (int l = 0; l < L && ok; ++l) {
     const Lin* lin = p.lin + 7 * l;
     const Lin* prev = l > 0 ? p.lin + 7 * (l - 1) : nullptr;
     // P1
-    if (!(ok = tab_acquire())) break;
-    {
-      const uint8_t* tU = s.tab;
-      const uint8_t* tV = prev ? s.tab + table_bytes_cluster<TC>(prev[6].w_out, prev[6].m_out) : s.tab;
-      ok = chain_residual<TC>(p, s, X, prev ? prev + 6 : nullptr, p.zpd, p.nk_f, lin + p.asg_qkv[c], l == 0, r, ct, tU,
-                          tV);
-    }
-    tab_release();
-    if (!ok) break;
+    if (!(ok = residual_any<TM>(p, s, X, res, prev ? prev + 6 : nullptr, p.zpd, p.nk_f, lin + p.asg_qkv[c], r,
+                                ct)))
+      break;
     // P2
     if (!(ok = run_units<BITS>(p, s, units<BITS>(p, l, 0, c, (int)r), kring, ct))) break;
     if (!(ok = grid_barrier(p, l * 5 + 0, ct))) break;
     // P3
-    if (!(ok = tab_acquire())) break;
-    ok = chain_attn<TC>(p, s, X, lin + 2, lin + 3, r, ct, s.tab,
-                    s.tab + table_bytes_cluster<TC>(lin[2].w_out, lin[2].m_out));
-    tab_release();
-    if (!ok) break;
+    if (!(ok = p.eb_h == 10 ? attn_eb<TM, 10>(p, s, X, lin + 2, lin + 3, r, ct)
+                            : attn_eb<TM, 9>(p, s, X, lin + 2, lin + 3, r, ct)))
+      break;
     // P4
     if (!(ok = run_units<BITS>(p, s, units<BITS>(p, l, 1, c, (int)r), kring, ct))) break;
     if (!(ok = grid_barrier(p, l * 5 + 1, ct))) break;
     // P5
-    if (!(ok = tab_acquire())) break;
-    ok = chain_residual<TC>(p, s, X, lin + 3, p.zpo, p.nk_h, lin + 4 + p.asg_gu[c], false, r, ct, s.tab,
-                        s.tab + table_bytes_cluster<TC>(lin[3].w_out, lin[3].m_out));
-    tab_release();
-    if (!ok) break;
+    if (!(ok = residual_any<TM>(p, s, X, res, lin + 3, p.zpo, p.nk_h, lin + 4 + p.asg_gu[c], r, ct))) break;
     // P6
     if (!(ok = run_units<BITS>(p, s, units<BITS>(p, l, 2, c, (int)r), kring, ct))) break;
     if (!(ok = grid_barrier(p, l * 5 + 2, ct))) break;
     // P7
-    if (!(ok = tab_acquire())) break;
+    if (!(ok = mlp_any<TM>(p, s, X, lin, c, r, ct))) break;
     {
-      if (t_cta < nblocks) block_chain<TC>(p, s, lin + 4, lin + 5, lin + 6, t_cta, ct, s.tab);
       const int qk = c == qk_cluster(p, 0) ? 0 : (c == qk_cluster(p, 1) ? 1 : -1);
       if (qk >= 0) {
         float* out = qk == 0 ? p.qout + (int64_t)l * lin[0].n_out : p.kout + (int64_t)l * lin[1].n_out;
         const float* zp = qk == 0 ? p.zpq + (int64_t)l * p.nk_h * lin[0].n_out
                                   : p.zpk + (int64_t)l * p.nk_h * lin[1].n_out;
-        ok = chain_out_only<TC>(p, s, X, lin + qk, zp, out, r, ct, s.tab);
+        if (!(ok = out_only_any<TM>(p, s, X, qk == 0 ? p.eb_h : p.eb_kv, lin + qk, zp, out, r, ct))) break;
       }
     }
-    tab_release();
-    if (!ok) break;
     if (!(ok = grid_barrier(p, l * 5 + 3, ct))) break;
     // P8: the down projection's operand from global
     {
@@ -1166,12 +1173,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     if (!(ok = grid_barrier(p, l * 5 + 4, ct))) break;
   }
   // final: out = h_{L-1} + F_U_down(z_down)
-  if (ok && (ok = tab_acquire())) {
+  if (ok) {
     const Lin* last = p.lin + 7 * (L - 1);
-    ok = chain_residual<TC>(p, s, X, last + 6, p.zpd, p.nk_f, nullptr, false, r, ct, s.tab, s.tab);
-    if (ok && c == 0)
-      for (int L2 = ct; L2 < p.E; L2 += kNT) store_act(p.y_out, gidx_b(L2, p.E, r), p.yt, s.res[L2]);
-    tab_release();
+    ok = residual_any<TM>(p, s, X, res, last + 6, p.zpd, p.nk_f, nullptr, r, ct);
+    if (ok && c == 0) {
+      const int E = p.hidden / kC;
+      for (int sl = 0; sl < 2; ++sl) {
+        if (sl * kNT >= E || ct >= (E < kNT ? E : kNT)) continue;
+        const int run = E / kC;
+        const int g = (ct & 7) * E + (int)r * run + (((ct & 31) >> 3) | ((ct >> 5) << 2) | (sl << 6));
+        store_act(p.y_out, g, p.yt, res[sl]);
+      }
+    }
   }
   cluster_sync_all();
 }
@@ -1179,9 +1192,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 // ------------------------------------------------------------------ host side
 template <int BITS>
 size_t smem_bytes(const Params& p) {
-  return 1024 + (size_t)p.ring_stages * Geo<BITS>::kStageBytes + p.tab_bytes + 4 * kSgnSlot + 12 * (size_t)p.E + 64 +
+  return 1024 + (size_t)p.ring_stages * FGeo<BITS>::kStageBytes + 3 * 4 * (size_t)kRxFloats + 4 * 32 +
          (size_t)4 * kCW * 32 * p.ring_stages + 4 * ((p.ring_stages + 3) & ~3) + p.xq_bytes +
-         8 * (2 * (size_t)p.ring_stages + 3);
+         8 * (2 * (size_t)p.ring_stages + 2);
 }
 
 template <int BITS>
@@ -1191,6 +1204,9 @@ const void* kernel_ptr(int tm) {
                        : reinterpret_cast<const void*>(decode_kernel<BITS, kTmCS>);
 }
 
+// The grid barriers need every CTA resident at once. The launch asks for that explicitly
+// (cooperative), so a grid that cannot be co-resident -- because other work holds SMs --
+// is refused at launch instead of timing out in its first barrier.
 template <int BITS>
 cudaError_t launch_bits(const Params& p, cudaStream_t st) {
   const size_t smem = smem_bytes<BITS>(p);
@@ -1202,16 +1218,39 @@ cudaError_t launch_bits(const Params& p, cudaStream_t st) {
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = kC;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeCooperative;
+  attr[1].val.cooperative = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (p.tm == kTmHad) return cudaLaunchKernelEx(&cfg, decode_kernel<BITS, kTmHad>, p);
-  if (p.tm == kTmQ8) return cudaLaunchKernelEx(&cfg, decode_kernel<BITS, kTmQ8>, p);
-  return cudaLaunchKernelEx(&cfg, decode_kernel<BITS, kTmCS>, p);
+  // A driver that does not take the cooperative attribute together with cluster dimensions
+  // gets the plain cluster launch (co-residency then rests on the occupancy query made at
+  // set-up); a grid too large to be co-resident is refused either way.
+  static int coop_ok[64] = {0};  // 0 unknown, 1 accepted, -1 not accepted (per device)
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+  const bool coop = p.cooperative && coop_ok[dev] >= 0;
+  cfg.numAttrs = coop ? 2 : 1;
+  auto go = [&]() -> cudaError_t {
+    if (p.tm == kTmHad) return cudaLaunchKernelEx(&cfg, decode_kernel<BITS, kTmHad>, p);
+    if (p.tm == kTmQ8) return cudaLaunchKernelEx(&cfg, decode_kernel<BITS, kTmQ8>, p);
+    return cudaLaunchKernelEx(&cfg, decode_kernel<BITS, kTmCS>, p);
+  };
+  e = go();
+  if (coop && coop_ok[dev] == 0) {
+    if (e == cudaSuccess) {
+      coop_ok[dev] = 1;
+    } else if (e != cudaErrorCooperativeLaunchTooLarge) {
+      cudaGetLastError();
+      coop_ok[dev] = -1;
+      cfg.numAttrs = 1;
+      e = go();
+    }
+  }
+  return e;
 }
 
 cudaError_t launch(const Params& p, cudaStream_t st) {
@@ -1232,7 +1271,7 @@ size_t smem_for(const Params& p) {
 }
 
 int chunk_cols_for(int bits) {
-  return bits == 2 ? Geo<2>::kChunkCols : (bits == 3 ? Geo<3>::kChunkCols : Geo<4>::kChunkCols);
+  return bits == 2 ? FGeo<2>::kChunkCols : (bits == 3 ? FGeo<3>::kChunkCols : FGeo<4>::kChunkCols);
 }
 
 cudaError_t max_clusters(const Params& p, int* out) {

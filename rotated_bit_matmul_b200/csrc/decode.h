@@ -11,7 +11,7 @@ namespace dec {
 constexpr int kC = 8;                // CTAs per cluster
 constexpr int kCW = 16;              // consumer warps per CTA
 constexpr int kNT = 32 * kCW;        // consumer threads
-constexpr int kThreads = kNT + 64;   // + a weight-ring producer warp and a table producer warp
+constexpr int kThreads = kNT + 32;   // + the weight-ring producer warp
 constexpr int kMaxClusters = 64;
 
 // How the butterflies of a fused stack keep their angles (one kernel instantiation each):
@@ -34,8 +34,9 @@ struct Params {
   int L, hidden, ffn, n_heads, n_kv, head_dim, rep, bits;
   float eps;
   int G;           // clusters in the grid
-  int E;           // hidden / kC
-  int m_hidden;    // log2(hidden)
+  // log2 of the per-CTA share of a hidden-wide (eb_h) and a kv-wide (eb_kv) butterfly,
+  // log2 of the MLP block width (eb_blk; <= 9: one CTA per block, else one cluster)
+  int eb_h, eb_kv, eb_blk, nblocks;
   const void* x_in;
   int xt;
   void* y_out;
@@ -52,8 +53,9 @@ struct Params {
   long long wait_cycles;  // bound of every wait, in SM clock cycles
   int barrier_extra;      // testing hook: grid barrier whose target is raised by one (-1: none)
   int tm;   // kTmCS, kTmHad or kTmQ8: how every butterfly of the stack keeps its angles
-  int ring_stages, tab_bytes, xq_bytes;
-  int pf_dist;  // units the L2 prefetch runs ahead of the ring (0: none)
+  int ring_stages, xq_bytes;
+  int pf_dist;      // units the L2 prefetch runs ahead of the ring (0: none)
+  int cooperative;  // launch with the cooperative attribute (all CTAs co-resident or refused)
   int asg_qkv[kMaxClusters], idx_qkv[kMaxClusters], cnt_qkv[3];
   int asg_gu[kMaxClusters], idx_gu[kMaxClusters], cnt_gu[2];
 };

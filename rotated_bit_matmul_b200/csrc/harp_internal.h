@@ -8,6 +8,8 @@
 
 #include "harp.h"
 
+struct harp_mr_plan_s;
+
 namespace harp {
 
 enum { DT_F32 = 0, DT_BF16 = 1, DT_F16 = 2 };
@@ -77,6 +79,9 @@ struct GemvParams {
 struct Layer {
   int64_t n_in, n_out;
   int bits, group, w_in, w_out, m_in, m_out;
+  // mixed-radix sides (harp_create_layer_mr): borrowed plans, or null for radix-2 sides
+  const harp_mr_plan_s* mrV;
+  const harp_mr_plan_s* mrU;
   float2* csV;   // [m_in][n_in/2]
   float2* csU;   // [m_out][n_out/2]
   uint8_t* q8V;  // int8 angle storage of the input side (kQ8Head + m_in * n_in/2 bytes), or null
@@ -98,6 +103,8 @@ struct Layer {
 // Workspace carve-up for a linear forward with `batch` rows. Below kMinBatchMma rows
 // (GEMV): xq, xs, xsum, z. From kMinBatchMma rows (tensor cores): xf, x16, rowscale, zpart.
 struct LinearWs {
+  float* xmr;         // mixed-radix layers: [batch][n_in] transformed input (GEMV path)
+  float* zmr;         // mixed-radix layers: [batch][n_out] sum of the split partials (tensor-core path)
   int32_t* xq;
   float* xs;
   float* xsum;
@@ -115,6 +122,16 @@ LinearWs linear_ws_layout(const Layer& L, int batch, void* base);
 int xq_words_per_row(int64_t n_in, int bits);
 
 cudaError_t launch_butterfly(const BflyParams& p, int batch, cudaStream_t st);
+// mixed-radix transform of `batch` contiguous rows (plan forward, or its transpose)
+cudaError_t launch_mr(const harp_mr_plan_s* plan, int inverse, int batch, const void* x, int xt, void* y, int yt,
+                      cudaStream_t st);
+int64_t mr_plan_d(const harp_mr_plan_s* plan);
+int mr_plan_device(const harp_mr_plan_s* plan);
+// int16 GEMV operand of `batch` fp32 rows of n (groups of 64): xq words, xs, xsum
+cudaError_t launch_operand_prep(const float* x, int64_t n, int bits, int batch, int32_t* xq, int64_t xq_stride,
+                                float* xs, float* xsum, int64_t g_stride, cudaStream_t st);
+// z[i] = sum over s of part[s][i], s in fixed order (count elements per split)
+cudaError_t launch_sum_splits(const float* part, int splits, int64_t count, float* z, cudaStream_t st);
 cudaError_t launch_gemv(const Layer& L, const GemvParams& p, cudaStream_t st);
 cudaError_t launch_quantize(int64_t n_out, int64_t n_in, int bits, const float* W, void* codes,
                             void* scale_zero, cudaStream_t st);

@@ -299,6 +299,33 @@ harp_status harp_mr_plan_destroy(harp_mr_plan plan) {
   return HARP_OK;
 }
 
+}  // extern "C"
+
+namespace harp {
+
+cudaError_t launch_mr(const harp_mr_plan_s* plan, int inverse, int batch, const void* x, int xt, void* y, int yt,
+                      cudaStream_t st) {
+  if (batch <= 0) return cudaSuccess;
+  MrParams p = plan->p;
+  p.inverse = inverse;
+  p.x = x;
+  p.xt = xt;
+  p.y = y;
+  p.yt = yt;
+  const size_t smem = sizeof(float) * 2 * (size_t)p.d;
+  cudaError_t e = cudaFuncSetAttribute(mr_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  mr_kernel<<<(unsigned)batch, kMrThreads, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+int64_t mr_plan_d(const harp_mr_plan_s* plan) { return plan->p.d; }
+int mr_plan_device(const harp_mr_plan_s* plan) { return plan->device; }
+
+}  // namespace harp
+
+extern "C" {
+
 static harp_status mr_apply(harp_mr_plan plan, int batch, const void* x, harp_dtype xt, void* y, harp_dtype yt,
                             void* stream, int inverse) {
   if (!plan || !x || !y) return set_error(HARP_ERR_INVALID_ARG, "mr_butterfly: null pointer");
@@ -309,18 +336,7 @@ static harp_status mr_apply(harp_mr_plan plan, int batch, const void* x, harp_dt
     return set_error(HARP_ERR_INVALID_ARG, "mr_butterfly: device pointers must be 16-byte aligned");
   if (x == y && xt != yt) return set_error(HARP_ERR_INVALID_ARG, "mr_butterfly: in-place needs equal dtypes");
   if (batch == 0) return HARP_OK;
-  MrParams p = plan->p;
-  p.inverse = inverse;
-  p.x = x;
-  p.xt = xt;
-  p.y = y;
-  p.yt = yt;
-  const size_t smem = sizeof(float) * 2 * (size_t)p.d;
-  cudaError_t e = cudaFuncSetAttribute(mr_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e == cudaSuccess) {
-    mr_kernel<<<(unsigned)batch, kMrThreads, smem, static_cast<cudaStream_t>(stream)>>>(p);
-    e = cudaGetLastError();
-  }
+  const cudaError_t e = launch_mr(plan, inverse, batch, x, xt, y, yt, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return set_error(HARP_ERR_CUDA, "mr_butterfly launch: %s", cudaGetErrorString(e));
   return HARP_OK;
 }

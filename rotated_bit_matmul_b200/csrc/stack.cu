@@ -218,7 +218,9 @@ void setup_fused(harp_stack_s* S) {
   if (dq != H) return no("n_heads * head_dim must equal hidden");
   if (dkv < 256 || dkv > H || (dkv & (dkv - 1))) return no("n_kv_heads * head_dim must be a power of two in [256, hidden]");
   const int wb = S->layers[4]->L.w_out;
-  if (wb < 64 || wb > 512) return no("gate/up output blocks must be 64..512 wide");
+  // MLP blocks: up to 512 wide one CTA each, 4096 or 8192 wide one cluster each
+  if (!((wb >= 64 && wb <= 512) || wb == 4096 || wb == 8192))
+    return no("gate/up output blocks must be 64..512, 4096 or 8192 wide");
   for (int l = 0; l < S->n_layers; ++l) {
     const Layer* L[7];
     for (int i = 0; i < 7; ++i) L[i] = &S->layers[7 * l + i]->L;
@@ -233,7 +235,7 @@ void setup_fused(harp_stack_s* S) {
     if (L[6]->w_out != H) return no("down output butterfly must be hidden-wide");
   }
   // every butterfly in one form: fp32 angles (cos/sin tables), int8 angles, or Theta == 0.
-  // One kernel instantiation per form, so none pays for another in its rotation rounds.
+  // One kernel instantiation per form, so none pays for another in its rotations.
   int n_cs = 0, n_q8 = 0, n_had = 0;
   for (const harp_layer l : S->layers) {
     const Layer& L = l->L;
@@ -264,37 +266,32 @@ void setup_fused(harp_stack_s* S) {
   p.rep = S->n_heads / S->n_kv_heads;
   p.bits = bits;
   p.eps = S->eps;
-  p.E = H / dec::kC;
-  p.m_hidden = ilog2(H);
-  // shared-memory budget: tables of the largest chain, operand of the widest input
-  // tables are staged as (cos, sin) pairs whatever the layer keeps (int8 angles are expanded)
-  const int esz = 8, head = 0;
-  auto tb = [&](int w) { return head + esz * ilog2(w) * (w / dec::kC / 2); };
-  int tab = 2 * tb(H);
-  tab = std::max(tab, tb(dkv) + tb(H));
-  tab = std::max(tab, tb(dq));
-  const int wbm = ilog2(wb);
-  tab = std::max(tab, 3 * (head + esz * wbm * (wb / 2)));
-  p.tab_bytes = (tab + 15) & ~15;  // the sign slices after it take 16-byte bulk copies
+  p.eb_h = ilog2(H / dec::kC);
+  p.eb_kv = ilog2(dkv / dec::kC);
+  p.eb_blk = ilog2(wb);
+  p.nblocks = F / wb;
+  // shared memory: the operand of the widest input, then as many ring stages as fit
+  // (each also carries its reduction scratch and barriers)
   auto xqb = [&](int n) { return 4 * ((bits == 3 ? n : n / 2) + 2 * (n / 64)); };
   p.xq_bytes = (std::max(xqb(H), xqb(F)) + 15) & ~15;  // keeps the mbarriers after it 8-byte aligned
   int optin = 0;
   cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, S->device);
-  // as many ring stages as fit (each also carries its reduction scratch and barriers)
   p.ring_stages = 16;
   while (p.ring_stages >= 2 && dec::smem_for(p) > (size_t)optin) --p.ring_stages;
   if (p.ring_stages < 2) return no("not enough shared memory for the weight ring");
-  // L2 prefetch distance: HARP_PF_DIST overrides (a tuning knob), else 16 units
-  p.pf_dist = 16;
+  // L2 prefetch distance in units (tuning knob HARP_PF_DIST); cooperative launch unless
+  // HARP_COOPERATIVE=0
+  p.pf_dist = 24;
   if (const char* e = getenv("HARP_PF_DIST")) p.pf_dist = std::max(0, atoi(e));
+  p.cooperative = 1;
+  if (const char* e = getenv("HARP_COOPERATIVE")) p.cooperative = atoi(e) != 0;
   int G = 0;
   cudaError_t e = dec::max_clusters(p, &G);
   if (e != cudaSuccess || G < 1) return no(std::string("cluster occupancy query failed: ") + cudaGetErrorString(e));
   if (G > dec::kMaxClusters) G = dec::kMaxClusters;
-  const int nblocks = F / wb;
-  // P7: block CTAs come first, the last two clusters apply F_U_q / F_U_k
-  while (G > 3 && nblocks > (G - 2) * dec::kC) --G;
-  if (G < 3 || nblocks > (G - 2) * dec::kC) return no("too few co-resident clusters");
+  // P7: MLP-block CTAs (or clusters) come first, the last two clusters apply F_U_q / F_U_k
+  const int cap = wb <= 512 ? dec::kC : 1;
+  if (G < 3 || p.nblocks > (G - 2) * cap) return no("too few co-resident clusters");
   p.G = G;
   const int rq[3] = {dq, dkv, dkv}, rg[2] = {F, F};
   assign(G, rq, 3, p.asg_qkv, p.idx_qkv, p.cnt_qkv);
