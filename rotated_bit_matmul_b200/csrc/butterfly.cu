@@ -21,6 +21,7 @@
 // pi/4 + delta_t q are evaluated as each rotation needs them.
 // The forward epilogue can also emit the GEMV operand: per group of 64 outputs an
 // int16 copy in dp2a pair order, the power-of-two scale and the fp32 group sum.
+#include "bfly_engine.cuh"
 #include "common.cuh"
 
 namespace harp {
@@ -28,6 +29,8 @@ namespace harp {
 namespace {
 
 constexpr int kBflyThreads = 256;
+// the engine-based forward path (fast_bfly_kernel) serves the forward calls it covers
+constexpr bool kDisableFastButterfly = false;
 constexpr float kRsqrt2 = 0.70710678118654752440f;  // cos(pi/4) = sin(pi/4)
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -307,10 +310,150 @@ __global__ void __launch_bounds__(kBflyThreads) bfly_kernel(BflyParams p, int C)
 
 int cluster_for(int w) { return w >= 4096 ? 8 : (w == 2048 ? 4 : (w == 1024 ? 2 : 1)); }
 
+// ------------------------------------------------------------------ fast forward path
+// The forward transform with the layer's tables (or Theta == 0) on the butterfly engines:
+// one CTA per (row, block) up to 512 wide, one cluster of 8 per (row, block) from 1024 to
+// 8192. 512 threads, one element each (two at 8192); coefficients straight from the tables.
+template <int EB, int TM, bool CLUSTER>
+__global__ void __launch_bounds__(dec::kNT) fast_bfly_kernel(BflyParams p) {
+  using namespace dec;
+  __shared__ __align__(16) float sm_T[kRxFloats];
+  __shared__ __align__(16) float sm_rx[2][CLUSTER ? kRxFloats : 1];
+  __shared__ uint64_t sm_bar[2];
+  EngCtx ctx;
+  ctx.T = sm_T;
+  ctx.rx[0] = sm_rx[0];
+  ctx.rx[1] = sm_rx[1];
+  ctx.xbar = sm_bar;
+  const int ct = threadIdx.x, warp = ct >> 5, lane = ct & 31;
+  const int64_t row = blockIdx.y;
+  if (ct == 0) {
+    s_wait_cycles = p.wait_cycles > 0 ? p.wait_cycles : 4000000000ll;
+    mbar_init(&sm_bar[0], 1);
+    mbar_init(&sm_bar[1], 1);
+    fence_mbar_init();
+  }
+  if (CLUSTER) cluster_sync_all();
+  else __syncthreads();
+  const uint8_t* tab = TM == kTmCS ? reinterpret_cast<const uint8_t*>(p.cs) : (TM == kTmQ8 ? p.q8 : nullptr);
+  using M = Map<CLUSTER ? EB : EB>;
+  const int64_t w = CLUSTER ? (int64_t)kC * M::E : (int64_t)M::E;
+  const int64_t blk = CLUSTER ? blockIdx.x / kC : blockIdx.x;
+  auto in = [&](int64_t g) {
+    float v = load_act(p.x, row * p.x_stride + g, p.xt);
+    for (int k = 1; k < p.nsum; ++k) v += load_act(p.x, k * p.sum_stride + row * p.x_stride + g, p.xt);
+    return v * (float)__ldg(p.sign + g);
+  };
+  int16_t* xq16 = p.xq ? reinterpret_cast<int16_t*>(p.xq + row * p.xq_stride) : nullptr;
+  if constexpr (CLUSTER) {
+    using BF = ClusterBfly<EB, TM>;
+    const uint32_t r = cta_rank();
+    BF bf;
+    bf.fetch(tab, p.n >> 1, blk, r, ct);
+    float v[2] = {0.f, 0.f};
+    if (ct < M::NT)
+#pragma unroll
+      for (int s = 0; s < M::P; ++s) v[s] = in(blk * w + BF::ga(r, ct, s));
+    Xch x;
+    const bool ok = bf.run(v, ctx, x, r, ct, p.status, 20);
+    if (ok && p.y && ct < M::NT)
+#pragma unroll
+      for (int s = 0; s < M::P; ++s) store_act(p.y, row * p.y_stride + blk * w + BF::gb(r, ct, s), p.yt, v[s]);
+    if constexpr (M::RUN >= 64) {
+      if (ok && xq16) {  // groups of 64 lie inside the layout-B runs
+        constexpr int GPR = M::RUN / 64, NGL = M::E / 64;
+        if (ct < M::NT)
+#pragma unroll
+          for (int s = 0; s < M::P; ++s) sm_T[M::idx_b(M::bj(ct), M::bii(ct, s))] = v[s];
+        cbar();
+        if (warp < NGL) {
+          const int j = warp / GPR, kk = warp - j * GPR;
+          const int64_t G = (blk * w + j * M::E + (int)r * M::RUN + 64 * kk) >> 6;
+          prep_group(sm_T + j * M::PAD + 64 * kk, p.bits, xq16 + G * 64, xq16 + p.n + G * 64,
+                     p.xs + row * p.g_stride + G, p.xsum + row * p.g_stride + G, lane);
+        }
+      }
+    }
+    cluster_sync_all();  // no CTA leaves while a peer may still store into it
+  } else {
+    LocalBfly<EB, TM> lb;
+    lb.fetch(tab, p.n >> 1, blk, ct);
+    float v = ct < M::NT ? in(blk * w + M::e1(ct, 0)) : 0.f;
+    lb.run(v, ctx, ct);
+    if (ct < M::NT) {
+      if (p.y) store_act(p.y, row * p.y_stride + blk * w + M::e2(ct, 0), p.yt, v);
+      if (xq16) sm_T[M::e2(ct, 0)] = v;  // natural order for the groups
+    }
+    if (xq16) {
+      cbar();
+      if (warp < (M::E >> 6)) {
+        const int64_t G = ((blk * w) >> 6) + warp;
+        prep_group(sm_T + 64 * warp, p.bits, xq16 + G * 64, xq16 + p.n + G * 64, p.xs + row * p.g_stride + G,
+                   p.xsum + row * p.g_stride + G, lane);
+      }
+    }
+  }
+}
+
+template <int TM, bool CLUSTER>
+const void* fast_kernel_for(int eb) {
+  if (CLUSTER) {
+    switch (eb) {
+      case 7: return reinterpret_cast<const void*>(fast_bfly_kernel<7, TM, true>);
+      case 8: return reinterpret_cast<const void*>(fast_bfly_kernel<8, TM, true>);
+      case 9: return reinterpret_cast<const void*>(fast_bfly_kernel<9, TM, true>);
+      case 10: return reinterpret_cast<const void*>(fast_bfly_kernel<10, TM, true>);
+    }
+  } else {
+    switch (eb) {
+      case 6: return reinterpret_cast<const void*>(fast_bfly_kernel<6, TM, false>);
+      case 7: return reinterpret_cast<const void*>(fast_bfly_kernel<7, TM, false>);
+      case 8: return reinterpret_cast<const void*>(fast_bfly_kernel<8, TM, false>);
+      case 9: return reinterpret_cast<const void*>(fast_bfly_kernel<9, TM, false>);
+    }
+  }
+  return nullptr;
+}
+
+// true (and *e set) when the fast path took the call
+bool launch_fast(const BflyParams& p, int batch, cudaStream_t st, cudaError_t* e) {
+  if (p.inverse || (!p.cs && !p.q8 && p.theta)) return false;  // transposes and raw angles: the general kernel
+  const int w = p.w;
+  const bool local = w >= 64 && w <= 512, cluster = w >= 1024 && w <= 8192;
+  if (!local && !cluster) return false;
+  if (cluster && p.xq && w < 4096) return false;  // operand groups would straddle CTAs
+  int eb = 0;
+  while ((1 << eb) < (cluster ? w / dec::kC : w)) ++eb;
+  const int tm = p.q8 ? dec::kTmQ8 : (p.cs ? dec::kTmCS : dec::kTmHad);
+  const void* fn = nullptr;
+  if (tm == dec::kTmCS) fn = cluster ? fast_kernel_for<dec::kTmCS, true>(eb) : fast_kernel_for<dec::kTmCS, false>(eb);
+  else if (tm == dec::kTmQ8) fn = cluster ? fast_kernel_for<dec::kTmQ8, true>(eb) : fast_kernel_for<dec::kTmQ8, false>(eb);
+  else fn = cluster ? fast_kernel_for<dec::kTmHad, true>(eb) : fast_kernel_for<dec::kTmHad, false>(eb);
+  if (!fn) return false;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((p.n / w) * (cluster ? dec::kC : 1)), (unsigned)batch, 1);
+  cfg.blockDim = dim3(dec::kNT, 1, 1);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cluster ? dec::kC : 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  void* args[] = {const_cast<BflyParams*>(&p)};
+  *e = cudaLaunchKernelExC(&cfg, fn, args);
+  return true;
+}
+
 }  // namespace
 
 cudaError_t launch_butterfly(const BflyParams& p, int batch, cudaStream_t st) {
   if (batch <= 0) return cudaSuccess;
+  if (!kDisableFastButterfly) {
+    cudaError_t e = cudaSuccess;
+    if (launch_fast(p, batch, st, &e)) return e;
+  }
   const int C = cluster_for(p.w);
   const int E = p.w / C;
   const int tm = p.q8 ? kTabQ8 : (p.cs ? kTabCS : kTabTheta);

@@ -46,6 +46,7 @@ struct BflyParams {
   int nsum;            // forward input: sum of nsum fp32 partial arrays sum_stride apart (<= 1: one)
   int64_t sum_stride;
   int* status;
+  long long wait_cycles;  // bound of the fast kernel's exchange waits (SM cycles; 0: the default)
 };
 
 // Testing hooks (harp_test_set_faults): off by default. wait_ns bounds every mbarrier
