@@ -327,21 +327,36 @@ __global__ void __launch_bounds__(kThreads, 1) mma_kernel(const __grid_constant_
 }
 
 // ------------------------------------------------------------------ fp16 operand prep
-// One CTA per token row: max |v| -> scale 2^e with max |v| 2^e in [256, 512) (so the group
-// sums stay below 2^15), then the scaled values in pair order and the group sums.
+// One CTA of 1024 threads per token row: max |v| -> scale 2^e with max |v| 2^e in
+// [256, 512) (so the group sums stay below 2^15), then the scaled values in pair order and
+// the group sums. Each warp owns whole groups of 64 and keeps them in registers between
+// the two passes (16 groups per warp, 32768 inputs; wider rows re-read the rest).
+constexpr int kPrepThreads = 1024;
+constexpr int kPrepGroupsPerWarp = 16;
+
 template <int BITS>
-__global__ void __launch_bounds__(256) x16_prep_kernel(const float* __restrict__ xt, int n_in, int64_t ld,
-                                                       __half* __restrict__ x16, float* __restrict__ rowscale) {
-  __shared__ float red[8];
+__global__ void __launch_bounds__(kPrepThreads) x16_prep_kernel(const float* __restrict__ xt, int n_in, int64_t ld,
+                                                                __half* __restrict__ x16, float* __restrict__ rowscale) {
+  __shared__ float red[kPrepThreads / 32];
   __shared__ int bad_s;
   const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int NW = kPrepThreads / 32;
   const float* x = xt + (int64_t)b * n_in;
+  const int G = n_in / 64;
+  float2 v[kPrepGroupsPerWarp];
   float amax = 0.f;
   int bad = 0;
-  for (int j = tid; j < n_in; j += 256) {
-    const float v = x[j];
-    bad |= !isfinite(v);
-    amax = fmaxf(amax, fabsf(v));
+#pragma unroll
+  for (int i = 0; i < kPrepGroupsPerWarp; ++i) {
+    const int g = warp + i * NW;
+    v[i] = g < G ? *reinterpret_cast<const float2*>(x + g * 64 + 2 * lane) : make_float2(0.f, 0.f);
+    bad |= !(isfinite(v[i].x) && isfinite(v[i].y));
+    amax = fmaxf(amax, fmaxf(fabsf(v[i].x), fabsf(v[i].y)));
+  }
+  for (int g = warp + kPrepGroupsPerWarp * NW; g < G; g += NW) {  // rows wider than the cache
+    const float2 t = *reinterpret_cast<const float2*>(x + g * 64 + 2 * lane);
+    bad |= !(isfinite(t.x) && isfinite(t.y));
+    amax = fmaxf(amax, fmaxf(fabsf(t.x), fabsf(t.y)));
   }
   bad = __any_sync(0xffffffffu, bad);
 #pragma unroll
@@ -354,7 +369,7 @@ __global__ void __launch_bounds__(256) x16_prep_kernel(const float* __restrict__
   }
   __syncthreads();
   amax = red[0];
-  for (int i = 1; i < 8; ++i) amax = fmaxf(amax, red[i]);
+  for (int i = 1; i < NW; ++i) amax = fmaxf(amax, red[i]);
   int e = 0;
   if (amax > 0.f) {
     const int field = (int)((__float_as_uint(amax) >> 23) & 0xffu);
@@ -363,10 +378,18 @@ __global__ void __launch_bounds__(256) x16_prep_kernel(const float* __restrict__
   }
   const float sc = pow2f(e);
   __half* out = x16 + (int64_t)b * ld;
-  const int G = n_in / 64;
-  for (int g = warp; g < G; g += 8) {
-    const int j0 = g * 64 + 2 * lane;
-    const float v0 = x[j0] * sc, v1 = x[j0 + 1] * sc;
+  for (int i = 0;; ++i) {
+    const int g = warp + i * NW;
+    if (g >= G) break;
+    float2 t;
+    if (i < kPrepGroupsPerWarp) {
+#pragma unroll
+      for (int k = 0; k < kPrepGroupsPerWarp; ++k)
+        if (k == i) t = v[k];
+    } else {
+      t = *reinterpret_cast<const float2*>(x + g * 64 + 2 * lane);
+    }
+    const float v0 = t.x * sc, v1 = t.y * sc;
     float s = v0 + v1;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
@@ -377,17 +400,17 @@ __global__ void __launch_bounds__(256) x16_prep_kernel(const float* __restrict__
       const int j = jj[k];
       int pos;
       if (BITS == 4) {
-        const int c = j >> 3, i = j & 7;
-        pos = 8 * c + (i < 4 ? 2 * i : 2 * (i - 4) + 1);
+        const int c = j >> 3, q = j & 7;
+        pos = 8 * c + (q < 4 ? 2 * q : 2 * (q - 4) + 1);
       } else {
-        const int c = j >> 4, i = j & 15;
-        pos = 16 * c + (i < 8 ? 2 * i : 2 * (i - 8) + 1);
+        const int c = j >> 4, q = j & 15;
+        pos = 16 * c + (q < 8 ? 2 * q : 2 * (q - 8) + 1);
       }
       out[g * 64 + pos] = __float2half_rn(vv[k]);
     }
     if (lane == 0) out[n_in + g] = __float2half_rn(s);
   }
-  for (int64_t j = n_in + G + tid; j < ld; j += 256) out[j] = __float2half_rn(0.f);
+  for (int64_t j = n_in + G + tid; j < ld; j += kPrepThreads) out[j] = __float2half_rn(0.f);
   if (tid == 0) rowscale[b] = bad_s ? __int_as_float(0x7fc00000) : pow2f(-e);
 }
 
@@ -413,9 +436,9 @@ cudaError_t launch_x16_prep(const float* xt, int64_t n_in, int bits, int batch, 
   (void)status;
   const int64_t ld = x16_ld(n_in);
   if (bits == 4)
-    x16_prep_kernel<4><<<batch, 256, 0, st>>>(xt, (int)n_in, ld, x16, rowscale);
+    x16_prep_kernel<4><<<batch, kPrepThreads, 0, st>>>(xt, (int)n_in, ld, x16, rowscale);
   else
-    x16_prep_kernel<2><<<batch, 256, 0, st>>>(xt, (int)n_in, ld, x16, rowscale);
+    x16_prep_kernel<2><<<batch, kPrepThreads, 0, st>>>(xt, (int)n_in, ld, x16, rowscale);
   return cudaGetLastError();
 }
 
