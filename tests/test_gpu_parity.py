@@ -352,3 +352,38 @@ def test_full_7b_stack_in_the_bench_configuration():
     print(f"32-block fused vs per-linear rel-L2 {err:.3e}")
     assert err < GATE
     assert np.array_equal(y_lin[0], y_lin[1])
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_int16_operand_error_within_its_bound(bits):
+    """The dequant-GEMV carries x~ = F_V(x) as int16 with one power-of-two scale per group of
+    64 (max |x~| 2^e in [2^14, 2^15)), so each element is off by at most half a step,
+    2^-15 max_g |x~|, and row r of z = deq(codes) x~ by at most
+        b_r = sum_g 2^-15 max_g |x~| sum_{j in g} |s16 q_j + zero16|.
+    F_U is orthogonal, so ||y_gpu - y_oracle|| <= ||b|| plus the fp32 rounding of the
+    butterflies. x~ is built on the host with a x20 outlier in one group and a x1000 one in
+    another (small entries next to them keep only a few bits), and x = F_V^T x~."""
+    import rotated_bit_matmul_b200 as rb
+    n_out, n_in, w_in, w_out = 512, 1024, 1024, 512
+    case = oracle_layer(n_out, n_in, w_in, w_out, bits, workload=13)
+    rng = np.random.default_rng(13)
+    xt = rng.standard_normal(n_in)
+    xt[70] *= 20.0     # group 1: one x20 outlier
+    xt[700] *= 1000.0  # group 10: one x1000 outlier
+    x = oracle.butterfly_inv(xt[None], case["thV"], case["sV"], w_in).astype(np.float32)
+    L = device_layer(case)
+    got = L(_dev(x, torch.float32), out_dtype=torch.float32).cpu().numpy()[0]
+    L.close()
+    want = oracle.linear_fwd(case["lay"], x.astype(np.float64))[0]
+    xt_exact = oracle.butterfly_fwd(x.astype(np.float64), case["thV"], case["sV"], w_in)[0]
+    gmax = np.abs(xt_exact).reshape(-1, 64).max(axis=1)
+    q = oracle.unpack(case["lay"].packed, n_out, n_in, bits).astype(np.float64)
+    s16 = oracle.f16_to_f64(case["s16"])
+    z16 = oracle.f16_to_f64(case["z16"])
+    deq = np.abs(np.repeat(s16, 64, axis=1) * q + np.repeat(z16, 64, axis=1))
+    b = (deq.reshape(n_out, -1, 64).sum(axis=2) * gmax[None, :] * 2.0 ** -15).sum(axis=1)
+    err = np.linalg.norm(got - want)
+    bound = np.linalg.norm(b) + 1e-5 * np.linalg.norm(want)
+    print(f"{bits}-bit: error {err:.3e}, bound {bound:.3e}, rel-L2 {err / np.linalg.norm(want):.3e}")
+    assert err <= bound, (err, bound)
+    assert err / np.linalg.norm(want) < GATE
