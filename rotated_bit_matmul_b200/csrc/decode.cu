@@ -77,9 +77,12 @@ struct FGeo {
 };
 
 // ------------------------------------------------------------------ shared memory carve-up
+constexpr int kMaxWon = 16;  // MLP blocks one CTA can complete in a block's gate/up phase
+
 struct Smem : EngCtx {
   uint8_t* ring;
   float* misc;     // [0, 8) rms partials by source CTA, [8, 24) per-warp scratch
+  int* won;        // [0]: count, then up to kMaxWon MLP blocks whose last unit this CTA completed
   int32_t* xq;     // GEMV operand: xq words, then xs [ng], then xsum [ng]
   float* red;      // GEMV reduction scratch: ring_stages x 16 warps x 32 lanes
   int* ucnt;       // per ring stage: warps of the half done with the unit
@@ -99,6 +102,8 @@ __device__ __forceinline__ Smem carve(const Params& p, int stage_bytes) {
   s.rx[1] = reinterpret_cast<float*>(b);
   b += 4 * kRxFloats;
   s.misc = reinterpret_cast<float*>(b);
+  b += 4 * 32;
+  s.won = reinterpret_cast<int*>(b);
   b += 4 * 32;
   s.red = reinterpret_cast<float*>(b);
   b += (size_t)4 * kCW * 32 * p.ring_stages;
@@ -516,8 +521,11 @@ __device__ __forceinline__ void prefetch_unit(const Range& g, int u) {
 // half to finish a unit reduces its 8 per-warp partial rows and writes the unit's sums.
 constexpr int kHalf = kCW / 2;
 
+// tickets: with MLP-block tickets in the gate/up phase, the per-block completion counters of
+// this block (else null); per_block: gate and up units of one MLP block
 template <int BITS>
-__device__ __forceinline__ bool run_units(const Params& p, Smem& s, const Range& g, uint32_t& kring, int ct) {
+__device__ __forceinline__ bool run_units(const Params& p, Smem& s, const Range& g, uint32_t& kring, int ct,
+                                          unsigned* tickets = nullptr, unsigned per_block = 0, int wb = 0) {
   using Gm = FGeo<BITS>;
   const int warp = ct >> 5, lane = ct & 31;
   const int hv = warp / kHalf, hw = warp - hv * kHalf;  // half, warp within the half
@@ -568,6 +576,21 @@ __device__ __forceinline__ bool run_units(const Params& p, Smem& s, const Range&
 #pragma unroll
       for (int w = 0; w < kHalf; ++w) t += red[w * 32 + lane];
       if (ok && row0 + lane < n_out) g.zp[(int64_t)kc * n_out + row0 + lane] = t;
+      if (tickets) {
+        // the partials are visible device-wide before the block's ticket counts them; the
+        // CTA that brings the count to per_block runs the block's chain after this phase
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) {
+          const int blk = row0 / wb;
+          unsigned old;
+          asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(tickets + blk) : "memory");
+          if (old + 1 == per_block) {
+            const int i = atomicAdd(&s.won[0], 1);
+            if (i < kMaxWon) s.won[1 + i] = blk;
+          }
+        }
+      }
       __syncwarp();
       if (lane == 0) s.ucnt[slot] = 0;
     }
@@ -668,6 +691,17 @@ __device__ __forceinline__ bool mlp_any(const Params& p, Smem& sm, Xch& x, const
   }
 }
 
+// one local MLP block (width <= 512) by index
+template <int TM>
+__device__ __forceinline__ void mlp_local_blk(const Params& p, Smem& sm, const Lin* lin, int blk, int ct) {
+  switch (p.eb_blk) {
+    case 6: mlp_block_local<6, TM>(p, sm, lin + 4, lin + 5, lin + 6, blk, ct); break;
+    case 7: mlp_block_local<7, TM>(p, sm, lin + 4, lin + 5, lin + 6, blk, ct); break;
+    case 8: mlp_block_local<8, TM>(p, sm, lin + 4, lin + 5, lin + 6, blk, ct); break;
+    default: mlp_block_local<9, TM>(p, sm, lin + 4, lin + 5, lin + 6, blk, ct); break;
+  }
+}
+
 // P7 roles: MLP-block CTAs or clusters first, the last two clusters apply F_U_q / F_U_k
 __device__ __forceinline__ int qk_cluster(const Params& p, int which) { return p.G - 1 - which; }
 
@@ -684,6 +718,7 @@ __global__ void __maxnreg__(120) decode_kernel(const __grid_constant__ Params p)
 
   if (tid == 0) {
     s_wait_cycles = p.wait_cycles;
+    s.won[0] = 0;
     for (int i = 0; i < p.ring_stages; ++i) {
       mbar_init(&s.full[i], 1);
       mbar_init(&s.empty[i], kHalf);  // the 8 warps of the half that consumed the unit
@@ -794,10 +829,23 @@ __global__ void __maxnreg__(120) decode_kernel(const __grid_constant__ Params p)
     // P5
     if (!(ok = residual_any<TM>(p, s, X, res, lin + 3, p.zpo, p.nk_h, lin + 4 + p.asg_gu[c], r, ct))) break;
     // P6
-    if (!(ok = run_units<BITS>(p, s, units<BITS>(p, l, 2, c, (int)r), kring, ct))) break;
-    if (!(ok = grid_barrier(p, l * 5 + 2, ct))) break;
-    // P7
-    if (!(ok = mlp_any<TM>(p, s, X, lin, c, r, ct))) break;
+    if (p.mlp_tickets) {
+      const int wb = lin[4].w_out;
+      const unsigned per_block = (unsigned)(2 * (wb / 32) * p.nk_h);
+      unsigned* tickets = p.counters + 5 * L + (size_t)l * p.nblocks;
+      if (!(ok = run_units<BITS>(p, s, units<BITS>(p, l, 2, c, (int)r), kring, ct, tickets, per_block, wb))) break;
+      // P7 for the MLP blocks this CTA completed (their partials are all written)
+      const int nw = min(s.won[0], kMaxWon);
+      if (s.won[0] > kMaxWon) report(p.status, 6, 70);  // cannot happen: a CTA's units span few blocks
+      for (int i = 0; i < nw; ++i) mlp_local_blk<TM>(p, s, lin, s.won[1 + i], ct);
+      cbar();
+      if (ct == 0) s.won[0] = 0;
+    } else {
+      if (!(ok = run_units<BITS>(p, s, units<BITS>(p, l, 2, c, (int)r), kring, ct))) break;
+      if (!(ok = grid_barrier(p, l * 5 + 2, ct))) break;
+      // P7
+      if (!(ok = mlp_any<TM>(p, s, X, lin, c, r, ct))) break;
+    }
     {
       const int qk = c == qk_cluster(p, 0) ? 0 : (c == qk_cluster(p, 1) ? 1 : -1);
       if (qk >= 0) {
@@ -845,7 +893,7 @@ __global__ void __maxnreg__(120) decode_kernel(const __grid_constant__ Params p)
 // ------------------------------------------------------------------ host side
 template <int BITS>
 size_t smem_bytes(const Params& p) {
-  return 1024 + (size_t)p.ring_stages * FGeo<BITS>::kStageBytes + 3 * 4 * (size_t)kRxFloats + 4 * 32 +
+  return 1024 + (size_t)p.ring_stages * FGeo<BITS>::kStageBytes + 3 * 4 * (size_t)kRxFloats + 4 * 32 + 4 * 32 +
          (size_t)4 * kCW * 32 * p.ring_stages + 4 * ((p.ring_stages + 3) & ~3) + p.xq_bytes +
          8 * (2 * (size_t)p.ring_stages + 2);
 }

@@ -48,7 +48,8 @@ struct Params {
   int32_t* xq_down;
   float* xs_down;
   float* xsum_down;
-  unsigned* counters;  // [L][5], zero at launch
+  unsigned* counters;  // [L][5] grid barriers, then [L][nblocks] MLP-block tickets; zero at launch
+  int mlp_tickets;     // 1: an MLP block's chain runs in the CTA that completes its last gate/up unit
   int* status;
   long long wait_cycles;  // bound of every wait, in SM clock cycles
   int barrier_extra;      // testing hook: grid barrier whose target is raised by one (-1: none)

@@ -143,7 +143,8 @@ size_t fused_ws(const harp_stack_s* S, dec::Params* p, void* base) {
   char* xq = take(4 * words);
   char* xs = take(4 * ngf);
   char* xsum = take(4 * ngf);
-  char* cnt = take(4 * 5 * L);
+  const size_t nblk = (size_t)(F / (size_t)S->layers[4]->L.w_out);
+  char* cnt = take(4 * (5 + nblk) * L);
   if (p) {
     p->nk_h = (int)nkh;
     p->nk_f = (int)nkf;
@@ -285,6 +286,10 @@ void setup_fused(harp_stack_s* S) {
   if (const char* e = getenv("HARP_PF_DIST")) p.pf_dist = std::max(0, atoi(e));
   p.cooperative = 1;
   if (const char* e = getenv("HARP_COOPERATIVE")) p.cooperative = atoi(e) != 0;
+  // MLP blocks up to 512 wide: the chain runs where the block's last gate/up unit completes
+  // (one grid barrier less per block); HARP_MLP_TICKETS=0 keeps the barrier
+  p.mlp_tickets = wb <= 512 && F % 32 == 0;
+  if (const char* e = getenv("HARP_MLP_TICKETS")) p.mlp_tickets = p.mlp_tickets && atoi(e) != 0;
   int G = 0;
   cudaError_t e = dec::max_clusters(p, &G);
   if (e != cudaSuccess || G < 1) return no(std::string("cluster occupancy query failed: ") + cudaGetErrorString(e));
@@ -416,7 +421,8 @@ harp_status harp_stack_step(harp_stack S, int batch, const void* x, harp_dtype x
     const TestHooks th = test_hooks();
     p.wait_cycles = th.wait_cycles;
     p.barrier_extra = th.decode_barrier_extra;
-    cudaError_t e = cudaMemsetAsync(p.counters, 0, sizeof(unsigned) * 5 * (size_t)S->n_layers, st);
+    cudaError_t e =
+        cudaMemsetAsync(p.counters, 0, sizeof(unsigned) * (5 + (size_t)p.nblocks) * (size_t)S->n_layers, st);
     if (e == cudaSuccess) e = dec::launch(p, st);
     if (e != cudaSuccess) return sfail(HARP_ERR_CUDA, std::string("fused decode step: ") + cudaGetErrorString(e));
     return HARP_OK;
