@@ -324,8 +324,9 @@ harp_status harp_stack_workspace_size(harp_stack stack, int batch, size_t* bytes
 
 /* 1 when harp_stack_step with this batch runs the fused single-kernel decode step
  * (batch 1, hidden a power of two in [4096, 8192], n_heads*head_dim == hidden, single-block
- * q/k/v/o/down butterflies, gate/up output blocks 64..512 wide, one bit width), else 0
- * (the step then runs one launch sequence per linear). */
+ * q/k/v/o/down butterflies, gate/up output blocks 64..512, 4096 or 8192 wide, one bit width,
+ * one form of the angles), else 0
+ * (the step then runs one launch sequence per linear; harp_last_error() then says why). */
 int harp_stack_uses_fused_step(harp_stack stack, int batch);
 
 /* One decode step: out = stack(x). x, out: device [batch][hidden] of dtypes xt / ot

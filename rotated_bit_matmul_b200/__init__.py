@@ -305,8 +305,14 @@ class HarpStack:
         return n.value
 
     def uses_fused_step(self, batch: int = 1) -> bool:
-        """True when a step of this batch runs the single-kernel fused decode path."""
+        """True when a step of this batch runs the single-kernel fused decode path (when the
+        stack's shapes keep it on the per-linear path, harp_last_error says why)."""
         return bool(load().harp_stack_uses_fused_step(self.handle, int(batch)))
+
+    def fused_reason(self) -> str:
+        """Why the fused decode step is not taken ('' when it is)."""
+        lib = load()
+        return "" if lib.harp_stack_uses_fused_step(self.handle, 1) else lib.harp_last_error().decode()
 
     def workspace(self, batch: int):
         ws = self._ws.get(batch)

@@ -199,6 +199,19 @@ struct Map {
   __device__ static int idx_b(int j, int ii) { return j * PAD + ii; }
 };
 
+// the lane bit a stage pairs on: t in phase 1, t - 5 in phase 2, t - EB across the cluster
+__device__ __forceinline__ int stage_lane_bit(int EB, int t) { return t < (EB < 5 ? EB : 5) ? t : (t < EB ? t - 5 : t - EB); }
+// the lane with bit b removed (4 bits) / a 4-bit value with a zero inserted at bit b
+__device__ __forceinline__ int rm_bit(int x, int b) { return ((x >> (b + 1)) << b) | (x & ((1 << b) - 1)); }
+__device__ __forceinline__ int ins0(int x, int b) { return ((x >> b) << (b + 1)) | (x & ((1 << b) - 1)); }
+// Thread-order coefficient tables: for every stage the two lanes of a pair share one slot,
+// (warp << 4) | (lane without the stage's lane bit), so a warp reads 16 consecutive entries.
+// Layout [block][cta r][stage t][slot s][NT/2 slots]; entries are (cos, sin) float2, or the
+// angle pi/4 + delta_t q as a float for int8 layers.
+__device__ __forceinline__ int stage_slot(int EB, int t, int ct) {
+  return ((ct >> 5) << 4) | rm_bit(ct & 31, stage_lane_bit(EB, t));
+}
+
 // layout-A buffer index: xor swizzle keeps a warp's phase-1 and phase-2 accesses on
 // (nearly) distinct banks
 __device__ __forceinline__ int idx_a(int e) { return e ^ ((e >> 5) & 31); }
@@ -237,6 +250,15 @@ __device__ __forceinline__ Cf<TM> fetch_cf(const uint8_t* tab, int64_t half_n, i
     const int8_t code = __ldg(reinterpret_cast<const int8_t*>(tab + kQ8Head) + (int64_t)t * half_n + q);
     c.psi = fmaf(step, (float)code, kQuarterPi);
   }
+  return c;
+}
+
+// one entry of a thread-order table (see stage_slot)
+template <int TM>
+__device__ __forceinline__ Cf<TM> fetch_rt(const uint8_t* rt, int64_t idx) {
+  Cf<TM> c;
+  if constexpr (TM == kTmCS) c.v = __ldg(reinterpret_cast<const float2*>(rt) + idx);
+  else if constexpr (TM == kTmQ8) c.psi = __ldg(reinterpret_cast<const float*>(rt) + idx);
   return c;
 }
 
@@ -285,6 +307,19 @@ struct ClusterBfly {
         for (int t = 0; t < NS; ++t)
           cf[t][s] = fetch_cf<TM>(tab, half_n, t, pair_of(t < 5 ? g1 : (t < EB ? g2 : gb), t));
       }
+    }
+  }
+
+  // the same coefficients from a thread-order table (block blk of the side)
+  __device__ __forceinline__ void fetch_rt(const uint8_t* rt, int64_t blk, uint32_t r, int ct) {
+    if constexpr (TM != kTmHad) {
+      if (ct >= M::NT) return;
+      const int64_t base = (blk * kC + r) * (int64_t)NS;
+#pragma unroll
+      for (int t = 0; t < NS; ++t)
+#pragma unroll
+        for (int s = 0; s < M::P; ++s)
+          cf[t][s] = dec::fetch_rt<TM>(rt, ((base + t) * M::P + s) * (M::NT / 2) + stage_slot(EB, t, ct));
     }
   }
 
@@ -358,6 +393,15 @@ struct LocalBfly {
     }
   }
 
+  __device__ __forceinline__ void fetch_rt(const uint8_t* rt, int64_t blk, int ct) {
+    if constexpr (TM != kTmHad) {
+      if (ct >= M::NT) return;
+#pragma unroll
+      for (int t = 0; t < EB; ++t)
+        cf[t] = dec::fetch_rt<TM>(rt, (blk * EB + t) * (int64_t)(M::NT / 2) + stage_slot(EB, t, ct));
+    }
+  }
+
   __device__ __forceinline__ void run(float& v, EngCtx& sm, int ct) {
     const bool act = ct < M::NT;
     if (act)
@@ -375,6 +419,42 @@ struct LocalBfly {
     }
   }
 };
+
+// Builds a thread-order table for nblk blocks of a side (block width w = 8 * 2^EB spread
+// over a cluster when cluster, else w = 2^EB in one CTA) from the layer's storage (tab:
+// float2 (cos, sin) [m][n/2], or int8 after a 64-byte head of steps). One thread per entry.
+template <int EB, int TM, bool CLUSTER>
+__global__ void repack_kernel(const uint8_t* tab, int64_t half_n, int nblk, uint8_t* rt) {
+  using M = Map<EB>;
+  constexpr int NS = CLUSTER ? EB + 3 : EB, P = CLUSTER ? M::P : 1, NR = CLUSTER ? kC : 1, H = M::NT / 2;
+  const int64_t total = (int64_t)nblk * NR * NS * P * H;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+    int64_t k = i;
+    const int slot = (int)(k % H);
+    k /= H;
+    const int s = (int)(k % P);
+    k /= P;
+    const int t = (int)(k % NS);
+    k /= NS;
+    const int r = (int)(k % NR);
+    const int64_t blk = k / NR;
+    const int b = stage_lane_bit(EB, t);
+    const int ct = ((slot >> 4) << 5) | ins0(slot & 15, b);  // the lane of the pair with the bit clear
+    int64_t g;
+    if (t < (EB < 5 ? EB : 5)) g = (int64_t)r * M::E + M::e1(ct, s);
+    else if (t < EB) g = (int64_t)r * M::E + M::e2(ct, s);
+    else g = (int64_t)M::bj(ct) * M::E + (int64_t)r * M::RUN + M::bii(ct, s);
+    const int64_t w = (int64_t)NR * M::E;
+    const int64_t q = blk * (w >> 1) + pair_of(g, t);
+    if constexpr (TM == kTmCS) {
+      reinterpret_cast<float2*>(rt)[i] = reinterpret_cast<const float2*>(tab)[(int64_t)t * half_n + q];
+    } else {
+      const float step = reinterpret_cast<const float*>(tab)[t];
+      const int8_t code = reinterpret_cast<const int8_t*>(tab + kQ8Head)[(int64_t)t * half_n + q];
+      reinterpret_cast<float*>(rt)[i] = fmaf(step, (float)code, kQuarterPi);
+    }
+  }
+}
 
 }  // namespace dec
 }  // namespace harp

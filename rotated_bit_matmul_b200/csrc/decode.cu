@@ -117,6 +117,20 @@ __device__ __forceinline__ Smem carve(const Params& p, int stage_bytes) {
   return s;
 }
 
+// a butterfly's coefficients: from the side's thread-order table when the stack built one
+template <int EB, int TM>
+__device__ __forceinline__ void fetch_side(ClusterBfly<EB, TM>& bf, const uint8_t* rt, const uint8_t* tab,
+                                           int64_t half_n, int64_t blk, uint32_t r, int ct) {
+  if (rt) bf.fetch_rt(rt, blk, r, ct);
+  else bf.fetch(tab, half_n, blk, r, ct);
+}
+template <int EB, int TM>
+__device__ __forceinline__ void fetch_side(LocalBfly<EB, TM>& bf, const uint8_t* rt, const uint8_t* tab,
+                                           int64_t half_n, int64_t blk, int ct) {
+  if (rt) bf.fetch_rt(rt, blk, ct);
+  else bf.fetch(tab, half_n, blk, ct);
+}
+
 // ------------------------------------------------------------------ GEMV operand
 // x~ of a hidden-wide input in layout B (runs of >= 64): the CTA's groups into its own
 // operand buffer, then to every peer's (one exchange)
@@ -189,7 +203,7 @@ __device__ __noinline__ bool chain_residual(const Params& p, Smem& sm, Xch& x, f
       for (int s = 0; s < M::P; ++s) res[s] = load_act(p.x_in, BF::gb(r, ct, s), p.xt);
   } else {
     BF fu;
-    fu.fetch(U->tU, (int64_t)U->n_out / 2, 0, r, ct);
+    fetch_side(fu, U->rU, U->tU, (int64_t)U->n_out / 2, 0, r, ct);
     float v[2] = {0.f, 0.f};
     if (act)
 #pragma unroll
@@ -204,7 +218,7 @@ __device__ __noinline__ bool chain_residual(const Params& p, Smem& sm, Xch& x, f
   }
   if (!V || !ok) return ok;
   BF fv;
-  fv.fetch(V->tV, (int64_t)V->n_in / 2, 0, r, ct);
+  fetch_side(fv, V->rV, V->tV, (int64_t)V->n_in / 2, 0, r, ct);
   // sum of squares: warps, then the CTA (fixed order), then to every peer's slot r along
   // with the residual values each peer holds in layout A for F_V
   float acc = 0.f;
@@ -252,7 +266,7 @@ __device__ __noinline__ bool chain_attn(const Params& p, Smem& sm, Xch& x, const
   using MU = Map<EBU>;
   using M = Map<EB>;
   ClusterBfly<EBU, TM> fu;
-  fu.fetch(Lv->tU, (int64_t)Lv->n_out / 2, 0, r, ct);
+  fetch_side(fu, Lv->rU, Lv->tU, (int64_t)Lv->n_out / 2, 0, r, ct);
   float v[2] = {0.f, 0.f};
   if (ct < MU::NT)
 #pragma unroll
@@ -262,7 +276,7 @@ __device__ __noinline__ bool chain_attn(const Params& p, Smem& sm, Xch& x, const
     }
   if (!fu.run(v, sm, x, r, ct, p.status, 44)) return false;
   ClusterBfly<EB, TM> fv;
-  fv.fetch(Lo->tV, (int64_t)Lo->n_in / 2, 0, r, ct);
+  fetch_side(fv, Lo->rV, Lo->tV, (int64_t)Lo->n_in / 2, 0, r, ct);
   // every v value to the layout-A owners of the query-head elements that copy it
   const int hd = p.head_dim, rep = p.rep;
   int self = 0;
@@ -303,7 +317,7 @@ __device__ __noinline__ bool chain_out_only(const Params& p, Smem& sm, Xch& x, c
   using M = Map<EB>;
   using BF = ClusterBfly<EB, TM>;
   BF fu;
-  fu.fetch(Lq->tU, (int64_t)Lq->n_out / 2, 0, r, ct);
+  fetch_side(fu, Lq->rU, Lq->tU, (int64_t)Lq->n_out / 2, 0, r, ct);
   float v[2] = {0.f, 0.f};
   if (ct < M::NT)
 #pragma unroll
@@ -327,9 +341,9 @@ __device__ __noinline__ void mlp_block_local(const Params& p, Smem& sm, const Li
                                              int blk, int ct) {
   using M = Map<EB>;
   LocalBfly<EB, TM> fg, fu, fd;
-  fg.fetch(Lg->tU, (int64_t)Lg->n_out / 2, blk, ct);
-  fu.fetch(Lu->tU, (int64_t)Lu->n_out / 2, blk, ct);
-  fd.fetch(Ld->tV, (int64_t)Ld->n_in / 2, blk, ct);
+  fetch_side(fg, Lg->rU, Lg->tU, (int64_t)Lg->n_out / 2, blk, ct);
+  fetch_side(fu, Lu->rU, Lu->tU, (int64_t)Lu->n_out / 2, blk, ct);
+  fetch_side(fd, Ld->rV, Ld->tV, (int64_t)Ld->n_in / 2, blk, ct);
   const bool act = ct < M::NT;
   const int64_t base = (int64_t)blk * M::E;
   float vg = 0.f, vu = 0.f;
@@ -377,7 +391,7 @@ __device__ __noinline__ bool mlp_block_cluster(const Params& p, Smem& sm, Xch& x
   float vg[2] = {0.f, 0.f}, vu[2] = {0.f, 0.f};
   {
     BF fg;
-    fg.fetch(Lg->tU, (int64_t)Lg->n_out / 2, blk, r, ct);
+    fetch_side(fg, Lg->rU, Lg->tU, (int64_t)Lg->n_out / 2, blk, r, ct);
     if (act)
 #pragma unroll
       for (int s = 0; s < M::P; ++s) {
@@ -388,7 +402,7 @@ __device__ __noinline__ bool mlp_block_cluster(const Params& p, Smem& sm, Xch& x
   }
   {
     BF fu;
-    fu.fetch(Lu->tU, (int64_t)Lu->n_out / 2, blk, r, ct);
+    fetch_side(fu, Lu->rU, Lu->tU, (int64_t)Lu->n_out / 2, blk, r, ct);
     if (act)
 #pragma unroll
       for (int s = 0; s < M::P; ++s) {
@@ -398,7 +412,7 @@ __device__ __noinline__ bool mlp_block_cluster(const Params& p, Smem& sm, Xch& x
     if (!fu.run(vu, sm, x, r, ct, p.status, 49)) return false;
   }
   BF fd;
-  fd.fetch(Ld->tV, (int64_t)Ld->n_in / 2, blk, r, ct);
+  fetch_side(fd, Ld->rV, Ld->tV, (int64_t)Ld->n_in / 2, blk, r, ct);
   // h = silu(gate) * up in layout B, to the layout-A owners
   xch_begin(sm, x, 4u * M::RUN * (kC - 1), ct);
   if (act)
@@ -888,6 +902,38 @@ __global__ void __maxnreg__(120) decode_kernel(const __grid_constant__ Params p)
     }
   }
   cluster_sync_all();
+}
+
+// ------------------------------------------------------------------ thread-order tables
+size_t repack_bytes(int tm, int eb, bool cluster, int nblk) {
+  if (tm == kTmHad) return 0;
+  const int E = 1 << eb, nt = E < kNT ? E : kNT, P = cluster && E > kNT ? E / kNT : 1;
+  const int ns = cluster ? eb + 3 : eb, nr = cluster ? kC : 1;
+  return (size_t)nblk * nr * ns * P * (nt / 2) * (tm == kTmCS ? 8 : 4);
+}
+
+template <int TM, bool CLUSTER>
+static cudaError_t repack_t(int eb, int nblk, const uint8_t* tab, int64_t half_n, uint8_t* rt, cudaStream_t st) {
+  const int grid = 296, thr = 256;
+  switch (eb) {
+    case 5: if (CLUSTER) repack_kernel<5, TM, CLUSTER><<<grid, thr, 0, st>>>(tab, half_n, nblk, rt); else return cudaErrorInvalidValue; break;
+    case 6: repack_kernel<6, TM, CLUSTER><<<grid, thr, 0, st>>>(tab, half_n, nblk, rt); break;
+    case 7: repack_kernel<7, TM, CLUSTER><<<grid, thr, 0, st>>>(tab, half_n, nblk, rt); break;
+    case 8: repack_kernel<8, TM, CLUSTER><<<grid, thr, 0, st>>>(tab, half_n, nblk, rt); break;
+    case 9: repack_kernel<9, TM, CLUSTER><<<grid, thr, 0, st>>>(tab, half_n, nblk, rt); break;
+    case 10: if (CLUSTER) repack_kernel<10, TM, CLUSTER><<<grid, thr, 0, st>>>(tab, half_n, nblk, rt); else return cudaErrorInvalidValue; break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t repack_side(int tm, int eb, bool cluster, int nblk, const uint8_t* tab, int64_t half_n, uint8_t* rt,
+                        cudaStream_t st) {
+  if (tm == kTmCS) return cluster ? repack_t<kTmCS, true>(eb, nblk, tab, half_n, rt, st)
+                                  : repack_t<kTmCS, false>(eb, nblk, tab, half_n, rt, st);
+  if (tm == kTmQ8) return cluster ? repack_t<kTmQ8, true>(eb, nblk, tab, half_n, rt, st)
+                                  : repack_t<kTmQ8, false>(eb, nblk, tab, half_n, rt, st);
+  return cudaSuccess;
 }
 
 // ------------------------------------------------------------------ host side

@@ -26,6 +26,8 @@ struct alignas(64) Lin {
   const uint8_t* tU;  // output-side angle storage
   const int8_t* sV;
   const int8_t* sU;
+  const uint8_t* rV;  // thread-order copies of the angle storage (see repack_side), or null
+  const uint8_t* rU;
   int n_in, n_out, w_in, w_out, m_in, m_out, pad0, pad1;
 };
 
@@ -62,6 +64,12 @@ struct Params {
 };
 
 cudaError_t launch(const Params& p, cudaStream_t st);
+// Thread-order copy of one side's angles for the fused step: nblk blocks, each spread over a
+// cluster (per-CTA share 2^eb) or held by one CTA (width 2^eb). Bytes of the copy, and the
+// kernel that builds it from the layer's storage (tab) on `st`.
+size_t repack_bytes(int tm, int eb, bool cluster, int nblk);
+cudaError_t repack_side(int tm, int eb, bool cluster, int nblk, const uint8_t* tab, int64_t half_n, uint8_t* rt,
+                        cudaStream_t st);
 size_t smem_for(const Params& p);
 int chunk_cols_for(int bits);
 cudaError_t max_clusters(const Params& p, int* out);

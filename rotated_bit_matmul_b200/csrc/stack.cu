@@ -2,6 +2,7 @@
 // layers: RMSNorm, residual adds, SiLU * up, and the key/value-group broadcast of a
 // one-key attention (its output is the value), around harp linear forwards.
 #include <algorithm>
+#include <cstdio>
 #include <cstdlib>
 #include <cstring>
 #include <new>
@@ -21,6 +22,7 @@ struct harp_stack_s {
   // fused batch-1 decode step (null when this stack's shapes are outside its domain)
   bool fused = false;
   dec::Lin* d_lin = nullptr;
+  uint8_t* d_rt = nullptr;  // thread-order angle tables of every butterfly (one allocation)
   dec::Params fp{};
   std::string fused_why;
 };
@@ -292,12 +294,17 @@ void setup_fused(harp_stack_s* S) {
   if (const char* e = getenv("HARP_MLP_TICKETS")) p.mlp_tickets = p.mlp_tickets && atoi(e) != 0;
   int G = 0;
   cudaError_t e = dec::max_clusters(p, &G);
-  if (e != cudaSuccess || G < 1) return no(std::string("cluster occupancy query failed: ") + cudaGetErrorString(e));
+  if (e != cudaSuccess || G < 1)
+    return no(std::string("cluster occupancy query failed: ") + cudaGetErrorString(e) + ", G=" + std::to_string(G) +
+              ", smem " + std::to_string(dec::smem_for(p)) + ", ring stages " + std::to_string(p.ring_stages));
   if (G > dec::kMaxClusters) G = dec::kMaxClusters;
   // P7: MLP-block CTAs (or clusters) come first, the last two clusters apply F_U_q / F_U_k
   const int cap = wb <= 512 ? dec::kC : 1;
   if (G < 3 || p.nblocks > (G - 2) * cap) return no("too few co-resident clusters");
   p.G = G;
+  if (getenv("HARP_DEBUG"))
+    fprintf(stderr, "harp fused step: G=%d ring_stages=%d smem=%zu xq_bytes=%d eb_h=%d eb_kv=%d eb_blk=%d nblocks=%d tm=%d\n",
+            G, p.ring_stages, dec::smem_for(p), p.xq_bytes, p.eb_h, p.eb_kv, p.eb_blk, p.nblocks, p.tm);
   const int rq[3] = {dq, dkv, dkv}, rg[2] = {F, F};
   assign(G, rq, 3, p.asg_qkv, p.idx_qkv, p.cnt_qkv);
   assign(G, rg, 2, p.asg_gu, p.idx_gu, p.cnt_gu);
@@ -320,6 +327,48 @@ void setup_fused(harp_stack_s* S) {
     d.w_out = L.w_out;
     d.m_in = L.m_in;
     d.m_out = L.m_out;
+  }
+  // thread-order copies of the angle tables (HARP_REPACK=0 reads the layers' own tables)
+  bool repack = tm != dec::kTmHad;
+  if (const char* e = getenv("HARP_REPACK")) repack = repack && atoi(e) != 0;
+  if (repack) {
+    struct Side {
+      size_t i;
+      bool u, cl;
+      int eb, nblk;
+    };
+    std::vector<Side> sides;
+    auto mlp = [&](size_t i, bool u) {
+      if (wb <= 512) sides.push_back({i, u, false, p.eb_blk, p.nblocks});
+      else sides.push_back({i, u, true, p.eb_blk - 3, p.nblocks});
+    };
+    for (size_t i = 0; i < h.size(); ++i) {
+      const int li = (int)(i % 7);
+      if (li <= 5) sides.push_back({i, false, true, p.eb_h, 1});
+      else mlp(i, false);
+      if (li == 0 || li == 3 || li == 6) sides.push_back({i, true, true, p.eb_h, 1});
+      else if (li == 1 || li == 2) sides.push_back({i, true, true, p.eb_kv, 1});
+      else mlp(i, true);
+    }
+    size_t total = 0;
+    for (const Side& sd : sides) total += (dec::repack_bytes(tm, sd.eb, sd.cl, sd.nblk) + 255) & ~size_t(255);
+    if (cudaMalloc(&S->d_rt, total) != cudaSuccess) return no("cudaMalloc of the thread-order tables failed");
+    size_t off = 0;
+    for (const Side& sd : sides) {
+      dec::Lin& d = h[sd.i];
+      const Layer& L = S->layers[sd.i]->L;
+      uint8_t* dst = S->d_rt + off;
+      off += (dec::repack_bytes(tm, sd.eb, sd.cl, sd.nblk) + 255) & ~size_t(255);
+      const uint8_t* src = sd.u ? d.tU : d.tV;
+      if (dec::repack_side(tm, sd.eb, sd.cl, sd.nblk, src, (sd.u ? L.n_out : L.n_in) / 2, dst, 0) != cudaSuccess) {
+        cudaFree(S->d_rt);
+        S->d_rt = nullptr;
+        return no("building the thread-order tables failed");
+      }
+      if (sd.u) d.rU = dst;
+      else d.rV = dst;
+    }
+    if (cudaStreamSynchronize(0) != cudaSuccess) return no("building the thread-order tables failed");
   }
   if (cudaMalloc(&S->d_lin, sizeof(dec::Lin) * h.size()) != cudaSuccess) return no("cudaMalloc failed");
   if (cudaMemcpy(S->d_lin, h.data(), sizeof(dec::Lin) * h.size(), cudaMemcpyHostToDevice) != cudaSuccess) {
@@ -373,19 +422,23 @@ harp_status harp_stack_create(harp_stack* out, int n_layers, int hidden, int ffn
 
 harp_status harp_stack_destroy(harp_stack stack) {
   if (!stack) return HARP_OK;
-  if (stack->d_lin) {
+  if (stack->d_lin || stack->d_rt) {
     int prev = 0;
     cudaGetDevice(&prev);
     cudaSetDevice(stack->device);
     cudaDeviceSynchronize();
     cudaFree(stack->d_lin);
+    cudaFree(stack->d_rt);
     cudaSetDevice(prev);
   }
   delete stack;
   return HARP_OK;
 }
 
-int harp_stack_uses_fused_step(harp_stack stack, int batch) { return stack && stack->fused && batch == 1; }
+int harp_stack_uses_fused_step(harp_stack stack, int batch) {
+  if (stack && !stack->fused) set_error(HARP_OK, "fused step not taken: %s", stack->fused_why.c_str());
+  return stack && stack->fused && batch == 1;
+}
 
 harp_status harp_stack_workspace_size(harp_stack stack, int batch, size_t* bytes) {
   if (!stack || !bytes) return sfail(HARP_ERR_INVALID_ARG, "stack_workspace_size: null pointer");
