@@ -538,7 +538,7 @@ constexpr int kHalf = kCW / 2;
 // tickets: with MLP-block tickets in the gate/up phase, the per-block completion counters of
 // this block (else null); per_block: gate and up units of one MLP block
 template <int BITS>
-__device__ __forceinline__ bool run_units(const Params& p, Smem& s, const Range& g, uint32_t& kring, int ct,
+__device__ __noinline__ bool run_units(const Params& p, Smem& s, const Range& g, uint32_t& kring, int ct,
                                           unsigned* tickets = nullptr, unsigned per_block = 0, int wb = 0) {
   using Gm = FGeo<BITS>;
   const int warp = ct >> 5, lane = ct & 31;
@@ -719,11 +719,111 @@ __device__ __forceinline__ void mlp_local_blk(const Params& p, Smem& sm, const L
 // P7 roles: MLP-block CTAs or clusters first, the last two clusters apply F_U_q / F_U_k
 __device__ __forceinline__ int qk_cluster(const Params& p, int which) { return p.G - 1 - which; }
 
+// ---------------- producer warp: the weight ring, every unit of the step in consumer
+// order. Every lane runs the same loop (the warp never diverges around a blocking wait);
+// lane 0 waits and issues. A second cursor runs p.pf_dist units ahead and asks for those
+// units' boxes in L2, so HBM keeps streaming while the chains run and the ring's copies are
+// served from L2.
+// L2 hint for this CTA's slice of a side's thread-order table (cluster layout: CTA r's
+// entries are contiguous) and of its sign vector
+__device__ __forceinline__ void prefetch_side(const uint8_t* rt, const int8_t* sign, int eb, int tm, uint32_t r) {
+  if (!rt) return;
+  const int E = 1 << eb, nt = E < kNT ? E : kNT, P = E > kNT ? E / kNT : 1;
+  const uint32_t bytes = (uint32_t)((eb + 3) * P * (nt / 2) * (tm == kTmCS ? 8 : 4));
+  bulk_prefetch_l2(rt + (size_t)r * bytes, bytes);
+  if (E % 16 == 0) bulk_prefetch_l2(sign + (size_t)r * E, (uint32_t)E);
+}
+
+// the tables of the chain that follows GEMV phase ph of block l (lane 0 of the producer)
+__device__ __forceinline__ void prefetch_chain(const Params& p, int l, int ph, int c, uint32_t r) {
+  const Lin* lin = p.lin + 7 * l;
+  if (ph == 0) {  // P3: F_U of v, F_V of o
+    prefetch_side(lin[2].rU, lin[2].sU, p.eb_kv, p.tm, r);
+    prefetch_side(lin[3].rV, lin[3].sV, p.eb_h, p.tm, r);
+  } else if (ph == 1) {  // P5: F_U of o, F_V of the cluster's gate or up
+    prefetch_side(lin[3].rU, lin[3].sU, p.eb_h, p.tm, r);
+    prefetch_side(lin[4 + p.asg_gu[c]].rV, lin[4 + p.asg_gu[c]].sV, p.eb_h, p.tm, r);
+  } else if (ph == 3) {  // next P1: F_U of down, F_V of the cluster's q, k or v in block l + 1
+    prefetch_side(lin[6].rU, lin[6].sU, p.eb_h, p.tm, r);
+    if (l + 1 < p.L) {
+      const Lin* nx = lin + 7 + p.asg_qkv[c];
+      prefetch_side(nx->rV, nx->sV, p.eb_h, p.tm, r);
+    }
+  }
+}
+
+template <int BITS>
+__device__ __noinline__ void producer(const Params& p, Smem& s, int c, uint32_t r, int tid) {
+  using Gm = FGeo<BITS>;
+  const int L = p.L;
+  const int lane = tid & 31;
+  UnitCursor pf;
+  pf.l = 0;
+  pf.ph = 0;
+  pf.g = units<BITS>(p, 0, 0, c, (int)r);
+  pf.u = pf.g.u0;
+  pf.normalize<BITS>(p, c, (int)r);
+  if (lane == 0)
+    for (int d = 0; d < p.pf_dist && pf.l < L; ++d) {
+      prefetch_unit<BITS>(pf.g, pf.u);
+      pf.next<BITS>(p, c, (int)r);
+    }
+  uint32_t k = 0;
+  bool ok = true;
+  for (int l = 0; l < L && ok; ++l)
+    for (int ph = 0; ph < 4 && ok; ++ph) {
+      const Range g = units<BITS>(p, l, ph, c, (int)r);
+      const int ngroups = g.L->n_in / 64;
+      if (lane == 0 && p.tm != kTmHad) prefetch_chain(p, l, ph, c, r);
+      for (int u = g.u0; u < g.u1; ++u) {
+        const int slot = k % p.ring_stages;
+        int go = 1;
+        if (lane == 0) {
+          if (pf.l < L) {
+            prefetch_unit<BITS>(pf.g, pf.u);
+            pf.next<BITS>(p, c, (int)r);
+          }
+          if (k >= (uint32_t)p.ring_stages &&
+              !wait_phase<false, true>(&s.empty[slot], ((k / p.ring_stages) - 1) & 1, p.status, 53)) {
+            go = 0;
+          } else {
+            const int tile = u / g.nk, kc = u - tile * g.nk;
+            const int g0 = kc * Gm::kChunkGroups, gc = min(Gm::kChunkGroups, ngroups - g0);
+            const int cslabs = (gc + Gm::kGroupsPerSlab - 1) / Gm::kGroupsPerSlab;
+            const int hslabs = BITS == 3 ? (gc + 15) / 16 : 0;
+            uint8_t* st = s.ring + (size_t)slot * Gm::kStageBytes;
+            mbar_arrive_expect_tx(&s.full[slot], (uint32_t)((cslabs + hslabs + (gc + 31) / 32) * kSlab));
+            const int code_x0 = g0 * (BITS == 4 ? 32 : 16) / 8;
+            for (int q = 0; q < cslabs; ++q)
+              tma_load_2d(st + q * kSlab, &g.L->tm_codes, &s.full[slot], code_x0 + q * 16, tile * 32);
+            if (BITS == 3)
+              for (int q = 0; q < hslabs; ++q)
+                tma_load_2d(st + (Gm::kCodeSlabs + q) * kSlab, &g.L->tm_hi, &s.full[slot], g0 + q * 16, tile * 32);
+            for (int q = 0; q < (gc + 31) / 32; ++q)
+              tma_load_2d(st + (Gm::kCodeSlabs + Gm::kHiSlabs + q) * kSlab, &g.L->tm_sz, &s.full[slot],
+                          g0 + q * 32, tile * 32);
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, go, 0) != 0;
+        if (!ok) break;
+        ++k;  // k counts the stages issued so far
+      }
+    }
+  // drain: the copies still in flight must land before the CTA may exit (bounded, and
+  // not cut short by the abort word: these are this CTA's own copies)
+  if (lane == 0) {
+    const uint32_t nwait = k < (uint32_t)p.ring_stages ? k : (uint32_t)p.ring_stages;
+    for (uint32_t q = k - nwait; q < k; ++q)
+      wait_phase<false, true, false>(&s.full[q % p.ring_stages], (q / p.ring_stages) & 1, p.status, 54);
+  }
+  __syncwarp();
+}
+
 // ------------------------------------------------------------------ the kernel
 // TM: how every butterfly of the stack keeps its angles (kTmCS, kTmHad, kTmQ8); each form
 // has its own instantiation, so no rotation branches on it.
 template <int BITS, int TM>
-__global__ void __maxnreg__(120) decode_kernel(const __grid_constant__ Params p) {
+__global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_constant__ Params p) {
   using Gm = FGeo<BITS>;
   Smem s = carve(p, Gm::kStageBytes);
   const uint32_t r = cta_rank();
@@ -747,71 +847,7 @@ __global__ void __maxnreg__(120) decode_kernel(const __grid_constant__ Params p)
   const int L = p.L;
 
   if (tid >= kNT) {
-    // ---------------- producer warp: the weight ring, every unit of the step in consumer
-    // order. Every lane runs the same loop (the warp never diverges around a blocking
-    // wait); lane 0 waits and issues. A second cursor runs p.pf_dist units ahead and asks
-    // for those units' boxes in L2, so HBM keeps streaming while the chains run and the
-    // ring's copies are served from L2.
-    const int lane = tid & 31;
-    UnitCursor pf;
-    pf.l = 0;
-    pf.ph = 0;
-    pf.g = units<BITS>(p, 0, 0, c, (int)r);
-    pf.u = pf.g.u0;
-    pf.normalize<BITS>(p, c, (int)r);
-    if (lane == 0)
-      for (int d = 0; d < p.pf_dist && pf.l < L; ++d) {
-        prefetch_unit<BITS>(pf.g, pf.u);
-        pf.next<BITS>(p, c, (int)r);
-      }
-    uint32_t k = 0;
-    bool ok = true;
-    for (int l = 0; l < L && ok; ++l)
-      for (int ph = 0; ph < 4 && ok; ++ph) {
-        const Range g = units<BITS>(p, l, ph, c, (int)r);
-        const int ngroups = g.L->n_in / 64;
-        for (int u = g.u0; u < g.u1; ++u) {
-          const int slot = k % p.ring_stages;
-          int go = 1;
-          if (lane == 0) {
-            if (pf.l < L) {
-              prefetch_unit<BITS>(pf.g, pf.u);
-              pf.next<BITS>(p, c, (int)r);
-            }
-            if (k >= (uint32_t)p.ring_stages &&
-                !wait_phase<false, true>(&s.empty[slot], ((k / p.ring_stages) - 1) & 1, p.status, 53)) {
-              go = 0;
-            } else {
-              const int tile = u / g.nk, kc = u - tile * g.nk;
-              const int g0 = kc * Gm::kChunkGroups, gc = min(Gm::kChunkGroups, ngroups - g0);
-              const int cslabs = (gc + Gm::kGroupsPerSlab - 1) / Gm::kGroupsPerSlab;
-              const int hslabs = BITS == 3 ? (gc + 15) / 16 : 0;
-              uint8_t* st = s.ring + (size_t)slot * Gm::kStageBytes;
-              mbar_arrive_expect_tx(&s.full[slot], (uint32_t)((cslabs + hslabs + (gc + 31) / 32) * kSlab));
-              const int code_x0 = g0 * (BITS == 4 ? 32 : 16) / 8;
-              for (int q = 0; q < cslabs; ++q)
-                tma_load_2d(st + q * kSlab, &g.L->tm_codes, &s.full[slot], code_x0 + q * 16, tile * 32);
-              if (BITS == 3)
-                for (int q = 0; q < hslabs; ++q)
-                  tma_load_2d(st + (Gm::kCodeSlabs + q) * kSlab, &g.L->tm_hi, &s.full[slot], g0 + q * 16, tile * 32);
-              for (int q = 0; q < (gc + 31) / 32; ++q)
-                tma_load_2d(st + (Gm::kCodeSlabs + Gm::kHiSlabs + q) * kSlab, &g.L->tm_sz, &s.full[slot],
-                            g0 + q * 32, tile * 32);
-            }
-          }
-          ok = __shfl_sync(0xffffffffu, go, 0) != 0;
-          if (!ok) break;
-          ++k;  // k counts the stages issued so far
-        }
-      }
-    // drain: the copies still in flight must land before the CTA may exit (bounded, and
-    // not cut short by the abort word: these are this CTA's own copies)
-    if (lane == 0) {
-      const uint32_t nwait = k < (uint32_t)p.ring_stages ? k : (uint32_t)p.ring_stages;
-      for (uint32_t q = k - nwait; q < k; ++q)
-        wait_phase<false, true, false>(&s.full[q % p.ring_stages], (q / p.ring_stages) & 1, p.status, 54);
-    }
-    __syncwarp();
+    producer<BITS>(p, s, c, r, tid);
     cluster_sync_all();
     return;
   }
