@@ -88,7 +88,7 @@ def algorithmic_bytes_per_step(n_layers, batch=BATCH, bits=BITS):
 # reported only while those sources are unchanged.
 TRAFFIC_PER_BLOCK = {"bytes": {"fp32": 270_965_248 // 4, "int8": 258_862_848 // 4},
                      "sources_sha256_16": "a7a80626b48c905c"}
-KERNEL_SOURCES = ("decode.cu", "decode.h", "common.cuh", "gemv_core.cuh")
+KERNEL_SOURCES = ("decode.cu", "decode.h", "common.cuh", "gemv_core.cuh", "bfly_engine.cuh")
 
 
 def traffic_per_step(n_layers, angles="fp32"):

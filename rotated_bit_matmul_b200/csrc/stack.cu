@@ -288,10 +288,11 @@ void setup_fused(harp_stack_s* S) {
   if (const char* e = getenv("HARP_PF_DIST")) p.pf_dist = std::max(0, atoi(e));
   p.cooperative = 1;
   if (const char* e = getenv("HARP_COOPERATIVE")) p.cooperative = atoi(e) != 0;
-  // MLP blocks up to 512 wide: the chain runs where the block's last gate/up unit completes
-  // (one grid barrier less per block); HARP_MLP_TICKETS=0 keeps the barrier
-  p.mlp_tickets = wb <= 512 && F % 32 == 0;
-  if (const char* e = getenv("HARP_MLP_TICKETS")) p.mlp_tickets = p.mlp_tickets && atoi(e) != 0;
+  // HARP_MLP_TICKETS=1 (MLP blocks up to 512 wide): the chain runs where the block's last
+  // gate/up unit completes, one grid barrier less per block. Off by default: the chains then
+  // pile onto the CTAs that finish last, and the step measured slower than with the barrier.
+  p.mlp_tickets = 0;
+  if (const char* e = getenv("HARP_MLP_TICKETS")) p.mlp_tickets = wb <= 512 && F % 32 == 0 && atoi(e) != 0;
   int G = 0;
   cudaError_t e = dec::max_clusters(p, &G);
   if (e != cudaSuccess || G < 1)

@@ -2,9 +2,10 @@
 harp_create_layer_mr against the oracle's mr_linear_fwd, which is pinned on the CPU
 (exact change of basis, the all-radix-2 case equal to the radix-2 linear, its own codes).
 
-The widths are the pages' non-power-of-two cases: 11008 = 2^8 * 43 (Llama-2-7B FFN) and
-28672 = 2^12 * 7 (Llama-70B FFN), on the output side (gate/up) and the input side (down),
-plus a radix-8 Cayley side. Gates as for the radix-2 layers: rel-L2 2e-3 on the GEMV path
+The widths are the pages' non-power-of-two cases: 11008 = 2^8 * 43 (Llama-2-7B FFN) on the
+output side (gate/up) and the input side (down), a radix-7 side of 14336 = 2^11 * 7 (the
+70B FFN's 28672 = 2^12 * 7 exceeds the 16384 one mixed-radix row holds on the device), and
+radix-8 Cayley sides. Gates as for the radix-2 layers: rel-L2 2e-3 on the GEMV path
 (1 and 4 tokens) and on the tensor-core path (16 tokens).
 """
 import numpy as np
@@ -34,27 +35,31 @@ def _cuda():
 
 
 def _side(radices, seed):
+    """Seeded fp32 parameters, signs and one fp32 Gaussian per stage (the QR mixer's fixed
+    matrix; read only for radices that are not powers of two)."""
     rng = np.random.default_rng(seed)
     d = int(np.prod(radices))
-    npar = sum((d // b) * oracle.mr_param_count(b) for b in radices)
-    theta = rng.uniform(-0.05, 0.05, npar)
+    theta = rng.uniform(-0.05, 0.05, oracle.mr_theta_size(radices)).astype(np.float32)
     sign = (rng.integers(0, 2, d) * 2 - 1).astype(np.int8)
-    gauss = np.concatenate([rng.standard_normal(b * b) for b in radices]) if any(b & (b - 1) for b in radices) else None
-    return oracle.MixedRadixSide(radices, theta, sign, gauss)
+    gauss = [rng.standard_normal((b, b)).astype(np.float32) for b in radices]
+    return oracle.MixedRadixSide(radices, theta, sign, [g.astype(np.float64) for g in gauss])
 
 
 def _device_plan(side):
     from rotated_bit_matmul_b200 import HarpMixedRadix
     dev = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a)).to("cuda", dtype=dt)
+    flat = np.concatenate([np.asarray(g, np.float32).reshape(-1) for g in side.gauss])
     return HarpMixedRadix(side.radices, dev(side.theta, torch.float32), dev(side.sign, torch.int8),
-                          dev(side.gauss, torch.float32) if side.gauss is not None else None)
+                          dev(flat, torch.float32))
 
 
 CASES = [
-    # (n_out radices, n_in radices): gate/up of 7B, down of 7B, a 70B FFN side, radix-8 Cayley
+    # (n_out radices, n_in radices): gate/up of 7B (11008 = 2^8 * 43 out), down of 7B
+    # (11008 in), a radix-7 side (14336 = 2^11 * 7; 70B's 28672 = 2^12 * 7 is twice the
+    # 16384 the mixed-radix kernel holds per row), radix-8 Cayley sides
     ((2, 2, 2, 2, 2, 2, 2, 2, 43), (16, 16, 16)),
     ((16, 16, 16), (43, 2, 2, 2, 2, 2, 2, 2, 2)),
-    ((8, 8, 8, 8, 7), (8, 8, 8)),
+    ((8, 8, 8, 4, 7), (8, 8, 8)),
     ((8, 8, 8), (8, 8, 8)),
 ]
 
