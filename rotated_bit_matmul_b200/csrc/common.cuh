@@ -55,6 +55,10 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
 }
 
 // raises the barrier's expected transaction bytes without arriving
+// orders this thread's earlier generic-proxy accesses of shared memory before its later
+// async-proxy ones (a TMA load into a buffer that was just read)
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
 }
@@ -201,8 +205,10 @@ __device__ __forceinline__ float pow2f(int e) { return __int_as_float((e + 127) 
 // 2^e with max |v| 2^e in [2^14, 2^15), in dp2a pair order (and the 1-bit-plane order for
 // 3-bit codes); lane 0 writes the scale 2^-e and the fp32 group sum. A non-finite value
 // makes the group's scale and sum NaN.
+// key: the group's 16-byte chunks are stored at chunk ^ key (0: in order; a consumer that
+// keeps one group per lane swizzles them to spread its reads over the banks)
 __device__ __forceinline__ void prep_group(const float* v, int bits, int16_t* grp, int16_t* grp_hi, float* xs,
-                                           float* xsum, int lane) {
+                                           float* xsum, int lane, int key = 0) {
   const float v0 = v[2 * lane], v1 = v[2 * lane + 1];
   float amax = fmaxf(fabsf(v0), fabsf(v1));
   float sum = v0 + v1;
@@ -217,11 +223,12 @@ __device__ __forceinline__ void prep_group(const float* v, int bits, int16_t* gr
   const float sc = pow2f(ex);
   const int q0 = max(-32767, min(32767, __float2int_rn(v0 * sc)));
   const int q1 = max(-32767, min(32767, __float2int_rn(v1 * sc)));
-  grp[xq_pos_lo(bits, 2 * lane)] = (int16_t)q0;
-  grp[xq_pos_lo(bits, 2 * lane + 1)] = (int16_t)q1;
+  const int kx = key << 3;  // 8 int16 per chunk
+  grp[xq_pos_lo(bits, 2 * lane) ^ kx] = (int16_t)q0;
+  grp[xq_pos_lo(bits, 2 * lane + 1) ^ kx] = (int16_t)q1;
   if (bits == 3) {
-    grp_hi[xq_pos_hi(2 * lane)] = (int16_t)q0;
-    grp_hi[xq_pos_hi(2 * lane + 1)] = (int16_t)q1;
+    grp_hi[xq_pos_hi(2 * lane) ^ kx] = (int16_t)q0;
+    grp_hi[xq_pos_hi(2 * lane + 1) ^ kx] = (int16_t)q1;
   }
   if (lane == 0) {
     *xs = bad ? __int_as_float(0x7fc00000) : pow2f(-ex);

@@ -5,15 +5,16 @@
 // output butterfly) plus the glue; at batch 1 every launch is short and the
 // launch/ramp/drain overheads dominate. Here one kernel does the whole step:
 //
-//  * Weights never depend on activations, so a producer warp per CTA streams that
-//    CTA's share of every GEMV of the step, in order, with 2-D TMA tile loads (no
-//    multicast) into a ring of shared-memory stages, while the activation chain runs.
-//    A second cursor runs ahead of the ring and asks for the boxes of later units in L2
-//    (bulk tensor prefetch), so HBM keeps streaming while the chains run. A GEMV is cut
-//    into units of 32 output rows x 2048 input columns (split-K); each unit's partial
-//    sums go to a buffer the next chain adds up in a fixed order. The 16 consumer warps
-//    form two halves that take alternate units; the last warp of a half to finish a
-//    unit reduces it.
+//  * Weights never depend on activations, so each CTA streams its share of every GEMV of
+//    the step, in order, with 2-D TMA tile loads (no multicast) into a ring of
+//    shared-memory stages: the warp that finishes a stage's unit last issues the load
+//    that refills it, and asks for a later unit's boxes in L2 (bulk tensor prefetch), so
+//    HBM keeps streaming while the chains run. No warp is set aside for the loads: the
+//    16 warps leave each thread 128 registers. A GEMV is cut into units of 32 output
+//    rows x 2048 input columns (split-K); each unit's partial sums go to a buffer the
+//    next chain adds up in a fixed order. The warps form four quads that take the units
+//    in turn; a lane holds one group of 64 input columns, with its operand words in
+//    registers, for eight rows.
 //  * CTAs form clusters of 8. Each cluster computes the activation chain between two
 //    GEMVs itself (redundantly with the other clusters): a w-wide butterfly is spread
 //    over the 8 CTAs, w/8 elements each. Every consumer thread holds one (two when
@@ -84,9 +85,11 @@ struct Smem : EngCtx {
   float* misc;     // [0, 8) rms partials by source CTA, [8, 24) per-warp scratch
   int* won;        // [0]: count, then up to kMaxWon MLP blocks whose last unit this CTA completed
   int32_t* xq;     // GEMV operand: xq words, then xs [ng], then xsum [ng]
-  float* red;      // GEMV reduction scratch: ring_stages x 16 warps x 32 lanes
-  int* ucnt;       // per ring stage: warps of the half done with the unit
-  uint64_t *full, *empty;
+  float* red;      // GEMV row partials: 16 warps x 8 rows x 33 (32 lanes, padded)
+  int* ucnt;       // per ring stage: warps of the quad done with its unit
+  int* lastk;      // per ring stage: the last stage index issued into it (-1: none)
+  struct Plan* plan;
+  uint64_t* full;
 };
 
 __device__ __forceinline__ Smem carve(const Params& p, int stage_bytes) {
@@ -105,15 +108,18 @@ __device__ __forceinline__ Smem carve(const Params& p, int stage_bytes) {
   b += 4 * 32;
   s.won = reinterpret_cast<int*>(b);
   b += 4 * 32;
-  s.red = reinterpret_cast<float*>(b);
-  b += (size_t)4 * kCW * 32 * p.ring_stages;
-  s.ucnt = reinterpret_cast<int*>(b);
-  b += 4 * ((p.ring_stages + 3) & ~3);
   s.xq = reinterpret_cast<int32_t*>(b);
   b += p.xq_bytes;
+  s.red = reinterpret_cast<float*>(b);
+  b += 4 * kCW * 8 * 33;
+  s.ucnt = reinterpret_cast<int*>(b);
+  b += 4 * 16;
+  s.lastk = reinterpret_cast<int*>(b);
+  b += 4 * 16;
+  s.plan = reinterpret_cast<struct Plan*>(b);
+  b += 512;
   s.full = reinterpret_cast<uint64_t*>(b);
-  s.empty = s.full + p.ring_stages;
-  s.xbar = s.empty + p.ring_stages;
+  s.xbar = s.full + p.ring_stages;
   return s;
 }
 
@@ -154,7 +160,7 @@ __device__ bool prep_broadcast(const float (&v)[2], int n_in, int bits, Smem& sm
     const int j = warp / GPR, kk = warp - j * GPR;
     const int G = (j * M::E + (int)r * M::RUN + 64 * kk) >> 6;
     prep_group(sm.T + j * M::PAD + 64 * kk, bits, xq16 + (int64_t)G * 64, xq16 + n_in + (int64_t)G * 64, xsA + G,
-               xsumA + G, lane);
+               xsumA + G, lane, G & 7);
   }
   const int planes = bits == 3 ? 2 : 1;
   xch_begin(sm, x, (uint32_t)((kC - 1) * NGL * (128 * planes + 8)), ct);  // starts with a barrier: prep is done
@@ -373,7 +379,7 @@ __device__ __noinline__ void mlp_block_local(const Params& p, Smem& sm, const Li
   if (warp < (M::E >> 6)) {
     const int G = (int)(base >> 6) + warp;
     prep_group(sm.T + 64 * warp, p.bits, xq16 + (int64_t)G * 64, xq16 + n_in + (int64_t)G * 64, p.xs_down + G,
-               p.xsum_down + G, lane);
+               p.xsum_down + G, lane, G & 7);
   }
 }
 
@@ -442,17 +448,24 @@ __device__ __noinline__ bool mlp_block_cluster(const Params& p, Smem& sm, Xch& x
     const int j = warp / GPR, kk = warp - j * GPR;
     const int G = (int)((base + j * M::E + (int)r * M::RUN + 64 * kk) >> 6);
     prep_group(sm.T + j * M::PAD + 64 * kk, p.bits, xq16 + (int64_t)G * 64, xq16 + n_in + (int64_t)G * 64,
-               p.xs_down + G, p.xsum_down + G, lane);
+               p.xs_down + G, p.xsum_down + G, lane, G & 7);
   }
   return true;
 }
 
 // ------------------------------------------------------------------ GEMV work units
 // A unit is 32 output rows x one 2048-column chunk of one linear: exactly one ring stage.
+// Units are numbered chunk-major (u = kc * tiles + tile), so the consecutive units a CTA
+// takes mostly share their chunk of the operand.
 struct Range {
   const Lin* L;
   float* zp;  // partial sums [nk][n_out]
-  int nk, u0, u1;
+  int n_in, n_out;
+  int nk, nt, u0, u1;  // chunks, 32-row tiles, the CTA's units [u0, u1)
+  __device__ __forceinline__ void tk(int u, int& tile, int& kc) const {
+    kc = u / nt;
+    tile = u - kc * nt;
+  }
 };
 
 __device__ __forceinline__ int split(int n, int i, int parts) { return (int)(((int64_t)n * i) / parts); }
@@ -483,43 +496,23 @@ __device__ __forceinline__ Range units(const Params& p, int l, int ph, int c, in
     parts = p.G * kC;
     g.zp = ph == 1 ? p.zpo : p.zpd;
   }
-  g.nk = (g.L->n_in + FGeo<BITS>::kChunkCols - 1) / FGeo<BITS>::kChunkCols;
-  const int U = ((g.L->n_out + 31) / 32) * g.nk;
+  g.n_in = g.L->n_in;
+  g.n_out = g.L->n_out;
+  g.nk = (g.n_in + FGeo<BITS>::kChunkCols - 1) / FGeo<BITS>::kChunkCols;
+  g.nt = (g.n_out + 31) / 32;
+  const int U = g.nt * g.nk;
   g.u0 = split(U, i, parts);
   g.u1 = split(U, i + 1, parts);
   return g;
 }
 
-// Cursor over a CTA's units in consumer order (block, phase, unit), used to run the L2
-// prefetch ahead of the ring.
-struct UnitCursor {
-  int l, ph, u;
-  Range g;
-  template <int BITS>
-  __device__ __forceinline__ void normalize(const Params& p, int c, int r) {
-    while (l < p.L && u >= g.u1) {
-      if (++ph == 4) {
-        ph = 0;
-        ++l;
-      }
-      if (l >= p.L) return;
-      g = units<BITS>(p, l, ph, c, r);
-      u = g.u0;
-    }
-  }
-  template <int BITS>
-  __device__ __forceinline__ void next(const Params& p, int c, int r) {
-    ++u;
-    normalize<BITS>(p, c, r);
-  }
-};
-
 // the boxes of one unit, as the ring loads them, requested into L2
 template <int BITS>
 __device__ __forceinline__ void prefetch_unit(const Range& g, int u) {
   using Gm = FGeo<BITS>;
-  const int ngroups = g.L->n_in / 64;
-  const int tile = u / g.nk, kc = u - tile * g.nk;
+  const int ngroups = g.n_in / 64;
+  int tile, kc;
+  g.tk(u, tile, kc);
   const int g0 = kc * Gm::kChunkGroups, gc = min(Gm::kChunkGroups, ngroups - g0);
   const int cslabs = (gc + Gm::kGroupsPerSlab - 1) / Gm::kGroupsPerSlab;
   const int code_x0 = g0 * (BITS == 4 ? 32 : 16) / 8;
@@ -529,87 +522,261 @@ __device__ __forceinline__ void prefetch_unit(const Range& g, int u) {
   for (int q = 0; q < (gc + 31) / 32; ++q) tma_prefetch_l2_2d(&g.L->tm_sz, g0 + q * 32, tile * 32);
 }
 
+// ---------------- the weight ring. A CTA's units of the whole step form one sequence of
+// stages K = 0, 1, ... (block, phase, unit order); stage K lives in ring slot K % S. The
+// first S stages are issued at the start; after that, the consumer warp that completes a
+// slot's unit last issues stage K + S into it (and asks for stage K + pf_dist in L2), so no
+// warp is set aside for the loads and a slot is refilled the moment it is free.
+// The CTA's ranges of block 0 by phase, and how they move per block (the next block's
+// linears are 7 Lin further; q and k partials have a buffer per block): worked out once and
+// kept in shared memory, so finding a stage's unit chases no pointer in global memory.
+struct Plan {
+  Range r0[4];
+  long long zstride[4];  // partial-sum offset per block
+  int nb;                // the CTA's units per block
+};
+
+template <int BITS>
+__device__ __forceinline__ void make_plan(const Params& p, int c, int r, Plan& q) {
+  q.nb = 0;
+  for (int ph = 0; ph < 4; ++ph) {
+    q.r0[ph] = units<BITS>(p, 0, ph, c, r);
+    q.zstride[ph] = p.L > 1 ? units<BITS>(p, 1, ph, c, r).zp - q.r0[ph].zp : 0;
+    q.nb += q.r0[ph].u1 - q.r0[ph].u0;
+  }
+}
+
+__device__ __forceinline__ Range range_of(const Plan& q, int l, int ph) {
+  Range g = q.r0[ph];
+  g.L += 7 * l;
+  g.zp += (long long)l * q.zstride[ph];
+  return g;
+}
+
+// stage K -> its range and unit; false past the step's last stage
+__device__ __forceinline__ bool locate(const Params& p, const Plan& q, uint32_t K, Range& g, int& u) {
+  if (q.nb == 0) return false;
+  const int l = (int)(K / (uint32_t)q.nb);
+  if (l >= p.L) return false;
+  int rem = (int)(K - (uint32_t)l * (uint32_t)q.nb), ph = 0;
+  while (rem >= q.r0[ph].u1 - q.r0[ph].u0) {
+    rem -= q.r0[ph].u1 - q.r0[ph].u0;
+    ++ph;
+  }
+  g = range_of(q, l, ph);
+  u = g.u0 + rem;
+  return true;
+}
+
+// one lane: stage K into its slot (2-D TMA tile loads, no multicast, completing on the
+// slot's full barrier), then the L2 request for stage K + pf_dist
+template <int BITS>
+__device__ void issue_stage(const Params& p, Smem& s, uint32_t K) {
+  using Gm = FGeo<BITS>;
+  const Plan& q = *s.plan;
+  Range g;
+  int u;
+  if (locate(p, q, K, g, u)) {
+    const int slot = (int)(K % (uint32_t)p.ring_stages);
+    const int ngroups = g.n_in / 64;
+    int tile, kc;
+    g.tk(u, tile, kc);
+    const int g0 = kc * Gm::kChunkGroups, gc = min(Gm::kChunkGroups, ngroups - g0);
+    const int cslabs = (gc + Gm::kGroupsPerSlab - 1) / Gm::kGroupsPerSlab;
+    const int hslabs = BITS == 3 ? (gc + 15) / 16 : 0;
+    uint8_t* st = s.ring + (size_t)slot * Gm::kStageBytes;
+    s.lastk[slot] = (int)K;
+    fence_proxy_async();  // the slot's earlier contents were read through the generic proxy
+    mbar_arrive_expect_tx(&s.full[slot], (uint32_t)((cslabs + hslabs + (gc + 31) / 32) * kSlab));
+    const int code_x0 = g0 * (BITS == 4 ? 32 : 16) / 8;
+    for (int t = 0; t < cslabs; ++t)
+      tma_load_2d(st + t * kSlab, &g.L->tm_codes, &s.full[slot], code_x0 + t * 16, tile * 32);
+    if (BITS == 3)
+      for (int t = 0; t < hslabs; ++t)
+        tma_load_2d(st + (Gm::kCodeSlabs + t) * kSlab, &g.L->tm_hi, &s.full[slot], g0 + t * 16, tile * 32);
+    for (int t = 0; t < (gc + 31) / 32; ++t)
+      tma_load_2d(st + (Gm::kCodeSlabs + Gm::kHiSlabs + t) * kSlab, &g.L->tm_sz, &s.full[slot], g0 + t * 32,
+                  tile * 32);
+  }
+  if (p.pf_dist > 0 && locate(p, q, K + (uint32_t)p.pf_dist, g, u)) prefetch_unit<BITS>(g, u);
+}
+
 // ------------------------------------------------------------------ GEMV (consumer side)
-// The 16 consumer warps form two halves that take alternate units of the CTA's range,
-// so two units are in flight and each warp covers 4 groups of a unit; the last warp of a
-// half to finish a unit reduces its 8 per-warp partial rows and writes the unit's sums.
-constexpr int kHalf = kCW / 2;
+// The 16 consumer warps form four quads, and a CTA's units go to the quads in turn. In a
+// unit, warp w of the quad takes rows 8w..8w+7 and lane l the unit's group l (64 input
+// columns): the lane's operand words stay in registers for all its rows, and for the
+// warp's next unit too when that has the same chunk, so shared memory serves only the
+// codes and the scale/zero words. A warp's per-lane row partials go through its own
+// 8 x 32 scratch in shared memory: four lanes add up each row, in a fixed order.
+constexpr int kQuads = 4, kQuadWarps = kCW / kQuads, kRowsW = 32 / kQuadWarps;
+constexpr int kRedRow = 33;  // scratch row stride: the adders' reads hit 32 distinct banks
+
+// 16-byte chunk k of operand group G in shared memory (and in the down operand in global):
+// swizzled by G, so that lanes holding consecutive groups read distinct banks
+__device__ __forceinline__ int xq_chunk(int G, int k) { return (G << 3) | (k ^ (G & 7)); }
+
+// exact integer dot product of one row's group (codes of unit row `row`, group l of the
+// chunk) with the operand words x of that group; xh: the 1-bit plane's operand (3-bit)
+template <int BITS>
+__device__ __forceinline__ int row_dot(const uint8_t* st, int row, int l, const int4 (&x)[8], const int4* xh,
+                                       int G) {
+  using Gm = FGeo<BITS>;
+  if constexpr (BITS == 2 || BITS == 3) {
+    const uint4 cw = *reinterpret_cast<const uint4*>(swz(st + (l >> 3) * kSlab, row, l & 7));
+    const uint32_t wv[4] = {cw.x, cw.y, cw.z, cw.w};
+    int a0 = 0, a1 = 0, a2 = 0, a3 = 0, b0 = 0, b1 = 0, b2 = 0, b3 = 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int4 xa = x[2 * k], xb = x[2 * k + 1];
+      const uint32_t w = wv[k];
+      const uint32_t m0 = w & 0x03030303u, m1 = w & 0x0C0C0C0Cu, m2 = w & 0x30303030u, m3 = w & 0xC0C0C0C0u;
+      a0 = dp2a_lo(xa.x, m0, a0);
+      b0 = dp2a_hi(xa.y, m0, b0);
+      a1 = dp2a_lo(xa.z, m1, a1);
+      b1 = dp2a_hi(xa.w, m1, b1);
+      a2 = dp2a_lo(xb.x, m2, a2);
+      b2 = dp2a_hi(xb.y, m2, b2);
+      a3 = dp2a_lo(xb.z, m3, a3);
+      b3 = dp2a_hi(xb.w, m3, b3);
+    }
+    int acc = (a0 + b0) + ((a1 + b1) >> 2) + ((a2 + b2) >> 4) + ((a3 + b3) >> 6);  // exact shifts
+    if constexpr (BITS == 3) {
+      const int gh = l & 15;
+      const uint2 hw = *reinterpret_cast<const uint2*>(
+          swz(st + (Gm::kCodeSlabs + (l >> 4)) * kSlab, row, gh >> 1) + (gh & 1) * 8);
+      const uint32_t hv[2] = {hw.x, hw.y};
+      int h = 0;
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+#pragma unroll
+        for (int mm = 0; mm < 8; mm += 2) {
+          const int4 xa = xh[xq_chunk(G, 4 * k + mm / 2)];
+          const uint32_t ma = hv[k] & (0x01010101u << mm), mb = hv[k] & (0x01010101u << (mm + 1));
+          int ha = 0, hb = 0;
+          ha = dp2a_lo(xa.x, ma, ha);
+          ha = dp2a_hi(xa.y, ma, ha);
+          hb = dp2a_lo(xa.z, mb, hb);
+          hb = dp2a_hi(xa.w, mb, hb);
+          h += (ha >> mm) + (hb >> (mm + 1));
+        }
+      }
+      acc += 4 * h;
+    }
+    return acc;
+  } else {  // 4-bit: two 16-byte chunks per group, 8 codes per word
+    const uint8_t* slab = st + (l >> 2) * kSlab;
+    const int c0 = (l & 3) * 2;
+    const uint4 ca = *reinterpret_cast<const uint4*>(swz(slab, row, c0));
+    const uint4 cb = *reinterpret_cast<const uint4*>(swz(slab, row, c0 + 1));
+    const uint32_t wv[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
+    int lo = 0, hi = 0, lo2 = 0, hi2 = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int4 xa = x[k];
+      const uint32_t ml = wv[k] & 0x0F0F0F0Fu, mh = wv[k] & 0xF0F0F0F0u;
+      lo = dp2a_lo(xa.x, ml, lo);
+      lo2 = dp2a_hi(xa.y, ml, lo2);
+      hi = dp2a_lo(xa.z, mh, hi);
+      hi2 = dp2a_hi(xa.w, mh, hi2);
+    }
+    return (lo + lo2) + ((hi + hi2) >> 4);
+  }
+}
 
 // tickets: with MLP-block tickets in the gate/up phase, the per-block completion counters of
-// this block (else null); per_block: gate and up units of one MLP block
-template <int BITS>
+// this block (else null); per_block: (unit, warp) items of one MLP block's gate and up rows
+template <int BITS, bool TICKETS = false>
 __device__ __noinline__ bool run_units(const Params& p, Smem& s, const Range& g, uint32_t& kring, int ct,
                                           unsigned* tickets = nullptr, unsigned per_block = 0, int wb = 0) {
   using Gm = FGeo<BITS>;
+  static_assert(kRowsW == 8, "four lanes add up each of a warp's eight rows");
   const int warp = ct >> 5, lane = ct & 31;
-  const int hv = warp / kHalf, hw = warp - hv * kHalf;  // half, warp within the half
-  const int n_out = g.L->n_out, n_in = g.L->n_in, ngroups = n_in / 64;
+  const int quad = warp / kQuadWarps, qw = warp - quad * kQuadWarps;
+  const int n_out = g.n_out, n_in = g.n_in, ngroups = n_in / 64;
   const int words = BITS == 3 ? n_in : n_in / 2;
   const float* xsA = reinterpret_cast<const float*>(s.xq + words);
   const float* xsumA = xsA + ngroups;
+  const int4* xlo = reinterpret_cast<const int4*>(s.xq);
+  const int4* xhi = reinterpret_cast<const int4*>(s.xq + n_in / 2);
   const int nu = g.u1 - g.u0;
+  int4 xr[8];
+  float xs = 0.f, xsum = 0.f;
+  int kc_have = -1;
   bool ok = true;
-  for (int i = hv; i < nu; i += 2) {
+  float* red = s.red + warp * (kRowsW * kRedRow);
+  // unit i of the phase is the CTA's (kring + i)-th stage and goes to quad (kring + i) % 4
+  for (int i = (quad - (int)(kring & 3)) & 3; i < nu; i += kQuads) {
     const uint32_t kr = kring + (uint32_t)i;
     const int slot = kr % p.ring_stages;
-    const int u = g.u0 + i;
     if (ok) {
       int w = 1;
       if (lane == 0) w = wait_phase<false>(&s.full[slot], (kr / p.ring_stages) & 1, p.status, 52);
       ok = __shfl_sync(0xffffffffu, w, 0) != 0;
     }
-    const int tile = u / g.nk, kc = u - tile * g.nk, row0 = tile * 32;
+    int tile, kc;
+    g.tk(g.u0 + i, tile, kc);
     const int g0 = kc * Gm::kChunkGroups, gc = min(Gm::kChunkGroups, ngroups - g0);
-    float zacc = 0.f;
-    if (ok) {
-      const uint8_t* st = s.ring + (size_t)slot * Gm::kStageBytes;
-      const uint8_t* szs = st + (Gm::kCodeSlabs + Gm::kHiSlabs) * kSlab;
-      for (int gl = hw; gl < gc; gl += kHalf) {
-        const int gg = g0 + gl;
-        const uint32_t szw = sz_word(szs, lane, gl);
+    const bool act = lane < gc;
+    const int G = g0 + lane;
+    if (kc != kc_have) {
+      kc_have = kc;
+      if (act) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) xr[k] = xlo[xq_chunk(G, k)];
+        xs = xsA[G];
+        xsum = xsumA[G];
+      }
+    }
+    const uint8_t* st = s.ring + (size_t)slot * Gm::kStageBytes;
+    const uint8_t* szs = st + (Gm::kCodeSlabs + Gm::kHiSlabs) * kSlab;
+#pragma unroll 1
+    for (int rr = 0; rr < kRowsW; ++rr) {
+      const int row = qw * kRowsW + rr;
+      float z = 0.f;
+      if (ok && act) {
+        const uint32_t szw = sz_word(szs, row, lane);
         const float s16 = __half2float(__ushort_as_half((unsigned short)(szw & 0xffffu)));
         const float z16 = __half2float(__ushort_as_half((unsigned short)(szw >> 16)));
-        const int4* xg = reinterpret_cast<const int4*>(s.xq + (int64_t)gg * 32);
-        const int4* xgh = reinterpret_cast<const int4*>(s.xq + n_in / 2 + (int64_t)gg * 32);
-        const int acc = group_dot<BITS, true>(st, st + Gm::kCodeSlabs * kSlab, lane, gl, xg, xgh);
-        zacc = fmaf(s16, (float)acc * xsA[gg], fmaf(z16, xsumA[gg], zacc));
+        const int acc = row_dot<BITS>(st, row, lane, xr, xhi, G);
+        z = fmaf(s16, (float)acc * xs, z16 * xsum);
       }
+      red[rr * kRedRow + lane] = z;
     }
-    float* red = s.red + (size_t)slot * kCW * 32;
-    red[hw * 32 + lane] = zacc;
     __syncwarp();
-    int last = 0;
-    if (lane == 0) {
-      __threadfence_block();
-      last = atomicAdd(&s.ucnt[slot], 1) == kHalf - 1;
-    }
-    last = __shfl_sync(0xffffffffu, last, 0);
-    if (last) {
-      __threadfence_block();
-      float t = 0.f;
+    // row (lane >> 2) of the octet: lane & 3 adds lanes (lane & 3) * 8 .. + 7, then the quad
+    float t = 0.f;
+    {
+      const float* rp = red + (lane >> 2) * kRedRow + (lane & 3) * 8;
 #pragma unroll
-      for (int w = 0; w < kHalf; ++w) t += red[w * 32 + lane];
-      if (ok && row0 + lane < n_out) g.zp[(int64_t)kc * n_out + row0 + lane] = t;
-      if (tickets) {
-        // the partials are visible device-wide before the block's ticket counts them; the
-        // CTA that brings the count to per_block runs the block's chain after this phase
-        __threadfence();
-        __syncwarp();
-        if (lane == 0) {
-          const int blk = row0 / wb;
-          unsigned old;
-          asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(tickets + blk) : "memory");
-          if (old + 1 == per_block) {
-            const int i = atomicAdd(&s.won[0], 1);
-            if (i < kMaxWon) s.won[1 + i] = blk;
-          }
+      for (int k = 0; k < 8; ++k) t += rp[k];
+    }
+    t += __shfl_xor_sync(0xffffffffu, t, 1);
+    t += __shfl_xor_sync(0xffffffffu, t, 2);
+    __syncwarp();  // the scratch is free for the warp's next unit
+    const int rowo = tile * 32 + qw * kRowsW + (lane >> 2);
+    if (ok && (lane & 3) == 0 && rowo < n_out) g.zp[(int64_t)kc * n_out + rowo] = t;
+    if constexpr (TICKETS) {
+      // the partials are visible device-wide before the block's ticket counts them; the
+      // CTA that brings the count to per_block runs the block's chain after this phase
+      __threadfence();
+      __syncwarp();
+      if (lane == 0) {
+        const int blk = tile * 32 / wb;
+        unsigned old;
+        asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(tickets + blk) : "memory");
+        if (old + 1 == per_block) {
+          const int k = atomicAdd(&s.won[0], 1);
+          if (k < kMaxWon) s.won[1 + k] = blk;
         }
       }
-      __syncwarp();
-      if (lane == 0) s.ucnt[slot] = 0;
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&s.empty[slot]);
+    // the quad's last warp to finish (its reads of the slot all fed the sums above) refills it
+    if (lane == 0 && atomicAdd(&s.ucnt[slot], 1) == kQuadWarps - 1) {
+      s.ucnt[slot] = 0;
+      issue_stage<BITS>(p, s, kr + (uint32_t)p.ring_stages);
+    }
+    __syncwarp();
   }
   kring += (uint32_t)nu;
   return cbar_and(ok);
@@ -719,11 +886,6 @@ __device__ __forceinline__ void mlp_local_blk(const Params& p, Smem& sm, const L
 // P7 roles: MLP-block CTAs or clusters first, the last two clusters apply F_U_q / F_U_k
 __device__ __forceinline__ int qk_cluster(const Params& p, int which) { return p.G - 1 - which; }
 
-// ---------------- producer warp: the weight ring, every unit of the step in consumer
-// order. Every lane runs the same loop (the warp never diverges around a blocking wait);
-// lane 0 waits and issues. A second cursor runs p.pf_dist units ahead and asks for those
-// units' boxes in L2, so HBM keeps streaming while the chains run and the ring's copies are
-// served from L2.
 // L2 hint for this CTA's slice of a side's thread-order table (cluster layout: CTA r's
 // entries are contiguous) and of its sign vector
 __device__ __forceinline__ void prefetch_side(const uint8_t* rt, const int8_t* sign, int eb, int tm, uint32_t r) {
@@ -734,7 +896,8 @@ __device__ __forceinline__ void prefetch_side(const uint8_t* rt, const int8_t* s
   if (E % 16 == 0) bulk_prefetch_l2(sign + (size_t)r * E, (uint32_t)E);
 }
 
-// the tables of the chain that follows GEMV phase ph of block l (lane 0 of the producer)
+// the tables of the chain that follows GEMV phase ph of block l (one thread, as the phase
+// starts)
 __device__ __forceinline__ void prefetch_chain(const Params& p, int l, int ph, int c, uint32_t r) {
   const Lin* lin = p.lin + 7 * l;
   if (ph == 0) {  // P3: F_U of v, F_V of o
@@ -752,73 +915,6 @@ __device__ __forceinline__ void prefetch_chain(const Params& p, int l, int ph, i
   }
 }
 
-template <int BITS>
-__device__ __noinline__ void producer(const Params& p, Smem& s, int c, uint32_t r, int tid) {
-  using Gm = FGeo<BITS>;
-  const int L = p.L;
-  const int lane = tid & 31;
-  UnitCursor pf;
-  pf.l = 0;
-  pf.ph = 0;
-  pf.g = units<BITS>(p, 0, 0, c, (int)r);
-  pf.u = pf.g.u0;
-  pf.normalize<BITS>(p, c, (int)r);
-  if (lane == 0)
-    for (int d = 0; d < p.pf_dist && pf.l < L; ++d) {
-      prefetch_unit<BITS>(pf.g, pf.u);
-      pf.next<BITS>(p, c, (int)r);
-    }
-  uint32_t k = 0;
-  bool ok = true;
-  for (int l = 0; l < L && ok; ++l)
-    for (int ph = 0; ph < 4 && ok; ++ph) {
-      const Range g = units<BITS>(p, l, ph, c, (int)r);
-      const int ngroups = g.L->n_in / 64;
-      if (lane == 0 && p.tm != kTmHad) prefetch_chain(p, l, ph, c, r);
-      for (int u = g.u0; u < g.u1; ++u) {
-        const int slot = k % p.ring_stages;
-        int go = 1;
-        if (lane == 0) {
-          if (pf.l < L) {
-            prefetch_unit<BITS>(pf.g, pf.u);
-            pf.next<BITS>(p, c, (int)r);
-          }
-          if (k >= (uint32_t)p.ring_stages &&
-              !wait_phase<false, true>(&s.empty[slot], ((k / p.ring_stages) - 1) & 1, p.status, 53)) {
-            go = 0;
-          } else {
-            const int tile = u / g.nk, kc = u - tile * g.nk;
-            const int g0 = kc * Gm::kChunkGroups, gc = min(Gm::kChunkGroups, ngroups - g0);
-            const int cslabs = (gc + Gm::kGroupsPerSlab - 1) / Gm::kGroupsPerSlab;
-            const int hslabs = BITS == 3 ? (gc + 15) / 16 : 0;
-            uint8_t* st = s.ring + (size_t)slot * Gm::kStageBytes;
-            mbar_arrive_expect_tx(&s.full[slot], (uint32_t)((cslabs + hslabs + (gc + 31) / 32) * kSlab));
-            const int code_x0 = g0 * (BITS == 4 ? 32 : 16) / 8;
-            for (int q = 0; q < cslabs; ++q)
-              tma_load_2d(st + q * kSlab, &g.L->tm_codes, &s.full[slot], code_x0 + q * 16, tile * 32);
-            if (BITS == 3)
-              for (int q = 0; q < hslabs; ++q)
-                tma_load_2d(st + (Gm::kCodeSlabs + q) * kSlab, &g.L->tm_hi, &s.full[slot], g0 + q * 16, tile * 32);
-            for (int q = 0; q < (gc + 31) / 32; ++q)
-              tma_load_2d(st + (Gm::kCodeSlabs + Gm::kHiSlabs + q) * kSlab, &g.L->tm_sz, &s.full[slot],
-                          g0 + q * 32, tile * 32);
-          }
-        }
-        ok = __shfl_sync(0xffffffffu, go, 0) != 0;
-        if (!ok) break;
-        ++k;  // k counts the stages issued so far
-      }
-    }
-  // drain: the copies still in flight must land before the CTA may exit (bounded, and
-  // not cut short by the abort word: these are this CTA's own copies)
-  if (lane == 0) {
-    const uint32_t nwait = k < (uint32_t)p.ring_stages ? k : (uint32_t)p.ring_stages;
-    for (uint32_t q = k - nwait; q < k; ++q)
-      wait_phase<false, true, false>(&s.full[q % p.ring_stages], (q / p.ring_stages) & 1, p.status, 54);
-  }
-  __syncwarp();
-}
-
 // ------------------------------------------------------------------ the kernel
 // TM: how every butterfly of the stack keeps its angles (kTmCS, kTmHad, kTmQ8); each form
 // has its own instantiation, so no rotation branches on it.
@@ -831,28 +927,27 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   const int tid = threadIdx.x;
 
   if (tid == 0) {
+    make_plan<BITS>(p, c, (int)r, *s.plan);
     s_wait_cycles = p.wait_cycles;
     s.won[0] = 0;
     for (int i = 0; i < p.ring_stages; ++i) {
       mbar_init(&s.full[i], 1);
-      mbar_init(&s.empty[i], kHalf);  // the 8 warps of the half that consumed the unit
       s.ucnt[i] = 0;
+      s.lastk[i] = -1;
     }
     mbar_init(&s.xbar[0], 1);
     mbar_init(&s.xbar[1], 1);
     fence_mbar_init();
+    // the ring's first stages, after the L2 requests for those the refills will ask for
+    Range g;
+    int u;
+    for (int k = p.ring_stages; k < p.pf_dist; ++k)
+      if (locate(p, *s.plan, (uint32_t)k, g, u)) prefetch_unit<BITS>(g, u);
+    for (int k = 0; k < p.ring_stages; ++k) issue_stage<BITS>(p, s, (uint32_t)k);
   }
   cluster_sync_all();  // every CTA's barriers exist before any remote store signals one
 
   const int L = p.L;
-
-  if (tid >= kNT) {
-    producer<BITS>(p, s, c, r, tid);
-    cluster_sync_all();
-    return;
-  }
-
-  // ---------------- consumers
   const int ct = tid;
   uint32_t kring = 0;
   Xch X;
@@ -866,24 +961,26 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     if (!(ok = residual_any<TM>(p, s, X, res, prev ? prev + 6 : nullptr, p.zpd, p.nk_f, lin + p.asg_qkv[c], r,
                                 ct)))
       break;
-    // P2
-    if (!(ok = run_units<BITS>(p, s, units<BITS>(p, l, 0, c, (int)r), kring, ct))) break;
+    // P2 (L2 requests for the tables of the chain that follows, as every GEMV phase)
+    if (ct == 0 && p.tm != kTmHad) prefetch_chain(p, l, 0, c, r);
+    if (!(ok = run_units<BITS>(p, s, range_of(*s.plan, l, 0), kring, ct))) break;
     if (!(ok = grid_barrier(p, l * 5 + 0, ct))) break;
     // P3
     if (!(ok = p.eb_h == 10 ? attn_eb<TM, 10>(p, s, X, lin + 2, lin + 3, r, ct)
                             : attn_eb<TM, 9>(p, s, X, lin + 2, lin + 3, r, ct)))
       break;
     // P4
-    if (!(ok = run_units<BITS>(p, s, units<BITS>(p, l, 1, c, (int)r), kring, ct))) break;
+    if (ct == 0 && p.tm != kTmHad) prefetch_chain(p, l, 1, c, r);
+    if (!(ok = run_units<BITS>(p, s, range_of(*s.plan, l, 1), kring, ct))) break;
     if (!(ok = grid_barrier(p, l * 5 + 1, ct))) break;
     // P5
     if (!(ok = residual_any<TM>(p, s, X, res, lin + 3, p.zpo, p.nk_h, lin + 4 + p.asg_gu[c], r, ct))) break;
     // P6
     if (p.mlp_tickets) {
       const int wb = lin[4].w_out;
-      const unsigned per_block = (unsigned)(2 * (wb / 32) * p.nk_h);
+      const unsigned per_block = (unsigned)(2 * (wb / 32) * p.nk_h * kQuadWarps);
       unsigned* tickets = p.counters + 5 * L + (size_t)l * p.nblocks;
-      if (!(ok = run_units<BITS>(p, s, units<BITS>(p, l, 2, c, (int)r), kring, ct, tickets, per_block, wb))) break;
+      if (!(ok = run_units<BITS, true>(p, s, range_of(*s.plan, l, 2), kring, ct, tickets, per_block, wb))) break;
       // P7 for the MLP blocks this CTA completed (their partials are all written)
       const int nw = min(s.won[0], kMaxWon);
       if (s.won[0] > kMaxWon) report(p.status, 6, 70);  // cannot happen: a CTA's units span few blocks
@@ -891,7 +988,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       cbar();
       if (ct == 0) s.won[0] = 0;
     } else {
-      if (!(ok = run_units<BITS>(p, s, units<BITS>(p, l, 2, c, (int)r), kring, ct))) break;
+      if (!(ok = run_units<BITS>(p, s, range_of(*s.plan, l, 2), kring, ct))) break;
       if (!(ok = grid_barrier(p, l * 5 + 2, ct))) break;
       // P7
       if (!(ok = mlp_any<TM>(p, s, X, lin, c, r, ct))) break;
@@ -919,7 +1016,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         xsA[ng + g] = __ldcg(p.xsum_down + g);
       }
       cbar();
-      if (!(ok = run_units<BITS>(p, s, units<BITS>(p, l, 3, c, (int)r), kring, ct))) break;
+      if (ct == 0 && p.tm != kTmHad) prefetch_chain(p, l, 3, c, r);
+      if (!(ok = run_units<BITS>(p, s, range_of(*s.plan, l, 3), kring, ct))) break;
     }
     if (!(ok = grid_barrier(p, l * 5 + 4, ct))) break;
   }
@@ -937,6 +1035,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       }
     }
   }
+  // copies still in flight (a step that ended early) land before the CTA exits: bounded,
+  // and not cut short by the abort word, since these are this CTA's own copies
+  if (ct == 0)
+    for (int i = 0; i < p.ring_stages; ++i)
+      if (s.lastk[i] >= 0)
+        wait_phase<false, true, false>(&s.full[i], ((uint32_t)s.lastk[i] / (uint32_t)p.ring_stages) & 1, p.status,
+                                       54);
   cluster_sync_all();
 }
 
@@ -976,8 +1081,7 @@ cudaError_t repack_side(int tm, int eb, bool cluster, int nblk, const uint8_t* t
 template <int BITS>
 size_t smem_bytes(const Params& p) {
   return 1024 + (size_t)p.ring_stages * FGeo<BITS>::kStageBytes + 3 * 4 * (size_t)kRxFloats + 4 * 32 + 4 * 32 +
-         (size_t)4 * kCW * 32 * p.ring_stages + 4 * ((p.ring_stages + 3) & ~3) + p.xq_bytes +
-         8 * (2 * (size_t)p.ring_stages + 2);
+         p.xq_bytes + 4 * kCW * 8 * 33 + 2 * 4 * 16 + 512 + 8 * ((size_t)p.ring_stages + 2);
 }
 
 template <int BITS>

@@ -11,7 +11,7 @@ namespace dec {
 constexpr int kC = 8;                // CTAs per cluster
 constexpr int kCW = 16;              // consumer warps per CTA
 constexpr int kNT = 32 * kCW;        // consumer threads
-constexpr int kThreads = kNT + 32;   // + the weight-ring producer warp
+constexpr int kThreads = kNT;        // every warp consumes; the ring is refilled by them
 constexpr int kMaxClusters = 64;
 
 // How the butterflies of a fused stack keep their angles (one kernel instantiation each):
