@@ -5,16 +5,14 @@
 // output butterfly) plus the glue; at batch 1 every launch is short and the
 // launch/ramp/drain overheads dominate. Here one kernel does the whole step:
 //
-//  * Weights never depend on activations, so each CTA streams its share of every GEMV of
-//    the step, in order, with 2-D TMA tile loads (no multicast) into a ring of
-//    shared-memory stages: the warp that finishes a stage's unit last issues the load
-//    that refills it, and asks for a later unit's boxes in L2 (bulk tensor prefetch), so
-//    HBM keeps streaming while the chains run. No warp is set aside for the loads: the
-//    16 warps leave each thread 128 registers. A GEMV is cut into units of 32 output
-//    rows x 2048 input columns (split-K); each unit's partial sums go to a buffer the
-//    next chain adds up in a fixed order. The warps form four quads that take the units
-//    in turn; a lane holds one group of 64 input columns, with its operand words in
-//    registers, for eight rows.
+//  * Weights never depend on activations, so as each GEMV phase starts, every warp asks
+//    for its rows of the next phase's weights in L2 (plain per-lane line prefetches), and
+//    HBM streams them while the chains run. A GEMV is cut into units of 32 output rows x
+//    2048 input columns (split-K); each unit's partial sums go to a buffer the next chain
+//    adds up in a fixed order. The 16 warps form four quads that take the units in turn;
+//    a lane holds one group of 64 input columns, with its operand words in registers, for
+//    eight rows, and loads that group's codes and scale/zero words of those rows straight
+//    from L2 (a warp reads each row's chunk as one contiguous span).
 //  * CTAs form clusters of 8. Each cluster computes the activation chain between two
 //    GEMVs itself (redundantly with the other clusters): a w-wide butterfly is spread
 //    over the 8 CTAs, w/8 elements each. Every consumer thread holds one (two when
@@ -64,40 +62,30 @@ namespace dec {
 using namespace gemv_core;
 
 // ------------------------------------------------------------------ GEMV unit geometry
-// 32 output rows x 2048 input columns per unit and ring stage (20 / 28 / 36 KB of codes
-// and scale/zero at 2 / 3 / 4 bits).
+// 32 output rows x 2048 input columns (one group of 64 columns per lane) per unit.
 template <int BITS>
 struct FGeo {
   static constexpr int kChunkCols = 2048;
   static constexpr int kChunkGroups = kChunkCols / 64;
-  static constexpr int kGroupsPerSlab = BITS == 4 ? 4 : 8;
-  static constexpr int kCodeSlabs = kChunkGroups / kGroupsPerSlab;
-  static constexpr int kHiSlabs = BITS == 3 ? kChunkGroups / 16 : 0;
-  static constexpr int kSzSlabs = 1;
-  static constexpr int kStageBytes = (kCodeSlabs + kHiSlabs + kSzSlabs) * kSlab;
+  static constexpr int kGroupBytes = BITS == 4 ? 32 : 16;  // a group's codes (first plane)
+  static constexpr int kRowBatch = 4;  // rows whose loads are in flight at once
 };
 
 // ------------------------------------------------------------------ shared memory carve-up
 constexpr int kMaxWon = 16;  // MLP blocks one CTA can complete in a block's gate/up phase
 
 struct Smem : EngCtx {
-  uint8_t* ring;
   float* misc;     // [0, 8) rms partials by source CTA, [8, 24) per-warp scratch
   int* won;        // [0]: count, then up to kMaxWon MLP blocks whose last unit this CTA completed
   int32_t* xq;     // GEMV operand: xq words, then xs [ng], then xsum [ng]
   float* red;      // GEMV row partials: 16 warps x 8 rows x 33 (32 lanes, padded)
-  int* ucnt;       // per ring stage: warps of the quad done with its unit
-  int* lastk;      // per ring stage: the last stage index issued into it (-1: none)
   struct Plan* plan;
-  uint64_t* full;
 };
 
-__device__ __forceinline__ Smem carve(const Params& p, int stage_bytes) {
+__device__ __forceinline__ Smem carve(const Params& p) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* b = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* b = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 15) & ~uintptr_t(15));
   Smem s;
-  s.ring = b;
-  b += (size_t)p.ring_stages * stage_bytes;
   s.T = reinterpret_cast<float*>(b);
   b += 4 * kRxFloats;
   s.rx[0] = reinterpret_cast<float*>(b);
@@ -112,14 +100,9 @@ __device__ __forceinline__ Smem carve(const Params& p, int stage_bytes) {
   b += p.xq_bytes;
   s.red = reinterpret_cast<float*>(b);
   b += 4 * kCW * 8 * 33;
-  s.ucnt = reinterpret_cast<int*>(b);
-  b += 4 * 16;
-  s.lastk = reinterpret_cast<int*>(b);
-  b += 4 * 16;
   s.plan = reinterpret_cast<struct Plan*>(b);
   b += 512;
-  s.full = reinterpret_cast<uint64_t*>(b);
-  s.xbar = s.full + p.ring_stages;
+  s.xbar = reinterpret_cast<uint64_t*>(b);
   return s;
 }
 
@@ -454,7 +437,7 @@ __device__ __noinline__ bool mlp_block_cluster(const Params& p, Smem& sm, Xch& x
 }
 
 // ------------------------------------------------------------------ GEMV work units
-// A unit is 32 output rows x one 2048-column chunk of one linear: exactly one ring stage.
+// A unit is 32 output rows x one 2048-column chunk of one linear.
 // Units are numbered chunk-major (u = kc * tiles + tile), so the consecutive units a CTA
 // takes mostly share their chunk of the operand.
 struct Range {
@@ -506,30 +489,35 @@ __device__ __forceinline__ Range units(const Params& p, int l, int ph, int c, in
   return g;
 }
 
-// the boxes of one unit, as the ring loads them, requested into L2
-template <int BITS>
-__device__ __forceinline__ void prefetch_unit(const Range& g, int u) {
-  using Gm = FGeo<BITS>;
-  const int ngroups = g.n_in / 64;
-  int tile, kc;
-  g.tk(u, tile, kc);
-  const int g0 = kc * Gm::kChunkGroups, gc = min(Gm::kChunkGroups, ngroups - g0);
-  const int cslabs = (gc + Gm::kGroupsPerSlab - 1) / Gm::kGroupsPerSlab;
-  const int code_x0 = g0 * (BITS == 4 ? 32 : 16) / 8;
-  for (int q = 0; q < cslabs; ++q) tma_prefetch_l2_2d(&g.L->tm_codes, code_x0 + q * 16, tile * 32);
-  if (BITS == 3)
-    for (int q = 0; q < (gc + 15) / 16; ++q) tma_prefetch_l2_2d(&g.L->tm_hi, g0 + q * 16, tile * 32);
-  for (int q = 0; q < (gc + 31) / 32; ++q) tma_prefetch_l2_2d(&g.L->tm_sz, g0 + q * 32, tile * 32);
+__device__ __forceinline__ void prefetch_line_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
-// ---------------- the weight ring. A CTA's units of the whole step form one sequence of
-// stages K = 0, 1, ... (block, phase, unit order); stage K lives in ring slot K % S. The
-// first S stages are issued at the start; after that, the consumer warp that completes a
-// slot's unit last issues stage K + S into it (and asks for stage K + pf_dist in L2), so no
-// warp is set aside for the loads and a slot is refilled the moment it is free.
+// L2 requests for this warp's rows of its units in range g (the units of a phase go to the
+// quads in turn from quad k0 % 4): lane l asks for 128-byte line l % 4 (and + 4, ...) of
+// row l / 4's codes and 1-bit plane in the chunk, lanes 0, 4, ... for its scale/zero words.
+// Plain prefetches from every lane: nothing queues behind the TMA unit.
+template <int BITS>
+__device__ __forceinline__ void prefetch_rows(const Range& g, uint32_t k0, int quad, int qw, int lane) {
+  using Gm = FGeo<BITS>;
+  const int ngroups = g.n_in / 64, row_bytes = ngroups * Gm::kGroupBytes;
+  const int line = lane & 3;
+  for (int i = (quad - (int)(k0 & 3)) & 3; i < g.u1 - g.u0; i += 4) {
+    int tile, kc;
+    g.tk(g.u0 + i, tile, kc);
+    const int row = tile * 32 + qw * 8 + (lane >> 2);
+    if (row >= g.n_out) continue;
+    const int g0 = kc * Gm::kChunkGroups, gc = min(Gm::kChunkGroups, ngroups - g0);
+    const uint8_t* cb = g.L->codes + (size_t)row * row_bytes + (size_t)g0 * Gm::kGroupBytes;
+    for (int o = line * 128; o < gc * Gm::kGroupBytes; o += 512) prefetch_line_l2(cb + o);
+    if (BITS == 3 && line * 128 < gc * 8) prefetch_line_l2(g.L->hi + (size_t)row * (ngroups * 8) + (size_t)g0 * 8 + line * 128);
+    if (line == 0) prefetch_line_l2(g.L->sz + (size_t)row * ngroups + g0);
+  }
+}
+
 // The CTA's ranges of block 0 by phase, and how they move per block (the next block's
 // linears are 7 Lin further; q and k partials have a buffer per block): worked out once and
-// kept in shared memory, so finding a stage's unit chases no pointer in global memory.
+// kept in shared memory, so finding a unit chases no pointer in global memory.
 struct Plan {
   Range r0[4];
   long long zstride[4];  // partial-sum offset per block
@@ -553,61 +541,16 @@ __device__ __forceinline__ Range range_of(const Plan& q, int l, int ph) {
   return g;
 }
 
-// stage K -> its range and unit; false past the step's last stage
-__device__ __forceinline__ bool locate(const Params& p, const Plan& q, uint32_t K, Range& g, int& u) {
-  if (q.nb == 0) return false;
-  const int l = (int)(K / (uint32_t)q.nb);
-  if (l >= p.L) return false;
-  int rem = (int)(K - (uint32_t)l * (uint32_t)q.nb), ph = 0;
-  while (rem >= q.r0[ph].u1 - q.r0[ph].u0) {
-    rem -= q.r0[ph].u1 - q.r0[ph].u0;
-    ++ph;
-  }
-  g = range_of(q, l, ph);
-  u = g.u0 + rem;
-  return true;
-}
-
-// one lane: stage K into its slot (2-D TMA tile loads, no multicast, completing on the
-// slot's full barrier), then the L2 request for stage K + pf_dist
-template <int BITS>
-__device__ void issue_stage(const Params& p, Smem& s, uint32_t K) {
-  using Gm = FGeo<BITS>;
-  const Plan& q = *s.plan;
-  Range g;
-  int u;
-  if (locate(p, q, K, g, u)) {
-    const int slot = (int)(K % (uint32_t)p.ring_stages);
-    const int ngroups = g.n_in / 64;
-    int tile, kc;
-    g.tk(u, tile, kc);
-    const int g0 = kc * Gm::kChunkGroups, gc = min(Gm::kChunkGroups, ngroups - g0);
-    const int cslabs = (gc + Gm::kGroupsPerSlab - 1) / Gm::kGroupsPerSlab;
-    const int hslabs = BITS == 3 ? (gc + 15) / 16 : 0;
-    uint8_t* st = s.ring + (size_t)slot * Gm::kStageBytes;
-    s.lastk[slot] = (int)K;
-    fence_proxy_async();  // the slot's earlier contents were read through the generic proxy
-    mbar_arrive_expect_tx(&s.full[slot], (uint32_t)((cslabs + hslabs + (gc + 31) / 32) * kSlab));
-    const int code_x0 = g0 * (BITS == 4 ? 32 : 16) / 8;
-    for (int t = 0; t < cslabs; ++t)
-      tma_load_2d(st + t * kSlab, &g.L->tm_codes, &s.full[slot], code_x0 + t * 16, tile * 32);
-    if (BITS == 3)
-      for (int t = 0; t < hslabs; ++t)
-        tma_load_2d(st + (Gm::kCodeSlabs + t) * kSlab, &g.L->tm_hi, &s.full[slot], g0 + t * 16, tile * 32);
-    for (int t = 0; t < (gc + 31) / 32; ++t)
-      tma_load_2d(st + (Gm::kCodeSlabs + Gm::kHiSlabs + t) * kSlab, &g.L->tm_sz, &s.full[slot], g0 + t * 32,
-                  tile * 32);
-  }
-  if (p.pf_dist > 0 && locate(p, q, K + (uint32_t)p.pf_dist, g, u)) prefetch_unit<BITS>(g, u);
-}
-
-// ------------------------------------------------------------------ GEMV (consumer side)
-// The 16 consumer warps form four quads, and a CTA's units go to the quads in turn. In a
-// unit, warp w of the quad takes rows 8w..8w+7 and lane l the unit's group l (64 input
-// columns): the lane's operand words stay in registers for all its rows, and for the
-// warp's next unit too when that has the same chunk, so shared memory serves only the
-// codes and the scale/zero words. A warp's per-lane row partials go through its own
-// 8 x 32 scratch in shared memory: four lanes add up each row, in a fixed order.
+// ------------------------------------------------------------------ GEMV
+// The 16 warps form four quads, and a CTA's units go to the quads in turn. In a unit, warp
+// w of the quad takes rows 8w..8w+7 and lane l the unit's group l (64 input columns). The
+// lane loads its own bytes of every row straight from global memory (a warp reads each
+// row's chunk as one contiguous, coalesced span; the phase's weights were requested into
+// L2 a phase earlier), with a batch of rows in flight at once, and keeps its operand words
+// in registers for all its rows, and for the warp's next unit too when that has the same
+// chunk. No data passes between warps but the row sums: a warp's per-lane partials go
+// through its own 8 x 32 scratch in shared memory, and four lanes add up each row, in a
+// fixed order.
 constexpr int kQuads = 4, kQuadWarps = kCW / kQuads, kRowsW = 32 / kQuadWarps;
 constexpr int kRedRow = 33;  // scratch row stride: the adders' reads hit 32 distinct banks
 
@@ -615,15 +558,31 @@ constexpr int kRedRow = 33;  // scratch row stride: the adders' reads hit 32 dis
 // swizzled by G, so that lanes holding consecutive groups read distinct banks
 __device__ __forceinline__ int xq_chunk(int G, int k) { return (G << 3) | (k ^ (G & 7)); }
 
-// exact integer dot product of one row's group (codes of unit row `row`, group l of the
-// chunk) with the operand words x of that group; xh: the 1-bit plane's operand (3-bit)
+// one row's data for one lane: the group's codes (first plane), its 1-bit plane (3-bit)
+// and its scale/zero word
 template <int BITS>
-__device__ __forceinline__ int row_dot(const uint8_t* st, int row, int l, const int4 (&x)[8], const int4* xh,
-                                       int G) {
+struct RowW {
+  uint4 c[BITS == 4 ? 2 : 1];
+  uint2 h;
+  uint32_t sz;
+};
+
+template <int BITS>
+__device__ __forceinline__ void load_row(RowW<BITS>& w, const Range& g, int row, int G, int ngroups) {
   using Gm = FGeo<BITS>;
+  const uint4* cp = reinterpret_cast<const uint4*>(g.L->codes + ((size_t)row * ngroups + G) * Gm::kGroupBytes);
+  w.c[0] = ldg_nc_u4(cp);
+  if constexpr (BITS == 4) w.c[1] = ldg_nc_u4(cp + 1);
+  if constexpr (BITS == 3) w.h = ldg_nc_u2(reinterpret_cast<const uint2*>(g.L->hi + ((size_t)row * ngroups + G) * 8));
+  w.sz = ldg_nc_u32(g.L->sz + (size_t)row * ngroups + G);
+}
+
+// exact integer dot product of one row's group with the operand words x of that group;
+// xh: the 1-bit plane's operand (3-bit)
+template <int BITS>
+__device__ __forceinline__ int row_dot(const RowW<BITS>& rw, const int4 (&x)[8], const int4* xh, int G) {
   if constexpr (BITS == 2 || BITS == 3) {
-    const uint4 cw = *reinterpret_cast<const uint4*>(swz(st + (l >> 3) * kSlab, row, l & 7));
-    const uint32_t wv[4] = {cw.x, cw.y, cw.z, cw.w};
+    const uint32_t wv[4] = {rw.c[0].x, rw.c[0].y, rw.c[0].z, rw.c[0].w};
     int a0 = 0, a1 = 0, a2 = 0, a3 = 0, b0 = 0, b1 = 0, b2 = 0, b3 = 0;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -641,10 +600,7 @@ __device__ __forceinline__ int row_dot(const uint8_t* st, int row, int l, const 
     }
     int acc = (a0 + b0) + ((a1 + b1) >> 2) + ((a2 + b2) >> 4) + ((a3 + b3) >> 6);  // exact shifts
     if constexpr (BITS == 3) {
-      const int gh = l & 15;
-      const uint2 hw = *reinterpret_cast<const uint2*>(
-          swz(st + (Gm::kCodeSlabs + (l >> 4)) * kSlab, row, gh >> 1) + (gh & 1) * 8);
-      const uint32_t hv[2] = {hw.x, hw.y};
+      const uint32_t hv[2] = {rw.h.x, rw.h.y};
       int h = 0;
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
@@ -664,11 +620,7 @@ __device__ __forceinline__ int row_dot(const uint8_t* st, int row, int l, const 
     }
     return acc;
   } else {  // 4-bit: two 16-byte chunks per group, 8 codes per word
-    const uint8_t* slab = st + (l >> 2) * kSlab;
-    const int c0 = (l & 3) * 2;
-    const uint4 ca = *reinterpret_cast<const uint4*>(swz(slab, row, c0));
-    const uint4 cb = *reinterpret_cast<const uint4*>(swz(slab, row, c0 + 1));
-    const uint32_t wv[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
+    const uint32_t wv[8] = {rw.c[0].x, rw.c[0].y, rw.c[0].z, rw.c[0].w, rw.c[1].x, rw.c[1].y, rw.c[1].z, rw.c[1].w};
     int lo = 0, hi = 0, lo2 = 0, hi2 = 0;
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
@@ -684,11 +636,12 @@ __device__ __forceinline__ int row_dot(const uint8_t* st, int row, int l, const 
 }
 
 // tickets: with MLP-block tickets in the gate/up phase, the per-block completion counters of
-// this block (else null); per_block: (unit, warp) items of one MLP block's gate and up rows
+// this block; per_block: (unit, warp) items of one MLP block's gate and up rows
 template <int BITS, bool TICKETS = false>
 __device__ __noinline__ bool run_units(const Params& p, Smem& s, const Range& g, uint32_t& kring, int ct,
                                           unsigned* tickets = nullptr, unsigned per_block = 0, int wb = 0) {
   using Gm = FGeo<BITS>;
+  constexpr int RB = Gm::kRowBatch;
   static_assert(kRowsW == 8, "four lanes add up each of a warp's eight rows");
   const int warp = ct >> 5, lane = ct & 31;
   const int quad = warp / kQuadWarps, qw = warp - quad * kQuadWarps;
@@ -702,22 +655,15 @@ __device__ __noinline__ bool run_units(const Params& p, Smem& s, const Range& g,
   int4 xr[8];
   float xs = 0.f, xsum = 0.f;
   int kc_have = -1;
-  bool ok = true;
   float* red = s.red + warp * (kRowsW * kRedRow);
-  // unit i of the phase is the CTA's (kring + i)-th stage and goes to quad (kring + i) % 4
+  // unit i of the phase is the CTA's (kring + i)-th and goes to quad (kring + i) % 4
   for (int i = (quad - (int)(kring & 3)) & 3; i < nu; i += kQuads) {
-    const uint32_t kr = kring + (uint32_t)i;
-    const int slot = kr % p.ring_stages;
-    if (ok) {
-      int w = 1;
-      if (lane == 0) w = wait_phase<false>(&s.full[slot], (kr / p.ring_stages) & 1, p.status, 52);
-      ok = __shfl_sync(0xffffffffu, w, 0) != 0;
-    }
     int tile, kc;
     g.tk(g.u0 + i, tile, kc);
     const int g0 = kc * Gm::kChunkGroups, gc = min(Gm::kChunkGroups, ngroups - g0);
     const bool act = lane < gc;
     const int G = g0 + lane;
+    const int row0 = tile * 32 + qw * kRowsW;
     if (kc != kc_have) {
       kc_have = kc;
       if (act) {
@@ -727,20 +673,23 @@ __device__ __noinline__ bool run_units(const Params& p, Smem& s, const Range& g,
         xsum = xsumA[G];
       }
     }
-    const uint8_t* st = s.ring + (size_t)slot * Gm::kStageBytes;
-    const uint8_t* szs = st + (Gm::kCodeSlabs + Gm::kHiSlabs) * kSlab;
 #pragma unroll 1
-    for (int rr = 0; rr < kRowsW; ++rr) {
-      const int row = qw * kRowsW + rr;
-      float z = 0.f;
-      if (ok && act) {
-        const uint32_t szw = sz_word(szs, row, lane);
-        const float s16 = __half2float(__ushort_as_half((unsigned short)(szw & 0xffffu)));
-        const float z16 = __half2float(__ushort_as_half((unsigned short)(szw >> 16)));
-        const int acc = row_dot<BITS>(st, row, lane, xr, xhi, G);
-        z = fmaf(s16, (float)acc * xs, z16 * xsum);
+    for (int rb = 0; rb < kRowsW; rb += RB) {
+      RowW<BITS> w[RB];
+#pragma unroll
+      for (int j = 0; j < RB; ++j)
+        if (act && row0 + rb + j < n_out) load_row<BITS>(w[j], g, row0 + rb + j, G, ngroups);
+#pragma unroll
+      for (int j = 0; j < RB; ++j) {
+        float z = 0.f;
+        if (act && row0 + rb + j < n_out) {
+          const float s16 = __half2float(__ushort_as_half((unsigned short)(w[j].sz & 0xffffu)));
+          const float z16 = __half2float(__ushort_as_half((unsigned short)(w[j].sz >> 16)));
+          const int acc = row_dot<BITS>(w[j], xr, xhi, G);
+          z = fmaf(s16, (float)acc * xs, z16 * xsum);
+        }
+        red[(rb + j) * kRedRow + lane] = z;
       }
-      red[rr * kRedRow + lane] = z;
     }
     __syncwarp();
     // row (lane >> 2) of the octet: lane & 3 adds lanes (lane & 3) * 8 .. + 7, then the quad
@@ -753,8 +702,8 @@ __device__ __noinline__ bool run_units(const Params& p, Smem& s, const Range& g,
     t += __shfl_xor_sync(0xffffffffu, t, 1);
     t += __shfl_xor_sync(0xffffffffu, t, 2);
     __syncwarp();  // the scratch is free for the warp's next unit
-    const int rowo = tile * 32 + qw * kRowsW + (lane >> 2);
-    if (ok && (lane & 3) == 0 && rowo < n_out) g.zp[(int64_t)kc * n_out + rowo] = t;
+    const int rowo = row0 + (lane >> 2);
+    if ((lane & 3) == 0 && rowo < n_out) g.zp[(int64_t)kc * n_out + rowo] = t;
     if constexpr (TICKETS) {
       // the partials are visible device-wide before the block's ticket counts them; the
       // CTA that brings the count to per_block runs the block's chain after this phase
@@ -770,16 +719,24 @@ __device__ __noinline__ bool run_units(const Params& p, Smem& s, const Range& g,
         }
       }
     }
-    __syncwarp();
-    // the quad's last warp to finish (its reads of the slot all fed the sums above) refills it
-    if (lane == 0 && atomicAdd(&s.ucnt[slot], 1) == kQuadWarps - 1) {
-      s.ucnt[slot] = 0;
-      issue_stage<BITS>(p, s, kr + (uint32_t)p.ring_stages);
-    }
-    __syncwarp();
   }
   kring += (uint32_t)nu;
-  return cbar_and(ok);
+  return cbar_and(true);
+}
+
+// as GEMV phase ph of block l starts (its first unit is the CTA's kring-th): this
+// warp's rows of the following phase into L2
+template <int BITS>
+__device__ __forceinline__ void prefetch_next(const Params& p, Smem& s, int l, int ph, uint32_t kring, int ct) {
+  if (p.pf_dist == 0) return;
+  const Plan& q = *s.plan;
+  const uint32_t k0 = kring + (uint32_t)(q.r0[ph].u1 - q.r0[ph].u0);
+  if (++ph == 4) {
+    ph = 0;
+    if (++l >= p.L) return;
+  }
+  const int warp = ct >> 5;
+  prefetch_rows<BITS>(range_of(q, l, ph), k0, warp / kQuadWarps, warp % kQuadWarps, ct & 31);
 }
 
 // ------------------------------------------------------------------ grid barrier
@@ -921,7 +878,7 @@ __device__ __forceinline__ void prefetch_chain(const Params& p, int l, int ph, i
 template <int BITS, int TM>
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_constant__ Params p) {
   using Gm = FGeo<BITS>;
-  Smem s = carve(p, Gm::kStageBytes);
+  Smem s = carve(p);
   const uint32_t r = cta_rank();
   const int c = (int)cluster_id_x();
   const int tid = threadIdx.x;
@@ -930,25 +887,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     make_plan<BITS>(p, c, (int)r, *s.plan);
     s_wait_cycles = p.wait_cycles;
     s.won[0] = 0;
-    for (int i = 0; i < p.ring_stages; ++i) {
-      mbar_init(&s.full[i], 1);
-      s.ucnt[i] = 0;
-      s.lastk[i] = -1;
-    }
     mbar_init(&s.xbar[0], 1);
     mbar_init(&s.xbar[1], 1);
     fence_mbar_init();
-    // the ring's first stages, after the L2 requests for those the refills will ask for
-    Range g;
-    int u;
-    for (int k = p.ring_stages; k < p.pf_dist; ++k)
-      if (locate(p, *s.plan, (uint32_t)k, g, u)) prefetch_unit<BITS>(g, u);
-    for (int k = 0; k < p.ring_stages; ++k) issue_stage<BITS>(p, s, (uint32_t)k);
   }
   cluster_sync_all();  // every CTA's barriers exist before any remote store signals one
 
   const int L = p.L;
   const int ct = tid;
+  // the first GEMV phase's weights into L2 while the first chain runs
+  if (p.pf_dist > 0)
+    prefetch_rows<BITS>(range_of(*s.plan, 0, 0), 0, (ct >> 5) / kQuadWarps, (ct >> 5) % kQuadWarps, ct & 31);
   uint32_t kring = 0;
   Xch X;
   float res[2] = {0.f, 0.f};  // the residual stream, this CTA's layout-B share
@@ -963,6 +912,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       break;
     // P2 (L2 requests for the tables of the chain that follows, as every GEMV phase)
     if (ct == 0 && p.tm != kTmHad) prefetch_chain(p, l, 0, c, r);
+    prefetch_next<BITS>(p, s, l, 0, kring, ct);
     if (!(ok = run_units<BITS>(p, s, range_of(*s.plan, l, 0), kring, ct))) break;
     if (!(ok = grid_barrier(p, l * 5 + 0, ct))) break;
     // P3
@@ -971,11 +921,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       break;
     // P4
     if (ct == 0 && p.tm != kTmHad) prefetch_chain(p, l, 1, c, r);
+    prefetch_next<BITS>(p, s, l, 1, kring, ct);
     if (!(ok = run_units<BITS>(p, s, range_of(*s.plan, l, 1), kring, ct))) break;
     if (!(ok = grid_barrier(p, l * 5 + 1, ct))) break;
     // P5
     if (!(ok = residual_any<TM>(p, s, X, res, lin + 3, p.zpo, p.nk_h, lin + 4 + p.asg_gu[c], r, ct))) break;
     // P6
+    prefetch_next<BITS>(p, s, l, 2, kring, ct);
     if (p.mlp_tickets) {
       const int wb = lin[4].w_out;
       const unsigned per_block = (unsigned)(2 * (wb / 32) * p.nk_h * kQuadWarps);
@@ -1017,6 +969,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       }
       cbar();
       if (ct == 0 && p.tm != kTmHad) prefetch_chain(p, l, 3, c, r);
+      prefetch_next<BITS>(p, s, l, 3, kring, ct);
       if (!(ok = run_units<BITS>(p, s, range_of(*s.plan, l, 3), kring, ct))) break;
     }
     if (!(ok = grid_barrier(p, l * 5 + 4, ct))) break;
@@ -1035,13 +988,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       }
     }
   }
-  // copies still in flight (a step that ended early) land before the CTA exits: bounded,
-  // and not cut short by the abort word, since these are this CTA's own copies
-  if (ct == 0)
-    for (int i = 0; i < p.ring_stages; ++i)
-      if (s.lastk[i] >= 0)
-        wait_phase<false, true, false>(&s.full[i], ((uint32_t)s.lastk[i] / (uint32_t)p.ring_stages) & 1, p.status,
-                                       54);
   cluster_sync_all();
 }
 
@@ -1080,8 +1026,7 @@ cudaError_t repack_side(int tm, int eb, bool cluster, int nblk, const uint8_t* t
 // ------------------------------------------------------------------ host side
 template <int BITS>
 size_t smem_bytes(const Params& p) {
-  return 1024 + (size_t)p.ring_stages * FGeo<BITS>::kStageBytes + 3 * 4 * (size_t)kRxFloats + 4 * 32 + 4 * 32 +
-         p.xq_bytes + 4 * kCW * 8 * 33 + 2 * 4 * 16 + 512 + 8 * ((size_t)p.ring_stages + 2);
+  return 16 + 3 * 4 * (size_t)kRxFloats + 4 * 32 + 4 * 32 + p.xq_bytes + 4 * kCW * 8 * 33 + 512 + 8 * 2;
 }
 
 template <int BITS>

@@ -21,7 +21,9 @@ enum { kTmCS = 0, kTmHad = 1, kTmQ8 = 2 };
 
 // One linear as the fused kernel sees it (device array, 64-byte aligned for the maps).
 struct alignas(64) Lin {
-  CUtensorMap tm_codes, tm_hi, tm_sz;
+  const uint8_t* codes;  // [n_out][n_in/64] groups of 16 bytes (2-bit) or 32 (4-bit); 3-bit: the 2-bit plane
+  const uint8_t* hi;     // 3-bit: the 1-bit plane, [n_out][n_in/64] x 8 bytes; else null
+  const uint32_t* sz;    // scale/zero words [n_out][n_in/64]
   const uint8_t* tV;  // input-side angle storage in the stack's form (see kTm*), or null
   const uint8_t* tU;  // output-side angle storage
   const int8_t* sV;
@@ -56,8 +58,8 @@ struct Params {
   long long wait_cycles;  // bound of every wait, in SM clock cycles
   int barrier_extra;      // testing hook: grid barrier whose target is raised by one (-1: none)
   int tm;   // kTmCS, kTmHad or kTmQ8: how every butterfly of the stack keeps its angles
-  int ring_stages, xq_bytes;
-  int pf_dist;      // units the L2 prefetch runs ahead of the ring (0: none)
+  int xq_bytes;
+  int pf_dist;      // nonzero: each GEMV phase asks for the next phase's weights in L2
   int cooperative;  // launch with the cooperative attribute (all CTAs co-resident or refused)
   int asg_qkv[kMaxClusters], idx_qkv[kMaxClusters], cnt_qkv[3];
   int asg_gu[kMaxClusters], idx_gu[kMaxClusters], cnt_gu[2];

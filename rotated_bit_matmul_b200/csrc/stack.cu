@@ -273,18 +273,15 @@ void setup_fused(harp_stack_s* S) {
   p.eb_kv = ilog2(dkv / dec::kC);
   p.eb_blk = ilog2(wb);
   p.nblocks = F / wb;
-  // shared memory: the operand of the widest input, then as many ring stages as fit
-  // (each also carries its reduction scratch and barriers)
+  // shared memory: the operand of the widest input and the chain buffers
   auto xqb = [&](int n) { return 4 * ((bits == 3 ? n : n / 2) + 2 * (n / 64)); };
-  p.xq_bytes = (std::max(xqb(H), xqb(F)) + 15) & ~15;  // keeps the mbarriers after it 8-byte aligned
+  p.xq_bytes = (std::max(xqb(H), xqb(F)) + 15) & ~15;  // keeps what follows it 16-byte aligned
   int optin = 0;
   cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, S->device);
-  p.ring_stages = 16;
-  while (p.ring_stages >= 2 && dec::smem_for(p) > (size_t)optin) --p.ring_stages;
-  if (p.ring_stages < 2) return no("not enough shared memory for the weight ring");
-  // L2 prefetch distance in units (tuning knob HARP_PF_DIST); cooperative launch unless
-  // HARP_COOPERATIVE=0
-  p.pf_dist = 24;
+  if (dec::smem_for(p) > (size_t)optin) return no("not enough shared memory for the operand");
+  // HARP_PF_DIST=0 turns off the L2 requests for the next GEMV phase's weights; cooperative
+  // launch unless HARP_COOPERATIVE=0
+  p.pf_dist = 1;
   if (const char* e = getenv("HARP_PF_DIST")) p.pf_dist = std::max(0, atoi(e));
   p.cooperative = 1;
   if (const char* e = getenv("HARP_COOPERATIVE")) p.cooperative = atoi(e) != 0;
@@ -297,15 +294,15 @@ void setup_fused(harp_stack_s* S) {
   cudaError_t e = dec::max_clusters(p, &G);
   if (e != cudaSuccess || G < 1)
     return no(std::string("cluster occupancy query failed: ") + cudaGetErrorString(e) + ", G=" + std::to_string(G) +
-              ", smem " + std::to_string(dec::smem_for(p)) + ", ring stages " + std::to_string(p.ring_stages));
+              ", smem " + std::to_string(dec::smem_for(p)));
   if (G > dec::kMaxClusters) G = dec::kMaxClusters;
   // P7: MLP-block CTAs (or clusters) come first, the last two clusters apply F_U_q / F_U_k
   const int cap = wb <= 512 ? dec::kC : 1;
   if (G < 3 || p.nblocks > (G - 2) * cap) return no("too few co-resident clusters");
   p.G = G;
   if (getenv("HARP_DEBUG"))
-    fprintf(stderr, "harp fused step: G=%d ring_stages=%d smem=%zu xq_bytes=%d eb_h=%d eb_kv=%d eb_blk=%d nblocks=%d tm=%d\n",
-            G, p.ring_stages, dec::smem_for(p), p.xq_bytes, p.eb_h, p.eb_kv, p.eb_blk, p.nblocks, p.tm);
+    fprintf(stderr, "harp fused step: G=%d smem=%zu xq_bytes=%d eb_h=%d eb_kv=%d eb_blk=%d nblocks=%d tm=%d\n", G,
+            dec::smem_for(p), p.xq_bytes, p.eb_h, p.eb_kv, p.eb_blk, p.nblocks, p.tm);
   const int rq[3] = {dq, dkv, dkv}, rg[2] = {F, F};
   assign(G, rq, 3, p.asg_qkv, p.idx_qkv, p.cnt_qkv);
   assign(G, rg, 2, p.asg_gu, p.idx_gu, p.cnt_gu);
@@ -315,9 +312,9 @@ void setup_fused(harp_stack_s* S) {
     const Layer& L = S->layers[i]->L;
     dec::Lin& d = h[i];
     memset(&d, 0, sizeof d);
-    d.tm_codes = L.tm_codes;
-    d.tm_hi = L.tm_hi;
-    d.tm_sz = L.tm_sz;
+    d.codes = static_cast<const uint8_t*>(L.codes);
+    d.hi = L.bits == 3 ? static_cast<const uint8_t*>(L.codes) + L.n_out * L.n_in / 4 : nullptr;
+    d.sz = static_cast<const uint32_t*>(L.scale_zero);
     d.tV = L.q8V ? L.q8V : reinterpret_cast<const uint8_t*>(L.csV);
     d.tU = L.q8U ? L.q8U : reinterpret_cast<const uint8_t*>(L.csU);
     d.sV = L.sV;
