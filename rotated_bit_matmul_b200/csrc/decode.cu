@@ -169,10 +169,18 @@ __device__ bool prep_broadcast(const float (&v)[2], int n_in, int bits, Smem& sm
   return xch_end(sm, x, status, 40, ct);
 }
 
-// sum of the split-K partials of element i (fixed order)
+// sum of the split-K partials of element i (fixed order); the loads are independent and
+// go out together (one L2 round trip for up to 16 partials)
 __device__ __forceinline__ float zsum(const float* zp, int nk, int64_t n, int64_t i) {
-  float t = __ldcg(zp + i);
-  for (int k = 1; k < nk; ++k) t += __ldcg(zp + (int64_t)k * n + i);
+  constexpr int kMaxK = 16;
+  float v[kMaxK];
+#pragma unroll
+  for (int k = 0; k < kMaxK; ++k) v[k] = k < nk ? __ldcg(zp + (int64_t)k * n + i) : 0.f;
+  float t = v[0];
+#pragma unroll
+  for (int k = 1; k < kMaxK; ++k)
+    if (k < nk) t += v[k];
+  for (int k = kMaxK; k < nk; ++k) t += __ldcg(zp + (int64_t)k * n + i);
   return t;
 }
 
@@ -208,6 +216,10 @@ __device__ __noinline__ bool chain_residual(const Params& p, Smem& sm, Xch& x, f
   if (!V || !ok) return ok;
   BF fv;
   fetch_side(fv, V->rV, V->tV, (int64_t)V->n_in / 2, 0, r, ct);
+  float sgn[2] = {0.f, 0.f};  // F_V's signs, read before the exchange (its wait orders memory)
+  if (act)
+#pragma unroll
+    for (int s = 0; s < M::P; ++s) sgn[s] = (float)__ldg(V->sV + (int)r * M::E + M::e1(ct, s));
   // sum of squares: warps, then the CTA (fixed order), then to every peer's slot r along
   // with the residual values each peer holds in layout A for F_V
   float acc = 0.f;
@@ -241,7 +253,7 @@ __device__ __noinline__ bool chain_residual(const Params& p, Smem& sm, Xch& x, f
 #pragma unroll
     for (int s = 0; s < M::P; ++s) {
       const int e = M::e1(ct, s);
-      v[s] = rx[idx_a(e)] * inv * (float)__ldg(V->sV + (int)r * M::E + e);
+      v[s] = rx[idx_a(e)] * inv * sgn[s];
     }
   if (!(ok = fv.run(v, sm, x, r, ct, p.status, 43))) return false;
   return prep_broadcast<EB>(v, V->n_in, p.bits, sm, x, r, ct, p.status);
@@ -266,6 +278,10 @@ __device__ __noinline__ bool chain_attn(const Params& p, Smem& sm, Xch& x, const
   if (!fu.run(v, sm, x, r, ct, p.status, 44)) return false;
   ClusterBfly<EB, TM> fv;
   fetch_side(fv, Lo->rV, Lo->tV, (int64_t)Lo->n_in / 2, 0, r, ct);
+  float sgn[2] = {0.f, 0.f};  // F_V's signs, read before the exchange
+  if (ct < M::NT)
+#pragma unroll
+    for (int s = 0; s < M::P; ++s) sgn[s] = (float)__ldg(Lo->sV + (int)r * M::E + M::e1(ct, s));
   // every v value to the layout-A owners of the query-head elements that copy it
   const int hd = p.head_dim, rep = p.rep;
   int self = 0;
@@ -293,7 +309,7 @@ __device__ __noinline__ bool chain_attn(const Params& p, Smem& sm, Xch& x, const
 #pragma unroll
     for (int s = 0; s < M::P; ++s) {
       const int e = M::e1(ct, s);
-      w[s] = rx[idx_a(e)] * (float)__ldg(Lo->sV + (int)r * M::E + e);
+      w[s] = rx[idx_a(e)] * sgn[s];
     }
   if (!fv.run(w, sm, x, r, ct, p.status, 46)) return false;
   return prep_broadcast<EB>(w, Lo->n_in, p.bits, sm, x, r, ct, p.status);
@@ -335,20 +351,18 @@ __device__ __noinline__ void mlp_block_local(const Params& p, Smem& sm, const Li
   fetch_side(fd, Ld->rV, Ld->tV, (int64_t)Ld->n_in / 2, blk, ct);
   const bool act = ct < M::NT;
   const int64_t base = (int64_t)blk * M::E;
-  float vg = 0.f, vu = 0.f;
+  float vg = 0.f, vu = 0.f, sd = 0.f;
   if (act) {
     const int64_t g = base + M::e1(ct, 0);
     vg = zsum(p.zpg, p.nk_h, Lg->n_out, g) * (float)__ldg(Lg->sU + g);
     vu = zsum(p.zpu, p.nk_h, Lu->n_out, g) * (float)__ldg(Lu->sU + g);
+    sd = (float)__ldg(Ld->sV + base + M::e2(ct, 0));  // F_V_down's sign, read up front
   }
   fg.run(vg, sm, ct);
   fu.run(vu, sm, ct);
   // both in phase-2 order; F_V_down starts from phase-1 order
   float h = 0.f;
-  if (act) {
-    const int64_t g = base + M::e2(ct, 0);
-    h = silu(vg) * vu * (float)__ldg(Ld->sV + g);
-  }
+  if (act) h = silu(vg) * vu * sd;
   cbar();
   if (act) sm.T[idx_a(M::e2(ct, 0))] = h;
   cbar();
@@ -402,6 +416,10 @@ __device__ __noinline__ bool mlp_block_cluster(const Params& p, Smem& sm, Xch& x
   }
   BF fd;
   fetch_side(fd, Ld->rV, Ld->tV, (int64_t)Ld->n_in / 2, blk, r, ct);
+  float sgn[2] = {0.f, 0.f};  // F_V_down's signs, read before the exchange
+  if (act)
+#pragma unroll
+    for (int s = 0; s < M::P; ++s) sgn[s] = (float)__ldg(Ld->sV + base + (int)r * M::E + M::e1(ct, s));
   // h = silu(gate) * up in layout B, to the layout-A owners
   xch_begin(sm, x, 4u * M::RUN * (kC - 1), ct);
   if (act)
@@ -415,7 +433,7 @@ __device__ __noinline__ bool mlp_block_cluster(const Params& p, Smem& sm, Xch& x
 #pragma unroll
     for (int s = 0; s < M::P; ++s) {
       const int e = M::e1(ct, s);
-      v[s] = rx[idx_a(e)] * (float)__ldg(Ld->sV + base + (int)r * M::E + e);
+      v[s] = rx[idx_a(e)] * sgn[s];
     }
   if (!fd.run(v, sm, x, r, ct, p.status, 51)) return false;
   // groups of 64 inside the runs, to the global down operand
@@ -853,6 +871,16 @@ __device__ __forceinline__ void prefetch_side(const uint8_t* rt, const int8_t* s
   if (E % 16 == 0) bulk_prefetch_l2(sign + (size_t)r * E, (uint32_t)E);
 }
 
+// L2 hint for one block of a side kept in the local (one CTA per block) thread order, and
+// for that block's signs
+__device__ __forceinline__ void prefetch_block(const uint8_t* rt, const int8_t* sign, int eb, int tm, int blk) {
+  if (!rt) return;
+  const int E = 1 << eb, nt = E < kNT ? E : kNT;
+  const uint32_t bytes = (uint32_t)(eb * (nt / 2) * (tm == kTmCS ? 8 : 4));
+  bulk_prefetch_l2(rt + (size_t)blk * bytes, bytes);
+  if (E % 16 == 0) bulk_prefetch_l2(sign + (size_t)blk * E, (uint32_t)E);
+}
+
 // the tables of the chain that follows GEMV phase ph of block l (one thread, as the phase
 // starts)
 __device__ __forceinline__ void prefetch_chain(const Params& p, int l, int ph, int c, uint32_t r) {
@@ -863,6 +891,15 @@ __device__ __forceinline__ void prefetch_chain(const Params& p, int l, int ph, i
   } else if (ph == 1) {  // P5: F_U of o, F_V of the cluster's gate or up
     prefetch_side(lin[3].rU, lin[3].sU, p.eb_h, p.tm, r);
     prefetch_side(lin[4 + p.asg_gu[c]].rV, lin[4 + p.asg_gu[c]].sV, p.eb_h, p.tm, r);
+  } else if (ph == 2) {  // P7: the MLP block this CTA runs (up to 512 wide), F_U of q or k
+    const int t_cta = c * kC + (int)r;
+    if (p.eb_blk <= 9 && t_cta < p.nblocks) {
+      prefetch_block(lin[4].rU, lin[4].sU, p.eb_blk, p.tm, t_cta);
+      prefetch_block(lin[5].rU, lin[5].sU, p.eb_blk, p.tm, t_cta);
+      prefetch_block(lin[6].rV, lin[6].sV, p.eb_blk, p.tm, t_cta);
+    }
+    if (c == qk_cluster(p, 0)) prefetch_side(lin[0].rU, lin[0].sU, p.eb_h, p.tm, r);
+    if (c == qk_cluster(p, 1)) prefetch_side(lin[1].rU, lin[1].sU, p.eb_kv, p.tm, r);
   } else if (ph == 3) {  // next P1: F_U of down, F_V of the cluster's q, k or v in block l + 1
     prefetch_side(lin[6].rU, lin[6].sU, p.eb_h, p.tm, r);
     if (l + 1 < p.L) {
@@ -927,6 +964,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     // P5
     if (!(ok = residual_any<TM>(p, s, X, res, lin + 3, p.zpo, p.nk_h, lin + 4 + p.asg_gu[c], r, ct))) break;
     // P6
+    if (ct == 0 && p.tm != kTmHad) prefetch_chain(p, l, 2, c, r);
     prefetch_next<BITS>(p, s, l, 2, kring, ct);
     if (p.mlp_tickets) {
       const int wb = lin[4].w_out;
