@@ -83,11 +83,11 @@ def algorithmic_bytes_per_step(n_layers, batch=BATCH, bits=BITS):
 
 # DRAM bytes (read + write) of one fused decode launch per transformer block, from an
 # ncu capture of the 4-block stack (dram__bytes_read.sum + dram__bytes_write.sum, scaled
-# by blocks): 270.97 MB per launch with fp32 cos/sin tables, 258.86 MB with
-# int8 angles. With them, a hash of the kernel's sources at capture time: the figures are
-# reported only while those sources are unchanged.
-TRAFFIC_PER_BLOCK = {"bytes": {"fp32": 270_965_248 // 4, "int8": 258_862_848 // 4},
-                     "sources_sha256_16": "a7a80626b48c905c"}
+# by blocks): 291.40 MB per 4-block launch with fp32 cos/sin tables (int8 angles: not
+# captured for these sources). With them, a hash of the kernel's sources at capture time:
+# the figures are reported only while those sources are unchanged.
+TRAFFIC_PER_BLOCK = {"bytes": {"fp32": 291_404_288 // 4, "int8": None},
+                     "sources_sha256_16": "7a655f9784ea80d5"}
 KERNEL_SOURCES = ("decode.cu", "decode.h", "common.cuh", "gemv_core.cuh", "bfly_engine.cuh")
 
 
@@ -100,7 +100,8 @@ def traffic_per_step(n_layers, angles="fp32"):
             h.update(fh.read())
     if h.hexdigest()[:16] != TRAFFIC_PER_BLOCK["sources_sha256_16"]:
         return None
-    return TRAFFIC_PER_BLOCK["bytes"][angles] * n_layers
+    b = TRAFFIC_PER_BLOCK["bytes"][angles]
+    return None if b is None else b * n_layers
 
 
 def measured_tc_peak():
@@ -414,6 +415,20 @@ def run_linear_configs(args):
                 total_us += mult[i] * us
                 total_bytes += mult[i] * r["alg_bytes"]
     if args.config == 2:
+        # the FFN side as one mixed-radix butterfly (11008 = 2^8 * 43) against 43 blocks of 256
+        for side, nm in (("U", "gate/up 11008x4096, output side 2^8*43"), ("V", "down 4096x11008, input side 43*2^8")):
+            with ClockSampler(0) as clk:
+                m = lt.time_mixed_radix(side)
+            ach = m["alg_bytes"] / m["us_mixed_radix"] / 1e3
+            _line(f"rotated 2-bit linear {nm} mixed-radix, batch 1: time per call", m["us_mixed_radix"], "us/call",
+                  False, {"workload": f"config 2: {nm} as one mixed-radix butterfly, bf16 x [1,{m['n_in']}]",
+                          "batch": 1, "distinct_layers": m["layers"], "l2": "cold L2: distinct layer copies per call"},
+                  {"bound": "hbm", "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
+                   "frac": round(ach / peak, 4), "traffic": None, "peak_kind": peak_kind,
+                   "algorithmic_bytes_per_call": m["alg_bytes"], "kernel": "whole harp_linear_fwd, mixed-radix sides"},
+                  launches=None, clocks=clk.summary(),
+                  extra={"block_diagonal_us_per_call": m["us_block_diagonal"],
+                         "mixed_radix_over_block_diagonal": round(m["us_mixed_radix"] / m["us_block_diagonal"], 3)})
         ach = total_bytes / total_us / 1e3
         _line("the seven linears of a 7B-shaped block, batch 1: time per block", round(total_us, 2), "us/block",
               False, {"workload": "config 2: q/k/v/o 4096x4096, gate/up 11008x4096, down 4096x11008, batch 1",
