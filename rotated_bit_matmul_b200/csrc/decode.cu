@@ -9,10 +9,11 @@
 //    for its rows of the next phase's weights in L2 (plain per-lane line prefetches), and
 //    HBM streams them while the chains run. A GEMV is cut into units of 32 output rows x
 //    2048 input columns (split-K); each unit's partial sums go to a buffer the next chain
-//    adds up in a fixed order. The 16 warps form four quads that take the units in turn;
-//    a lane holds one group of 64 input columns, with its operand words in registers, for
-//    eight rows, and loads that group's codes and scale/zero words of those rows straight
-//    from L2 (a warp reads each row's chunk as one contiguous span).
+//    adds up in a fixed order. Each of the 16 warps takes two rows of every unit; a
+//    lane holds one group of 64 input columns, with its operand words in registers, and
+//    loads that group's codes and scale/zero words of its rows straight from L2 (a warp
+//    reads each row's chunk as one contiguous span). The down projection reads its
+//    operand from the global buffer the MLP blocks wrote.
 //  * CTAs form clusters of 8. Each cluster computes the activation chain between two
 //    GEMVs itself (redundantly with the other clusters): a w-wide butterfly is spread
 //    over the 8 CTAs, w/8 elements each. Every consumer thread holds one (two when
@@ -45,7 +46,7 @@
 //   P7 MLP blocks (one CTA each up to 512 wide, one cluster each from 2048): F_U_gate,
 //      F_U_up, silu*up, F_V_down, operand to global; the two last clusters apply F_U_q
 //      and F_U_k of this block                  -> grid barrier
-//   P8 GEMV down                                -> grid barrier
+//   P8 GEMV down (operand from global)          -> grid barrier
 // and after the last block: out = h_{L-1} + F_U_down(z_down).
 //
 // Every wait is bounded (about 2 s of SM clock unless the testing hook shortens it) and
@@ -511,25 +512,43 @@ __device__ __forceinline__ void prefetch_line_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
-// L2 requests for this warp's rows of its units in range g (the units of a phase go to the
-// quads in turn from quad k0 % 4): lane l asks for 128-byte line l % 4 (and + 4, ...) of
-// row l / 4's codes and 1-bit plane in the chunk, lanes 0, 4, ... for its scale/zero words.
-// Plain prefetches from every lane: nothing queues behind the TMA unit.
+// L2 requests for this warp's rows of range g, the same rows run_units will take (rows
+// rw and rw + 16 of every unit, rw turned by the phase's first unit index k0): lanes 0..7
+// (0..15 at 4 bits) ask for the 128-byte lines of the two rows' codes in the chunk, lanes
+// 16, 17 for their scale/zero words, lanes 18..21 for their 1-bit plane (3 bits). Plain
+// prefetches from every lane: nothing queues behind the TMA unit.
 template <int BITS>
-__device__ __forceinline__ void prefetch_rows(const Range& g, uint32_t k0, int quad, int qw, int lane) {
+__device__ __forceinline__ void prefetch_rows(const Range& g, uint32_t k0, int warp, int lane) {
   using Gm = FGeo<BITS>;
   const int ngroups = g.n_in / 64, row_bytes = ngroups * Gm::kGroupBytes;
-  const int line = lane & 3;
-  for (int i = (quad - (int)(k0 & 3)) & 3; i < g.u1 - g.u0; i += 4) {
+  const int rw = (warp - (int)(k0 & 15)) & 15;
+  constexpr int LPR = 2048 * (BITS == 4 ? 4 : 2) / 8 / 128;  // code lines per row of a chunk
+  for (int i = 0; i < g.u1 - g.u0; ++i) {
     int tile, kc;
     g.tk(g.u0 + i, tile, kc);
-    const int row = tile * 32 + qw * 8 + (lane >> 2);
-    if (row >= g.n_out) continue;
     const int g0 = kc * Gm::kChunkGroups, gc = min(Gm::kChunkGroups, ngroups - g0);
-    const uint8_t* cb = g.L->codes + (size_t)row * row_bytes + (size_t)g0 * Gm::kGroupBytes;
-    for (int o = line * 128; o < gc * Gm::kGroupBytes; o += 512) prefetch_line_l2(cb + o);
-    if (BITS == 3 && line * 128 < gc * 8) prefetch_line_l2(g.L->hi + (size_t)row * (ngroups * 8) + (size_t)g0 * 8 + line * 128);
-    if (line == 0) prefetch_line_l2(g.L->sz + (size_t)row * ngroups + g0);
+    int row, bytes = 0;
+    const uint8_t* src = nullptr;
+    if (lane < 2 * LPR) {
+      row = tile * 32 + rw + 16 * (lane / LPR);
+      const int o = (lane % LPR) * 128;
+      if (o < gc * Gm::kGroupBytes) {
+        src = g.L->codes + (size_t)row * row_bytes + (size_t)g0 * Gm::kGroupBytes + o;
+        bytes = 1;
+      }
+    } else if (lane == 16 || lane == 17) {
+      row = tile * 32 + rw + 16 * (lane - 16);
+      src = reinterpret_cast<const uint8_t*>(g.L->sz + (size_t)row * ngroups + g0);
+      bytes = 1;
+    } else if (BITS == 3 && lane >= 18 && lane < 22) {
+      row = tile * 32 + rw + 16 * ((lane - 18) >> 1);
+      const int o = ((lane - 18) & 1) * 128;
+      if (o < gc * 8) {
+        src = g.L->hi + (size_t)row * (ngroups * 8) + (size_t)g0 * 8 + o;
+        bytes = 1;
+      }
+    }
+    if (bytes && row < g.n_out) prefetch_line_l2(src);
   }
 }
 
@@ -560,16 +579,15 @@ __device__ __forceinline__ Range range_of(const Plan& q, int l, int ph) {
 }
 
 // ------------------------------------------------------------------ GEMV
-// The 16 warps form four quads, and a CTA's units go to the quads in turn. In a unit, warp
-// w of the quad takes rows 8w..8w+7 and lane l the unit's group l (64 input columns). The
-// lane loads its own bytes of every row straight from global memory (a warp reads each
-// row's chunk as one contiguous, coalesced span; the phase's weights were requested into
-// L2 a phase earlier), with a batch of rows in flight at once, and keeps its operand words
-// in registers for all its rows, and for the warp's next unit too when that has the same
-// chunk. No data passes between warps but the row sums: a warp's per-lane partials go
-// through its own 8 x 32 scratch in shared memory, and four lanes add up each row, in a
-// fixed order.
-constexpr int kQuads = 4, kQuadWarps = kCW / kQuads, kRowsW = 32 / kQuadWarps;
+// Every warp takes two rows of every unit of the CTA's range (rows rw and rw + 16, rw
+// turned by the CTA's unit count from phase to phase), and lane l the unit's group l (64
+// input columns). The lane loads its own bytes of each row straight from global memory (a
+// warp reads each row's chunk as one contiguous, coalesced span; the phase's weights were
+// requested into L2 a phase earlier), two units' rows in flight at once when they share a
+// chunk, and keeps its operand words in registers while the chunk stays the same. No data
+// passes between warps but the row sums: a warp's per-lane partials go through its own
+// scratch in shared memory, and eight lanes add up each row, in a fixed order.
+constexpr int kRowsW = 8;  // rows of scratch per warp (four are used)
 constexpr int kRedRow = 33;  // scratch row stride: the adders' reads hit 32 distinct banks
 
 // 16-byte chunk k of operand group G in shared memory (and in the down operand in global):
@@ -598,7 +616,7 @@ __device__ __forceinline__ void load_row(RowW<BITS>& w, const Range& g, int row,
 // exact integer dot product of one row's group with the operand words x of that group;
 // xh: the 1-bit plane's operand (3-bit)
 template <int BITS>
-__device__ __forceinline__ int row_dot(const RowW<BITS>& rw, const int4 (&x)[8], const int4* xh, int G) {
+__device__ __forceinline__ int row_dot(const RowW<BITS>& rw, const int4 (&x)[8], const int4* xh, int G, bool xg) {
   if constexpr (BITS == 2 || BITS == 3) {
     const uint32_t wv[4] = {rw.c[0].x, rw.c[0].y, rw.c[0].z, rw.c[0].w};
     int a0 = 0, a1 = 0, a2 = 0, a3 = 0, b0 = 0, b1 = 0, b2 = 0, b3 = 0;
@@ -624,7 +642,7 @@ __device__ __forceinline__ int row_dot(const RowW<BITS>& rw, const int4 (&x)[8],
       for (int k = 0; k < 2; ++k) {
 #pragma unroll
         for (int mm = 0; mm < 8; mm += 2) {
-          const int4 xa = xh[xq_chunk(G, 4 * k + mm / 2)];
+          const int4 xa = xg ? __ldcg(xh + xq_chunk(G, 4 * k + mm / 2)) : xh[xq_chunk(G, 4 * k + mm / 2)];
           const uint32_t ma = hv[k] & (0x01010101u << mm), mb = hv[k] & (0x01010101u << (mm + 1));
           int ha = 0, hb = 0;
           ha = dp2a_lo(xa.x, ma, ha);
@@ -657,78 +675,94 @@ __device__ __forceinline__ int row_dot(const RowW<BITS>& rw, const int4 (&x)[8],
 // this block; per_block: (unit, warp) items of one MLP block's gate and up rows
 template <int BITS, bool TICKETS = false>
 __device__ __noinline__ bool run_units(const Params& p, Smem& s, const Range& g, uint32_t& kring, int ct,
-                                          unsigned* tickets = nullptr, unsigned per_block = 0, int wb = 0) {
+                                          const int32_t* xglob = nullptr, unsigned* tickets = nullptr,
+                                          unsigned per_block = 0, int wb = 0) {
   using Gm = FGeo<BITS>;
-  constexpr int RB = Gm::kRowBatch;
-  static_assert(kRowsW == 8, "four lanes add up each of a warp's eight rows");
   const int warp = ct >> 5, lane = ct & 31;
-  const int quad = warp / kQuadWarps, qw = warp - quad * kQuadWarps;
   const int n_out = g.n_out, n_in = g.n_in, ngroups = n_in / 64;
   const int words = BITS == 3 ? n_in : n_in / 2;
-  const float* xsA = reinterpret_cast<const float*>(s.xq + words);
-  const float* xsumA = xsA + ngroups;
-  const int4* xlo = reinterpret_cast<const int4*>(s.xq);
-  const int4* xhi = reinterpret_cast<const int4*>(s.xq + n_in / 2);
+  // the operand: shared memory, or (xglob) the global buffer another phase of this kernel
+  // wrote, read through L2
+  const int32_t* xw = xglob ? xglob : s.xq;
+  const float* xsA = xglob ? p.xs_down : reinterpret_cast<const float*>(s.xq + words);
+  const float* xsumA = xglob ? p.xsum_down : xsA + ngroups;
+  const int4* xlo = reinterpret_cast<const int4*>(xw);
+  const int4* xhi = reinterpret_cast<const int4*>(xw + n_in / 2);
   const int nu = g.u1 - g.u0;
+  // rows rw and rw + 16 of every unit; the mapping turns with the CTA's unit count so that
+  // no warp keeps the same rows phase after phase
+  const int rw = (warp - (int)(kring & 15)) & 15;
   int4 xr[8];
   float xs = 0.f, xsum = 0.f;
   int kc_have = -1;
   float* red = s.red + warp * (kRowsW * kRedRow);
-  // unit i of the phase is the CTA's (kring + i)-th and goes to quad (kring + i) % 4
-  for (int i = (quad - (int)(kring & 3)) & 3; i < nu; i += kQuads) {
-    int tile, kc;
-    g.tk(g.u0 + i, tile, kc);
+  for (int i = 0; i < nu;) {
+    // this unit and, when it has the same chunk, the next: up to four rows in flight
+    int tile[2], kc;
+    g.tk(g.u0 + i, tile[0], kc);
+    tile[1] = tile[0];
+    int nb = 1;
+    if (i + 1 < nu) {
+      int t1, k1;
+      g.tk(g.u0 + i + 1, t1, k1);
+      if (k1 == kc) {
+        tile[1] = t1;
+        nb = 2;
+      }
+    }
     const int g0 = kc * Gm::kChunkGroups, gc = min(Gm::kChunkGroups, ngroups - g0);
     const bool act = lane < gc;
     const int G = g0 + lane;
-    const int row0 = tile * 32 + qw * kRowsW;
     if (kc != kc_have) {
       kc_have = kc;
       if (act) {
 #pragma unroll
-        for (int k = 0; k < 8; ++k) xr[k] = xlo[xq_chunk(G, k)];
-        xs = xsA[G];
-        xsum = xsumA[G];
+        for (int k = 0; k < 8; ++k) xr[k] = xglob ? __ldcg(xlo + xq_chunk(G, k)) : xlo[xq_chunk(G, k)];
+        xs = xglob ? __ldcg(xsA + G) : xsA[G];
+        xsum = xglob ? __ldcg(xsumA + G) : xsumA[G];
       }
     }
-#pragma unroll 1
-    for (int rb = 0; rb < kRowsW; rb += RB) {
-      RowW<BITS> w[RB];
+    RowW<BITS> w[4];
 #pragma unroll
-      for (int j = 0; j < RB; ++j)
-        if (act && row0 + rb + j < n_out) load_row<BITS>(w[j], g, row0 + rb + j, G, ngroups);
+    for (int j = 0; j < 4; ++j) {
+      const int row = tile[j >> 1] * 32 + rw + 16 * (j & 1);
+      if ((j >> 1) < nb && act && row < n_out) load_row<BITS>(w[j], g, row, G, ngroups);
+    }
 #pragma unroll
-      for (int j = 0; j < RB; ++j) {
-        float z = 0.f;
-        if (act && row0 + rb + j < n_out) {
-          const float s16 = __half2float(__ushort_as_half((unsigned short)(w[j].sz & 0xffffu)));
-          const float z16 = __half2float(__ushort_as_half((unsigned short)(w[j].sz >> 16)));
-          const int acc = row_dot<BITS>(w[j], xr, xhi, G);
-          z = fmaf(s16, (float)acc * xs, z16 * xsum);
-        }
-        red[(rb + j) * kRedRow + lane] = z;
+    for (int j = 0; j < 4; ++j) {
+      const int row = tile[j >> 1] * 32 + rw + 16 * (j & 1);
+      float z = 0.f;
+      if ((j >> 1) < nb && act && row < n_out) {
+        const float s16 = __half2float(__ushort_as_half((unsigned short)(w[j].sz & 0xffffu)));
+        const float z16 = __half2float(__ushort_as_half((unsigned short)(w[j].sz >> 16)));
+        const int acc = row_dot<BITS>(w[j], xr, xhi, G, xglob != nullptr);
+        z = fmaf(s16, (float)acc * xs, z16 * xsum);
       }
+      red[j * kRedRow + lane] = z;
     }
     __syncwarp();
-    // row (lane >> 2) of the octet: lane & 3 adds lanes (lane & 3) * 8 .. + 7, then the quad
+    // row j = lane / 8: lane % 8 adds lanes 4 (lane % 8) .. + 3, then the eight
     float t = 0.f;
     {
-      const float* rp = red + (lane >> 2) * kRedRow + (lane & 3) * 8;
+      const float* rp = red + (lane >> 3) * kRedRow + (lane & 7) * 4;
 #pragma unroll
-      for (int k = 0; k < 8; ++k) t += rp[k];
+      for (int k = 0; k < 4; ++k) t += rp[k];
     }
     t += __shfl_xor_sync(0xffffffffu, t, 1);
     t += __shfl_xor_sync(0xffffffffu, t, 2);
-    __syncwarp();  // the scratch is free for the warp's next unit
-    const int rowo = row0 + (lane >> 2);
-    if ((lane & 3) == 0 && rowo < n_out) g.zp[(int64_t)kc * n_out + rowo] = t;
+    t += __shfl_xor_sync(0xffffffffu, t, 4);
+    __syncwarp();  // the scratch is free for the next rows
+    {
+      const int j = lane >> 3, row = tile[j >> 1] * 32 + rw + 16 * (j & 1);
+      if ((lane & 7) == 0 && (j >> 1) < nb && row < n_out) g.zp[(int64_t)kc * n_out + row] = t;
+    }
     if constexpr (TICKETS) {
       // the partials are visible device-wide before the block's ticket counts them; the
       // CTA that brings the count to per_block runs the block's chain after this phase
       __threadfence();
       __syncwarp();
-      if (lane == 0) {
-        const int blk = tile * 32 / wb;
+      if (lane < nb) {
+        const int blk = tile[lane] * 32 / wb;
         unsigned old;
         asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(tickets + blk) : "memory");
         if (old + 1 == per_block) {
@@ -737,6 +771,7 @@ __device__ __noinline__ bool run_units(const Params& p, Smem& s, const Range& g,
         }
       }
     }
+    i += nb;
   }
   kring += (uint32_t)nu;
   return cbar_and(true);
@@ -753,8 +788,7 @@ __device__ __forceinline__ void prefetch_next(const Params& p, Smem& s, int l, i
     ph = 0;
     if (++l >= p.L) return;
   }
-  const int warp = ct >> 5;
-  prefetch_rows<BITS>(range_of(q, l, ph), k0, warp / kQuadWarps, warp % kQuadWarps, ct & 31);
+  prefetch_rows<BITS>(range_of(q, l, ph), k0, ct >> 5, ct & 31);
 }
 
 // ------------------------------------------------------------------ grid barrier
@@ -934,7 +968,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   const int ct = tid;
   // the first GEMV phase's weights into L2 while the first chain runs
   if (p.pf_dist > 0)
-    prefetch_rows<BITS>(range_of(*s.plan, 0, 0), 0, (ct >> 5) / kQuadWarps, (ct >> 5) % kQuadWarps, ct & 31);
+    prefetch_rows<BITS>(range_of(*s.plan, 0, 0), 0, ct >> 5, ct & 31);
   uint32_t kring = 0;
   Xch X;
   float res[2] = {0.f, 0.f};  // the residual stream, this CTA's layout-B share
@@ -968,9 +1002,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     prefetch_next<BITS>(p, s, l, 2, kring, ct);
     if (p.mlp_tickets) {
       const int wb = lin[4].w_out;
-      const unsigned per_block = (unsigned)(2 * (wb / 32) * p.nk_h * kQuadWarps);
+      const unsigned per_block = (unsigned)(2 * (wb / 32) * p.nk_h * kCW);
       unsigned* tickets = p.counters + 5 * L + (size_t)l * p.nblocks;
-      if (!(ok = run_units<BITS, true>(p, s, range_of(*s.plan, l, 2), kring, ct, tickets, per_block, wb))) break;
+      if (!(ok = run_units<BITS, true>(p, s, range_of(*s.plan, l, 2), kring, ct, nullptr, tickets, per_block, wb))) break;
       // P7 for the MLP blocks this CTA completed (their partials are all written)
       const int nw = min(s.won[0], kMaxWon);
       if (s.won[0] > kMaxWon) report(p.status, 6, 70);  // cannot happen: a CTA's units span few blocks
@@ -993,22 +1027,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       }
     }
     if (!(ok = grid_barrier(p, l * 5 + 3, ct))) break;
-    // P8: the down projection's operand from global
+    // P8: the down projection, its operand read from the global buffer the MLP blocks wrote
     {
-      const int n_in = lin[6].n_in, ng = n_in / 64;
-      const int words = BITS == 3 ? n_in : n_in / 2;
-      const int4* src = reinterpret_cast<const int4*>(p.xq_down);
-      int4* dst = reinterpret_cast<int4*>(s.xq);
-      for (int i = ct; i < words / 4; i += kNT) dst[i] = __ldcg(src + i);
-      float* xsA = reinterpret_cast<float*>(s.xq + words);
-      for (int g = ct; g < ng; g += kNT) {
-        xsA[g] = __ldcg(p.xs_down + g);
-        xsA[ng + g] = __ldcg(p.xsum_down + g);
-      }
-      cbar();
       if (ct == 0 && p.tm != kTmHad) prefetch_chain(p, l, 3, c, r);
       prefetch_next<BITS>(p, s, l, 3, kring, ct);
-      if (!(ok = run_units<BITS>(p, s, range_of(*s.plan, l, 3), kring, ct))) break;
+      if (!(ok = run_units<BITS>(p, s, range_of(*s.plan, l, 3), kring, ct, p.xq_down))) break;
     }
     if (!(ok = grid_barrier(p, l * 5 + 4, ct))) break;
   }
