@@ -346,6 +346,48 @@ template <int EB, int TM>
 __device__ __noinline__ void mlp_block_local(const Params& p, Smem& sm, const Lin* Lg, const Lin* Lu, const Lin* Ld,
                                              int blk, int ct) {
   using M = Map<EB>;
+  if constexpr (2 * M::E <= kNT) {
+    // blocks up to 256 wide: F_U(gate) on threads [0, E) and F_U(up) on [E, 2E) at once,
+    // each half with its own transpose buffer; the up half then hands its values over
+    const bool up = ct >= M::E;
+    const int cl = up ? ct - M::E : ct;  // the thread within its half (>= E: idle)
+    const Lin* Lx = up ? Lu : Lg;
+    LocalBfly<EB, TM> fx, fd;
+    fetch_side(fx, Lx->rU, Lx->tU, (int64_t)Lx->n_out / 2, blk, cl);
+    if (!up) fetch_side(fd, Ld->rV, Ld->tV, (int64_t)Ld->n_in / 2, blk, cl);
+    const bool act = cl < M::NT;
+    const int64_t base = (int64_t)blk * M::E;
+    float v = 0.f, sd = 0.f;
+    if (act) {
+      const int64_t g = base + M::e1(cl, 0);
+      v = zsum(up ? p.zpu : p.zpg, p.nk_h, Lx->n_out, g) * (float)__ldg(Lx->sU + g);
+      if (!up) sd = (float)__ldg(Ld->sV + base + M::e2(cl, 0));  // F_V_down's sign, read up front
+    }
+    EngCtx half = sm;
+    if (up) half.T += 512;
+    fx.run(v, half, cl);
+    cbar();  // the gate half has read its transpose buffer
+    if (act && up) sm.T[idx_a(M::e2(cl, 0))] = v;  // both halves hold phase-2 order
+    cbar();
+    float h = 0.f;
+    if (act && !up) h = silu(v) * sm.T[idx_a(M::e2(cl, 0))] * sd;
+    cbar();
+    if (act && !up) sm.T[idx_a(M::e2(cl, 0))] = h;
+    cbar();
+    if (act && !up) h = sm.T[idx_a(M::e1(cl, 0))];
+    fd.run(h, sm, up ? M::NT : cl);  // F_V_down from phase-1 order, on the gate half
+    cbar();
+    if (act && !up) sm.T[M::e2(cl, 0)] = h;  // natural order for the groups
+    cbar();
+    const int warp = ct >> 5, lane = ct & 31, n_in = Ld->n_in;
+    int16_t* xq16 = reinterpret_cast<int16_t*>(p.xq_down);
+    if (warp < (M::E >> 6)) {
+      const int G = (int)(base >> 6) + warp;
+      prep_group(sm.T + 64 * warp, p.bits, xq16 + (int64_t)G * 64, xq16 + n_in + (int64_t)G * 64, p.xs_down + G,
+                 p.xsum_down + G, lane, G & 7);
+    }
+    return;
+  }
   LocalBfly<EB, TM> fg, fu, fd;
   fetch_side(fg, Lg->rU, Lg->tU, (int64_t)Lg->n_out / 2, blk, ct);
   fetch_side(fu, Lu->rU, Lu->tU, (int64_t)Lu->n_out / 2, blk, ct);
@@ -796,8 +838,9 @@ __device__ __noinline__ bool grid_barrier(const Params& p, int idx, int ct) {
   cbar();
   bool mine = true;
   if (ct == 0) {
+    // the CTA barrier above orders every thread's writes before this release, which makes
+    // them visible with the count at gpu scope (no separate fence)
     unsigned* c = p.counters + idx;
-    __threadfence();
     asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(c) : "memory");
     const unsigned target = (unsigned)(p.G * kC) + (idx == p.barrier_extra ? 1u : 0u);  // + testing hook
     const long long t0 = clock64();
