@@ -12,8 +12,7 @@
 //    adds up in a fixed order. Each of the 16 warps takes two rows of every unit; a
 //    lane holds one group of 64 input columns, with its operand words in registers, and
 //    loads that group's codes and scale/zero words of its rows straight from L2 (a warp
-//    reads each row's chunk as one contiguous span). The down projection reads its
-//    operand from the global buffer the MLP blocks wrote.
+//    reads each row's chunk as one contiguous span).
 //  * CTAs form clusters of 8. Each cluster computes the activation chain between two
 //    GEMVs itself (redundantly with the other clusters): a w-wide butterfly is spread
 //    over the 8 CTAs, w/8 elements each. Every consumer thread holds one (two when
@@ -46,7 +45,7 @@
 //   P7 MLP blocks (one CTA each up to 512 wide, one cluster each from 2048): F_U_gate,
 //      F_U_up, silu*up, F_V_down, operand to global; the two last clusters apply F_U_q
 //      and F_U_k of this block                  -> grid barrier
-//   P8 GEMV down (operand from global)          -> grid barrier
+//   P8 GEMV down                                -> grid barrier
 // and after the last block: out = h_{L-1} + F_U_down(z_down).
 //
 // Every wait is bounded (about 2 s of SM clock unless the testing hook shortens it) and
@@ -658,7 +657,7 @@ __device__ __forceinline__ void load_row(RowW<BITS>& w, const Range& g, int row,
 // exact integer dot product of one row's group with the operand words x of that group;
 // xh: the 1-bit plane's operand (3-bit)
 template <int BITS>
-__device__ __forceinline__ int row_dot(const RowW<BITS>& rw, const int4 (&x)[8], const int4* xh, int G, bool xg) {
+__device__ __forceinline__ int row_dot(const RowW<BITS>& rw, const int4 (&x)[8], const int4* xh, int G) {
   if constexpr (BITS == 2 || BITS == 3) {
     const uint32_t wv[4] = {rw.c[0].x, rw.c[0].y, rw.c[0].z, rw.c[0].w};
     int a0 = 0, a1 = 0, a2 = 0, a3 = 0, b0 = 0, b1 = 0, b2 = 0, b3 = 0;
@@ -684,7 +683,7 @@ __device__ __forceinline__ int row_dot(const RowW<BITS>& rw, const int4 (&x)[8],
       for (int k = 0; k < 2; ++k) {
 #pragma unroll
         for (int mm = 0; mm < 8; mm += 2) {
-          const int4 xa = xg ? __ldcg(xh + xq_chunk(G, 4 * k + mm / 2)) : xh[xq_chunk(G, 4 * k + mm / 2)];
+          const int4 xa = xh[xq_chunk(G, 4 * k + mm / 2)];
           const uint32_t ma = hv[k] & (0x01010101u << mm), mb = hv[k] & (0x01010101u << (mm + 1));
           int ha = 0, hb = 0;
           ha = dp2a_lo(xa.x, ma, ha);
@@ -717,19 +716,15 @@ __device__ __forceinline__ int row_dot(const RowW<BITS>& rw, const int4 (&x)[8],
 // this block; per_block: (unit, warp) items of one MLP block's gate and up rows
 template <int BITS, bool TICKETS = false>
 __device__ __noinline__ bool run_units(const Params& p, Smem& s, const Range& g, uint32_t& kring, int ct,
-                                          const int32_t* xglob = nullptr, unsigned* tickets = nullptr,
-                                          unsigned per_block = 0, int wb = 0) {
+                                          unsigned* tickets = nullptr, unsigned per_block = 0, int wb = 0) {
   using Gm = FGeo<BITS>;
   const int warp = ct >> 5, lane = ct & 31;
   const int n_out = g.n_out, n_in = g.n_in, ngroups = n_in / 64;
   const int words = BITS == 3 ? n_in : n_in / 2;
-  // the operand: shared memory, or (xglob) the global buffer another phase of this kernel
-  // wrote, read through L2
-  const int32_t* xw = xglob ? xglob : s.xq;
-  const float* xsA = xglob ? p.xs_down : reinterpret_cast<const float*>(s.xq + words);
-  const float* xsumA = xglob ? p.xsum_down : xsA + ngroups;
-  const int4* xlo = reinterpret_cast<const int4*>(xw);
-  const int4* xhi = reinterpret_cast<const int4*>(xw + n_in / 2);
+  const float* xsA = reinterpret_cast<const float*>(s.xq + words);
+  const float* xsumA = xsA + ngroups;
+  const int4* xlo = reinterpret_cast<const int4*>(s.xq);
+  const int4* xhi = reinterpret_cast<const int4*>(s.xq + n_in / 2);
   const int nu = g.u1 - g.u0;
   // rows rw and rw + 16 of every unit; the mapping turns with the CTA's unit count so that
   // no warp keeps the same rows phase after phase
@@ -759,9 +754,9 @@ __device__ __noinline__ bool run_units(const Params& p, Smem& s, const Range& g,
       kc_have = kc;
       if (act) {
 #pragma unroll
-        for (int k = 0; k < 8; ++k) xr[k] = xglob ? __ldcg(xlo + xq_chunk(G, k)) : xlo[xq_chunk(G, k)];
-        xs = xglob ? __ldcg(xsA + G) : xsA[G];
-        xsum = xglob ? __ldcg(xsumA + G) : xsumA[G];
+        for (int k = 0; k < 8; ++k) xr[k] = xlo[xq_chunk(G, k)];
+        xs = xsA[G];
+        xsum = xsumA[G];
       }
     }
     RowW<BITS> w[4];
@@ -777,7 +772,7 @@ __device__ __noinline__ bool run_units(const Params& p, Smem& s, const Range& g,
       if ((j >> 1) < nb && act && row < n_out) {
         const float s16 = __half2float(__ushort_as_half((unsigned short)(w[j].sz & 0xffffu)));
         const float z16 = __half2float(__ushort_as_half((unsigned short)(w[j].sz >> 16)));
-        const int acc = row_dot<BITS>(w[j], xr, xhi, G, xglob != nullptr);
+        const int acc = row_dot<BITS>(w[j], xr, xhi, G);
         z = fmaf(s16, (float)acc * xs, z16 * xsum);
       }
       red[j * kRedRow + lane] = z;
@@ -1047,7 +1042,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       const int wb = lin[4].w_out;
       const unsigned per_block = (unsigned)(2 * (wb / 32) * p.nk_h * kCW);
       unsigned* tickets = p.counters + 5 * L + (size_t)l * p.nblocks;
-      if (!(ok = run_units<BITS, true>(p, s, range_of(*s.plan, l, 2), kring, ct, nullptr, tickets, per_block, wb))) break;
+      if (!(ok = run_units<BITS, true>(p, s, range_of(*s.plan, l, 2), kring, ct, tickets, per_block, wb))) break;
       // P7 for the MLP blocks this CTA completed (their partials are all written)
       const int nw = min(s.won[0], kMaxWon);
       if (s.won[0] > kMaxWon) report(p.status, 6, 70);  // cannot happen: a CTA's units span few blocks
@@ -1070,11 +1065,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       }
     }
     if (!(ok = grid_barrier(p, l * 5 + 3, ct))) break;
-    // P8: the down projection, its operand read from the global buffer the MLP blocks wrote
+    // P8: the down projection's operand from global into shared memory, then the GEMV
     {
+      const int n_in = lin[6].n_in, ng = n_in / 64;
+      const int words = BITS == 3 ? n_in : n_in / 2;
+      const int4* src = reinterpret_cast<const int4*>(p.xq_down);
+      int4* dst = reinterpret_cast<int4*>(s.xq);
+      for (int i = ct; i < words / 4; i += kNT) dst[i] = __ldcg(src + i);
+      float* xsA = reinterpret_cast<float*>(s.xq + words);
+      for (int g = ct; g < ng; g += kNT) {
+        xsA[g] = __ldcg(p.xs_down + g);
+        xsA[ng + g] = __ldcg(p.xsum_down + g);
+      }
+      cbar();
       if (ct == 0 && p.tm != kTmHad) prefetch_chain(p, l, 3, c, r);
       prefetch_next<BITS>(p, s, l, 3, kring, ct);
-      if (!(ok = run_units<BITS>(p, s, range_of(*s.plan, l, 3), kring, ct, p.xq_down))) break;
+      if (!(ok = run_units<BITS>(p, s, range_of(*s.plan, l, 3), kring, ct))) break;
     }
     if (!(ok = grid_barrier(p, l * 5 + 4, ct))) break;
   }
