@@ -1020,7 +1020,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                                 ct)))
       break;
     // P2 (L2 requests for the tables of the chain that follows, as every GEMV phase)
-    if (ct == 0 && p.tm != kTmHad) prefetch_chain(p, l, 0, c, r);
+    if (ct == 0 && p.table_pf && p.tm != kTmHad) prefetch_chain(p, l, 0, c, r);
     prefetch_next<BITS>(p, s, l, 0, kring, ct);
     if (!(ok = run_units<BITS>(p, s, range_of(*s.plan, l, 0), kring, ct))) break;
     if (!(ok = grid_barrier(p, l * 5 + 0, ct))) break;
@@ -1029,14 +1029,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                             : attn_eb<TM, 9>(p, s, X, lin + 2, lin + 3, r, ct)))
       break;
     // P4
-    if (ct == 0 && p.tm != kTmHad) prefetch_chain(p, l, 1, c, r);
+    if (ct == 0 && p.table_pf && p.tm != kTmHad) prefetch_chain(p, l, 1, c, r);
     prefetch_next<BITS>(p, s, l, 1, kring, ct);
     if (!(ok = run_units<BITS>(p, s, range_of(*s.plan, l, 1), kring, ct))) break;
     if (!(ok = grid_barrier(p, l * 5 + 1, ct))) break;
     // P5
     if (!(ok = residual_any<TM>(p, s, X, res, lin + 3, p.zpo, p.nk_h, lin + 4 + p.asg_gu[c], r, ct))) break;
     // P6
-    if (ct == 0 && p.tm != kTmHad) prefetch_chain(p, l, 2, c, r);
+    if (ct == 0 && p.table_pf && p.tm != kTmHad) prefetch_chain(p, l, 2, c, r);
     prefetch_next<BITS>(p, s, l, 2, kring, ct);
     if (p.mlp_tickets) {
       const int wb = lin[4].w_out;
@@ -1078,7 +1078,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         xsA[ng + g] = __ldcg(p.xsum_down + g);
       }
       cbar();
-      if (ct == 0 && p.tm != kTmHad) prefetch_chain(p, l, 3, c, r);
+      if (ct == 0 && p.table_pf && p.tm != kTmHad) prefetch_chain(p, l, 3, c, r);
       prefetch_next<BITS>(p, s, l, 3, kring, ct);
       if (!(ok = run_units<BITS>(p, s, range_of(*s.plan, l, 3), kring, ct))) break;
     }

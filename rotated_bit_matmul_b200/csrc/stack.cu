@@ -279,10 +279,15 @@ void setup_fused(harp_stack_s* S) {
   int optin = 0;
   cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, S->device);
   if (dec::smem_for(p) > (size_t)optin) return no("not enough shared memory for the operand");
-  // HARP_PF_DIST=0 turns off the L2 requests for the next GEMV phase's weights; cooperative
-  // launch unless HARP_COOPERATIVE=0
-  p.pf_dist = 1;
+  // HARP_PF_DIST=1: each GEMV phase asks for the next phase's weights in L2 (per-lane line
+  // prefetches). Off by default: the burst of requests stalls the issuing warps for longer
+  // than the L2 hits save (same-box A/B: 2.924 ms/step without, 3.101 ms with).
+  // HARP_TABLE_PF=0: no bulk L2 requests for the next chain's tables. Cooperative launch
+  // unless HARP_COOPERATIVE=0.
+  p.pf_dist = 0;
   if (const char* e = getenv("HARP_PF_DIST")) p.pf_dist = std::max(0, atoi(e));
+  p.table_pf = 1;
+  if (const char* e = getenv("HARP_TABLE_PF")) p.table_pf = atoi(e) != 0;
   p.cooperative = 1;
   if (const char* e = getenv("HARP_COOPERATIVE")) p.cooperative = atoi(e) != 0;
   // HARP_MLP_TICKETS=1 (MLP blocks up to 512 wide): the chain runs where the block's last
