@@ -828,9 +828,44 @@ __device__ __forceinline__ void prefetch_next(const Params& p, Smem& s, int l, i
   prefetch_rows<BITS>(range_of(q, l, ph), k0, ct >> 5, ct & 31);
 }
 
+// This CTA's rows of GEMV phase (l, ph) into L2, spread over the lanes of warps 1..15 while
+// thread 0 polls a grid barrier (those warps would only wait): line by line, codes and
+// 1-bit plane of each row's chunk, then its scale/zero words.
+template <int BITS>
+__device__ __forceinline__ void prefetch_phase_l2(const Params& p, const Smem& s, int l, int ph, int ct) {
+  using Gm = FGeo<BITS>;
+  if (l >= p.L) return;
+  const Range g = range_of(*s.plan, l, ph);
+  const int ngroups = g.n_in / 64, row_bytes = ngroups * Gm::kGroupBytes;
+  constexpr int kLines = 2048 * (BITS == 4 ? 4 : 2) / 8 / 128 + (BITS == 3 ? 2 : 0) + 1;  // per row of a chunk
+  const int per_unit = 32 * kLines;
+  for (int it = ct - 32; it < (g.u1 - g.u0) * per_unit; it += kNT - 32) {
+    const int i = it / per_unit, rest = it - i * per_unit, row_in = rest / kLines, ln = rest - row_in * kLines;
+    int tile, kc;
+    g.tk(g.u0 + i, tile, kc);
+    const int row = tile * 32 + row_in;
+    if (row >= g.n_out) continue;
+    const int g0 = kc * Gm::kChunkGroups, gc = min(Gm::kChunkGroups, ngroups - g0);
+    constexpr int kCodeLines = 2048 * (BITS == 4 ? 4 : 2) / 8 / 128;
+    if (ln < kCodeLines) {
+      if (ln * 128 < gc * Gm::kGroupBytes)
+        prefetch_line_l2(g.L->codes + (size_t)row * row_bytes + (size_t)g0 * Gm::kGroupBytes + ln * 128);
+    } else if (BITS == 3 && ln < kCodeLines + 2) {
+      if ((ln - kCodeLines) * 128 < gc * 8)
+        prefetch_line_l2(g.L->hi + (size_t)row * (ngroups * 8) + (size_t)g0 * 8 + (ln - kCodeLines) * 128);
+    } else {
+      prefetch_line_l2(g.L->sz + (size_t)row * ngroups + g0);
+    }
+  }
+}
+
 // ------------------------------------------------------------------ grid barrier
-__device__ __noinline__ bool grid_barrier(const Params& p, int idx, int ct) {
+// pf_l, pf_ph: a GEMV phase whose rows warps 1..15 ask for in L2 meanwhile (pf_l < 0: none)
+template <int BITS>
+__device__ __noinline__ bool grid_barrier(const Params& p, const Smem& s, int idx, int ct, int pf_l = -1,
+                                          int pf_ph = 0) {
   cbar();
+  if (ct >= 32 && pf_l >= 0 && p.bar_pf) prefetch_phase_l2<BITS>(p, s, pf_l, pf_ph, ct);
   bool mine = true;
   if (ct == 0) {
     // the CTA barrier above orders every thread's writes before this release, which makes
@@ -1023,7 +1058,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     if (ct == 0 && p.table_pf && p.tm != kTmHad) prefetch_chain(p, l, 0, c, r);
     prefetch_next<BITS>(p, s, l, 0, kring, ct);
     if (!(ok = run_units<BITS>(p, s, range_of(*s.plan, l, 0), kring, ct))) break;
-    if (!(ok = grid_barrier(p, l * 5 + 0, ct))) break;
+    if (!(ok = grid_barrier<BITS>(p, s, l * 5 + 0, ct, l, 1))) break;
     // P3
     if (!(ok = p.eb_h == 10 ? attn_eb<TM, 10>(p, s, X, lin + 2, lin + 3, r, ct)
                             : attn_eb<TM, 9>(p, s, X, lin + 2, lin + 3, r, ct)))
@@ -1032,7 +1067,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     if (ct == 0 && p.table_pf && p.tm != kTmHad) prefetch_chain(p, l, 1, c, r);
     prefetch_next<BITS>(p, s, l, 1, kring, ct);
     if (!(ok = run_units<BITS>(p, s, range_of(*s.plan, l, 1), kring, ct))) break;
-    if (!(ok = grid_barrier(p, l * 5 + 1, ct))) break;
+    if (!(ok = grid_barrier<BITS>(p, s, l * 5 + 1, ct, l, 2))) break;
     // P5
     if (!(ok = residual_any<TM>(p, s, X, res, lin + 3, p.zpo, p.nk_h, lin + 4 + p.asg_gu[c], r, ct))) break;
     // P6
@@ -1051,7 +1086,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       if (ct == 0) s.won[0] = 0;
     } else {
       if (!(ok = run_units<BITS>(p, s, range_of(*s.plan, l, 2), kring, ct))) break;
-      if (!(ok = grid_barrier(p, l * 5 + 2, ct))) break;
+      if (!(ok = grid_barrier<BITS>(p, s, l * 5 + 2, ct, l, 3))) break;
       // P7
       if (!(ok = mlp_any<TM>(p, s, X, lin, c, r, ct))) break;
     }
@@ -1064,7 +1099,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         if (!(ok = out_only_any<TM>(p, s, X, qk == 0 ? p.eb_h : p.eb_kv, lin + qk, zp, out, r, ct))) break;
       }
     }
-    if (!(ok = grid_barrier(p, l * 5 + 3, ct))) break;
+    if (!(ok = grid_barrier<BITS>(p, s, l * 5 + 3, ct))) break;
     // P8: the down projection's operand from global into shared memory, then the GEMV
     {
       const int n_in = lin[6].n_in, ng = n_in / 64;
@@ -1082,7 +1117,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       prefetch_next<BITS>(p, s, l, 3, kring, ct);
       if (!(ok = run_units<BITS>(p, s, range_of(*s.plan, l, 3), kring, ct))) break;
     }
-    if (!(ok = grid_barrier(p, l * 5 + 4, ct))) break;
+    if (!(ok = grid_barrier<BITS>(p, s, l * 5 + 4, ct, l + 1, 0))) break;
   }
   // final: out = h_{L-1} + F_U_down(z_down)
   if (ok) {

@@ -61,6 +61,7 @@ struct Params {
   int xq_bytes;
   int pf_dist;      // nonzero: each GEMV phase asks for the next phase's weights in L2
   int table_pf;     // nonzero: each GEMV phase asks for the next chain's tables in L2
+  int bar_pf;       // nonzero: while a grid barrier polls, the idle warps ask for the next GEMV phase's rows in L2
   int cooperative;  // launch with the cooperative attribute (all CTAs co-resident or refused)
   int asg_qkv[kMaxClusters], idx_qkv[kMaxClusters], cnt_qkv[3];
   int asg_gu[kMaxClusters], idx_gu[kMaxClusters], cnt_gu[2];

@@ -288,6 +288,10 @@ void setup_fused(harp_stack_s* S) {
   if (const char* e = getenv("HARP_PF_DIST")) p.pf_dist = std::max(0, atoi(e));
   p.table_pf = 1;
   if (const char* e = getenv("HARP_TABLE_PF")) p.table_pf = atoi(e) != 0;
+  // HARP_BAR_PF=0: the warps idle at a grid barrier do not ask for the next GEMV phase's
+  // rows in L2
+  p.bar_pf = 1;
+  if (const char* e = getenv("HARP_BAR_PF")) p.bar_pf = atoi(e) != 0;
   p.cooperative = 1;
   if (const char* e = getenv("HARP_COOPERATIVE")) p.cooperative = atoi(e) != 0;
   // HARP_MLP_TICKETS=1 (MLP blocks up to 512 wide): the chain runs where the block's last
