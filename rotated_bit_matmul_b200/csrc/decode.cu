@@ -72,11 +72,9 @@ struct FGeo {
 };
 
 // ------------------------------------------------------------------ shared memory carve-up
-constexpr int kMaxWon = 16;  // MLP blocks one CTA can complete in a block's gate/up phase
 
 struct Smem : EngCtx {
   float* misc;     // [0, 8) rms partials by source CTA, [8, 24) per-warp scratch
-  int* won;        // [0]: count, then up to kMaxWon MLP blocks whose last unit this CTA completed
   int32_t* xq;     // GEMV operand: xq words, then xs [ng], then xsum [ng]
   float* red;      // GEMV row partials: 16 warps x 8 rows x 33 (32 lanes, padded)
   struct Plan* plan;
@@ -93,8 +91,6 @@ __device__ __forceinline__ Smem carve(const Params& p) {
   s.rx[1] = reinterpret_cast<float*>(b);
   b += 4 * kRxFloats;
   s.misc = reinterpret_cast<float*>(b);
-  b += 4 * 32;
-  s.won = reinterpret_cast<int*>(b);
   b += 4 * 32;
   s.xq = reinterpret_cast<int32_t*>(b);
   b += p.xq_bytes;
@@ -712,11 +708,8 @@ __device__ __forceinline__ int row_dot(const RowW<BITS>& rw, const int4 (&x)[8],
   }
 }
 
-// tickets: with MLP-block tickets in the gate/up phase, the per-block completion counters of
-// this block; per_block: (unit, warp) items of one MLP block's gate and up rows
-template <int BITS, bool TICKETS = false>
-__device__ __noinline__ bool run_units(const Params& p, Smem& s, const Range& g, uint32_t& kring, int ct,
-                                          unsigned* tickets = nullptr, unsigned per_block = 0, int wb = 0) {
+template <int BITS>
+__device__ __noinline__ bool run_units(const Params& p, Smem& s, const Range& g, uint32_t& kring, int ct) {
   using Gm = FGeo<BITS>;
   const int warp = ct >> 5, lane = ct & 31;
   const int n_out = g.n_out, n_in = g.n_in, ngroups = n_in / 64;
@@ -793,21 +786,6 @@ __device__ __noinline__ bool run_units(const Params& p, Smem& s, const Range& g,
       const int j = lane >> 3, row = tile[j >> 1] * 32 + rw + 16 * (j & 1);
       if ((lane & 7) == 0 && (j >> 1) < nb && row < n_out) g.zp[(int64_t)kc * n_out + row] = t;
     }
-    if constexpr (TICKETS) {
-      // the partials are visible device-wide before the block's ticket counts them; the
-      // CTA that brings the count to per_block runs the block's chain after this phase
-      __threadfence();
-      __syncwarp();
-      if (lane < nb) {
-        const int blk = tile[lane] * 32 / wb;
-        unsigned old;
-        asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(tickets + blk) : "memory");
-        if (old + 1 == per_block) {
-          const int k = atomicAdd(&s.won[0], 1);
-          if (k < kMaxWon) s.won[1 + k] = blk;
-        }
-      }
-    }
     i += nb;
   }
   kring += (uint32_t)nu;
@@ -857,6 +835,33 @@ __device__ __forceinline__ void prefetch_phase_l2(const Params& p, const Smem& s
       prefetch_line_l2(g.L->sz + (size_t)row * ngroups + g0);
     }
   }
+}
+
+// ------------------------------------------------------------------ waits on global counters
+// CTA-wide: thread 0 polls until *c >= target (acquire), bounded like every wait here
+__device__ __noinline__ bool wait_count(const Params& p, const unsigned* c, unsigned target, int where, int ct) {
+  bool mine = true;
+  if (ct == 0) {
+    const long long t0 = clock64();
+    for (uint32_t it = 0;; ++it) {
+      unsigned v;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(c) : "memory");
+      if (v >= target) break;
+      if ((it & 15) == 15) {
+        const long long dt = clock64() - t0;
+        if (dt > kAbortCheckCycles && aborted(p.status)) {
+          mine = false;
+          break;
+        }
+        if (dt > s_wait_cycles) {
+          report(p.status, 5, where);
+          mine = false;
+          break;
+        }
+      }
+    }
+  }
+  return cbar_and(mine);
 }
 
 // ------------------------------------------------------------------ grid barrier
@@ -1030,7 +1035,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   if (tid == 0) {
     make_plan<BITS>(p, c, (int)r, *s.plan);
     s_wait_cycles = p.wait_cycles;
-    s.won[0] = 0;
     mbar_init(&s.xbar[0], 1);
     mbar_init(&s.xbar[1], 1);
     fence_mbar_init();
@@ -1073,17 +1077,40 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     // P6
     if (ct == 0 && p.table_pf && p.tm != kTmHad) prefetch_chain(p, l, 2, c, r);
     prefetch_next<BITS>(p, s, l, 2, kring, ct);
-    if (p.mlp_tickets) {
+    if (p.mlp_ready) {
+      // no grid barrier: each CTA adds its gate/up units, once they are all written, to the
+      // counters of the MLP blocks they belong to (one fence for the lot), and CTA b runs
+      // MLP block b as soon as its count reaches the block's 2 x wb/32 x nk units
+      const Range g6 = range_of(*s.plan, l, 2);
+      if (!(ok = run_units<BITS>(p, s, g6, kring, ct))) break;
       const int wb = lin[4].w_out;
-      const unsigned per_block = (unsigned)(2 * (wb / 32) * p.nk_h * kCW);
-      unsigned* tickets = p.counters + 5 * L + (size_t)l * p.nblocks;
-      if (!(ok = run_units<BITS, true>(p, s, range_of(*s.plan, l, 2), kring, ct, tickets, per_block, wb))) break;
-      // P7 for the MLP blocks this CTA completed (their partials are all written)
-      const int nw = min(s.won[0], kMaxWon);
-      if (s.won[0] > kMaxWon) report(p.status, 6, 70);  // cannot happen: a CTA's units span few blocks
-      for (int i = 0; i < nw; ++i) mlp_local_blk<TM>(p, s, lin, s.won[1 + i], ct);
-      cbar();
-      if (ct == 0) s.won[0] = 0;
+      unsigned* ready = p.counters + 5 * L + (size_t)l * p.nblocks;
+      if (ct == 0) {
+        __threadfence();
+        int cur = -1;
+        unsigned cnt = 0;
+        for (int u = g6.u0; u <= g6.u1; ++u) {
+          int b = -2;
+          if (u < g6.u1) {
+            int tile, kc;
+            g6.tk(u, tile, kc);
+            b = tile * 32 / wb;
+          }
+          if (b != cur) {
+            if (cnt) asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(ready + cur), "r"(cnt) : "memory");
+            cur = b;
+            cnt = 0;
+          }
+          ++cnt;
+        }
+      }
+      const int t_cta = c * kC + (int)r;
+      if (t_cta < p.nblocks) {
+        if (!(ok = wait_count(p, ready + t_cta, (unsigned)(2 * (wb / 32) * p.nk_h), 70, ct))) break;
+        mlp_local_blk<TM>(p, s, lin, t_cta, ct);
+      } else if (ct >= 32 && p.bar_pf) {
+        prefetch_phase_l2<BITS>(p, s, l, 3, ct);  // idle until the MLP blocks are done
+      }
     } else {
       if (!(ok = run_units<BITS>(p, s, range_of(*s.plan, l, 2), kring, ct))) break;
       if (!(ok = grid_barrier<BITS>(p, s, l * 5 + 2, ct, l, 3))) break;
@@ -1171,7 +1198,7 @@ cudaError_t repack_side(int tm, int eb, bool cluster, int nblk, const uint8_t* t
 // ------------------------------------------------------------------ host side
 template <int BITS>
 size_t smem_bytes(const Params& p) {
-  return 16 + 3 * 4 * (size_t)kRxFloats + 4 * 32 + 4 * 32 + p.xq_bytes + 4 * kCW * 8 * 33 + 512 + 8 * 2;
+  return 16 + 3 * 4 * (size_t)kRxFloats + 4 * 32 + p.xq_bytes + 4 * kCW * 8 * 33 + 512 + 8 * 2;
 }
 
 template <int BITS>

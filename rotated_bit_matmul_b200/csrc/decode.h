@@ -53,7 +53,7 @@ struct Params {
   float* xs_down;
   float* xsum_down;
   unsigned* counters;  // [L][5] grid barriers, then [L][nblocks] MLP-block tickets; zero at launch
-  int mlp_tickets;     // 1: an MLP block's chain runs in the CTA that completes its last gate/up unit
+  int mlp_ready;       // 1: CTA b runs MLP block b once its counter says the block's gate/up rows are in (no grid barrier)
   int* status;
   long long wait_cycles;  // bound of every wait, in SM clock cycles
   int barrier_extra;      // testing hook: grid barrier whose target is raised by one (-1: none)

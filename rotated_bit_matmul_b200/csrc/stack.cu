@@ -294,11 +294,11 @@ void setup_fused(harp_stack_s* S) {
   if (const char* e = getenv("HARP_BAR_PF")) p.bar_pf = atoi(e) != 0;
   p.cooperative = 1;
   if (const char* e = getenv("HARP_COOPERATIVE")) p.cooperative = atoi(e) != 0;
-  // HARP_MLP_TICKETS=1 (MLP blocks up to 512 wide): the chain runs where the block's last
-  // gate/up unit completes, one grid barrier less per block. Off by default: the chains then
-  // pile onto the CTAs that finish last, and the step measured slower than with the barrier.
-  p.mlp_tickets = 0;
-  if (const char* e = getenv("HARP_MLP_TICKETS")) p.mlp_tickets = wb <= 512 && F % 32 == 0 && atoi(e) != 0;
+  // MLP blocks up to 512 wide, one CTA each: CTA b starts block b's chain as soon as that
+  // block's gate and up rows are in (a counter per block that each CTA adds its units to
+  // once), without a grid barrier; HARP_MLP_READY=0 waits for the whole phase instead
+  p.mlp_ready = wb <= 512 && F % 32 == 0;
+  if (const char* e = getenv("HARP_MLP_READY")) p.mlp_ready = p.mlp_ready && atoi(e) != 0;
   int G = 0;
   cudaError_t e = dec::max_clusters(p, &G);
   if (e != cudaSuccess || G < 1)

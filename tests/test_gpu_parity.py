@@ -249,12 +249,13 @@ def test_stack_matches_oracle(dims, n_layers, block, batch):
 
 
 # ------------------------------------------------------------------ fused decode step
-@pytest.mark.parametrize("n_layers,bits,tickets", [(2, 2, 0), (1, 3, 0), (1, 4, 0), (2, 2, 1)])
-def test_fused_decode_step_matches_oracle(n_layers, bits, tickets, monkeypatch):
-    """The single-kernel batch-1 decode step on 7B-wide blocks against the oracle (tickets=1:
-    the opt-in variant whose MLP chains run in the CTA that completes a block's last unit)."""
+@pytest.mark.parametrize("n_layers,bits,ready", [(2, 2, 1), (1, 3, 1), (1, 4, 1), (2, 2, 0)])
+def test_fused_decode_step_matches_oracle(n_layers, bits, ready, monkeypatch):
+    """The single-kernel batch-1 decode step on 7B-wide blocks against the oracle (ready=1,
+    the default: each MLP block starts once its own gate/up rows are counted in; 0: after
+    a grid barrier)."""
     import rotated_bit_matmul_b200 as rb
-    monkeypatch.setenv("HARP_MLP_TICKETS", str(tickets))
+    monkeypatch.setenv("HARP_MLP_READY", str(ready))
     dims = (4096, 11008, 32, 32, 128)
     hidden, ffn = dims[0], dims[1]
     shapes = [(4096, hidden), (4096, hidden), (4096, hidden), (hidden, 4096), (ffn, hidden), (ffn, hidden),
