@@ -865,11 +865,13 @@ __device__ __noinline__ bool wait_count(const Params& p, const unsigned* c, unsi
 }
 
 // ------------------------------------------------------------------ grid barrier
-// pf_l, pf_ph: a GEMV phase whose rows warps 1..15 ask for in L2 meanwhile (pf_l < 0: none)
+// pf_l, pf_ph: a GEMV phase whose rows warps 1..15 ask for in L2 meanwhile (pf_l < 0: none);
+// synced: the caller has just passed a CTA barrier (a GEMV phase's end), so every thread's
+// writes are already ordered before thread 0's release
 template <int BITS>
 __device__ __noinline__ bool grid_barrier(const Params& p, const Smem& s, int idx, int ct, int pf_l = -1,
-                                          int pf_ph = 0) {
-  cbar();
+                                          int pf_ph = 0, bool synced = false) {
+  if (!synced) cbar();
   if (ct >= 32 && pf_l >= 0 && p.bar_pf) prefetch_phase_l2<BITS>(p, s, pf_l, pf_ph, ct);
   bool mine = true;
   if (ct == 0) {
@@ -1062,7 +1064,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     if (ct == 0 && p.table_pf && p.tm != kTmHad) prefetch_chain(p, l, 0, c, r);
     prefetch_next<BITS>(p, s, l, 0, kring, ct);
     if (!(ok = run_units<BITS>(p, s, range_of(*s.plan, l, 0), kring, ct))) break;
-    if (!(ok = grid_barrier<BITS>(p, s, l * 5 + 0, ct, l, 1))) break;
+    if (!(ok = grid_barrier<BITS>(p, s, l * 5 + 0, ct, l, 1, true))) break;
     // P3
     if (!(ok = p.eb_h == 10 ? attn_eb<TM, 10>(p, s, X, lin + 2, lin + 3, r, ct)
                             : attn_eb<TM, 9>(p, s, X, lin + 2, lin + 3, r, ct)))
@@ -1071,7 +1073,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     if (ct == 0 && p.table_pf && p.tm != kTmHad) prefetch_chain(p, l, 1, c, r);
     prefetch_next<BITS>(p, s, l, 1, kring, ct);
     if (!(ok = run_units<BITS>(p, s, range_of(*s.plan, l, 1), kring, ct))) break;
-    if (!(ok = grid_barrier<BITS>(p, s, l * 5 + 1, ct, l, 2))) break;
+    if (!(ok = grid_barrier<BITS>(p, s, l * 5 + 1, ct, l, 2, true))) break;
     // P5
     if (!(ok = residual_any<TM>(p, s, X, res, lin + 3, p.zpo, p.nk_h, lin + 4 + p.asg_gu[c], r, ct))) break;
     // P6
@@ -1113,7 +1115,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       }
     } else {
       if (!(ok = run_units<BITS>(p, s, range_of(*s.plan, l, 2), kring, ct))) break;
-      if (!(ok = grid_barrier<BITS>(p, s, l * 5 + 2, ct, l, 3))) break;
+      if (!(ok = grid_barrier<BITS>(p, s, l * 5 + 2, ct, l, 3, true))) break;
       // P7
       if (!(ok = mlp_any<TM>(p, s, X, lin, c, r, ct))) break;
     }
@@ -1144,7 +1146,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       prefetch_next<BITS>(p, s, l, 3, kring, ct);
       if (!(ok = run_units<BITS>(p, s, range_of(*s.plan, l, 3), kring, ct))) break;
     }
-    if (!(ok = grid_barrier<BITS>(p, s, l * 5 + 4, ct, l + 1, 0))) break;
+    if (!(ok = grid_barrier<BITS>(p, s, l * 5 + 4, ct, l + 1, 0, true))) break;
   }
   // final: out = h_{L-1} + F_U_down(z_down)
   if (ok) {
