@@ -83,11 +83,11 @@ def algorithmic_bytes_per_step(n_layers, batch=BATCH, bits=BITS):
 
 # DRAM bytes (read + write) of one fused decode launch per transformer block, from an
 # ncu capture of the 4-block stack (dram__bytes_read.sum + dram__bytes_write.sum, scaled
-# by blocks): 291.40 MB per 4-block launch with fp32 cos/sin tables (int8 angles: not
-# captured for these sources). With them, a hash of the kernel's sources at capture time:
-# the figures are reported only while those sources are unchanged.
-TRAFFIC_PER_BLOCK = {"bytes": {"fp32": 291_404_288 // 4, "int8": None},
-                     "sources_sha256_16": "7a655f9784ea80d5"}
+# by blocks): 278.45 MB per 4-block launch with fp32 cos/sin tables, 270.19 MB with int8
+# angles. With them, a hash of the kernel's sources at capture time: the figures are
+# reported only while those sources are unchanged.
+TRAFFIC_PER_BLOCK = {"bytes": {"fp32": 278_446_336 // 4, "int8": 270_192_384 // 4},
+                     "sources_sha256_16": "dbd501af0bd7bebb"}
 KERNEL_SOURCES = ("decode.cu", "decode.h", "common.cuh", "gemv_core.cuh", "bfly_engine.cuh")
 
 
