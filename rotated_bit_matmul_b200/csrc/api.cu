@@ -242,7 +242,8 @@ static harp_status mr_linear_forward(const Layer& L, int batch, const void* x, i
     }
     z = w.z;
   }
-  HARP_CUDA(launch_mr(L.mrU, 0, batch, z, DT_F32, y, yt, st), "output transform launch");
+  // z is this call's own workspace: the transform may use it between its launches
+  HARP_CUDA(launch_mr(L.mrU, 0, batch, z, DT_F32, y, yt, st, const_cast<float*>(z)), "output transform launch");
   return HARP_OK;
 }
 

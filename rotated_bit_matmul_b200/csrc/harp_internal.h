@@ -123,9 +123,12 @@ LinearWs linear_ws_layout(const Layer& L, int batch, void* base);
 int xq_words_per_row(int64_t n_in, int bits);
 
 cudaError_t launch_butterfly(const BflyParams& p, int batch, cudaStream_t st);
-// mixed-radix transform of `batch` contiguous rows (plan forward, or its transpose)
+// mixed-radix transform of `batch` contiguous rows (plan forward, or its transpose).
+// For fewer than 8 rows the stages run in several launches with fp32 rows in between,
+// held in y when y is fp32, else in `scratch` (batch x d floats, may be x); with neither,
+// one CTA per row runs every stage.
 cudaError_t launch_mr(const harp_mr_plan_s* plan, int inverse, int batch, const void* x, int xt, void* y, int yt,
-                      cudaStream_t st);
+                      cudaStream_t st, float* scratch = nullptr);
 int64_t mr_plan_d(const harp_mr_plan_s* plan);
 int mr_plan_device(const harp_mr_plan_s* plan);
 // int16 GEMV operand of `batch` fp32 rows of n (groups of 64): xq words, xs, xsum

@@ -15,10 +15,17 @@
 //                  twice over the Gaussian's columns;
 //   blocks_kernel  one thread per group: the Cayley map by Gauss-Jordan elimination with
 //                  partial pivoting, then B = Q G.
-// The transform keeps a whole row (d <= 16384) in shared memory. A stage computes every
-// output i of group c as sum_j B_{t,c}[i][j] v[base_c + j s_t] (B^T for the transpose)
-// into a second buffer, and the two buffers swap after each stage.
+// For many rows the transform keeps a whole row (d <= 16384) in shared memory, one CTA per
+// row. A stage computes every output i of group c as sum_j B_{t,c}[i][j] v[base_c + j s_t]
+// (B^T for the transpose) into a second buffer, and the two buffers swap after each stage.
+// For a few rows (one CTA per row would leave the GPU idle) the stages are cut into runs of
+// consecutive stages whose radices multiply to at most 256: within a run the row falls into
+// d / (b_t0 ... b_t1-1) independent sub-problems (the indices that share every digit outside
+// the run), and one launch per run spreads them over many CTAs, each keeping a few
+// sub-problems and all the blocks the run applies to them in shared memory; fp32 results
+// pass between runs through global memory.
 #include <algorithm>
+#include <cstdlib>
 #include <new>
 
 #include "common.cuh"
@@ -30,6 +37,14 @@ constexpr int kMrMaxStages = 32;
 constexpr int kMrMaxRadix = 64;
 constexpr int64_t kMrMaxD = 16384;
 constexpr int kMrThreads = 512;
+// Below kMrSegRows rows the transform runs run by run: runs of at most kMrSegRun
+// coordinates, at most kMrSegElems coordinates and kMrSegSmem bytes of shared memory per CTA.
+constexpr int kMrSegRows = 8;
+constexpr int kMrSegRun = 256;
+constexpr int kMrSegElems = 1024;
+constexpr int kMrSegSmem = 96 * 1024;
+constexpr int kMrSegThreads = 512;
+static_assert(kMrSegRun <= 256, "a run holds at most 8 stages");
 
 struct MrParams {
   int64_t d;
@@ -44,6 +59,199 @@ struct MrParams {
   void* y;
   int yt;
 };
+
+struct SegParams {
+  MrParams mp;
+  int t0, t1;       // the run: stages t0 .. t1-1
+  int K;            // sub-problems per CTA
+  int first, last;  // reads x (and applies the forward signs) / writes y (and the transpose's signs)
+  int s0, br;       // stride of the run's first digit, product of the run's radices
+  int sumb;         // sum of the run's radices
+  const float* src; // fp32 input of a run that is not the first
+  float* dst;       // fp32 output of a run that is not the last
+};
+
+// Integer quotient a / d for 0 <= a < 2^20 and d >= 1 from d's fp32 reciprocal: the
+// product is within 0.25 of a / d, so the truncated estimate is off by at most one, and
+// the remainder's sign and size correct it. (Every index here is below 2^17.)
+struct Div {
+  int d;
+  float r;
+};
+__device__ __forceinline__ Div mkdiv(int d) { return Div{d, 1.0f / (float)d}; }
+__device__ __forceinline__ int qdiv(int a, Div v) {
+  int q = __float2int_rz(__int2float_rn(a) * v.r);
+  const int r = a - q * v.d;
+  q += (r >= v.d) - (r < 0);
+  return q;
+}
+
+// One run of stages over K sub-problems per CTA (blockIdx.x: row, then sub-problem block).
+// Shared memory: the sub-problems' coordinates twice (the stage buffers), every block the
+// run applies to them, gathered before the first stage so that their loads overlap (stage
+// t's block of sub-problem qi, group gl, at off_t + (qi (br / b_t) + gl) b_t^2), and the
+// global group number of each of those blocks (at goff_t + qi (br / b_t) + gl).
+__global__ void __launch_bounds__(kMrSegThreads) mr_seg_kernel(SegParams sp) {
+  extern __shared__ __align__(16) float mr_sm[];
+  const MrParams& p = sp.mp;
+  const int d = (int)p.d, s0 = sp.s0, br = sp.br, nsub = d / br;
+  const int nblk = (nsub + sp.K - 1) / sp.K;
+  const int64_t row = blockIdx.x / nblk;
+  const int q0 = (int)(blockIdx.x % nblk) * sp.K;
+  const int K = nsub - q0 < sp.K ? nsub - q0 : sp.K;
+  const int n = K * br;
+  const Div dbr = mkdiv(br), dK = mkdiv(K), ds0 = mkdiv(s0);
+  float* a = mr_sm;
+  float* b2 = mr_sm + n;
+  float* bs = mr_sm + 2 * n;
+  int* gidx = reinterpret_cast<int*>(bs + n * sp.sumb);
+  // element lam of sub-problem q: the lower digits q mod s0, the run's digits lam, the
+  // higher digits q div s0
+  auto goff = [&](int qi, int lam) {
+    const int q = q0 + qi, hi = qdiv(q, ds0);
+    return (q - hi * s0) + s0 * lam + hi * s0 * br;
+  };
+  // load and store order: along the row when the run starts at stride 1, else across the
+  // sub-problems (neighbouring lower digits sit next to each other)
+  auto split = [&](int o, int& qi, int& lam) {
+    if (s0 == 1) {
+      qi = qdiv(o, dbr);
+      lam = o - qi * br;
+    } else {
+      lam = qdiv(o, dK);
+      qi = o - lam * K;
+    }
+  };
+  // the run's stage parameters (at most 8 stages: a run holds at most 256 coordinates):
+  // radix, global and local stride, offsets of the stage's blocks and group numbers
+  __shared__ int s_b[8], s_st[8], s_ls[8], s_off[8], s_go[8];
+  __shared__ const float* s_blk[8];
+  const int ns = sp.t1 - sp.t0;
+  if (threadIdx.x == 0) {
+    int off = 0, go = 0;
+    for (int i = 0; i < ns; ++i) {
+      const int t = sp.t0 + i, b = p.radix[t];
+      s_b[i] = b;
+      s_st[i] = (int)p.stride[t];
+      s_ls[i] = (int)p.stride[t] / s0;
+      s_off[i] = off;
+      s_go[i] = go;
+      s_blk[i] = p.blocks + p.block_off[t];
+      off += n * b;
+      go += n / b;
+    }
+  }
+  __syncthreads();
+  // group numbers: group gl of stage i in sub-problem qi starts at local coordinate
+  // (gl mod ls) + (gl div ls) ls b; the global group of coordinate gb at stride st is
+  // (gb mod st) + (gb div (st b)) st
+  for (int i = 0; i < ns; ++i) {
+    const int b = s_b[i], st = s_st[i], ls = s_ls[i], ng = br / b, go = s_go[i];
+    const Div dng = mkdiv(ng), dls = mkdiv(ls), dst = mkdiv(st), db = mkdiv(b);
+    for (int gq = threadIdx.x; gq < n / b; gq += blockDim.x) {  // gq = qi (br / b) + gl
+      const int qi = qdiv(gq, dng), gl = gq - qi * ng;
+      const int gb = goff(qi, gl + qdiv(gl, dls) * ls * (b - 1));
+      const int u = qdiv(gb, dst), w = qdiv(u, db);
+      gidx[go + gq] = (gb - u * st) + w * st;
+    }
+  }
+  // the x (or previous run's) values: at most kX per thread, loaded into registers first so
+  // that their latency overlaps the gather's
+  constexpr int kX = kMrSegElems / kMrSegThreads;
+  float xv[kX];
+#pragma unroll
+  for (int k = 0; k < kX; ++k) {
+    const int o = threadIdx.x + k * kMrSegThreads;
+    xv[k] = 0.f;
+    if (o < n) {
+      int qi, lam;
+      split(o, qi, lam);
+      const int g = goff(qi, lam);
+      if (sp.first) {
+        xv[k] = load_act(p.x, row * d + g, p.xt);
+        if (!p.inverse) xv[k] *= (float)p.sign[g];
+      } else {
+        xv[k] = sp.src[row * d + g];
+      }
+    }
+  }
+  __syncthreads();
+  // the gather over every stage of the run at once, kG independent loads per thread in
+  // flight: a thread issues them all before it stores any
+  constexpr int kG = 8;
+  const int total = n * sp.sumb;
+  for (int o0 = threadIdx.x; o0 < total; o0 += kMrSegThreads * kG) {
+    float v[kG];
+#pragma unroll
+    for (int k = 0; k < kG; ++k) {
+      const int o = o0 + k * kMrSegThreads;
+      v[k] = 0.f;
+      if (o < total) {
+        int i = 0;
+        while (i + 1 < ns && o >= s_off[i + 1]) ++i;
+        const int bb = s_b[i] * s_b[i], r = o - s_off[i], gq = qdiv(r, mkdiv(bb));
+        v[k] = __ldg(s_blk[i] + (int64_t)gidx[s_go[i] + gq] * bb + (r - gq * bb));
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kG; ++k)
+      if (o0 + k * kMrSegThreads < total) bs[o0 + k * kMrSegThreads] = v[k];
+  }
+#pragma unroll
+  for (int k = 0; k < kX; ++k) {
+    const int o = threadIdx.x + k * kMrSegThreads;
+    if (o < n) {
+      int qi, lam;
+      split(o, qi, lam);
+      a[qi * br + lam] = xv[k];
+    }
+  }
+  __syncthreads();
+  // the stages: the thread's elements o = qi br + lam stay the same through the run
+  int eq[kX], el[kX];
+#pragma unroll
+  for (int k = 0; k < kX; ++k) {
+    const int o = threadIdx.x + k * kMrSegThreads;
+    eq[k] = qdiv(o, dbr);
+    el[k] = o - eq[k] * br;
+  }
+  for (int step = 0; step < ns; ++step) {
+    const int i = p.inverse ? ns - 1 - step : step;
+    const int off = s_off[i], b = s_b[i], ls = s_ls[i], ng = br / b;
+    const Div dls = mkdiv(ls), db = mkdiv(b);
+#pragma unroll
+    for (int k = 0; k < kX; ++k) {
+      const int o = threadIdx.x + k * kMrSegThreads;
+      if (o < n) {
+        const int lam = el[k], t1 = qdiv(lam, dls), hi = qdiv(t1, db), digit = t1 - hi * b;
+        const int gl = (lam - t1 * ls) + hi * ls;  // lam's group: its digit i taken out
+        const float* Bc = bs + off + (eq[k] * ng + gl) * b * b;
+        const float* av = a + eq[k] * br + (lam - digit * ls);
+        float acc = 0.f;
+        if (p.inverse)
+          for (int j = 0; j < b; ++j) acc = fmaf(Bc[j * b + digit], av[j * ls], acc);
+        else
+          for (int j = 0; j < b; ++j) acc = fmaf(Bc[digit * b + j], av[j * ls], acc);
+        b2[o] = acc;
+      }
+    }
+    __syncthreads();
+    float* tmp = a;
+    a = b2;
+    b2 = tmp;
+  }
+  for (int k = 0; k < kX; ++k) {
+    const int o = threadIdx.x + k * kMrSegThreads;
+    if (o < n) {
+      int qi, lam;
+      split(o, qi, lam);
+      const int g = goff(qi, lam);
+      const float v = a[qi * br + lam];
+      if (sp.last) store_act(p.y, row * d + g, p.yt, p.inverse ? v * (float)p.sign[g] : v);
+      else sp.dst[row * d + g] = v;
+    }
+  }
+}
 
 __global__ void __launch_bounds__(kMrThreads) mr_kernel(MrParams p) {
   extern __shared__ __align__(16) float mr_sm[];
@@ -304,7 +512,7 @@ harp_status harp_mr_plan_destroy(harp_mr_plan plan) {
 namespace harp {
 
 cudaError_t launch_mr(const harp_mr_plan_s* plan, int inverse, int batch, const void* x, int xt, void* y, int yt,
-                      cudaStream_t st) {
+                      cudaStream_t st, float* scratch) {
   if (batch <= 0) return cudaSuccess;
   MrParams p = plan->p;
   p.inverse = inverse;
@@ -312,6 +520,63 @@ cudaError_t launch_mr(const harp_mr_plan_s* plan, int inverse, int batch, const 
   p.xt = xt;
   p.y = y;
   p.yt = yt;
+  // few rows: runs of stages over many CTAs, fp32 between runs in y (when fp32) or scratch
+  float* buf = yt == DT_F32 ? static_cast<float*>(y) : scratch;
+  if (batch < kMrSegRows && buf) {
+    static const int run_cap = [] {
+      const char* e = getenv("HARP_MR_RUN");
+      return e ? std::max(2, std::min(kMrSegRun, atoi(e))) : kMrSegRun;
+    }();
+    int runs[kMrMaxStages + 1], nr = 0;  // run boundaries in stage order
+    runs[nr++] = 0;
+    int64_t prod = 1;
+    for (int t = 0; t < p.m; ++t) {
+      if (prod * p.radix[t] > run_cap && prod > 1) {
+        runs[nr++] = t;
+        prod = 1;
+      }
+      prod *= p.radix[t];
+    }
+    runs[nr] = p.m;
+    for (int k = 0; k < nr; ++k) {
+      const int r = inverse ? nr - 1 - k : k;  // the transpose runs the stages backwards
+      SegParams sp;
+      sp.mp = p;
+      sp.t0 = runs[r];
+      sp.t1 = runs[r + 1];
+      if (sp.t1 - sp.t0 > 8) return cudaErrorInvalidValue;
+      sp.s0 = (int)p.stride[sp.t0];
+      sp.br = 1;
+      sp.sumb = 0;
+      for (int t = sp.t0; t < sp.t1; ++t) {
+        sp.br *= p.radix[t];
+        sp.sumb += p.radix[t];
+      }
+      const int nsub = (int)(p.d / sp.br);
+      // enough sub-problems per CTA to fill about one CTA per SM, within the caps
+      int K = (nsub * batch + 147) / 148;
+      K = std::min(K, std::max(1, kMrSegElems / sp.br));
+      int ngrp = 0;  // blocks per sub-problem over the run
+      for (int t = sp.t0; t < sp.t1; ++t) ngrp += sp.br / p.radix[t];
+      const int per = (sp.br * (2 + sp.sumb) + ngrp) * (int)sizeof(float);  // shared bytes per sub-problem
+      K = std::max(1, std::min(K, kMrSegSmem / per));
+      sp.K = K;
+      sp.first = k == 0;
+      sp.last = k == nr - 1;
+      sp.src = buf;
+      sp.dst = buf;
+      const int nblk = (nsub + K - 1) / K;
+      const size_t smem = (size_t)K * per;
+      if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(mr_seg_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+      }
+      mr_seg_kernel<<<(unsigned)(nblk * batch), kMrSegThreads, smem, st>>>(sp);
+      const cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+  }
   const size_t smem = sizeof(float) * 2 * (size_t)p.d;
   cudaError_t e = cudaFuncSetAttribute(mr_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

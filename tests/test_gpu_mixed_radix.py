@@ -44,12 +44,15 @@ def _case(radices, seed, scale=0.2):
 @pytest.mark.parametrize("radices", [(8, 8, 8, 5, 2), (2, 2, 2, 2, 2, 2, 2, 2, 43), (3, 4, 5), (2,) * 8, (16, 4),
                                      (7, 64), (64, 64, 4)])
 @pytest.mark.parametrize("inverse", [False, True])
-def test_mixed_radix_matches_oracle(radices, inverse):
+@pytest.mark.parametrize("rows", [3, 9])
+def test_mixed_radix_matches_oracle(radices, inverse, rows):
+    """3 rows: the stages run in runs of at most 4096 coordinates over many CTAs; 9 rows: one
+    CTA per row holds the whole row."""
     import rotated_bit_matmul_b200 as rb
     d, th, sign, gauss = _case(radices, sum(radices))
     plan = rb.HarpMixedRadix(radices, torch.from_numpy(th).cuda(), torch.from_numpy(sign).cuda(),
                              torch.from_numpy(np.concatenate([g.reshape(-1) for g in gauss])).cuda())
-    x = np.random.default_rng(d).standard_normal((3, d)).astype(np.float32)
+    x = np.random.default_rng(d).standard_normal((rows, d)).astype(np.float32)
     f = plan.inv if inverse else plan.fwd
     got = f(torch.from_numpy(x).cuda()).cpu().numpy()
     torch.cuda.synchronize()
@@ -57,7 +60,7 @@ def test_mixed_radix_matches_oracle(radices, inverse):
     g64 = [g.astype(np.float64) for g in gauss]
     want = (oracle.mr_butterfly_inv if inverse else oracle.mr_butterfly_fwd)(x, radices, th, sign, g64)
     err = rel_l2(got, want)
-    print(f"mixed radix {radices} inverse={inverse}: rel-L2 {err:.2e}")
+    print(f"mixed radix {radices} inverse={inverse} rows={rows}: rel-L2 {err:.2e}")
     assert err < GATE
 
 
