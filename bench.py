@@ -396,6 +396,14 @@ def run_linear_configs(args):
     for i, shp in enumerate(shapes):
         with ClockSampler(0) as clk:
             rows = lt.time_shape(*shp, 2, batches)
+        fused = {}
+        if args.config == 3 and shp[3] <= 256:
+            # the output blocks of 256 finished inside the tensor-core kernel (opt-in)
+            os.environ["HARP_MMA_FUSE"] = "1"
+            try:
+                fused = {r["batch"]: r["us_per_call"] for r in lt.time_shape(*shp, 2, [b for b in batches if b >= 16])}
+            finally:
+                del os.environ["HARP_MMA_FUSE"]
         for r in rows:
             us, B = r["us_per_call"], r["batch"]
             ach = r["alg_bytes"] / us / 1e3
@@ -410,7 +418,8 @@ def run_linear_configs(args):
             _line(f"rotated 2-bit linear {names[i]}, batch {B}: time per call", us, "us/call", False,
                   {"workload": f"config {args.config}: {names[i]} rotated 2-bit linear, bf16 x [{B},{shp[1]}]",
                    "batch": B, "distinct_layers": r["layers"], "l2": "cold L2: distinct layer copies per call"},
-                  roof, launches=3 if B < 16 else 4, clocks=clk.summary())
+                  roof, launches=3 if B < 16 else 4, clocks=clk.summary(),
+                  extra={"fused_epilogue_us_per_call": fused[B]} if B in fused else None)
             if args.config == 2:
                 total_us += mult[i] * us
                 total_bytes += mult[i] * r["alg_bytes"]

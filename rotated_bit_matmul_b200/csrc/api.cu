@@ -280,6 +280,13 @@ harp_status linear_forward_status(const Layer& L, int batch, const void* x, int 
     c.zpart = w.zpart;
     c.batch = batch;
     c.status = status;
+    if (mma::fuses(L, batch)) {  // output butterfly inside the tensor-core kernel
+      c.y = y;
+      c.yt = yt;
+      c.y_stride = y_stride;
+      HARP_CUDA(mma::launch(L, c, st), "dequant-MMA launch");
+      return HARP_OK;
+    }
     HARP_CUDA(mma::launch(L, c, st), "dequant-MMA launch");
   } else {
     pv.y = nullptr;

@@ -13,6 +13,16 @@
 // * warps 2..9 then read the accumulator with tcgen05.ld and store the split's fp32
 //   partial sums. The output butterfly adds the splits in a fixed order.
 //
+// Fused epilogue (output blocks of w_out = 128 or 256 rows, HARP Sec. 2.4: the stride
+// stages fused with the contraction). The H = w_out / 128 tiles of one output block and
+// all S splits run as one thread-block cluster of H S CTAs. Each CTA writes its scaled
+// partial tile into its own (by then idle) ring, token-major. After a cluster barrier each
+// CTA takes a share of the token columns, one warp per column: it reads the block's H S
+// partial tiles through distributed shared memory, adds the splits in split order, applies
+// the signs and the block's stride stages (the layer's cos/sin pairs, int8 angles, or
+// Theta = 0) in registers and warp shuffles, and writes y. A second cluster barrier keeps every tile alive until its last
+// reader is done. No partial array and no output-butterfly launch remain.
+//
 // Zero term. deq(q) = s q + m for each (row, group), so
 //   z = sum_j (s q_j) x_j + sum_g m_g X_g,
 // where X_g is a group sum of the operand. The second sum runs on the tensor core as one
@@ -26,6 +36,7 @@
 #include "mma.h"
 
 #include <algorithm>
+#include <cstdlib>
 
 namespace harp {
 namespace mma {
@@ -91,6 +102,15 @@ __device__ __forceinline__ void st_shared_v4(void* p, uint32_t a, uint32_t b, ui
                : "memory");
 }
 
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t h2u(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 __device__ __forceinline__ __half2 u2h(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
 
@@ -112,7 +132,16 @@ struct Params {
   const float* rowscale;
   float* zpart;
   int* status;
+  // fused epilogue (fuse != 0): cluster of H tiles x all splits per w_out-row block
+  int fuse, H, w_out, m_out;
+  const int8_t* sign;  // [n_out] output-side signs
+  const float2* cs;    // [m_out][n_out/2] (cos, sin), or null
+  const uint8_t* q8;   // int8 angles (fp32 steps head, then [m_out][n_out/2]), or null
+  void* y;
+  int yt;
+  int64_t y_stride;
 };
+
 
 template <int BITS>
 struct Geo {
@@ -121,14 +150,121 @@ struct Geo {
 };
 
 // Dynamic shared memory: [ring: stages x (A 16 KB | X N*128 | codes 128*cb)] [sz 128*gs*4]
-// [hi 128*gs*8] [barriers]; the ring starts 1024-byte aligned (swizzle atoms).
+// [hi 128*gs*8] [barriers, 256 B] [fused epilogue: the output block's (cos, sin) pairs];
+// the ring starts 1024-byte aligned (swizzle atoms).
+constexpr int kCfBytes = 8 * 128 * 8;  // log2 256 stages x 128 pairs x (cos, sin)
 template <int BITS>
 __host__ __device__ inline int stage_bytes(int N) {
   return Geo<BITS>::kA + N * 128 + kBM * Geo<BITS>::kCodeBytes;
 }
 template <int BITS>
-__host__ __device__ inline int fixed_bytes(int gs) {
-  return kBM * gs * 4 + (BITS == 3 ? kBM * gs * 8 : 0) + 256 + 1024;  // + barriers + alignment slack
+__host__ __device__ inline int fixed_bytes(int gs, bool fuse) {
+  // + barriers + alignment slack (+ the fused epilogue's coefficients)
+  return kBM * gs * 4 + (BITS == 3 ? kBM * gs * 8 : 0) + 256 + 1024 + (fuse ? kCfBytes : 0);
+}
+
+// (cos, sin) of pi/4 + theta_t for pair q of the output side's stage t (global slot)
+__device__ __forceinline__ void out_coef(const Params& p, int t, int64_t slot, float& c, float& s) {
+  if (p.q8) {
+    const float step = __ldg(reinterpret_cast<const float*>(p.q8) + t);
+    const int8_t a = reinterpret_cast<const int8_t*>(p.q8 + kQ8Head)[(int64_t)t * (p.n_out >> 1) + slot];
+    sincosf(fmaf(step, (float)a, 0.785398163397448309616f), &s, &c);
+  } else if (p.cs) {
+    const float2 v = __ldg(p.cs + (int64_t)t * (p.n_out >> 1) + slot);
+    c = v.x;
+    s = v.y;
+  } else {
+    c = s = 0.70710678118654752440f;  // Theta = 0
+  }
+}
+
+// four fp32 at `local` (16-byte aligned, this CTA's shared memory) in cluster CTA `cta`'s copy
+__device__ __forceinline__ float4 ld_peer4(const float* local, uint32_t cta) {
+  uint32_t ra;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(local)), "r"(cta));
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(ra)
+               : "memory");
+  return v;
+}
+
+// The cluster's output block of W rows: split sums, signs, stride stages and the store of y
+// for this CTA's share of the token columns. Every CTA of the cluster takes both cluster
+// barriers. One warp per token column, W / 32 consecutive rows per lane: stages of stride
+// below W / 32 stay inside a lane, the wider ones pair lanes through shuffles. `tile` is
+// this CTA's partial tile; `cf` holds the block's log2 W x W/2 (cos, sin) pairs, stage-major.
+template <int W>
+__device__ __noinline__ void fused_epilogue(const Params& p, const float* tile, const float2* cf, int tile_idx, int b0) {
+  constexpr int EPL = W / 32, LE = EPL == 8 ? 3 : 2, LW = W == 256 ? 8 : 7, HW = W / 2;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int H = p.H, S = (int)gridDim.y, R = H * S;
+  const int blk = tile_idx / H;
+  const uint32_t rank = cluster_rank();
+  cluster_sync_all();  // every partial tile of the cluster written
+  const int nval = min(p.N, p.batch - b0);
+  const int per = (nval + R - 1) / R;
+  const int c_lo = min(nval, (int)rank * per), c_hi = min(nval, c_lo + per);
+  const int e0 = lane * EPL, h0 = e0 >> 7;
+  const int8_t* sg = p.sign + (int64_t)blk * W + e0;
+  float sgn[EPL];
+#pragma unroll
+  for (int j = 0; j < EPL; ++j) sgn[j] = (float)__ldg(sg + j);
+  for (int col = c_lo + warp; col < c_hi; col += kThreads / 32) {
+    const float* src = tile + col * kBM + (e0 & (kBM - 1));
+    float v[EPL];
+#pragma unroll
+    for (int k = 0; k < EPL / 4; ++k) {
+      const float4 a = ld_peer4(src + 4 * k, (uint32_t)h0);  // split 0 of tile h0: cluster rank h0
+      v[4 * k] = a.x;
+      v[4 * k + 1] = a.y;
+      v[4 * k + 2] = a.z;
+      v[4 * k + 3] = a.w;
+    }
+    for (int sp = 1; sp < S; ++sp) {
+#pragma unroll
+      for (int k = 0; k < EPL / 4; ++k) {
+        const float4 a = ld_peer4(src + 4 * k, (uint32_t)(h0 + sp * H));
+        v[4 * k] += a.x;
+        v[4 * k + 1] += a.y;
+        v[4 * k + 2] += a.z;
+        v[4 * k + 3] += a.w;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) v[j] *= sgn[j];
+    // stages inside the lane: pairs (j, j + 2^t)
+#pragma unroll
+    for (int t = 0; t < LE; ++t) {
+      const int hs = 1 << t;
+#pragma unroll
+      for (int j = 0; j < EPL; ++j) {
+        if (j & hs) continue;
+        const int i = e0 + j, q = ((i >> (t + 1)) << t) | (i & (hs - 1));
+        const float2 k2 = cf[t * HW + q];
+        const float a = v[j], b = v[j + hs];
+        v[j] = fmaf(k2.x, a, k2.y * b);
+        v[j + hs] = fmaf(k2.y, a, -k2.x * b);
+      }
+    }
+    // stages across lanes: lane bit t - LE pairs row i (bit clear) with i + 2^t
+#pragma unroll
+    for (int t = LE; t < LW; ++t) {
+      const int lb = 1 << (t - LE), hs = 1 << t;
+      const bool upper = (lane & lb) != 0;
+      const int il = (lane & ~lb) * EPL;  // the lower lane's first row
+#pragma unroll
+      for (int j = 0; j < EPL; ++j) {
+        const float o = __shfl_xor_sync(0xffffffffu, v[j], lb);
+        const int i = il + j, q = ((i >> (t + 1)) << t) | (i & (hs - 1));
+        const float2 k2 = cf[t * HW + q];
+        v[j] = upper ? fmaf(k2.y, o, -k2.x * v[j]) : fmaf(k2.x, v[j], k2.y * o);
+      }
+    }
+    const int64_t yo = (int64_t)(b0 + col) * p.y_stride + (int64_t)blk * W + e0;
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) store_act(p.y, yo + j, p.yt, v[j]);
+  }
+  cluster_sync_all();  // no tile leaves while a peer may still read it
 }
 
 template <int BITS>
@@ -148,6 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1) mma_kernel(const __grid_constant_
   uint64_t* pre = bars + 3 * kMaxStages;    // scale/zero (and hi plane) of the split landed
   uint64_t* accb = pre + 1;                 // accumulator complete
   uint32_t* tslot = reinterpret_cast<uint32_t*>(accb + 1);
+  float2* cf_s = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(bars) + 256);  // fused epilogue only
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int tile = blockIdx.x, split = blockIdx.y, b0 = blockIdx.z * kMaxN;
@@ -233,6 +370,16 @@ __global__ void __launch_bounds__(kThreads, 1) mma_kernel(const __grid_constant_
       if (lane == 0) w = mbar_wait_sleep(bar, ph, p.status, where);
       return __shfl_sync(0xffffffffu, w, 0) != 0;
     };
+    if (p.fuse) {
+      // the output block's coefficients, for the fused epilogue: loaded now, so that their
+      // latency hides under the ring's first copies
+      const int hw = p.w_out >> 1, blk = tile / p.H;
+      for (int k = t; k < p.m_out * hw; k += 32 * kDqWarps) {
+        float c, s;
+        out_coef(p, k / hw, (int64_t)blk * hw + (k % hw), c, s);
+        cf_s[k] = make_float2(c, s);
+      }
+    }
     bool ok = warp_wait(pre, 0, 86);
     for (int k = 0; ok && k < nst; ++k) {
       const int slot = k % ST, ph = (k / ST) & 1;
@@ -307,13 +454,17 @@ __global__ void __launch_bounds__(kThreads, 1) mma_kernel(const __grid_constant_
       const int r = row0 + 32 * q + lane;
       const int half = p.N >> 1;
       float* zp = p.zpart + (int64_t)split * p.batch * p.n_out;
+      float* ptile = reinterpret_cast<float*>(ring);  // fused: [N][128] in the idle ring
       for (int c0 = ch * half; c0 < (ch + 1) * half; c0 += 8) {
         float v[8];
         tmem_ld8(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int b = b0 + c0 + j;
-          if (b < p.batch && r < p.n_out) zp[(int64_t)b * p.n_out + r] = v[j] * p.rowscale[b];
+          if (p.fuse)
+            ptile[(c0 + j) * kBM + 32 * q + lane] = b < p.batch ? v[j] * p.rowscale[b] : 0.f;
+          else if (b < p.batch && r < p.n_out)
+            zp[(int64_t)b * p.n_out + r] = v[j] * p.rowscale[b];
         }
       }
     }
@@ -323,6 +474,10 @@ __global__ void __launch_bounds__(kThreads, 1) mma_kernel(const __grid_constant_
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, (uint32_t)p.ncols);
+  }
+  if (p.fuse) {
+    if (p.w_out == 256) fused_epilogue<256>(p, reinterpret_cast<const float*>(ring), cf_s, tile, b0);
+    else fused_epilogue<128>(p, reinterpret_cast<const float*>(ring), cf_s, tile, b0);
   }
 }
 
@@ -442,6 +597,32 @@ cudaError_t launch_x16_prep(const float* xt, int64_t n_in, int bits, int batch, 
   return cudaGetLastError();
 }
 
+// ring stages for N tokens within the opt-in shared memory (0: does not fit)
+template <int BITS>
+static int ring_stages(int N, int gs, bool fuse, int optin) {
+  return std::min(kMaxStages, (optin - fixed_bytes<BITS>(gs, fuse)) / stage_bytes<BITS>(N));
+}
+
+static int optin_smem() {
+  int dev = 0, optin = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  return optin;
+}
+
+template <int BITS>
+static bool fuses_t(const Layer& L, int batch) {
+  // opt-in (HARP_MMA_FUSE=1): measured slower than the separate output butterfly so far
+  const char* e = getenv("HARP_MMA_FUSE");
+  const bool on = e && atoi(e) != 0;
+  if (!on || (L.w_out != 128 && L.w_out != 256) || (1 << L.m_out) != L.w_out || L.n_out % L.w_out != 0) return false;
+  if ((L.w_out / kBM) * L.msplits > 8) return false;  // portable cluster size
+  const int N = (std::min(batch, kMaxN) + 15) / 16 * 16;
+  const int stages = ring_stages<BITS>(N, L.mgs, true, optin_smem());
+  // the idle ring holds the N x 128 partial tile
+  return stages >= 2 && (int64_t)stages * stage_bytes<BITS>(N) >= (int64_t)N * kBM * 4;
+}
+
 template <int BITS>
 static cudaError_t launch_t(const Layer& L, const Call& c, cudaStream_t st) {
   Params p{};
@@ -460,13 +641,24 @@ static cudaError_t launch_t(const Layer& L, const Call& c, cudaStream_t st) {
   p.rowscale = c.rowscale;
   p.zpart = c.zpart;
   p.status = c.status;
+  p.fuse = c.y && fuses_t<BITS>(L, c.batch);
+  if (c.y && !p.fuse) return cudaErrorInvalidValue;  // the caller asked without checking fuses()
+  p.H = L.w_out / kBM;
+  p.w_out = L.w_out;
+  p.m_out = L.m_out;
+  p.sign = L.sU;
+  p.cs = L.q8U ? nullptr : L.csU;
+  p.q8 = L.q8U;
+  p.y = c.y;
+  p.yt = c.yt;
+  p.y_stride = c.y_stride;
 
   int dev = 0, optin = 0, sm_smem = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   cudaDeviceGetAttribute(&sm_smem, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
-  const int SB = stage_bytes<BITS>(p.N), FB = fixed_bytes<BITS>(p.gs);
-  p.stages = std::min(kMaxStages, (optin - FB) / SB);
+  const int SB = stage_bytes<BITS>(p.N), FB = fixed_bytes<BITS>(p.gs, p.fuse);
+  p.stages = ring_stages<BITS>(p.N, p.gs, p.fuse, optin);
   if (p.stages < 2) return cudaErrorInvalidConfiguration;
   int smem = FB + p.stages * SB;
   // tensor memory: CTAs resident on one SM must fit in its 512 columns
@@ -487,8 +679,29 @@ static cudaError_t launch_t(const Layer& L, const Call& c, cudaStream_t st) {
   const int tiles = (p.n_out + kBM - 1) / kBM;
   const int splits = (p.G + p.gs - 1) / p.gs;
   const int chunks = (c.batch + kMaxN - 1) / kMaxN;
-  mma_kernel<BITS><<<dim3(tiles, splits, chunks), kThreads, smem, st>>>(p);
-  return cudaGetLastError();
+  if (!p.fuse) {
+    mma_kernel<BITS><<<dim3(tiles, splits, chunks), kThreads, smem, st>>>(p);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)tiles, (unsigned)splits, (unsigned)chunks);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)p.H;
+  attr[0].val.clusterDim.y = (unsigned)splits;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, mma_kernel<BITS>, p);
+}
+
+bool fuses(const Layer& L, int batch) {
+  if (L.bits == 2) return fuses_t<2>(L, batch);
+  if (L.bits == 3) return fuses_t<3>(L, batch);
+  return fuses_t<4>(L, batch);
 }
 
 cudaError_t launch(const Layer& L, const Call& c, cudaStream_t st) {

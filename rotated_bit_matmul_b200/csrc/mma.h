@@ -30,10 +30,21 @@ struct Call {
   const __half* x16;     // [batch][ld]
   int64_t ld;
   const float* rowscale; // [batch] 2^-e
-  float* zpart;          // [splits][batch][n_out]
+  float* zpart;          // [splits][batch][n_out] (unused when y is set)
   int batch;
   int* status;
+  // set only when fuses(L, batch): the kernel adds the splits and applies the output
+  // side's butterfly itself, writing y ([batch] rows of n_out, y_stride apart, dtype yt)
+  void* y = nullptr;
+  int yt = 0;
+  int64_t y_stride = 0;
 };
+
+// true when the fused epilogue is switched on (HARP_MMA_FUSE=1, read at each call; off by
+// default) and the layer's output blocks (w_out = 128 or 256 rows) can be finished inside
+// the tensor-core kernel at this batch: a cluster of (w_out / 128) x splits <= 8 CTAs, and
+// the ring holds the partial tile.
+bool fuses(const Layer& L, int batch);
 
 cudaError_t launch_x16_prep(const float* xt, int64_t n_in, int bits, int batch, __half* x16, float* rowscale,
                             int* status, cudaStream_t st);

@@ -120,6 +120,61 @@ def test_ragged(bits, batch):
     _check(case, batch, 9)
 
 
+@pytest.mark.parametrize("bits", [2, 3, 4])
+@pytest.mark.parametrize("batch", [17, 300])
+@pytest.mark.parametrize("w_out", [128, 256])
+def test_fused_epilogue_ragged(bits, batch, w_out, monkeypatch):
+    """Output blocks of 128 or 256 rows finish inside the tensor-core kernel (a cluster of
+    the block's tiles and all splits; switched on by HARP_MMA_FUSE=1): 17 tokens (N padded
+    to 32, columns shared unevenly over the cluster) and 300 tokens (two token chunks)."""
+    monkeypatch.setenv("HARP_MMA_FUSE", "1")
+    case = oracle_layer(768, 1024, 1024, w_out, bits, workload=9)
+    _check(case, batch, 9)
+
+
+@pytest.mark.parametrize("batch", [16, 256])
+def test_fused_epilogue_11008(batch, monkeypatch):
+    """The fused epilogue on gate/up of 7B (43 output blocks of 256, two splits)."""
+    monkeypatch.setenv("HARP_MMA_FUSE", "1")
+    case = oracle_layer(11008, 4096, 4096, 256, 2, workload=3, linear=4)
+    _check(case, batch, 3)
+
+
+def test_fused_epilogue_q8_and_rht(monkeypatch):
+    """The fused epilogue with int8 angles and with Theta = 0 on the output side."""
+    monkeypatch.setenv("HARP_MMA_FUSE", "1")
+    import test_gpu_q8 as q8
+    import test_gpu_rht as rht
+    c = q8._q8_case(11008, 4096, 4096, 256, 3)
+    x = synth.activations(16, 4096, 12, step=16)
+    L = q8._device(c)
+    got = L(_dev(x, torch.bfloat16), out_dtype=torch.float32).cpu().numpy()
+    torch.cuda.synchronize()
+    L.close()
+    assert rel_l2(got, oracle.linear_fwd(c["lay"], x.astype(np.float64))) < GATE
+    c = rht._rht_case(11008, 4096, 4096, 256, 2, True, True)
+    x = synth.activations(16, 4096, 10, step=16)
+    L = rht._device(c)
+    got = L(_dev(x, torch.bfloat16), out_dtype=torch.float32).cpu().numpy()
+    torch.cuda.synchronize()
+    L.close()
+    assert rel_l2(got, oracle.linear_fwd(c["lay"], x.astype(np.float64))) < GATE
+
+
+def test_fused_epilogue_bf16_output(monkeypatch):
+    """The fused epilogue's bf16 store: the fp32 result rounded once."""
+    monkeypatch.setenv("HARP_MMA_FUSE", "1")
+    case = oracle_layer(11008, 4096, 4096, 256, 2, workload=3, linear=4)
+    x = synth.activations(16, 4096, 3, step=16)
+    L = device_layer(case)
+    xd = _dev(x, torch.bfloat16)
+    y32 = L(xd, out_dtype=torch.float32)
+    y16 = L(xd, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    L.close()
+    assert torch.equal(y16, y32.to(torch.bfloat16))
+
+
 def test_fp32_input_config1_shape():
     case = oracle_layer(1024, 1024, 1024, 1024, 2, workload=1)
     _check(case, 32, 1, xdt=torch.float32)
