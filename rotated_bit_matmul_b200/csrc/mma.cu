@@ -579,11 +579,28 @@ Split choose_split(int64_t n_out, int64_t n_in, int bits) {
   const int gmax = bits == 3 ? 32 : kMaxGs;  // the 1-bit plane box holds 8 bytes per group
   // gs is a multiple of 8 so that every split's first group sum (fp16 column n_in + g0)
   // starts a TMA box on a 16-byte boundary
-  int s = std::max(1, (148 + tiles - 1) / tiles);
-  int gs = (G + s - 1) / s;
-  gs = std::min(gmax, std::max(8, (gs + 7) / 8 * 8));
-  s = (G + gs - 1) / gs;
-  return Split{s, gs};
+  auto fit = [&](int s) {
+    int gs = (G + s - 1) / s;
+    gs = std::min(gmax, std::max(8, (gs + 7) / 8 * 8));
+    return Split{(G + gs - 1) / gs, gs};
+  };
+  if (const char* e = getenv("HARP_MMA_SPLITS")) return fit(std::max(1, atoi(e)));  // tuning: a fixed request
+  // About one CTA per SM. The dequant threads read their row's scale/zero word at
+  // sz_s[m gs + g], a stride of gs words across the warp's 32 rows: gs = 32 or 64 puts all
+  // 32 lanes on one bank. Such a split moves to the next request whose gs avoids that
+  // (on B200, 7B gate/up: 3 splits of 24 groups, 50.9 us per call at 16 tokens, against
+  // 66.5 us with 2 of 32; down, 4096 x 11008, keeps 5 of 40: 47.0 us, against 69.2 us with
+  // 6 of 32).
+  const int s0 = std::max(1, (148 + tiles - 1) / tiles);
+  const char* m = getenv("HARP_MMA_SPLIT_MODEL");
+  const Split base = fit(s0);
+  if ((m && atoi(m) == 0) || base.gs % 32 != 0) return base;
+  for (int s = s0 + 1; s <= G / 8; ++s) {  // at most one more wave of CTAs
+    const Split c = fit(s);
+    if ((int64_t)tiles * c.splits > (int64_t)tiles * base.splits + 148) break;
+    if (c.gs % 32 != 0) return c;
+  }
+  return base;
 }
 
 cudaError_t launch_x16_prep(const float* xt, int64_t n_in, int bits, int batch, __half* x16, float* rowscale,
