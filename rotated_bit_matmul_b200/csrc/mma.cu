@@ -585,12 +585,11 @@ Split choose_split(int64_t n_out, int64_t n_in, int bits) {
     return Split{(G + gs - 1) / gs, gs};
   };
   if (const char* e = getenv("HARP_MMA_SPLITS")) return fit(std::max(1, atoi(e)));  // tuning: a fixed request
-  // About one CTA per SM. The dequant threads read their row's scale/zero word at
-  // sz_s[m gs + g], a stride of gs words across the warp's 32 rows: gs = 32 or 64 puts all
-  // 32 lanes on one bank. Such a split moves to the next request whose gs avoids that
-  // (on B200, 7B gate/up: 3 splits of 24 groups, 50.9 us per call at 16 tokens, against
-  // 66.5 us with 2 of 32; down, 4096 x 11008, keeps 5 of 40: 47.0 us, against 69.2 us with
-  // 6 of 32).
+  // About one CTA per SM, and no split of 32 or 64 groups, which measured slow on B200:
+  // 7B gate/up ran 3 splits of 24 groups in 50.9 us per call at 16 tokens against 66.5 us
+  // with 2 of 32, and down (4096 x 11008) 5 of 40 in 47.0 us against 69.2 us with 6 of 32.
+  // The cause is not known: the scale/zero reads' bank conflicts at those widths were
+  // ruled out (a tile transposed to group-major changed nothing).
   const int s0 = std::max(1, (148 + tiles - 1) / tiles);
   const char* m = getenv("HARP_MMA_SPLIT_MODEL");
   const Split base = fit(s0);
