@@ -178,6 +178,17 @@ __device__ __forceinline__ void out_coef(const Params& p, int t, int64_t slot, f
   }
 }
 
+// the output block's (cos, sin) pairs into cf, stage-major, by the 256 dequant threads (t);
+// out of line, so that the int8 angles' sincosf does not weigh on the main loop's registers
+__device__ __noinline__ void stage_out_coefs(const Params& p, float2* cf, int blk, int t) {
+  const int hw = p.w_out >> 1;
+  for (int k = t; k < p.m_out * hw; k += 32 * kDqWarps) {
+    float c, s;
+    out_coef(p, k / hw, (int64_t)blk * hw + (k % hw), c, s);
+    cf[k] = make_float2(c, s);
+  }
+}
+
 // four fp32 at `local` (16-byte aligned, this CTA's shared memory) in cluster CTA `cta`'s copy
 __device__ __forceinline__ float4 ld_peer4(const float* local, uint32_t cta) {
   uint32_t ra;
@@ -370,16 +381,9 @@ __global__ void __launch_bounds__(kThreads, 1) mma_kernel(const __grid_constant_
       if (lane == 0) w = mbar_wait_sleep(bar, ph, p.status, where);
       return __shfl_sync(0xffffffffu, w, 0) != 0;
     };
-    if (p.fuse) {
-      // the output block's coefficients, for the fused epilogue: loaded now, so that their
-      // latency hides under the ring's first copies
-      const int hw = p.w_out >> 1, blk = tile / p.H;
-      for (int k = t; k < p.m_out * hw; k += 32 * kDqWarps) {
-        float c, s;
-        out_coef(p, k / hw, (int64_t)blk * hw + (k % hw), c, s);
-        cf_s[k] = make_float2(c, s);
-      }
-    }
+    // the output block's coefficients, for the fused epilogue: loaded now, so that their
+    // latency hides under the ring's first copies
+    if (p.fuse) stage_out_coefs(p, cf_s, tile / p.H, t);
     bool ok = warp_wait(pre, 0, 86);
     for (int k = 0; ok && k < nst; ++k) {
       const int slot = k % ST, ph = (k / ST) & 1;
