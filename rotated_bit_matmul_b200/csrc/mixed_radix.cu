@@ -15,9 +15,12 @@
 //                  twice over the Gaussian's columns;
 //   blocks_kernel  one thread per group: the Cayley map by Gauss-Jordan elimination with
 //                  partial pivoting, then B = Q G.
-// For many rows the transform keeps a whole row (d <= 16384) in shared memory, one CTA per
-// row. A stage computes every output i of group c as sum_j B_{t,c}[i][j] v[base_c + j s_t]
-// (B^T for the transpose) into a second buffer, and the two buffers swap after each stage.
+// A plan whose radices are all 2 (64 <= d <= 8192) is the radix-2 butterfly of width d: it
+// runs on the butterfly kernels, with a (cos, sin) table taken from its blocks.
+// Otherwise, for many rows the transform keeps a whole row (d <= 16384) in shared memory,
+// one CTA per row. A stage computes every output i of group c as
+// sum_j B_{t,c}[i][j] v[base_c + j s_t] (B^T for the transpose) into a second buffer, and
+// the two buffers swap after each stage.
 // For a few rows (one CTA per row would leave the GPU idle) the stages are cut into runs of
 // consecutive stages whose radices multiply to at most 256: within a run the row falls into
 // d / (b_t0 ... b_t1-1) independent sub-problems (the indices that share every digit outside
@@ -253,6 +256,16 @@ __global__ void __launch_bounds__(kMrSegThreads) mr_seg_kernel(SegParams sp) {
   }
 }
 
+// all-radix-2 plans: (cos, sin) of stage t, pair c from the block's first row (stage t's
+// blocks start at t 2d, four floats per group)
+__global__ void cs_of_blocks_kernel(const float* blocks, int64_t d, int m, float2* cs) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (int64_t)m * (d / 2)) return;
+  const int64_t t = i / (d / 2), c = i - t * (d / 2);
+  const float* B = blocks + t * 2 * d + 4 * c;
+  cs[i] = make_float2(B[0], B[1]);
+}
+
 __global__ void __launch_bounds__(kMrThreads) mr_kernel(MrParams p) {
   extern __shared__ __align__(16) float mr_sm[];
   const int64_t d = p.d, row = blockIdx.x;
@@ -404,6 +417,9 @@ struct harp_mr_plan_s {
   MrParams p{};
   float* blocks = nullptr;
   int8_t* sign = nullptr;
+  // all radices 2 and 64 <= d <= 8192: the radix-2 butterfly's (cos, sin) table [m][d/2],
+  // taken from the blocks, so that the transform runs on the butterfly kernels
+  float2* cs2 = nullptr;
   int device = 0;
 };
 
@@ -457,6 +473,7 @@ harp_status harp_mr_plan_create(harp_mr_plan* out, int64_t d, int m, const int* 
     if (s != HARP_OK) {
       cudaFree(h->blocks);
       cudaFree(h->sign);
+      cudaFree(h->cs2);
       delete h;
     }
     return s;
@@ -483,6 +500,18 @@ harp_status harp_mr_plan_create(harp_mr_plan* out, int64_t d, int m, const int* 
     toff += groups * mr_params_of(b);
     goff += (int64_t)b * b;
   }
+  bool all2 = (d & (d - 1)) == 0 && d >= 64 && d <= 8192;
+  for (int t = 0; t < m; ++t) all2 = all2 && radix[t] == 2;
+  if (all2) {
+    // stage t's group c is the butterfly's pair c of stage t (both number a pair by its
+    // lower index with bit t removed), and its block's first row is (cos p, sin p)
+    if ((e = cudaMalloc(&h->cs2, sizeof(float2) * (size_t)m * (d / 2))) != cudaSuccess)
+      return done(set_error(HARP_ERR_CUDA, "mr_plan_create: cudaMalloc: %s", cudaGetErrorString(e)));
+    const int64_t n = (int64_t)m * (d / 2);
+    cs_of_blocks_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(h->blocks, d, m, h->cs2);
+    if ((e = cudaGetLastError()) != cudaSuccess)
+      return done(set_error(HARP_ERR_CUDA, "mr_plan_create: table launch: %s", cudaGetErrorString(e)));
+  }
   int hbad = 0;
   if ((e = cudaMemcpyAsync(&hbad, bad, sizeof(int), cudaMemcpyDeviceToHost, st)) != cudaSuccess ||
       (e = cudaStreamSynchronize(st)) != cudaSuccess)
@@ -502,6 +531,7 @@ harp_status harp_mr_plan_destroy(harp_mr_plan plan) {
   cudaDeviceSynchronize();
   cudaFree(plan->blocks);
   cudaFree(plan->sign);
+  cudaFree(plan->cs2);
   cudaSetDevice(prev);
   delete plan;
   return HARP_OK;
@@ -514,6 +544,23 @@ namespace harp {
 cudaError_t launch_mr(const harp_mr_plan_s* plan, int inverse, int batch, const void* x, int xt, void* y, int yt,
                       cudaStream_t st, float* scratch) {
   if (batch <= 0) return cudaSuccess;
+  if (plan->cs2) {  // all radices 2: the radix-2 butterfly of width d with the plan's table
+    BflyParams bp{};
+    bp.n = plan->p.d;
+    bp.w = (int)plan->p.d;
+    bp.m = plan->p.m;
+    bp.inverse = inverse;
+    bp.cs = plan->cs2;
+    bp.sign = plan->sign;
+    bp.x = x;
+    bp.xt = xt;
+    bp.x_stride = plan->p.d;
+    bp.y = y;
+    bp.yt = yt;
+    bp.y_stride = plan->p.d;
+    bp.nsum = 1;
+    return launch_butterfly(bp, batch, st);
+  }
   MrParams p = plan->p;
   p.inverse = inverse;
   p.x = x;

@@ -42,7 +42,7 @@ def _case(radices, seed, scale=0.2):
 
 
 @pytest.mark.parametrize("radices", [(8, 8, 8, 5, 2), (2, 2, 2, 2, 2, 2, 2, 2, 43), (3, 4, 5), (2,) * 8, (16, 4),
-                                     (7, 64), (64, 64, 4)])
+                                     (7, 64), (64, 64, 4), (2,) * 12, (2,) * 5])
 @pytest.mark.parametrize("inverse", [False, True])
 @pytest.mark.parametrize("rows", [3, 9])
 def test_mixed_radix_matches_oracle(radices, inverse, rows):

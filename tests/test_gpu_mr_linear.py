@@ -61,6 +61,8 @@ CASES = [
     ((16, 16, 16), (43, 2, 2, 2, 2, 2, 2, 2, 2)),
     ((8, 8, 8, 4, 7), (8, 8, 8)),
     ((8, 8, 8), (8, 8, 8)),
+    # all radices 2 on both sides: the plans run on the radix-2 butterfly kernels
+    ((2,) * 9, (2,) * 12),
 ]
 
 
