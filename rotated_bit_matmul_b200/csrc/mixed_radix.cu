@@ -417,9 +417,11 @@ struct harp_mr_plan_s {
   MrParams p{};
   float* blocks = nullptr;
   int8_t* sign = nullptr;
-  // all radices 2 and 64 <= d <= 8192: the radix-2 butterfly's (cos, sin) table [m][d/2],
-  // taken from the blocks, so that the transform runs on the butterfly kernels
+  // the first P stages of radix 2 with 64 <= 2^P <= 8192: they are the block-diagonal
+  // radix-2 butterfly of width 2^P over the row, whose (cos, sin) table [P][d/2] is taken
+  // from the blocks, so that they run on the butterfly kernels (P = m: the whole plan)
   float2* cs2 = nullptr;
+  int P = 0;
   int device = 0;
 };
 
@@ -500,15 +502,17 @@ harp_status harp_mr_plan_create(harp_mr_plan* out, int64_t d, int m, const int* 
     toff += groups * mr_params_of(b);
     goff += (int64_t)b * b;
   }
-  bool all2 = (d & (d - 1)) == 0 && d >= 64 && d <= 8192;
-  for (int t = 0; t < m; ++t) all2 = all2 && radix[t] == 2;
-  if (all2) {
-    // stage t's group c is the butterfly's pair c of stage t (both number a pair by its
-    // lower index with bit t removed), and its block's first row is (cos p, sin p)
-    if ((e = cudaMalloc(&h->cs2, sizeof(float2) * (size_t)m * (d / 2))) != cudaSuccess)
+  int P = 0;  // leading stages of radix 2
+  while (P < m && radix[P] == 2) ++P;
+  if (P >= 6 && P <= 13) {
+    // stage t < P: group c is the butterfly's pair c of stage t (both number a pair by its
+    // lower index with bit t removed, block after block), and its block's first row is
+    // (cos p, sin p)
+    h->P = P;
+    if ((e = cudaMalloc(&h->cs2, sizeof(float2) * (size_t)P * (d / 2))) != cudaSuccess)
       return done(set_error(HARP_ERR_CUDA, "mr_plan_create: cudaMalloc: %s", cudaGetErrorString(e)));
-    const int64_t n = (int64_t)m * (d / 2);
-    cs_of_blocks_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(h->blocks, d, m, h->cs2);
+    const int64_t n = (int64_t)P * (d / 2);
+    cs_of_blocks_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(h->blocks, d, P, h->cs2);
     if ((e = cudaGetLastError()) != cudaSuccess)
       return done(set_error(HARP_ERR_CUDA, "mr_plan_create: table launch: %s", cudaGetErrorString(e)));
   }
@@ -544,7 +548,7 @@ namespace harp {
 cudaError_t launch_mr(const harp_mr_plan_s* plan, int inverse, int batch, const void* x, int xt, void* y, int yt,
                       cudaStream_t st, float* scratch) {
   if (batch <= 0) return cudaSuccess;
-  if (plan->cs2) {  // all radices 2: the radix-2 butterfly of width d with the plan's table
+  if (plan->cs2 && plan->P == plan->p.m) {  // all radices 2: the radix-2 butterfly of width d
     BflyParams bp{};
     bp.n = plan->p.d;
     bp.w = (int)plan->p.d;
@@ -570,14 +574,35 @@ cudaError_t launch_mr(const harp_mr_plan_s* plan, int inverse, int batch, const 
   // few rows: runs of stages over many CTAs, fp32 between runs in y (when fp32) or scratch
   float* buf = yt == DT_F32 ? static_cast<float*>(y) : scratch;
   if (batch < kMrSegRows && buf) {
+    // forward with leading radix-2 stages: those first, on the butterfly kernels (signs
+    // included), into buf; the runs then start at stage P
+    // (in place only up to width 512, where one CTA reads its whole block before writing)
+    const bool pre2 = plan->cs2 && !inverse && (x != buf || plan->P <= 9);
+    if (pre2) {
+      BflyParams bp{};
+      bp.n = p.d;
+      bp.w = 1 << plan->P;
+      bp.m = plan->P;
+      bp.cs = plan->cs2;
+      bp.sign = plan->sign;
+      bp.x = x;
+      bp.xt = xt;
+      bp.x_stride = p.d;
+      bp.y = buf;
+      bp.yt = DT_F32;
+      bp.y_stride = p.d;
+      bp.nsum = 1;
+      const cudaError_t e = launch_butterfly(bp, batch, st);
+      if (e != cudaSuccess) return e;
+    }
     static const int run_cap = [] {
       const char* e = getenv("HARP_MR_RUN");
       return e ? std::max(2, std::min(kMrSegRun, atoi(e))) : kMrSegRun;
     }();
     int runs[kMrMaxStages + 1], nr = 0;  // run boundaries in stage order
-    runs[nr++] = 0;
+    runs[nr++] = pre2 ? plan->P : 0;
     int64_t prod = 1;
-    for (int t = 0; t < p.m; ++t) {
+    for (int t = runs[0]; t < p.m; ++t) {
       if (prod * p.radix[t] > run_cap && prod > 1) {
         runs[nr++] = t;
         prod = 1;
@@ -608,7 +633,7 @@ cudaError_t launch_mr(const harp_mr_plan_s* plan, int inverse, int batch, const 
       const int per = (sp.br * (2 + sp.sumb) + ngrp) * (int)sizeof(float);  // shared bytes per sub-problem
       K = std::max(1, std::min(K, kMrSegSmem / per));
       sp.K = K;
-      sp.first = k == 0;
+      sp.first = k == 0 && !pre2;
       sp.last = k == nr - 1;
       sp.src = buf;
       sp.dst = buf;
